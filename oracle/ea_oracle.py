@@ -1,0 +1,270 @@
+"""Plain, slow CPU oracle for Elastic Attention's prefill hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module; only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use it.  It shares no code with the CUDA path.
+
+What it computes, and where the pages define it
+-----------------------------------------------
+Sources are two pages about one method:
+
+* the blog post "Elastic Attention：将 MoE 路由引入 Attention，让大模型长文本推理
+  '该省省，该花花'" (bxzpzcl.cn), cited here as *EA blog*, and its copy with the
+  results section on tiemojia.cn, cited as *EA blog (results copy)*;
+* the explainer page "Elastic Attention: Test-time Adaptive Sparsity Ratios for
+  Efficient Transformers" (gist.science), cited as *EA explainer*.
+
+1. Attention Router (EA blog §2.1 "核心架构：Attention Router"): the router reads the
+   layer's Key hidden states and a simple MLP emits one routing signal r per
+   head; r = 0 sends the head to Full Attention (FA), r = 1 to Sparse
+   Attention (SA).  The pages fix neither pooling, activation nor widths.
+   Readings taken here (all plain, all listed in the design doc):
+     - pooled input x[b] = mean over all N positions of K[b, :, n, :], flattened
+       in (kv_head, channel) order;
+     - h = ReLU(W1 x + b1), z = W2 h + b2 (nn.Linear convention, W is out x in);
+     - hard decision r = 1 iff z > threshold (threshold 0), a tie goes to FA.
+       Training uses Gumbel-Softmax with a straight-through estimator (EA blog
+       §2.1, "训练Trick"); at inference no noise is drawn.
+   The router size 0.27M parameters per layer for an 8B model (EA blog §2.2)
+   matches 1024 -> 256 -> 32 with biases (270,624 parameters).
+
+2. Full attention (EA blog §1 and §2.1): causal softmax attention over every
+   earlier token, softmax(q k^T * scale + causal mask) v, scale = 1/sqrt(d).
+
+3. Sparse attention (EA blog §1: heads that "only look locally or at a
+   sliding window"): fixed here as streaming attention, S sink tokens plus a
+   causal local window of W tokens.  Key j is visible from query i iff
+   j <= i and (j < S or i - j < W).  The window counts the diagonal.
+
+4. Result concat (EA blog §2.1 "结果融合"): every head writes its own slot of
+   out[B, Hq, N, d]; there is no separate concat step.
+
+GQA (not on the pages; the named backbones use it): query head h reads kv
+head h // (Hq // Hkv).
+
+Precision: everything in float64 from inputs the caller has already rounded
+to bf16 (the tests convert the same bf16 tensors the GPU receives).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "router_param_count",
+    "router_pool",
+    "router_mlp",
+    "router_decide",
+    "visible",
+    "visible_keys",
+    "attention_rows",
+    "attention",
+    "attention_weights",
+    "brute_force_attention",
+    "count_visible_pairs",
+]
+
+
+# --------------------------------------------------------------------------
+# Attention Router (EA blog §2.1; size from EA blog §2.2)
+# --------------------------------------------------------------------------
+
+def router_param_count(in_dim: int, hidden: int, out_dim: int) -> int:
+    """Parameters of a two-layer MLP with biases (EA blog §2.2: 0.27M/layer)."""
+    return in_dim * hidden + hidden + hidden * out_dim + out_dim
+
+
+def router_pool(k: np.ndarray) -> np.ndarray:
+    """Mean of the key states over the sequence.
+
+    k: [B, Hkv, N, d] (float64 values of the bf16 keys).
+    Returns x: [B, Hkv * d], flattened in (kv_head, channel) order.
+    Written as an explicit sum over positions divided by N.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    B, Hkv, N, d = k.shape
+    total = np.zeros((B, Hkv, d), dtype=np.float64)
+    for n in range(N):
+        total += k[:, :, n, :]
+    return (total / N).reshape(B, Hkv * d)
+
+
+def router_mlp(x: np.ndarray, w1: np.ndarray, b1: np.ndarray,
+               w2: np.ndarray, b2: np.ndarray) -> np.ndarray:
+    """z = W2 ReLU(W1 x + b1) + b2, per batch row.  W is [out, in]."""
+    x = np.asarray(x, dtype=np.float64)
+    w1 = np.asarray(w1, dtype=np.float64)
+    b1 = np.asarray(b1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64)
+    b2 = np.asarray(b2, dtype=np.float64)
+    pre = x @ w1.T + b1
+    h = np.where(pre > 0.0, pre, 0.0)
+    return h @ w2.T + b2
+
+
+def router_decide(k, w1, b1, w2, b2, threshold: float = 0.0):
+    """Route mask [B, Hq] (uint8, 1 = SA, 0 = FA) and the logits z [B, Hq].
+
+    r = 1 (sparse) iff z > threshold; z == threshold routes to FA.
+    """
+    z = router_mlp(router_pool(k), w1, b1, w2, b2)
+    mask = (z > threshold).astype(np.uint8)
+    return mask, z
+
+
+# --------------------------------------------------------------------------
+# Visibility: FA = causal; SA = sink S + causal local window W (EA blog §1)
+# --------------------------------------------------------------------------
+
+def visible(i: int, j: int, sparse: bool, sink: int, window: int) -> bool:
+    """Is key j visible from query i?  Square causal prefill, no offset."""
+    if j > i:
+        return False
+    if not sparse:
+        return True
+    return j < sink or (i - j) < window
+
+
+def visible_keys(i: int, sparse: bool, sink: int, window: int) -> np.ndarray:
+    """Sorted indices of the keys query i sees (each key once)."""
+    if not sparse:
+        return np.arange(i + 1)
+    lo = max(0, i - window + 1)
+    sink_part = np.arange(min(sink, lo))          # sink keys left of the window
+    return np.concatenate([sink_part, np.arange(lo, i + 1)])
+
+
+def count_visible_pairs(n: int, sparse: bool, sink: int, window: int) -> int:
+    """Number of visible (i, j) pairs of one head, by enumeration of rows."""
+    return int(sum(len(visible_keys(i, sparse, sink, window)) for i in range(n)))
+
+
+# --------------------------------------------------------------------------
+# Attention
+# --------------------------------------------------------------------------
+
+def _softmax_row_weighted(scores: np.ndarray, vals: np.ndarray) -> np.ndarray:
+    """softmax(scores) @ vals for a block of rows; scores may hold -inf."""
+    m = np.max(scores, axis=-1, keepdims=True)
+    e = np.exp(scores - m)
+    return (e @ vals) / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention_rows(q, k, v, mask, b: int, h: int, rows, sink: int, window: int,
+                   scale: float | None = None) -> np.ndarray:
+    """Output rows out[b, h, rows, :] in float64.
+
+    Each row is an exact function of that row alone, so any subset of rows can
+    be checked.  Scores use only the keys the row sees (EA blog §1, §2.1).
+    """
+    Hq = q.shape[1]
+    Hkv = k.shape[1]
+    d = q.shape[3]
+    g = Hq // Hkv
+    hk = h // g
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    sparse = bool(mask[b, h])
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.empty((len(rows), d), dtype=np.float64)
+    qh = np.asarray(q[b, h], dtype=np.float64)
+    kh = np.asarray(k[b, hk], dtype=np.float64)
+    vh = np.asarray(v[b, hk], dtype=np.float64)
+    for r, i in enumerate(rows):
+        keys = visible_keys(int(i), sparse, sink, window)
+        s = (kh[keys] @ qh[i]) * scale
+        out[r] = _softmax_row_weighted(s[None, :], vh[keys])[0]
+    return out
+
+
+def attention(q, k, v, mask, sink: int, window: int, scale: float | None = None,
+              block: int = 256) -> np.ndarray:
+    """Full output out[B, Hq, N, d] in float64.
+
+    Rows are processed in blocks; each block forms scores against the union of
+    the keys its rows may see and then applies the exact element mask, so the
+    result equals the row-by-row definition.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.empty((B, Hq, N, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // g
+            sparse = bool(mask[b, h])
+            for i0 in range(0, N, block):
+                i1 = min(N, i0 + block)
+                if sparse:
+                    lo = max(0, i0 - window + 1)
+                    keys = np.concatenate([np.arange(min(sink, lo)),
+                                           np.arange(lo, i1)])
+                else:
+                    keys = np.arange(i1)
+                s = (q[b, h, i0:i1] @ k[b, hk, keys].T) * scale
+                ii = np.arange(i0, i1)[:, None]
+                jj = keys[None, :]
+                vis = jj <= ii
+                if sparse:
+                    vis &= (jj < sink) | ((ii - jj) < window)
+                s = np.where(vis, s, -np.inf)
+                out[b, h, i0:i1] = _softmax_row_weighted(s, v[b, hk, keys])
+    return out
+
+
+def attention_weights(q, k, mask, b: int, h: int, sink: int, window: int,
+                      scale: float | None = None) -> np.ndarray:
+    """Dense N x N attention weights of one head (small N only)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    Hq, N, d = q.shape[1], q.shape[2], q.shape[3]
+    g = Hq // k.shape[1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    sparse = bool(mask[b, h])
+    s = (q[b, h] @ k[b, h // g].T) * scale
+    vis = np.array([[visible(i, j, sparse, sink, window) for j in range(N)]
+                    for i in range(N)])
+    s = np.where(vis, s, -np.inf)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def brute_force_attention(q, k, v, mask, sink: int, window: int,
+                          scale: float | None = None) -> np.ndarray:
+    """Per-element loops, for N <= 64: independent of the blocked version."""
+    B, Hq, N, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv = len(k[0])
+    g = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.zeros((B, Hq, N, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // g
+            sparse = bool(mask[b][h])
+            for i in range(N):
+                scores = []
+                keys = []
+                for j in range(N):
+                    if visible(i, j, sparse, sink, window):
+                        dot = 0.0
+                        for c in range(d):
+                            dot += float(q[b][h][i][c]) * float(k[b][hk][j][c])
+                        scores.append(dot * scale)
+                        keys.append(j)
+                mx = max(scores)
+                w = [math.exp(s - mx) for s in scores]
+                tot = sum(w)
+                for c in range(d):
+                    acc = 0.0
+                    for wj, j in zip(w, keys):
+                        acc += wj * float(v[b][hk][j][c])
+                    out[b, h, i, c] = acc / tot
+    return out

@@ -1,0 +1,92 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check that
+the pins in test_oracle_pins.py catch every one of them."""
+import importlib.util
+import inspect
+import os
+import types
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "ea_oracle.py")
+
+MUTATIONS = {
+    "window_off_by_one_visible": ("return j < sink or (i - j) < window",
+                                  "return j < sink or (i - j) <= window"),
+    "window_off_by_one_blocked": ("vis &= (jj < sink) | ((ii - jj) < window)",
+                                  "vis &= (jj < sink) | ((ii - jj) <= window)"),
+    "window_off_by_one_rows": ("lo = max(0, i - window + 1)",
+                               "lo = max(0, i - window)"),
+    "causal_strict": ("if j > i:", "if j >= i:"),
+    "gqa_modulo_mapping": ("    hk = h // g\n", "    hk = h % Hkv\n"),
+    "gqa_modulo_mapping_blocked": ("            hk = h // g\n", "            hk = h % Hkv\n"),
+    "scale_one_over_d": ("        scale = 1.0 / math.sqrt(d)\n    sparse = bool(mask[b, h])\n    rows",
+                         "        scale = 1.0 / d\n    sparse = bool(mask[b, h])\n    rows"),
+    "scale_one_over_d_blocked": ("        scale = 1.0 / math.sqrt(d)\n    out = np.empty((B, Hq, N, d)",
+                                 "        scale = 1.0 / d\n    out = np.empty((B, Hq, N, d)"),
+    "relu_dropped": ("h = np.where(pre > 0.0, pre, 0.0)", "h = pre"),
+    "bias2_dropped": ("return h @ w2.T + b2", "return h @ w2.T"),
+    "bias1_dropped": ("pre = x @ w1.T + b1", "pre = x @ w1.T"),
+    "w1_transposed": ("pre = x @ w1.T + b1", "pre = x @ w1 + b1"),
+    "tie_to_sparse": ("mask = (z > threshold)", "mask = (z >= threshold)"),
+    "pool_divisor": ("return (total / N)", "return (total / (N - 1))"),
+    "pool_flatten_order": ("return (total / N).reshape(B, Hkv * d)",
+                           "return (total / N).transpose(0, 2, 1).reshape(B, Hkv * d)"),
+    "sink_double_count": ("sink_part = np.arange(min(sink, lo))",
+                          "sink_part = np.arange(min(sink, i + 1))"),
+    "softmax_unnormalised": ("return (e @ vals) / np.sum(e, axis=-1, keepdims=True)",
+                             "return (e @ vals)"),
+    "sink_ignored_blocked": ("vis &= (jj < sink) | ((ii - jj) < window)",
+                             "vis &= ((ii - jj) < window)"),
+}
+
+
+def _mutant(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation {name} does not apply"
+    src = src.replace(old, new, 1)
+    mod = types.ModuleType(f"oracle_mutant_{name}")
+    exec(compile(src, f"<mutant {name}>", "exec"), mod.__dict__)
+    return mod
+
+
+def _pin_calls():
+    """Every pin with a fixed argument set (parametrised pins expanded)."""
+    calls = []
+    for fname, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not fname.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if not params:
+            calls.append((fname, fn, {}))
+            continue
+        argnames, values = params[0].args[0], params[0].args[1]
+        names = [a.strip() for a in argnames.split(",")]
+        for val in values:
+            vals = val if isinstance(val, tuple) else (val,)
+            calls.append((fname, fn, dict(zip(names, vals))))
+    return calls
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    mutant = _mutant(name)
+    monkeypatch.setattr(pins, "oracle", mutant)
+    caught = []
+    for fname, fn, kwargs in _pin_calls():
+        try:
+            fn(**kwargs)
+        except Exception:       # an assertion, or a shape error from the slip
+            caught.append(fname)
+    assert caught, f"no pin catches mutation {name}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert pins.oracle is oracle
+    for fname, fn, kwargs in _pin_calls():
+        fn(**kwargs)

@@ -1,0 +1,261 @@
+"""Pins for the CPU oracle: facts fixed by the pages or by mathematics, not by
+the oracle itself.  Each test is chosen so that a plausible slip in the
+oracle (a dropped term, a wrong sign, an off-by-one window, a transposed
+operand, a wrong GQA mapping, a wrong scale) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, dtype=np.float64):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal(shape).astype(dtype)
+
+
+def _bf16(x):
+    """Round float64 values to bf16 exactly as the GPU inputs are rounded."""
+    return torch.from_numpy(np.asarray(x)).to(torch.bfloat16).double().numpy()
+
+
+def _qkv(B, Hq, Hkv, N, d, seed):
+    q = _bf16(_rand((B, Hq, N, d), seed))
+    k = _bf16(_rand((B, Hkv, N, d), seed + 1))
+    v = _bf16(_rand((B, Hkv, N, d), seed + 2))
+    return q, k, v
+
+
+# --------------------------------------------------------------------------
+# Router pins
+# --------------------------------------------------------------------------
+
+def test_router_size_matches_printed_value():
+    """EA blog §2.2 prints 0.27M router parameters per layer (8B model)."""
+    g = json.load(open(os.path.join(GOLDEN, "router_size.json")))
+    n = oracle.router_param_count(*g["dims"])
+    assert n == 270624
+    assert abs(n - g["printed_params_per_layer"]) <= g["printed_precision"]
+    # a router without biases or with a 2-way output per head would not round
+    # to the printed value
+    assert abs(1024 * 256 + 256 * 64 + 256 + 64 - 270000) > 5000
+
+
+def test_router_pool_closed_forms():
+    B, Hkv, N, d = 2, 3, 37, 5
+    k = np.zeros((B, Hkv, N, d))
+    for b in range(B):
+        for h in range(Hkv):
+            for n in range(N):
+                for c in range(d):
+                    k[b, h, n, c] = 1000.0 * h + c + 0.5 * n + 7.0 * b
+    x = oracle.router_pool(k)
+    assert x.shape == (B, Hkv * d)
+    for b in range(B):
+        for h in range(Hkv):
+            for c in range(d):
+                # mean of 0.5 n over n = 0..N-1 is 0.25 (N - 1)
+                want = 1000.0 * h + c + 0.25 * (N - 1) + 7.0 * b
+                assert x[b, h * d + c] == pytest.approx(want, abs=1e-9)
+
+
+def test_router_mlp_hand_example():
+    """A hand-worked two-layer MLP: ReLU kills the negative pre-activation,
+    the biases enter once, a logit exactly at the threshold routes to FA."""
+    x = np.array([[1.0, -2.0, 3.0]])
+    w1 = np.eye(3)
+    b1 = np.array([0.0, 0.0, -1.0])         # pre = [1, -2, 2] -> h = [1, 0, 2]
+    w2 = np.array([[1.0, 1.0, 1.0], [0.0, -1.0, 0.0], [-1.0, 0.0, 0.0]])
+    b2 = np.array([0.5, 0.0, 0.25])         # z = [3.5, 0, -0.75]
+    z = oracle.router_mlp(x, w1, b1, w2, b2)
+    np.testing.assert_allclose(z, [[3.5, 0.0, -0.75]], atol=0, rtol=0)
+    k = np.broadcast_to(np.array([1.0, -2.0, 3.0]), (1, 1, 4, 3)).copy()
+    mask, z2 = oracle.router_decide(k, w1, b1, w2, b2, threshold=0.0)
+    np.testing.assert_array_equal(mask, [[1, 0, 0]])   # r=1 -> SA, tie -> FA
+    mask_hi, _ = oracle.router_decide(k, w1, b1, w2, b2, threshold=3.5)
+    np.testing.assert_array_equal(mask_hi, [[0, 0, 0]])
+
+
+def test_router_matches_torch_linear():
+    """Cross-check with torch's nn.functional.linear in float64."""
+    B, Hkv, N, d, hid, Hq = 2, 2, 19, 8, 16, 4
+    k = _rand((B, Hkv, N, d), 5)
+    w1, b1 = _rand((hid, Hkv * d), 6), _rand((hid,), 7)
+    w2, b2 = _rand((Hq, hid), 8), _rand((Hq,), 9)
+    z = oracle.router_mlp(oracle.router_pool(k), w1, b1, w2, b2)
+    kt = torch.from_numpy(k)
+    x = kt.mean(dim=2).reshape(B, Hkv * d)
+    h = torch.relu(torch.nn.functional.linear(x, torch.from_numpy(w1), torch.from_numpy(b1)))
+    zt = torch.nn.functional.linear(h, torch.from_numpy(w2), torch.from_numpy(b2))
+    np.testing.assert_allclose(z, zt.numpy(), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Attention pins
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,d", [(1, 8), (63, 16), (300, 32)])
+def test_all_fa_is_dense_causal_sdpa(N, d):
+    """An all-zero mask is dense causal attention: torch SDPA in float64."""
+    B, Hq, Hkv = 2, 4, 2
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 11)
+    mask = np.zeros((B, Hq), np.uint8)
+    out = oracle.attention(q, k, v, mask, sink=3, window=5, block=64)
+    g = Hq // Hkv
+    kt = torch.from_numpy(k).repeat_interleave(g, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(g, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), kt, vt, is_causal=True)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_sparse_equals_full_when_window_covers_sequence():
+    B, Hq, Hkv, N, d = 1, 4, 4, 90, 16
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 12)
+    full = oracle.attention(q, k, v, np.zeros((B, Hq), np.uint8), 10, 80, block=32)
+    for S, W in [(10, 80), (0, 90), (90, 1), (45, 45), (5, 200)]:
+        sa = oracle.attention(q, k, v, np.ones((B, Hq), np.uint8), S, W, block=32)
+        np.testing.assert_array_equal(sa, full)
+    # one key short of covering: a late row must differ
+    sa = oracle.attention(q, k, v, np.ones((B, Hq), np.uint8), 10, 79, block=32)
+    assert np.max(np.abs(sa[..., -1, :] - full[..., -1, :])) > 1e-6
+
+
+def test_window_one_no_sink_returns_own_value():
+    """S = 0, W = 1: each query sees only itself, out[i] = v[i] (GQA h // G)."""
+    B, Hq, Hkv, N, d = 2, 6, 2, 40, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 13)
+    out = oracle.attention(q, k, v, np.ones((B, Hq), np.uint8), 0, 1, block=16)
+    for h in range(Hq):
+        np.testing.assert_array_equal(out[:, h], v[:, h // 3])
+
+
+def test_sink_one_window_one_two_key_closed_form():
+    """S = 1, W = 1: query i > 0 sees keys {0, i}.  With a = (q.k0 - q.ki)/sqrt(d),
+    out[i] = sigma(a) v0 + (1 - sigma(a)) vi, and out[0] = v0."""
+    B, Hq, Hkv, N, d = 1, 2, 1, 30, 16
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 14)
+    out = oracle.attention(q, k, v, np.ones((B, Hq), np.uint8), 1, 1, block=8)
+    for h in range(Hq):
+        np.testing.assert_allclose(out[0, h, 0], v[0, 0, 0], atol=1e-15)
+        for i in range(1, N):
+            a = (q[0, h, i] @ k[0, 0, 0] - q[0, h, i] @ k[0, 0, i]) / math.sqrt(d)
+            sig = 1.0 / (1.0 + math.exp(-a))
+            want = sig * v[0, 0, 0] + (1.0 - sig) * v[0, 0, i]
+            np.testing.assert_allclose(out[0, h, i], want, rtol=0, atol=1e-13)
+
+
+def test_explicit_scale_enters_scores():
+    B, Hq, Hkv, N, d = 1, 1, 1, 12, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 15)
+    m = np.ones((1, 1), np.uint8)
+    out = oracle.attention(q, k, v, m, 1, 1, scale=0.25, block=4)
+    i = 7
+    a = 0.25 * (q[0, 0, i] @ k[0, 0, 0] - q[0, 0, i] @ k[0, 0, i])
+    sig = 1.0 / (1.0 + math.exp(-a))
+    np.testing.assert_allclose(out[0, 0, i], sig * v[0, 0, 0] + (1 - sig) * v[0, 0, i],
+                               atol=1e-13)
+
+
+def test_constant_values_give_constant_output():
+    B, Hq, Hkv, N, d = 1, 4, 2, 77, 8
+    q, k, _ = _qkv(B, Hq, Hkv, N, d, 16)
+    v = np.broadcast_to(np.arange(d, dtype=np.float64) - 2.5, (B, Hkv, N, d)).copy()
+    mask = np.array([[0, 1, 1, 0]], np.uint8)
+    out = oracle.attention(q, k, v, mask, 4, 9, block=16)
+    np.testing.assert_allclose(out, np.broadcast_to(v[:, :1], out.shape), atol=1e-13)
+
+
+def test_weights_sum_to_one_and_vanish_off_pattern():
+    B, Hq, Hkv, N, d = 1, 2, 1, 50, 8
+    q, k, _ = _qkv(B, Hq, Hkv, N, d, 17)
+    mask = np.array([[0, 1]], np.uint8)
+    S, W = 3, 7
+    for h in range(Hq):
+        w = oracle.attention_weights(q, k, mask, 0, h, S, W)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, atol=1e-14)
+        for i in range(N):
+            for j in range(N):
+                causal = j <= i
+                seen = causal and (h == 0 or j < S or i - j < W)
+                if not seen:
+                    assert w[i, j] == 0.0
+                else:
+                    assert w[i, j] > 0.0
+    # visible-key counts per row of the SA head
+    counts = [(oracle.attention_weights(q, k, mask, 0, 1, S, W)[i] > 0).sum()
+              for i in range(N)]
+    for i, c in enumerate(counts):
+        assert c == min(i + 1, W + min(S, max(0, i - W + 1)))
+
+
+def test_head_permutation_equivariance():
+    """Permuting kv groups and heads within a group, together with their mask
+    bits, permutes the outputs the same way."""
+    B, Hq, Hkv, N, d = 2, 6, 3, 45, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 18)
+    rng = np.random.default_rng(3)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    out = oracle.attention(q, k, v, mask, 2, 6, block=16)
+    gperm = np.array([2, 0, 1])
+    inner = np.array([1, 0])
+    hperm = np.array([gp * 2 + inner[i] for gp in gperm for i in range(2)])
+    out2 = oracle.attention(q[:, hperm], k[:, gperm], v[:, gperm], mask[:, hperm], 2, 6,
+                            block=16)
+    np.testing.assert_allclose(out2, out[:, hperm], atol=1e-14, rtol=0)
+
+
+def test_batch_rows_independent():
+    B, Hq, Hkv, N, d = 3, 2, 1, 33, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 19)
+    mask = np.array([[0, 1], [1, 1], [0, 0]], np.uint8)
+    out = oracle.attention(q, k, v, mask, 2, 5, block=8)
+    for b in range(B):
+        one = oracle.attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], mask[b:b + 1], 2, 5,
+                               block=8)
+        np.testing.assert_array_equal(one[0], out[b])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_brute_force_agrees(seed):
+    rng = np.random.default_rng(100 + seed)
+    Hkv = int(rng.integers(1, 3))
+    g = int(rng.integers(1, 3))
+    Hq = Hkv * g
+    B = int(rng.integers(1, 3))
+    N = int(rng.integers(1, 65))
+    d = int(rng.choice([4, 8]))
+    S = int(rng.integers(0, 9))
+    W = int(rng.integers(1, 20))
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 200 + seed)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    fast = oracle.attention(q, k, v, mask, S, W, block=int(rng.integers(1, 40)))
+    slow = oracle.brute_force_attention(q.tolist(), k.tolist(), v.tolist(), mask.tolist(),
+                                        S, W)
+    np.testing.assert_allclose(fast, slow, rtol=0, atol=1e-12)
+    rows = sorted(set(int(r) for r in rng.integers(0, N, size=5)))
+    for b in range(B):
+        for h in range(Hq):
+            part = oracle.attention_rows(q, k, v, mask, b, h, rows, S, W)
+            np.testing.assert_allclose(part, slow[b, h, rows], rtol=0, atol=1e-12)
+
+
+def test_visible_pair_counts_closed_forms():
+    for N in [1, 2, 17, 300]:
+        assert oracle.count_visible_pairs(N, False, 5, 7) == N * (N + 1) // 2
+    # pure sliding window: row i sees min(i + 1, W) keys
+    for N, W in [(50, 7), (10, 20), (129, 128)]:
+        want = sum(min(i + 1, W) for i in range(N))
+        assert oracle.count_visible_pairs(N, True, 0, W) == want
+    # sink + window: a row past S + W - 1 sees exactly S + W keys
+    S, W, N = 4, 6, 40
+    assert len(oracle.visible_keys(N - 1, True, S, W)) == S + W
+    assert len(oracle.visible_keys(S + W - 1, True, S, W)) == S + W
+    assert len(oracle.visible_keys(S + W - 2, True, S, W)) == S + W - 1
