@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark of the Elastic Attention prefill hot path on B200.
+
+One step = one attention layer's prefill: the Attention Router
+(ea_router_decide) on the key states, then the fused hybrid FA/SA attention
+(ea_hybrid_attn_prefill), on seeded synthetic inputs already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Multi-GPU runs (torchrun, one rank per GPU)
+are independent replicas of the workload on every rank (the path splits into
+independent (batch, head) problems, so there is no data-path collective); the
+time is the max over ranks and `value` counts the work of all ranks.
+
+--impl reference times the CPU oracle (float64 numpy, the plain definition of
+the method) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "effective prefill attention TFLOPS and tokens/s at 1 B200; % of bf16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+# ---------------------------------------------------------------- helpers
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the host-buffer end-to-end measurement (default: --steps)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed region only: no comparators, e2e or CPU baseline")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w: workloads.Workload, mask_frac: float) -> str:
+    s = (f"{w.name}: B{w.batch} N{w.seq} Hq{w.hq} Hkv{w.hkv} d{w.d} sink{w.sink} "
+         f"window{w.window}")
+    if w.use_router:
+        s += f" router {w.hkv * w.d}-{w.router_hidden}-{w.hq}"
+    s += f" sparse-head fraction {mask_frac:.3f}"
+    if w.layers > 1:
+        s += f" x{w.layers} layers"
+    return s
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def visible_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids) and ids[local_rank].strip().isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def traffic_for_current_kernel():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, only if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    src = os.path.join(ROOT, "sparse_attention_head_b200", "csrc", "ea_attn.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("kernel_sha256_16") != h:
+        return None
+    return d.get("dram_bytes_per_launch_full_workload")
+
+
+# ---------------------------------------------------------------- inputs
+def make_layer(w: workloads.Workload, layer: int, rank: int, device):
+    seed = workloads.layer_seed(w, layer) + 7919 * rank
+    q, k, v = workloads.make_qkv(w, seed, device=device)
+    if w.use_router:
+        frac = workloads.layer_sparse_frac(w, layer)
+        heads = workloads.sparse_head_set(w.hq, frac, seed)
+        w1, b1, w2, b2 = workloads.make_router_weights(w.hkv * w.d, w.router_hidden, w.hq,
+                                                       heads, seed)
+        router = tuple(t.to(device) for t in (w1, b1, w2, b2))
+        mask = None
+    else:
+        router = None
+        mask = workloads.make_fixed_mask(w, seed).to(device)
+    return {"q": q, "k": k, "v": v, "router": router, "mask": mask, "seed": seed}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (EA_SELECT_FA, EA_SELECT_SA, HostPrefill,
+                                                attn_workspace, ea_get_device_status,
+                                                ea_hybrid_attn_prefill, ea_router_decide,
+                                                ea_router_workspace_size, make_params)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
+    nlayers = w.layers
+    # qwen8b36-style multi-layer workloads keep one layer resident at a time
+    # per step would need regeneration; here every layer's inputs stay
+    # resident only when they fit in a quarter of the device memory.
+    layers = [make_layer(w, l, rank, dev) for l in range(nlayers)]
+    p = make_params(B, Hq, Hkv, N, d, w.sink, w.window)
+    aws = attn_workspace(p, dev)
+    rws = torch.empty(max(ea_router_workspace_size(B, Hkv, N, d), 16), dtype=torch.uint8,
+                      device=dev)
+    outs = [torch.empty_like(L["q"]) for L in layers]
+    masks = [torch.empty((B, Hq), dtype=torch.uint8, device=dev) if L["router"] is not None
+             else L["mask"] for L in layers]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        for li, L in enumerate(layers):
+            if ev is not None:
+                ev[li][0].record(stream)
+            if L["router"] is not None:
+                ea_router_decide(L["k"], *L["router"], workspace=rws, route_mask=masks[li],
+                                 want_logits=False)
+            if ev is not None:
+                ev[li][1].record(stream)
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], masks[li], w.sink, w.window,
+                                   out=outs[li], workspace=aws)
+            if ev is not None:
+                ev[li][2].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if ea_get_device_status(aws) != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+
+    mask_host = [m.cpu().numpy() for m in masks]
+    eff = sum(flops.effective_flops(m, N, d, w.sink, w.window) for m in mask_host)
+    tile = sum(flops.tile_flops(m, N, d, w.sink, w.window) for m in mask_host)
+    sparse_frac = float(np.mean([m.mean() for m in mask_host]))
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlayers)]
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(visible_gpu_index(local_rank)) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = t0.elapsed_time(t1)
+    attn_ms = [evs[i][l][1].elapsed_time(evs[i][l][2]) for i in range(K) for l in range(nlayers)]
+    router_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K)
+                 for l in range(nlayers)]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if ea_get_device_status(aws) != 0:
+        raise RuntimeError("device status word reports an error after the timed region")
+
+    ms_per_step = total_ms / K
+    value = eff * world / (ms_per_step * 1e-3) / 1e12
+    tokens_per_s = B * N * world / (ms_per_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = (eff / nlayers) / (attn_avg_ms * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(w, sparse_frac), "global_batch": B * world,
+                   "seq_len": N, "parallelism": f"replicas x{world}",
+                   "l2": "inputs exceed L2 (Q+K+V %.0f MiB > 126 MB), no flush"
+                         % ((B * (Hq + 2 * Hkv) * N * d * 2) / 2 ** 20)},
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_bf16_peak": round(100.0 * value / world / peak, 2),
+        "tile_granular_tflops": round(tile * world / (ms_per_step * 1e-3) / 1e12, 2),
+        "attn_ms": round(attn_avg_ms, 4),
+        "router_ms": round(statistics.mean(router_ms), 4),
+        "gpu_launches": K * nlayers * (3 if layers[0]["router"] is not None else 1),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "traffic": traffic_for_current_kernel(),
+                     "kernel": "ea_hybrid_attn_kernel<128>"},
+        "clocks": clocks,
+    }
+
+    if not args.quick and world == 1:
+        # comparators on the same inputs (outside the timed region)
+        L = layers[0]
+        m0 = masks[0]
+
+        def timeit(fn, reps=5):
+            fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+
+        out_tmp = torch.empty_like(L["q"])
+
+        def split_pass():
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], m0, w.sink, w.window,
+                                   select=EA_SELECT_FA, out=out_tmp, workspace=aws)
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], m0, w.sink, w.window,
+                                   select=EA_SELECT_SA, out=out_tmp, workspace=aws)
+
+        def fused():
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], m0, w.sink, w.window,
+                                   out=out_tmp, workspace=aws)
+        all_fa = torch.zeros_like(m0)
+
+        def full_causal():
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], all_fa, w.sink, w.window,
+                                   out=out_tmp, workspace=aws)
+        fused_ms = timeit(fused)
+        split_ms = timeit(split_pass)
+        full_ms = timeit(full_causal, reps=3)
+        full_eff = flops.effective_flops(all_fa.cpu().numpy(), N, d, w.sink, w.window)
+        result["comparators"] = {
+            "fused_attn_ms": round(fused_ms, 4),
+            "split_fa_then_sa_ms": round(split_ms, 4),
+            "fused_speedup_vs_split": round(split_ms / fused_ms, 3),
+            "full_causal_ms": round(full_ms, 4),
+            "full_causal_tflops": round(full_eff / (full_ms * 1e-3) / 1e12, 2),
+            "elastic_speedup_vs_full_causal": round(full_ms / fused_ms, 3),
+        }
+        # end to end through the public API with host buffers
+        if L["router"] is not None:
+            ek = args.e2e_steps or K
+            hp = HostPrefill(B, Hq, Hkv, N, d, *L["router"], w.sink, w.window, device=dev)
+            qh = L["q"].cpu().pin_memory()
+            kh = L["k"].cpu().pin_memory()
+            vh = L["v"].cpu().pin_memory()
+            for _ in range(2):
+                hp(qh, kh, vh)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(ek):
+                hp(qh, kh, vh)
+            b.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms = a.elapsed_time(b) / ek
+            result["e2e"] = {"value": round(eff / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                             "h2d_bytes_per_step": hp.h2d_bytes(),
+                             "d2h_bytes_per_step": hp.d2h_bytes(),
+                             "ms_per_step": round(e2e_ms, 4),
+                             "path": "HostPrefill: pinned host q,k,v -> ea_router_decide -> "
+                                     "ea_hybrid_attn_prefill -> pinned host out"}
+        if rank == 0:
+            result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
+    return result
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(w, L_cpu, mask_np, target_s, rng):
+    """Time the oracle on a bounded sample: the full router (when the workload
+    has one) and sampled query rows of every head.  Returns (flops, seconds,
+    description)."""
+    import oracle
+    q, k, v = L_cpu["q"], L_cpu["k"], L_cpu["v"]
+    N, d = w.seq, w.d
+    t_start = time.perf_counter()
+    if L_cpu.get("router") is not None:
+        w1, b1, w2, b2 = L_cpu["router"]
+        oracle.router_decide(k, w1, b1, w2, b2)
+    t_router = time.perf_counter() - t_start
+    fl = 0.0
+    rows_done = 0
+    heads = [(b, h) for b in range(w.batch) for h in range(w.hq)]
+    t_att = 0.0
+    while t_att < max(0.5, target_s - t_router):
+        b, h = heads[rows_done % len(heads)]
+        rows = rng.integers(0, N, size=4)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, mask_np, b, h, rows, w.sink, w.window)
+        t_att += time.perf_counter() - t0
+        sparse = bool(mask_np[b, h])
+        for i in rows:
+            fl += 4.0 * d * len(oracle.visible_keys(int(i), sparse, w.sink, w.window))
+        rows_done += 1
+    desc = (f"oracle router on the full key tensor plus {4 * rows_done} sampled query rows "
+            f"over all heads")
+    return fl, t_router + t_att, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def host_layer(L):
+    """float64 host copies of one layer's inputs for the oracle."""
+    out = {"q": L["q"].float().cpu().double().numpy(), "k": L["k"].float().cpu().double().numpy(),
+           "v": L["v"].float().cpu().double().numpy(), "router": None}
+    if L["router"] is not None:
+        out["router"] = tuple(t.cpu().double().numpy() for t in L["router"])
+    return out
+
+
+def cpu_baseline(w, L, mask_np, target_s):
+    Lc = host_layer(L)
+    fl, secs, desc = oracle_sample(w, Lc, mask_np, target_s, np.random.default_rng(5))
+    return {"value": round(fl / secs / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle", "sample": desc + f"; {secs:.1f} s of CPU time"}
+
+
+def run_reference(args):
+    w = workloads.get(args.workload)
+    L = make_layer(w, 0, 0, "cpu")
+    if L["router"] is not None:
+        import oracle
+        Lc = host_layer(L)
+        mask_np, _ = oracle.router_decide(Lc["k"], *Lc["router"])
+    else:
+        Lc = host_layer(L)
+        mask_np = L["mask"].numpy()
+    rng = np.random.default_rng(11)
+    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, Lc, mask_np, per_step * 0.25, rng)
+    tot_fl, tot_s = 0.0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        fl, s, desc = oracle_sample(w, Lc, mask_np, per_step, rng)
+        tot_fl += fl
+        tot_s += s
+    value = tot_fl / tot_s / 1e12
+    sparse_frac = float(mask_np.mean())
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch,
+                   "seq_len": w.seq, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc + " per step"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=180),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

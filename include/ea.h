@@ -1,0 +1,178 @@
+/*
+ * ea.h — C ABI of the Elastic Attention prefill library (libea.so), sm_100a.
+ *
+ * The method (Elastic Attention blog, bxzpzcl.cn, §2.1 "Attention Router" and
+ * §3 "Fused Kernel"): a light router reads the layer's key states and emits,
+ * for every head, a routing bit r; r = 0 sends the head to Full Attention
+ * (causal softmax attention over all earlier tokens), r = 1 to Sparse
+ * Attention (here: S sink tokens plus a causal local window of W tokens).
+ * The routing bits are passed to one fused kernel as metadata, and that one
+ * launch computes the FA heads and the SA heads together.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are dense, contiguous, row-major, in BHSD order:
+ *      q, out : bf16 [B][Hq][N][d]      k, v : bf16 [B][Hkv][N][d]
+ *    Query head h reads kv head h / (Hq / Hkv).
+ *  - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *    never allocates, frees or keeps device memory of its own.  Parameter
+ *    structs are HOST pointers, read before the call returns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; no entry point synchronises except ea_get_device_status.
+ *  - Argument errors are returned synchronously, before anything is
+ *    enqueued.  Launch failures return EA_ERR_CUDA.  A device-side wait that
+ *    runs out (EA_ERR_TIMEOUT) is recorded in a device status word and read
+ *    back with ea_get_device_status.
+ *  - Calls on different streams may run concurrently as long as each has its
+ *    own workspace and output buffers.
+ */
+#ifndef EA_H_
+#define EA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ea_status {
+  EA_OK = 0,
+  EA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad enum   */
+  EA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle   */
+  EA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned            */
+  EA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed           */
+  EA_ERR_TIMEOUT = 5,       /* a device-side wait ran out (see status)     */
+  EA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required  */
+} ea_status;
+
+/* Which heads one attention call computes.  EA_SELECT_ALL is the fused
+ * single launch; EA_SELECT_FA / EA_SELECT_SA compute only the heads routed
+ * to that mode (two such calls form the split "serial dispatch" pass that
+ * the Elastic Attention blog, §3, contrasts with the fused kernel). */
+typedef enum ea_select {
+  EA_SELECT_ALL = 0,
+  EA_SELECT_FA = 1,
+  EA_SELECT_SA = 2
+} ea_select;
+
+/* Static string for a status code (never NULL). */
+const char* ea_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int ea_version(void);
+
+/* ------------------------------------------------------------------------
+ * Attention Router (Elastic Attention blog §2.1: the router takes the key
+ * hidden states and a simple MLP emits one routing signal per head; r = 0 is
+ * Full Attention, r = 1 is Sparse Attention; §2.2: 0.27M parameters per
+ * layer for an 8B model = 1024 -> 256 -> 32 with biases).
+ *
+ *   x[b]          = (1/N) * sum_n K[b, :, n, :]   flattened (kv_head, channel)
+ *   h             = ReLU(W1 x + b1)              W1: [hidden][Hkv*d], b1: [hidden]
+ *   z[b, :]       = W2 h + b2                    W2: [Hq][hidden],    b2: [Hq]
+ *   route_mask[b, j] = (z[b, j] > threshold) ? 1 : 0     (a tie routes to FA)
+ *
+ * k          : device bf16 [B][Hkv][N][d].
+ * w1,b1,w2,b2: device fp32, row-major (out x in), 16-byte aligned;
+ *              Hkv*d and hidden must be multiples of 4.
+ * route_mask : device uint8 [B][Hq], written (1 = sparse, 0 = full).
+ * logits_out : device fp32 [B][Hq] or NULL; receives z when non-NULL.
+ * workspace  : device scratch of at least ea_router_workspace_size(...)
+ *              bytes, 256-byte aligned; its contents need no initialisation
+ *              and are overwritten.
+ * Limits: d in {64, 128}; Hkv*d <= 8192; hidden <= 4096; Hq <= 1024.
+ * Pooling sums in fp32 in a fixed order (bit-reproducible run to run).
+ * ---------------------------------------------------------------------- */
+size_t ea_router_workspace_size(int B, int Hkv, int N, int d);
+
+ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d,
+                           const float* w1, const float* b1, int hidden,
+                           const float* w2, const float* b2, int Hq,
+                           float threshold, uint8_t* route_mask,
+                           float* logits_out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fused hybrid prefill attention (Elastic Attention blog §3: the routing
+ * decision enters the kernel as metadata and one launch serves the FA heads
+ * and the SA heads together; §2.1 "结果融合": each head's result lands in
+ * its own slot of the output, which is the concatenation).
+ *
+ * For each (b, h) with r = route_mask[b*Hq + h] and kv head hk = h / (Hq/Hkv):
+ *   visible(i, j) = j <= i                                  if r == 0 (FA)
+ *                 = j <= i && (j < sink || i - j < window)  if r == 1 (SA)
+ *   out[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:].k[b,hk,j,:] | visible) v[b,hk,j,:]
+ * with scale = softmax_scale > 0 ? softmax_scale : 1/sqrt(d).
+ * Square causal prefill: query i and key i are the same position.
+ *
+ * Arithmetic: bf16 operands on the tensor cores, fp32 scores, fp32 online
+ * softmax, P rounded to bf16 for the P.V product, fp32 accumulation, output
+ * rounded to bf16 (round to nearest even).
+ * ---------------------------------------------------------------------- */
+typedef struct ea_attn_params {
+  int B, Hq, Hkv, N, d;
+  int sink;              /* S >= 0 sink tokens seen by SA heads             */
+  int window;            /* W >= 1, the local window including the diagonal */
+  float softmax_scale;   /* <= 0 selects 1/sqrt(d)                          */
+  int select;            /* ea_select                                       */
+} ea_attn_params;
+
+/* Bytes of workspace ea_hybrid_attn_prefill needs (a status word and the
+ * schedule's scratch); 0 if p is invalid. */
+size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p);
+
+/* q, k, v   : device bf16, BHSD as above, 16-byte aligned.
+ * route_mask: device uint8 [B][Hq], 0 = FA, 1 = SA (any nonzero is SA).
+ * p         : host pointer.
+ * out       : device bf16 [B][Hq][N][d]; rows of heads not selected by
+ *             p->select are left untouched.
+ * workspace : device, >= ea_hybrid_attn_workspace_size(p) bytes, ZEROED
+ *             once before its first use; the kernel only ever writes a
+ *             nonzero error code into it (cleared by ea_get_device_status).
+ * Limits: d in {64, 128}; Hq % Hkv == 0; B*Hq <= 4096; N < 2^30.
+ */
+ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
+                                 const uint8_t* route_mask,
+                                 const ea_attn_params* p, void* out,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word kept
+ * in `workspace` (an attention workspace).  *status_out receives EA_OK or
+ * the error a kernel recorded (EA_ERR_TIMEOUT when a bounded device wait ran
+ * out).  Returns EA_ERR_CUDA if the synchronisation or the copy fails. */
+ea_status ea_get_device_status(void* workspace, void* stream, int* status_out);
+
+/* ------------------------------------------------------------------------
+ * Host-side view of the fused kernel's work schedule, for inspection and
+ * tests (no GPU needed).  A unit is (mode, b, h, pair): 256 query rows
+ * [256*pair, 256*pair + 256) of head h in batch b, run by one CTA.  Units
+ * are ordered longest first and dealt to CTAs in a snake order.
+ *
+ * mask        : host uint8 [B][Hq].
+ * units_out   : host int32 [max_units][5] = {sparse, b, h, pair, n_kv_tiles}
+ *               in schedule rank order (may be NULL to only count).
+ * Returns the number of units (>= 0), or -1 on invalid arguments.
+ * ---------------------------------------------------------------------- */
+int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p,
+                      int32_t* units_out, int max_units);
+
+/* The KV tiles (128 keys each) unit `rank` visits, in visiting order, and
+ * per tile and query slot (slot 0: rows 256*pair..+127, slot 1: the next
+ * 128) a code: 0 = skipped, 1 = every pair visible, 2 = needs the element
+ * mask.  tiles_out: host int32 [max_tiles]; codes_out: host int32
+ * [max_tiles][2].  Returns the tile count, or -1 on invalid arguments. */
+int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p,
+                           int rank, int32_t* tiles_out, int32_t* codes_out,
+                           int max_tiles);
+
+/* Number of CTAs the fused kernel launches for these params when the device
+ * has `num_sms` SMs: min(num_sms, B*Hq*ceil(N/256)); 0 if p is invalid.  CTAs
+ * left without units by the mask exit at once. */
+int ea_attn_grid_size(const ea_attn_params* p, int num_sms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EA_H_ */

@@ -57,6 +57,7 @@ __all__ = [
     "router_mlp",
     "router_decide",
     "visible",
+    "visible_spans",
     "visible_keys",
     "attention_rows",
     "attention",
@@ -126,13 +127,23 @@ def visible(i: int, j: int, sparse: bool, sink: int, window: int) -> bool:
     return j < sink or (i - j) < window
 
 
+def visible_spans(i: int, sparse: bool, sink: int, window: int) -> list:
+    """The keys query i sees as sorted, disjoint half-open spans [a, b)."""
+    if not sparse:
+        return [(0, i + 1)]
+    lo = max(0, i - window + 1)
+    spans = []
+    sink_end = min(sink, lo)                       # sink keys left of the window
+    if sink_end > 0:
+        spans.append((0, sink_end))
+    spans.append((lo, i + 1))
+    return spans
+
+
 def visible_keys(i: int, sparse: bool, sink: int, window: int) -> np.ndarray:
     """Sorted indices of the keys query i sees (each key once)."""
-    if not sparse:
-        return np.arange(i + 1)
-    lo = max(0, i - window + 1)
-    sink_part = np.arange(min(sink, lo))          # sink keys left of the window
-    return np.concatenate([sink_part, np.arange(lo, i + 1)])
+    return np.concatenate([np.arange(a, b) for a, b in
+                           visible_spans(i, sparse, sink, window)])
 
 
 def count_visible_pairs(n: int, sparse: bool, sink: int, window: int) -> int:
@@ -172,9 +183,14 @@ def attention_rows(q, k, v, mask, b: int, h: int, rows, sink: int, window: int,
     kh = np.asarray(k[b, hk], dtype=np.float64)
     vh = np.asarray(v[b, hk], dtype=np.float64)
     for r, i in enumerate(rows):
-        keys = visible_keys(int(i), sparse, sink, window)
-        s = (kh[keys] @ qh[i]) * scale
-        out[r] = _softmax_row_weighted(s[None, :], vh[keys])[0]
+        spans = visible_spans(int(i), sparse, sink, window)
+        if len(spans) == 1:
+            kk, vv = kh[spans[0][0]:spans[0][1]], vh[spans[0][0]:spans[0][1]]
+        else:
+            kk = np.concatenate([kh[j0:j1] for j0, j1 in spans])
+            vv = np.concatenate([vh[j0:j1] for j0, j1 in spans])
+        s = (kk @ qh[i]) * scale
+        out[r] = _softmax_row_weighted(s[None, :], vv)[0]
     return out
 
 

@@ -1,0 +1,217 @@
+"""Python binding of the C ABI (include/ea.h), one function per entry point.
+
+Argument marshalling only: PyTorch provides device memory and the current
+CUDA stream; every step of the computation runs in libea.so's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import EA_SELECT_ALL, EA_SELECT_FA, EA_SELECT_SA, EaAttnParams, check  # noqa: F401
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale=0.0,
+                select=EA_SELECT_ALL) -> EaAttnParams:
+    return EaAttnParams(int(B), int(Hq), int(Hkv), int(N), int(d), int(sink), int(window),
+                        float(softmax_scale), int(select))
+
+
+# ---------------------------------------------------------------- router
+def ea_router_workspace_size(B: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib.load().ea_router_workspace_size(B, Hkv, N, d))
+
+
+def ea_router_decide(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+                     b2: torch.Tensor, threshold: float = 0.0, *,
+                     workspace: Optional[torch.Tensor] = None,
+                     route_mask: Optional[torch.Tensor] = None,
+                     logits: Optional[torch.Tensor] = None, want_logits: bool = True,
+                     stream: Optional[torch.cuda.Stream] = None
+                     ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Route mask uint8 [B, Hq] (1 = sparse) and logits fp32 [B, Hq]."""
+    lib = _lib.load()
+    _need(k, "k", torch.bfloat16, 4)
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+        _need(t, name, torch.float32, nd)
+    B, Hkv, N, d = k.shape
+    hidden = w1.shape[0]
+    Hq = w2.shape[0]
+    if w1.shape[1] != Hkv * d or b1.shape[0] != hidden or w2.shape[1] != hidden \
+            or b2.shape[0] != Hq:
+        raise ValueError("router weight shapes do not match the key states")
+    dev = k.device
+    need = lib.ea_router_workspace_size(B, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if route_mask is None:
+        route_mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+    if logits is None and want_logits:
+        logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    rc = lib.ea_router_decide(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(), hidden,
+                              w2.data_ptr(), b2.data_ptr(), Hq, float(threshold),
+                              route_mask.data_ptr(),
+                              logits.data_ptr() if logits is not None else None,
+                              workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
+    check(rc, "ea_router_decide")
+    return route_mask, logits
+
+
+# ---------------------------------------------------------------- attention
+def ea_hybrid_attn_workspace_size(p: EaAttnParams) -> int:
+    return int(_lib.load().ea_hybrid_attn_workspace_size(ctypes.byref(p)))
+
+
+def attn_workspace(p: EaAttnParams, device) -> torch.Tensor:
+    """A zeroed attention workspace (the status word starts at 0)."""
+    n = ea_hybrid_attn_workspace_size(p)
+    if n == 0:
+        raise ValueError("invalid attention parameters")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def ea_hybrid_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           route_mask: torch.Tensor, sink: int, window: int, *,
+                           softmax_scale: float = 0.0, select: int = EA_SELECT_ALL,
+                           out: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Fused hybrid prefill attention; returns out bf16 [B, Hq, N, d]."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    if route_mask.numel() != B * Hq:
+        raise ValueError("route_mask must hold B * Hq entries")
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale, select)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if workspace is None:
+        workspace = attn_workspace(p, q.device)
+    rc = lib.ea_hybrid_attn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                    route_mask.data_ptr(), ctypes.byref(p), out.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel(),
+                                    _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill")
+    return out
+
+
+def ea_get_device_status(workspace: torch.Tensor,
+                         stream: Optional[torch.cuda.Stream] = None) -> int:
+    lib = _lib.load()
+    st = ctypes.c_int(0)
+    rc = lib.ea_get_device_status(workspace.data_ptr(), _stream_ptr(stream, workspace.device),
+                                  ctypes.byref(st))
+    check(rc, "ea_get_device_status")
+    return int(st.value)
+
+
+# ---------------------------------------------------------------- schedule view
+def _host_mask(mask) -> np.ndarray:
+    m = mask.detach().cpu().numpy() if isinstance(mask, torch.Tensor) else np.asarray(mask)
+    return np.ascontiguousarray(m.astype(np.uint8).reshape(-1))
+
+
+def ea_schedule_units(mask, p: EaAttnParams) -> np.ndarray:
+    """[U, 5] int32 rows (sparse, b, h, pair, n_kv_tiles) in schedule order."""
+    lib = _lib.load()
+    m = _host_mask(mask)
+    n = lib.ea_schedule_units(m.ctypes.data, ctypes.byref(p), None, 0)
+    if n < 0:
+        raise ValueError("invalid schedule arguments")
+    out = np.zeros((max(n, 1), 5), dtype=np.int32)
+    lib.ea_schedule_units(m.ctypes.data, ctypes.byref(p), out.ctypes.data, n)
+    return out[:n]
+
+
+def ea_schedule_unit_tiles(mask, p: EaAttnParams, rank: int):
+    """(tiles int32 [T], codes int32 [T, 2]) of one unit."""
+    lib = _lib.load()
+    m = _host_mask(mask)
+    cap = (p.N + 127) // 128 + 1
+    tiles = np.zeros(cap, dtype=np.int32)
+    codes = np.zeros((cap, 2), dtype=np.int32)
+    n = lib.ea_schedule_unit_tiles(m.ctypes.data, ctypes.byref(p), int(rank), tiles.ctypes.data,
+                                   codes.ctypes.data, cap)
+    if n < 0:
+        raise ValueError("invalid schedule arguments")
+    return tiles[:n], codes[:n]
+
+
+def ea_attn_grid_size(p: EaAttnParams, num_sms: int) -> int:
+    return int(_lib.load().ea_attn_grid_size(ctypes.byref(p), int(num_sms)))
+
+
+# ---------------------------------------------------------------- host-buffer path
+class HostPrefill:
+    """One layer's prefill from HOST buffers: copies q, k, v (pinned host) to
+    the device, runs ea_router_decide then ea_hybrid_attn_prefill, and copies
+    the output back into a pinned host buffer.  Device buffers are allocated
+    once and reused across calls."""
+
+    def __init__(self, B, Hq, Hkv, N, d, w1, b1, w2, b2, sink, window, device="cuda",
+                 threshold=0.0):
+        self.shape_q = (B, Hq, N, d)
+        self.shape_kv = (B, Hkv, N, d)
+        self.sink, self.window, self.threshold = int(sink), int(window), float(threshold)
+        dev = torch.device(device)
+        self.q = torch.empty(self.shape_q, dtype=torch.bfloat16, device=dev)
+        self.k = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(self.shape_q, dtype=torch.bfloat16, device=dev)
+        self.w1, self.b1 = w1.to(dev).contiguous(), b1.to(dev).contiguous()
+        self.w2, self.b2 = w2.to(dev).contiguous(), b2.to(dev).contiguous()
+        self.mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+        self.rws = torch.empty(max(ea_router_workspace_size(B, Hkv, N, d), 16),
+                               dtype=torch.uint8, device=dev)
+        self.aws = attn_workspace(make_params(B, Hq, Hkv, N, d, sink, window), dev)
+        self.out_host = torch.empty(self.shape_q, dtype=torch.bfloat16, pin_memory=True)
+
+    def h2d_bytes(self) -> int:
+        return (self.q.numel() + self.k.numel() + self.v.numel()) * 2
+
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * 2
+
+    def __call__(self, q_host, k_host, v_host, stream=None):
+        self.q.copy_(q_host, non_blocking=True)
+        self.k.copy_(k_host, non_blocking=True)
+        self.v.copy_(v_host, non_blocking=True)
+        ea_router_decide(self.k, self.w1, self.b1, self.w2, self.b2, self.threshold,
+                         workspace=self.rws, route_mask=self.mask, want_logits=False,
+                         stream=stream)
+        ea_hybrid_attn_prefill(self.q, self.k, self.v, self.mask, self.sink, self.window,
+                               out=self.out, workspace=self.aws, stream=stream)
+        self.out_host.copy_(self.out, non_blocking=True)
+        return self.out_host

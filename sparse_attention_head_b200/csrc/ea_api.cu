@@ -1,0 +1,269 @@
+// ea_api.cu — the C ABI of libea.so: argument checks, TMA descriptor
+// encoding and kernel launches.  See include/ea.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "ea.h"
+#include "ea_internal.h"
+#include "ea_sched.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the attention params; EA_OK if the kernels can run them.
+ea_status check_params(const ea_attn_params* p) {
+  if (!p) return EA_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->N <= 0 || p->d <= 0)
+    return EA_ERR_INVALID_ARG;
+  if (p->sink < 0 || p->window < 1) return EA_ERR_INVALID_ARG;
+  if (p->select < EA_SELECT_ALL || p->select > EA_SELECT_SA) return EA_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return EA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return EA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->Hq > EA_MAX_ENTRIES) return EA_ERR_UNSUPPORTED;
+  if (p->N >= (1 << 30)) return EA_ERR_UNSUPPORTED;
+  if (!(p->softmax_scale <= 0.f) && !(p->softmax_scale > 0.f)) return EA_ERR_INVALID_ARG;  // NaN
+  return EA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 [rows3][n][d] tensor, box 64 x 128 x 1, 128-byte swizzle, OOB -> 0.
+bool encode_bhsd(CUtensorMap* m, const void* ptr, int d, int n, int rows3) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                        static_cast<cuuint64_t>(rows3)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(n)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices && sms[dev]) return sms[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) sms[dev] = n;
+  return n;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long ns = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    double ms = 2000.0;
+    if (const char* e = getenv("EA_WAIT_TIMEOUT_MS")) {
+      double v = atof(e);
+      if (v > 0) ms = v;
+    }
+    ns = static_cast<unsigned long long>(ms * 1e6);
+  });
+  return ns;
+}
+
+constexpr size_t kAttnWorkspace = 256;
+
+}  // namespace
+
+extern "C" {
+
+const char* ea_status_string(int status) {
+  switch (status) {
+    case EA_OK: return "ok";
+    case EA_ERR_INVALID_ARG: return "invalid argument";
+    case EA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case EA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case EA_ERR_CUDA: return "CUDA call failed";
+    case EA_ERR_TIMEOUT: return "device wait timed out";
+    case EA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int ea_version(void) { return (1 << 16) | 0; }
+
+// ------------------------------------------------------------------ router
+size_t ea_router_workspace_size(int B, int Hkv, int N, int d) {
+  if (B <= 0 || Hkv <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+  const int ns = ea::router_num_splits(B, Hkv, N);
+  return static_cast<size_t>(B) * Hkv * ns * d * sizeof(float);
+}
+
+ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                           const float* b1, int hidden, const float* w2, const float* b2,
+                           int Hq, float threshold, uint8_t* route_mask, float* logits_out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k || !w1 || !b1 || !w2 || !b2 || !route_mask) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || hidden <= 0 || Hq <= 0)
+    return EA_ERR_INVALID_ARG;
+  if (threshold != threshold) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192 || hidden > 4096 || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  const size_t need = ea_router_workspace_size(B, Hkv, N, d);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  const int ns = ea::router_num_splits(B, Hkv, N);
+  cudaError_t err = ea::launch_router(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold,
+                                      route_mask, logits_out, static_cast<float*>(workspace), ns,
+                                      static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ attention
+size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p) {
+  return check_params(p) == EA_OK ? kAttnWorkspace : 0;
+}
+
+int ea_attn_grid_size(const ea_attn_params* p, int num_sms) {
+  if (check_params(p) != EA_OK || num_sms <= 0) return 0;
+  const long long units =
+      static_cast<long long>(p->B) * p->Hq * ((p->N + EA_UNIT_ROWS - 1) / EA_UNIT_ROWS);
+  return static_cast<int>(units < num_sms ? units : num_sms);
+}
+
+ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
+                                 const uint8_t* route_mask, const ea_attn_params* p, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (!q || !k || !v || !route_mask || !out) return EA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+
+  ea::AttnArgs args;
+  if (!encode_bhsd(&args.tm_q, q, p->d, p->N, p->B * p->Hq) ||
+      !encode_bhsd(&args.tm_k, k, p->d, p->N, p->B * p->Hkv) ||
+      !encode_bhsd(&args.tm_v, v, p->d, p->N, p->B * p->Hkv))
+    return EA_ERR_CUDA;
+  args.mask = route_mask;
+  args.out = out;
+  args.status = static_cast<int*>(workspace);
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->N;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  const int grid = ea_attn_grid_size(p, sms);
+  cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status ea_get_device_status(void* workspace, void* stream, int* status_out) {
+  if (!workspace || !status_out) return EA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return EA_ERR_CUDA;
+  if (cudaMemcpy(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EA_ERR_CUDA;
+  if (host != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return EA_ERR_CUDA;
+  *status_out = host;
+  return EA_OK;
+}
+
+// ------------------------------------------------------------------ schedule view
+static int count_entries(const uint8_t* mask, const ea_attn_params* p, int* nfa, int* nsa,
+                         int* ent) {
+  const int BH = p->B * p->Hq;
+  int f = 0, s = 0;
+  for (int i = 0; i < BH; ++i)
+    if (!mask[i] && p->select != EA_SELECT_SA) ent[f++] = i;
+  for (int i = 0; i < BH; ++i)
+    if (mask[i] && p->select != EA_SELECT_FA) ent[f + s++] = i;
+  *nfa = f;
+  *nsa = s;
+  return f + s;
+}
+
+int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p, int32_t* units_out,
+                      int max_units) {
+  if (!mask || check_params(p) != EA_OK) return -1;
+  static thread_local int ent[EA_MAX_ENTRIES];
+  int nfa, nsa;
+  count_entries(mask, p, &nfa, &nsa, ent);
+  const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
+  const int total = ea_num_units(sh, nfa, nsa);
+  if (units_out) {
+    for (int r = 0; r < total && r < max_units; ++r) {
+      int sparse, e, pair;
+      ea_unit_of_rank(sh, nfa, nsa, r, &sparse, &e, &pair);
+      const int idx = ent[sparse ? nfa + e : e];
+      const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
+      int32_t* u = units_out + 5 * r;
+      u[0] = sparse;
+      u[1] = idx / p->Hq;
+      u[2] = idx % p->Hq;
+      u[3] = pair;
+      u[4] = ut.n;
+    }
+  }
+  return total;
+}
+
+int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int rank,
+                           int32_t* tiles_out, int32_t* codes_out, int max_tiles) {
+  if (!mask || check_params(p) != EA_OK) return -1;
+  static thread_local int ent[EA_MAX_ENTRIES];
+  int nfa, nsa;
+  count_entries(mask, p, &nfa, &nsa, ent);
+  const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
+  const int total = ea_num_units(sh, nfa, nsa);
+  if (rank < 0 || rank >= total) return -1;
+  int sparse, e, pair;
+  ea_unit_of_rank(sh, nfa, nsa, rank, &sparse, &e, &pair);
+  const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
+  for (int i = 0; i < ut.n && i < max_tiles; ++i) {
+    const int t = ea_tile_at(ut, i);
+    if (tiles_out) tiles_out[i] = t;
+    if (codes_out) {
+      codes_out[2 * i] = ea_tile_code(sh, ut, sparse, 0, t);
+      codes_out[2 * i + 1] = ea_tile_code(sh, ut, sparse, 1, t);
+    }
+  }
+  return ut.n;
+}
+
+}  // extern "C"

@@ -1,0 +1,509 @@
+// ea_attn.cu — fused hybrid FA/SA causal prefill attention for sm_100a.
+//
+// Elastic Attention blog (bxzpzcl.cn) §3 "Fused Kernel": the per-head routing
+// decision is passed to the kernel as metadata, and one launch serves the
+// heads routed to Full Attention and those routed to Sparse Attention.  The
+// sparse pattern is streaming attention (S sink keys plus a causal window of
+// W keys including the diagonal); full heads are plain causal attention.
+//
+// Design (one persistent CTA per SM, 10 warps):
+//   warps 0-3  softmax/correction/epilogue of query slot 0 (rows r0..r0+127)
+//   warps 4-7  the same for slot 1 (rows r0+128..r0+255)
+//   warp  8    TMA producer: Q slots once per unit, then K and V tiles of the
+//              unit's tile list through a ring of shared-memory stages
+//   warp  9    tcgen05 issuer (one thread): S_s = Q_s K^T into TMEM, then
+//              O_s += P_s V with P read from TMEM (P overwrites S in place)
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+d)  O1 [384,384+d).
+// The MMA order per tile i is PV0(i), S0(i+1), PV1(i), S1(i+1), so one
+// slot's softmax overlaps the other slot's tensor-core work.
+//
+// Softmax runs one query row per thread in fp32 on the log2 scale.  The row
+// reference max is only moved when a tile's max exceeds it by more than 8
+// (2^8 headroom in fp32/bf16), so most tiles need no O rescale; the final
+// O / l uses the same reference, so the result is unchanged.
+//
+// Every wait is bounded: on timeout the kernel records EA_ERR_TIMEOUT in the
+// status word, every role leaves its loop, in-flight copies and MMAs are
+// drained with bounded waits, TMEM is freed and the CTA exits.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ea.h"
+#include "ea_internal.h"
+#include "ea_ptx.cuh"
+#include "ea_sched.h"
+#include "ea_tmem.cuh"
+
+namespace ea {
+
+template <int D>
+struct AttnCfg {
+  static constexpr int kThreads = 320;
+  static constexpr int kBlockBytes = 128 * 128;             // 128 rows x 64 bf16
+  static constexpr int kDBlocks = D / 64;                   // 128-byte column blocks
+  static constexpr int kTileBytes = 128 * D * 2;            // one Q slot / K / V tile
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  // q_full, q_empty, drain, kv_full[kStages], kv_empty[kStages],
+  // s_full[2], p_full[2], o_done[2], o_empty[2]
+  static constexpr int kNumBars = 3 + 2 * kStages + 8;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, counts
+  static constexpr int kOffEnt = kOffMisc + 64;
+  static constexpr int kSmem = kOffEnt + EA_MAX_ENTRIES * 2 + 1024;  // + alignment slack
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+};
+
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[128]) {
+  tmem_ld128_wait(taddr, r);
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld64_wait(taddr, r);
+}
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[128]) {
+  tmem_st128(taddr, r);
+}
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[64]) {
+  tmem_st64(taddr, r);
+}
+
+struct Bars {
+  uint64_t* q_full;
+  uint64_t* q_empty;
+  uint64_t* drain;
+  uint64_t* kv_full;
+  uint64_t* kv_empty;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_done;
+  uint64_t* o_empty;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sKV = smem + C::kOffKV;
+  uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  Bars bars;
+  bars.q_full = bar_base + 0;
+  bars.q_empty = bar_base + 1;
+  bars.drain = bar_base + 2;
+  bars.kv_full = bar_base + 3;
+  bars.kv_empty = bars.kv_full + C::kStages;
+  bars.s_full = bars.kv_empty + C::kStages;
+  bars.p_full = bars.s_full + 2;
+  bars.o_done = bars.p_full + 2;
+  bars.o_empty = bars.o_done + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int* s_counts = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // nFA, nSA
+  uint16_t* s_ent = reinterpret_cast<uint16_t*>(smem + C::kOffEnt);
+
+  const int BH = args.B * args.Hq;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full, 1);
+    mbar_init(bars.q_empty, 1);
+    mbar_init(bars.drain, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(bars.kv_full + i, 1);
+      mbar_init(bars.kv_empty + i, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bars.s_full + s, 1);
+      mbar_init(bars.p_full + s, 128);
+      mbar_init(bars.o_done + s, 1);
+      mbar_init(bars.o_empty + s, 128);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&args.tm_q);
+    tma_prefetch_desc(&args.tm_k);
+    tma_prefetch_desc(&args.tm_v);
+  }
+  if (warp == 9) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  // Entry lists: FA heads first, then SA heads, each in (b, h) order, filtered
+  // by args.select.  Warp 0 builds them with ballots.
+  if (warp == 0) {
+    int nfa = 0;
+    for (int base = 0; base < BH; base += 32) {
+      int idx = base + lane;
+      bool ok = idx < BH && args.mask[idx] == 0 && args.select != EA_SELECT_SA;
+      unsigned bits = __ballot_sync(0xffffffffu, ok);
+      if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
+      nfa += __popc(bits);
+    }
+    int nsa = 0;
+    for (int base = 0; base < BH; base += 32) {
+      int idx = base + lane;
+      bool ok = idx < BH && args.mask[idx] != 0 && args.select != EA_SELECT_FA;
+      unsigned bits = __ballot_sync(0xffffffffu, ok);
+      if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
+      nsa += __popc(bits);
+    }
+    if (lane == 0) {
+      s_counts[0] = nfa;
+      s_counts[1] = nsa;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = *s_tmem;
+  const int nFA = s_counts[0];
+  const int nSA = s_counts[1];
+  const EaShape shape = ea_make_shape(args.N, args.sink, args.window);
+  const int total = ea_num_units(shape, nFA, nSA);
+  const int G = args.Hq / args.Hkv;
+  const uint64_t tlim = args.timeout_ns;
+  int* status = args.status;
+
+  if (warp == 8) {
+    // ============================================================ producer
+    if (lane == 0) {
+      uint32_t kv_pos = 0;
+      uint32_t n_units = 0;
+      bool ok = true;
+      for (int kk = 0; ok; ++kk) {
+        const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+        if (r < 0) break;
+        int sparse, e, pair;
+        ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+        const int idx = s_ent[sparse ? nFA + e : e];
+        const int b = idx / args.Hq, h = idx % args.Hq;
+        const int kvrow = b * args.Hkv + h / G;
+        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+        if (n_units > 0) {
+          ok = mbar_wait(bars.q_empty, (n_units - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(bars.q_full, ut.nslots * C::kTileBytes);
+        for (int s = 0; s < ut.nslots; ++s)
+          for (int c = 0; c < C::kDBlocks; ++c)
+            tma_load_3d(sQ + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
+                        c * 64, ut.r0 + s * EA_BM, idx);
+        ++n_units;
+        for (int i = 0; i < ut.n && ok; ++i) {
+          const int t = ea_tile_at(ut, i);
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t st = kv_pos % C::kStages;
+            if (kv_pos >= static_cast<uint32_t>(C::kStages)) {
+              ok = mbar_wait(bars.kv_empty + st, ((kv_pos / C::kStages) - 1) & 1, s_abort, status,
+                             tlim, EA_ERR_TIMEOUT);
+              if (!ok) break;
+            }
+            mbar_arrive_expect_tx(bars.kv_full + st, C::kTileBytes);
+            const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
+            for (int c = 0; c < C::kDBlocks; ++c)
+              tma_load_3d(sKV + st * C::kTileBytes + c * C::kBlockBytes, map, bars.kv_full + st,
+                          c * 64, t * EA_BN, kvrow);
+            ++kv_pos;
+          }
+        }
+      }
+      // Drain: every copy this thread issued must land before the CTA exits.
+      const uint32_t nst = kv_pos < static_cast<uint32_t>(C::kStages) ? kv_pos : C::kStages;
+      for (uint32_t p = kv_pos - nst; p < kv_pos; ++p)
+        mbar_wait_drain(bars.kv_full + (p % C::kStages), (p / C::kStages) & 1, 200000000ull);
+      if (n_units > 0) mbar_wait_drain(bars.q_full, (n_units - 1) & 1, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      uint32_t kv_pos = 0;
+      uint32_t n_units = 0;
+      uint32_t p_cnt[2] = {0, 0};
+      uint32_t u_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int kk = 0; ok; ++kk) {
+        const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+        if (r < 0) break;
+        int sparse, e, pair;
+        ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+
+        ok = mbar_wait(bars.q_full, n_units & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        if (!ok) break;
+        ++n_units;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(sQ);
+        const uint32_t kv_base = smem_u32(sKV);
+
+        auto issue_s = [&](int s, uint32_t st) {
+          const uint32_t a0 = q_base + s * C::kTileBytes;
+          const uint32_t b0 = kv_base + st * C::kTileBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::kBlockBytes + (k & 3) * 32;
+            mma_ss(tmem + s * 128, smem_desc_sw128(a0 + off, 16, 1024),
+                   smem_desc_sw128(b0 + off, 16, 1024), C::kIdescS, k > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_pv = [&](int s, uint32_t st, bool acc) {
+          const uint32_t b0 = kv_base + st * C::kTileBytes;
+#pragma unroll
+          for (int k = 0; k < EA_BN / 16; ++k) {
+            mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
+                   smem_desc_sw128(b0 + k * 2048, C::kBlockBytes, 1024), C::kIdescPV,
+                   (acc || k > 0) ? 1u : 0u);
+          }
+        };
+
+        // K of the first tile, then S for every slot that sees it.
+        {
+          const uint32_t st = kv_pos % C::kStages;
+          ok = mbar_wait(bars.kv_full + st, (kv_pos / C::kStages) & 1, s_abort, status, tlim,
+                         EA_ERR_TIMEOUT);
+          if (!ok) break;
+          tc_fence_after();
+          const int t0 = ea_tile_at(ut, 0);
+          for (int s = 0; s < 2; ++s)
+            if (ea_tile_code(shape, ut, sparse, s, t0)) {
+              issue_s(s, st);
+              mma_commit(bars.s_full + s);
+            }
+          mma_commit(bars.kv_empty + st);
+        }
+        bool first_pv[2] = {true, true};
+        for (int i = 0; i < ut.n && ok; ++i) {
+          const uint32_t vpos = kv_pos + 2 * i + 1;
+          const uint32_t vst = vpos % C::kStages;
+          ok = mbar_wait(bars.kv_full + vst, (vpos / C::kStages) & 1, s_abort, status, tlim,
+                         EA_ERR_TIMEOUT);
+          if (!ok) break;
+          const bool has_next = i + 1 < ut.n;
+          uint32_t kst = 0;
+          if (has_next) {
+            const uint32_t kpos = kv_pos + 2 * (i + 1);
+            kst = kpos % C::kStages;
+            ok = mbar_wait(bars.kv_full + kst, (kpos / C::kStages) & 1, s_abort, status, tlim,
+                           EA_ERR_TIMEOUT);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const int t = ea_tile_at(ut, i);
+          const int tn = has_next ? ea_tile_at(ut, i + 1) : 0;
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (ea_tile_code(shape, ut, sparse, s, t)) {
+              ok = mbar_wait(bars.p_full + s, p_cnt[s] & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+              if (!ok) break;
+              ++p_cnt[s];
+              if (first_pv[s]) {
+                if (u_cnt[s] > 0) {
+                  ok = mbar_wait(bars.o_empty + s, (u_cnt[s] - 1) & 1, s_abort, status, tlim,
+                                 EA_ERR_TIMEOUT);
+                  if (!ok) break;
+                }
+                ++u_cnt[s];
+              }
+              tc_fence_after();
+              issue_pv(s, vst, !first_pv[s]);
+              first_pv[s] = false;
+              mma_commit(bars.o_done + s);
+            }
+            if (has_next && ea_tile_code(shape, ut, sparse, s, tn)) {
+              issue_s(s, kst);
+              mma_commit(bars.s_full + s);
+            }
+          }
+          if (!ok) break;
+          mma_commit(bars.kv_empty + vst);
+          if (has_next) mma_commit(bars.kv_empty + kst);
+        }
+        if (!ok) break;
+        mma_commit(bars.q_empty);
+        kv_pos += 2 * ut.n;
+      }
+      // Drain: wait for every MMA this thread issued.
+      mma_commit(bars.drain);
+      mbar_wait_drain(bars.drain, 0, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ softmax
+    const int slot = warp >> 2;
+    const int wq = warp & 3;
+    const int row_local = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + slot * 128;
+    const uint32_t tO = tmem + lane_off + 256 + slot * 128;
+    const float sl2 = args.scale_log2;
+    uint32_t s_cnt = 0;
+    uint32_t pv_cnt = 0;
+    bool ok = true;
+    for (int kk = 0; ok; ++kk) {
+      const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+      if (r < 0) break;
+      int sparse, e, pair;
+      ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+      const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+      if (slot >= ut.nslots) continue;
+      const int idx = s_ent[sparse ? nFA + e : e];
+      const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      bool has_o = false;
+      for (int i = 0; i < ut.n; ++i) {
+        const int t = ea_tile_at(ut, i);
+        const int code = ea_tile_code(shape, ut, sparse, slot, t);
+        if (!code) continue;
+        ok = mbar_wait(bars.s_full + slot, s_cnt & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t raw[128];
+          tmem_ld128_wait(tS, raw);
+#pragma unroll
+          for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(raw[j]);
+        }
+        if (code == 2) {
+          const int c0 = t * EA_BN;
+          // visible key j (local): j <= row - c0, and for SA also
+          // (j < sink - c0 || j >= row - window + 1 - c0)
+          const int lim = row - c0;
+          const int sink_hi = sparse ? args.sink - c0 : 1 << 30;
+          const int win_lo = sparse ? row - args.window + 1 - c0 : -(1 << 30);
+#pragma unroll
+          for (int j = 0; j < 128; ++j) {
+            const bool vis = (j <= lim) && (j < sink_hi || j >= win_lo);
+            if (!vis) x[j] = -INFINITY;
+          }
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, x[j]);
+        const float m_tile = mx * sl2;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (m_tile > m_ref + 8.f) {
+          alpha = ex2_approx(m_ref - m_tile);
+          rescale = has_o && (m_ref != -INFINITY);
+          l *= alpha;
+          m_ref = m_tile;
+        }
+        const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * j], sl2, -msub));
+            const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * j + 1], sl2, -msub));
+            pk[j] = pack_bf16x2(p0, p1);
+            // the row sum uses the bf16 values the P.V product sees, so the
+            // weights applied to V sum to one
+            rs += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        l += rs;
+        if (__any_sync(0xffffffffu, rescale)) {
+          ok = mbar_wait(bars.o_done + slot, (pv_cnt - 1) & 1, s_abort, status, tlim,
+                         EA_ERR_TIMEOUT);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const float a = rescale ? alpha : 1.f;
+          uint32_t o[D];
+          tmem_ld_wait(tO, o);
+#pragma unroll
+          for (int j = 0; j < D; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a);
+          tmem_st(tO, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars.p_full + slot);
+        ++pv_cnt;
+        has_o = true;
+      }
+      if (!ok) break;
+      // Epilogue: O / l -> bf16 -> out[b, h, row, :].
+      ok = mbar_wait(bars.o_done + slot, (pv_cnt - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) +
+                            (static_cast<size_t>(idx) * args.N + row) * D;
+      {
+        uint32_t o[D];
+        tmem_ld_wait(tO, o);
+        if (row < args.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int q = 0; q < D / 8; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              w[j] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * j]) * inv_l,
+                                 __uint_as_float(o[8 * q + 2 * j + 1]) * inv_l);
+            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bars.o_empty + slot);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int attn_smem_bytes(int D) {
+  return D == 128 ? AttnCfg<128>::kSmem : AttnCfg<64>::kSmem;
+}
+
+template <int D>
+static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream) {
+  const int smem = AttnCfg<D>::kSmem;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && !configured[dev]) {
+    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    configured[dev] = 1;
+  }
+  ea_hybrid_attn_kernel<D><<<grid, AttnCfg<D>::kThreads, smem, stream>>>(args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stream) {
+  if (D == 128) return launch_d<128>(args, grid, stream);
+  if (D == 64) return launch_d<64>(args, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ea

@@ -1,0 +1,40 @@
+// ea_internal.h — declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ea {
+
+// Arguments of the fused hybrid attention kernel.  The tensor maps describe
+// q [B*Hq][N][d], k and v [B*Hkv][N][d] (bf16, inner dim d) with a
+// 64 x 128 x 1 box and 128-byte swizzle.
+struct alignas(64) AttnArgs {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  const uint8_t* mask;      // [B*Hq], nonzero = sparse
+  void* out;                // bf16 [B][Hq][N][d]
+  int* status;              // device status word
+  int B, Hq, Hkv, N;
+  int sink, window;
+  float scale_log2;         // softmax scale * log2(e)
+  int select;               // ea_select
+  unsigned long long timeout_ns;
+};
+
+// Dynamic shared memory the kernel for head dim D needs.
+int attn_smem_bytes(int D);
+
+// Launch the fused kernel (D in {64, 128}) with `grid` CTAs.
+cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stream);
+
+// Router: pooled partial sums, then the MLP and the threshold.
+int router_num_splits(int B, int Hkv, int N);
+cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                          const float* b1, int hidden, const float* w2, const float* b2,
+                          int Hq, float threshold, uint8_t* mask, float* logits,
+                          float* partials, int nsplit, cudaStream_t stream);
+
+}  // namespace ea

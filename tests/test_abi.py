@@ -1,0 +1,131 @@
+"""The C-ABI library loads, exports every symbol include/ea.h declares, and
+rejects bad arguments before touching the GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_head_b200 import _lib, build
+from sparse_attention_head_b200.api import make_params
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ea.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(ea_[a-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("ea_router_decide", "ea_hybrid_attn_prefill", "ea_status_string",
+                 "ea_router_workspace_size", "ea_hybrid_attn_workspace_size",
+                 "ea_get_device_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(_lib.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), f"libea.so does not export {n}"
+
+
+def test_library_is_built_for_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH_FLAGS)
+    assert os.path.exists(_lib.LIB_PATH)
+
+
+def test_status_strings(lib):
+    for code in range(0, 7):
+        s = _lib.status_string(code)
+        assert isinstance(s, str) and s
+    assert _lib.status_string(5) == "device wait timed out"
+    assert _lib.status_string(99) == "unknown status"
+    assert lib.ea_version() >> 16 == 1
+
+
+def _attn(lib, p, q=16, k=16, v=16, mask=16, out=16, ws=256, wsbytes=256):
+    return lib.ea_hybrid_attn_prefill(q, k, v, mask, ctypes.byref(p), out, ws, wsbytes, None)
+
+
+def test_attention_argument_errors(lib):
+    good = make_params(1, 4, 2, 512, 64, 16, 128)
+    cases = [
+        (make_params(0, 4, 2, 512, 64, 16, 128), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 3, 512, 64, 16, 128), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 2, 0, 64, 16, 128), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 2, 512, 64, -1, 128), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 2, 512, 64, 16, 0), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 2, 512, 64, 16, 128, select=3), {}, _lib.EA_ERR_INVALID_ARG),
+        (make_params(1, 4, 2, 512, 96, 16, 128), {}, _lib.EA_ERR_UNSUPPORTED),
+        (make_params(2, 4096, 4096, 512, 64, 16, 128), {}, _lib.EA_ERR_UNSUPPORTED),
+        (make_params(1, 4, 2, 512, 64, 16, 128, softmax_scale=float("nan")), {},
+         _lib.EA_ERR_INVALID_ARG),
+        (good, {"q": 0}, _lib.EA_ERR_INVALID_ARG),
+        (good, {"mask": 0}, _lib.EA_ERR_INVALID_ARG),
+        (good, {"out": 0}, _lib.EA_ERR_INVALID_ARG),
+        (good, {"k": 24}, _lib.EA_ERR_MISALIGNED),
+        (good, {"out": 8}, _lib.EA_ERR_MISALIGNED),
+        (good, {"ws": 0}, _lib.EA_ERR_WORKSPACE),
+        (good, {"wsbytes": 4}, _lib.EA_ERR_WORKSPACE),
+    ]
+    for p, kw, want in cases:
+        assert _attn(lib, p, **kw) == want, (p.B, p.Hq, p.Hkv, p.N, p.d, kw)
+    assert lib.ea_hybrid_attn_prefill(16, 16, 16, 16, None, 16, 16, 256, None) == \
+        _lib.EA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(lib):
+    p = make_params(1, 32, 8, 32768, 128, 64, 1024)
+    assert lib.ea_hybrid_attn_workspace_size(ctypes.byref(p)) >= 4
+    bad = make_params(1, 32, 8, 32768, 100, 64, 1024)
+    assert lib.ea_hybrid_attn_workspace_size(ctypes.byref(bad)) == 0
+    n = lib.ea_router_workspace_size(1, 8, 32768, 128)
+    assert n > 0 and n % (128 * 4) == 0
+    assert lib.ea_router_workspace_size(1, 8, 32768, 96) == 0
+
+
+def test_router_argument_errors(lib):
+    def call(k=16, B=1, Hkv=8, N=64, d=128, w1=16, b1=16, hidden=256, w2=16, b2=16, Hq=32,
+             thr=0.0, mask=16, ws=256, wsb=1 << 20):
+        return lib.ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, thr, mask, None,
+                                    ws, wsb, None)
+    assert call(k=0) == _lib.EA_ERR_INVALID_ARG
+    assert call(mask=0) == _lib.EA_ERR_INVALID_ARG
+    assert call(N=0) == _lib.EA_ERR_INVALID_ARG
+    assert call(thr=float("nan")) == _lib.EA_ERR_INVALID_ARG
+    assert call(d=96) == _lib.EA_ERR_UNSUPPORTED
+    assert call(hidden=8192) == _lib.EA_ERR_UNSUPPORTED
+    assert call(hidden=254) == _lib.EA_ERR_UNSUPPORTED
+    assert call(w1=20) == _lib.EA_ERR_MISALIGNED
+    assert call(ws=0) == _lib.EA_ERR_WORKSPACE
+    assert call(wsb=8) == _lib.EA_ERR_WORKSPACE
+
+
+def test_grid_size(lib):
+    p = make_params(1, 4, 2, 512, 64, 16, 128)
+    assert lib.ea_attn_grid_size(ctypes.byref(p), 148) == 8      # 4 heads x 2 units
+    p = make_params(1, 32, 8, 32768, 128, 64, 1024)
+    assert lib.ea_attn_grid_size(ctypes.byref(p), 148) == 148
+
+
+def test_product_path_has_no_oracle_import():
+    """The package never imports the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "sparse_attention_head_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f

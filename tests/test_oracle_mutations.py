@@ -35,8 +35,7 @@ MUTATIONS = {
     "pool_divisor": ("return (total / N)", "return (total / (N - 1))"),
     "pool_flatten_order": ("return (total / N).reshape(B, Hkv * d)",
                            "return (total / N).transpose(0, 2, 1).reshape(B, Hkv * d)"),
-    "sink_double_count": ("sink_part = np.arange(min(sink, lo))",
-                          "sink_part = np.arange(min(sink, i + 1))"),
+    "sink_double_count": ("sink_end = min(sink, lo)", "sink_end = min(sink, i + 1)"),
     "softmax_unnormalised": ("return (e @ vals) / np.sum(e, axis=-1, keepdims=True)",
                              "return (e @ vals)"),
     "sink_ignored_blocked": ("vis &= (jj < sink) | ((ii - jj) < window)",

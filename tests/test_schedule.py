@@ -1,0 +1,147 @@
+"""Host logic of the fused kernel's schedule (no GPU): every selected
+(b, h, query row) is covered by exactly one unit slot, every tile a slot
+needs is visited with the right masking code, units are ordered longest
+first, and the snake deal gives each rank to exactly one CTA."""
+import numpy as np
+import pytest
+
+import oracle
+from sparse_attention_head_b200 import flops
+from sparse_attention_head_b200.api import (ea_schedule_unit_tiles, ea_schedule_units,
+                                            make_params)
+
+
+def brute_codes(N, sparse, S, W, r0, tile):
+    """0/1/2 code of (128-row slot at r0, 128-key tile) from the definition."""
+    rows = [i for i in range(r0, r0 + 128)]
+    keys = range(tile * 128, tile * 128 + 128)
+    any_vis = False
+    all_vis = True
+    for i in rows:
+        for j in keys:
+            v = oracle.visible(i, j, sparse, S, W)
+            if i < N and v:
+                any_vis = True
+            if not v:
+                all_vis = False
+    if not any_vis:
+        return 0
+    return 1 if all_vis else 2
+
+
+CASES = [
+    # B, Hq, Hkv, N, d, S, W, select
+    (1, 4, 2, 512, 64, 16, 128, 0),
+    (1, 4, 2, 300, 64, 0, 1, 0),
+    (2, 4, 1, 700, 128, 130, 200, 0),
+    (1, 2, 2, 1, 64, 5, 3, 0),
+    (1, 4, 4, 1000, 128, 64, 1024, 0),
+    (1, 4, 2, 640, 64, 1, 129, 1),
+    (1, 4, 2, 640, 64, 1, 129, 2),
+    (2, 6, 3, 257, 64, 300, 5, 0),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,S,W,sel", CASES)
+def test_units_cover_rows_once(B, Hq, Hkv, N, d, S, W, sel):
+    rng = np.random.default_rng(N + S + W + sel)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    p = make_params(B, Hq, Hkv, N, d, S, W, select=sel)
+    units = ea_schedule_units(mask, p)
+    covered = np.zeros((B, Hq, N), dtype=np.int32)
+    for sparse, b, h, pair, ntiles in units:
+        assert sparse == mask[b, h]
+        assert sel == 0 or (sel == 1 and not sparse) or (sel == 2 and sparse)
+        r0 = 256 * pair
+        covered[b, h, r0:min(N, r0 + 256)] += 1
+    for b in range(B):
+        for h in range(Hq):
+            selected = sel == 0 or (sel == 1) == (mask[b, h] == 0)
+            want = 1 if selected else 0
+            assert np.all(covered[b, h] == want)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,S,W,sel", CASES)
+def test_unit_tiles_match_definition(B, Hq, Hkv, N, d, S, W, sel):
+    rng = np.random.default_rng(7 * N + S)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    p = make_params(B, Hq, Hkv, N, d, S, W, select=sel)
+    units = ea_schedule_units(mask, p)
+    ntiles_total = (N + 127) // 128
+    seen_kinds = set()
+    for rank, (sparse, b, h, pair, n) in enumerate(units):
+        key = (sparse, pair)
+        if key in seen_kinds:
+            continue
+        seen_kinds.add(key)
+        tiles, codes = ea_schedule_unit_tiles(mask, p, rank)
+        assert len(tiles) == n
+        assert len(set(tiles.tolist())) == n and list(tiles) == sorted(tiles)
+        r0 = 256 * pair
+        for slot in range(2):
+            rs = r0 + 128 * slot
+            for t in range(ntiles_total):
+                want = brute_codes(N, bool(sparse), S, W, rs, t) if rs < N else 0
+                if t in tiles:
+                    got = codes[list(tiles).index(t), slot]
+                    assert got == want, (rank, slot, t)
+                else:
+                    assert want == 0, (rank, slot, t)
+        # every listed tile is needed by some slot
+        assert np.all(codes.max(axis=1) > 0)
+
+
+def test_order_longest_first_and_snake_deal():
+    B, Hq, Hkv, N, d, S, W = 1, 32, 8, 32768, 128, 64, 1024
+    mask = np.zeros((B, Hq), np.uint8)
+    mask[0, [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]] = 1
+    p = make_params(B, Hq, Hkv, N, d, S, W)
+    units = ea_schedule_units(mask, p)
+    cost = units[:, 4]
+    sa_cap = max(cost[units[:, 0] == 1])
+    nfa = int((mask == 0).sum())
+    # long FA units first, strictly non-increasing
+    long_fa = units[: nfa * (128 - sa_cap // 2)]
+    assert np.all(long_fa[:, 0] == 0)
+    assert np.all(np.diff(long_fa[:, 4]) <= 0)
+    assert np.all(long_fa[:, 4] > sa_cap)
+    # then SA units, then the short FA units
+    rest = units[len(long_fa):]
+    assert np.all(rest[: 22 * 128, 0] == 1)
+    assert np.all(rest[22 * 128:, 0] == 0)
+    assert np.all(rest[22 * 128:, 4] <= sa_cap)
+    # snake deal: each rank exactly once, loads within one longest unit
+    G = 148
+    total = len(units)
+    owner = -np.ones(total, dtype=np.int64)
+    load = np.zeros(G, dtype=np.int64)
+    for c in range(G):
+        k = 0
+        while True:
+            r = k * G + ((G - 1 - c) if (k & 1) else c)
+            if r >= total:
+                break
+            assert owner[r] == -1
+            owner[r] = c
+            load[c] += cost[r]
+            k += 1
+    assert np.all(owner >= 0)
+    assert load.max() - load.min() <= cost.max()
+
+
+@pytest.mark.parametrize("N,S,W", [(1, 0, 1), (77, 3, 5), (512, 16, 128), (300, 400, 2)])
+def test_pair_counts_match_oracle(N, S, W):
+    for sparse in (False, True):
+        assert flops.attn_visible_pairs(N, sparse, S, W) == \
+            oracle.count_visible_pairs(N, sparse, S, W)
+
+
+def test_effective_and_tile_flops():
+    mask = np.array([[0, 1, 0, 1]], np.uint8)
+    eff = flops.effective_flops(mask, 512, 64, 16, 128)
+    pairs = 2 * oracle.count_visible_pairs(512, False, 16, 128) + \
+        2 * oracle.count_visible_pairs(512, True, 16, 128)
+    assert eff == 4 * 64 * pairs
+    # tile-granular: FA 512 rows -> 1+2+3+4 tiles; SA (S=16, W=128): tiles per
+    # row tile m are {0, m-1, m} -> 1, 2, 3, 3
+    assert flops.tile_flops(mask, 512, 64, 16, 128) == 4 * 64 * 128 * 128 * (2 * 10 + 2 * 9)
