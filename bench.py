@@ -18,6 +18,7 @@ the method) on a bounded sample of the same workload, on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -55,6 +56,8 @@ def parse_args():
                     help="steps of the host-buffer end-to-end measurement (default: --steps)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="override the workload's sequence length (profiling cases)")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
     return ap.parse_args()
@@ -181,11 +184,11 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = workloads.get(args.workload)
+    if args.seq:
+        w = dataclasses.replace(w, seq=args.seq)
     B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
     nlayers = w.layers
-    # qwen8b36-style multi-layer workloads keep one layer resident at a time
-    # per step would need regeneration; here every layer's inputs stay
-    # resident only when they fit in a quarter of the device memory.
+    # every layer's inputs stay resident in HBM (36 x 768 MiB for qwen8b36)
     layers = [make_layer(w, l, rank, dev) for l in range(nlayers)]
     p = make_params(B, Hq, Hkv, N, d, w.sink, w.window)
     aws = attn_workspace(p, dev)
@@ -415,6 +418,8 @@ def cpu_baseline(w, L, mask_np, target_s):
 
 def run_reference(args):
     w = workloads.get(args.workload)
+    if args.seq:
+        w = dataclasses.replace(w, seq=args.seq)
     L = make_layer(w, 0, 0, "cpu")
     if L["router"] is not None:
         import oracle
