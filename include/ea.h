@@ -42,7 +42,9 @@ typedef enum ea_status {
   EA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned            */
   EA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed           */
   EA_ERR_TIMEOUT = 5,       /* a device-side wait ran out (see status)     */
-  EA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required  */
+  EA_ERR_WORKSPACE = 6,     /* workspace missing or smaller than required  */
+  EA_ERR_SCRATCH_LIMIT = 7  /* too large for ea_router_decide_noalloc's
+                               fixed scratch (EA_ROUTER_NOALLOC_MAX_BYTES)  */
 } ea_status;
 
 /* Which heads one attention call computes.  EA_SELECT_ALL is the fused
@@ -91,6 +93,41 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d,
                            float threshold, uint8_t* route_mask,
                            float* logits_out, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * ea_router_decide without a caller-supplied workspace.
+ *
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory at the point they route a layer — code that
+ * runs inside a host framework which owns all device memory and forbids its
+ * plug-ins to call cudaMalloc, or a serving loop that must not allocate
+ * after warm-up because cudaMalloc/cudaFree can synchronise the device and
+ * take the allocator's locks.
+ *
+ * Same inputs, outputs and result bits as ea_router_decide.  The pooling
+ * scratch lives in a fixed device array inside libea.so, of
+ * EA_ROUTER_NOALLOC_MAX_BYTES bytes, which every GPU that loads the library
+ * keeps until the process exits.  A problem whose scratch need,
+ * ea_router_workspace_size(B, Hkv, N, d), exceeds that size is rejected with
+ * EA_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *
+ * The first call on a device looks up that device's copy of the array (a
+ * runtime symbol query, no allocation), so make the first call on each
+ * device before any stream capture.  The entry point never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *
+ * All calls on one device share the array: two calls whose work overlaps on
+ * the GPU (different streams, no ordering between them) race on it and give
+ * undefined results.  Calls ordered on one stream are safe; each call
+ * overwrites every scratch value it reads, so stale contents never matter.
+ * ---------------------------------------------------------------------- */
+#define EA_ROUTER_NOALLOC_MAX_BYTES (1u << 20)
+
+ea_status ea_router_decide_noalloc(const void* k, int B, int Hkv, int N, int d,
+                                   const float* w1, const float* b1, int hidden,
+                                   const float* w2, const float* b2, int Hq,
+                                   float threshold, uint8_t* route_mask,
+                                   float* logits_out, void* stream);
 
 /* ------------------------------------------------------------------------
  * Fused hybrid prefill attention (Elastic Attention blog §3: the routing

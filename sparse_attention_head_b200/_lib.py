@@ -19,6 +19,10 @@ EA_ERR_MISALIGNED = 3
 EA_ERR_CUDA = 4
 EA_ERR_TIMEOUT = 5
 EA_ERR_WORKSPACE = 6
+EA_ERR_SCRATCH_LIMIT = 7
+
+# bytes of the fixed device scratch behind ea_router_decide_noalloc
+EA_ROUTER_NOALLOC_MAX_BYTES = 1 << 20
 
 EA_SELECT_ALL = 0
 EA_SELECT_FA = 1
@@ -26,7 +30,7 @@ EA_SELECT_SA = 2
 
 EXPORTED = [
     "ea_status_string", "ea_version",
-    "ea_router_workspace_size", "ea_router_decide",
+    "ea_router_workspace_size", "ea_router_decide", "ea_router_decide_noalloc",
     "ea_hybrid_attn_workspace_size", "ea_hybrid_attn_prefill",
     "ea_get_device_status", "ea_schedule_units", "ea_schedule_unit_tiles",
     "ea_attn_grid_size",
@@ -74,6 +78,9 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_router_decide.restype = c_int
     lib.ea_router_decide.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp,
                                      c_int, c_float, vp, vp, vp, c_size, vp]
+    lib.ea_router_decide_noalloc.restype = c_int
+    lib.ea_router_decide_noalloc.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, c_int, vp,
+                                             vp, c_int, c_float, vp, vp, vp]
     lib.ea_hybrid_attn_workspace_size.restype = c_size
     lib.ea_hybrid_attn_workspace_size.argtypes = [pparams]
     lib.ea_hybrid_attn_prefill.restype = c_int

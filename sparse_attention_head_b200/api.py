@@ -79,6 +79,28 @@ def ea_router_decide(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: to
     return route_mask, logits
 
 
+def ea_router_decide_noalloc(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
+                             w2: torch.Tensor, b2: torch.Tensor, threshold: float = 0.0, *,
+                             route_mask: torch.Tensor, logits: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> None:
+    """The router without a workspace argument, for callers that cannot
+    allocate device memory when they route a layer (its scratch is a fixed
+    array inside libea.so).  The caller passes the output buffers; this
+    wrapper allocates nothing either."""
+    lib = _lib.load()
+    _need(k, "k", torch.bfloat16, 4)
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+        _need(t, name, torch.float32, nd)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hkv, N, d = k.shape
+    rc = lib.ea_router_decide_noalloc(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(),
+                                      w1.shape[0], w2.data_ptr(), b2.data_ptr(), w2.shape[0],
+                                      float(threshold), route_mask.data_ptr(),
+                                      logits.data_ptr() if logits is not None else None,
+                                      _stream_ptr(stream, k.device))
+    check(rc, "ea_router_decide_noalloc")
+
+
 # ---------------------------------------------------------------- attention
 def ea_hybrid_attn_workspace_size(p: EaAttnParams) -> int:
     return int(_lib.load().ea_hybrid_attn_workspace_size(ctypes.byref(p)))

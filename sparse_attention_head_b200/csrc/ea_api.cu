@@ -108,6 +108,7 @@ const char* ea_status_string(int status) {
     case EA_ERR_CUDA: return "CUDA call failed";
     case EA_ERR_TIMEOUT: return "device wait timed out";
     case EA_ERR_WORKSPACE: return "workspace missing or too small";
+    case EA_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }

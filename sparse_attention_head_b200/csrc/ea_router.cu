@@ -20,6 +20,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
+#include "ea.h"
 #include "ea_internal.h"
 
 namespace ea {
@@ -166,3 +169,49 @@ cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const flo
 }
 
 }  // namespace ea
+
+// ---------------------------------------------------------------------------
+// ea_router_decide_noalloc: the router for callers that cannot allocate.
+//
+// The pooling partial sums go to a fixed array that lives in this library's
+// device image instead of a caller-supplied workspace.  Host code must not
+// pass the array's name to a kernel: on the host it only stands for the
+// symbol, not a device address.  The device address is looked up once per
+// device with cudaGetSymbolAddress while that device is current.
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_router_noalloc_scratch[EA_ROUTER_NOALLOC_MAX_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {nullptr};
+
+// Device address of this device's scratch array, or nullptr on failure.
+void* noalloc_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_router_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" ea_status ea_router_decide_noalloc(const void* k, int B, int Hkv, int N, int d,
+                                              const float* w1, const float* b1, int hidden,
+                                              const float* w2, const float* b2, int Hq,
+                                              float threshold, uint8_t* route_mask,
+                                              float* logits_out, void* stream) {
+  const size_t need = ea_router_workspace_size(B, Hkv, N, d);
+  if (need > EA_ROUTER_NOALLOC_MAX_BYTES) return EA_ERR_SCRATCH_LIMIT;
+  if (need == 0) return ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold,
+                                         route_mask, logits_out, nullptr, 0, stream);
+  void* scratch = noalloc_scratch_for_current_device();
+  if (!scratch) return EA_ERR_CUDA;
+  return ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold, route_mask,
+                          logits_out, scratch, EA_ROUTER_NOALLOC_MAX_BYTES, stream);
+}
