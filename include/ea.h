@@ -80,8 +80,9 @@ int ea_version(void);
  * route_mask : device uint8 [B][Hq], written (1 = sparse, 0 = full).
  * logits_out : device fp32 [B][Hq] or NULL; receives z when non-NULL.
  * workspace  : device scratch of at least ea_router_workspace_size(...)
- *              bytes, 256-byte aligned; its contents need no initialisation
- *              and are overwritten.
+ *              bytes (pooled partial sums, the pooled vector and the hidden
+ *              activations), 16-byte aligned; its contents need no
+ *              initialisation and are overwritten.
  * Limits: d in {64, 128}; Hkv*d <= 8192; hidden <= 4096; Hq <= 1024.
  * Pooling sums in fp32 in a fixed order (bit-reproducible run to run).
  * ---------------------------------------------------------------------- */

@@ -94,6 +94,7 @@ unsigned long long wait_timeout_ns() {
 }
 
 constexpr size_t kAttnWorkspace = 256;
+constexpr int kRouterMaxHidden = 4096;
 
 }  // namespace
 
@@ -116,10 +117,11 @@ const char* ea_status_string(int status) {
 int ea_version(void) { return (1 << 16) | 0; }
 
 // ------------------------------------------------------------------ router
+// Pooled partial sums, the pooled vector x and the hidden activations h (sized
+// for the largest supported hidden width, so the size does not depend on it).
 size_t ea_router_workspace_size(int B, int Hkv, int N, int d) {
   if (B <= 0 || Hkv <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
-  const int ns = ea::router_num_splits(B, Hkv, N);
-  return static_cast<size_t>(B) * Hkv * ns * d * sizeof(float);
+  return ea::router_workspace_bytes(B, Hkv, N, d, kRouterMaxHidden);
 }
 
 ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const float* w1,
@@ -131,7 +133,7 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const fl
     return EA_ERR_INVALID_ARG;
   if (threshold != threshold) return EA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
-  if (Hkv * d > 8192 || hidden > 4096 || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
   if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
   if (!aligned16(k) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
   const size_t need = ea_router_workspace_size(B, Hkv, N, d);

@@ -6,13 +6,17 @@
 // sparse pattern is streaming attention (S sink keys plus a causal window of
 // W keys including the diagonal); full heads are plain causal attention.
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 12 warps = 3 warpgroups):
 //   warps 0-3  softmax/correction/epilogue of query slot 0 (rows r0..r0+127)
 //   warps 4-7  the same for slot 1 (rows r0+128..r0+255)
 //   warp  8    TMA producer: Q slots once per unit, then K and V tiles of the
 //              unit's tile list through a ring of shared-memory stages
 //   warp  9    tcgen05 issuer (one thread): S_s = Q_s K^T into TMEM, then
 //              O_s += P_s V with P read from TMEM (P overwrites S in place)
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: launched at 168 per thread (384 x 168 = 64512); the third
+// warpgroup drops to 120 and the two softmax warpgroups rise to 192
+// (2 x 128 x 192 + 128 x 120 = 64512).
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+d)  O1 [384,384+d).
 // The MMA order per tile i is PV0(i), S0(i+1), PV1(i), S1(i+1), so one
 // slot's softmax overlaps the other slot's tensor-core work.
@@ -32,15 +36,22 @@
 
 #include "ea.h"
 #include "ea_internal.h"
+#include "ea_math.cuh"
 #include "ea_ptx.cuh"
 #include "ea_sched.h"
 #include "ea_tmem.cuh"
 
 namespace ea {
 
+// Of every 8 exp2 pairs of a score row, this many run as a polynomial on the
+// FMA pipe instead of the MUFU (the two units then share the work).
+constexpr int kEmuPairs = 0;
+
 template <int D>
 struct AttnCfg {
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegsSoftmax = 192;
+  static constexpr uint32_t kRegsOther = 120;
   static constexpr int kBlockBytes = 128 * 128;             // 128 rows x 64 bf16
   static constexpr int kDBlocks = D / 64;                   // 128-byte column blocks
   static constexpr int kTileBytes = 128 * D * 2;            // one Q slot / K / V tile
@@ -58,33 +69,22 @@ struct AttnCfg {
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
 };
 
-__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[128]) {
-  tmem_ld128_wait(taddr, r);
-}
-__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[64]) {
-  tmem_ld64_wait(taddr, r);
-}
-__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[128]) {
-  tmem_st128(taddr, r);
-}
-__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[64]) {
-  tmem_st64(taddr, r);
-}
-
+// Shared-memory addresses (32-bit) of the kernel's mbarriers; the arrays
+// (kv_full, kv_empty, s_full, ...) are consecutive 8-byte barriers.
 struct Bars {
-  uint64_t* q_full;
-  uint64_t* q_empty;
-  uint64_t* drain;
-  uint64_t* kv_full;
-  uint64_t* kv_empty;
-  uint64_t* s_full;
-  uint64_t* p_full;
-  uint64_t* o_done;
-  uint64_t* o_empty;
+  uint32_t q_full;
+  uint32_t q_empty;
+  uint32_t drain;
+  uint32_t kv_full;
+  uint32_t kv_empty;
+  uint32_t s_full;
+  uint32_t p_full;
+  uint32_t o_done;
+  uint32_t o_empty;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
+__global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -97,15 +97,18 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
   uint8_t* sKV = smem + C::kOffKV;
   uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   Bars bars;
-  bars.q_full = bar_base + 0;
-  bars.q_empty = bar_base + 1;
-  bars.drain = bar_base + 2;
-  bars.kv_full = bar_base + 3;
-  bars.kv_empty = bars.kv_full + C::kStages;
-  bars.s_full = bars.kv_empty + C::kStages;
-  bars.p_full = bars.s_full + 2;
-  bars.o_done = bars.p_full + 2;
-  bars.o_empty = bars.o_done + 2;
+  {
+    const uint32_t b0 = smem_u32(bar_base);
+    bars.q_full = b0;
+    bars.q_empty = b0 + 8;
+    bars.drain = b0 + 16;
+    bars.kv_full = b0 + 24;
+    bars.kv_empty = bars.kv_full + 8 * C::kStages;
+    bars.s_full = bars.kv_empty + 8 * C::kStages;
+    bars.p_full = bars.s_full + 16;
+    bars.o_done = bars.p_full + 16;
+    bars.o_empty = bars.o_done + 16;
+  }
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_counts = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // nFA, nSA
@@ -115,18 +118,20 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    mbar_init(bars.q_full, 1);
-    mbar_init(bars.q_empty, 1);
-    mbar_init(bars.drain, 1);
+    // bar_base layout: q_full, q_empty, drain, kv_full[kStages],
+    // kv_empty[kStages], s_full[2], p_full[2], o_done[2], o_empty[2]
+    mbar_init(bar_base + 0, 1);                        // q_full: producer
+    mbar_init(bar_base + 1, 1);                        // q_empty: MMA issuer
+    mbar_init(bar_base + 2, 1);                        // drain: MMA issuer
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(bars.kv_full + i, 1);
-      mbar_init(bars.kv_empty + i, 1);
+      mbar_init(bar_base + 3 + i, 1);                  // kv_full: producer
+      mbar_init(bar_base + 3 + C::kStages + i, 1);     // kv_empty: MMA issuer
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bars.s_full + s, 1);
-      mbar_init(bars.p_full + s, 128);
-      mbar_init(bars.o_done + s, 1);
-      mbar_init(bars.o_empty + s, 128);
+      mbar_init(bar_base + 3 + 2 * C::kStages + s, 1);        // s_full
+      mbar_init(bar_base + 3 + 2 * C::kStages + 2 + s, 128);  // p_full
+      mbar_init(bar_base + 3 + 2 * C::kStages + 4 + s, 1);    // o_done
+      mbar_init(bar_base + 3 + 2 * C::kStages + 6 + s, 128);  // o_empty
     }
     *s_abort = 0;
     fence_mbar_init();
@@ -177,7 +182,11 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
   const uint64_t tlim = args.timeout_ns;
   int* status = args.status;
 
-  if (warp == 8) {
+  static_assert(2 * 128 * C::kRegsSoftmax + 128 * C::kRegsOther <= 384 * 168,
+                "register split exceeds the launch budget");
+  if (warp >= 8) {
+    regs_dec<C::kRegsOther>();
+    if (warp == 8) {
     // ============================================================ producer
     if (lane == 0) {
       uint32_t kv_pos = 0;
@@ -199,7 +208,7 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
         mbar_arrive_expect_tx(bars.q_full, ut.nslots * C::kTileBytes);
         for (int s = 0; s < ut.nslots; ++s)
           for (int c = 0; c < C::kDBlocks; ++c)
-            tma_load_3d(sQ + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
+            tma_load_3d(smem_u32(sQ) + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
                         c * 64, ut.r0 + s * EA_BM, idx);
         ++n_units;
         for (int i = 0; i < ut.n && ok; ++i) {
@@ -207,14 +216,14 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
           for (int which = 0; which < 2; ++which) {
             const uint32_t st = kv_pos % C::kStages;
             if (kv_pos >= static_cast<uint32_t>(C::kStages)) {
-              ok = mbar_wait(bars.kv_empty + st, ((kv_pos / C::kStages) - 1) & 1, s_abort, status,
+              ok = mbar_wait(bars.kv_empty + 8 * st, ((kv_pos / C::kStages) - 1) & 1, s_abort, status,
                              tlim, EA_ERR_TIMEOUT);
               if (!ok) break;
             }
-            mbar_arrive_expect_tx(bars.kv_full + st, C::kTileBytes);
+            mbar_arrive_expect_tx(bars.kv_full + 8 * st, C::kTileBytes);
             const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
             for (int c = 0; c < C::kDBlocks; ++c)
-              tma_load_3d(sKV + st * C::kTileBytes + c * C::kBlockBytes, map, bars.kv_full + st,
+              tma_load_3d(smem_u32(sKV) + st * C::kTileBytes + c * C::kBlockBytes, map, bars.kv_full + 8 * st,
                           c * 64, t * EA_BN, kvrow);
             ++kv_pos;
           }
@@ -223,18 +232,48 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
       // Drain: every copy this thread issued must land before the CTA exits.
       const uint32_t nst = kv_pos < static_cast<uint32_t>(C::kStages) ? kv_pos : C::kStages;
       for (uint32_t p = kv_pos - nst; p < kv_pos; ++p)
-        mbar_wait_drain(bars.kv_full + (p % C::kStages), (p / C::kStages) & 1, 200000000ull);
+        mbar_wait_drain(bars.kv_full + 8 * (p % C::kStages), (p / C::kStages) & 1, 200000000ull);
       if (n_units > 0) mbar_wait_drain(bars.q_full, (n_units - 1) & 1, 200000000ull);
     }
     __syncwarp();
-  } else if (warp == 9) {
+    } else if (warp == 9) {
     // ============================================================ MMA issuer
+    // One thread issues both slots' MMAs in the order PV0(i), S0(i+1),
+    // PV1(i), S1(i+1): each group of eight MMAs is contiguous, and the
+    // tensor pipe always has the other slot's group queued while a softmax
+    // runs.  The pipe's queue is shallow, so the thread keeps everything but
+    // MMAs and the waits they need off this path (K/V waits come from the
+    // async proxy and need no tcgen05 fence; only P handoffs do).
     if (lane == 0) {
       uint32_t kv_pos = 0;
       uint32_t n_units = 0;
       uint32_t p_cnt[2] = {0, 0};
       uint32_t u_cnt[2] = {0, 0};
       bool ok = true;
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t kv_base = smem_u32(sKV);
+      // Descriptors are built once; K steps add their byte offset >> 4 to the
+      // 14-bit start-address field (all of shared memory is below 256 KB, so
+      // the field never overflows).
+      const uint64_t dq = smem_desc_sw128(q_base, 16, 1024);
+      const uint64_t dkv_k = smem_desc_sw128(kv_base, 16, 1024);
+      const uint64_t dkv_v = smem_desc_sw128(kv_base, C::kBlockBytes, 1024);
+      auto issue_s = [&](int s, uint32_t st) {
+        const uint64_t a0 = dq + ((s * C::kTileBytes) >> 4);
+        const uint64_t b0 = dkv_k + ((st * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
+          mma_ss(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int s, uint32_t st, bool acc) {
+        const uint64_t b0 = dkv_v + ((st * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < EA_BN / 16; ++k)
+          mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8, b0 + ((k * 2048) >> 4),
+                 C::kIdescPV, (acc || k > 0) ? 1u : 0u);
+      };
       for (int kk = 0; ok; ++kk) {
         const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
         if (r < 0) break;
@@ -245,50 +284,26 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
         ok = mbar_wait(bars.q_full, n_units & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
         if (!ok) break;
         ++n_units;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ);
-        const uint32_t kv_base = smem_u32(sKV);
-
-        auto issue_s = [&](int s, uint32_t st) {
-          const uint32_t a0 = q_base + s * C::kTileBytes;
-          const uint32_t b0 = kv_base + st * C::kTileBytes;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::kBlockBytes + (k & 3) * 32;
-            mma_ss(tmem + s * 128, smem_desc_sw128(a0 + off, 16, 1024),
-                   smem_desc_sw128(b0 + off, 16, 1024), C::kIdescS, k > 0 ? 1u : 0u);
-          }
-        };
-        auto issue_pv = [&](int s, uint32_t st, bool acc) {
-          const uint32_t b0 = kv_base + st * C::kTileBytes;
-#pragma unroll
-          for (int k = 0; k < EA_BN / 16; ++k) {
-            mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
-                   smem_desc_sw128(b0 + k * 2048, C::kBlockBytes, 1024), C::kIdescPV,
-                   (acc || k > 0) ? 1u : 0u);
-          }
-        };
 
         // K of the first tile, then S for every slot that sees it.
         {
           const uint32_t st = kv_pos % C::kStages;
-          ok = mbar_wait(bars.kv_full + st, (kv_pos / C::kStages) & 1, s_abort, status, tlim,
+          ok = mbar_wait(bars.kv_full + 8 * st, (kv_pos / C::kStages) & 1, s_abort, status, tlim,
                          EA_ERR_TIMEOUT);
           if (!ok) break;
-          tc_fence_after();
           const int t0 = ea_tile_at(ut, 0);
           for (int s = 0; s < 2; ++s)
             if (ea_tile_code(shape, ut, sparse, s, t0)) {
               issue_s(s, st);
-              mma_commit(bars.s_full + s);
+              mma_commit(bars.s_full + 8 * s);
             }
-          mma_commit(bars.kv_empty + st);
+          mma_commit(bars.kv_empty + 8 * st);
         }
         bool first_pv[2] = {true, true};
         for (int i = 0; i < ut.n && ok; ++i) {
           const uint32_t vpos = kv_pos + 2 * i + 1;
           const uint32_t vst = vpos % C::kStages;
-          ok = mbar_wait(bars.kv_full + vst, (vpos / C::kStages) & 1, s_abort, status, tlim,
+          ok = mbar_wait(bars.kv_full + 8 * vst, (vpos / C::kStages) & 1, s_abort, status, tlim,
                          EA_ERR_TIMEOUT);
           if (!ok) break;
           const bool has_next = i + 1 < ut.n;
@@ -296,21 +311,22 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
           if (has_next) {
             const uint32_t kpos = kv_pos + 2 * (i + 1);
             kst = kpos % C::kStages;
-            ok = mbar_wait(bars.kv_full + kst, (kpos / C::kStages) & 1, s_abort, status, tlim,
-                           EA_ERR_TIMEOUT);
+            ok = mbar_wait(bars.kv_full + 8 * kst, (kpos / C::kStages) & 1, s_abort, status,
+                           tlim, EA_ERR_TIMEOUT);
             if (!ok) break;
           }
-          tc_fence_after();
           const int t = ea_tile_at(ut, i);
           const int tn = has_next ? ea_tile_at(ut, i + 1) : 0;
-          for (int s = 0; s < 2 && ok; ++s) {
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
             if (ea_tile_code(shape, ut, sparse, s, t)) {
-              ok = mbar_wait(bars.p_full + s, p_cnt[s] & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+              ok = mbar_wait(bars.p_full + 8 * s, p_cnt[s] & 1, s_abort, status, tlim,
+                             EA_ERR_TIMEOUT);
               if (!ok) break;
               ++p_cnt[s];
               if (first_pv[s]) {
                 if (u_cnt[s] > 0) {
-                  ok = mbar_wait(bars.o_empty + s, (u_cnt[s] - 1) & 1, s_abort, status, tlim,
+                  ok = mbar_wait(bars.o_empty + 8 * s, (u_cnt[s] - 1) & 1, s_abort, status, tlim,
                                  EA_ERR_TIMEOUT);
                   if (!ok) break;
                 }
@@ -319,16 +335,16 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
               tc_fence_after();
               issue_pv(s, vst, !first_pv[s]);
               first_pv[s] = false;
-              mma_commit(bars.o_done + s);
+              mma_commit(bars.o_done + 8 * s);
             }
             if (has_next && ea_tile_code(shape, ut, sparse, s, tn)) {
               issue_s(s, kst);
-              mma_commit(bars.s_full + s);
+              mma_commit(bars.s_full + 8 * s);
             }
           }
           if (!ok) break;
-          mma_commit(bars.kv_empty + vst);
-          if (has_next) mma_commit(bars.kv_empty + kst);
+          mma_commit(bars.kv_empty + 8 * vst);
+          if (has_next) mma_commit(bars.kv_empty + 8 * kst);
         }
         if (!ok) break;
         mma_commit(bars.q_empty);
@@ -339,7 +355,9 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
       mbar_wait_drain(bars.drain, 0, 200000000ull);
     }
     __syncwarp();
+    }
   } else {
+    regs_inc<C::kRegsSoftmax>();
     // ============================================================ softmax
     const int slot = warp >> 2;
     const int wq = warp & 3;
@@ -367,7 +385,7 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
         const int t = ea_tile_at(ut, i);
         const int code = ea_tile_code(shape, ut, sparse, slot, t);
         if (!code) continue;
-        ok = mbar_wait(bars.s_full + slot, s_cnt & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        ok = mbar_wait(bars.s_full + 8 * slot, s_cnt & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++s_cnt;
@@ -392,9 +410,17 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
             if (!vis) x[j] = -INFINITY;
           }
         }
-        float mx = x[0];
+        // row max: eight independent chains of three-input max, then a tree
+        float mk[8];
 #pragma unroll
-        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, x[j]);
+        for (int k = 0; k < 8; ++k) mk[k] = x[k];
+#pragma unroll
+        for (int j = 8; j < 128; j += 16) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], x[j + k], x[j + 8 + k]);
+        }
+        const float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]),
+                               fmaxf(mk[6], mk[7]));
         const float m_tile = mx * sl2;
         bool rescale = false;
         float alpha = 1.f;
@@ -405,57 +431,72 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
           m_ref = m_tile;
         }
         const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs = 0.f;
+        // p = 2^(s * scale * log2e - m): packed FMA, then exp2 on the MUFU for
+        // most pairs and on the FMA pipe for kEmuPairs of every 8 pairs
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * j], sl2, -msub));
-            const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * j + 1], sl2, -msub));
+            float p0, p1;
+            fma2_sc(p0, p1, x[c * 32 + 2 * j], x[c * 32 + 2 * j + 1], sl2, -msub);
+            if ((j & 7) < kEmuPairs) {
+              exp2_poly2(p0, p1);
+            } else {
+              p0 = ex2_approx(p0);
+              p1 = ex2_approx(p1);
+            }
             pk[j] = pack_bf16x2(p0, p1);
-            // the row sum uses the bf16 values the P.V product sees, so the
-            // weights applied to V sum to one
-            rs += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+            // the row sum adds the bf16 values the P.V product sees, so the
+            // weights applied to V sum to one even in rows with few keys
+            add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], __uint_as_float(pk[j] << 16),
+                     __uint_as_float(pk[j] & 0xffff0000u));
           }
           tmem_st16(tS + c * 16, pk);
         }
-        l += rs;
+        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         if (__any_sync(0xffffffffu, rescale)) {
-          ok = mbar_wait(bars.o_done + slot, (pv_cnt - 1) & 1, s_abort, status, tlim,
+          ok = mbar_wait(bars.o_done + 8 * slot, (pv_cnt - 1) & 1, s_abort, status, tlim,
                          EA_ERR_TIMEOUT);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
           const float a = rescale ? alpha : 1.f;
-          uint32_t o[D];
-          tmem_ld_wait(tO, o);
 #pragma unroll
-          for (int j = 0; j < D; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a);
-          tmem_st(tO, o);
+          for (int h = 0; h < D / 64; ++h) {
+            uint32_t o[64];
+            tmem_ld64_wait(tO + h * 64, o);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a);
+            tmem_st64(tO + h * 64, o);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bars.p_full + slot);
+        mbar_arrive(bars.p_full + 8 * slot);
         ++pv_cnt;
         has_o = true;
       }
       if (!ok) break;
       // Epilogue: O / l -> bf16 -> out[b, h, row, :].
-      ok = mbar_wait(bars.o_done + slot, (pv_cnt - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+      ok = mbar_wait(bars.o_done + 8 * slot, (pv_cnt - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) +
                             (static_cast<size_t>(idx) * args.N + row) * D;
-      {
-        uint32_t o[D];
-        tmem_ld_wait(tO, o);
-        if (row < args.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int q = 0; q < D / 8; ++q) {
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t o[64];
+        tmem_ld64_wait(tO + h * 64, o);
+        if (row < args.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + h * 64);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
             uint32_t w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -466,7 +507,7 @@ __global__ void __launch_bounds__(320, 1) ea_hybrid_attn_kernel(const __grid_con
         }
       }
       tc_fence_before();
-      mbar_arrive(bars.o_empty + slot);
+      mbar_arrive(bars.o_empty + 8 * slot);
     }
   }
 

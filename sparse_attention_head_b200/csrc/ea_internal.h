@@ -32,6 +32,7 @@ cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stre
 
 // Router: pooled partial sums, then the MLP and the threshold.
 int router_num_splits(int B, int Hkv, int N);
+size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden);
 cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const float* w1,
                           const float* b1, int hidden, const float* w2, const float* b2,
                           int Hq, float threshold, uint8_t* mask, float* logits,

@@ -12,10 +12,10 @@
 // Kernel 1 (HBM-bound): CTA (split, kv head, batch) sums its chunk of rows
 //   into fp32, 8 channels per thread with 16-byte loads, and reduces the
 //   row groups in a fixed order into partials[b][hk][split][d].
-// Kernel 2: one CTA per batch row sums the partials in split order, divides
-//   by N, runs h = ReLU(W1 x + b1) and z = W2 h + b2 with one warp per output
-//   (fixed shuffle order), writes z and the mask z > threshold.
-// Both kernels are deterministic: the same inputs give the same bits.
+// Kernel 2 sums the partials in split order and divides by N (x); kernels 3
+//   and 4 run h = ReLU(W1 x + b1) and z = W2 h + b2 with one warp per output
+//   spread over many CTAs (fixed shuffle order), and write z and the mask
+//   z > threshold.  All kernels are deterministic: same inputs, same bits.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -69,60 +69,52 @@ __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
   }
 }
 
-__global__ void __launch_bounds__(kMlpThreads) ea_router_mlp_kernel(
-    const float* __restrict__ partials, int Hkv, int N, int d, int nsplit,
-    const float* __restrict__ w1, const float* __restrict__ b1, int hidden,
-    const float* __restrict__ w2, const float* __restrict__ b2, int Hq, float threshold,
-    uint8_t* __restrict__ mask, float* __restrict__ logits) {
-  extern __shared__ float sm[];
-  const int in_dim = Hkv * d;
-  float* x = sm;                 // [in_dim]
-  float* h = sm + in_dim;        // [hidden]
-  const int b = blockIdx.x;
+// x[b][hk*d + c] = (sum over splits, in split order) / N; one thread per channel.
+__global__ void ea_router_reduce_kernel(const float* __restrict__ partials, int Hkv, int N, int d,
+                                        int nsplit, float* __restrict__ x) {
+  const int b = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;   // j = hk * d + c
+  if (j >= Hkv * d) return;
+  const int hk = j / d, c = j % d;
+  const float* p = partials + (static_cast<size_t>(b) * Hkv + hk) * nsplit * d + c;
+  float s = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) s += p[static_cast<size_t>(sp) * d];
+  x[static_cast<size_t>(b) * Hkv * d + j] = s * (1.0f / static_cast<float>(N));
+}
+
+// One warp per output: y[b][o] = act(W[o] . x[b] + bias[o]), float4 over the
+// input, lanes reduced in a fixed shuffle order.  For the last layer the
+// output is the logit z, and the route bit z > threshold is written too.
+template <bool kLast>
+__global__ void __launch_bounds__(kMlpThreads) ea_router_layer_kernel(
+    const float* __restrict__ x, int in_dim, const float* __restrict__ w,
+    const float* __restrict__ bias, int out_dim, float* __restrict__ y, float threshold,
+    uint8_t* __restrict__ mask) {
+  const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = kMlpThreads / 32;
-  const float inv_n = 1.0f / static_cast<float>(N);
-  for (int j = threadIdx.x; j < in_dim; j += kMlpThreads) {
-    const int hk = j / d, c = j % d;
-    const float* p = partials + (static_cast<size_t>(b) * Hkv + hk) * nsplit * d + c;
-    float s = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) s += p[static_cast<size_t>(sp) * d];
-    x[j] = s * inv_n;
+  const int o = blockIdx.x * (kMlpThreads / 32) + warp;
+  if (o >= out_dim) return;
+  const float4* wr = reinterpret_cast<const float4*>(w + static_cast<size_t>(o) * in_dim);
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * in_dim);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int j = lane; j < in_dim / 4; j += 32) {
+    const float4 wv = __ldg(wr + j);
+    const float4 xv = xr[j];
+    acc = fmaf(wv.x, xv.x, acc);
+    acc = fmaf(wv.y, xv.y, acc);
+    acc = fmaf(wv.z, xv.z, acc);
+    acc = fmaf(wv.w, xv.w, acc);
   }
-  __syncthreads();
-  // layer 1: one warp per hidden unit, float4 over the input
-  for (int o = warp; o < hidden; o += nwarps) {
-    const float4* wr = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(o) * in_dim);
-    float acc = 0.f;
-    for (int j = lane; j < in_dim / 4; j += 32) {
-      const float4 w = __ldg(wr + j);
-      acc = fmaf(w.x, x[4 * j], acc);
-      acc = fmaf(w.y, x[4 * j + 1], acc);
-      acc = fmaf(w.z, x[4 * j + 2], acc);
-      acc = fmaf(w.w, x[4 * j + 3], acc);
-    }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) h[o] = fmaxf(acc + b1[o], 0.f);
-  }
-  __syncthreads();
-  // layer 2: one warp per head
-  for (int q = warp; q < Hq; q += nwarps) {
-    const float4* wr = reinterpret_cast<const float4*>(w2 + static_cast<size_t>(q) * hidden);
-    float acc = 0.f;
-    for (int j = lane; j < hidden / 4; j += 32) {
-      const float4 w = __ldg(wr + j);
-      acc = fmaf(w.x, h[4 * j], acc);
-      acc = fmaf(w.y, h[4 * j + 1], acc);
-      acc = fmaf(w.z, h[4 * j + 2], acc);
-      acc = fmaf(w.w, h[4 * j + 3], acc);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      const float z = acc + b2[q];
-      mask[static_cast<size_t>(b) * Hq + q] = (z > threshold) ? 1 : 0;
-      if (logits) logits[static_cast<size_t>(b) * Hq + q] = z;
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    const float v = acc + bias[o];
+    if (kLast) {
+      if (y) y[static_cast<size_t>(b) * out_dim + o] = v;
+      mask[static_cast<size_t>(b) * out_dim + o] = (v > threshold) ? 1 : 0;
+    } else {
+      y[static_cast<size_t>(b) * out_dim + o] = fmaxf(v, 0.f);
     }
   }
 }
@@ -137,11 +129,22 @@ int router_num_splits(int B, int Hkv, int N) {
   return per;
 }
 
+size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden) {
+  const int ns = router_num_splits(B, Hkv, N);
+  const size_t parts = static_cast<size_t>(B) * Hkv * ns * d;
+  const size_t x = static_cast<size_t>(B) * Hkv * d;
+  const size_t h = static_cast<size_t>(B) * hidden;
+  return (parts + x + h) * sizeof(float);
+}
+
 cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const float* w1,
                           const float* b1, int hidden, const float* w2, const float* b2,
                           int Hq, float threshold, uint8_t* mask, float* logits,
                           float* partials, int nsplit, cudaStream_t stream) {
   const int chunk = (N + nsplit - 1) / nsplit;
+  const int in_dim = Hkv * d;
+  float* xbuf = partials + static_cast<size_t>(B) * Hkv * nsplit * d;
+  float* hbuf = xbuf + static_cast<size_t>(B) * in_dim;
   dim3 grid(nsplit, Hkv, B);
   if (d == 128)
     ea_router_pool_kernel<128><<<grid, kPoolThreads, 0, stream>>>(
@@ -151,20 +154,17 @@ cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const flo
         static_cast<const __nv_bfloat16*>(k), N, nsplit, chunk, partials);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const size_t smem = static_cast<size_t>(Hkv * d + hidden) * sizeof(float);
-  static int configured[64] = {0};
-  int dev = 0;
-  err = cudaGetDevice(&dev);
+  ea_router_reduce_kernel<<<dim3((in_dim + 255) / 256, B), 256, 0, stream>>>(partials, Hkv, N,
+                                                                             d, nsplit, xbuf);
+  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  if (smem > 48 * 1024 && dev < 64 && !configured[dev]) {
-    err = cudaFuncSetAttribute(ea_router_mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (8192 + 4096) * static_cast<int>(sizeof(float)));
-    if (err != cudaSuccess) return err;
-    configured[dev] = 1;
-  }
-  ea_router_mlp_kernel<<<B, kMlpThreads, smem, stream>>>(partials, Hkv, N, d, nsplit, w1, b1,
-                                                         hidden, w2, b2, Hq, threshold, mask,
-                                                         logits);
+  constexpr int kWarps = kMlpThreads / 32;
+  ea_router_layer_kernel<false><<<dim3((hidden + kWarps - 1) / kWarps, B), kMlpThreads, 0,
+                                  stream>>>(xbuf, in_dim, w1, b1, hidden, hbuf, 0.f, nullptr);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ea_router_layer_kernel<true><<<dim3((Hq + kWarps - 1) / kWarps, B), kMlpThreads, 0,
+                                 stream>>>(hbuf, hidden, w2, b2, Hq, logits, threshold, mask);
   return cudaGetLastError();
 }
 
