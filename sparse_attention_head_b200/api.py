@@ -198,12 +198,14 @@ def ea_attn_grid_size(p: EaAttnParams, num_sms: int) -> int:
 # ---------------------------------------------------------------- host-buffer path
 class HostPrefill:
     """One layer's prefill from HOST buffers: copies q, k, v (pinned host) to
-    the device, runs ea_router_decide then ea_hybrid_attn_prefill, and copies
-    the output back into a pinned host buffer.  Device buffers are allocated
-    once and reused across calls."""
+    the device, runs ea_router_decide (or, with no router weights, copies the
+    caller's route mask) then ea_hybrid_attn_prefill, and copies the output
+    back into a pinned host buffer.  Device buffers are allocated once and
+    reused across calls."""
 
     def __init__(self, B, Hq, Hkv, N, d, w1, b1, w2, b2, sink, window, device="cuda",
                  threshold=0.0):
+        self.has_router = w1 is not None
         self.shape_q = (B, Hq, N, d)
         self.shape_kv = (B, Hkv, N, d)
         self.sink, self.window, self.threshold = int(sink), int(window), float(threshold)
@@ -212,8 +214,9 @@ class HostPrefill:
         self.k = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
         self.v = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
         self.out = torch.empty(self.shape_q, dtype=torch.bfloat16, device=dev)
-        self.w1, self.b1 = w1.to(dev).contiguous(), b1.to(dev).contiguous()
-        self.w2, self.b2 = w2.to(dev).contiguous(), b2.to(dev).contiguous()
+        if self.has_router:
+            self.w1, self.b1 = w1.to(dev).contiguous(), b1.to(dev).contiguous()
+            self.w2, self.b2 = w2.to(dev).contiguous(), b2.to(dev).contiguous()
         self.mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
         self.rws = torch.empty(max(ea_router_workspace_size(B, Hkv, N, d), 16),
                                dtype=torch.uint8, device=dev)
@@ -221,18 +224,22 @@ class HostPrefill:
         self.out_host = torch.empty(self.shape_q, dtype=torch.bfloat16, pin_memory=True)
 
     def h2d_bytes(self) -> int:
-        return (self.q.numel() + self.k.numel() + self.v.numel()) * 2
+        n = (self.q.numel() + self.k.numel() + self.v.numel()) * 2
+        return n if self.has_router else n + self.mask.numel()
 
     def d2h_bytes(self) -> int:
         return self.out.numel() * 2
 
-    def __call__(self, q_host, k_host, v_host, stream=None):
+    def __call__(self, q_host, k_host, v_host, mask_host=None, stream=None):
         self.q.copy_(q_host, non_blocking=True)
         self.k.copy_(k_host, non_blocking=True)
         self.v.copy_(v_host, non_blocking=True)
-        ea_router_decide(self.k, self.w1, self.b1, self.w2, self.b2, self.threshold,
-                         workspace=self.rws, route_mask=self.mask, want_logits=False,
-                         stream=stream)
+        if self.has_router:
+            ea_router_decide(self.k, self.w1, self.b1, self.w2, self.b2, self.threshold,
+                             workspace=self.rws, route_mask=self.mask, want_logits=False,
+                             stream=stream)
+        else:
+            self.mask.copy_(mask_host.reshape(self.mask.shape), non_blocking=True)
         ea_hybrid_attn_prefill(self.q, self.k, self.v, self.mask, self.sink, self.window,
                                out=self.out, workspace=self.aws, stream=stream)
         self.out_host.copy_(self.out, non_blocking=True)
