@@ -157,9 +157,24 @@ def traffic_for_current_kernel():
     return d.get("dram_bytes_per_launch_full_workload")
 
 
+# ---------------------------------------------------------------- ranks
+def rank_seed(w: workloads.Workload, layer: int, rank: int) -> int:
+    """Each rank runs its own replica of the workload with its own inputs."""
+    return workloads.layer_seed(w, layer) + 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time (every rank takes part; no-op on one rank)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- inputs
 def make_layer(w: workloads.Workload, layer: int, rank: int, device):
-    seed = workloads.layer_seed(w, layer) + 7919 * rank
+    seed = rank_seed(w, layer, rank)
     q, k, v = workloads.make_qkv(w, seed, device=device)
     if w.use_router:
         frac = workloads.layer_sparse_frac(w, layer)
@@ -247,10 +262,7 @@ def run_ours(args, rank, world, local_rank):
     attn_ms = [evs[i][l][1].elapsed_time(evs[i][l][2]) for i in range(K) for l in range(nlayers)]
     router_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K)
                  for l in range(nlayers)]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     if ea_get_device_status(aws) != 0:
         raise RuntimeError("device status word reports an error after the timed region")
 
@@ -435,7 +447,8 @@ def run_reference(args):
         Lc = host_layer(L)
         mask_np = L["mask"].numpy()
     rng = np.random.default_rng(11)
-    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    # each step is a bounded sample; the whole run stays within about two minutes
+    per_step = max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, Lc, mask_np, per_step * 0.25, rng)
     tot_fl, tot_s = 0.0, 0.0

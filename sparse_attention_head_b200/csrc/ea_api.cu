@@ -93,6 +93,17 @@ unsigned long long wait_timeout_ns() {
   return ns;
 }
 
+// EA_DEBUG_DROP_KV_POS=<n> makes the attention producer skip K/V ring
+// position n of every CTA (a test of the bounded waits; off by default).
+int debug_drop_kv_pos() {
+  static int pos = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (const char* e = getenv("EA_DEBUG_DROP_KV_POS")) pos = atoi(e);
+  });
+  return pos;
+}
+
 constexpr size_t kAttnWorkspace = 256;
 constexpr int kRouterMaxHidden = 4096;
 
@@ -187,6 +198,7 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   args.scale_log2 = scale * 1.4426950408889634f;
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = debug_drop_kv_pos();
 
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;

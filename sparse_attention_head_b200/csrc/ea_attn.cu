@@ -220,6 +220,10 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                              tlim, EA_ERR_TIMEOUT);
               if (!ok) break;
             }
+            if (static_cast<int>(kv_pos) == args.debug_drop_kv_pos) {
+              ++kv_pos;           // test hook: this copy never happens
+              continue;
+            }
             mbar_arrive_expect_tx(bars.kv_full + 8 * st, C::kTileBytes);
             const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
             for (int c = 0; c < C::kDBlocks; ++c)

@@ -22,6 +22,9 @@ struct alignas(64) AttnArgs {
   float scale_log2;         // softmax scale * log2(e)
   int select;               // ea_select
   unsigned long long timeout_ns;
+  // Failure-detection test hook (-1 = off): the producer skips the copy of
+  // this K/V ring position, so the kernel's bounded wait for it runs out.
+  int debug_drop_kv_pos;
 };
 
 // Dynamic shared memory the kernel for head dim D needs.
