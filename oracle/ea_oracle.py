@@ -64,6 +64,9 @@ __all__ = [
     "attention_weights",
     "brute_force_attention",
     "count_visible_pairs",
+    "kv_head_sparse",
+    "compact_slot",
+    "decode_step",
 ]
 
 
@@ -283,4 +286,56 @@ def brute_force_attention(q, k, v, mask, sink: int, window: int,
                     for wj, j in zip(w, keys):
                         acc += wj * float(v[b][hk][j][c])
                     out[b, h, i, c] = acc / tot
+    return out
+
+
+# --------------------------------------------------------------------------
+# Decode step with a per-head KV-cache policy (EA blog §3: the fused kernel
+# lowers memory use; a head routed to SA only ever needs its S sink tokens
+# and its last W tokens).  Readings: query position t of sequence b sees the
+# same keys as prefill row t (FA: 0..t; SA: sink + window); a kv head keeps a
+# compact sink + window cache iff every query head that reads it is SA.
+# --------------------------------------------------------------------------
+
+def kv_head_sparse(mask, hq: int, hkv: int) -> np.ndarray:
+    """[B, Hkv] uint8: 1 iff all query heads of the kv group route to SA."""
+    m = np.asarray(mask, dtype=np.uint8).reshape(-1, hq)
+    g = hq // hkv
+    return np.all(m.reshape(m.shape[0], hkv, g) != 0, axis=2).astype(np.uint8)
+
+
+def compact_slot(p: int, sink: int, window: int) -> int:
+    """Cache slot of position p in a sink + window cache: sinks stay put, the
+    rest cycle through a ring of W slots after them."""
+    if p < sink:
+        return p
+    return sink + (p - sink) % window
+
+
+def decode_step(q, k_hist, v_hist, pos, mask, sink: int, window: int,
+                scale: float | None = None) -> np.ndarray:
+    """out[b, h, :] for one new token per sequence.
+
+    q      : [B, Hq, d]      the new token's queries
+    k_hist : [B, Hkv, L, d]  every key up to and including position pos[b]
+    v_hist : [B, Hkv, L, d]
+    pos    : [B]             the new token's position t_b (its key is at t_b)
+    Each output is the prefill row t_b of the same head (EA blog §2.1: r
+    decides FA or SA per head)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    Hkv = k_hist.shape[1]
+    g = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    for b in range(B):
+        t = int(pos[b])
+        for h in range(Hq):
+            hk = h // g
+            keys = visible_keys(t, bool(mask[b][h]), sink, window)
+            kk = np.asarray(k_hist[b, hk], dtype=np.float64)[keys]
+            vv = np.asarray(v_hist[b, hk], dtype=np.float64)[keys]
+            s = (kk @ q[b, h]) * scale
+            out[b, h] = _softmax_row_weighted(s[None, :], vv)[0]
     return out

@@ -40,6 +40,11 @@ MUTATIONS = {
                              "return (e @ vals)"),
     "sink_ignored_blocked": ("vis &= (jj < sink) | ((ii - jj) < window)",
                              "vis &= ((ii - jj) < window)"),
+    "ring_slot_unshifted": ("return sink + (p - sink) % window", "return sink + p % window"),
+    "kv_policy_any": ("np.all(m.reshape(m.shape[0], hkv, g) != 0, axis=2)",
+                      "np.any(m.reshape(m.shape[0], hkv, g) != 0, axis=2)"),
+    "decode_gqa_modulo": ("            hk = h // g\n            keys = visible_keys",
+                          "            hk = h % Hkv\n            keys = visible_keys"),
 }
 
 

@@ -259,3 +259,58 @@ def test_visible_pair_counts_closed_forms():
     assert len(oracle.visible_keys(N - 1, True, S, W)) == S + W
     assert len(oracle.visible_keys(S + W - 1, True, S, W)) == S + W
     assert len(oracle.visible_keys(S + W - 2, True, S, W)) == S + W - 1
+
+
+# --------------------------------------------------------------------------
+# Decode-step pins
+# --------------------------------------------------------------------------
+
+def test_decode_step_is_the_prefill_row():
+    """A decode step at position t gives prefill row t of the same head."""
+    B, Hq, Hkv, N, d = 2, 4, 2, 70, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 31)
+    mask = np.array([[0, 1, 1, 1], [1, 0, 0, 1]], np.uint8)
+    S, W = 3, 9
+    pos = np.array([N - 1, 37])
+    full = oracle.attention(q, k, v, mask, S, W, block=16)
+    qt = np.stack([q[b, :, pos[b]] for b in range(B)])
+    out = oracle.decode_step(qt, k, v, pos, mask, S, W)
+    for b in range(B):
+        np.testing.assert_allclose(out[b], full[b, :, pos[b]], rtol=0, atol=1e-13)
+
+
+def test_decode_step_closed_forms():
+    B, Hq, Hkv, N, d = 1, 2, 1, 30, 8
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 32)
+    qt = q[:, :, 17]
+    out = oracle.decode_step(qt, k, v, [17], np.ones((1, 2), np.uint8), 0, 1)
+    np.testing.assert_array_equal(out[0, 0], v[0, 0, 17])   # W=1, S=0: its own value
+    out = oracle.decode_step(qt, k, v, [17], np.ones((1, 2), np.uint8), 1, 1)
+    a = (qt[0, 1] @ k[0, 0, 0] - qt[0, 1] @ k[0, 0, 17]) / math.sqrt(d)
+    sig = 1.0 / (1.0 + math.exp(-a))
+    np.testing.assert_allclose(out[0, 1], sig * v[0, 0, 0] + (1 - sig) * v[0, 0, 17], atol=1e-13)
+
+
+def test_compact_cache_slots():
+    S, W = 4, 6
+    # sinks never move
+    assert [oracle.compact_slot(p, S, W) for p in range(S)] == list(range(S))
+    # the last W positions (>= S) of any query occupy distinct ring slots
+    for t in range(S, 60):
+        window = [p for p in range(max(S, t - W + 1), t + 1)]
+        slots = [oracle.compact_slot(p, S, W) for p in window]
+        assert len(set(slots)) == len(slots)
+        assert all(S <= s < S + W for s in slots)
+    # the ring wraps with period W
+    assert oracle.compact_slot(S + 3, S, W) == oracle.compact_slot(S + 3 + W, S, W)
+    # layout convention (part of the cache API): the first position after the
+    # sinks fills the first ring slot, and the ring restarts there every W
+    assert oracle.compact_slot(S, S, W) == S
+    assert oracle.compact_slot(S + W, S, W) == S
+    assert oracle.compact_slot(S + W - 1, S, W) == S + W - 1
+
+
+def test_kv_head_sparse_requires_all_query_heads():
+    mask = np.array([[1, 1, 0, 1, 1, 1], [0, 0, 1, 1, 1, 0]], np.uint8)
+    np.testing.assert_array_equal(oracle.kv_head_sparse(mask, 6, 3), [[1, 0, 1], [0, 1, 0]])
+    np.testing.assert_array_equal(oracle.kv_head_sparse(mask, 6, 6), mask)
