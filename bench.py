@@ -58,6 +58,10 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--seq", type=int, default=None,
                     help="override the workload's sequence length (profiling cases)")
+    ap.add_argument("--decode-batch", type=int, default=16,
+                    help="sequences in the decode measurement (0 skips it)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
     return ap.parse_args()
@@ -372,7 +376,104 @@ def run_ours(args, rank, world, local_rank):
                                  + (" (layer 0)" if nlayers > 1 else "")}
         if rank == 0:
             result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
+    if not args.quick and world == 1 and args.decode_batch > 0:
+        result["decode"] = measure_decode(w, args.decode_batch, max(args.steps, 10),
+                                          max(args.warmup, 3), dev, stream)
     return result
+
+
+# ---------------------------------------------------------------- decode
+def measure_decode(w: workloads.Workload, batch: int, steps: int, warmup: int, dev, stream):
+    """One decode step per sequence of a ragged serving batch (positions in
+    [seq/2, seq)), caches under the per-head policy, timed with CUDA events;
+    then the same step with every head FA (every kv head on a full cache)."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (decode_workspace, ea_decode_kv_policy,
+                                                ea_get_device_status, ea_hybrid_attn_decode,
+                                                make_decode_params)
+    B, Hq, Hkv, d, S, W = batch, w.hq, w.hkv, w.d, w.sink, w.window
+    seed = workloads.layer_seed(w, 0) + 5000
+    frac = workloads.layer_sparse_frac(w, 0)
+    mask = workloads.make_fixed_mask(dataclasses.replace(w, batch=B, sparse_frac=frac,
+                                                         layers=1), seed)
+    pos0 = workloads.decode_positions(w, B, seed)
+    max_len = int(pos0.max()) + steps + warmup + 1
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+
+    def rand(*shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    def setup(m):
+        slots, n_full, n_sa = ea_decode_kv_policy(m, Hkv)
+        kf = rand(n_full, max_len, d) if n_full else None
+        vf = rand(n_full, max_len, d) if n_full else None
+        ks = rand(n_sa, S + W, d) if n_sa else None
+        vs = rand(n_sa, S + W, d) if n_sa else None
+        return slots, n_full, n_sa, (kf, vf, ks, vs)
+
+    q = rand(B, Hq, d)
+    kn = rand(B, Hkv, d)
+    vn = rand(B, Hkv, d)
+    # positions of step i: pos0 + i (each step appends one token per sequence)
+    pos_steps = [(pos0 + i).to(dev) for i in range(warmup + steps)]
+    out = torch.empty_like(q)
+
+    def run(m):
+        slots_np, n_full, n_sa, caches = setup(m)
+        slots = torch.as_tensor(slots_np, device=dev)
+        m_dev = m.to(dev)
+        ws = decode_workspace(make_decode_params(B, Hq, Hkv, d, S, W, max_len, n_full, n_sa),
+                              dev)
+        cache_bytes = sum(c.numel() * 2 for c in caches if c is not None)
+
+        def step(i):
+            ea_hybrid_attn_decode(q, kn, vn, pos_steps[i], m_dev, slots, *caches, S, W,
+                                  max_len, out=out, workspace=ws, stream=stream)
+        for i in range(warmup):
+            step(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            step(warmup + i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if ea_get_device_status(ws) != 0:
+            raise RuntimeError("decode status word reports an error")
+        ms = a.elapsed_time(b) / steps
+        mid = (pos0 + warmup + (steps - 1) // 2).numpy()
+        byts = flops.decode_bytes(m.numpy(), mid, Hkv, d, S, W)
+        del caches
+        return ms, byts, cache_bytes
+
+    ms, byts, cache_bytes = run(mask)
+    full_mask = torch.zeros_like(mask)
+    ms_full, byts_full, cache_full = run(full_mask)
+    peaks, src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = byts["total"] / (ms * 1e-3) / 1e9
+    return {
+        "workload": f"{w.name} decode: B={B} Hq={Hq} Hkv={Hkv} d={d} S={S} W={W}, positions "
+                    f"ragged in [{w.seq // 2}, {w.seq}) + step, SA heads {mask.float().mean():.2f},"
+                    f" all-SA kv groups {byts['n_sa_groups']}/{byts['n_groups']}",
+        "steps": steps, "warmup": warmup,
+        "us_per_step": round(ms * 1e3, 2),
+        "tokens_per_s": round(B / (ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "peak_source": f"{src} hbm_gbs",
+                     "bytes_per_step": byts["total"],
+                     "scope": "whole step (append + split-K attention + combine) over its "
+                              "algorithmic bytes"},
+        "gpu_launches_per_step": 3,
+        "all_fa_us_per_step": round(ms_full * 1e3, 2),
+        "all_fa_gbs": round(byts_full["total"] / (ms_full * 1e-3) / 1e9, 1),
+        "speedup_vs_all_fa": round(ms_full / ms, 3),
+        "cache_bytes": cache_bytes,
+        "all_fa_cache_bytes": cache_full,
+        "cache_saved_frac": round(1.0 - cache_bytes / cache_full, 4),
+        "l2": "per-step bytes exceed L2" if byts["total"] > 126e6 else "per-step bytes fit L2",
+    }
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -483,6 +584,17 @@ def main():
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.decode_only:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = measure_decode(w, max(args.decode_batch, 1), args.steps, max(args.warmup, 3), dev,
+                             torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
         return 0
     if world > 1:
         torch.cuda.set_device(local_rank)

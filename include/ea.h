@@ -182,6 +182,63 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
 ea_status ea_get_device_status(void* workspace, void* stream, int* status_out);
 
 /* ------------------------------------------------------------------------
+ * Decode step with a per-head KV-cache policy.
+ *
+ * Elastic Attention blog §3: the fused treatment of FA and SA heads lowers
+ * memory use as well as time.  In decode the saving is the cache: a head
+ * routed to SA only reads its S sink keys and its last W keys, so a kv head
+ * whose query heads are ALL routed SA keeps a compact cache of S + W rows;
+ * any other kv head keeps every position.  The query at position t sees the
+ * keys prefill row t sees (FA: 0..t; SA: j < S or t - j < W).
+ *
+ * Caches (caller-owned, device, bf16, d contiguous):
+ *   full    k_full, v_full [n_full][max_len][d]   row p holds position p
+ *   compact k_sa,   v_sa   [n_sa][sink+window][d] position p < S at row p,
+ *                                                 p >= S at S + (p - S) % W
+ * cache_slot[b*Hkv + hk] (device int32) picks a kv head's cache: c >= 0 is
+ * full cache c, c < 0 is compact cache -c-1.  A compact cache may back only
+ * a kv head whose query heads are all SA (ea_decode_kv_policy builds such an
+ * assignment); otherwise the step records EA_ERR_INVALID_ARG in the status
+ * word and FA heads of that group see only sink + window keys.  A slot
+ * outside its pool, pos[b] < 0, or pos[b] >= max_len on a full cache also
+ * records EA_ERR_INVALID_ARG: that (b, kv head) is neither written nor read
+ * and its outputs are zero.
+ *
+ * One step, per sequence b: the new k_new, v_new [B][Hkv][d] are written at
+ * position pos[b] (device int32 [B]; 0 <= pos[b] < max_len for full caches),
+ * then every query head attends: out[b, h, :] (bf16 [B][Hq][d]) from
+ * q [B][Hq][d].  Sequences may sit at different positions.  fp32 softmax
+ * and accumulation; the partial results of the split key range live in the
+ * workspace (ea_decode_workspace_size bytes, zeroed once: its first word is
+ * the status word read by ea_get_device_status).
+ * ---------------------------------------------------------------------- */
+typedef struct ea_decode_params {
+  int B, Hq, Hkv, d;
+  int sink, window;
+  int max_len;           /* positions a full cache holds                 */
+  float softmax_scale;   /* <= 0 selects 1/sqrt(d)                       */
+  int n_full, n_sa;      /* caches in each pool; every cache_slot entry
+                            must name one of them                        */
+} ea_decode_params;
+
+size_t ea_decode_workspace_size(const ea_decode_params* p);
+
+ea_status ea_hybrid_attn_decode(const void* q, const void* k_new, const void* v_new,
+                                const int32_t* pos, const uint8_t* route_mask,
+                                const int32_t* cache_slot, void* k_full, void* v_full,
+                                void* k_sa, void* v_sa, const ea_decode_params* p,
+                                void* out, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Host helper: from a host route mask [B][Hq], assign every (b, kv head) a
+ * full cache (some query head is FA) or a compact cache (all are SA):
+ * cache_slot (host int32 [B][Hkv]) gets the encoding above, numbered in
+ * (b, hk) order; *n_full and *n_sa receive the pool sizes.  Returns 0, or -1
+ * on invalid arguments. */
+int ea_decode_kv_policy(const uint8_t* mask, int B, int Hq, int Hkv, int32_t* cache_slot,
+                        int* n_full, int* n_sa);
+
+/* ------------------------------------------------------------------------
  * Host-side view of the fused kernel's work schedule, for inspection and
  * tests (no GPU needed).  A unit is (mode, b, h, pair): 256 query rows
  * [256*pair, 256*pair + 256) of head h in batch b, run by one CTA.  Units

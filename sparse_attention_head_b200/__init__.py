@@ -9,7 +9,8 @@ libea.so; this package only marshals arguments.
 from ._lib import (EA_OK, EA_ERR_CUDA, EA_ERR_INVALID_ARG, EA_ERR_MISALIGNED,  # noqa: F401
                    EA_ERR_TIMEOUT, EA_ERR_UNSUPPORTED, EA_ERR_WORKSPACE, EA_SELECT_ALL,
                    EA_SELECT_FA, EA_SELECT_SA, EaAttnParams, EaError, LIB_PATH)
-from .api import (HostPrefill, attn_workspace, ea_attn_grid_size, ea_get_device_status,  # noqa: F401
+from .api import (HostPrefill, attn_workspace, decode_workspace, ea_decode_kv_policy,  # noqa: F401
+                  ea_hybrid_attn_decode, make_decode_params, ea_attn_grid_size, ea_get_device_status,  # noqa: F401
                   ea_hybrid_attn_prefill, ea_hybrid_attn_workspace_size, ea_router_decide,
                   ea_router_workspace_size, ea_schedule_unit_tiles, ea_schedule_units,
                   make_params)

@@ -33,7 +33,8 @@ EXPORTED = [
     "ea_router_workspace_size", "ea_router_decide", "ea_router_decide_noalloc",
     "ea_hybrid_attn_workspace_size", "ea_hybrid_attn_prefill",
     "ea_get_device_status", "ea_schedule_units", "ea_schedule_unit_tiles",
-    "ea_attn_grid_size",
+    "ea_attn_grid_size", "ea_decode_workspace_size", "ea_hybrid_attn_decode",
+    "ea_decode_kv_policy",
 ]
 
 
@@ -42,6 +43,13 @@ class EaAttnParams(ctypes.Structure):
                 ("N", ctypes.c_int), ("d", ctypes.c_int), ("sink", ctypes.c_int),
                 ("window", ctypes.c_int), ("softmax_scale", ctypes.c_float),
                 ("select", ctypes.c_int)]
+
+
+class EaDecodeParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("d", ctypes.c_int), ("sink", ctypes.c_int), ("window", ctypes.c_int),
+                ("max_len", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+                ("n_full", ctypes.c_int), ("n_sa", ctypes.c_int)]
 
 
 class EaError(RuntimeError):
@@ -93,6 +101,14 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_schedule_unit_tiles.argtypes = [vp, pparams, c_int, vp, vp, c_int]
     lib.ea_attn_grid_size.restype = c_int
     lib.ea_attn_grid_size.argtypes = [pparams, c_int]
+    pdec = ctypes.POINTER(EaDecodeParams)
+    lib.ea_decode_workspace_size.restype = c_size
+    lib.ea_decode_workspace_size.argtypes = [pdec]
+    lib.ea_hybrid_attn_decode.restype = c_int
+    lib.ea_hybrid_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, pdec, vp, vp,
+                                          c_size, vp]
+    lib.ea_decode_kv_policy.restype = c_int
+    lib.ea_decode_kv_policy.argtypes = [vp, c_int, c_int, c_int, vp, vp, vp]
     _lib = lib
     return lib
 

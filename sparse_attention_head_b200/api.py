@@ -12,7 +12,8 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import EA_SELECT_ALL, EA_SELECT_FA, EA_SELECT_SA, EaAttnParams, check  # noqa: F401
+from ._lib import (EA_SELECT_ALL, EA_SELECT_FA, EA_SELECT_SA, EaAttnParams,  # noqa: F401
+                   EaDecodeParams, check)
 
 
 def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> int:
@@ -244,3 +245,77 @@ class HostPrefill:
                                out=self.out, workspace=self.aws, stream=stream)
         self.out_host.copy_(self.out, non_blocking=True)
         return self.out_host
+
+
+# ---------------------------------------------------------------- decode
+def ea_decode_kv_policy(mask, Hkv: int):
+    """(cache_slot int32 [B, Hkv], n_full, n_sa): a compact cache for every kv
+    head whose query heads are all SA, a full cache for the others."""
+    lib = _lib.load()
+    m = np.ascontiguousarray(
+        (mask.detach().cpu().numpy() if isinstance(mask, torch.Tensor) else np.asarray(mask))
+        .astype(np.uint8))
+    B, Hq = m.shape
+    slots = np.zeros((B, Hkv), dtype=np.int32)
+    nf, ns = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib.ea_decode_kv_policy(m.ctypes.data, B, Hq, Hkv, slots.ctypes.data, ctypes.byref(nf),
+                                 ctypes.byref(ns))
+    if rc != 0:
+        raise ValueError("invalid kv policy arguments")
+    return slots, int(nf.value), int(ns.value)
+
+
+def make_decode_params(B, Hq, Hkv, d, sink, window, max_len, n_full, n_sa,
+                       softmax_scale=0.0) -> EaDecodeParams:
+    return EaDecodeParams(int(B), int(Hq), int(Hkv), int(d), int(sink), int(window),
+                          int(max_len), float(softmax_scale), int(n_full), int(n_sa))
+
+
+def decode_workspace(p: EaDecodeParams, device) -> torch.Tensor:
+    n = int(_lib.load().ea_decode_workspace_size(ctypes.byref(p)))
+    if n == 0:
+        raise ValueError("invalid decode parameters")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def ea_hybrid_attn_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                          pos: torch.Tensor, route_mask: torch.Tensor, cache_slot: torch.Tensor,
+                          k_full, v_full, k_sa, v_sa, sink: int, window: int, max_len: int, *,
+                          softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One decode step: append k_new/v_new at pos, attend, return out [B, Hq, d]."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(pos, "pos", torch.int32, 1)
+    _need(route_mask, "route_mask", torch.uint8)
+    _need(cache_slot, "cache_slot", torch.int32)
+    B, Hq, d = q.shape
+    Hkv = k_new.shape[1]
+    for name, t in (("k_full", k_full), ("v_full", v_full), ("k_sa", k_sa), ("v_sa", v_sa)):
+        if t is not None:
+            _need(t, name, torch.bfloat16, 3)
+    n_full = k_full.shape[0] if k_full is not None else 0
+    n_sa = k_sa.shape[0] if k_sa is not None else 0
+    if k_full is not None and tuple(k_full.shape[1:]) != (max_len, d):
+        raise ValueError("k_full must be [n_full, max_len, d]")
+    if k_sa is not None and tuple(k_sa.shape[1:]) != (sink + window, d):
+        raise ValueError("k_sa must be [n_sa, sink + window, d]")
+    for a, b_, name in ((k_full, v_full, "v_full"), (k_sa, v_sa, "v_sa")):
+        if (a is None) != (b_ is None) or (a is not None and a.shape != b_.shape):
+            raise ValueError(f"{name} must match its k cache")
+    p = make_decode_params(B, Hq, Hkv, d, sink, window, max_len, n_full, n_sa, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(p, q.device)
+    ptr = (lambda t: t.data_ptr() if t is not None else None)
+    rc = lib.ea_hybrid_attn_decode(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+                                   pos.data_ptr(), route_mask.data_ptr(), cache_slot.data_ptr(),
+                                   ptr(k_full), ptr(v_full), ptr(k_sa), ptr(v_sa),
+                                   ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel(), _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_decode")
+    return out

@@ -52,3 +52,33 @@ def tile_flops(mask, N: int, d: int, sink: int, window: int) -> float:
     tiles = n_fa * _visible_tiles(N, False, sink, window) + \
         n_sa * _visible_tiles(N, True, sink, window)
     return 4.0 * d * 128 * 128 * tiles
+
+
+# ---------------------------------------------------------------- decode
+def decode_group_rows(t: int, all_sparse: bool, sink: int, window: int) -> int:
+    """Cache rows one kv group reads for the query at position t: every
+    position 0..t when some query head of the group is FA, else the sink and
+    window positions (j < S or t - j < W)."""
+    if not all_sparse:
+        return t + 1
+    lo = max(0, t - window + 1)
+    return min(sink, lo) + (t - lo + 1)
+
+
+def decode_bytes(mask, pos, hkv: int, d: int, sink: int, window: int) -> dict:
+    """Algorithmic HBM bytes of one decode step (bf16 everywhere):
+    kv   = K and V rows every kv group reads once for all its query heads;
+    io   = q read + out write + the new k, v rows read and appended."""
+    m = np.asarray(mask, dtype=np.uint8)
+    B, hq = m.shape
+    g = hq // hkv
+    all_sa = np.all(m.reshape(B, hkv, g) != 0, axis=2)
+    row = 2 * d                                    # bytes of one bf16 row
+    kv = 0
+    for b in range(B):
+        t = int(pos[b])
+        for hk in range(hkv):
+            kv += 2 * row * decode_group_rows(t, bool(all_sa[b, hk]), sink, window)
+    io = 2 * B * hq * row + 2 * 2 * B * hkv * row
+    return {"kv": kv, "io": io, "total": kv + io, "n_sa_groups": int(all_sa.sum()),
+            "n_groups": int(B * hkv)}

@@ -145,3 +145,21 @@ def test_effective_and_tile_flops():
     # tile-granular: FA 512 rows -> 1+2+3+4 tiles; SA (S=16, W=128): tiles per
     # row tile m are {0, m-1, m} -> 1, 2, 3, 3
     assert flops.tile_flops(mask, 512, 64, 16, 128) == 4 * 64 * 128 * 128 * (2 * 10 + 2 * 9)
+
+
+@pytest.mark.parametrize("t,S,W", [(0, 4, 16), (5, 4, 16), (19, 4, 16), (20, 4, 16),
+                                   (1000, 64, 256), (7, 0, 1), (300, 500, 8)])
+def test_decode_group_rows_match_oracle(t, S, W):
+    assert flops.decode_group_rows(t, False, S, W) == len(oracle.visible_keys(t, False, S, W))
+    assert flops.decode_group_rows(t, True, S, W) == len(oracle.visible_keys(t, True, S, W))
+
+
+def test_decode_bytes():
+    mask = np.array([[1, 1, 0, 1], [1, 1, 1, 1]], np.uint8)
+    pos = [100, 9]
+    got = flops.decode_bytes(mask, pos, 2, 64, 2, 8)
+    row = 128
+    # b0: group 0 all SA (2 + 8 rows), group 1 mixed (101 rows); b1: both SA (2 + 8)
+    assert got["kv"] == 2 * row * (10 + 101 + 10 + 10)
+    assert got["io"] == 2 * 2 * 4 * row + 4 * 2 * 2 * row
+    assert got["n_sa_groups"] == 3 and got["n_groups"] == 4

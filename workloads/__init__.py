@@ -21,7 +21,7 @@ import torch
 
 __all__ = ["Workload", "WORKLOADS", "get", "make_qkv", "make_router_weights",
            "make_fixed_mask", "sparse_head_set", "layer_seed",
-           "layer_sparse_frac"]
+           "layer_sparse_frac", "decode_positions"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -153,3 +153,11 @@ def layer_sparse_frac(w: Workload, layer: int) -> float:
     g = _gen(layer_seed(w, layer) + 29, "cpu")
     u = torch.rand((1,), generator=g, dtype=torch.float64).item()
     return w.sparse_lo + (w.sparse_hi - w.sparse_lo) * u
+
+
+def decode_positions(w: Workload, batch: int, seed: int) -> torch.Tensor:
+    """int32 [batch] decode positions, ragged: uniform in [seq/2, seq - 1]
+    (a serving batch whose prompts finished prefill at different lengths)."""
+    g = _gen(seed + 211, "cpu")
+    lo = max(0, w.seq // 2)
+    return torch.randint(lo, w.seq, (batch,), generator=g, dtype=torch.int64).to(torch.int32)
