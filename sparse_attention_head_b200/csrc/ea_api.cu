@@ -12,7 +12,41 @@
 #include "ea_internal.h"
 #include "ea_sched.h"
 
+namespace ea {
+
+constexpr int kMaxSmDevices = 64;
+
+int device_sms() {
+  static int sms[kMaxSmDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < kMaxSmDevices && sms[dev]) return sms[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxSmDevices) sms[dev] = n;
+  return n;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long ns = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    double ms = 2000.0;
+    if (const char* e = getenv("EA_WAIT_TIMEOUT_MS")) {
+      double v = atof(e);
+      if (v > 0) ms = v;
+    }
+    ns = static_cast<unsigned long long>(ms * 1e6);
+  });
+  return ns;
+}
+
+}  // namespace ea
+
 namespace {
+
+using ea::device_sms;
+using ea::wait_timeout_ns;
 
 constexpr int kMaxDevices = 64;
 
@@ -66,31 +100,6 @@ bool encode_bhsd(CUtensorMap* m, const void* ptr, int d, int n, int rows3) {
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-int device_sms() {
-  static int sms[kMaxDevices] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices && sms[dev]) return sms[dev];
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) sms[dev] = n;
-  return n;
-}
-
-unsigned long long wait_timeout_ns() {
-  static unsigned long long ns = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    double ms = 2000.0;
-    if (const char* e = getenv("EA_WAIT_TIMEOUT_MS")) {
-      double v = atof(e);
-      if (v > 0) ms = v;
-    }
-    ns = static_cast<unsigned long long>(ms * 1e6);
-  });
-  return ns;
 }
 
 // EA_DEBUG_DROP_KV_POS=<n> makes the attention producer skip K/V ring

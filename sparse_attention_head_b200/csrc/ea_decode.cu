@@ -11,11 +11,15 @@
 //
 // Step, all on the caller's stream:
 //   1. append: the new k, v of every (b, kv head) go to their cache slot;
-//   2. attention: CTA (split, kv head, b) reads one chunk of the group's
-//      visible keys once for all G query heads (16 lanes per key row, 16-byte
-//      loads), keeps an fp32 online softmax per head and writes a partial
-//      (max, sum, o) to the workspace;
-//   3. combine: the partials of each (b, query head) are merged in split
+//   2. attention: one persistent CTA per SM walks the (kv group, 512-key
+//      chunk) items that hold visible keys.  A producer warp streams each
+//      item's cache rows into shared memory with bulk copies (a group's
+//      visible keys are at most four contiguous row runs of its cache:
+//      sinks, window, and the two sides of the ring wrap); eight consumer
+//      warps read every row once for all G query heads of the group, keep an
+//      fp32 online softmax per head and write one partial (o, max, sum) per
+//      item and head to the workspace;
+//   3. combine: the partials of each (b, query head) are merged in chunk
 //      order and written as bf16.
 // The step is HBM-bound: its work is one read of every visible cache row.
 #include <cuda_bf16.h>
@@ -25,11 +29,12 @@
 
 #include "ea.h"
 #include "ea_internal.h"
+#include "ea_math.cuh"
+#include "ea_ptx.cuh"
 
 namespace ea {
 
-constexpr int kDecThreads = 256;         // 8 warps, 16 key rows in flight per step
-constexpr int kDecChunk = 512;           // visible keys per CTA (at most)
+constexpr int kDecChunk = 512;           // visible keys per work item (at most)
 
 struct DecodeArgs {
   const __nv_bfloat16* q;      // [B][Hq][d]
@@ -47,6 +52,7 @@ struct DecodeArgs {
   int* status;
   int B, Hq, Hkv, d, sink, window, max_len, nsplit, n_full, n_sa;
   float scale_log2;
+  unsigned long long timeout_ns;   // bound of every barrier wait
 };
 
 __device__ __forceinline__ int dec_compact_slot(int p, int sink, int window) {
@@ -83,6 +89,14 @@ __global__ void ea_decode_append_kernel(DecodeArgs args) {
     if (threadIdx.x == 0) atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);
     return;
   }
+  if (slot < 0 && threadIdx.x == 0) {   // a compact cache behind an FA query head
+    const int G = args.Hq / args.Hkv;
+    for (int g = 0; g < G; ++g)
+      if (args.mask[b * args.Hq + hk * G + g] == 0) {
+        atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);
+        break;
+      }
+  }
   __nv_bfloat16* kd;
   __nv_bfloat16* vd;
   size_t row;
@@ -105,177 +119,415 @@ __global__ void ea_decode_append_kernel(DecodeArgs args) {
   }
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads) ea_decode_attn_kernel(DecodeArgs args) {
-  constexpr int kLanesPerRow = D / 8;                 // 16 (d=128) or 8 (d=64)
-  constexpr int kRowsPerWarp = 32 / kLanesPerRow;     // 2 or 4
-  constexpr int kWarps = kDecThreads / 32;
-  constexpr int kRowsPerStep = kWarps * kRowsPerWarp;
-  constexpr int kGroups = kDecThreads / kLanesPerRow; // independent softmax states
-  __shared__ float s_q[G][D];
-  __shared__ float s_m[kGroups][G];
-  __shared__ float s_l[kGroups][G];
-  __shared__ float s_o[G][D];
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int t = args.pos[b];
-  const int slot = args.cache_slot[b * args.Hkv + hk];
-  const bool compact = slot < 0;
+// Visible keys of kv group (b, hk) at this step and the heads' routing.
+struct DecGroup {
+  int t, slot, a, lo, nvis;
+  bool compact;
+  uint32_t sparse_bits;   // bit g: query head hk*G + g routes to SA
+};
+
+__device__ __forceinline__ DecGroup dec_group(const DecodeArgs& args, int b, int hk, int G) {
+  DecGroup g;
+  g.t = args.pos[b];
+  g.slot = args.cache_slot[b * args.Hkv + hk];
+  g.compact = g.slot < 0;
+  g.sparse_bits = 0;
   bool all_sparse = true;
-  bool head_sparse[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    head_sparse[g] = args.mask[b * args.Hq + hk * G + g] != 0;
-    all_sparse = all_sparse && head_sparse[g];
+  for (int i = 0; i < G; ++i) {
+    const bool sp = args.mask[b * args.Hq + hk * G + i] != 0;
+    g.sparse_bits |= static_cast<uint32_t>(sp) << i;
+    all_sparse = all_sparse && sp;
   }
-  if (compact && !all_sparse && threadIdx.x == 0 && split == 0)
-    atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);   // an FA head on a compact cache
-  int a, lo;
-  dec_group_keys(all_sparse || compact, t, args.sink, args.window, &a, &lo);
-  const int nvis = dec_slot_ok(args, slot, t) ? a + (t - lo + 1) : 0;
-  const int k0 = split * kDecChunk;
-  const int k1 = min(nvis, k0 + kDecChunk);
+  dec_group_keys(all_sparse || g.compact, g.t, args.sink, args.window, &g.a, &g.lo);
+  g.nvis = dec_slot_ok(args, g.slot, g.t) ? g.a + (g.t - g.lo + 1) : 0;
+  return g;
+}
 
-  for (int i = threadIdx.x; i < G * D; i += kDecThreads) {
-    const int g = i / D, c = i % D;
-    s_q[g][c] = __bfloat162float(
-                    args.q[(static_cast<size_t>(b) * args.Hq + hk * G + g) * D + c]) *
-                args.scale_log2;
-  }
-  __syncthreads();
+// One 64-row stage of an item, written by the producer before it arms the
+// stage's full barrier.  n < 0 ends the stream.
+struct DecDesc {
+  int n, js, t, a, lo, b, hk, chunk, first, last;
+  uint32_t sparse_bits;
+  int pad[5];
+};
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane / kLanesPerRow;                // key row within the warp step
-  const int cl = lane % kLanesPerRow;                 // 8-channel column block
-  const int grp = warp * kRowsPerWarp + sub;          // softmax state index
-  const __nv_bfloat16* kbase;
-  const __nv_bfloat16* vbase;
-  if (nvis == 0) {   // nothing to read; the pointers are never used
-    kbase = vbase = nullptr;
-  } else if (compact) {
-    const size_t c = static_cast<size_t>(-slot - 1) * (args.sink + args.window);
-    kbase = args.k_sa + c * D;
-    vbase = args.v_sa + c * D;
-  } else {
-    const size_t c = static_cast<size_t>(slot) * args.max_len;
-    kbase = args.k_full + c * D;
-    vbase = args.v_full + c * D;
-  }
-  float qv[G][8];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qv[g][e] = s_q[g][cl * 8 + e];
+constexpr int kDecConsumerWarps = 8;                              // warpgroups 0 and 1
+constexpr int kDecKernelThreads = (kDecConsumerWarps + 4) * 32;   // + producer warpgroup
+// Register split (setmaxnreg): launched at 65536 / 384 = 168 per thread, the
+// producer warpgroup gives back down to 56 and the consumers take 224:
+// 128 * 56 + 256 * 224 = 64512 = 384 * 168.
+constexpr int kDecRegsProducer = 56;
+constexpr int kDecRegsConsumer = 224;
+static_assert(128 * kDecRegsProducer + 256 * kDecRegsConsumer <= kDecKernelThreads * 168,
+              "register split exceeds the launch's registers");
+constexpr int kDecStageRows = 64;
+constexpr int kDecMaxGroups = 4096;                                // B * Hkv
+constexpr float kDecNegBig = -1.0e30f;     // running max before the first key
+constexpr float kDecRescale = 8.0f;        // rescale only when the max grows by > 2^8
 
-  float m[G], l[G], o[G][8];
+template <int D, int G>
+struct DecLayout {
+  static constexpr int kDPL = (G == 8) ? 8 : 16;     // channels per lane
+  static constexpr int kLPR = D / kDPL;              // lanes per key row
+  static constexpr int kChunks = kDPL / 8;           // 16-byte chunks per lane
+  static constexpr int kRGW = 32 / kLPR;             // row groups per warp
+  static constexpr int kNG = kDecConsumerWarps * kRGW;
+  static constexpr int kRPS = kDecStageRows / kNG;   // rows per group per stage
+  static constexpr int kStages = (D == 128) ? 4 : 6;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kKV = kDecStageRows * kRowBytes;
+  static constexpr int kQ = G * D * 2;
+  static constexpr int off_k = 0;
+  static constexpr int off_v = off_k + kStages * kKV;
+  static constexpr int off_q = off_v + kStages * kKV;
+  static constexpr int off_desc = off_q + kStages * kQ;
+  static constexpr int off_full = off_desc + kStages * static_cast<int>(sizeof(DecDesc));
+  static constexpr int off_empty = off_full + kStages * 8;
+  static constexpr int off_flag = off_empty + kStages * 8;
+  static constexpr int off_mo = off_flag + 16;
+  static constexpr int off_ml = off_mo + kDecConsumerWarps * G * D * 4;
+  static constexpr int off_table = off_ml + kDecConsumerWarps * G * 2 * 4;
+  static constexpr int bytes(int ngroups) { return off_table + (ngroups + 1) * 4; }
+  static_assert(kDecStageRows % kNG == 0 && kRPS >= 1, "stage rows per row group");
+  static_assert(sizeof(DecDesc) == 64, "descriptor size");
+  static_assert(off_full % 8 == 0 && off_q % 16 == 0, "alignment");
+};
+
+__device__ __forceinline__ void named_bar_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
-  }
-  // warp-uniform loop (the shuffles below need every lane); rows past the
-  // chunk are loaded as zeros and skipped
-  for (int jb = k0 + warp * kRowsPerWarp; jb < k1; jb += kRowsPerStep) {
-    const int j = jb + sub;
-    const bool valid = j < k1;
-    const int p = !valid ? 0 : (j < a ? j : lo + (j - a));     // key position
-    const int crow = compact ? dec_compact_slot(p, args.sink, args.window) : p;
-    uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
-    if (valid) {
-      kraw = __ldg(reinterpret_cast<const uint4*>(kbase + static_cast<size_t>(crow) * D) + cl);
-      vraw = __ldg(reinterpret_cast<const uint4*>(vbase + static_cast<size_t>(crow) * D) + cl);
-    }
-    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vraw);
-    float kf[8], vf[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 kk = __bfloat1622float2(k2[e]);
-      const float2 vv = __bfloat1622float2(v2[e]);
-      kf[2 * e] = kk.x; kf[2 * e + 1] = kk.y;
-      vf[2 * e] = vv.x; vf[2 * e + 1] = vv.y;
-    }
-    const bool in_sa = p < args.sink || t - p < args.window;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float s = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s = fmaf(qv[g][e], kf[e], s);
-#pragma unroll
-      for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
-        s += __shfl_xor_sync(0xffffffffu, s, off);
-      if (!valid || (head_sparse[g] && !in_sa)) continue;   // not a key of this head
-      const float mn = fmaxf(m[g], s);
-      const float alpha = exp2f(m[g] - mn);
-      const float pr = exp2f(s - mn);
-      l[g] = l[g] * alpha + pr;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[g][e] = fmaf(o[g][e], alpha, pr * vf[e]);
-      m[g] = mn;
-    }
-  }
-  // merge the kGroups softmax states of this CTA, then write the partial
-  if (cl == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      s_m[grp][g] = m[g];
-      s_l[grp][g] = l[g];
-    }
-  }
-  for (int i = threadIdx.x; i < G * D; i += kDecThreads) (&s_o[0][0])[i] = 0.f;
-  __syncthreads();
-  float mg[G], sc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float mm = -INFINITY;
-    for (int r = 0; r < kGroups; ++r) mm = fmaxf(mm, s_m[r][g]);
-    mg[g] = mm;
-    sc[g] = (m[g] == -INFINITY) ? 0.f : exp2f(m[g] - mm);
-  }
-  // fixed-order merge of the o rows: one group at a time
-  for (int r = 0; r < kGroups; ++r) {
-    if (grp == r) {
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s_o[g][cl * 8 + e] += o[g][e] * sc[g];
-    }
-    __syncthreads();
-  }
-  float* pb = args.part + ((static_cast<size_t>(b) * args.Hq + hk * G) * args.nsplit + split) *
-                              (D + 2);
-  for (int i = threadIdx.x; i < G * D; i += kDecThreads) {
-    const int g = i / D, c = i % D;
-    pb[static_cast<size_t>(g) * args.nsplit * (D + 2) + c] = s_o[g][c];
-  }
-  if (threadIdx.x < G) {
-    const int g = threadIdx.x;
-    float ls = 0.f;
-    for (int r = 0; r < kGroups; ++r)
-      ls += (s_m[r][g] == -INFINITY) ? 0.f : s_l[r][g] * exp2f(s_m[r][g] - mg[g]);
-    pb[static_cast<size_t>(g) * args.nsplit * (D + 2) + D] = mg[g];
-    pb[static_cast<size_t>(g) * args.nsplit * (D + 2) + D + 1] = ls;
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
   }
 }
 
+// Persistent split-K decode attention.  Work item = (kv group, 512-key
+// chunk) with at least one visible key; CTA c takes items c, c + grid, ...
+// Warp 8 (producer) builds the item table, then streams each item's visible
+// cache rows (contiguous runs: sinks, window, ring wrap) and its G query rows
+// into a ring of 64-row stages with bulk copies.  Warps 0-7 (consumers) take
+// a stage: every key row is read by kLPR lanes, the G dot products reduced
+// by shuffles, and an fp32 online softmax kept per row group and head; the
+// last stage of an item merges the row groups and writes the item's partial
+// (o, max, sum) for every query head of the group.
+template <int D, int G>
+__global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(DecodeArgs args) {
+  using L = DecLayout<D, G>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  DecDesc* desc = reinterpret_cast<DecDesc*>(smem + L::off_desc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::off_flag);
+  int* table = reinterpret_cast<int*>(smem + L::off_table);
+  const uint32_t full0 = sbase + L::off_full, empty0 = sbase + L::off_empty;
+  const int ngroups = args.B * args.Hkv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * s) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s),
+                   "n"(kDecConsumerWarps) : "memory");
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp >= kDecConsumerWarps) {
+    regs_dec<kDecRegsProducer>();
+    if (warp != kDecConsumerWarps) return;
+    // ---------------- producer: item table (exclusive prefix of chunk counts)
+    int carry = 0;
+    for (int base = 0; base < ngroups; base += 32) {
+      const int gi = base + lane;
+      int cnt = 0;
+      if (gi < ngroups) {
+        const DecGroup g = dec_group(args, gi / args.Hkv, gi % args.Hkv, G);
+        cnt = (g.nvis + kDecChunk - 1) / kDecChunk;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (gi < ngroups) table[gi + 1] = carry + incl;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) table[0] = 0;
+    __syncwarp();
+    if (lane != 0) return;
+
+    // ---------------- producer: stream the stages
+    const int total = table[ngroups];
+    int u = 0;                 // stage uses issued
+    int gi = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      while (table[gi + 1] <= it) ++gi;
+      const int b = gi / args.Hkv, hk = gi % args.Hkv;
+      const int chunk = it - table[gi];
+      const DecGroup g = dec_group(args, b, hk, G);
+      const __nv_bfloat16* kbase;
+      const __nv_bfloat16* vbase;
+      if (g.compact) {
+        const size_t c = static_cast<size_t>(-g.slot - 1) * (args.sink + args.window);
+        kbase = args.k_sa + c * D;
+        vbase = args.v_sa + c * D;
+      } else {
+        const size_t c = static_cast<size_t>(g.slot) * args.max_len;
+        kbase = args.k_full + c * D;
+        vbase = args.v_full + c * D;
+      }
+      const int j0 = chunk * kDecChunk, j1 = min(g.nvis, j0 + kDecChunk);
+      for (int js = j0; js < j1; js += kDecStageRows) {
+        const int slot = u % L::kStages, round = u / L::kStages;
+        if (round > 0 && !mbar_wait(empty0 + 8 * slot, (round - 1) & 1, abort_flag, args.status,
+                                    args.timeout_ns, EA_ERR_TIMEOUT)) {
+          ok = false;
+          break;
+        }
+        const int n = min(kDecStageRows, j1 - js);
+        DecDesc& d = desc[slot];
+        d.n = n; d.js = js; d.t = g.t; d.a = g.a; d.lo = g.lo; d.b = b; d.hk = hk;
+        d.chunk = chunk; d.first = js == j0; d.last = js + kDecStageRows >= j1;
+        d.sparse_bits = g.sparse_bits;
+        const uint32_t bar = full0 + 8 * slot;
+        mbar_arrive_expect_tx(bar, 2u * n * L::kRowBytes + (js == j0 ? L::kQ : 0));
+        const uint32_t kdst = sbase + L::off_k + slot * L::kKV;
+        const uint32_t vdst = sbase + L::off_v + slot * L::kKV;
+        for (int j = js; j < js + n;) {
+          int crow, run;
+          if (j < g.a) {                       // sink keys: rows 0.. of either cache
+            crow = j;
+            run = min(js + n, g.a) - j;
+          } else {
+            const int p = g.lo + (j - g.a);
+            if (!g.compact) {
+              crow = p;
+              run = js + n - j;
+            } else if (p < args.sink) {
+              crow = p;
+              run = min(js + n - j, args.sink - p);
+            } else {                           // ring: stop at the wrap
+              const int r = (p - args.sink) % args.window;
+              crow = args.sink + r;
+              run = min(js + n - j, args.window - r);
+            }
+          }
+          const uint32_t off = static_cast<uint32_t>(j - js) * L::kRowBytes;
+          bulk_load(kdst + off, kbase + static_cast<size_t>(crow) * D, run * L::kRowBytes, bar);
+          bulk_load(vdst + off, vbase + static_cast<size_t>(crow) * D, run * L::kRowBytes, bar);
+          j += run;
+        }
+        if (js == j0)
+          bulk_load(sbase + L::off_q + slot * L::kQ,
+                    args.q + (static_cast<size_t>(b) * args.Hq + hk * G) * D, L::kQ, bar);
+        ++u;
+      }
+    }
+    if (ok) {
+      // end of stream
+      const int slot = u % L::kStages, round = u / L::kStages;
+      if (round == 0 || mbar_wait(empty0 + 8 * slot, (round - 1) & 1, abort_flag, args.status,
+                                  args.timeout_ns, EA_ERR_TIMEOUT)) {
+        desc[slot].n = -1;
+        mbar_arrive(full0 + 8 * slot);
+        return;
+      }
+    }
+    // aborted: let the copies in flight land before the CTA exits
+    for (int v = max(0, u - L::kStages); v < u; ++v)
+      mbar_wait_drain(full0 + 8 * (v % L::kStages), (v / L::kStages) & 1, args.timeout_ns);
+    return;
+  }
+
+  // ---------------- consumers
+  regs_inc<kDecRegsConsumer>();
+  const int sub = lane / L::kLPR, cl = lane % L::kLPR;
+  const int rg = warp * L::kRGW + sub;
+  float qf[G][L::kDPL], o[G][L::kDPL], m[G], l[G];
+  uint32_t sparse_bits = 0;
+  int t = 0, a = 0, lo = 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m[g] = kDecNegBig;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < L::kDPL; ++e) { o[g][e] = 0.f; qf[g][e] = 0.f; }
+  }
+  for (int u = 0;; ++u) {
+    const int slot = u % L::kStages, round = u / L::kStages;
+    if (!mbar_wait(full0 + 8 * slot, round & 1, abort_flag, args.status, args.timeout_ns,
+                   EA_ERR_TIMEOUT))
+      break;
+    const DecDesc d = desc[slot];
+    if (d.n < 0) break;
+    if (d.first) {
+      sparse_bits = d.sparse_bits;
+      t = d.t; a = d.a; lo = d.lo;
+      const uint8_t* qs = smem + L::off_q + slot * L::kQ;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int i = 0; i < L::kChunks; ++i) {
+          const uint4 raw =
+              *reinterpret_cast<const uint4*>(qs + (g * D + (cl + i * L::kLPR) * 8) * 2);
+          float f[8];
+          bf16x8_to_f32(raw, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) qf[g][i * 8 + e] = f[e] * args.scale_log2;
+        }
+        m[g] = kDecNegBig;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
+      }
+    }
+    const uint8_t* ks = smem + L::off_k + slot * L::kKV;
+    const uint8_t* vs = smem + L::off_v + slot * L::kKV;
+#pragma unroll
+    for (int k = 0; k < L::kRPS; ++k) {
+      const int r = rg + k * L::kNG;
+      const bool valid = r < d.n;
+      float kf[L::kDPL], vf[L::kDPL];
+#pragma unroll
+      for (int i = 0; i < L::kChunks; ++i) {
+        const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + off), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kf[i * 8 + e] = f[e];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + off), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) vf[i * 8 + e] = f[e];
+      }
+      float sc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < L::kDPL; e += 2) fma2_acc(s0, s1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1]);
+        sc[g] = s0 + s1;
+      }
+#pragma unroll
+      for (int off = L::kLPR / 2; off > 0; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
+      if (valid) {
+        const int j = d.js + r;
+        const int p = j < a ? j : lo + (j - a);
+        const bool in_sa = p < args.sink || t - p < args.window;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const bool seen = in_sa || !((sparse_bits >> g) & 1u);
+          const float sg = seen ? sc[g] : -INFINITY;
+          if (sg > m[g] + kDecRescale) {
+            const float alpha = ex2_approx(m[g] - sg);
+            l[g] *= alpha;
+#pragma unroll
+            for (int e = 0; e < L::kDPL; ++e) o[g][e] *= alpha;
+            m[g] = sg;
+          }
+          const float pr = ex2_approx(sg - m[g]);
+          l[g] += pr;
+#pragma unroll
+          for (int e = 0; e < L::kDPL; e += 2) fma2_acc(o[g][e], o[g][e + 1], pr, pr, vf[e], vf[e + 1]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+
+    if (d.last) {
+      // merge the row groups of this warp (lanes cl, cl + kLPR, ...)
+#pragma unroll
+      for (int off = L::kLPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
+          const float lo_ = __shfl_xor_sync(0xffffffffu, l[g], off);
+          const float mn = fmaxf(m[g], mo);
+          const float as = ex2_approx(m[g] - mn), ao = ex2_approx(mo - mn);
+          l[g] = l[g] * as + lo_ * ao;
+#pragma unroll
+          for (int e = 0; e < L::kDPL; ++e) {
+            const float oo = __shfl_xor_sync(0xffffffffu, o[g][e], off);
+            o[g][e] = o[g][e] * as + oo * ao;
+          }
+          m[g] = mn;
+        }
+      }
+      float* s_mo = reinterpret_cast<float*>(smem + L::off_mo);
+      float* s_ml = reinterpret_cast<float*>(smem + L::off_ml);
+      if (sub == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+          for (int i = 0; i < L::kChunks; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              s_mo[(warp * G + g) * D + (cl + i * L::kLPR) * 8 + e] = o[g][i * 8 + e];
+          if (cl == 0) {
+            s_ml[(warp * G + g) * 2] = m[g];
+            s_ml[(warp * G + g) * 2 + 1] = l[g];
+          }
+        }
+      }
+      named_bar_consumers();
+      const int hq0 = d.b * args.Hq + d.hk * G;
+      for (int idx = threadIdx.x; idx < G * (D + 2); idx += kDecConsumerWarps * 32) {
+        const int g = idx / (D + 2), c = idx % (D + 2);
+        float mx = kDecNegBig;
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) mx = fmaxf(mx, s_ml[(w * G + g) * 2]);
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) {
+          const float sw = ex2_approx(s_ml[(w * G + g) * 2] - mx);
+          const float x = c < D ? s_mo[(w * G + g) * D + c] : s_ml[(w * G + g) * 2 + 1];
+          acc += x * sw;
+        }
+        float* pb = args.part + ((static_cast<size_t>(hq0 + g)) * args.nsplit + d.chunk) * (D + 2);
+        pb[c == D + 1 ? D + 1 : c] = (c == D) ? mx : acc;
+      }
+      named_bar_consumers();
+      // reset for the next item (also done when its first stage arrives)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        m[g] = kDecNegBig;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
+      }
+    }
+  }
+}
+
+// out[b, h] = merge of the item partials of (b, h) in chunk order.
 __global__ void ea_decode_combine_kernel(DecodeArgs args) {
   const int hq = blockIdx.x, b = blockIdx.y;
   const int D = args.d;
+  const int G = args.Hq / args.Hkv;
+  const DecGroup grp = dec_group(args, b, hq / G, G);
+  const int nused = (grp.nvis + kDecChunk - 1) / kDecChunk;
   const float* pb = args.part + (static_cast<size_t>(b) * args.Hq + hq) * args.nsplit * (D + 2);
-  float mm = -INFINITY;
-  for (int s = 0; s < args.nsplit; ++s) mm = fmaxf(mm, pb[static_cast<size_t>(s) * (D + 2) + D]);
+  float mm = kDecNegBig;
+  for (int s = 0; s < nused; ++s) mm = fmaxf(mm, pb[static_cast<size_t>(s) * (D + 2) + D]);
   float ls = 0.f;
-  for (int s = 0; s < args.nsplit; ++s) {
-    const float ms = pb[static_cast<size_t>(s) * (D + 2) + D];
-    if (ms != -INFINITY) ls += pb[static_cast<size_t>(s) * (D + 2) + D + 1] * exp2f(ms - mm);
-  }
+  for (int s = 0; s < nused; ++s)
+    ls += pb[static_cast<size_t>(s) * (D + 2) + D + 1] *
+          ex2_approx(pb[static_cast<size_t>(s) * (D + 2) + D] - mm);
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float acc = 0.f;
-    for (int s = 0; s < args.nsplit; ++s) {
-      const float ms = pb[static_cast<size_t>(s) * (D + 2) + D];
-      if (ms != -INFINITY) acc += pb[static_cast<size_t>(s) * (D + 2) + c] * exp2f(ms - mm);
-    }
+    for (int s = 0; s < nused; ++s)
+      acc += pb[static_cast<size_t>(s) * (D + 2) + c] *
+             ex2_approx(pb[static_cast<size_t>(s) * (D + 2) + D] - mm);
     // no visible key (a rejected slot or position): zero output
     args.out[(static_cast<size_t>(b) * args.Hq + hq) * D + c] =
         __float2bfloat16_rn(ls > 0.f ? acc / ls : 0.f);
@@ -284,17 +536,35 @@ __global__ void ea_decode_combine_kernel(DecodeArgs args) {
 
 int decode_num_splits(int max_len) { return (max_len + kDecChunk - 1) / kDecChunk; }
 
+template <int D, int G>
+static cudaError_t launch_attn_dec_g(const DecodeArgs& a, cudaStream_t stream) {
+  using L = DecLayout<D, G>;
+  static int configured[64] = {0};   // per device: the attribute is per context
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev >= 64 || !configured[dev]) {
+    err = cudaFuncSetAttribute(ea_decode_attn_kernel<D, G>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::bytes(kDecMaxGroups));
+    if (err != cudaSuccess) return err;
+    if (dev < 64) configured[dev] = 1;
+  }
+  const int grid = device_sms();
+  if (grid <= 0) return cudaErrorInvalidDevice;
+  ea_decode_attn_kernel<D, G><<<grid, kDecKernelThreads, L::bytes(a.B * a.Hkv), stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_attn_dec(const DecodeArgs& a, int G, cudaStream_t stream) {
-  dim3 grid(a.nsplit, a.Hkv, a.B);
   switch (G) {
-    case 1: ea_decode_attn_kernel<D, 1><<<grid, kDecThreads, 0, stream>>>(a); break;
-    case 2: ea_decode_attn_kernel<D, 2><<<grid, kDecThreads, 0, stream>>>(a); break;
-    case 4: ea_decode_attn_kernel<D, 4><<<grid, kDecThreads, 0, stream>>>(a); break;
-    case 8: ea_decode_attn_kernel<D, 8><<<grid, kDecThreads, 0, stream>>>(a); break;
+    case 1: return launch_attn_dec_g<D, 1>(a, stream);
+    case 2: return launch_attn_dec_g<D, 2>(a, stream);
+    case 4: return launch_attn_dec_g<D, 4>(a, stream);
+    case 8: return launch_attn_dec_g<D, 8>(a, stream);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
@@ -325,6 +595,7 @@ ea_status check_decode(const ea_decode_params* p) {
   if (G != 1 && G != 2 && G != 4 && G != 8) return EA_ERR_UNSUPPORTED;
   if (p->max_len >= (1 << 30)) return EA_ERR_UNSUPPORTED;
   if (p->n_full < 0 || p->n_sa < 0 || p->n_full + p->n_sa <= 0) return EA_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->B) * p->Hkv > ea::kDecMaxGroups) return EA_ERR_UNSUPPORTED;
   return EA_OK;
 }
 }  // namespace
@@ -401,6 +672,7 @@ ea_status ea_hybrid_attn_decode(const void* q, const void* k_new, const void* v_
                                                                      : p->sink + p->window);
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = ea::wait_timeout_ns();
   cudaError_t err = ea::launch_decode(a, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }

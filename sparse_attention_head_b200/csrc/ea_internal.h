@@ -27,6 +27,11 @@ struct alignas(64) AttnArgs {
   int debug_drop_kv_pos;
 };
 
+// SM count of the current device (cached per device); 0 on error.
+int device_sms();
+// Bound of every device-side wait, from EA_WAIT_TIMEOUT_MS (default 2 s).
+unsigned long long wait_timeout_ns();
+
 // Dynamic shared memory the kernel for head dim D needs.
 int attn_smem_bytes(int D);
 

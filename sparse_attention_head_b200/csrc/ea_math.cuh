@@ -26,6 +26,19 @@ __device__ __forceinline__ void fma2_sc(float& y0, float& y1, float x0, float x1
       : "f"(x0), "f"(x1), "f"(s), "f"(c));
 }
 
+// (c0, c1) = (a0 * b0 + c0, a1 * b1 + c1), one packed instruction.
+__device__ __forceinline__ void fma2_acc(float& c0, float& c1, float a0, float a1, float b0,
+                                         float b1) {
+  asm("{\n\t.reg .b64 ab, bb, cb;\n\t"
+      "mov.b64 ab, {%2, %3};\n\t"
+      "mov.b64 bb, {%4, %5};\n\t"
+      "mov.b64 cb, {%0, %1};\n\t"
+      "fma.rn.f32x2 cb, ab, bb, cb;\n\t"
+      "mov.b64 {%0, %1}, cb;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // (a0, a1) += (x0, x1), one packed instruction.
 __device__ __forceinline__ void add2_acc(float& a0, float& a1, float x0, float x1) {
   asm("{\n\t.reg .b64 ab, xb;\n\t"
