@@ -9,7 +9,7 @@
 // FA query head keeps every position.  The query at position t sees exactly
 // the keys prefill row t sees (FA: 0..t; SA: sink + window).
 //
-// Step, all on the caller's stream:
+// Step, two launches on the caller's stream:
 //   1. append: the new k, v of every (b, kv head) go to their cache slot;
 //   2. attention: one persistent CTA per SM walks the (kv group, 512-key
 //      chunk) items that hold visible keys.  A producer warp streams each
@@ -19,8 +19,8 @@
 //      warps read every row once for all G query heads of the group, keep an
 //      fp32 online softmax per head and write one partial (o, max, sum) per
 //      item and head to the workspace;
-//   3. combine: the partials of each (b, query head) are merged in chunk
-//      order and written as bf16.
+//      the CTA that completes a group's last item merges the group's partials
+//      in chunk order and writes the bf16 output.
 // The step is HBM-bound: its work is one read of every visible cache row.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -49,6 +49,7 @@ struct DecodeArgs {
   __nv_bfloat16* v_sa;
   __nv_bfloat16* out;          // [B][Hq][d]
   float* part;                 // [B][Hq][nsplit][d + 2]: o, max, sum
+  int* counters;               // [B][Hkv]: items of the group finished this step
   int* status;
   int B, Hq, Hkv, d, sink, window, max_len, nsplit, n_full, n_sa;
   float scale_log2;
@@ -85,8 +86,13 @@ __global__ void ea_decode_append_kernel(DecodeArgs args) {
   const int b = blockIdx.y, hk = blockIdx.x;
   const int t = args.pos[b];
   const int slot = args.cache_slot[b * args.Hkv + hk];
+  if (threadIdx.x == 0) args.counters[b * args.Hkv + hk] = 0;
   if (!dec_slot_ok(args, slot, t)) {
     if (threadIdx.x == 0) atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);
+    // no work item reads or writes this group: its outputs are zero
+    const int G = args.Hq / args.Hkv;
+    __nv_bfloat16* o = args.out + (static_cast<size_t>(b) * args.Hq + hk * G) * args.d;
+    for (int i = threadIdx.x; i < G * args.d; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
     return;
   }
   if (slot < 0 && threadIdx.x == 0) {   // a compact cache behind an FA query head
@@ -143,13 +149,28 @@ __device__ __forceinline__ DecGroup dec_group(const DecodeArgs& args, int b, int
   return g;
 }
 
-// One 64-row stage of an item, written by the producer before it arms the
-// stage's full barrier.  n < 0 ends the stream.
+// One stage of an item, written by the producer before it arms the stage's
+// full barrier.  n < 0 ends the stream.
 struct DecDesc {
-  int n, js, t, a, lo, b, hk, chunk, first, last;
+  int n, js, t, a, lo, b, hk;
+  int seg, nseg;       // this CTA's segment of the group, and the group's segment count
+  int first, last;     // first / last stage of the segment
   uint32_t sparse_bits;
-  int pad[5];
+  int pad[4];
 };
+
+// Balanced contiguous split of `total` items over `grid` CTAs: CTA c owns
+// [dec_range_begin(c), dec_range_begin(c + 1)).
+__device__ __forceinline__ int dec_range_begin(int c, int total, int grid) {
+  const int q = total / grid, r = total % grid;
+  return c * q + min(c, r);
+}
+// The CTA whose range holds item i.
+__device__ __forceinline__ int dec_cta_of(int i, int total, int grid) {
+  const int q = total / grid, r = total % grid;
+  const int big = r * (q + 1);
+  return i < big ? i / (q + 1) : r + (i - big) / q;
+}
 
 constexpr int kDecConsumerWarps = 8;                              // warpgroups 0 and 1
 constexpr int kDecKernelThreads = (kDecConsumerWarps + 4) * 32;   // + producer warpgroup
@@ -160,8 +181,8 @@ constexpr int kDecRegsProducer = 56;
 constexpr int kDecRegsConsumer = 224;
 static_assert(128 * kDecRegsProducer + 256 * kDecRegsConsumer <= kDecKernelThreads * 168,
               "register split exceeds the launch's registers");
-constexpr int kDecStageRows = 64;
-constexpr int kDecMaxGroups = 4096;                                // B * Hkv
+constexpr int kDecStageBytes = 16384;      // K (or V) bytes per stage: 64 rows of d = 128
+constexpr int kDecMaxGroups = 4096;        // B * Hkv
 constexpr float kDecNegBig = -1.0e30f;     // running max before the first key
 constexpr float kDecRescale = 8.0f;        // rescale only when the max grows by > 2^8
 
@@ -172,10 +193,12 @@ struct DecLayout {
   static constexpr int kChunks = kDPL / 8;           // 16-byte chunks per lane
   static constexpr int kRGW = 32 / kLPR;             // row groups per warp
   static constexpr int kNG = kDecConsumerWarps * kRGW;
-  static constexpr int kRPS = kDecStageRows / kNG;   // rows per group per stage
-  static constexpr int kStages = (D == 128) ? 4 : 6;
   static constexpr int kRowBytes = D * 2;
-  static constexpr int kKV = kDecStageRows * kRowBytes;
+  static constexpr int kStageRows = kDecStageBytes / kRowBytes;   // 64 or 128
+  static constexpr int kRPS = kStageRows / kNG;      // rows per group per stage
+  static constexpr int kRB = (G == 8) ? 2 : kRPS;    // rows per batch (registers)
+  static constexpr int kStages = 4;
+  static constexpr int kKV = kDecStageBytes;
   static constexpr int kQ = G * D * 2;
   static constexpr int off_k = 0;
   static constexpr int off_v = off_k + kStages * kKV;
@@ -183,12 +206,12 @@ struct DecLayout {
   static constexpr int off_desc = off_q + kStages * kQ;
   static constexpr int off_full = off_desc + kStages * static_cast<int>(sizeof(DecDesc));
   static constexpr int off_empty = off_full + kStages * 8;
-  static constexpr int off_flag = off_empty + kStages * 8;
+  static constexpr int off_flag = off_empty + kStages * 8;    // abort flag, last-item flag
   static constexpr int off_mo = off_flag + 16;
   static constexpr int off_ml = off_mo + kDecConsumerWarps * G * D * 4;
   static constexpr int off_table = off_ml + kDecConsumerWarps * G * 2 * 4;
   static constexpr int bytes(int ngroups) { return off_table + (ngroups + 1) * 4; }
-  static_assert(kDecStageRows % kNG == 0 && kRPS >= 1, "stage rows per row group");
+  static_assert(kStageRows % kNG == 0 && kRPS >= 1 && kRPS % kRB == 0, "stage rows");
   static_assert(sizeof(DecDesc) == 64, "descriptor size");
   static_assert(off_full % 8 == 0 && off_q % 16 == 0, "alignment");
 };
@@ -207,14 +230,18 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
 }
 
 // Persistent split-K decode attention.  Work item = (kv group, 512-key
-// chunk) with at least one visible key; CTA c takes items c, c + grid, ...
-// Warp 8 (producer) builds the item table, then streams each item's visible
-// cache rows (contiguous runs: sinks, window, ring wrap) and its G query rows
-// into a ring of 64-row stages with bulk copies.  Warps 0-7 (consumers) take
-// a stage: every key row is read by kLPR lanes, the G dot products reduced
-// by shuffles, and an fp32 online softmax kept per row group and head; the
-// last stage of an item merges the row groups and writes the item's partial
-// (o, max, sum) for every query head of the group.
+// chunk) with at least one visible key, ordered by group then chunk; CTA c
+// owns one contiguous, balanced range of items, so a group's chunks fall in
+// one or a few consecutive CTAs (its segments).  Warp 8 (producer) builds the
+// item table, then streams its items' visible cache rows (contiguous runs:
+// sinks, window, ring wrap) and, once per segment, the G query rows into a
+// ring of 32 KB stages with bulk copies.  Warps 0-7 (consumers) take a stage:
+// every key row is read by kLPR lanes, the G dot products of a batch of rows
+// reduced by interleaved shuffles, and an fp32 online softmax kept per row
+// group and head (one max update per batch) across the whole segment.  The
+// segment's last stage merges the row groups and writes one partial
+// (o, max, sum) per query head; the CTA that completes a group's last segment
+// merges its partials in segment order and writes the bf16 output.
 template <int D, int G>
 __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(DecodeArgs args) {
   using L = DecLayout<D, G>;
@@ -223,6 +250,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
   const uint32_t sbase = smem_u32(smem);
   DecDesc* desc = reinterpret_cast<DecDesc*>(smem + L::off_desc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::off_flag);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::off_flag + 4);
   int* table = reinterpret_cast<int*>(smem + L::off_table);
   const uint32_t full0 = sbase + L::off_full, empty0 = sbase + L::off_empty;
   const int ngroups = args.B * args.Hkv;
@@ -234,6 +262,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
                    "n"(kDecConsumerWarps) : "memory");
     }
     *abort_flag = 0;
+    *last_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -265,13 +294,20 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
 
     // ---------------- producer: stream the stages
     const int total = table[ngroups];
+    const int grid = gridDim.x, cta = blockIdx.x;
+    const int i0 = dec_range_begin(cta, total, grid), i1 = dec_range_begin(cta + 1, total, grid);
     int u = 0;                 // stage uses issued
     int gi = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+    for (int it = i0; it < i1 && ok; ++it) {
       while (table[gi + 1] <= it) ++gi;
       const int b = gi / args.Hkv, hk = gi % args.Hkv;
       const int chunk = it - table[gi];
+      const bool seg_first = it == i0 || chunk == 0;
+      const bool seg_last = it == i1 - 1 || it == table[gi + 1] - 1;
+      const int cta_first = dec_cta_of(table[gi], total, grid);
+      const int seg = cta - cta_first;
+      const int nseg = dec_cta_of(table[gi + 1] - 1, total, grid) - cta_first + 1;
       const DecGroup g = dec_group(args, b, hk, G);
       const __nv_bfloat16* kbase;
       const __nv_bfloat16* vbase;
@@ -285,20 +321,22 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         vbase = args.v_full + c * D;
       }
       const int j0 = chunk * kDecChunk, j1 = min(g.nvis, j0 + kDecChunk);
-      for (int js = j0; js < j1; js += kDecStageRows) {
+      for (int js = j0; js < j1; js += L::kStageRows) {
         const int slot = u % L::kStages, round = u / L::kStages;
         if (round > 0 && !mbar_wait(empty0 + 8 * slot, (round - 1) & 1, abort_flag, args.status,
                                     args.timeout_ns, EA_ERR_TIMEOUT)) {
           ok = false;
           break;
         }
-        const int n = min(kDecStageRows, j1 - js);
+        const int n = min(L::kStageRows, j1 - js);
         DecDesc& d = desc[slot];
         d.n = n; d.js = js; d.t = g.t; d.a = g.a; d.lo = g.lo; d.b = b; d.hk = hk;
-        d.chunk = chunk; d.first = js == j0; d.last = js + kDecStageRows >= j1;
+        d.seg = seg; d.nseg = nseg;
+        const bool first = seg_first && js == j0;
+        d.first = first; d.last = seg_last && js + L::kStageRows >= j1;
         d.sparse_bits = g.sparse_bits;
         const uint32_t bar = full0 + 8 * slot;
-        mbar_arrive_expect_tx(bar, 2u * n * L::kRowBytes + (js == j0 ? L::kQ : 0));
+        mbar_arrive_expect_tx(bar, 2u * n * L::kRowBytes + (first ? L::kQ : 0));
         const uint32_t kdst = sbase + L::off_k + slot * L::kKV;
         const uint32_t vdst = sbase + L::off_v + slot * L::kKV;
         for (int j = js; j < js + n;) {
@@ -325,7 +363,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
           bulk_load(vdst + off, vbase + static_cast<size_t>(crow) * D, run * L::kRowBytes, bar);
           j += run;
         }
-        if (js == j0)
+        if (first)
           bulk_load(sbase + L::off_q + slot * L::kQ,
                     args.q + (static_cast<size_t>(b) * args.Hq + hk * G) * D, L::kQ, bar);
         ++u;
@@ -349,11 +387,10 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
 
   // ---------------- consumers
   regs_inc<kDecRegsConsumer>();
+  constexpr uint32_t kAllBits = (1u << G) - 1u;
   const int sub = lane / L::kLPR, cl = lane % L::kLPR;
   const int rg = warp * L::kRGW + sub;
   float qf[G][L::kDPL], o[G][L::kDPL], m[G], l[G];
-  uint32_t sparse_bits = 0;
-  int t = 0, a = 0, lo = 0;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m[g] = kDecNegBig;
@@ -369,8 +406,6 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
     const DecDesc d = desc[slot];
     if (d.n < 0) break;
     if (d.first) {
-      sparse_bits = d.sparse_bits;
-      t = d.t; a = d.a; lo = d.lo;
       const uint8_t* qs = smem + L::off_q + slot * L::kQ;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -389,55 +424,96 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
       }
     }
+    const bool full = d.n == L::kStageRows;
+    // only a group with both FA and SA heads tests key positions
+    const bool mixed = d.sparse_bits != 0 && d.sparse_bits != kAllBits;
     const uint8_t* ks = smem + L::off_k + slot * L::kKV;
     const uint8_t* vs = smem + L::off_v + slot * L::kKV;
 #pragma unroll
-    for (int k = 0; k < L::kRPS; ++k) {
-      const int r = rg + k * L::kNG;
-      const bool valid = r < d.n;
-      float kf[L::kDPL], vf[L::kDPL];
+    for (int kb = 0; kb < L::kRPS; kb += L::kRB) {
+      uint4 kr[L::kRB][L::kChunks], vr[L::kRB][L::kChunks];
+      bool valid[L::kRB];
 #pragma unroll
-      for (int i = 0; i < L::kChunks; ++i) {
-        const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
-        float f[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + off), f);
+      for (int kk = 0; kk < L::kRB; ++kk) {
+        const int r = rg + (kb + kk) * L::kNG;
+        valid[kk] = full || r < d.n;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kf[i * 8 + e] = f[e];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + off), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) vf[i * 8 + e] = f[e];
+        for (int i = 0; i < L::kChunks; ++i) {
+          const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
+          kr[kk][i] = *reinterpret_cast<const uint4*>(ks + off);
+          // rows past the stage's end hold stale bytes: never multiply them
+          vr[kk][i] = valid[kk] ? *reinterpret_cast<const uint4*>(vs + off)
+                                : make_uint4(0, 0, 0, 0);
+        }
       }
-      float sc[G];
+      float sc[L::kRB][G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float s0 = 0.f, s1 = 0.f;
+      for (int kk = 0; kk < L::kRB; ++kk) {
+        float a0[G], a1[G];
 #pragma unroll
-        for (int e = 0; e < L::kDPL; e += 2) fma2_acc(s0, s1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1]);
-        sc[g] = s0 + s1;
+        for (int g = 0; g < G; ++g) { a0[g] = 0.f; a1[g] = 0.f; }
+#pragma unroll
+        for (int i = 0; i < L::kChunks; ++i) {
+          float kf[8];
+          bf16x8_to_f32(kr[kk][i], kf);
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < 8; e += 2)
+              fma2_acc(a0[g], a1[g], qf[g][i * 8 + e], qf[g][i * 8 + e + 1], kf[e], kf[e + 1]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) sc[kk][g] = a0[g] + a1[g];
       }
 #pragma unroll
       for (int off = L::kLPR / 2; off > 0; off >>= 1)
 #pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
-      if (valid) {
-        const int j = d.js + r;
-        const int p = j < a ? j : lo + (j - a);
-        const bool in_sa = p < args.sink || t - p < args.window;
+        for (int kk = 0; kk < L::kRB; ++kk)
+#pragma unroll
+          for (int g = 0; g < G; ++g) sc[kk][g] += __shfl_xor_sync(0xffffffffu, sc[kk][g], off);
+      if (!full || mixed) {
+#pragma unroll
+        for (int kk = 0; kk < L::kRB; ++kk) {
+          const int j = d.js + rg + (kb + kk) * L::kNG;
+          const int p = j < d.a ? j : d.lo + (j - d.a);
+          const bool in_sa = p < args.sink || d.t - p < args.window;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const bool seen = valid[kk] && (in_sa || !((d.sparse_bits >> g) & 1u));
+            sc[kk][g] = seen ? sc[kk][g] : -INFINITY;
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mx = sc[0][g];
+#pragma unroll
+        for (int kk = 1; kk < L::kRB; ++kk) mx = fmaxf(mx, sc[kk][g]);
+        if (mx > m[g] + kDecRescale) {
+          const float alpha = ex2_approx(m[g] - mx);
+          l[g] *= alpha;
+#pragma unroll
+          for (int e = 0; e < L::kDPL; ++e) o[g][e] *= alpha;
+          m[g] = mx;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < L::kRB; ++kk) {
+        float pr[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const bool seen = in_sa || !((sparse_bits >> g) & 1u);
-          const float sg = seen ? sc[g] : -INFINITY;
-          if (sg > m[g] + kDecRescale) {
-            const float alpha = ex2_approx(m[g] - sg);
-            l[g] *= alpha;
+          pr[g] = ex2_approx(sc[kk][g] - m[g]);
+          l[g] += pr[g];
+        }
 #pragma unroll
-            for (int e = 0; e < L::kDPL; ++e) o[g][e] *= alpha;
-            m[g] = sg;
-          }
-          const float pr = ex2_approx(sg - m[g]);
-          l[g] += pr;
+        for (int i = 0; i < L::kChunks; ++i) {
+          float vf[8];
+          bf16x8_to_f32(vr[kk][i], vf);
 #pragma unroll
-          for (int e = 0; e < L::kDPL; e += 2) fma2_acc(o[g][e], o[g][e + 1], pr, pr, vf[e], vf[e + 1]);
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < 8; e += 2)
+              fma2_acc(o[g][i * 8 + e], o[g][i * 8 + e + 1], pr[g], pr[g], vf[e], vf[e + 1]);
         }
       }
     }
@@ -493,11 +569,37 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
           const float x = c < D ? s_mo[(w * G + g) * D + c] : s_ml[(w * G + g) * 2 + 1];
           acc += x * sw;
         }
-        float* pb = args.part + ((static_cast<size_t>(hq0 + g)) * args.nsplit + d.chunk) * (D + 2);
-        pb[c == D + 1 ? D + 1 : c] = (c == D) ? mx : acc;
+        float* pb = args.part + ((static_cast<size_t>(hq0 + g)) * args.nsplit + d.seg) * (D + 2);
+        pb[c] = (c == D) ? mx : acc;
+      }
+      // publish the partial; the CTA that completes the group merges it
+      __threadfence();
+      named_bar_consumers();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(args.counters + d.b * args.Hkv + d.hk, 1);
+        *last_flag = prev == d.nseg - 1;
+        __threadfence();
       }
       named_bar_consumers();
-      // reset for the next item (also done when its first stage arrives)
+      if (*last_flag) {
+        for (int idx = threadIdx.x; idx < G * D; idx += kDecConsumerWarps * 32) {
+          const int g = idx / D, c = idx % D;
+          const float* pb = args.part + static_cast<size_t>(hq0 + g) * args.nsplit * (D + 2);
+          float mx = kDecNegBig;
+          for (int sp = 0; sp < d.nseg; ++sp)
+            mx = fmaxf(mx, __ldcg(pb + static_cast<size_t>(sp) * (D + 2) + D));
+          float acc = 0.f, sum = 0.f;
+          for (int sp = 0; sp < d.nseg; ++sp) {
+            const float* ps = pb + static_cast<size_t>(sp) * (D + 2);
+            const float w = ex2_approx(__ldcg(ps + D) - mx);
+            acc += __ldcg(ps + c) * w;
+            sum += __ldcg(ps + D + 1) * w;
+          }
+          args.out[static_cast<size_t>(hq0 + g) * D + c] =
+              __float2bfloat16_rn(sum > 0.f ? acc / sum : 0.f);
+        }
+      }
+      // reset for the next segment (also done when its first stage arrives)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m[g] = kDecNegBig;
@@ -506,31 +608,6 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
       }
     }
-  }
-}
-
-// out[b, h] = merge of the item partials of (b, h) in chunk order.
-__global__ void ea_decode_combine_kernel(DecodeArgs args) {
-  const int hq = blockIdx.x, b = blockIdx.y;
-  const int D = args.d;
-  const int G = args.Hq / args.Hkv;
-  const DecGroup grp = dec_group(args, b, hq / G, G);
-  const int nused = (grp.nvis + kDecChunk - 1) / kDecChunk;
-  const float* pb = args.part + (static_cast<size_t>(b) * args.Hq + hq) * args.nsplit * (D + 2);
-  float mm = kDecNegBig;
-  for (int s = 0; s < nused; ++s) mm = fmaxf(mm, pb[static_cast<size_t>(s) * (D + 2) + D]);
-  float ls = 0.f;
-  for (int s = 0; s < nused; ++s)
-    ls += pb[static_cast<size_t>(s) * (D + 2) + D + 1] *
-          ex2_approx(pb[static_cast<size_t>(s) * (D + 2) + D] - mm);
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < nused; ++s)
-      acc += pb[static_cast<size_t>(s) * (D + 2) + c] *
-             ex2_approx(pb[static_cast<size_t>(s) * (D + 2) + D] - mm);
-    // no visible key (a rejected slot or position): zero output
-    args.out[(static_cast<size_t>(b) * args.Hq + hq) * D + c] =
-        __float2bfloat16_rn(ls > 0.f ? acc / ls : 0.f);
   }
 }
 
@@ -572,10 +649,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int G = a.Hq / a.Hkv;
-  err = a.d == 128 ? launch_attn_dec<128>(a, G, stream) : launch_attn_dec<64>(a, G, stream);
-  if (err != cudaSuccess) return err;
-  ea_decode_combine_kernel<<<dim3(a.Hq, a.B), 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  return a.d == 128 ? launch_attn_dec<128>(a, G, stream) : launch_attn_dec<64>(a, G, stream);
 }
 
 }  // namespace ea
@@ -583,6 +657,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 // ------------------------------------------------------------------ C ABI
 namespace {
 bool dec_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace: status word (256 B), per-group item counters (rounded up to
+// 256 B), then the partials.
+size_t dec_counter_bytes(const ea_decode_params* p) {
+  const size_t n = static_cast<size_t>(p->B) * p->Hkv * sizeof(int);
+  return (n + 255) / 256 * 256;
+}
 
 ea_status check_decode(const ea_decode_params* p) {
   if (!p) return EA_ERR_INVALID_ARG;
@@ -606,7 +687,7 @@ size_t ea_decode_workspace_size(const ea_decode_params* p) {
   if (check_decode(p) != EA_OK) return 0;
   const size_t ns = ea::decode_num_splits(p->max_len > p->sink + p->window
                                               ? p->max_len : p->sink + p->window);
-  return 256 + static_cast<size_t>(p->B) * p->Hq * ns * (p->d + 2) * sizeof(float);
+  return 256 + dec_counter_bytes(p) + static_cast<size_t>(p->B) * p->Hq * ns * (p->d + 2) * sizeof(float);
 }
 
 int ea_decode_kv_policy(const uint8_t* mask, int B, int Hq, int Hkv, int32_t* cache_slot,
@@ -658,7 +739,8 @@ ea_status ea_hybrid_attn_decode(const void* q, const void* k_new, const void* v_
   a.v_sa = static_cast<__nv_bfloat16*>(v_sa);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.status = static_cast<int*>(workspace);
-  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256);
+  a.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + 256);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256 + dec_counter_bytes(p));
   a.B = p->B;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
