@@ -34,7 +34,7 @@
 
 namespace ea {
 
-constexpr int kDecChunk = 512;           // visible keys per work item (at most)
+constexpr int kDecChunk = 512;           // smallest work item (keys): bounds the partials
 
 struct DecodeArgs {
   const __nv_bfloat16* q;      // [B][Hq][d]
@@ -172,33 +172,43 @@ __device__ __forceinline__ int dec_cta_of(int i, int total, int grid) {
   return i < big ? i / (q + 1) : r + (i - big) / q;
 }
 
-constexpr int kDecConsumerWarps = 8;                              // warpgroups 0 and 1
-constexpr int kDecKernelThreads = (kDecConsumerWarps + 4) * 32;   // + producer warpgroup
-// Register split (setmaxnreg): launched at 65536 / 384 = 168 per thread, the
-// producer warpgroup gives back down to 56 and the consumers take 224:
-// 128 * 56 + 256 * 224 = 64512 = 384 * 168.
-constexpr int kDecRegsProducer = 56;
-constexpr int kDecRegsConsumer = 224;
-static_assert(128 * kDecRegsProducer + 256 * kDecRegsConsumer <= kDecKernelThreads * 168,
-              "register split exceeds the launch's registers");
-constexpr int kDecStageBytes = 16384;      // K (or V) bytes per stage: 64 rows of d = 128
+// Consumer warps: 3 warpgroups for G <= 2 (q and o of a lane take at most
+// 16 + 16 register pairs), 2 for G = 4 and 8 (32 + 32 pairs: 16 channels x 4
+// heads, 8 channels x 8 heads); 3 warpgroups at 8 channels per lane measured
+// slower for G = 4 (one more shuffle level per key).  The last warpgroup is
+// the producer.  Register split (setmaxnreg) against the launch's 65536:
+//   G <= 2:   512 threads launched at 128: 128 * 32 + 384 * 160 = 65536
+//   G = 4, 8: 384 threads launched at 168: 128 * 56 + 256 * 224 = 64512
+template <int G>
+struct DecWarps {
+  static constexpr int kConsumers = (G <= 2) ? 12 : 8;
+  static constexpr int kThreads = (kConsumers + 4) * 32;
+  static constexpr int kLaunchRegs = (G <= 2) ? 128 : 168;
+  static constexpr int kRegsProducer = (G <= 2) ? 32 : 56;
+  static constexpr int kRegsConsumer = (G <= 2) ? 160 : 224;
+  static_assert(128 * kRegsProducer + kConsumers * 32 * kRegsConsumer <= kThreads * kLaunchRegs,
+                "register split exceeds the launch's registers");
+  static_assert(kThreads * kLaunchRegs <= 65536, "launch registers");
+};
 constexpr int kDecMaxGroups = 4096;        // B * Hkv
 constexpr float kDecNegBig = -1.0e30f;     // running max before the first key
 constexpr float kDecRescale = 8.0f;        // rescale only when the max grows by > 2^8
 
 template <int D, int G>
 struct DecLayout {
+  static constexpr int kCW = DecWarps<G>::kConsumers;
   static constexpr int kDPL = (G == 8) ? 8 : 16;     // channels per lane
   static constexpr int kLPR = D / kDPL;              // lanes per key row
   static constexpr int kChunks = kDPL / 8;           // 16-byte chunks per lane
   static constexpr int kRGW = 32 / kLPR;             // row groups per warp
-  static constexpr int kNG = kDecConsumerWarps * kRGW;
+  static constexpr int kNG = kCW * kRGW;
   static constexpr int kRowBytes = D * 2;
-  static constexpr int kStageRows = kDecStageBytes / kRowBytes;   // 64 or 128
+  static constexpr int kStageRows = kNG * ((kDPL == 8) ? 4 : 2);   // rows per group: 4 or 2
+  static constexpr int kChunkRows = (kCW == 12) ? 576 : 512;  // keys per work item
   static constexpr int kRPS = kStageRows / kNG;      // rows per group per stage
   static constexpr int kRB = (G == 8) ? 2 : kRPS;    // rows per batch (registers)
-  static constexpr int kStages = 4;
-  static constexpr int kKV = kDecStageBytes;
+  static constexpr int kStages = (kCW == 12) ? 3 : 4;
+  static constexpr int kKV = kStageRows * kRowBytes;
   static constexpr int kQ = G * D * 2;
   static constexpr int off_k = 0;
   static constexpr int off_v = off_k + kStages * kKV;
@@ -206,18 +216,48 @@ struct DecLayout {
   static constexpr int off_desc = off_q + kStages * kQ;
   static constexpr int off_full = off_desc + kStages * static_cast<int>(sizeof(DecDesc));
   static constexpr int off_empty = off_full + kStages * 8;
-  static constexpr int off_flag = off_empty + kStages * 8;    // abort flag, last-item flag
+  static constexpr int off_flag = off_empty + kStages * 8;    // abort flag, last-segment flag
   static constexpr int off_mo = off_flag + 16;
-  static constexpr int off_ml = off_mo + kDecConsumerWarps * G * D * 4;
-  static constexpr int off_table = off_ml + kDecConsumerWarps * G * 2 * 4;
+  static constexpr int off_ml = off_mo + kCW * G * D * 4;
+  static constexpr int off_table = off_ml + kCW * G * 2 * 4;
   static constexpr int bytes(int ngroups) { return off_table + (ngroups + 1) * 4; }
   static_assert(kStageRows % kNG == 0 && kRPS >= 1 && kRPS % kRB == 0, "stage rows");
+  static_assert(kChunkRows % kStageRows == 0 && kChunkRows >= kDecChunk, "chunk rows");
   static_assert(sizeof(DecDesc) == 64, "descriptor size");
-  static_assert(off_full % 8 == 0 && off_q % 16 == 0, "alignment");
+  static_assert(off_full % 8 == 0 && off_q % 16 == 0 && kKV % 16 == 0, "alignment");
 };
 
+template <int kCW>
 __device__ __forceinline__ void named_bar_consumers() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+}
+
+// Packed f32x2 values held in one 64-bit register pair (low word = first
+// element), so the paired FMA needs no moves.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("{\n\t.reg .b32 lo, hi;\n\t"
+      "shl.b32 lo, %1, 16;\n\t"
+      "and.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 %0, {lo, hi};\n\t}"
+      : "=l"(r) : "r"(w));
+  return r;
+}
+__device__ __forceinline__ void ffma2(uint64_t& c, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(c) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t pack2(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t a, float& x, float& y) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a));
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
@@ -232,10 +272,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
 // Persistent split-K decode attention.  Work item = (kv group, 512-key
 // chunk) with at least one visible key, ordered by group then chunk; CTA c
 // owns one contiguous, balanced range of items, so a group's chunks fall in
-// one or a few consecutive CTAs (its segments).  Warp 8 (producer) builds the
+// one or a few consecutive CTAs (its segments).  The producer warp builds the
 // item table, then streams its items' visible cache rows (contiguous runs:
 // sinks, window, ring wrap) and, once per segment, the G query rows into a
-// ring of 32 KB stages with bulk copies.  Warps 0-7 (consumers) take a stage:
+// ring of 64- to 192-row stages with bulk copies.  The consumer warps take a stage:
 // every key row is read by kLPR lanes, the G dot products of a batch of rows
 // reduced by interleaved shuffles, and an fp32 online softmax kept per row
 // group and head (one max update per batch) across the whole segment.  The
@@ -243,8 +283,9 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
 // (o, max, sum) per query head; the CTA that completes a group's last segment
 // merges its partials in segment order and writes the bf16 output.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(DecodeArgs args) {
+__global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kernel(DecodeArgs args) {
   using L = DecLayout<D, G>;
+  using W = DecWarps<G>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = smem_u32(smem);
@@ -259,7 +300,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
     for (int s = 0; s < L::kStages; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * s) : "memory");
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s),
-                   "n"(kDecConsumerWarps) : "memory");
+                   "n"(L::kCW) : "memory");
     }
     *abort_flag = 0;
     *last_flag = 0;
@@ -267,9 +308,9 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
   }
   __syncthreads();
 
-  if (warp >= kDecConsumerWarps) {
-    regs_dec<kDecRegsProducer>();
-    if (warp != kDecConsumerWarps) return;
+  if (warp >= L::kCW) {
+    regs_dec<W::kRegsProducer>();
+    if (warp != L::kCW) return;
     // ---------------- producer: item table (exclusive prefix of chunk counts)
     int carry = 0;
     for (int base = 0; base < ngroups; base += 32) {
@@ -277,7 +318,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
       int cnt = 0;
       if (gi < ngroups) {
         const DecGroup g = dec_group(args, gi / args.Hkv, gi % args.Hkv, G);
-        cnt = (g.nvis + kDecChunk - 1) / kDecChunk;
+        cnt = (g.nvis + L::kChunkRows - 1) / L::kChunkRows;
       }
       int incl = cnt;
 #pragma unroll
@@ -320,7 +361,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         kbase = args.k_full + c * D;
         vbase = args.v_full + c * D;
       }
-      const int j0 = chunk * kDecChunk, j1 = min(g.nvis, j0 + kDecChunk);
+      const int j0 = chunk * L::kChunkRows, j1 = min(g.nvis, j0 + L::kChunkRows);
       for (int js = j0; js < j1; js += L::kStageRows) {
         const int slot = u % L::kStages, round = u / L::kStages;
         if (round > 0 && !mbar_wait(empty0 + 8 * slot, (round - 1) & 1, abort_flag, args.status,
@@ -386,18 +427,21 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
   }
 
   // ---------------- consumers
-  regs_inc<kDecRegsConsumer>();
+  regs_inc<W::kRegsConsumer>();
   constexpr uint32_t kAllBits = (1u << G) - 1u;
+  constexpr int kP = L::kDPL / 2;                    // channel pairs per lane
   const int sub = lane / L::kLPR, cl = lane % L::kLPR;
   const int rg = warp * L::kRGW + sub;
-  float qf[G][L::kDPL], o[G][L::kDPL], m[G], l[G];
+  uint64_t q2[G][kP], o2[G][kP];
+  float m[G], l[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m[g] = kDecNegBig;
     l[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < L::kDPL; ++e) { o[g][e] = 0.f; qf[g][e] = 0.f; }
+    for (int e = 0; e < kP; ++e) { o2[g][e] = 0ull; q2[g][e] = 0ull; }
   }
+  const uint64_t scale2 = pack2(args.scale_log2, args.scale_log2);
   for (int u = 0;; ++u) {
     const int slot = u % L::kStages, round = u / L::kStages;
     if (!mbar_wait(full0 + 8 * slot, round & 1, abort_flag, args.status, args.timeout_ns,
@@ -413,15 +457,14 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         for (int i = 0; i < L::kChunks; ++i) {
           const uint4 raw =
               *reinterpret_cast<const uint4*>(qs + (g * D + (cl + i * L::kLPR) * 8) * 2);
-          float f[8];
-          bf16x8_to_f32(raw, f);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) qf[g][i * 8 + e] = f[e] * args.scale_log2;
+          for (int e = 0; e < 4; ++e) q2[g][i * 4 + e] = fmul2(bf16x2_to_f32x2(w[e]), scale2);
         }
         m[g] = kDecNegBig;
         l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
+        for (int e = 0; e < kP; ++e) o2[g][e] = 0ull;
       }
     }
     const bool full = d.n == L::kStageRows;
@@ -449,21 +492,25 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
       float sc[L::kRB][G];
 #pragma unroll
       for (int kk = 0; kk < L::kRB; ++kk) {
-        float a0[G], a1[G];
+        uint64_t acc[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) { a0[g] = 0.f; a1[g] = 0.f; }
+        for (int g = 0; g < G; ++g) acc[g] = 0ull;
 #pragma unroll
         for (int i = 0; i < L::kChunks; ++i) {
-          float kf[8];
-          bf16x8_to_f32(kr[kk][i], kf);
+          const uint32_t w[4] = {kr[kk][i].x, kr[kk][i].y, kr[kk][i].z, kr[kk][i].w};
 #pragma unroll
-          for (int g = 0; g < G; ++g)
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t k2 = bf16x2_to_f32x2(w[e]);
 #pragma unroll
-            for (int e = 0; e < 8; e += 2)
-              fma2_acc(a0[g], a1[g], qf[g][i * 8 + e], qf[g][i * 8 + e + 1], kf[e], kf[e + 1]);
+            for (int g = 0; g < G; ++g) ffma2(acc[g], q2[g][i * 4 + e], k2);
+          }
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g) sc[kk][g] = a0[g] + a1[g];
+        for (int g = 0; g < G; ++g) {
+          float x, y;
+          unpack2(acc[g], x, y);
+          sc[kk][g] = x + y;
+        }
       }
 #pragma unroll
       for (int off = L::kLPR / 2; off > 0; off >>= 1)
@@ -492,28 +539,30 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         if (mx > m[g] + kDecRescale) {
           const float alpha = ex2_approx(m[g] - mx);
           l[g] *= alpha;
+          const uint64_t a2 = pack2(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < L::kDPL; ++e) o[g][e] *= alpha;
+          for (int e = 0; e < kP; ++e) o2[g][e] = fmul2(o2[g][e], a2);
           m[g] = mx;
         }
       }
 #pragma unroll
       for (int kk = 0; kk < L::kRB; ++kk) {
-        float pr[G];
+        uint64_t p2[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          pr[g] = ex2_approx(sc[kk][g] - m[g]);
-          l[g] += pr[g];
+          const float pr = ex2_approx(sc[kk][g] - m[g]);
+          l[g] += pr;
+          p2[g] = pack2(pr, pr);
         }
 #pragma unroll
         for (int i = 0; i < L::kChunks; ++i) {
-          float vf[8];
-          bf16x8_to_f32(vr[kk][i], vf);
+          const uint32_t w[4] = {vr[kk][i].x, vr[kk][i].y, vr[kk][i].z, vr[kk][i].w};
 #pragma unroll
-          for (int g = 0; g < G; ++g)
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t v2 = bf16x2_to_f32x2(w[e]);
 #pragma unroll
-            for (int e = 0; e < 8; e += 2)
-              fma2_acc(o[g][i * 8 + e], o[g][i * 8 + e + 1], pr[g], pr[g], vf[e], vf[e + 1]);
+            for (int g = 0; g < G; ++g) ffma2(o2[g][i * 4 + e], p2[g], v2);
+          }
         }
       }
     }
@@ -532,9 +581,12 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
           const float as = ex2_approx(m[g] - mn), ao = ex2_approx(mo - mn);
           l[g] = l[g] * as + lo_ * ao;
 #pragma unroll
-          for (int e = 0; e < L::kDPL; ++e) {
-            const float oo = __shfl_xor_sync(0xffffffffu, o[g][e], off);
-            o[g][e] = o[g][e] * as + oo * ao;
+          for (int e = 0; e < kP; ++e) {
+            float x, y;
+            unpack2(o2[g][e], x, y);
+            const float ox = __shfl_xor_sync(0xffffffffu, x, off);
+            const float oy = __shfl_xor_sync(0xffffffffu, y, off);
+            o2[g][e] = pack2(x * as + ox * ao, y * as + oy * ao);
           }
           m[g] = mn;
         }
@@ -547,24 +599,29 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
 #pragma unroll
           for (int i = 0; i < L::kChunks; ++i)
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              s_mo[(warp * G + g) * D + (cl + i * L::kLPR) * 8 + e] = o[g][i * 8 + e];
+            for (int e = 0; e < 4; ++e) {
+              float x, y;
+              unpack2(o2[g][i * 4 + e], x, y);
+              float* dst = s_mo + (warp * G + g) * D + (cl + i * L::kLPR) * 8 + 2 * e;
+              dst[0] = x;
+              dst[1] = y;
+            }
           if (cl == 0) {
             s_ml[(warp * G + g) * 2] = m[g];
             s_ml[(warp * G + g) * 2 + 1] = l[g];
           }
         }
       }
-      named_bar_consumers();
+      named_bar_consumers<L::kCW>();
       const int hq0 = d.b * args.Hq + d.hk * G;
-      for (int idx = threadIdx.x; idx < G * (D + 2); idx += kDecConsumerWarps * 32) {
+      for (int idx = threadIdx.x; idx < G * (D + 2); idx += L::kCW * 32) {
         const int g = idx / (D + 2), c = idx % (D + 2);
         float mx = kDecNegBig;
 #pragma unroll
-        for (int w = 0; w < kDecConsumerWarps; ++w) mx = fmaxf(mx, s_ml[(w * G + g) * 2]);
+        for (int w = 0; w < L::kCW; ++w) mx = fmaxf(mx, s_ml[(w * G + g) * 2]);
         float acc = 0.f;
 #pragma unroll
-        for (int w = 0; w < kDecConsumerWarps; ++w) {
+        for (int w = 0; w < L::kCW; ++w) {
           const float sw = ex2_approx(s_ml[(w * G + g) * 2] - mx);
           const float x = c < D ? s_mo[(w * G + g) * D + c] : s_ml[(w * G + g) * 2 + 1];
           acc += x * sw;
@@ -574,15 +631,15 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
       }
       // publish the partial; the CTA that completes the group merges it
       __threadfence();
-      named_bar_consumers();
+      named_bar_consumers<L::kCW>();
       if (threadIdx.x == 0) {
         const int prev = atomicAdd(args.counters + d.b * args.Hkv + d.hk, 1);
         *last_flag = prev == d.nseg - 1;
         __threadfence();
       }
-      named_bar_consumers();
+      named_bar_consumers<L::kCW>();
       if (*last_flag) {
-        for (int idx = threadIdx.x; idx < G * D; idx += kDecConsumerWarps * 32) {
+        for (int idx = threadIdx.x; idx < G * D; idx += L::kCW * 32) {
           const int g = idx / D, c = idx % D;
           const float* pb = args.part + static_cast<size_t>(hq0 + g) * args.nsplit * (D + 2);
           float mx = kDecNegBig;
@@ -605,7 +662,7 @@ __global__ void __launch_bounds__(kDecKernelThreads, 1) ea_decode_attn_kernel(De
         m[g] = kDecNegBig;
         l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < L::kDPL; ++e) o[g][e] = 0.f;
+        for (int e = 0; e < kP; ++e) o2[g][e] = 0ull;
       }
     }
   }
@@ -629,7 +686,7 @@ static cudaError_t launch_attn_dec_g(const DecodeArgs& a, cudaStream_t stream) {
   }
   const int grid = device_sms();
   if (grid <= 0) return cudaErrorInvalidDevice;
-  ea_decode_attn_kernel<D, G><<<grid, kDecKernelThreads, L::bytes(a.B * a.Hkv), stream>>>(a);
+  ea_decode_attn_kernel<D, G><<<grid, DecWarps<G>::kThreads, L::bytes(a.B * a.Hkv), stream>>>(a);
   return cudaGetLastError();
 }
 
