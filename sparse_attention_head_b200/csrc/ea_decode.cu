@@ -484,10 +484,16 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
         for (int i = 0; i < L::kChunks; ++i) {
           const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
           kr[kk][i] = *reinterpret_cast<const uint4*>(ks + off);
-          // rows past the stage's end hold stale bytes: never multiply them
-          vr[kk][i] = valid[kk] ? *reinterpret_cast<const uint4*>(vs + off)
-                                : make_uint4(0, 0, 0, 0);
+          vr[kk][i] = *reinterpret_cast<const uint4*>(vs + off);
         }
+      }
+      if (!full) {
+        // rows past the stage's end hold stale bytes: never multiply them
+#pragma unroll
+        for (int kk = 0; kk < L::kRB; ++kk)
+#pragma unroll
+          for (int i = 0; i < L::kChunks; ++i)
+            if (!valid[kk]) vr[kk][i] = make_uint4(0, 0, 0, 0);
       }
       float sc[L::kRB][G];
 #pragma unroll
@@ -531,18 +537,26 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
           }
         }
       }
+      // one branch per batch: rescale every head whose max grew by > 2^8
+      float mx[G];
+      bool grow = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float mx = sc[0][g];
+        mx[g] = sc[0][g];
 #pragma unroll
-        for (int kk = 1; kk < L::kRB; ++kk) mx = fmaxf(mx, sc[kk][g]);
-        if (mx > m[g] + kDecRescale) {
-          const float alpha = ex2_approx(m[g] - mx);
+        for (int kk = 1; kk < L::kRB; ++kk) mx[g] = fmaxf(mx[g], sc[kk][g]);
+        grow = grow || mx[g] > m[g] + kDecRescale;
+      }
+      if (grow) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const bool up = mx[g] > m[g] + kDecRescale;
+          const float alpha = up ? ex2_approx(m[g] - mx[g]) : 1.0f;
+          m[g] = up ? mx[g] : m[g];
           l[g] *= alpha;
           const uint64_t a2 = pack2(alpha, alpha);
 #pragma unroll
           for (int e = 0; e < kP; ++e) o2[g][e] = fmul2(o2[g][e], a2);
-          m[g] = mx;
         }
       }
 #pragma unroll
