@@ -48,7 +48,6 @@ namespace {
 using ea::device_sms;
 using ea::wait_timeout_ns;
 
-constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -49,7 +49,7 @@ struct DecodeArgs {
   __nv_bfloat16* v_sa;
   __nv_bfloat16* out;          // [B][Hq][d]
   float* part;                 // [B][Hq][nsplit][d + 2]: o, max, sum
-  int* counters;               // [B][Hkv]: items of the group finished this step
+  int* counters;               // [B][Hkv][2]: segments of each virtual group finished this step
   int* status;
   int B, Hq, Hkv, d, sink, window, max_len, nsplit, n_full, n_sa;
   float scale_log2;
@@ -86,7 +86,7 @@ __global__ void ea_decode_append_kernel(DecodeArgs args) {
   const int b = blockIdx.y, hk = blockIdx.x;
   const int t = args.pos[b];
   const int slot = args.cache_slot[b * args.Hkv + hk];
-  if (threadIdx.x == 0) args.counters[b * args.Hkv + hk] = 0;
+  if (threadIdx.x < 2) args.counters[2 * (b * args.Hkv + hk) + threadIdx.x] = 0;
   if (!dec_slot_ok(args, slot, t)) {
     if (threadIdx.x == 0) atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);
     // no work item reads or writes this group: its outputs are zero
@@ -125,38 +125,52 @@ __global__ void ea_decode_append_kernel(DecodeArgs args) {
   }
 }
 
-// Visible keys of kv group (b, hk) at this step and the heads' routing.
-struct DecGroup {
-  int t, slot, a, lo, nvis;
+// Keys and query heads of virtual group (b, hk, part) at this step.  A kv
+// group whose query heads are all FA or all SA (or that sits on a compact
+// cache) is one virtual group, part 0.  A group on a full cache with both
+// kinds of heads is two: part 0 = its FA heads over every position 0..t,
+// part 1 = its SA heads over the sink and window positions.  Every head of a
+// virtual group sees exactly the group's key list, so nothing is masked
+// inside a list and no SA head spends work on keys it does not see.
+struct DecVGroup {
+  int t, slot, a, lo, nvis;   // keys: [0, a) then [lo, t]; nvis of them (0: empty part)
   bool compact;
-  uint32_t sparse_bits;   // bit g: query head hk*G + g routes to SA
+  uint32_t heads;             // bit g: query head hk * G + g belongs to this part
 };
 
-__device__ __forceinline__ DecGroup dec_group(const DecodeArgs& args, int b, int hk, int G) {
-  DecGroup g;
-  g.t = args.pos[b];
-  g.slot = args.cache_slot[b * args.Hkv + hk];
-  g.compact = g.slot < 0;
-  g.sparse_bits = 0;
-  bool all_sparse = true;
-  for (int i = 0; i < G; ++i) {
-    const bool sp = args.mask[b * args.Hq + hk * G + i] != 0;
-    g.sparse_bits |= static_cast<uint32_t>(sp) << i;
-    all_sparse = all_sparse && sp;
+__device__ __forceinline__ DecVGroup dec_vgroup(const DecodeArgs& args, int b, int hk, int part,
+                                                int G) {
+  DecVGroup v;
+  v.t = args.pos[b];
+  v.slot = args.cache_slot[b * args.Hkv + hk];
+  v.compact = v.slot < 0;
+  uint32_t sparse = 0;
+  for (int i = 0; i < G; ++i)
+    sparse |= static_cast<uint32_t>(args.mask[b * args.Hq + hk * G + i] != 0) << i;
+  const uint32_t all = (1u << G) - 1u;
+  const bool split = sparse != 0 && sparse != all && !v.compact;
+  bool sa_keys;
+  if (!split) {
+    v.heads = part == 0 ? all : 0u;
+    sa_keys = sparse == all || v.compact;
+  } else {
+    v.heads = part == 0 ? (all & ~sparse) : sparse;
+    sa_keys = part == 1;
   }
-  dec_group_keys(all_sparse || g.compact, g.t, args.sink, args.window, &g.a, &g.lo);
-  g.nvis = dec_slot_ok(args, g.slot, g.t) ? g.a + (g.t - g.lo + 1) : 0;
-  return g;
+  dec_group_keys(sa_keys, v.t, args.sink, args.window, &v.a, &v.lo);
+  v.nvis = (v.heads != 0 && dec_slot_ok(args, v.slot, v.t)) ? v.a + (v.t - v.lo + 1) : 0;
+  return v;
 }
 
-// One stage of an item, written by the producer before it arms the stage's
+// One stage of a segment, written by the producer before it arms the stage's
 // full barrier.  n < 0 ends the stream.
 struct DecDesc {
-  int n, js, t, a, lo, b, hk;
-  int seg, nseg;       // this CTA's segment of the group, and the group's segment count
+  int n;               // key rows in the stage
   int first, last;     // first / last stage of the segment
-  uint32_t sparse_bits;
-  int pad[4];
+  int b, hk, vg;       // batch row, kv head, virtual group (2 * (b * Hkv + hk) + part)
+  int seg, nseg;       // this CTA's segment of the virtual group, and its segment count
+  uint32_t heads;      // query heads of the virtual group (bit g: head hk * G + g)
+  int pad[7];
 };
 
 // Balanced contiguous split of `total` items over `grid` CTAs: CTA c owns
@@ -200,6 +214,7 @@ struct DecLayout {
   static constexpr int kDPL = (G == 8) ? 8 : 16;     // channels per lane
   static constexpr int kLPR = D / kDPL;              // lanes per key row
   static constexpr int kChunks = kDPL / 8;           // 16-byte chunks per lane
+  static constexpr int kP = kDPL / 2;                // channel pairs per lane
   static constexpr int kRGW = 32 / kLPR;             // row groups per warp
   static constexpr int kNG = kCW * kRGW;
   static constexpr int kRowBytes = D * 2;
@@ -220,7 +235,9 @@ struct DecLayout {
   static constexpr int off_mo = off_flag + 16;
   static constexpr int off_ml = off_mo + kCW * G * D * 4;
   static constexpr int off_table = off_ml + kCW * G * 2 * 4;
-  static constexpr int bytes(int ngroups) { return off_table + (ngroups + 1) * 4; }
+  // item table: one entry per virtual group (two per kv group) plus one
+  static constexpr int bytes(int ngroups) { return off_table + (2 * ngroups + 1) * 4; }
+  static_assert(bytes(kDecMaxGroups) <= 232448, "shared memory per CTA");
   static_assert(kStageRows % kNG == 0 && kRPS >= 1 && kRPS % kRB == 0, "stage rows");
   static_assert(kChunkRows % kStageRows == 0 && kChunkRows >= kDecChunk, "chunk rows");
   static_assert(sizeof(DecDesc) == 64, "descriptor size");
@@ -260,28 +277,151 @@ __device__ __forceinline__ void unpack2(uint64_t a, float& x, float& y) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a));
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+// One stage of a virtual group whose NA query heads sit in slots 0..NA-1 of
+// the state arrays.  Every row of the stage is a key all NA heads see; rows
+// at and past n (a partial last stage) hold stale bytes and are skipped.
+// Per batch of rows: the NA dot products of each row (kLPR lanes, reduced by
+// interleaved shuffles), one running-max update (rescale only when the max
+// grows by more than 2^8), then P.V.
+template <class L, int G, int NA>
+__device__ __forceinline__ void dec_stage(int n, const uint8_t* ks, const uint8_t* vs, int rg,
+                                          int cl, const uint64_t (&q2)[G][L::kP],
+                                          uint64_t (&o2)[G][L::kP], float (&m)[G],
+                                          float (&l)[G]) {
+  const bool full = n == L::kStageRows;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    f[2 * e] = __uint_as_float(w[e] << 16);
-    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  for (int kb = 0; kb < L::kRPS; kb += L::kRB) {
+    uint4 kr[L::kRB][L::kChunks], vr[L::kRB][L::kChunks];
+    bool valid[L::kRB];
+#pragma unroll
+    for (int kk = 0; kk < L::kRB; ++kk) {
+      const int r = rg + (kb + kk) * L::kNG;
+      valid[kk] = full || r < n;
+#pragma unroll
+      for (int i = 0; i < L::kChunks; ++i) {
+        const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
+        kr[kk][i] = *reinterpret_cast<const uint4*>(ks + off);
+        vr[kk][i] = *reinterpret_cast<const uint4*>(vs + off);
+      }
+    }
+    if (!full) {
+      // never multiply stale bytes
+#pragma unroll
+      for (int kk = 0; kk < L::kRB; ++kk)
+#pragma unroll
+        for (int i = 0; i < L::kChunks; ++i)
+          if (!valid[kk]) vr[kk][i] = make_uint4(0, 0, 0, 0);
+    }
+    float sc[L::kRB][NA];
+#pragma unroll
+    for (int kk = 0; kk < L::kRB; ++kk) {
+      uint64_t acc[NA];
+#pragma unroll
+      for (int h = 0; h < NA; ++h) acc[h] = 0ull;
+#pragma unroll
+      for (int i = 0; i < L::kChunks; ++i) {
+        const uint32_t w[4] = {kr[kk][i].x, kr[kk][i].y, kr[kk][i].z, kr[kk][i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint64_t k2 = bf16x2_to_f32x2(w[e]);
+#pragma unroll
+          for (int h = 0; h < NA; ++h) ffma2(acc[h], q2[h][i * 4 + e], k2);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < NA; ++h) {
+        float x, y;
+        unpack2(acc[h], x, y);
+        sc[kk][h] = x + y;
+      }
+    }
+#pragma unroll
+    for (int off = L::kLPR / 2; off > 0; off >>= 1)
+#pragma unroll
+      for (int kk = 0; kk < L::kRB; ++kk)
+#pragma unroll
+        for (int h = 0; h < NA; ++h) sc[kk][h] += __shfl_xor_sync(0xffffffffu, sc[kk][h], off);
+    if (!full) {
+#pragma unroll
+      for (int kk = 0; kk < L::kRB; ++kk)
+#pragma unroll
+        for (int h = 0; h < NA; ++h) sc[kk][h] = valid[kk] ? sc[kk][h] : -INFINITY;
+    }
+    // one branch per batch: rescale every head whose max grew by > 2^8
+    float mx[NA];
+    bool grow = false;
+#pragma unroll
+    for (int h = 0; h < NA; ++h) {
+      mx[h] = sc[0][h];
+#pragma unroll
+      for (int kk = 1; kk < L::kRB; ++kk) mx[h] = fmaxf(mx[h], sc[kk][h]);
+      grow = grow || mx[h] > m[h] + kDecRescale;
+    }
+    if (grow) {
+#pragma unroll
+      for (int h = 0; h < NA; ++h) {
+        const bool up = mx[h] > m[h] + kDecRescale;
+        const float alpha = up ? ex2_approx(m[h] - mx[h]) : 1.0f;
+        m[h] = up ? mx[h] : m[h];
+        l[h] *= alpha;
+        const uint64_t a2 = pack2(alpha, alpha);
+#pragma unroll
+        for (int e = 0; e < L::kP; ++e) o2[h][e] = fmul2(o2[h][e], a2);
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < L::kRB; ++kk) {
+      uint64_t p2[NA];
+#pragma unroll
+      for (int h = 0; h < NA; ++h) {
+        const float pr = ex2_approx(sc[kk][h] - m[h]);
+        l[h] += pr;
+        p2[h] = pack2(pr, pr);
+      }
+#pragma unroll
+      for (int i = 0; i < L::kChunks; ++i) {
+        const uint32_t w[4] = {vr[kk][i].x, vr[kk][i].y, vr[kk][i].z, vr[kk][i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint64_t v2 = bf16x2_to_f32x2(w[e]);
+#pragma unroll
+          for (int h = 0; h < NA; ++h) ffma2(o2[h][i * 4 + e], p2[h], v2);
+        }
+      }
+    }
   }
 }
 
-// Persistent split-K decode attention.  Work item = (kv group, 512-key
-// chunk) with at least one visible key, ordered by group then chunk; CTA c
-// owns one contiguous, balanced range of items, so a group's chunks fall in
-// one or a few consecutive CTAs (its segments).  The producer warp builds the
-// item table, then streams its items' visible cache rows (contiguous runs:
-// sinks, window, ring wrap) and, once per segment, the G query rows into a
-// ring of 64- to 192-row stages with bulk copies.  The consumer warps take a stage:
-// every key row is read by kLPR lanes, the G dot products of a batch of rows
-// reduced by interleaved shuffles, and an fp32 online softmax kept per row
-// group and head (one max update per batch) across the whole segment.  The
-// segment's last stage merges the row groups and writes one partial
-// (o, max, sum) per query head; the CTA that completes a group's last segment
-// merges its partials in segment order and writes the bf16 output.
+// Run the stage body compiled for exactly `nact` heads (1 <= nact <= NA).
+// One body per head count: padding a smaller head set up to a larger body
+// measured slower on mixed groups than the extra code costs.
+template <class L, int G, int NA>
+__device__ __forceinline__ void dec_stage_dispatch(int nact, int n, const uint8_t* ks,
+                                                   const uint8_t* vs, int rg, int cl,
+                                                   const uint64_t (&q2)[G][L::kP],
+                                                   uint64_t (&o2)[G][L::kP], float (&m)[G],
+                                                   float (&l)[G]) {
+  if (NA == 1 || nact == NA) {
+    dec_stage<L, G, NA>(n, ks, vs, rg, cl, q2, o2, m, l);
+    return;
+  }
+  if constexpr (NA > 1) dec_stage_dispatch<L, G, NA - 1>(nact, n, ks, vs, rg, cl, q2, o2, m, l);
+}
+
+
+// Persistent split-K decode attention.  Work item = (virtual group, chunk of
+// its key list) with at least one key, ordered by virtual group then chunk;
+// CTA c owns one contiguous, balanced range of items, so a virtual group's
+// chunks fall in one or a few consecutive CTAs (its segments).  The producer
+// warp builds the item table, then streams its items' cache rows (contiguous
+// runs: sinks, window, ring wrap) and, once per segment, the group's query
+// rows into a ring of stages with bulk copies.  The consumer warps take a
+// stage: every key row is read by kLPR lanes for all the virtual group's
+// heads (a body compiled per head count), and an fp32 online softmax is kept
+// per row group and head across the whole segment.  The segment's last stage
+// merges the row groups and writes one partial (o, max, sum) per query head;
+// the CTA that completes a virtual group's last segment merges its partials
+// in segment order and writes the bf16 output.
 template <int D, int G>
 __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kernel(DecodeArgs args) {
   using L = DecLayout<D, G>;
@@ -312,12 +452,13 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
     regs_dec<W::kRegsProducer>();
     if (warp != L::kCW) return;
     // ---------------- producer: item table (exclusive prefix of chunk counts)
+    const int nvg = 2 * ngroups;   // virtual groups: (b, hk, part)
     int carry = 0;
-    for (int base = 0; base < ngroups; base += 32) {
+    for (int base = 0; base < nvg; base += 32) {
       const int gi = base + lane;
       int cnt = 0;
-      if (gi < ngroups) {
-        const DecGroup g = dec_group(args, gi / args.Hkv, gi % args.Hkv, G);
+      if (gi < nvg) {
+        const DecVGroup g = dec_vgroup(args, (gi / 2) / args.Hkv, (gi / 2) % args.Hkv, gi % 2, G);
         cnt = (g.nvis + L::kChunkRows - 1) / L::kChunkRows;
       }
       int incl = cnt;
@@ -326,7 +467,7 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
         const int y = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += y;
       }
-      if (gi < ngroups) table[gi + 1] = carry + incl;
+      if (gi < nvg) table[gi + 1] = carry + incl;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) table[0] = 0;
@@ -334,7 +475,7 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
     if (lane != 0) return;
 
     // ---------------- producer: stream the stages
-    const int total = table[ngroups];
+    const int total = table[nvg];
     const int grid = gridDim.x, cta = blockIdx.x;
     const int i0 = dec_range_begin(cta, total, grid), i1 = dec_range_begin(cta + 1, total, grid);
     int u = 0;                 // stage uses issued
@@ -342,14 +483,14 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
     bool ok = true;
     for (int it = i0; it < i1 && ok; ++it) {
       while (table[gi + 1] <= it) ++gi;
-      const int b = gi / args.Hkv, hk = gi % args.Hkv;
+      const int b = (gi / 2) / args.Hkv, hk = (gi / 2) % args.Hkv;
       const int chunk = it - table[gi];
       const bool seg_first = it == i0 || chunk == 0;
       const bool seg_last = it == i1 - 1 || it == table[gi + 1] - 1;
       const int cta_first = dec_cta_of(table[gi], total, grid);
       const int seg = cta - cta_first;
       const int nseg = dec_cta_of(table[gi + 1] - 1, total, grid) - cta_first + 1;
-      const DecGroup g = dec_group(args, b, hk, G);
+      const DecVGroup g = dec_vgroup(args, b, hk, gi % 2, G);
       const __nv_bfloat16* kbase;
       const __nv_bfloat16* vbase;
       if (g.compact) {
@@ -371,11 +512,11 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
         }
         const int n = min(L::kStageRows, j1 - js);
         DecDesc& d = desc[slot];
-        d.n = n; d.js = js; d.t = g.t; d.a = g.a; d.lo = g.lo; d.b = b; d.hk = hk;
+        d.n = n; d.b = b; d.hk = hk; d.vg = gi;
         d.seg = seg; d.nseg = nseg;
         const bool first = seg_first && js == j0;
         d.first = first; d.last = seg_last && js + L::kStageRows >= j1;
-        d.sparse_bits = g.sparse_bits;
+        d.heads = g.heads;
         const uint32_t bar = full0 + 8 * slot;
         mbar_arrive_expect_tx(bar, 2u * n * L::kRowBytes + (first ? L::kQ : 0));
         const uint32_t kdst = sbase + L::off_k + slot * L::kKV;
@@ -428,10 +569,11 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
 
   // ---------------- consumers
   regs_inc<W::kRegsConsumer>();
-  constexpr uint32_t kAllBits = (1u << G) - 1u;
-  constexpr int kP = L::kDPL / 2;                    // channel pairs per lane
+  constexpr int kP = L::kP;
   const int sub = lane / L::kLPR, cl = lane % L::kLPR;
   const int rg = warp * L::kRGW + sub;
+  // state of the segment's heads, packed: slot k holds the k-th head of the
+  // virtual group (the k-th set bit of its head mask)
   uint64_t q2[G][kP], o2[G][kP];
   float m[G], l[G];
 #pragma unroll
@@ -441,6 +583,8 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
 #pragma unroll
     for (int e = 0; e < kP; ++e) { o2[g][e] = 0ull; q2[g][e] = 0ull; }
   }
+  int nact = G;
+  uint32_t heads = (1u << G) - 1u;
   const uint64_t scale2 = pack2(args.scale_log2, args.scale_log2);
   for (int u = 0;; ++u) {
     const int slot = u % L::kStages, round = u / L::kStages;
@@ -450,141 +594,38 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
     const DecDesc d = desc[slot];
     if (d.n < 0) break;
     if (d.first) {
+      heads = d.heads;
+      nact = __popc(heads);
       const uint8_t* qs = smem + L::off_q + slot * L::kQ;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int k = 0; k < G; ++k) {
 #pragma unroll
-        for (int i = 0; i < L::kChunks; ++i) {
-          const uint4 raw =
-              *reinterpret_cast<const uint4*>(qs + (g * D + (cl + i * L::kLPR) * 8) * 2);
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int e = 0; e < kP; ++e) q2[k][e] = 0ull;   // slots past nact are never read
+        if (k < nact) {
+          const int g = __fns(heads, 0, k + 1);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) q2[g][i * 4 + e] = fmul2(bf16x2_to_f32x2(w[e]), scale2);
+          for (int i = 0; i < L::kChunks; ++i) {
+            const uint4 raw =
+                *reinterpret_cast<const uint4*>(qs + (g * D + (cl + i * L::kLPR) * 8) * 2);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q2[k][i * 4 + e] = fmul2(bf16x2_to_f32x2(w[e]), scale2);
+          }
         }
-        m[g] = kDecNegBig;
-        l[g] = 0.f;
+        m[k] = kDecNegBig;
+        l[k] = 0.f;
 #pragma unroll
-        for (int e = 0; e < kP; ++e) o2[g][e] = 0ull;
+        for (int e = 0; e < kP; ++e) o2[k][e] = 0ull;
       }
     }
-    const bool full = d.n == L::kStageRows;
-    // only a group with both FA and SA heads tests key positions
-    const bool mixed = d.sparse_bits != 0 && d.sparse_bits != kAllBits;
-    const uint8_t* ks = smem + L::off_k + slot * L::kKV;
-    const uint8_t* vs = smem + L::off_v + slot * L::kKV;
-#pragma unroll
-    for (int kb = 0; kb < L::kRPS; kb += L::kRB) {
-      uint4 kr[L::kRB][L::kChunks], vr[L::kRB][L::kChunks];
-      bool valid[L::kRB];
-#pragma unroll
-      for (int kk = 0; kk < L::kRB; ++kk) {
-        const int r = rg + (kb + kk) * L::kNG;
-        valid[kk] = full || r < d.n;
-#pragma unroll
-        for (int i = 0; i < L::kChunks; ++i) {
-          const int off = r * L::kRowBytes + (cl + i * L::kLPR) * 16;
-          kr[kk][i] = *reinterpret_cast<const uint4*>(ks + off);
-          vr[kk][i] = *reinterpret_cast<const uint4*>(vs + off);
-        }
-      }
-      if (!full) {
-        // rows past the stage's end hold stale bytes: never multiply them
-#pragma unroll
-        for (int kk = 0; kk < L::kRB; ++kk)
-#pragma unroll
-          for (int i = 0; i < L::kChunks; ++i)
-            if (!valid[kk]) vr[kk][i] = make_uint4(0, 0, 0, 0);
-      }
-      float sc[L::kRB][G];
-#pragma unroll
-      for (int kk = 0; kk < L::kRB; ++kk) {
-        uint64_t acc[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = 0ull;
-#pragma unroll
-        for (int i = 0; i < L::kChunks; ++i) {
-          const uint32_t w[4] = {kr[kk][i].x, kr[kk][i].y, kr[kk][i].z, kr[kk][i].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint64_t k2 = bf16x2_to_f32x2(w[e]);
-#pragma unroll
-            for (int g = 0; g < G; ++g) ffma2(acc[g], q2[g][i * 4 + e], k2);
-          }
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float x, y;
-          unpack2(acc[g], x, y);
-          sc[kk][g] = x + y;
-        }
-      }
-#pragma unroll
-      for (int off = L::kLPR / 2; off > 0; off >>= 1)
-#pragma unroll
-        for (int kk = 0; kk < L::kRB; ++kk)
-#pragma unroll
-          for (int g = 0; g < G; ++g) sc[kk][g] += __shfl_xor_sync(0xffffffffu, sc[kk][g], off);
-      if (!full || mixed) {
-#pragma unroll
-        for (int kk = 0; kk < L::kRB; ++kk) {
-          const int j = d.js + rg + (kb + kk) * L::kNG;
-          const int p = j < d.a ? j : d.lo + (j - d.a);
-          const bool in_sa = p < args.sink || d.t - p < args.window;
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const bool seen = valid[kk] && (in_sa || !((d.sparse_bits >> g) & 1u));
-            sc[kk][g] = seen ? sc[kk][g] : -INFINITY;
-          }
-        }
-      }
-      // one branch per batch: rescale every head whose max grew by > 2^8
-      float mx[G];
-      bool grow = false;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        mx[g] = sc[0][g];
-#pragma unroll
-        for (int kk = 1; kk < L::kRB; ++kk) mx[g] = fmaxf(mx[g], sc[kk][g]);
-        grow = grow || mx[g] > m[g] + kDecRescale;
-      }
-      if (grow) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const bool up = mx[g] > m[g] + kDecRescale;
-          const float alpha = up ? ex2_approx(m[g] - mx[g]) : 1.0f;
-          m[g] = up ? mx[g] : m[g];
-          l[g] *= alpha;
-          const uint64_t a2 = pack2(alpha, alpha);
-#pragma unroll
-          for (int e = 0; e < kP; ++e) o2[g][e] = fmul2(o2[g][e], a2);
-        }
-      }
-#pragma unroll
-      for (int kk = 0; kk < L::kRB; ++kk) {
-        uint64_t p2[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = ex2_approx(sc[kk][g] - m[g]);
-          l[g] += pr;
-          p2[g] = pack2(pr, pr);
-        }
-#pragma unroll
-        for (int i = 0; i < L::kChunks; ++i) {
-          const uint32_t w[4] = {vr[kk][i].x, vr[kk][i].y, vr[kk][i].z, vr[kk][i].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint64_t v2 = bf16x2_to_f32x2(w[e]);
-#pragma unroll
-            for (int g = 0; g < G; ++g) ffma2(o2[g][i * 4 + e], p2[g], v2);
-          }
-        }
-      }
-    }
+    dec_stage_dispatch<L, G, G>(nact, d.n, smem + L::off_k + slot * L::kKV,
+                                smem + L::off_v + slot * L::kKV, rg, cl, q2, o2, m, l);
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
 
     if (d.last) {
-      // merge the row groups of this warp (lanes cl, cl + kLPR, ...)
+      // merge the row groups of this warp (lanes cl, cl + kLPR, ...); slots
+      // past nact hold zeros and merge to zeros
 #pragma unroll
       for (int off = L::kLPR; off < 32; off <<= 1) {
 #pragma unroll
@@ -628,33 +669,34 @@ __global__ void __launch_bounds__(DecWarps<G>::kThreads, 1) ea_decode_attn_kerne
       }
       named_bar_consumers<L::kCW>();
       const int hq0 = d.b * args.Hq + d.hk * G;
-      for (int idx = threadIdx.x; idx < G * (D + 2); idx += L::kCW * 32) {
-        const int g = idx / (D + 2), c = idx % (D + 2);
+      for (int idx = threadIdx.x; idx < nact * (D + 2); idx += L::kCW * 32) {
+        const int k = idx / (D + 2), c = idx % (D + 2);
+        const int g = __fns(heads, 0, k + 1);
         float mx = kDecNegBig;
 #pragma unroll
-        for (int w = 0; w < L::kCW; ++w) mx = fmaxf(mx, s_ml[(w * G + g) * 2]);
+        for (int w = 0; w < L::kCW; ++w) mx = fmaxf(mx, s_ml[(w * G + k) * 2]);
         float acc = 0.f;
 #pragma unroll
         for (int w = 0; w < L::kCW; ++w) {
-          const float sw = ex2_approx(s_ml[(w * G + g) * 2] - mx);
-          const float x = c < D ? s_mo[(w * G + g) * D + c] : s_ml[(w * G + g) * 2 + 1];
+          const float sw = ex2_approx(s_ml[(w * G + k) * 2] - mx);
+          const float x = c < D ? s_mo[(w * G + k) * D + c] : s_ml[(w * G + k) * 2 + 1];
           acc += x * sw;
         }
         float* pb = args.part + ((static_cast<size_t>(hq0 + g)) * args.nsplit + d.seg) * (D + 2);
         pb[c] = (c == D) ? mx : acc;
       }
-      // publish the partial; the CTA that completes the group merges it
+      // publish the partial; the CTA that completes the virtual group merges it
       __threadfence();
       named_bar_consumers<L::kCW>();
       if (threadIdx.x == 0) {
-        const int prev = atomicAdd(args.counters + d.b * args.Hkv + d.hk, 1);
+        const int prev = atomicAdd(args.counters + d.vg, 1);
         *last_flag = prev == d.nseg - 1;
         __threadfence();
       }
       named_bar_consumers<L::kCW>();
       if (*last_flag) {
-        for (int idx = threadIdx.x; idx < G * D; idx += L::kCW * 32) {
-          const int g = idx / D, c = idx % D;
+        for (int idx = threadIdx.x; idx < nact * D; idx += L::kCW * 32) {
+          const int g = __fns(heads, 0, idx / D + 1), c = idx % D;
           const float* pb = args.part + static_cast<size_t>(hq0 + g) * args.nsplit * (D + 2);
           float mx = kDecNegBig;
           for (int sp = 0; sp < d.nseg; ++sp)
@@ -732,7 +774,7 @@ bool dec_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u
 // Workspace: status word (256 B), per-group item counters (rounded up to
 // 256 B), then the partials.
 size_t dec_counter_bytes(const ea_decode_params* p) {
-  const size_t n = static_cast<size_t>(p->B) * p->Hkv * sizeof(int);
+  const size_t n = 2 * static_cast<size_t>(p->B) * p->Hkv * sizeof(int);
   return (n + 255) / 256 * 256;
 }
 

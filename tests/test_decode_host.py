@@ -47,14 +47,14 @@ def test_kv_policy_invalid(lib):
 def test_decode_workspace_size(lib):
     p = make_decode_params(2, 32, 8, 128, 64, 1024, 4096, 10, 6)
     n = lib.ea_decode_workspace_size(ctypes.byref(p))
-    # status block, per-group item counters (256-byte block), and one
-    # (o, max, sum) partial per (b, head, 512-key split)
+    # status block, two segment counters per kv group (256-byte blocks), and
+    # one (o, max, sum) partial per (b, head, 512-key split)
     assert n == 256 + 256 + 2 * 32 * (4096 // 512) * (128 + 2) * 4
     # the compact cache alone can need more splits than max_len
     p = make_decode_params(1, 4, 4, 64, 600, 600, 100, 0, 4)
     assert lib.ea_decode_workspace_size(ctypes.byref(p)) == 256 + 256 + 4 * 3 * 66 * 4
-    p = make_decode_params(20, 32, 8, 128, 4, 16, 64, 160, 0)       # 160 counters: 640 B
-    assert lib.ea_decode_workspace_size(ctypes.byref(p)) == 256 + 768 + 20 * 32 * 1 * 130 * 4
+    p = make_decode_params(20, 32, 8, 128, 4, 16, 64, 160, 0)       # 320 counters: 1280 B
+    assert lib.ea_decode_workspace_size(ctypes.byref(p)) == 256 + 1280 + 20 * 32 * 1 * 130 * 4
     # more than 4096 kv groups per step is not supported
     p = make_decode_params(513, 32, 8, 128, 4, 16, 64, 513 * 8, 0)
     assert lib.ea_decode_workspace_size(ctypes.byref(p)) == 0
