@@ -67,6 +67,9 @@ __all__ = [
     "kv_head_sparse",
     "compact_slot",
     "decode_step",
+    "router_pool_varlen",
+    "router_decide_varlen",
+    "attention_varlen",
 ]
 
 
@@ -338,4 +341,63 @@ def decode_step(q, k_hist, v_hist, pos, mask, sink: int, window: int,
             vv = np.asarray(v_hist[b, hk], dtype=np.float64)[keys]
             s = (kk @ q[b, h]) * scale
             out[b, h] = _softmax_row_weighted(s[None, :], vv)[0]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Packed variable-length batches.  A serving prefill batch is ragged: sequence
+# b holds tokens [cu[b], cu[b+1]) of packed tensors q [T, Hq, d] and k, v
+# [T, Hkv, d] (token-major, heads, channels).  The method routes per input
+# (EA blog §2.1), so each sequence is its own square causal prefill: its
+# router input is the mean of its own keys, and its attention sees only its
+# own tokens, positions counted from the sequence's first token.  Reading
+# taken for an empty sequence: its pooled keys are zero (no tokens), so its
+# routing comes from the biases alone, and it has no output rows.
+# --------------------------------------------------------------------------
+
+def router_pool_varlen(k_packed, cu_seqlens) -> np.ndarray:
+    """x [B, Hkv * d]: per sequence, the explicit sum of its key rows divided
+    by its length (zeros for an empty sequence)."""
+    k = np.asarray(k_packed, dtype=np.float64)
+    cu = [int(c) for c in cu_seqlens]
+    B = len(cu) - 1
+    T, Hkv, d = k.shape
+    x = np.zeros((B, Hkv * d), dtype=np.float64)
+    for b in range(B):
+        n = cu[b + 1] - cu[b]
+        if n <= 0:
+            continue
+        total = np.zeros((Hkv, d), dtype=np.float64)
+        for t in range(cu[b], cu[b + 1]):
+            total += k[t]
+        x[b] = (total / n).reshape(Hkv * d)
+    return x
+
+
+def router_decide_varlen(k_packed, cu_seqlens, w1, b1, w2, b2, threshold: float = 0.0):
+    """Route mask [B, Hq] and logits z [B, Hq] of a packed batch."""
+    z = router_mlp(router_pool_varlen(k_packed, cu_seqlens), w1, b1, w2, b2)
+    return (z > threshold).astype(np.uint8), z
+
+
+def attention_varlen(q, k, v, cu_seqlens, mask, sink: int, window: int,
+                     scale: float | None = None, block: int = 256) -> np.ndarray:
+    """out [T, Hq, d] in float64: every sequence's tokens attend within the
+    sequence, each head in its own mode (mask [B, Hq])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cu = [int(c) for c in cu_seqlens]
+    T, Hq, d = q.shape
+    out = np.zeros((T, Hq, d), dtype=np.float64)
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        if t1 <= t0:
+            continue
+        # [n, H, d] -> [1, H, n, d]: the sequence as a batch of one
+        qs = q[t0:t1].transpose(1, 0, 2)[None]
+        ks = k[t0:t1].transpose(1, 0, 2)[None]
+        vs = v[t0:t1].transpose(1, 0, 2)[None]
+        o = attention(qs, ks, vs, np.asarray(mask)[b:b + 1], sink, window, scale, block)
+        out[t0:t1] = o[0].transpose(1, 0, 2)
     return out

@@ -45,6 +45,13 @@ MUTATIONS = {
                       "np.any(m.reshape(m.shape[0], hkv, g) != 0, axis=2)"),
     "decode_gqa_modulo": ("            hk = h // g\n            keys = visible_keys",
                           "            hk = h % Hkv\n            keys = visible_keys"),
+    "varlen_pool_total_divisor": ("x[b] = (total / n).reshape(Hkv * d)",
+                                  "x[b] = (total / T).reshape(Hkv * d)"),
+    "varlen_pool_drops_last_token": ("for t in range(cu[b], cu[b + 1]):",
+                                     "for t in range(cu[b], cu[b + 1] - 1):"),
+    "varlen_first_mask_row": ("np.asarray(mask)[b:b + 1]", "np.asarray(mask)[0:1]"),
+    "varlen_heads_as_positions": ("qs = q[t0:t1].transpose(1, 0, 2)[None]",
+                                  "qs = q[t0:t1].reshape(Hq, t1 - t0, d)[None]"),
 }
 
 

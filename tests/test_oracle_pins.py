@@ -314,3 +314,77 @@ def test_kv_head_sparse_requires_all_query_heads():
     mask = np.array([[1, 1, 0, 1, 1, 1], [0, 0, 1, 1, 1, 0]], np.uint8)
     np.testing.assert_array_equal(oracle.kv_head_sparse(mask, 6, 3), [[1, 0, 1], [0, 1, 0]])
     np.testing.assert_array_equal(oracle.kv_head_sparse(mask, 6, 6), mask)
+
+
+# --------------------------------------------------------------------------
+# Packed variable-length batches: every sequence is its own prefill
+# --------------------------------------------------------------------------
+
+def _packed(cu, Hq, Hkv, d, seed):
+    T = cu[-1]
+    q = _bf16(_rand((T, Hq, d), seed))
+    k = _bf16(_rand((T, Hkv, d), seed + 1))
+    v = _bf16(_rand((T, Hkv, d), seed + 2))
+    return q, k, v
+
+
+def test_varlen_matches_brute_force_per_sequence():
+    cu = [0, 5, 5, 17, 40]                      # includes an empty sequence
+    Hq, Hkv, d, S, W = 4, 2, 8, 2, 5
+    q, k, v = _packed(cu, Hq, Hkv, d, 61)
+    mask = np.array([[0, 1, 1, 0], [1, 1, 1, 1], [1, 0, 1, 0], [0, 0, 1, 1]], np.uint8)
+    out = oracle.attention_varlen(q, k, v, cu, mask, S, W)
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        if t1 == t0:
+            continue
+        # brute force on the sequence laid out as its own batch of one
+        qs = q[t0:t1].transpose(1, 0, 2)[None]
+        ks = k[t0:t1].transpose(1, 0, 2)[None]
+        vs = v[t0:t1].transpose(1, 0, 2)[None]
+        ref = oracle.brute_force_attention(qs, ks, vs, mask[b:b + 1], S, W)
+        np.testing.assert_allclose(out[t0:t1], ref[0].transpose(1, 0, 2), rtol=0, atol=1e-12)
+
+
+def test_varlen_positions_restart_per_sequence():
+    """The first token of every sequence sees only itself: out = its own v."""
+    cu = [0, 7, 19, 20, 33]
+    Hq, Hkv, d = 4, 2, 8
+    q, k, v = _packed(cu, Hq, Hkv, d, 62)
+    mask = np.array([[0, 1, 0, 1]] * 4, np.uint8)
+    out = oracle.attention_varlen(q, k, v, cu, mask, 3, 4)
+    for b in range(4):
+        for h in range(Hq):
+            np.testing.assert_array_equal(out[cu[b], h], v[cu[b], h // 2])
+
+
+def test_varlen_sequences_are_independent():
+    cu = [0, 9, 30, 44]
+    Hq, Hkv, d = 2, 1, 8
+    q, k, v = _packed(cu, Hq, Hkv, d, 63)
+    mask = np.array([[0, 1], [1, 0], [0, 0]], np.uint8)
+    out = oracle.attention_varlen(q, k, v, cu, mask, 2, 6)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[9:30] += 1.0
+    k2[9:30] -= 0.5
+    v2[9:30] *= 3.0
+    out2 = oracle.attention_varlen(q2, k2, v2, cu, mask, 2, 6)
+    np.testing.assert_array_equal(out2[:9], out[:9])
+    np.testing.assert_array_equal(out2[30:], out[30:])
+    assert not np.allclose(out2[9:30], out[9:30])
+
+
+def test_varlen_router_pool_closed_forms():
+    cu = [0, 4, 4, 11]
+    Hkv, d = 2, 3
+    T = cu[-1]
+    # key rows k[t, kh, c] = t + 100 kh + 1000 c: the mean over [t0, t1) is
+    # (t0 + t1 - 1) / 2 + 100 kh + 1000 c
+    k = np.array([[[t + 100 * kh + 1000 * c for c in range(d)] for kh in range(Hkv)]
+                  for t in range(T)], np.float64)
+    x = oracle.router_pool_varlen(k, cu)
+    assert x.shape == (3, Hkv * d)
+    for b, (t0, t1) in enumerate(zip(cu[:-1], cu[1:])):
+        want = np.zeros(Hkv * d) if t1 == t0 else np.array(
+            [(t0 + t1 - 1) / 2 + 100 * kh + 1000 * c for kh in range(Hkv) for c in range(d)])
+        np.testing.assert_allclose(x[b], want, rtol=0, atol=1e-9)
