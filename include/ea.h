@@ -167,7 +167,8 @@ size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p);
  * workspace : device, >= ea_hybrid_attn_workspace_size(p) bytes, ZEROED
  *             once before its first use; the kernel only ever writes a
  *             nonzero error code into it (cleared by ea_get_device_status).
- * Limits: d in {64, 128}; Hq % Hkv == 0; B*Hq <= 4096; N < 2^30.
+ * Limits: d in {64, 128}; Hq % Hkv == 0; B <= 1024; B*Hq <= 4096;
+ * N <= 32767 * 256.
  */
 ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
                                  const uint8_t* route_mask,
@@ -180,6 +181,47 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
  * the error a kernel recorded (EA_ERR_TIMEOUT when a bounded device wait ran
  * out).  Returns EA_ERR_CUDA if the synchronisation or the copy fails. */
 ea_status ea_get_device_status(void* workspace, void* stream, int* status_out);
+
+/* ------------------------------------------------------------------------
+ * Packed variable-length batch (the same attention; not on the pages, which
+ * route per input, EA blog §2.1: every sequence is its own square causal
+ * prefill).  Sequence b holds tokens [cu_seqlens[b], cu_seqlens[b+1]) of the
+ * packed tensors; positions restart at 0 in every sequence, and a sequence
+ * sees only its own tokens.
+ *
+ * q, out   : device bf16 [T][Hq][d] (token-major, then head, then channel).
+ * k, v     : device bf16 [T][Hkv][d].  All 16-byte aligned.
+ * cu_seqlens: device int32 [B+1], cu[0] = 0, non-decreasing, cu[B] = T.  An
+ *             inconsistent array runs nothing and records EA_ERR_INVALID_ARG
+ *             in the status word.  Empty sequences are allowed.
+ * route_mask: device uint8 [B][Hq], as for ea_hybrid_attn_prefill.
+ * p->max_seqlen bounds every length (it sizes the grid only).
+ * Workspace as for ea_hybrid_attn_prefill (ea_hybrid_attn_varlen_workspace_size).
+ * Limits: d in {64, 128}; Hq % Hkv == 0; B <= 1024; B*Hq <= 4096;
+ * max_seqlen <= 32767 * 256; T < 2^31.
+ * ---------------------------------------------------------------------- */
+typedef struct ea_varlen_params {
+  int B, Hq, Hkv;
+  int total;             /* T = cu_seqlens[B]                               */
+  int max_seqlen;        /* >= every cu_seqlens[b+1] - cu_seqlens[b]        */
+  int d;
+  int sink, window;
+  float softmax_scale;   /* <= 0 selects 1/sqrt(d)                          */
+  int select;            /* ea_select                                       */
+} ea_varlen_params;
+
+size_t ea_hybrid_attn_varlen_workspace_size(const ea_varlen_params* p);
+
+ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void* v,
+                                        const int32_t* cu_seqlens, const uint8_t* route_mask,
+                                        const ea_varlen_params* p, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* Host view of the packed batch's schedule, like ea_schedule_units below:
+ * cu_seqlens_host is a HOST int32 [B+1] copy; units_out rows are
+ * {sparse, b, h, pair, n_kv_tiles}.  Returns the unit count or -1. */
+int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
+                             const int32_t* cu_seqlens_host, int32_t* units_out, int max_units);
 
 /* ------------------------------------------------------------------------
  * Decode step with a per-head KV-cache policy.

@@ -34,7 +34,8 @@ EXPORTED = [
     "ea_hybrid_attn_workspace_size", "ea_hybrid_attn_prefill",
     "ea_get_device_status", "ea_schedule_units", "ea_schedule_unit_tiles",
     "ea_attn_grid_size", "ea_decode_workspace_size", "ea_hybrid_attn_decode",
-    "ea_decode_kv_policy",
+    "ea_decode_kv_policy", "ea_hybrid_attn_varlen_workspace_size",
+    "ea_hybrid_attn_prefill_varlen", "ea_schedule_units_varlen",
 ]
 
 
@@ -43,6 +44,13 @@ class EaAttnParams(ctypes.Structure):
                 ("N", ctypes.c_int), ("d", ctypes.c_int), ("sink", ctypes.c_int),
                 ("window", ctypes.c_int), ("softmax_scale", ctypes.c_float),
                 ("select", ctypes.c_int)]
+
+
+class EaVarlenParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("total", ctypes.c_int), ("max_seqlen", ctypes.c_int), ("d", ctypes.c_int),
+                ("sink", ctypes.c_int), ("window", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float), ("select", ctypes.c_int)]
 
 
 class EaDecodeParams(ctypes.Structure):
@@ -101,6 +109,13 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_schedule_unit_tiles.argtypes = [vp, pparams, c_int, vp, vp, c_int]
     lib.ea_attn_grid_size.restype = c_int
     lib.ea_attn_grid_size.argtypes = [pparams, c_int]
+    pvar = ctypes.POINTER(EaVarlenParams)
+    lib.ea_hybrid_attn_varlen_workspace_size.restype = c_size
+    lib.ea_hybrid_attn_varlen_workspace_size.argtypes = [pvar]
+    lib.ea_hybrid_attn_prefill_varlen.restype = c_int
+    lib.ea_hybrid_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, pvar, vp, vp, c_size, vp]
+    lib.ea_schedule_units_varlen.restype = c_int
+    lib.ea_schedule_units_varlen.argtypes = [vp, pvar, vp, vp, c_int]
     pdec = ctypes.POINTER(EaDecodeParams)
     lib.ea_decode_workspace_size.restype = c_size
     lib.ea_decode_workspace_size.argtypes = [pdec]

@@ -13,7 +13,7 @@ import torch
 
 from . import _lib
 from ._lib import (EA_SELECT_ALL, EA_SELECT_FA, EA_SELECT_SA, EaAttnParams,  # noqa: F401
-                   EaDecodeParams, check)
+                   EaDecodeParams, EaVarlenParams, check)
 
 
 def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> int:
@@ -150,6 +150,55 @@ def ea_hybrid_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out
 
 
+# ---------------------------------------------------------------- packed batches
+def make_varlen_params(B, Hq, Hkv, total, max_seqlen, d, sink, window, softmax_scale=0.0,
+                       select=EA_SELECT_ALL) -> EaVarlenParams:
+    return EaVarlenParams(int(B), int(Hq), int(Hkv), int(total), int(max_seqlen), int(d),
+                          int(sink), int(window), float(softmax_scale), int(select))
+
+
+def ea_hybrid_attn_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  cu_seqlens: torch.Tensor, route_mask: torch.Tensor,
+                                  max_seqlen: int, sink: int, window: int, *,
+                                  softmax_scale: float = 0.0, select: int = EA_SELECT_ALL,
+                                  out: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Packed batch: q [T, Hq, d], k, v [T, Hkv, d], cu_seqlens int32 [B + 1]
+    (device); returns out bf16 [T, Hq, d]."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    _need(route_mask, "route_mask", torch.uint8)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if k.shape != (T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [T, Hkv, d] matching q")
+    if route_mask.numel() != B * Hq:
+        raise ValueError("route_mask must hold B * Hq entries")
+    p = make_varlen_params(B, Hq, Hkv, T, max_seqlen, d, sink, window, softmax_scale, select)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if workspace is None:
+        n = int(lib.ea_hybrid_attn_varlen_workspace_size(ctypes.byref(p)))
+        if n == 0:
+            raise ValueError("invalid packed-batch parameters")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    rc = lib.ea_hybrid_attn_prefill_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           cu_seqlens.data_ptr(), route_mask.data_ptr(),
+                                           ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill_varlen")
+    return out
+
+
 def ea_get_device_status(workspace: torch.Tensor,
                          stream: Optional[torch.cuda.Stream] = None) -> int:
     lib = _lib.load()
@@ -175,6 +224,20 @@ def ea_schedule_units(mask, p: EaAttnParams) -> np.ndarray:
         raise ValueError("invalid schedule arguments")
     out = np.zeros((max(n, 1), 5), dtype=np.int32)
     lib.ea_schedule_units(m.ctypes.data, ctypes.byref(p), out.ctypes.data, n)
+    return out[:n]
+
+
+def ea_schedule_units_varlen(mask, p: EaVarlenParams, cu_seqlens) -> np.ndarray:
+    """Schedule of a packed batch (cu_seqlens on the host): [U, 5] int32 rows."""
+    lib = _lib.load()
+    m = _host_mask(mask)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    n = lib.ea_schedule_units_varlen(m.ctypes.data, ctypes.byref(p), cu.ctypes.data, None, 0)
+    if n < 0:
+        raise ValueError("invalid schedule arguments")
+    out = np.zeros((max(n, 1), 5), dtype=np.int32)
+    lib.ea_schedule_units_varlen(m.ctypes.data, ctypes.byref(p), cu.ctypes.data,
+                                 out.ctypes.data, n)
     return out[:n]
 
 

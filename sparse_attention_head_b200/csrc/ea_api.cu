@@ -6,7 +6,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "ea.h"
 #include "ea_internal.h"
@@ -51,6 +53,9 @@ using ea::wait_timeout_ns;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Unit counts per sequence are 16-bit in the kernel's tables.
+constexpr int kMaxSeqLen = 32767 * EA_UNIT_ROWS;
+
 // Validates the attention params; EA_OK if the kernels can run them.
 ea_status check_params(const ea_attn_params* p) {
   if (!p) return EA_ERR_INVALID_ARG;
@@ -61,7 +66,24 @@ ea_status check_params(const ea_attn_params* p) {
   if (p->Hq % p->Hkv != 0) return EA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return EA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->B) * p->Hq > EA_MAX_ENTRIES) return EA_ERR_UNSUPPORTED;
-  if (p->N >= (1 << 30)) return EA_ERR_UNSUPPORTED;
+  if (p->B > EA_MAX_SEQS) return EA_ERR_UNSUPPORTED;
+  if (p->N > kMaxSeqLen) return EA_ERR_UNSUPPORTED;
+  if (!(p->softmax_scale <= 0.f) && !(p->softmax_scale > 0.f)) return EA_ERR_INVALID_ARG;  // NaN
+  return EA_OK;
+}
+
+// Validates packed-batch params the same way.
+ea_status check_varlen(const ea_varlen_params* p) {
+  if (!p) return EA_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->total < 0 || p->max_seqlen < 0 || p->d <= 0)
+    return EA_ERR_INVALID_ARG;
+  if (p->sink < 0 || p->window < 1) return EA_ERR_INVALID_ARG;
+  if (p->select < EA_SELECT_ALL || p->select > EA_SELECT_SA) return EA_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return EA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return EA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->Hq > EA_MAX_ENTRIES) return EA_ERR_UNSUPPORTED;
+  if (p->B > EA_MAX_SEQS) return EA_ERR_UNSUPPORTED;
+  if (p->max_seqlen > kMaxSeqLen) return EA_ERR_UNSUPPORTED;
   if (!(p->softmax_scale <= 0.f) && !(p->softmax_scale > 0.f)) return EA_ERR_INVALID_ARG;  // NaN
   return EA_OK;
 }
@@ -99,6 +121,96 @@ bool encode_bhsd(CUtensorMap* m, const void* ptr, int d, int n, int rows3) {
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Packed [T][heads][d] memory as a (d, T, heads) tensor: tokens step by
+// heads * d elements, heads by d; the same 64 x 128 x 1 box.
+bool encode_packed(CUtensorMap* m, const void* ptr, int d, int total, int heads) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(total),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(heads) * static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Host copy of the kernel's sequence tables (EaSeqView): the schedule views
+// build exactly what the kernel's prologue builds.
+struct HostSched {
+  std::vector<int16_t> P;
+  std::vector<int32_t> prefFA, prefSA;
+  std::vector<int> ent, len;
+  int nfa = 0, nsa = 0;
+  EaSeqView view;
+};
+
+void build_host_sched(const uint8_t* mask, int B, int Hq, int select, const int* lens, int S,
+                      int W, HostSched& h) {
+  std::vector<int> order(B), pb(B);
+  for (int b = 0; b < B; ++b) {
+    order[b] = b;
+    pb[b] = ea_cdiv(lens[b], EA_UNIT_ROWS);
+  }
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return pb[x] > pb[y]; });
+  h.len.assign(lens, lens + B);
+  h.P.resize(B);
+  h.prefFA.assign(B + 1, 0);
+  h.prefSA.assign(B + 1, 0);
+  h.ent.clear();
+  for (int k = 0; k < B; ++k) {
+    h.P[k] = static_cast<int16_t>(pb[order[k]]);
+    h.prefFA[k] = static_cast<int32_t>(h.ent.size());
+    for (int hh = 0; hh < Hq; ++hh) {
+      const int idx = order[k] * Hq + hh;
+      if (!mask[idx] && select != EA_SELECT_SA) h.ent.push_back(idx);
+    }
+  }
+  h.nfa = static_cast<int>(h.ent.size());
+  h.prefFA[B] = h.nfa;
+  for (int k = 0; k < B; ++k) {
+    h.prefSA[k] = static_cast<int32_t>(h.ent.size()) - h.nfa;
+    for (int hh = 0; hh < Hq; ++hh) {
+      const int idx = order[k] * Hq + hh;
+      if (mask[idx] && select != EA_SELECT_FA) h.ent.push_back(idx);
+    }
+  }
+  h.nsa = static_cast<int>(h.ent.size()) - h.nfa;
+  h.prefSA[B] = h.nsa;
+  h.view.nseq = B;
+  h.view.P = h.P.data();
+  h.view.prefFA = h.prefFA.data();
+  h.view.prefSA = h.prefSA.data();
+  h.view.Pmax = B > 0 ? h.P[0] : 0;
+  h.view.pA = ea_split_pair(S, W, h.view.Pmax);
+}
+
+// Units of a schedule in rank order: {sparse, b, h, pair, n_kv_tiles}.
+int list_units(const HostSched& h, int Hq, int S, int W, int32_t* units_out, int max_units) {
+  const int total = ea_total_units(h.view);
+  if (units_out) {
+    EaCursor cur;
+    ea_cursor_init(cur, h.view);
+    for (int r = 0; r < total && r < max_units; ++r) {
+      int sparse, e, pair;
+      ea_cursor_seek(cur, h.view, r, &sparse, &e, &pair);
+      const int idx = h.ent[sparse ? h.nfa + e : e];
+      const EaShape sh = ea_make_shape(h.len[idx / Hq], S, W);
+      const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
+      int32_t* u = units_out + 5 * r;
+      u[0] = sparse;
+      u[1] = idx / Hq;
+      u[2] = idx % Hq;
+      u[3] = pair;
+      u[4] = ut.n;
+    }
+  }
+  return total;
 }
 
 // EA_DEBUG_DROP_KV_POS=<n> makes the attention producer skip K/V ring
@@ -196,6 +308,8 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   args.mask = route_mask;
   args.out = out;
   args.status = static_cast<int*>(workspace);
+  args.cu_seqlens = nullptr;
+  args.total = 0;
   args.B = p->B;
   args.Hq = p->Hq;
   args.Hkv = p->Hkv;
@@ -227,56 +341,91 @@ ea_status ea_get_device_status(void* workspace, void* stream, int* status_out) {
   return EA_OK;
 }
 
-// ------------------------------------------------------------------ schedule view
-static int count_entries(const uint8_t* mask, const ea_attn_params* p, int* nfa, int* nsa,
-                         int* ent) {
-  const int BH = p->B * p->Hq;
-  int f = 0, s = 0;
-  for (int i = 0; i < BH; ++i)
-    if (!mask[i] && p->select != EA_SELECT_SA) ent[f++] = i;
-  for (int i = 0; i < BH; ++i)
-    if (mask[i] && p->select != EA_SELECT_FA) ent[f + s++] = i;
-  *nfa = f;
-  *nsa = s;
-  return f + s;
+size_t ea_hybrid_attn_varlen_workspace_size(const ea_varlen_params* p) {
+  return check_varlen(p) == EA_OK ? kAttnWorkspace : 0;
 }
 
+ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void* v,
+                                        const int32_t* cu_seqlens, const uint8_t* route_mask,
+                                        const ea_varlen_params* p, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  ea_status st = check_varlen(p);
+  if (st != EA_OK) return st;
+  if (!q || !k || !v || !cu_seqlens || !route_mask || !out) return EA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  if (p->total == 0 || p->max_seqlen == 0) return EA_OK;   // no token: nothing to run
+
+  ea::AttnArgs args;
+  if (!encode_packed(&args.tm_q, q, p->d, p->total, p->Hq) ||
+      !encode_packed(&args.tm_k, k, p->d, p->total, p->Hkv) ||
+      !encode_packed(&args.tm_v, v, p->d, p->total, p->Hkv))
+    return EA_ERR_CUDA;
+  args.mask = route_mask;
+  args.out = out;
+  args.status = static_cast<int*>(workspace);
+  args.cu_seqlens = cu_seqlens;
+  args.total = p->total;
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->max_seqlen;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = debug_drop_kv_pos();
+
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  const long long units = static_cast<long long>(p->B) * p->Hq *
+                          ((p->max_seqlen + EA_UNIT_ROWS - 1) / EA_UNIT_ROWS);
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ schedule view
 int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p, int32_t* units_out,
                       int max_units) {
   if (!mask || check_params(p) != EA_OK) return -1;
-  static thread_local int ent[EA_MAX_ENTRIES];
-  int nfa, nsa;
-  count_entries(mask, p, &nfa, &nsa, ent);
-  const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
-  const int total = ea_num_units(sh, nfa, nsa);
-  if (units_out) {
-    for (int r = 0; r < total && r < max_units; ++r) {
-      int sparse, e, pair;
-      ea_unit_of_rank(sh, nfa, nsa, r, &sparse, &e, &pair);
-      const int idx = ent[sparse ? nfa + e : e];
-      const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
-      int32_t* u = units_out + 5 * r;
-      u[0] = sparse;
-      u[1] = idx / p->Hq;
-      u[2] = idx % p->Hq;
-      u[3] = pair;
-      u[4] = ut.n;
-    }
+  std::vector<int> lens(p->B, p->N);
+  HostSched h;
+  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  return list_units(h, p->Hq, p->sink, p->window, units_out, max_units);
+}
+
+int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
+                             const int32_t* cu_seqlens_host, int32_t* units_out, int max_units) {
+  if (!mask || !cu_seqlens_host || check_varlen(p) != EA_OK) return -1;
+  if (cu_seqlens_host[0] != 0 || cu_seqlens_host[p->B] != p->total) return -1;
+  std::vector<int> lens(p->B);
+  for (int b = 0; b < p->B; ++b) {
+    lens[b] = cu_seqlens_host[b + 1] - cu_seqlens_host[b];
+    if (lens[b] < 0) return -1;
   }
-  return total;
+  HostSched h;
+  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  return list_units(h, p->Hq, p->sink, p->window, units_out, max_units);
 }
 
 int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int rank,
                            int32_t* tiles_out, int32_t* codes_out, int max_tiles) {
   if (!mask || check_params(p) != EA_OK) return -1;
-  static thread_local int ent[EA_MAX_ENTRIES];
-  int nfa, nsa;
-  count_entries(mask, p, &nfa, &nsa, ent);
-  const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
-  const int total = ea_num_units(sh, nfa, nsa);
+  std::vector<int> lens(p->B, p->N);
+  HostSched h;
+  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  const int total = ea_total_units(h.view);
   if (rank < 0 || rank >= total) return -1;
+  EaCursor cur;
+  ea_cursor_init(cur, h.view);
   int sparse, e, pair;
-  ea_unit_of_rank(sh, nfa, nsa, rank, &sparse, &e, &pair);
+  ea_cursor_seek(cur, h.view, rank, &sparse, &e, &pair);
+  const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
   const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
   for (int i = 0; i < ut.n && i < max_tiles; ++i) {
     const int t = ea_tile_at(ut, i);

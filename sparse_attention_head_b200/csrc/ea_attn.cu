@@ -64,7 +64,16 @@ struct AttnCfg {
   static constexpr int kNumBars = 3 + 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, counts
   static constexpr int kOffEnt = kOffMisc + 64;
-  static constexpr int kSmem = kOffEnt + EA_MAX_ENTRIES * 2 + 1024;  // + alignment slack
+  // sequence tables: token offset and length by index, order and unit count by
+  // sorted position, FA / SA entry prefix counts by sorted position
+  static constexpr int kOffTok = kOffEnt + EA_MAX_ENTRIES * 2;
+  static constexpr int kOffLen = kOffTok + EA_MAX_SEQS * 4;
+  static constexpr int kOffPrefFA = kOffLen + EA_MAX_SEQS * 4;
+  static constexpr int kOffPrefSA = kOffPrefFA + (EA_MAX_SEQS + 1) * 4;
+  static constexpr int kOffOrder = kOffPrefSA + (EA_MAX_SEQS + 1) * 4;
+  static constexpr int kOffP = kOffOrder + EA_MAX_SEQS * 2;
+  static constexpr int kSmem = kOffP + EA_MAX_SEQS * 2 + 1024;  // + alignment slack
+  static_assert(kSmem <= 232448, "shared memory per CTA");
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
 };
@@ -145,26 +154,87 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
-  // Entry lists: FA heads first, then SA heads, each in (b, h) order, filtered
-  // by args.select.  Warp 0 builds them with ballots.
+  // Sequence tables.  Lengths and token offsets by sequence index: a padded
+  // batch has every length N; a packed batch reads cu_seqlens, and an
+  // inconsistent one (cu[0] != 0, decreasing, or cu[B] != T) runs no unit
+  // and records EA_ERR_INVALID_ARG.
+  int32_t* s_tok = reinterpret_cast<int32_t*>(smem + C::kOffTok);
+  int32_t* s_len = reinterpret_cast<int32_t*>(smem + C::kOffLen);
+  int32_t* s_prefFA = reinterpret_cast<int32_t*>(smem + C::kOffPrefFA);
+  int32_t* s_prefSA = reinterpret_cast<int32_t*>(smem + C::kOffPrefSA);
+  int16_t* s_order = reinterpret_cast<int16_t*>(smem + C::kOffOrder);
+  int16_t* s_P = reinterpret_cast<int16_t*>(smem + C::kOffP);
+  const bool packed = args.cu_seqlens != nullptr;
+  if (packed) {
+    bool good = true;
+    for (int b = threadIdx.x; b < args.B; b += blockDim.x) {
+      const int t0 = args.cu_seqlens[b], t1 = args.cu_seqlens[b + 1];
+      good = good && t1 >= t0 && t0 >= 0 && t1 <= args.total;
+      s_tok[b] = t0;
+      s_len[b] = t1 - t0;
+    }
+    if (threadIdx.x == 0)
+      good = good && args.cu_seqlens[0] == 0 && args.cu_seqlens[args.B] == args.total;
+    if (!__syncthreads_and(good)) {
+      for (int b = threadIdx.x; b < args.B; b += blockDim.x) s_len[b] = 0;
+      if (threadIdx.x == 0 && blockIdx.x == 0) atomicCAS(args.status, 0, EA_ERR_INVALID_ARG);
+    }
+  } else {
+    for (int b = threadIdx.x; b < args.B; b += blockDim.x) {
+      s_tok[b] = 0;
+      s_len[b] = args.N;
+    }
+  }
+  __syncthreads();
+  // Sorted order: by unit count, longest first, ties by index (a padded batch
+  // keeps the identity order).
+  for (int b = threadIdx.x; b < args.B; b += blockDim.x) {
+    const int pb = ea_cdiv(s_len[b], EA_UNIT_ROWS);
+    int rank = b;
+    if (packed) {
+      rank = 0;
+      for (int o = 0; o < args.B; ++o) {
+        const int po = ea_cdiv(s_len[o], EA_UNIT_ROWS);
+        rank += (po > pb) || (po == pb && o < b);
+      }
+    }
+    s_order[rank] = static_cast<int16_t>(b);
+    s_P[rank] = static_cast<int16_t>(pb);
+  }
+  __syncthreads();
+  // Entry lists: FA heads first, then SA heads, filtered by args.select, each
+  // grouped by sorted sequence with heads in order.  Warp 0 builds them with
+  // ballots, and the prefix counts per sorted position with them.
   if (warp == 0) {
     int nfa = 0;
-    for (int base = 0; base < BH; base += 32) {
-      int idx = base + lane;
-      bool ok = idx < BH && args.mask[idx] == 0 && args.select != EA_SELECT_SA;
-      unsigned bits = __ballot_sync(0xffffffffu, ok);
-      if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
-      nfa += __popc(bits);
+    for (int k = 0; k < args.B; ++k) {
+      const int b = s_order[k];
+      if (lane == 0) s_prefFA[k] = nfa;
+      for (int h0 = 0; h0 < args.Hq; h0 += 32) {
+        const int h = h0 + lane;
+        const int idx = b * args.Hq + h;
+        const bool ok = h < args.Hq && args.mask[idx] == 0 && args.select != EA_SELECT_SA;
+        const unsigned bits = __ballot_sync(0xffffffffu, ok);
+        if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
+        nfa += __popc(bits);
+      }
     }
     int nsa = 0;
-    for (int base = 0; base < BH; base += 32) {
-      int idx = base + lane;
-      bool ok = idx < BH && args.mask[idx] != 0 && args.select != EA_SELECT_FA;
-      unsigned bits = __ballot_sync(0xffffffffu, ok);
-      if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
-      nsa += __popc(bits);
+    for (int k = 0; k < args.B; ++k) {
+      const int b = s_order[k];
+      if (lane == 0) s_prefSA[k] = nsa;
+      for (int h0 = 0; h0 < args.Hq; h0 += 32) {
+        const int h = h0 + lane;
+        const int idx = b * args.Hq + h;
+        const bool ok = h < args.Hq && args.mask[idx] != 0 && args.select != EA_SELECT_FA;
+        const unsigned bits = __ballot_sync(0xffffffffu, ok);
+        if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
+        nsa += __popc(bits);
+      }
     }
     if (lane == 0) {
+      s_prefFA[args.B] = nfa;
+      s_prefSA[args.B] = nsa;
       s_counts[0] = nfa;
       s_counts[1] = nsa;
     }
@@ -175,9 +245,14 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
 
   const uint32_t tmem = *s_tmem;
   const int nFA = s_counts[0];
-  const int nSA = s_counts[1];
-  const EaShape shape = ea_make_shape(args.N, args.sink, args.window);
-  const int total = ea_num_units(shape, nFA, nSA);
+  EaSeqView view;
+  view.nseq = args.B;
+  view.P = s_P;
+  view.prefFA = s_prefFA;
+  view.prefSA = s_prefSA;
+  view.Pmax = args.B > 0 ? s_P[0] : 0;
+  view.pA = ea_split_pair(args.sink, args.window, view.Pmax);
+  const int total = ea_total_units(view);
   const int G = args.Hq / args.Hkv;
   const uint64_t tlim = args.timeout_ns;
   int* status = args.status;
@@ -192,14 +267,21 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       uint32_t kv_pos = 0;
       uint32_t n_units = 0;
       bool ok = true;
+      EaCursor cur;
+      ea_cursor_init(cur, view);
       for (int kk = 0; ok; ++kk) {
         const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
         if (r < 0) break;
         int sparse, e, pair;
-        ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+        ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
         const int idx = s_ent[sparse ? nFA + e : e];
         const int b = idx / args.Hq, h = idx % args.Hq;
-        const int kvrow = b * args.Hkv + h / G;
+        // tensor coordinates: padded batch (row, head index b*H + h); packed
+        // batch (token, head)
+        const int tok = s_tok[b];
+        const int qz = packed ? h : idx;
+        const int kvz = packed ? h / G : b * args.Hkv + h / G;
+        const EaShape shape = ea_make_shape(s_len[b], args.sink, args.window);
         const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
         if (n_units > 0) {
           ok = mbar_wait(bars.q_empty, (n_units - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
@@ -209,7 +291,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         for (int s = 0; s < ut.nslots; ++s)
           for (int c = 0; c < C::kDBlocks; ++c)
             tma_load_3d(smem_u32(sQ) + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
-                        c * 64, ut.r0 + s * EA_BM, idx);
+                        c * 64, tok + ut.r0 + s * EA_BM, qz);
         ++n_units;
         for (int i = 0; i < ut.n && ok; ++i) {
           const int t = ea_tile_at(ut, i);
@@ -228,7 +310,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
             const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
             for (int c = 0; c < C::kDBlocks; ++c)
               tma_load_3d(smem_u32(sKV) + st * C::kTileBytes + c * C::kBlockBytes, map, bars.kv_full + 8 * st,
-                          c * 64, t * EA_BN, kvrow);
+                          c * 64, tok + t * EA_BN, kvz);
             ++kv_pos;
           }
         }
@@ -278,11 +360,15 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8, b0 + ((k * 2048) >> 4),
                  C::kIdescPV, (acc || k > 0) ? 1u : 0u);
       };
+      EaCursor cur;
+      ea_cursor_init(cur, view);
       for (int kk = 0; ok; ++kk) {
         const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
         if (r < 0) break;
         int sparse, e, pair;
-        ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+        ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
+        const int idx = s_ent[sparse ? nFA + e : e];
+        const EaShape shape = ea_make_shape(s_len[idx / args.Hq], args.sink, args.window);
         const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
 
         ok = mbar_wait(bars.q_full, n_units & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
@@ -373,14 +459,19 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     uint32_t s_cnt = 0;
     uint32_t pv_cnt = 0;
     bool ok = true;
+    EaCursor cur;
+    ea_cursor_init(cur, view);
     for (int kk = 0; ok; ++kk) {
       const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
       if (r < 0) break;
       int sparse, e, pair;
-      ea_unit_of_rank(shape, nFA, nSA, r, &sparse, &e, &pair);
+      ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
+      const int idx = s_ent[sparse ? nFA + e : e];
+      const int seq = idx / args.Hq;
+      const int seq_len = s_len[seq];
+      const EaShape shape = ea_make_shape(seq_len, args.sink, args.window);
       const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
       if (slot >= ut.nslots) continue;
-      const int idx = s_ent[sparse ? nFA + e : e];
       const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
       float m_ref = -INFINITY;
       float l = 0.f;
@@ -491,13 +582,16 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) +
-                            (static_cast<size_t>(idx) * args.N + row) * D;
+      // out row: padded [B][Hq][N][d]; packed [T][Hq][d]
+      const size_t orow_index =
+          packed ? (static_cast<size_t>(s_tok[seq] + row) * args.Hq + idx % args.Hq)
+                 : (static_cast<size_t>(idx) * args.N + row);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) + orow_index * D;
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
         uint32_t o[64];
         tmem_ld64_wait(tO + h * 64, o);
-        if (row < args.N) {
+        if (row < seq_len) {
           uint4* dst = reinterpret_cast<uint4*>(orow + h * 64);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {

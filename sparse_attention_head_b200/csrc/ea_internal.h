@@ -8,15 +8,20 @@
 namespace ea {
 
 // Arguments of the fused hybrid attention kernel.  The tensor maps describe
-// q [B*Hq][N][d], k and v [B*Hkv][N][d] (bf16, inner dim d) with a
-// 64 x 128 x 1 box and 128-byte swizzle.
+// q [B*Hq][N][d], k and v [B*Hkv][N][d] (bf16, inner dim d), or for a packed
+// batch q as (d, T, Hq) and k, v as (d, T, Hkv) over [T][heads][d] memory,
+// all with a 64 x 128 x 1 box and 128-byte swizzle.
 struct alignas(64) AttnArgs {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   const uint8_t* mask;      // [B*Hq], nonzero = sparse
-  void* out;                // bf16 [B][Hq][N][d]
+  void* out;                // bf16 [B][Hq][N][d], or [T][Hq][d] for a packed batch
   int* status;              // device status word
+  // Packed batch (nullptr: padded BHSD of length N): sequence b holds tokens
+  // [cu_seqlens[b], cu_seqlens[b + 1]) of q [T][Hq][d], k, v [T][Hkv][d].
+  const int32_t* cu_seqlens;
+  int total;                // T, tokens of a packed batch
   int B, Hq, Hkv, N;
   int sink, window;
   float scale_log2;         // softmax scale * log2(e)

@@ -15,7 +15,8 @@
 //   order = longest first: FA units longer than any SA unit (largest pair
 //           first), then every SA unit, then the remaining FA units; inside
 //           one pair index the heads of one kv group are adjacent, so their
-//           K/V tiles are reused from L2.
+//           K/V tiles are reused from L2.  Sequences of a batch may differ in
+//           length (EaSeqView).
 //   deal  = rank r goes to CTA c in a snake: round k = r / G covers ranks
 //           [kG, kG+G) left to right when k is even, right to left when odd.
 #pragma once
@@ -60,24 +61,91 @@ EA_HD EaShape ea_make_shape(int N, int S, int W) {
   return s;
 }
 
-// Unit rank -> (sparse, entry index within its list, pair).
-EA_HD void ea_unit_of_rank(const EaShape& s, int nFA, int nSA, int r,
-                           int* sparse, int* e, int* pair) {
-  int nA = nFA * (s.P - s.pA);
-  if (r < nA) {
-    *sparse = 0; *pair = s.P - 1 - r / nFA; *e = r % nFA; return;
-  }
-  r -= nA;
-  int nB = nSA * s.P;
-  if (r < nB) {
-    *sparse = 1; *pair = s.P - 1 - r / nSA; *e = r % nSA; return;
-  }
-  r -= nB;
-  *sparse = 0; *pair = s.pA - 1 - r / nFA; *e = r % nFA;
+// Batches of sequences of different lengths (packed varlen batches; a
+// padded batch is the case where every length is the same).  Sequences are
+// viewed sorted by unit count, longest first (ties by index), and every entry
+// list (FA entries, then SA entries) is grouped by sorted sequence, heads in
+// order inside a sequence.  The units at pair p are then the entries of the
+// sequences that have more than p units: a prefix of each list.
+#define EA_MAX_SEQS 1024
+
+struct EaSeqView {
+  int nseq;                // sequences
+  const int16_t* P;        // [nseq] unit count of the k-th sorted sequence, non-increasing
+  const int32_t* prefFA;   // [nseq + 1] FA entries of sorted positions < k
+  const int32_t* prefSA;   // [nseq + 1] SA entries of sorted positions < k
+  int Pmax;                // P[0] (0 for an empty batch)
+  int pA;                  // FA units with pair >= pA are longer than any SA unit
+};
+
+// pA for a batch: an interior SA unit visits at most sa_cap tiles; FA unit
+// of pair p visits min(2p + 2, its tile count), longer than sa_cap when
+// p >= floor(sa_cap / 2).
+EA_HD int ea_split_pair(int S, int W, int Pmax) {
+  const int sa_cap = ea_cdiv(S, EA_BN) + 2 + ea_cdiv(W - 1, EA_BN);
+  return ea_min(sa_cap / 2, Pmax);
 }
 
-EA_HD int ea_num_units(const EaShape& s, int nFA, int nSA) {
-  return (nFA + nSA) * s.P;
+// Order (longest first): FA units with pair >= pA (pair descending), then
+// every SA unit (pair descending), then the FA units with pair < pA (pair
+// descending); inside one (phase, pair), entries in list order.  A cursor
+// walks it; ranks must be asked in increasing order.
+struct EaCursor {
+  int phase;   // 0: long FA, 1: SA, 2: short FA, 3: past the end
+  int p;       // pair
+  int base;    // rank of the first unit at (phase, p)
+  int cnt;     // units at (phase, p)
+  int m;       // sorted sequences with more than p units
+};
+
+EA_HD int ea_phase_top(const EaSeqView& v, int phase) {
+  return phase == 2 ? v.pA - 1 : v.Pmax - 1;
+}
+EA_HD int ea_phase_bottom(const EaSeqView& v, int phase) { return phase == 0 ? v.pA : 0; }
+
+EA_HD void ea_cursor_settle(EaCursor& c, const EaSeqView& v) {
+  while (c.phase < 3 && c.p < ea_phase_bottom(v, c.phase)) {
+    ++c.phase;
+    c.p = ea_phase_top(v, c.phase);
+    c.m = 0;
+  }
+  if (c.phase >= 3) {
+    c.cnt = 0;
+    return;
+  }
+  while (c.m < v.nseq && v.P[c.m] > c.p) ++c.m;
+  c.cnt = (c.phase == 1 ? v.prefSA : v.prefFA)[c.m];
+}
+
+EA_HD void ea_cursor_init(EaCursor& c, const EaSeqView& v) {
+  c.phase = 0;
+  c.p = ea_phase_top(v, 0);
+  c.base = 0;
+  c.m = 0;
+  ea_cursor_settle(c, v);
+}
+
+// Unit of rank r: (sparse, entry index within its list, pair); false past
+// the end.
+EA_HD bool ea_cursor_seek(EaCursor& c, const EaSeqView& v, int r, int* sparse, int* e,
+                          int* pair) {
+  while (c.phase < 3 && r >= c.base + c.cnt) {
+    c.base += c.cnt;
+    --c.p;
+    ea_cursor_settle(c, v);
+  }
+  if (c.phase >= 3) return false;
+  *sparse = c.phase == 1;
+  *e = r - c.base;
+  *pair = c.p;
+  return true;
+}
+
+EA_HD int ea_total_units(const EaSeqView& v) {
+  int total = 0;
+  for (int k = 0; k < v.nseq; ++k)
+    total += v.P[k] * ((v.prefFA[k + 1] - v.prefFA[k]) + (v.prefSA[k + 1] - v.prefSA[k]));
+  return total;
 }
 
 // k-th rank dealt to CTA c of G (or -1 past the end).

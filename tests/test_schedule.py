@@ -163,3 +163,98 @@ def test_decode_bytes():
     assert got["kv"] == 2 * row * (10 + 101 + 10 + 10)
     assert got["io"] == 2 * 2 * 4 * row + 4 * 2 * 2 * row
     assert got["n_sa_groups"] == 3 and got["n_groups"] == 4
+
+
+# ---------------------------------------------------------------- packed batches
+from sparse_attention_head_b200.api import ea_schedule_units_varlen, make_varlen_params  # noqa: E402
+
+VARLEN_CASES = [
+    # cu_seqlens, Hq, Hkv, d, S, W, select
+    ([0, 300, 300, 1000, 1077, 1600], 4, 2, 64, 16, 128, 0),
+    ([0, 1, 2, 515, 4611], 4, 1, 128, 64, 1024, 0),
+    ([0, 256, 512, 768], 2, 2, 64, 0, 1, 0),
+    ([0, 700, 900, 2000], 4, 2, 128, 130, 200, 1),
+    ([0, 700, 900, 2000], 4, 2, 128, 130, 200, 2),
+    ([0, 0, 0, 129], 2, 1, 64, 5, 3, 0),
+]
+
+
+def _units_cover(units, cu, mask, sel):
+    B, Hq = mask.shape
+    lens = np.diff(cu)
+    covered = [np.zeros((Hq, n), np.int32) for n in lens]
+    for sparse, b, h, pair, ntiles in units:
+        assert sparse == mask[b, h]
+        assert sel == 0 or (sel == 1 and not sparse) or (sel == 2 and sparse)
+        r0 = 256 * pair
+        assert r0 < lens[b]
+        covered[b][h, r0:min(lens[b], r0 + 256)] += 1
+    for b in range(B):
+        for h in range(Hq):
+            selected = sel == 0 or (sel == 1) == (mask[b, h] == 0)
+            assert np.all(covered[b][h] == (1 if selected else 0)), (b, h)
+
+
+@pytest.mark.parametrize("cu,Hq,Hkv,d,S,W,sel", VARLEN_CASES)
+def test_varlen_units_cover_rows_once(cu, Hq, Hkv, d, S, W, sel):
+    B = len(cu) - 1
+    rng = np.random.default_rng(cu[-1] + S)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    p = make_varlen_params(B, Hq, Hkv, cu[-1], max(np.diff(cu)), d, S, W, select=sel)
+    units = ea_schedule_units_varlen(mask, p, cu)
+    _units_cover(units, cu, mask, sel)
+    # each unit's tile count is that of its own sequence's shape
+    for sparse, b, h, pair, n in units:
+        N_b = cu[b + 1] - cu[b]
+        tiles = [t for t in range((N_b + 127) // 128)
+                 if any(brute_codes(N_b, bool(sparse), S, W, 256 * pair + 128 * s, t)
+                        for s in range(2) if 256 * pair + 128 * s < N_b)]
+        assert n == len(tiles), (b, pair, n, tiles)
+
+
+def test_varlen_equal_lengths_schedule_like_the_padded_batch():
+    B, Hq, Hkv, N, d, S, W = 3, 4, 2, 1000, 128, 64, 256
+    rng = np.random.default_rng(5)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    padded = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, d, S, W))
+    packed = ea_schedule_units_varlen(mask, make_varlen_params(B, Hq, Hkv, B * N, N, d, S, W),
+                                      [0, N, 2 * N, 3 * N])
+    np.testing.assert_array_equal(padded, packed)
+
+
+def test_varlen_order_longest_first_and_balance():
+    cu = np.cumsum([0, 32768, 1000, 9000, 300, 20000, 0, 4096]).tolist()
+    B, Hq, Hkv, d, S, W = len(cu) - 1, 32, 8, 128, 64, 1024
+    rng = np.random.default_rng(11)
+    mask = (rng.random((B, Hq)) < 0.7).astype(np.uint8)
+    p = make_varlen_params(B, Hq, Hkv, cu[-1], max(np.diff(cu)), d, S, W)
+    units = ea_schedule_units_varlen(mask, p, cu)
+    _units_cover(units, cu, mask, 0)
+    cost = units[:, 4]
+    sa_cap = int(np.ceil(S / 128)) + 2 + int(np.ceil((W - 1) / 128))
+    pA = sa_cap // 2
+    # long FA units first by pair, descending; then every SA unit; then short FA
+    nlong = int(np.sum((units[:, 0] == 0) & (units[:, 3] >= pA)))
+    assert np.all(units[:nlong, 0] == 0) and np.all(np.diff(units[:nlong, 3]) <= 0)
+    nsa = int(np.sum(units[:, 0] == 1))
+    assert np.all(units[nlong:nlong + nsa, 0] == 1)
+    assert np.all(units[nlong + nsa:, 0] == 0) and np.all(units[nlong + nsa:, 3] < pA)
+    # snake deal over 148 CTAs: loads within one longest unit
+    G = 148
+    load = np.zeros(G, np.int64)
+    for r in range(len(units)):
+        k = r // G
+        c = (r % G) if k % 2 == 0 else G - 1 - (r % G)
+        load[c] += cost[r]
+    assert load.max() - load.min() <= cost.max()
+
+
+def test_varlen_schedule_rejects_inconsistent_offsets():
+    mask = np.zeros((2, 2), np.uint8)
+    p = make_varlen_params(2, 2, 1, 10, 10, 64, 1, 4)
+    with pytest.raises(ValueError):
+        ea_schedule_units_varlen(mask, p, [1, 5, 10])
+    with pytest.raises(ValueError):
+        ea_schedule_units_varlen(mask, p, [0, 6, 4])
+    with pytest.raises(ValueError):
+        ea_schedule_units_varlen(mask, p, [0, 5, 9])
