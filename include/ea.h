@@ -95,6 +95,26 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d,
                            float* logits_out, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Router of a packed variable-length batch: the same pooling, MLP and
+ * threshold, where sequence b's router input is the mean of ITS OWN key rows
+ * (the method routes per input, EA blog §2.1).
+ * k          : device bf16 [total][Hkv][d], 16-byte aligned.
+ * cu_seqlens : device int32 [B+1] (as for ea_hybrid_attn_prefill_varlen).
+ *              An empty sequence pools to zero (its routing comes from the
+ *              biases alone); a sequence whose range is not inside [0, total]
+ *              pools nothing (zero) and is never read.
+ * max_seqlen : host bound of every length (sizes the workspace and split).
+ * workspace  : >= ea_router_varlen_workspace_size(B, Hkv, max_seqlen, d).
+ * Other arguments, limits and determinism as for ea_router_decide. */
+size_t ea_router_varlen_workspace_size(int B, int Hkv, int max_seqlen, int d);
+
+ea_status ea_router_decide_varlen(const void* k, const int32_t* cu_seqlens, int B, int Hkv,
+                                  int total, int max_seqlen, int d, const float* w1,
+                                  const float* b1, int hidden, const float* w2,
+                                  const float* b2, int Hq, float threshold,
+                                  uint8_t* route_mask, float* logits_out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * ea_router_decide without a caller-supplied workspace.
  *

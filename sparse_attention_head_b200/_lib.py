@@ -36,6 +36,7 @@ EXPORTED = [
     "ea_attn_grid_size", "ea_decode_workspace_size", "ea_hybrid_attn_decode",
     "ea_decode_kv_policy", "ea_hybrid_attn_varlen_workspace_size",
     "ea_hybrid_attn_prefill_varlen", "ea_schedule_units_varlen",
+    "ea_router_varlen_workspace_size", "ea_router_decide_varlen",
 ]
 
 
@@ -109,6 +110,12 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_schedule_unit_tiles.argtypes = [vp, pparams, c_int, vp, vp, c_int]
     lib.ea_attn_grid_size.restype = c_int
     lib.ea_attn_grid_size.argtypes = [pparams, c_int]
+    lib.ea_router_varlen_workspace_size.restype = c_size
+    lib.ea_router_varlen_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+    lib.ea_router_decide_varlen.restype = c_int
+    lib.ea_router_decide_varlen.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp,
+                                            c_int, vp, vp, c_int, ctypes.c_float, vp, vp, vp,
+                                            c_size, vp]
     pvar = ctypes.POINTER(EaVarlenParams)
     lib.ea_hybrid_attn_varlen_workspace_size.restype = c_size
     lib.ea_hybrid_attn_varlen_workspace_size.argtypes = [pvar]

@@ -80,6 +80,47 @@ def ea_router_decide(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: to
     return route_mask, logits
 
 
+def ea_router_decide_varlen(k: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int,
+                            w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+                            b2: torch.Tensor, threshold: float = 0.0, *,
+                            workspace: Optional[torch.Tensor] = None,
+                            route_mask: Optional[torch.Tensor] = None,
+                            logits: Optional[torch.Tensor] = None, want_logits: bool = True,
+                            stream: Optional[torch.cuda.Stream] = None
+                            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Router of a packed batch: k [T, Hkv, d], cu_seqlens int32 [B + 1] on the
+    device; route mask uint8 [B, Hq] and logits fp32 [B, Hq]."""
+    lib = _lib.load()
+    _need(k, "k", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+        _need(t, name, torch.float32, nd)
+    T, Hkv, d = k.shape
+    B = cu_seqlens.numel() - 1
+    hidden = w1.shape[0]
+    Hq = w2.shape[0]
+    if w1.shape[1] != Hkv * d or b1.shape[0] != hidden or w2.shape[1] != hidden \
+            or b2.shape[0] != Hq:
+        raise ValueError("router weight shapes do not match the key states")
+    dev = k.device
+    need = lib.ea_router_varlen_workspace_size(B, Hkv, int(max_seqlen), d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if route_mask is None:
+        route_mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+    if logits is None and want_logits:
+        logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    rc = lib.ea_router_decide_varlen(k.data_ptr(), cu_seqlens.data_ptr(), B, Hkv, T,
+                                     int(max_seqlen), d, w1.data_ptr(), b1.data_ptr(), hidden,
+                                     w2.data_ptr(), b2.data_ptr(), Hq, float(threshold),
+                                     route_mask.data_ptr(),
+                                     logits.data_ptr() if logits is not None else None,
+                                     workspace.data_ptr(), workspace.numel(),
+                                     _stream_ptr(stream, dev))
+    check(rc, "ea_router_decide_varlen")
+    return route_mask, logits
+
+
 def ea_router_decide_noalloc(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
                              w2: torch.Tensor, b2: torch.Tensor, threshold: float = 0.0, *,
                              route_mask: torch.Tensor, logits: Optional[torch.Tensor] = None,

@@ -271,8 +271,39 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const fl
   if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
   const int ns = ea::router_num_splits(B, Hkv, N);
-  cudaError_t err = ea::launch_router(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold,
-                                      route_mask, logits_out, static_cast<float*>(workspace), ns,
+  cudaError_t err = ea::launch_router(k, nullptr, B, Hkv, N, 0, d, w1, b1, hidden, w2, b2, Hq,
+                                      threshold, route_mask, logits_out,
+                                      static_cast<float*>(workspace), ns,
+                                      static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+size_t ea_router_varlen_workspace_size(int B, int Hkv, int max_seqlen, int d) {
+  if (B <= 0 || Hkv <= 0 || max_seqlen < 0 || (d != 64 && d != 128)) return 0;
+  return ea::router_workspace_bytes(B, Hkv, max_seqlen > 0 ? max_seqlen : 1, d,
+                                    kRouterMaxHidden);
+}
+
+ea_status ea_router_decide_varlen(const void* k, const int32_t* cu_seqlens, int B, int Hkv,
+                                  int total, int max_seqlen, int d, const float* w1,
+                                  const float* b1, int hidden, const float* w2, const float* b2,
+                                  int Hq, float threshold, uint8_t* route_mask, float* logits_out,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k || !cu_seqlens || !w1 || !b1 || !w2 || !b2 || !route_mask) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || total < 0 || max_seqlen < 0 || d <= 0 || hidden <= 0 || Hq <= 0)
+    return EA_ERR_INVALID_ARG;
+  if (threshold != threshold) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  const size_t need = ea_router_varlen_workspace_size(B, Hkv, max_seqlen, d);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  const int ns = ea::router_num_splits(B, Hkv, max_seqlen > 0 ? max_seqlen : 1);
+  cudaError_t err = ea::launch_router(k, cu_seqlens, B, Hkv, 0, total, d, w1, b1, hidden, w2, b2,
+                                      Hq, threshold, route_mask, logits_out,
+                                      static_cast<float*>(workspace), ns,
                                       static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }

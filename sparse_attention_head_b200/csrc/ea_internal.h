@@ -46,9 +46,11 @@ cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stre
 // Router: pooled partial sums, then the MLP and the threshold.
 int router_num_splits(int B, int Hkv, int N);
 size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden);
-cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const float* w1,
-                          const float* b1, int hidden, const float* w2, const float* b2,
-                          int Hq, float threshold, uint8_t* mask, float* logits,
+// cu == nullptr: padded K [B][Hkv][N][d]; else packed K [total][Hkv][d] with
+// sequence b at tokens [cu[b], cu[b + 1]).
+cudaError_t launch_router(const void* k, const int32_t* cu, int B, int Hkv, int N, int total,
+                          int d, const float* w1, const float* b1, int hidden, const float* w2,
+                          const float* b2, int Hq, float threshold, uint8_t* mask, float* logits,
                           float* partials, int nsplit, cudaStream_t stream);
 
 }  // namespace ea

@@ -12,7 +12,8 @@
 // Kernel 1 (HBM-bound): CTA (split, kv head, batch) sums its chunk of rows
 //   into fp32, 8 channels per thread with 16-byte loads, and reduces the
 //   row groups in a fixed order into partials[b][hk][split][d].
-// Kernel 2 sums the partials in split order and divides by N (x); kernels 3
+// Kernel 2 sums the partials in split order and divides by the sequence's
+//   row count (x; a packed batch pools each sequence's own tokens); kernels 3
 //   and 4 run h = ReLU(W1 x + b1) and z = W2 h + b2 with one warp per output
 //   spread over many CTAs (fixed shuffle order), and write z and the mask
 //   z > threshold.  All kernels are deterministic: same inputs, same bits.
@@ -30,10 +31,24 @@ namespace ea {
 constexpr int kPoolThreads = 256;
 constexpr int kMlpThreads = 256;
 
+// Rows of (b, kv head): padded K [B][Hkv][N][d] (cu == nullptr) or packed K
+// [T][Hkv][d] with sequence b at tokens [cu[b], cu[b + 1]).  A packed range
+// outside [0, T] (inconsistent offsets) pools nothing.
+__device__ __forceinline__ int router_seq_rows(const int32_t* cu, int N, int total, int b,
+                                               int* t0) {
+  if (!cu) {
+    *t0 = 0;
+    return N;
+  }
+  const int a = cu[b], e = cu[b + 1];
+  *t0 = a;
+  return (a >= 0 && e >= a && e <= total) ? e - a : 0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
-    const __nv_bfloat16* __restrict__ k, int N, int nsplit, int chunk,
-    float* __restrict__ partials) {
+    const __nv_bfloat16* __restrict__ k, const int32_t* __restrict__ cu, int N, int total,
+    int nsplit, float* __restrict__ partials) {
   constexpr int TPR = D / 8;                 // threads per row (8 channels each)
   constexpr int RPI = kPoolThreads / TPR;    // rows per iteration
   __shared__ float red[RPI][D];
@@ -41,16 +56,23 @@ __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
   const int Hkv = gridDim.y;
   const int cg = threadIdx.x % TPR;
   const int rs = threadIdx.x / TPR;
+  int t0;
+  const int len = router_seq_rows(cu, N, total, b, &t0);
+  const int chunk = (len + nsplit - 1) / nsplit;
   const int n0 = split * chunk;
-  const int n1 = min(N, n0 + chunk);
-  const __nv_bfloat16* base = k + (static_cast<size_t>(b) * Hkv + hk) * N * D + cg * 8;
+  const int n1 = min(len, n0 + chunk);
+  // padded: plane (b, hk) of N rows of D; packed: token rows of Hkv * D
+  const size_t row_stride = cu ? static_cast<size_t>(Hkv) * D : static_cast<size_t>(D);
+  const __nv_bfloat16* base =
+      (cu ? k + (static_cast<size_t>(t0) * Hkv + hk) * D
+          : k + (static_cast<size_t>(b) * Hkv + hk) * N * D) + cg * 8;
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
   int n = n0 + rs;
 #pragma unroll 4
   for (; n < n1; n += RPI) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(n) * D));
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(n) * row_stride));
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -69,17 +91,21 @@ __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
   }
 }
 
-// x[b][hk*d + c] = (sum over splits, in split order) / N; one thread per channel.
-__global__ void ea_router_reduce_kernel(const float* __restrict__ partials, int Hkv, int N, int d,
-                                        int nsplit, float* __restrict__ x) {
+// x[b][hk*d + c] = (sum over splits, in split order) / rows of sequence b
+// (zero for an empty sequence); one thread per channel.
+__global__ void ea_router_reduce_kernel(const float* __restrict__ partials,
+                                        const int32_t* __restrict__ cu, int Hkv, int N, int total,
+                                        int d, int nsplit, float* __restrict__ x) {
   const int b = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;   // j = hk * d + c
   if (j >= Hkv * d) return;
   const int hk = j / d, c = j % d;
+  int t0;
+  const int len = router_seq_rows(cu, N, total, b, &t0);
   const float* p = partials + (static_cast<size_t>(b) * Hkv + hk) * nsplit * d + c;
   float s = 0.f;
   for (int sp = 0; sp < nsplit; ++sp) s += p[static_cast<size_t>(sp) * d];
-  x[static_cast<size_t>(b) * Hkv * d + j] = s * (1.0f / static_cast<float>(N));
+  x[static_cast<size_t>(b) * Hkv * d + j] = len > 0 ? s * (1.0f / static_cast<float>(len)) : 0.f;
 }
 
 // One warp per output: y[b][o] = act(W[o] . x[b] + bias[o]), float4 over the
@@ -137,25 +163,24 @@ size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden) {
   return (parts + x + h) * sizeof(float);
 }
 
-cudaError_t launch_router(const void* k, int B, int Hkv, int N, int d, const float* w1,
-                          const float* b1, int hidden, const float* w2, const float* b2,
-                          int Hq, float threshold, uint8_t* mask, float* logits,
+cudaError_t launch_router(const void* k, const int32_t* cu, int B, int Hkv, int N, int total,
+                          int d, const float* w1, const float* b1, int hidden, const float* w2,
+                          const float* b2, int Hq, float threshold, uint8_t* mask, float* logits,
                           float* partials, int nsplit, cudaStream_t stream) {
-  const int chunk = (N + nsplit - 1) / nsplit;
   const int in_dim = Hkv * d;
   float* xbuf = partials + static_cast<size_t>(B) * Hkv * nsplit * d;
   float* hbuf = xbuf + static_cast<size_t>(B) * in_dim;
   dim3 grid(nsplit, Hkv, B);
   if (d == 128)
     ea_router_pool_kernel<128><<<grid, kPoolThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(k), N, nsplit, chunk, partials);
+        static_cast<const __nv_bfloat16*>(k), cu, N, total, nsplit, partials);
   else
     ea_router_pool_kernel<64><<<grid, kPoolThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(k), N, nsplit, chunk, partials);
+        static_cast<const __nv_bfloat16*>(k), cu, N, total, nsplit, partials);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  ea_router_reduce_kernel<<<dim3((in_dim + 255) / 256, B), 256, 0, stream>>>(partials, Hkv, N,
-                                                                             d, nsplit, xbuf);
+  ea_router_reduce_kernel<<<dim3((in_dim + 255) / 256, B), 256, 0, stream>>>(
+      partials, cu, Hkv, N, total, d, nsplit, xbuf);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   constexpr int kWarps = kMlpThreads / 32;

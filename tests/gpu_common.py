@@ -50,13 +50,18 @@ def sample_rows(N, S, W, n_random, seed):
     return sorted(rows)
 
 
-def margin_controlled_b2(k_f64, w1, b1, w2, b2, threshold=0.0, margin=MARGIN, shift=1e-2):
+def margin_controlled_b2(k_f64, w1, b1, w2, b2, threshold=0.0, margin=MARGIN, shift=1e-2,
+                         cu=None):
     """Return b2 shifted (per head, away from the threshold on its current side)
     until every oracle logit clears the margin; the routing is unchanged in
-    sign.  Uses only the oracle."""
+    sign.  Uses only the oracle.  With cu, k_f64 is a packed [T, Hkv, d]
+    batch with sequence offsets cu."""
     b2 = np.array(b2, dtype=np.float64)
     for _ in range(8):
-        _, z = oracle.router_decide(k_f64, w1, b1, w2, b2, threshold)
+        if cu is None:
+            _, z = oracle.router_decide(k_f64, w1, b1, w2, b2, threshold)
+        else:
+            _, z = oracle.router_decide_varlen(k_f64, cu, w1, b1, w2, b2, threshold)
         close = np.abs(z - threshold) < margin
         if not close.any():
             return b2

@@ -140,3 +140,60 @@ def test_varlen_large_ragged_batch_sampled_rows():
             ref = oracle.attention_rows(qs, ks, vs, mask[b:b + 1], 0, h, rows, S, W)
             err = np.abs(got[[t0 + r for r in rows], h] - ref)
             assert err.max() <= 1e-2, (b, h, float(err.max()))
+
+
+# ---------------------------------------------------------------- router
+from gpu_common import LOGIT_ABS, margin_controlled_b2  # noqa: E402
+from sparse_attention_head_b200.api import ea_router_decide, ea_router_decide_varlen  # noqa: E402
+
+
+def _router_weights(in_dim, hidden, Hq, seed):
+    g = torch.Generator().manual_seed(seed)
+    w1 = (torch.randn((hidden, in_dim), generator=g) * 0.05).float()
+    b1 = (torch.randn((hidden,), generator=g) * 0.1).float()
+    w2 = (torch.randn((Hq, hidden), generator=g) * 0.05).float()
+    b2 = (torch.randn((Hq,), generator=g) * 0.05).float()
+    return w1, b1, w2, b2
+
+
+@pytest.mark.parametrize("cu,Hkv,d", [([0, 300, 300, 1000, 1077, 5000], 8, 128),
+                                      ([0, 1, 4097, 4100], 4, 64)])
+def test_varlen_router_matches_oracle(cu, Hkv, d):
+    B, Hq, hidden = len(cu) - 1, 32, 256
+    T = cu[-1]
+    g = torch.Generator().manual_seed(T)
+    # per-sequence channel offsets make the pooled vectors (and so the
+    # routing) depend on each sequence's own keys
+    offs = torch.randn((B, Hkv, d), generator=g)
+    k = torch.randn((T, Hkv, d), generator=g)
+    for b in range(B):
+        k[cu[b]:cu[b + 1]] += offs[b]
+    k = k.to(torch.bfloat16)
+    w1, b1, w2, b2 = _router_weights(Hkv * d, hidden, Hq, seed=T + 1)
+    b2 = torch.as_tensor(margin_controlled_b2(f64(k), w1.double().numpy(), b1.double().numpy(),
+                                              w2.double().numpy(), b2.double().numpy(), cu=cu),
+                         dtype=torch.float32)
+    mask, z = ea_router_decide_varlen(k.to(DEV), torch.as_tensor(cu, dtype=torch.int32,
+                                                                  device=DEV),
+                                      int(max(np.diff(cu))), w1.to(DEV), b1.to(DEV), w2.to(DEV),
+                                      b2.to(DEV))
+    torch.cuda.synchronize()
+    ref_mask, ref_z = oracle.router_decide_varlen(f64(k), cu, w1.double().numpy(),
+                                                  b1.double().numpy(), w2.double().numpy(),
+                                                  b2.double().numpy())
+    np.testing.assert_array_equal(mask.cpu().numpy(), ref_mask)
+    assert np.abs(z.cpu().double().numpy() - ref_z).max() <= LOGIT_ABS
+    assert len(set(map(tuple, ref_mask.tolist()))) > 1      # sequences route differently
+
+
+def test_varlen_router_equal_lengths_match_the_padded_router_bitwise():
+    B, Hkv, N, d, Hq, hidden = 3, 8, 2000, 128, 32, 256
+    g = torch.Generator().manual_seed(12)
+    k4 = torch.randn((B, Hkv, N, d), generator=g).to(torch.bfloat16)
+    w1, b1, w2, b2 = (t.to(DEV) for t in _router_weights(Hkv * d, hidden, Hq, seed=13))
+    m_pad, z_pad = ea_router_decide(k4.to(DEV), w1, b1, w2, b2)
+    packed = k4.permute(0, 2, 1, 3).reshape(B * N, Hkv, d).contiguous().to(DEV)
+    cu = torch.as_tensor([0, N, 2 * N, 3 * N], dtype=torch.int32, device=DEV)
+    m_var, z_var = ea_router_decide_varlen(packed, cu, N, w1, b1, w2, b2)
+    torch.cuda.synchronize()
+    assert torch.equal(m_pad, m_var) and torch.equal(z_pad, z_var)
