@@ -62,6 +62,10 @@ def parse_args():
                     help="sequences in the decode measurement (0 skips it)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement and print its JSON object")
+    ap.add_argument("--packed-seqs", type=int, default=8,
+                    help="sequences in the packed-batch measurement (0 skips it)")
+    ap.add_argument("--packed-only", action="store_true",
+                    help="run only the packed-batch measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
     return ap.parse_args()
@@ -376,10 +380,113 @@ def run_ours(args, rank, world, local_rank):
                                  + (" (layer 0)" if nlayers > 1 else "")}
         if rank == 0:
             result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
+    if not args.quick and world == 1 and args.packed_seqs > 0:
+        result["packed"] = measure_packed(w, args.packed_seqs, max(args.steps, 5),
+                                          max(args.warmup, 3), dev, stream)
     if not args.quick and world == 1 and args.decode_batch > 0:
         result["decode"] = measure_decode(w, args.decode_batch, max(args.steps, 10),
                                           max(args.warmup, 3), dev, stream)
     return result
+
+
+# ---------------------------------------------------------------- packed batches
+def measure_packed(w: workloads.Workload, nseq: int, steps: int, warmup: int, dev, stream):
+    """A ragged prefill batch (lengths uniform in [seq/8, seq]) packed token-
+    major: router over each sequence's keys, then the fused attention, timed
+    with CUDA events; then the same batch padded to its longest sequence
+    through the padded entry points (the work a padded layout executes)."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_prefill,
+                                                ea_hybrid_attn_prefill_varlen, ea_router_decide,
+                                                ea_router_decide_varlen)
+    Hq, Hkv, d, S, W = w.hq, w.hkv, w.d, w.sink, w.window
+    seed = workloads.layer_seed(w, 0) + 7000
+    lens = workloads.packed_lengths(w, nseq, seed)
+    cu_host = np.cumsum([0] + lens).astype(np.int32)
+    T, Lmax = int(cu_host[-1]), int(max(lens))
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+
+    def rand(*shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    q, k, v = rand(T, Hq, d), rand(T, Hkv, d), rand(T, Hkv, d)
+    cu = torch.as_tensor(cu_host, device=dev)
+    frac = workloads.layer_sparse_frac(w, 0)
+    heads = workloads.sparse_head_set(Hq, frac, seed)
+    w1, b1, w2, b2 = (t.to(dev) for t in workloads.make_router_weights(Hkv * d, w.router_hidden,
+                                                                         Hq, heads, seed))
+    out = torch.empty_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    mask = torch.empty((nseq, Hq), dtype=torch.uint8, device=dev)
+    rws = torch.empty(1 << 24, dtype=torch.uint8, device=dev)
+
+    def step():
+        ea_router_decide_varlen(k, cu, Lmax, w1, b1, w2, b2, workspace=rws, route_mask=mask,
+                                want_logits=False, stream=stream)
+        ea_hybrid_attn_prefill_varlen(q, k, v, cu, mask, Lmax, S, W, out=out, workspace=ws,
+                                      stream=stream)
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ms = timed(step, steps)
+    if ea_get_device_status(ws) != 0:
+        raise RuntimeError("packed prefill status word reports an error")
+    m = mask.cpu().numpy()
+    eff = sum(flops.effective_flops(m[b:b + 1], lens[b], d, S, W) for b in range(nseq))
+    # padded comparator: [nseq, H, Lmax, d] with zero rows past every length
+    qp = torch.zeros((nseq, Hq, Lmax, d), dtype=torch.bfloat16, device=dev)
+    kp = torch.zeros((nseq, Hkv, Lmax, d), dtype=torch.bfloat16, device=dev)
+    vp = torch.zeros_like(kp)
+    for b in range(nseq):
+        t0, t1 = int(cu_host[b]), int(cu_host[b + 1])
+        qp[b, :, :t1 - t0] = q[t0:t1].transpose(0, 1)
+        kp[b, :, :t1 - t0] = k[t0:t1].transpose(0, 1)
+        vp[b, :, :t1 - t0] = v[t0:t1].transpose(0, 1)
+    outp = torch.empty_like(qp)
+    maskp = torch.empty_like(mask)
+
+    def padded_step():
+        # the padded router pools zero rows too (its mask is only timed); the
+        # attention runs the packed batch's routing, so both arms do the same
+        # heads in the same modes
+        ea_router_decide(kp, w1, b1, w2, b2, workspace=rws, route_mask=maskp, want_logits=False,
+                         stream=stream)
+        ea_hybrid_attn_prefill(qp, kp, vp, mask, S, W, out=outp, workspace=ws, stream=stream)
+
+    for _ in range(2):
+        padded_step()
+    torch.cuda.synchronize()
+    ms_pad = timed(padded_step, max(3, steps // 2))
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tf = eff / (ms * 1e-3) / 1e12
+    return {
+        "workload": f"{w.name} packed prefill: {nseq} sequences, lengths {lens} "
+                    f"(T={T}), Hq={Hq} Hkv={Hkv} d={d} S={S} W={W}, router-chosen mask "
+                    f"(SA heads {m.mean():.2f})",
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": round(ms, 4),
+        "effective_tflops": round(tf, 2),
+        "tokens_per_s": round(T / (ms * 1e-3), 1),
+        "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                     "peak_source": f"{src} bf16_tflops (burst)",
+                     "scope": "router + fused attention on the packed batch, effective flops"},
+        "gpu_launches_per_step": 5,
+        "padded_ms_per_step": round(ms_pad, 4),
+        "speedup_vs_padded": round(ms_pad / ms, 3),
+    }
 
 
 # ---------------------------------------------------------------- decode
@@ -584,6 +691,17 @@ def main():
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.packed_only:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = measure_packed(w, max(args.packed_seqs, 1), args.steps, max(args.warmup, 3), dev,
+                             torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
         return 0
     if args.decode_only:
         dev = torch.device("cuda", local_rank)

@@ -21,7 +21,7 @@ import torch
 
 __all__ = ["Workload", "WORKLOADS", "get", "make_qkv", "make_router_weights",
            "make_fixed_mask", "sparse_head_set", "layer_seed",
-           "layer_sparse_frac", "decode_positions"]
+           "layer_sparse_frac", "decode_positions", "packed_lengths"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -161,3 +161,11 @@ def decode_positions(w: Workload, batch: int, seed: int) -> torch.Tensor:
     g = _gen(seed + 211, "cpu")
     lo = max(0, w.seq // 2)
     return torch.randint(lo, w.seq, (batch,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+def packed_lengths(w: Workload, nseq: int, seed: int) -> list:
+    """Sequence lengths of a packed (ragged) prefill batch: uniform in
+    [seq/8, seq], so the batch mixes short prompts with full-length ones."""
+    g = _gen(seed + 307, "cpu")
+    lo = max(1, w.seq // 8)
+    return torch.randint(lo, w.seq + 1, (nseq,), generator=g, dtype=torch.int64).tolist()
