@@ -186,7 +186,8 @@ size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p);
  *             p->select are left untouched.
  * workspace : device, >= ea_hybrid_attn_workspace_size(p) bytes, ZEROED
  *             once before its first use; the kernel only ever writes a
- *             nonzero error code into it (cleared by ea_get_device_status).
+ *             nonzero error code into it (ea_get_device_status reads it and,
+ *             after an error, clears the 256-byte status block).
  * Limits: d in {64, 128}; Hq % Hkv == 0; B <= 1024; B*Hq <= 4096;
  * N <= 32767 * 256.
  */
@@ -236,6 +237,44 @@ ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void
                                         const int32_t* cu_seqlens, const uint8_t* route_mask,
                                         const ea_varlen_params* p, void* out, void* workspace,
                                         size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Router and attention in ONE launch (the router runs in the attention
+ * kernel's prologue, so a routed prefill layer is a single launch).  Same
+ * results, bit for bit, as ea_router_decide (ea_router_decide_varlen)
+ * followed by ea_hybrid_attn_prefill (ea_hybrid_attn_prefill_varlen): the
+ * prologue pools, reduces and runs both MLP layers with the router kernels'
+ * arithmetic, and its phases meet at grid barriers.  The launch is
+ * cooperative: every CTA is resident at once or the call returns EA_ERR_CUDA.
+ *
+ * Arguments: the attention call's, plus the router's (w1, b1, hidden, w2, b2,
+ * threshold as for ea_router_decide).  route_mask (device uint8 [B][Hq]) is
+ * WRITTEN with the decisions and logits_out (device fp32 [B][Hq] or NULL)
+ * with z.  workspace: >= the *_routed_workspace_size bytes, zeroed once
+ * before first use; its first 256 bytes hold the status word and the grid
+ * barrier, the rest the router's scratch.  A barrier that waits past
+ * EA_WAIT_TIMEOUT_MS records EA_ERR_TIMEOUT and the launch ends without
+ * running attention; ea_get_device_status then clears those 256 bytes.
+ * Packed batches need T > 0. */
+size_t ea_hybrid_attn_routed_workspace_size(const ea_attn_params* p, int hidden);
+
+ea_status ea_hybrid_attn_prefill_routed(const void* q, const void* k, const void* v,
+                                        const float* w1, const float* b1, int hidden,
+                                        const float* w2, const float* b2, float threshold,
+                                        uint8_t* route_mask, float* logits_out,
+                                        const ea_attn_params* p, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+size_t ea_hybrid_attn_varlen_routed_workspace_size(const ea_varlen_params* p, int hidden);
+
+ea_status ea_hybrid_attn_prefill_varlen_routed(const void* q, const void* k, const void* v,
+                                               const int32_t* cu_seqlens, const float* w1,
+                                               const float* b1, int hidden, const float* w2,
+                                               const float* b2, float threshold,
+                                               uint8_t* route_mask, float* logits_out,
+                                               const ea_varlen_params* p, void* out,
+                                               void* workspace, size_t workspace_bytes,
+                                               void* stream);
 
 /* Host view of the packed batch's schedule, like ea_schedule_units below:
  * cu_seqlens_host is a HOST int32 [B+1] copy; units_out rows are

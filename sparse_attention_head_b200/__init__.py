@@ -14,5 +14,6 @@ from .api import (HostPrefill, attn_workspace, decode_workspace, ea_decode_kv_po
                   ea_hybrid_attn_prefill, ea_hybrid_attn_workspace_size, ea_router_decide,
                   ea_router_workspace_size, ea_schedule_unit_tiles, ea_schedule_units,
                   make_params, ea_hybrid_attn_prefill_varlen, ea_schedule_units_varlen,
-                  make_varlen_params, ea_router_decide_varlen)
+                  make_varlen_params, ea_router_decide_varlen, ea_hybrid_attn_prefill_routed,
+                  ea_hybrid_attn_prefill_varlen_routed)
 from .flops import attn_visible_pairs, effective_flops, tile_flops  # noqa: F401

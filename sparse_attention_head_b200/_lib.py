@@ -37,6 +37,8 @@ EXPORTED = [
     "ea_decode_kv_policy", "ea_hybrid_attn_varlen_workspace_size",
     "ea_hybrid_attn_prefill_varlen", "ea_schedule_units_varlen",
     "ea_router_varlen_workspace_size", "ea_router_decide_varlen",
+    "ea_hybrid_attn_routed_workspace_size", "ea_hybrid_attn_prefill_routed",
+    "ea_hybrid_attn_varlen_routed_workspace_size", "ea_hybrid_attn_prefill_varlen_routed",
 ]
 
 
@@ -123,6 +125,18 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, pvar, vp, vp, c_size, vp]
     lib.ea_schedule_units_varlen.restype = c_int
     lib.ea_schedule_units_varlen.argtypes = [vp, pvar, vp, vp, c_int]
+    lib.ea_hybrid_attn_routed_workspace_size.restype = c_size
+    lib.ea_hybrid_attn_routed_workspace_size.argtypes = [pparams, c_int]
+    lib.ea_hybrid_attn_prefill_routed.restype = c_int
+    lib.ea_hybrid_attn_prefill_routed.argtypes = [vp, vp, vp, vp, vp, c_int, vp, vp,
+                                                  ctypes.c_float, vp, vp, pparams, vp, vp,
+                                                  c_size, vp]
+    lib.ea_hybrid_attn_varlen_routed_workspace_size.restype = c_size
+    lib.ea_hybrid_attn_varlen_routed_workspace_size.argtypes = [pvar, c_int]
+    lib.ea_hybrid_attn_prefill_varlen_routed.restype = c_int
+    lib.ea_hybrid_attn_prefill_varlen_routed.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, vp,
+                                                         ctypes.c_float, vp, vp, pvar, vp, vp,
+                                                         c_size, vp]
     pdec = ctypes.POINTER(EaDecodeParams)
     lib.ea_decode_workspace_size.restype = c_size
     lib.ea_decode_workspace_size.argtypes = [pdec]

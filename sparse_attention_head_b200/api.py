@@ -240,6 +240,104 @@ def ea_hybrid_attn_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
     return out
 
 
+# ---------------------------------------------------------------- router + attention, one launch
+def _router_shapes(w1, b1, w2, b2, in_dim):
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+        _need(t, name, torch.float32, nd)
+    hidden, Hq = w1.shape[0], w2.shape[0]
+    if w1.shape[1] != in_dim or b1.shape[0] != hidden or w2.shape[1] != hidden \
+            or b2.shape[0] != Hq:
+        raise ValueError("router weight shapes do not match the key states")
+    return hidden, Hq
+
+
+def ea_hybrid_attn_prefill_routed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+                                  b2: torch.Tensor, sink: int, window: int,
+                                  threshold: float = 0.0, *, softmax_scale: float = 0.0,
+                                  select: int = EA_SELECT_ALL,
+                                  route_mask: Optional[torch.Tensor] = None,
+                                  logits: Optional[torch.Tensor] = None,
+                                  out: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None):
+    """Router and attention in one launch (padded q [B, Hq, N, d]); returns
+    (out, route_mask, logits)."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    hidden, Hq_r = _router_shapes(w1, b1, w2, b2, Hkv * d)
+    if Hq_r != Hq or k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("shapes do not match")
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale, select)
+    dev = q.device
+    if route_mask is None:
+        route_mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = int(lib.ea_hybrid_attn_routed_workspace_size(ctypes.byref(p), hidden))
+        if n == 0:
+            raise ValueError("invalid parameters")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=dev)
+    rc = lib.ea_hybrid_attn_prefill_routed(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           w1.data_ptr(), b1.data_ptr(), hidden, w2.data_ptr(),
+                                           b2.data_ptr(), float(threshold), route_mask.data_ptr(),
+                                           logits.data_ptr() if logits is not None else None,
+                                           ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), _stream_ptr(stream, dev))
+    check(rc, "ea_hybrid_attn_prefill_routed")
+    return out, route_mask, logits
+
+
+def ea_hybrid_attn_prefill_varlen_routed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                         cu_seqlens: torch.Tensor, max_seqlen: int,
+                                         w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+                                         b2: torch.Tensor, sink: int, window: int,
+                                         threshold: float = 0.0, *, softmax_scale: float = 0.0,
+                                         select: int = EA_SELECT_ALL,
+                                         route_mask: Optional[torch.Tensor] = None,
+                                         logits: Optional[torch.Tensor] = None,
+                                         out: Optional[torch.Tensor] = None,
+                                         workspace: Optional[torch.Tensor] = None,
+                                         stream: Optional[torch.cuda.Stream] = None):
+    """Router and attention of a packed batch in one launch; returns
+    (out [T, Hq, d], route_mask [B, Hq], logits)."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    hidden, Hq_r = _router_shapes(w1, b1, w2, b2, Hkv * d)
+    if Hq_r != Hq or k.shape != (T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("shapes do not match")
+    p = make_varlen_params(B, Hq, Hkv, T, max_seqlen, d, sink, window, softmax_scale, select)
+    dev = q.device
+    if route_mask is None:
+        route_mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = int(lib.ea_hybrid_attn_varlen_routed_workspace_size(ctypes.byref(p), hidden))
+        if n == 0:
+            raise ValueError("invalid parameters")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=dev)
+    rc = lib.ea_hybrid_attn_prefill_varlen_routed(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens.data_ptr(), w1.data_ptr(),
+        b1.data_ptr(), hidden, w2.data_ptr(), b2.data_ptr(), float(threshold),
+        route_mask.data_ptr(), logits.data_ptr() if logits is not None else None,
+        ctypes.byref(p), out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream_ptr(stream, dev))
+    check(rc, "ea_hybrid_attn_prefill_varlen_routed")
+    return out, route_mask, logits
+
+
 def ea_get_device_status(workspace: torch.Tensor,
                          stream: Optional[torch.cuda.Stream] = None) -> int:
     lib = _lib.load()

@@ -331,7 +331,7 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
 
-  ea::AttnArgs args;
+  ea::AttnArgs args = {};
   if (!encode_bhsd(&args.tm_q, q, p->d, p->N, p->B * p->Hq) ||
       !encode_bhsd(&args.tm_k, k, p->d, p->N, p->B * p->Hkv) ||
       !encode_bhsd(&args.tm_v, v, p->d, p->N, p->B * p->Hkv))
@@ -367,7 +367,9 @@ ea_status ea_get_device_status(void* workspace, void* stream, int* status_out) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return EA_ERR_CUDA;
   if (cudaMemcpy(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return EA_ERR_CUDA;
-  if (host != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return EA_ERR_CUDA;
+  // an error clears the whole 256-byte status block: the status word and the
+  // routed launch's grid-barrier words (left mid-phase by a timeout)
+  if (host != 0 && cudaMemset(workspace, 0, kAttnWorkspace) != cudaSuccess) return EA_ERR_CUDA;
   *status_out = host;
   return EA_OK;
 }
@@ -389,7 +391,7 @@ ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
   if (p->total == 0 || p->max_seqlen == 0) return EA_OK;   // no token: nothing to run
 
-  ea::AttnArgs args;
+  ea::AttnArgs args = {};
   if (!encode_packed(&args.tm_q, q, p->d, p->total, p->Hq) ||
       !encode_packed(&args.tm_k, k, p->d, p->total, p->Hkv) ||
       !encode_packed(&args.tm_v, v, p->d, p->total, p->Hkv))
@@ -417,6 +419,150 @@ ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void
                           ((p->max_seqlen + EA_UNIT_ROWS - 1) / EA_UNIT_ROWS);
   const int grid = static_cast<int>(units < sms ? units : sms);
   cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ routed launches
+namespace {
+
+// Router argument checks shared by the routed entry points.
+ea_status check_router_args(const void* w1, const void* b1, const void* w2, const void* b2,
+                            const uint8_t* mask_out, int Hkv, int d, int hidden, int Hq,
+                            float threshold) {
+  if (!w1 || !b1 || !w2 || !b2 || !mask_out) return EA_ERR_INVALID_ARG;
+  if (hidden <= 0 || threshold != threshold) return EA_ERR_INVALID_ARG;
+  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  return EA_OK;
+}
+
+// Router fields of a routed launch; scratch after the 256-byte status block,
+// grid-barrier words inside it.
+void set_router_args(ea::AttnArgs& a, const void* k, const float* w1, const float* b1,
+                     int hidden, const float* w2, const float* b2, float threshold,
+                     uint8_t* mask_out, float* logits, void* workspace, int nsplit) {
+  a.k_raw = k;
+  a.w1 = w1;
+  a.b1 = b1;
+  a.w2 = w2;
+  a.b2 = b2;
+  a.hidden = hidden;
+  a.threshold = threshold;
+  a.mask_out = mask_out;
+  a.mask = mask_out;
+  a.logits = logits;
+  a.nsplit = nsplit;
+  char* ws = static_cast<char*>(workspace);
+  a.bar_count = reinterpret_cast<unsigned int*>(ws + 64);
+  a.bar_gen = reinterpret_cast<unsigned int*>(ws + 128);
+  a.partials = reinterpret_cast<float*>(ws + kAttnWorkspace);
+}
+
+}  // namespace
+
+size_t ea_hybrid_attn_routed_workspace_size(const ea_attn_params* p, int hidden) {
+  if (check_params(p) != EA_OK || hidden <= 0 || hidden > kRouterMaxHidden) return 0;
+  return kAttnWorkspace + ea::router_workspace_bytes(p->B, p->Hkv, p->N, p->d, hidden);
+}
+
+ea_status ea_hybrid_attn_prefill_routed(const void* q, const void* k, const void* v,
+                                        const float* w1, const float* b1, int hidden,
+                                        const float* w2, const float* b2, float threshold,
+                                        uint8_t* route_mask, float* logits_out,
+                                        const ea_attn_params* p, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (!q || !k || !v || !out) return EA_ERR_INVALID_ARG;
+  st = check_router_args(w1, b1, w2, b2, route_mask, p->Hkv, p->d, hidden, p->Hq, threshold);
+  if (st != EA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  const size_t need = ea_hybrid_attn_routed_workspace_size(p, hidden);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+
+  ea::AttnArgs args = {};
+  if (!encode_bhsd(&args.tm_q, q, p->d, p->N, p->B * p->Hq) ||
+      !encode_bhsd(&args.tm_k, k, p->d, p->N, p->B * p->Hkv) ||
+      !encode_bhsd(&args.tm_v, v, p->d, p->N, p->B * p->Hkv))
+    return EA_ERR_CUDA;
+  args.out = out;
+  args.status = static_cast<int*>(workspace);
+  args.cu_seqlens = nullptr;
+  args.total = 0;
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->N;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = debug_drop_kv_pos();
+  set_router_args(args, k, w1, b1, hidden, w2, b2, threshold, route_mask, logits_out, workspace,
+                  ea::router_num_splits(p->B, p->Hkv, p->N));
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  cudaError_t err = ea::launch_attn_routed(p->d, args, sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+size_t ea_hybrid_attn_varlen_routed_workspace_size(const ea_varlen_params* p, int hidden) {
+  if (check_varlen(p) != EA_OK || hidden <= 0 || hidden > kRouterMaxHidden) return 0;
+  return kAttnWorkspace +
+         ea::router_workspace_bytes(p->B, p->Hkv, p->max_seqlen > 0 ? p->max_seqlen : 1, p->d,
+                                    hidden);
+}
+
+ea_status ea_hybrid_attn_prefill_varlen_routed(const void* q, const void* k, const void* v,
+                                               const int32_t* cu_seqlens, const float* w1,
+                                               const float* b1, int hidden, const float* w2,
+                                               const float* b2, float threshold,
+                                               uint8_t* route_mask, float* logits_out,
+                                               const ea_varlen_params* p, void* out,
+                                               void* workspace, size_t workspace_bytes,
+                                               void* stream) {
+  ea_status st = check_varlen(p);
+  if (st != EA_OK) return st;
+  if (!q || !k || !v || !cu_seqlens || !out) return EA_ERR_INVALID_ARG;
+  st = check_router_args(w1, b1, w2, b2, route_mask, p->Hkv, p->d, hidden, p->Hq, threshold);
+  if (st != EA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  const size_t need = ea_hybrid_attn_varlen_routed_workspace_size(p, hidden);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  if (p->total == 0) return EA_ERR_UNSUPPORTED;   // the tensor maps need a token
+
+  ea::AttnArgs args = {};
+  if (!encode_packed(&args.tm_q, q, p->d, p->total, p->Hq) ||
+      !encode_packed(&args.tm_k, k, p->d, p->total, p->Hkv) ||
+      !encode_packed(&args.tm_v, v, p->d, p->total, p->Hkv))
+    return EA_ERR_CUDA;
+  args.out = out;
+  args.status = static_cast<int*>(workspace);
+  args.cu_seqlens = cu_seqlens;
+  args.total = p->total;
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->max_seqlen;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = debug_drop_kv_pos();
+  set_router_args(args, k, w1, b1, hidden, w2, b2, threshold, route_mask, logits_out, workspace,
+                  ea::router_num_splits(p->B, p->Hkv, p->max_seqlen > 0 ? p->max_seqlen : 1));
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  cudaError_t err = ea::launch_attn_routed(p->d, args, sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

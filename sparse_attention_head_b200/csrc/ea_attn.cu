@@ -38,6 +38,7 @@
 #include "ea_internal.h"
 #include "ea_math.cuh"
 #include "ea_ptx.cuh"
+#include "ea_router_dev.cuh"
 #include "ea_sched.h"
 #include "ea_tmem.cuh"
 
@@ -92,12 +93,105 @@ struct Bars {
   uint32_t o_empty;
 };
 
+// Route bit of entry idx, read through the coherent path: in a routed launch
+// other CTAs wrote it earlier in the same launch.  Out of range: 0.
+__device__ __forceinline__ uint8_t ld_mask(const uint8_t* mask, int idx) {
+  return idx >= 0 ? *reinterpret_cast<const volatile uint8_t*>(mask + idx) : 0;
+}
+
+// Grid barrier of the routed prologue.  Every CTA arrives once per phase;
+// the last arrival resets the count and advances the generation, which the
+// others wait for (no reset between launches is needed).  Bounded: returns
+// false, with EA_ERR_TIMEOUT in the status word, if the others do not arrive
+// in time.  Needs every CTA resident at once (a cooperative launch).
+__device__ bool grid_sync(const AttnArgs& args, volatile int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned int* gen = args.bar_gen;
+    const unsigned int g = *gen;
+    __threadfence();
+    const unsigned int arrived = atomicAdd(args.bar_count, 1u) + 1u;
+    bool ok = true;
+    if (arrived == gridDim.x) {
+      atomicExch(args.bar_count, 0u);
+      __threadfence();
+      atomicAdd(args.bar_gen, 1u);
+    } else {
+      const uint64_t t0 = global_ns();
+      for (uint32_t it = 0; *gen == g; ++it) {
+        if ((it & 63) == 63 && global_ns() - t0 > args.timeout_ns) {
+          atomicCAS(args.status, 0, EA_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *s_flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *s_flag != 0;
+}
+
+// The Attention Router inside the attention launch (EA blog §2.1), with the
+// standalone router kernels' arithmetic: pooling items (split, kv head, b)
+// by threads 0..255 exactly as ea_router_pool_kernel, x as
+// ea_router_reduce_kernel, then one warp per output of each MLP layer.  The
+// phases meet at grid barriers; the mask is complete before any CTA builds
+// its unit list.  Shared memory is free before the pipeline starts, so the
+// Q region holds the pooling reduction.
 template <int D>
+__device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile int* s_flag) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = args.B, Hkv = args.Hkv, ns = args.nsplit, hidden = args.hidden;
+  const int in_dim = Hkv * D;
+  float* partials = args.partials;
+  float* xbuf = partials + static_cast<size_t>(B) * Hkv * ns * D;
+  float* hbuf = xbuf + static_cast<size_t>(B) * in_dim;
+  if (tid < kPoolThreads) {
+    float* red = reinterpret_cast<float*>(smem);
+    const int items = ns * Hkv * B;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      const int split = it % ns, hk = (it / ns) % Hkv, b = it / (ns * Hkv);
+      router_pool_item<D>(static_cast<const __nv_bfloat16*>(args.k_raw), args.cu_seqlens, args.N,
+                          args.total, Hkv, b, hk, split, ns, partials, red, tid, 1);
+    }
+  }
+  if (!grid_sync(args, s_flag)) return false;
+  for (int i = blockIdx.x * blockDim.x + tid; i < B * in_dim; i += gridDim.x * blockDim.x)
+    xbuf[i] = router_x(partials, args.cu_seqlens, Hkv, args.N, args.total, D, ns, i / in_dim,
+                       i % in_dim);
+  if (!grid_sync(args, s_flag)) return false;
+  const int nw = blockDim.x / 32;
+  for (int o = blockIdx.x * nw + warp; o < B * hidden; o += gridDim.x * nw) {
+    const int b = o / hidden, oo = o % hidden;
+    const float v = router_warp_dot(xbuf + static_cast<size_t>(b) * in_dim, in_dim, args.w1,
+                                    args.b1, oo, lane);
+    if (lane == 0) hbuf[static_cast<size_t>(b) * hidden + oo] = fmaxf(v, 0.f);
+  }
+  if (!grid_sync(args, s_flag)) return false;
+  for (int o = blockIdx.x * nw + warp; o < B * args.Hq; o += gridDim.x * nw) {
+    const int b = o / args.Hq, oo = o % args.Hq;
+    const float v = router_warp_dot(hbuf + static_cast<size_t>(b) * hidden, hidden, args.w2,
+                                    args.b2, oo, lane);
+    if (lane == 0) {
+      if (args.logits) args.logits[o] = v;
+      args.mask_out[o] = (v > args.threshold) ? 1 : 0;
+    }
+  }
+  return grid_sync(args, s_flag);
+}
+
+template <int D, bool kRouted>
 __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  if constexpr (kRouted) {
+    if (!routed_prologue<D>(args, smem, reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16)))
+      return;   // a grid barrier timed out; nothing is allocated or in flight yet
+  }
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -213,7 +307,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       for (int h0 = 0; h0 < args.Hq; h0 += 32) {
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && args.mask[idx] == 0 && args.select != EA_SELECT_SA;
+        const bool ok = h < args.Hq && ld_mask(args.mask, idx) == 0 && args.select != EA_SELECT_SA;
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nfa += __popc(bits);
@@ -226,7 +320,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       for (int h0 = 0; h0 < args.Hq; h0 += 32) {
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && args.mask[idx] != 0 && args.select != EA_SELECT_FA;
+        const bool ok = h < args.Hq && ld_mask(args.mask, idx) != 0 && args.select != EA_SELECT_FA;
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nsa += __popc(bits);
@@ -622,26 +716,39 @@ int attn_smem_bytes(int D) {
   return D == 128 ? AttnCfg<128>::kSmem : AttnCfg<64>::kSmem;
 }
 
-template <int D>
+template <int D, bool kRouted>
 static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream) {
   const int smem = AttnCfg<D>::kSmem;
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !configured[dev]) {
-    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D>,
+  if (dev >= 64 || !configured[dev]) {
+    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D, kRouted>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    configured[dev] = 1;
+    if (dev < 64) configured[dev] = 1;
   }
-  ea_hybrid_attn_kernel<D><<<grid, AttnCfg<D>::kThreads, smem, stream>>>(args);
-  return cudaGetLastError();
+  if (!kRouted) {
+    ea_hybrid_attn_kernel<D, false><<<grid, AttnCfg<D>::kThreads, smem, stream>>>(args);
+    return cudaGetLastError();
+  }
+  // every CTA must be resident at once: the runtime refuses a cooperative
+  // launch that cannot be
+  void* params[] = {const_cast<AttnArgs*>(&args)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(ea_hybrid_attn_kernel<D, true>),
+                                     dim3(grid), dim3(AttnCfg<D>::kThreads), params, smem, stream);
 }
 
 cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stream) {
-  if (D == 128) return launch_d<128>(args, grid, stream);
-  if (D == 64) return launch_d<64>(args, grid, stream);
+  if (D == 128) return launch_d<128, false>(args, grid, stream);
+  if (D == 64) return launch_d<64, false>(args, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_routed(int D, const AttnArgs& args, int grid, cudaStream_t stream) {
+  if (D == 128) return launch_d<128, true>(args, grid, stream);
+  if (D == 64) return launch_d<64, true>(args, grid, stream);
   return cudaErrorInvalidValue;
 }
 

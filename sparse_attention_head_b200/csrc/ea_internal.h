@@ -30,6 +30,22 @@ struct alignas(64) AttnArgs {
   // Failure-detection test hook (-1 = off): the producer skips the copy of
   // this K/V ring position, so the kernel's bounded wait for it runs out.
   int debug_drop_kv_pos;
+  // Routed launch only: the router runs in the kernel's prologue (pool,
+  // x, MLP layer 1, layer 2 + threshold, separated by grid barriers) and
+  // writes the route mask (`mask` above points at the same buffer).
+  const void* k_raw;        // the key tensor as the router reads it
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  int hidden;
+  float threshold;
+  uint8_t* mask_out;
+  float* logits;            // may be nullptr
+  float* partials;          // router scratch: partials, then x, then h
+  int nsplit;
+  unsigned int* bar_count;  // grid barrier: arrivals of the current phase
+  unsigned int* bar_gen;    //               and its generation
 };
 
 // SM count of the current device (cached per device); 0 on error.
@@ -42,6 +58,9 @@ int attn_smem_bytes(int D);
 
 // Launch the fused kernel (D in {64, 128}) with `grid` CTAs.
 cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stream);
+// The routed kernel (router in the prologue), as a cooperative launch: all
+// CTAs resident at once (they meet at grid barriers), or an error.
+cudaError_t launch_attn_routed(int D, const AttnArgs& args, int grid, cudaStream_t stream);
 
 // Router: pooled partial sums, then the MLP and the threshold.
 int router_num_splits(int B, int Hkv, int N);

@@ -25,92 +25,34 @@
 
 #include "ea.h"
 #include "ea_internal.h"
+#include "ea_router_dev.cuh"
 
 namespace ea {
 
-constexpr int kPoolThreads = 256;
 constexpr int kMlpThreads = 256;
-
-// Rows of (b, kv head): padded K [B][Hkv][N][d] (cu == nullptr) or packed K
-// [T][Hkv][d] with sequence b at tokens [cu[b], cu[b + 1]).  A packed range
-// outside [0, T] (inconsistent offsets) pools nothing.
-__device__ __forceinline__ int router_seq_rows(const int32_t* cu, int N, int total, int b,
-                                               int* t0) {
-  if (!cu) {
-    *t0 = 0;
-    return N;
-  }
-  const int a = cu[b], e = cu[b + 1];
-  *t0 = a;
-  return (a >= 0 && e >= a && e <= total) ? e - a : 0;
-}
 
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
     const __nv_bfloat16* __restrict__ k, const int32_t* __restrict__ cu, int N, int total,
     int nsplit, float* __restrict__ partials) {
-  constexpr int TPR = D / 8;                 // threads per row (8 channels each)
-  constexpr int RPI = kPoolThreads / TPR;    // rows per iteration
-  __shared__ float red[RPI][D];
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int Hkv = gridDim.y;
-  const int cg = threadIdx.x % TPR;
-  const int rs = threadIdx.x / TPR;
-  int t0;
-  const int len = router_seq_rows(cu, N, total, b, &t0);
-  const int chunk = (len + nsplit - 1) / nsplit;
-  const int n0 = split * chunk;
-  const int n1 = min(len, n0 + chunk);
-  // padded: plane (b, hk) of N rows of D; packed: token rows of Hkv * D
-  const size_t row_stride = cu ? static_cast<size_t>(Hkv) * D : static_cast<size_t>(D);
-  const __nv_bfloat16* base =
-      (cu ? k + (static_cast<size_t>(t0) * Hkv + hk) * D
-          : k + (static_cast<size_t>(b) * Hkv + hk) * N * D) + cg * 8;
-  float acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  int n = n0 + rs;
-#pragma unroll 4
-  for (; n < n1; n += RPI) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(n) * row_stride));
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(p[j]);
-      acc[2 * j] += f.x;
-      acc[2 * j + 1] += f.y;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) red[rs][cg * 8 + j] = acc[j];
-  __syncthreads();
-  for (int c = threadIdx.x; c < D; c += kPoolThreads) {
-    float s = 0.f;
-    for (int r = 0; r < RPI; ++r) s += red[r][c];
-    partials[((static_cast<size_t>(b) * Hkv + hk) * nsplit + split) * D + c] = s;
-  }
+  __shared__ float red[(kPoolThreads / (D / 8)) * D];
+  router_pool_item<D>(k, cu, N, total, gridDim.y, blockIdx.z, blockIdx.y, blockIdx.x, nsplit,
+                      partials, red, threadIdx.x, 1);
 }
 
-// x[b][hk*d + c] = (sum over splits, in split order) / rows of sequence b
-// (zero for an empty sequence); one thread per channel.
+// x[b][j] for one channel per thread.
 __global__ void ea_router_reduce_kernel(const float* __restrict__ partials,
                                         const int32_t* __restrict__ cu, int Hkv, int N, int total,
                                         int d, int nsplit, float* __restrict__ x) {
   const int b = blockIdx.y;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;   // j = hk * d + c
   if (j >= Hkv * d) return;
-  const int hk = j / d, c = j % d;
-  int t0;
-  const int len = router_seq_rows(cu, N, total, b, &t0);
-  const float* p = partials + (static_cast<size_t>(b) * Hkv + hk) * nsplit * d + c;
-  float s = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) s += p[static_cast<size_t>(sp) * d];
-  x[static_cast<size_t>(b) * Hkv * d + j] = len > 0 ? s * (1.0f / static_cast<float>(len)) : 0.f;
+  x[static_cast<size_t>(b) * Hkv * d + j] = router_x(partials, cu, Hkv, N, total, d, nsplit, b, j);
 }
 
-// One warp per output: y[b][o] = act(W[o] . x[b] + bias[o]), float4 over the
-// input, lanes reduced in a fixed shuffle order.  For the last layer the
-// output is the logit z, and the route bit z > threshold is written too.
+// One warp per output: y[b][o] = act(W[o] . x[b] + bias[o]).  For the last
+// layer the output is the logit z, and the route bit z > threshold is
+// written too.
 template <bool kLast>
 __global__ void __launch_bounds__(kMlpThreads) ea_router_layer_kernel(
     const float* __restrict__ x, int in_dim, const float* __restrict__ w,
@@ -120,22 +62,8 @@ __global__ void __launch_bounds__(kMlpThreads) ea_router_layer_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o = blockIdx.x * (kMlpThreads / 32) + warp;
   if (o >= out_dim) return;
-  const float4* wr = reinterpret_cast<const float4*>(w + static_cast<size_t>(o) * in_dim);
-  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * in_dim);
-  float acc = 0.f;
-#pragma unroll 4
-  for (int j = lane; j < in_dim / 4; j += 32) {
-    const float4 wv = __ldg(wr + j);
-    const float4 xv = xr[j];
-    acc = fmaf(wv.x, xv.x, acc);
-    acc = fmaf(wv.y, xv.y, acc);
-    acc = fmaf(wv.z, xv.z, acc);
-    acc = fmaf(wv.w, xv.w, acc);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  const float v = router_warp_dot(x + static_cast<size_t>(b) * in_dim, in_dim, w, bias, o, lane);
   if (lane == 0) {
-    const float v = acc + bias[o];
     if (kLast) {
       if (y) y[static_cast<size_t>(b) * out_dim + o] = v;
       mask[static_cast<size_t>(b) * out_dim + o] = (v > threshold) ? 1 : 0;

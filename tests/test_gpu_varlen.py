@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import compare, f64, sample_rows
+from gpu_common import compare, f64, few_key_rows_packed, sample_rows
 from sparse_attention_head_b200 import _lib, build
 from sparse_attention_head_b200.api import (EA_SELECT_FA, EA_SELECT_SA, ea_get_device_status,
                                             ea_hybrid_attn_prefill,
@@ -62,7 +62,8 @@ def test_varlen_matches_oracle(cu, Hq, Hkv, d, S, W):
     out, ws = _run(q, k, v, cu, mask, S, W)
     assert ea_get_device_status(ws) == 0
     ref = oracle.attention_varlen(f64(q), f64(k), f64(v), cu, mask, S, W)
-    compare(out, ref, f"varlen cu={cu}", few_keys=W <= 2)
+    compare(out, ref, f"varlen cu={cu}", few_keys=W <= 2,
+            few_rows=None if W <= 2 else few_key_rows_packed(cu, mask, Hq, S, W))
 
 
 def test_varlen_equal_lengths_match_the_padded_kernel_bitwise():
