@@ -349,6 +349,32 @@ def run_ours(args, rank, world, local_rank):
             "full_causal_tflops": round(full_eff / (full_ms * 1e-3) / 1e12, 2),
             "elastic_speedup_vs_full_causal": round(full_ms / fused_ms, 3),
         }
+        if L["router"] is not None:
+            # router + attention: the two-launch pass against the one routed
+            # (cooperative) launch that runs the router in its prologue
+            from sparse_attention_head_b200.api import ea_hybrid_attn_prefill_routed
+            m_tmp = torch.empty_like(masks[0])
+            ws_routed = torch.zeros(1 << 24, dtype=torch.uint8, device=dev)
+
+            def two_launch():
+                ea_router_decide(L["k"], *L["router"], workspace=rws, route_mask=m_tmp,
+                                 want_logits=False)
+                ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], m_tmp, w.sink, w.window,
+                                       out=out_tmp, workspace=aws)
+
+            def routed():
+                ea_hybrid_attn_prefill_routed(L["q"], L["k"], L["v"], *L["router"], w.sink,
+                                              w.window, route_mask=m_tmp, out=out_tmp,
+                                              workspace=ws_routed)
+            two_ms = timeit(two_launch)
+            routed_ms = timeit(routed)
+            if ea_get_device_status(ws_routed) != 0:
+                raise RuntimeError("routed launch status word reports an error")
+            result["comparators"].update({
+                "router_then_attn_ms": round(two_ms, 4),
+                "routed_one_launch_ms": round(routed_ms, 4),
+                "routed_speedup_vs_two_launches": round(two_ms / routed_ms, 3),
+            })
         # end to end through the public API with host buffers (layer 0; for a
         # multi-layer workload the metric uses that layer's work only)
         ek = args.e2e_steps or K
