@@ -70,6 +70,10 @@ __all__ = [
     "router_pool_varlen",
     "router_decide_varlen",
     "attention_varlen",
+    "attention_lse",
+    "attention_backward",
+    "router_gumbel_forward",
+    "router_ste_backward",
 ]
 
 
@@ -401,3 +405,123 @@ def attention_varlen(q, k, v, cu_seqlens, mask, sink: int, window: int,
         o = attention(qs, ks, vs, np.asarray(mask)[b:b + 1], sink, window, scale, block)
         out[t0:t1] = o[0].transpose(1, 0, 2)
     return out
+
+
+# --------------------------------------------------------------------------
+# Backward pass (training).  EA blog §2.1, training trick: the discrete
+# routing decision is made differentiable with Gumbel-Softmax and a
+# straight-through estimator.  Readings taken here (the pages give no
+# formula): one logit z per head is the two-class pair (0, z); with Gumbel
+# noise g0, g1 (drawn by the caller and passed in) and temperature tau,
+#   r_soft = sigmoid((z + g1 - g0) / tau),   r_hard = [z + g1 - g0 > 0];
+# the forward uses r_hard (out = r_hard O_SA + (1 - r_hard) O_FA per head)
+# and the backward differentiates r_soft, so that
+#   dL/dr = sum over the head's rows and channels of dO * (O_SA - O_FA),
+#   dL/dz = dL/dr * r_soft (1 - r_soft) / tau,
+# and the gradient reaches the attention of the selected mode only.
+# --------------------------------------------------------------------------
+
+def _head_probs(q, k, mask, b, h, sink, window, scale):
+    """Dense softmax probabilities [N, N] of one head (zeros off the pattern)."""
+    Hq, N = q.shape[1], q.shape[2]
+    g = Hq // k.shape[1]
+    s = (q[b, h] @ k[b, h // g].T) * scale
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    vis = j <= i
+    if mask[b, h]:
+        vis &= (j < sink) | ((i - j) < window)
+    s = np.where(vis, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=1, keepdims=True), s
+
+
+def attention_lse(q, k, mask, sink: int, window: int, scale: float | None = None) -> np.ndarray:
+    """[B, Hq, N]: natural log of sum_j exp(scale q_i . k_j) over visible j."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.empty((B, Hq, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            _, s = _head_probs(q, k, mask, b, h, sink, window, scale)
+            m = np.max(s, axis=1)
+            out[b, h] = m + np.log(np.sum(np.exp(s - m[:, None]), axis=1))
+    return out
+
+
+def attention_backward(q, k, v, dout, mask, sink: int, window: int,
+                       scale: float | None = None):
+    """(dq [B,Hq,N,d], dk [B,Hkv,N,d], dv [B,Hkv,N,d]) of L = sum(dout * out),
+    out = attention(q, k, v, mask, ...); per head in its own mode, a kv
+    head's gradients summed over its query heads.  Dense per head (small N):
+      P = softmax(scale q k^T | visible), dV = P^T dO, dP = dO V^T,
+      D_i = sum_c dO_ic O_ic, dS = P * (dP - D), dQ = scale dS K,
+      dK = scale dS^T Q."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // g
+            p, _ = _head_probs(q, k, mask, b, h, sink, window, scale)
+            o = p @ v[b, hk]
+            dv[b, hk] += p.T @ dout[b, h]
+            dp = dout[b, h] @ v[b, hk].T
+            dd = np.sum(dout[b, h] * o, axis=1, keepdims=True)
+            ds = p * (dp - dd)
+            dq[b, h] = scale * (ds @ k[b, hk])
+            dk[b, hk] += scale * (ds.T @ q[b, h])
+    return dq, dk, dv
+
+
+def router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, tau: float):
+    """Training-time routing: (r_hard [B,Hq] uint8, r_soft [B,Hq], z [B,Hq])."""
+    z = router_mlp(router_pool(k), w1, b1, w2, b2)
+    u = (z + np.asarray(g1, dtype=np.float64) - np.asarray(g0, dtype=np.float64)) / tau
+    r_soft = 1.0 / (1.0 + np.exp(-u))
+    r_hard = (u > 0.0).astype(np.uint8)
+    return r_hard, r_soft, z
+
+
+def router_ste_backward(k, w1, b1, w2, b2, g0, g1, tau: float, dout, o_fa, o_sa):
+    """Router gradients through the straight-through estimator.
+
+    dout, o_fa, o_sa: [B, Hq, N, d] (the layer's output gradient and both
+    modes' outputs).  Returns (dr [B,Hq], dz [B,Hq], dw1, db1, dw2, db2,
+    dk_router [B,Hkv,N,d]) where dk_router is the keys' gradient through the
+    pooling (each position gets dx / N)."""
+    k = np.asarray(k, dtype=np.float64)
+    w1 = np.asarray(w1, dtype=np.float64)
+    b1 = np.asarray(b1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64)
+    B, Hkv, N, d = k.shape
+    dout = np.asarray(dout, dtype=np.float64)
+    diff = np.asarray(o_sa, dtype=np.float64) - np.asarray(o_fa, dtype=np.float64)
+    dr = np.sum(dout * diff, axis=(2, 3))
+    _, r_soft, _ = router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, tau)
+    dz = dr * r_soft * (1.0 - r_soft) / tau
+    x = router_pool(k)
+    pre = x @ w1.T + b1
+    h = np.where(pre > 0.0, pre, 0.0)
+    dw2 = dz.T @ h
+    db2 = np.sum(dz, axis=0)
+    dh = dz @ w2
+    dpre = np.where(pre > 0.0, dh, 0.0)
+    dw1 = dpre.T @ x
+    db1 = np.sum(dpre, axis=0)
+    dx = dpre @ w1
+    dk_router = np.broadcast_to((dx / N).reshape(B, Hkv, 1, d), (B, Hkv, N, d)).copy()
+    return dr, dz, dw1, db1, dw2, db2, dk_router

@@ -52,6 +52,17 @@ MUTATIONS = {
     "varlen_first_mask_row": ("np.asarray(mask)[b:b + 1]", "np.asarray(mask)[0:1]"),
     "varlen_heads_as_positions": ("qs = q[t0:t1].transpose(1, 0, 2)[None]",
                                   "qs = q[t0:t1].reshape(Hq, t1 - t0, d)[None]"),
+    "bwd_missing_rowsum": ("ds = p * (dp - dd)", "ds = p * dp"),
+    "bwd_dk_unscaled": ("dk[b, hk] += scale * (ds.T @ q[b, h])", "dk[b, hk] += ds.T @ q[b, h]"),
+    "bwd_dv_untransposed": ("dv[b, hk] += p.T @ dout[b, h]", "dv[b, hk] += p @ dout[b, h]"),
+    "bwd_gqa_overwrite": ("dv[b, hk] += p.T @ dout[b, h]", "dv[b, hk] = p.T @ dout[b, h]"),
+    "lse_without_max": ("out[b, h] = m + np.log(", "out[b, h] = np.log("),
+    "ste_missing_tau": ("dz = dr * r_soft * (1.0 - r_soft) / tau",
+                        "dz = dr * r_soft * (1.0 - r_soft)"),
+    "ste_relu_mask_dropped": ("dpre = np.where(pre > 0.0, dh, 0.0)", "dpre = dh"),
+    "ste_pool_not_divided": ("(dx / N).reshape(B, Hkv, 1, d)", "dx.reshape(B, Hkv, 1, d)"),
+    "ste_diff_sign": ("diff = np.asarray(o_sa, dtype=np.float64) - np.asarray(o_fa",
+                      "diff = np.asarray(o_fa, dtype=np.float64) - np.asarray(o_sa"),
 }
 
 

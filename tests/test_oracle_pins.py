@@ -388,3 +388,108 @@ def test_varlen_router_pool_closed_forms():
         want = np.zeros(Hkv * d) if t1 == t0 else np.array(
             [(t0 + t1 - 1) / 2 + 100 * kh + 1000 * c for kh in range(Hkv) for c in range(d)])
         np.testing.assert_allclose(x[b], want, rtol=0, atol=1e-9)
+
+
+# --------------------------------------------------------------------------
+# Backward pass and the straight-through router gradients
+# --------------------------------------------------------------------------
+
+def _fd_grad(f, x, eps=1e-6):
+    """Central finite differences of scalar f over every element of x."""
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + eps
+        fp = f()
+        x[i] = old - eps
+        fm = f()
+        x[i] = old
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+def test_attention_backward_matches_finite_differences():
+    """Gradients of L = sum(dout * out) against central differences of the
+    per-element brute-force forward (independent of the backward formulas);
+    GQA with FA and SA heads sharing kv heads."""
+    rng = np.random.default_rng(71)
+    B, Hq, Hkv, N, d, S, W = 1, 4, 2, 9, 3, 1, 3
+    q = rng.standard_normal((B, Hq, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    dout = rng.standard_normal((B, Hq, N, d))
+    mask = np.array([[0, 1, 1, 0]], np.uint8)
+
+    def loss():
+        return float(np.sum(dout * oracle.brute_force_attention(q, k, v, mask, S, W)))
+    dq, dk, dv = oracle.attention_backward(q, k, v, dout, mask, S, W)
+    np.testing.assert_allclose(dq, _fd_grad(loss, q), rtol=0, atol=1e-6)
+    np.testing.assert_allclose(dk, _fd_grad(loss, k), rtol=0, atol=1e-6)
+    np.testing.assert_allclose(dv, _fd_grad(loss, v), rtol=0, atol=1e-6)
+
+
+def test_attention_lse_matches_the_definition():
+    rng = np.random.default_rng(72)
+    B, Hq, Hkv, N, d, S, W = 1, 2, 1, 11, 4, 2, 3
+    q = rng.standard_normal((B, Hq, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    mask = np.array([[0, 1]], np.uint8)
+    lse = oracle.attention_lse(q, k, mask, S, W)
+    for h in range(Hq):
+        for i in range(N):
+            tot = 0.0
+            for j in range(N):
+                if oracle.visible(i, j, bool(mask[0, h]), S, W):
+                    tot += math.exp(float(q[0, h, i] @ k[0, 0, j]) / math.sqrt(d))
+            assert abs(lse[0, h, i] - math.log(tot)) < 1e-12
+
+
+def test_router_ste_backward_matches_the_soft_surrogate():
+    """The straight-through gradients equal the exact gradients of the soft
+    surrogate sum(dout * (r_soft O_SA + (1 - r_soft) O_FA)) with both
+    attention outputs held fixed (central differences)."""
+    rng = np.random.default_rng(73)
+    B, Hq, Hkv, N, d, hidden, tau = 2, 3, 2, 5, 2, 6, 0.7
+    k = rng.standard_normal((B, Hkv, N, d))
+    w1 = rng.standard_normal((hidden, Hkv * d)) * 0.7
+    b1 = rng.standard_normal(hidden) * 0.3
+    w2 = rng.standard_normal((Hq, hidden)) * 0.7
+    b2 = rng.standard_normal(Hq) * 0.3
+    g0 = rng.gumbel(size=(B, Hq))
+    g1 = rng.gumbel(size=(B, Hq))
+    dout = rng.standard_normal((B, Hq, 4, 3))
+    o_fa = rng.standard_normal((B, Hq, 4, 3))
+    o_sa = rng.standard_normal((B, Hq, 4, 3))
+
+    def loss():
+        x = k.mean(axis=2).reshape(B, Hkv * d)
+        pre = x @ w1.T + b1
+        z = np.maximum(pre, 0.0) @ w2.T + b2
+        r = 1.0 / (1.0 + np.exp(-(z + g1 - g0) / tau))
+        out = r[:, :, None, None] * o_sa + (1.0 - r[:, :, None, None]) * o_fa
+        return float(np.sum(dout * out))
+    dr, dz, dw1, db1, dw2, db2, dk = oracle.router_ste_backward(k, w1, b1, w2, b2, g0, g1, tau,
+                                                                dout, o_fa, o_sa)
+    np.testing.assert_allclose(dr, np.sum(dout * (o_sa - o_fa), axis=(2, 3)), atol=1e-12)
+    for got, x in ((dw1, w1), (db1, b1), (dw2, w2), (db2, b2), (dk, k)):
+        np.testing.assert_allclose(got, _fd_grad(loss, x), rtol=0, atol=1e-6)
+
+
+def test_gumbel_hard_decision_is_the_soft_argmax():
+    rng = np.random.default_rng(74)
+    B, Hkv, N, d, Hq, hidden = 3, 2, 6, 4, 5, 8
+    k = rng.standard_normal((B, Hkv, N, d))
+    w1, b1 = rng.standard_normal((hidden, Hkv * d)), rng.standard_normal(hidden)
+    w2, b2 = rng.standard_normal((Hq, hidden)), rng.standard_normal(Hq)
+    g0, g1 = rng.gumbel(size=(B, Hq)), rng.gumbel(size=(B, Hq))
+    r_hard, r_soft, z = oracle.router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, 0.5)
+    np.testing.assert_array_equal(r_hard, (r_soft > 0.5).astype(np.uint8))
+    # no noise: the hard decision is the inference threshold z > 0
+    r0, _, z0 = oracle.router_gumbel_forward(k, w1, b1, w2, b2, np.zeros_like(g0),
+                                             np.zeros_like(g1), 0.5)
+    np.testing.assert_array_equal(r0, oracle.router_decide(k, w1, b1, w2, b2)[0])
+    # a small temperature makes the soft decision hard
+    _, r_cold, _ = oracle.router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, 1e-6)
+    np.testing.assert_allclose(r_cold, r_hard, atol=1e-6)
