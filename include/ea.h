@@ -203,6 +203,38 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
  * out).  Returns EA_ERR_CUDA if the synchronisation or the copy fails. */
 ea_status ea_get_device_status(void* workspace, void* stream, int* status_out);
 
+/* Forward for training: ea_hybrid_attn_prefill plus the natural log-sum-exp
+ * of every row, lse (device fp32 [B][Hq][N]) = log sum_j exp(scale q_i.k_j)
+ * over the row's visible keys; the backward reads it. */
+ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v,
+                                     const uint8_t* route_mask, const ea_attn_params* p,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Backward pass (training; EA blog §2.1: the router is trained through a
+ * Gumbel-Softmax straight-through estimator, so the attention of each head's
+ * mode receives the output gradient).  With P the forward's softmax of a head
+ * (its own mode) and L = sum(dout * out):
+ *   dV = P^T dO, dP = dO V^T, D_i = sum_c dO_ic O_ic, dS = P * (dP - D),
+ *   dQ = scale dS K, dK = scale dS^T Q,
+ * dK and dV of a kv head summed over its query heads.
+ * q, k, v, out, dout : device bf16, padded BHSD (out and dout [B][Hq][N][d]).
+ * lse        : the forward's log-sum-exp (ea_hybrid_attn_prefill_lse).
+ * route_mask : the forward's mask.
+ * dq         : device bf16 [B][Hq][N][d]; dk, dv: [B][Hkv][N][d]; written.
+ * workspace  : >= ea_hybrid_attn_backward_workspace_size(p) bytes, zeroed
+ *              once; status word, then D (fp32 [B][Hq][N]).
+ * Arithmetic: bf16 tensor-core operands (P and dS rounded to bf16), fp32
+ * accumulation, bf16 results.  Limits: d = 128, p->select == EA_SELECT_ALL,
+ * plus those of ea_hybrid_attn_prefill. */
+size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p);
+
+ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                                  const void* dout, const float* lse, const uint8_t* route_mask,
+                                  const ea_attn_params* p, void* dq, void* dk, void* dv,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Packed variable-length batch (the same attention; not on the pages, which
  * route per input, EA blog §2.1: every sequence is its own square causal

@@ -39,6 +39,8 @@ EXPORTED = [
     "ea_router_varlen_workspace_size", "ea_router_decide_varlen",
     "ea_hybrid_attn_routed_workspace_size", "ea_hybrid_attn_prefill_routed",
     "ea_hybrid_attn_varlen_routed_workspace_size", "ea_hybrid_attn_prefill_varlen_routed",
+    "ea_hybrid_attn_prefill_lse", "ea_hybrid_attn_backward_workspace_size",
+    "ea_hybrid_attn_backward",
 ]
 
 
@@ -137,6 +139,13 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_prefill_varlen_routed.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, vp,
                                                          ctypes.c_float, vp, vp, pvar, vp, vp,
                                                          c_size, vp]
+    lib.ea_hybrid_attn_prefill_lse.restype = c_int
+    lib.ea_hybrid_attn_prefill_lse.argtypes = [vp, vp, vp, vp, pparams, vp, vp, vp, c_size, vp]
+    lib.ea_hybrid_attn_backward_workspace_size.restype = c_size
+    lib.ea_hybrid_attn_backward_workspace_size.argtypes = [pparams]
+    lib.ea_hybrid_attn_backward.restype = c_int
+    lib.ea_hybrid_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, pparams, vp, vp, vp, vp,
+                                            c_size, vp]
     pdec = ctypes.POINTER(EaDecodeParams)
     lib.ea_decode_workspace_size.restype = c_size
     lib.ea_decode_workspace_size.argtypes = [pdec]

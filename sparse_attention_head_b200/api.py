@@ -338,6 +338,68 @@ def ea_hybrid_attn_prefill_varlen_routed(q: torch.Tensor, k: torch.Tensor, v: to
     return out, route_mask, logits
 
 
+# ---------------------------------------------------------------- training
+def ea_hybrid_attn_prefill_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                               route_mask: torch.Tensor, sink: int, window: int, *,
+                               softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                               lse: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None,
+                               stream: Optional[torch.cuda.Stream] = None):
+    """Forward for training: (out bf16 [B, Hq, N, d], lse fp32 [B, Hq, N])."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(lse, "lse", torch.float32, 3)
+    if workspace is None:
+        workspace = attn_workspace(p, q.device)
+    rc = lib.ea_hybrid_attn_prefill_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        route_mask.data_ptr(), ctypes.byref(p), out.data_ptr(),
+                                        lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                        _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill_lse")
+    return out, lse
+
+
+def ea_hybrid_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
+                            route_mask: torch.Tensor, sink: int, window: int, *,
+                            softmax_scale: float = 0.0, dq: Optional[torch.Tensor] = None,
+                            dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None):
+    """(dq, dk, dv) bf16 of L = sum(dout * out) for the hybrid attention."""
+    lib = _lib.load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        n = int(lib.ea_hybrid_attn_backward_workspace_size(ctypes.byref(p)))
+        if n == 0:
+            raise ValueError("unsupported backward parameters (d must be 128)")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    rc = lib.ea_hybrid_attn_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     dout.data_ptr(), lse.data_ptr(), route_mask.data_ptr(),
+                                     ctypes.byref(p), dq.data_ptr(), dk.data_ptr(),
+                                     dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                     _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_backward")
+    return dq, dk, dv
+
+
 def ea_get_device_status(workspace: torch.Tensor,
                          stream: Optional[torch.cuda.Stream] = None) -> int:
     lib = _lib.load()

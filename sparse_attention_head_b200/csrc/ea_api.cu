@@ -1,6 +1,7 @@
 // ea_api.cu — the C ABI of libea.so: argument checks, TMA descriptor
 // encoding and kernel launches.  See include/ea.h for the contract.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -357,6 +358,94 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   if (sms <= 0) return EA_ERR_CUDA;
   const int grid = ea_attn_grid_size(p, sms);
   cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v,
+                                     const uint8_t* route_mask, const ea_attn_params* p,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (!q || !k || !v || !route_mask || !out || !lse) return EA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  ea::AttnArgs args = {};
+  if (!encode_bhsd(&args.tm_q, q, p->d, p->N, p->B * p->Hq) ||
+      !encode_bhsd(&args.tm_k, k, p->d, p->N, p->B * p->Hkv) ||
+      !encode_bhsd(&args.tm_v, v, p->d, p->N, p->B * p->Hkv))
+    return EA_ERR_CUDA;
+  args.mask = route_mask;
+  args.out = out;
+  args.lse = lse;
+  args.status = static_cast<int*>(workspace);
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->N;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = debug_drop_kv_pos();
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  cudaError_t err = ea::launch_attn(p->d, args, ea_attn_grid_size(p, sms),
+                                    static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p) {
+  if (check_params(p) != EA_OK || p->d != 128) return 0;
+  const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
+  return kAttnWorkspace + (rows * sizeof(float) + 255) / 256 * 256;
+}
+
+ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                                  const void* dout, const float* lse, const uint8_t* route_mask,
+                                  const ea_attn_params* p, void* dq, void* dk, void* dv,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (p->d != 128 || p->select != EA_SELECT_ALL) return EA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !dout || !lse || !route_mask || !dq || !dk || !dv)
+    return EA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return EA_ERR_MISALIGNED;
+  const size_t need = ea_hybrid_attn_backward_workspace_size(p);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  ea::BwdArgs a = {};
+  if (!encode_bhsd(&a.tm_q, q, p->d, p->N, p->B * p->Hq) ||
+      !encode_bhsd(&a.tm_k, k, p->d, p->N, p->B * p->Hkv) ||
+      !encode_bhsd(&a.tm_v, v, p->d, p->N, p->B * p->Hkv) ||
+      !encode_bhsd(&a.tm_do, dout, p->d, p->N, p->B * p->Hq))
+    return EA_ERR_CUDA;
+  float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + kAttnWorkspace);
+  a.lse = lse;
+  a.dvec = dvec;
+  a.mask = route_mask;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.status = static_cast<int*>(workspace);
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.N = p->N;
+  a.sink = p->sink;
+  a.window = p->window;
+  a.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.timeout_ns = wait_timeout_ns();
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  cudaError_t err = ea::launch_backward(a, dout, out, dvec, sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

@@ -217,7 +217,6 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   int* s_counts = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // nFA, nSA
   uint16_t* s_ent = reinterpret_cast<uint16_t*>(smem + C::kOffEnt);
 
-  const int BH = args.B * args.Hq;
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -676,6 +675,8 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
+      if (args.lse != nullptr && !packed && row < seq_len)   // log-sum-exp for the backward
+        args.lse[static_cast<size_t>(idx) * args.N + row] = (m_ref + __log2f(l)) * 0.6931471805599453f;
       // out row: padded [B][Hq][N][d]; packed [T][Hq][d]
       const size_t orow_index =
           packed ? (static_cast<size_t>(s_tok[seq] + row) * args.Hq + idx % args.Hq)

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +23,7 @@ struct alignas(64) AttnArgs {
   // [cu_seqlens[b], cu_seqlens[b + 1]) of q [T][Hq][d], k, v [T][Hkv][d].
   const int32_t* cu_seqlens;
   int total;                // T, tokens of a packed batch
+  float* lse;               // optional [B][Hq][N]: natural log-sum-exp of each row (padded only)
   int B, Hq, Hkv, N;
   int sink, window;
   float scale_log2;         // softmax scale * log2(e)
@@ -47,6 +49,24 @@ struct alignas(64) AttnArgs {
   unsigned int* bar_count;  // grid barrier: arrivals of the current phase
   unsigned int* bar_gen;    //               and its generation
 };
+
+// Arguments of the tcgen05 backward kernels (padded BHSD, d = 128).
+struct BwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // (d, N, B*heads) boxes of 64 x 128 x 1
+  const float* lse;                      // [B][Hq][N] natural log-sum-exp
+  const float* dvec;                     // [B][Hq][N] rowsum(dO * O) (computed first)
+  const uint8_t* mask;                   // [B][Hq]
+  __nv_bfloat16* dq;                     // [B][Hq][N][d]
+  __nv_bfloat16* dk;                     // [B][Hkv][N][d]
+  __nv_bfloat16* dv;
+  int* status;
+  int B, Hq, Hkv, N, sink, window;
+  float scale, scale_log2;
+  unsigned long long timeout_ns;
+};
+// D = rowsum(dO * O) into dvec, then the dK/dV and dQ kernels.
+cudaError_t launch_backward(const BwdArgs& a, const void* dout, const void* out, float* dvec,
+                            int grid_sms, cudaStream_t stream);
 
 // SM count of the current device (cached per device); 0 on error.
 int device_sms();

@@ -37,7 +37,8 @@ def compare(out_gpu: torch.Tensor, ref: np.ndarray, label="", few_keys=False, fe
 
     few_keys: rows that see only a handful of keys (window <= 2) output values
     of the size of V itself, and rounding the output to bf16 alone moves a
-    value by up to 2^-9 |out| (more than 1e-2 once |out| >= 4).  For such
+    value by up to 2^-8 |out| (bf16 unit roundoff; 2^-9 on average), more
+    than 1e-2 once |out| >= 2.6.  For such
     cases the bound adds that rounding: |err| <= 1e-2 + 2^-8 |ref| element-
     wise and mean |err| <= 1e-3 + mean(2^-9 |ref|).  few_rows marks such rows
     individually (the first rows of every sequence of a packed batch); the

@@ -1,0 +1,80 @@
+"""GPU parity of the training path (through the C ABI) against the oracle:
+the forward's log-sum-exp and the backward's dQ, dK, dV for mixed FA/SA
+heads under GQA."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_common import f64
+from sparse_attention_head_b200 import build
+from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_backward,
+                                            ea_hybrid_attn_prefill_lse)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+
+
+# log-sum-exp: the forward's row sum adds bf16-rounded probabilities; bf16
+# keeps 8 significand bits, so each is off by at most 2^-8 of itself (unit
+# roundoff) and log(l) moves by at most -log(1 - 2^-8) = 3.91e-3.
+LSE_ABS = 4.0e-3
+# Gradients: P and dS enter the tensor cores as bf16 (relative 2^-8 each),
+# sums are fp32, results are rounded to bf16 (relative 2^-8).  dS mixes signs,
+# so the bound is normwise: max |err| <= 2^-6 max |ref| (4 unit roundoffs) and
+# mean |err| <= 2^-7 mean |ref|.
+GRAD_MAX_REL = 2.0 ** -6
+GRAD_MEAN_REL = 2.0 ** -7
+
+
+def _inputs(B, Hq, Hkv, N, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, Hq, N, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Hkv, N, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, N, d), generator=g).to(torch.bfloat16)
+    dout = torch.randn((B, Hq, N, d), generator=g).to(torch.bfloat16)
+    return q, k, v, dout
+
+
+def _grad_report(got, ref):
+    err = np.abs(f64(got) - ref)
+    return float(err.max()), float(err.mean()), float(np.abs(ref).max()), float(np.abs(ref).mean())
+
+
+CASES = [
+    # B, Hq, Hkv, N, S, W, mask
+    (1, 4, 2, 300, 16, 64, [[0, 1, 1, 0]]),
+    (2, 8, 2, 513, 4, 200, [[1, 1, 1, 1, 0, 0, 0, 0], [0, 1, 0, 1, 0, 1, 0, 1]]),
+    (1, 2, 2, 128, 0, 1, [[1, 0]]),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,S,W,mask", CASES)
+def test_backward_matches_oracle(B, Hq, Hkv, N, S, W, mask):
+    d = 128
+    q, k, v, dout = _inputs(B, Hq, Hkv, N, d, seed=N + Hq)
+    m = torch.as_tensor(np.array(mask, np.uint8), device=DEV)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    out, lse = ea_hybrid_attn_prefill_lse(qd, kd, vd, m, S, W)
+    ws = torch.zeros(1 << 22, dtype=torch.uint8, device=DEV)
+    dq, dk, dv = ea_hybrid_attn_backward(qd, kd, vd, out, dod, lse, m, S, W, workspace=ws)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    mn = np.array(mask, np.uint8)
+    ref_lse = oracle.attention_lse(f64(q), f64(k), mn, S, W)
+    assert np.abs(lse.cpu().double().numpy() - ref_lse).max() <= LSE_ABS
+    rq, rk, rv = oracle.attention_backward(f64(q), f64(k), f64(v), f64(dout), mn, S, W)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        mx, mean, rmax, rmean = _grad_report(got, ref)
+        print(name, mx, mean, rmax, rmean)
+        assert np.all(np.isfinite(f64(got))), name
+        assert mx <= GRAD_MAX_REL * rmax and mean <= GRAD_MEAN_REL * rmean, \
+            (name, mx, mean, rmax, rmean)
