@@ -64,6 +64,8 @@ def parse_args():
                     help="run only the decode measurement and print its JSON object")
     ap.add_argument("--packed-seqs", type=int, default=8,
                     help="sequences in the packed-batch measurement (0 skips it)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="run only the training-step (forward + backward) measurement")
     ap.add_argument("--packed-only", action="store_true",
                     help="run only the packed-batch measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
@@ -515,6 +517,74 @@ def measure_packed(w: workloads.Workload, nseq: int, steps: int, warmup: int, de
     }
 
 
+# ---------------------------------------------------------------- backward
+def measure_backward(w: workloads.Workload, steps: int, warmup: int, dev, stream):
+    """Training step of one layer's attention: the forward with log-sum-exp,
+    then the backward (D, dK/dV, dQ), timed separately with CUDA events.
+    Work: the forward's effective flops, and 2.5x that for the backward (five
+    products of the forward's size against its two)."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_backward,
+                                                ea_hybrid_attn_prefill_lse)
+    B, Hq, Hkv, N, d, S, W = w.batch, w.hq, w.hkv, w.seq, w.d, w.sink, w.window
+    seed = workloads.layer_seed(w, 0) + 9000
+    q, k, v = workloads.make_qkv(w, seed, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    mask = workloads.make_fixed_mask(dataclasses.replace(w, sparse_frac=workloads.layer_sparse_frac(w, 0)),
+                                     seed).to(dev)
+    ws = torch.zeros(1 << 26, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def fwd():
+        ea_hybrid_attn_prefill_lse(q, k, v, mask, S, W, out=out, lse=lse, workspace=ws[:256],
+                                   stream=stream)
+
+    def bwd():
+        ea_hybrid_attn_backward(q, k, v, out, dout, lse, mask, S, W, dq=dq, dk=dk, dv=dv,
+                                workspace=ws, stream=stream)
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    for _ in range(warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    f_ms = timed(fwd, steps)
+    b_ms = timed(bwd, steps)
+    if ea_get_device_status(ws) != 0:
+        raise RuntimeError("backward status word reports an error")
+    eff = flops.effective_flops(mask.cpu().numpy(), N, d, S, W)
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    btf = 2.5 * eff / (b_ms * 1e-3) / 1e12
+    return {
+        "workload": f"{w.name} training step of one layer: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} "
+                    f"S={S} W={W}, SA heads {mask.float().mean():.2f}",
+        "steps": steps, "warmup": warmup,
+        "forward_lse_ms": round(f_ms, 4),
+        "forward_tflops": round(eff / (f_ms * 1e-3) / 1e12, 2),
+        "backward_ms": round(b_ms, 4),
+        "backward_tflops": round(btf, 2),
+        "roofline": {"bound": "tensor", "achieved": round(btf, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(btf / peak, 4),
+                     "peak_source": f"{src} bf16_tflops (burst)",
+                     "scope": "backward (rowdot + dK/dV + dQ kernels), 2.5x effective "
+                              "forward flops"},
+        "gpu_launches_per_step": 3,
+    }
+
+
 # ---------------------------------------------------------------- decode
 def measure_decode(w: workloads.Workload, batch: int, steps: int, warmup: int, dev, stream):
     """One decode step per sequence of a ragged serving batch (positions in
@@ -717,6 +787,17 @@ def main():
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.backward_only:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = measure_backward(w, args.steps, max(args.warmup, 3), dev,
+                               torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
         return 0
     if args.packed_only:
         dev = torch.device("cuda", local_rank)

@@ -78,3 +78,24 @@ def test_backward_matches_oracle(B, Hq, Hkv, N, S, W, mask):
         assert np.all(np.isfinite(f64(got))), name
         assert mx <= GRAD_MAX_REL * rmax and mean <= GRAD_MEAN_REL * rmean, \
             (name, mx, mean, rmax, rmean)
+
+
+def test_backward_llama_layer_shape():
+    """llama8b layer shape (32 query heads, 8 kv heads, d 128) at N = 2048,
+    router-like mask with most heads SA and mixed GQA groups."""
+    B, Hq, Hkv, N, S, W, d = 1, 32, 8, 2048, 64, 1024, 128
+    q, k, v, dout = _inputs(B, Hq, Hkv, N, d, seed=2048)
+    rng = np.random.default_rng(3)
+    mn = (rng.random((B, Hq)) < 0.68).astype(np.uint8)
+    m = torch.as_tensor(mn, device=DEV)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    out, lse = ea_hybrid_attn_prefill_lse(qd, kd, vd, m, S, W)
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device=DEV)
+    dq, dk, dv = ea_hybrid_attn_backward(qd, kd, vd, out, dod, lse, m, S, W, workspace=ws)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    rq, rk, rv = oracle.attention_backward(f64(q), f64(k), f64(v), f64(dout), mn, S, W)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        mx, mean, rmax, rmean = _grad_report(got, ref)
+        assert mx <= GRAD_MAX_REL * rmax and mean <= GRAD_MEAN_REL * rmean, \
+            (name, mx, mean, rmax, rmean)
