@@ -131,6 +131,8 @@ __device__ __forceinline__ bool bwd_block_full(int it, int jt, int N, bool sa, i
 // ---------------------------------------------------------------- units
 // kDkDv: unit (b, kv head, key tile), key tile 0 (the most queries) first;
 // else unit (b, head, query tile), the last query tile (the most keys) first.
+// Units are dealt to CTAs in a snake (ea_rank_for), so a CTA that takes one
+// of the first, longest units takes one of the last, shortest ones next.
 template <bool kDkDv>
 __device__ __forceinline__ void bwd_unit_of(const BwdArgs& a, int u, int* b, int* hx, int* tile) {
   const int nT = ea_cdiv(a.N, EA_BN);
@@ -213,7 +215,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     // ============================================================ producer
     uint32_t pos = 0, nu = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
+         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
       int b, hx, tile;
       bwd_unit_of<kDkDv>(args, u, &b, &hx, &tile);
       if (nu > 0) {
@@ -311,7 +314,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
       const uint64_t d_stg_mn = smem_desc_sw128(stg, C::kBlockBytes, 1024);
       uint32_t pos = 0, nu = 0, nsteps = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
+         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
         if (!(ok = mbar_wait(b_res_full, nu & 1, s_abort, status, tlim, EA_ERR_TIMEOUT))) break;
         if (nu > 0 && !(ok = mbar_wait(b_acc_empty, (nu - 1) & 1, s_abort, status, tlim,
                                        EA_ERR_TIMEOUT)))
@@ -376,7 +380,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     const float sl2 = args.scale_log2;
     uint32_t pos = 0, nsteps = 0, nu = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
+         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
       int b, hx, tile;
       bwd_unit_of<kDkDv>(args, u, &b, &hx, &tile);
       const int row = tile * EA_BM + t;
@@ -403,37 +408,64 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         const uint32_t step_parity = nsteps & 1;
         ++nsteps;
         tc_fence_after();
-        uint32_t sr[64], dr[64];
-        tmem_ld64_wait(tmem + lane_off + col0, sr);
-        tmem_ld64_wait(tmem + lane_off + 128 + col0, dr);
-        mbar_arrive(b_ld_done);          // this warp's S and dP columns are in registers
         const float* vl = vec + slot * 256;
+        // visible columns of this row as ranges (branch-free per element):
+        // kDkDv (row = key k, column c = query q0 + c): c in [lo_a, hi_a];
+        // else (row = query q, column c = key k0 + c): c in [0, hi_a] and
+        // (c < sink_c or c >= win_c)
+        int lo_a = 0, hi_a = 127, sink_c = 1 << 20, win_c = -(1 << 20);
+        if (!st.full) {
+          const bool sa = st.sa != 0;
+          if (kDkDv) {
+            const int k = row, q0 = st.it * EA_BM;
+            lo_a = k - q0;                                   // q >= k
+            hi_a = args.N - 1 - q0;                          // q < N
+            if (k >= args.N) hi_a = -1;
+            if (sa && k >= args.sink) hi_a = min(hi_a, k + args.window - 1 - q0);   // q - k < W
+          } else {
+            const int q = row, k0 = st.jt * EA_BN;
+            hi_a = (q < args.N) ? q - k0 : -1;               // k <= q (< N)
+            if (sa) {
+              sink_c = args.sink - k0;                       // k < S
+              win_c = q - args.window + 1 - k0;              // q - k < W
+            }
+          }
+        }
         uint32_t pp[32], ds[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int ch = 0; ch < 2; ++ch) {
+        // 32 columns at a time: S (or S^T) and dP (or dP^T) into registers
+        uint32_t sr[32], dr[32];
+        tmem_ld32_wait(tmem + lane_off + col0 + 32 * ch, sr);
+        tmem_ld32_wait(tmem + lane_off + 128 + col0 + 32 * ch, dr);
+        if (ch == 1) mbar_arrive(b_ld_done);   // all of this warp's columns are read
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = 16 * ch + jj;
           const int c = col0 + 2 * j;
-          // per column (kDkDv: query) or per row (dQ) -lse2 and -D
-          const float nl0 = kDkDv ? vl[c] : nl_row, nl1 = kDkDv ? vl[c + 1] : nl_row;
-          const float nd0 = kDkDv ? vl[128 + c] : nd_row, nd1 = kDkDv ? vl[128 + c + 1] : nd_row;
-          float x0 = nl0, x1 = nl1;
-          fma2_acc(x0, x1, __uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]), sl2, sl2);
-          if (!st.full) {
-            const int kq = kDkDv ? row : st.it * EA_BM + t;          // query of the pair
-            const int kk0 = kDkDv ? st.jt * EA_BN + t : st.jt * EA_BN + c;
-            // kDkDv: row = key, columns = queries; else row = query, columns = keys
-            const int q0 = kDkDv ? st.it * EA_BM + c : kq, q1 = kDkDv ? q0 + 1 : kq;
-            const int k0 = kk0, k1 = kDkDv ? kk0 : kk0 + 1;
-            const bool sa = st.sa != 0;
-            if (!(k0 < args.N && bwd_visible(q0, k0, args.N, sa, args.sink, args.window)))
-              x0 = -INFINITY;
-            if (!(k1 < args.N && bwd_visible(q1, k1, args.N, sa, args.sink, args.window)))
-              x1 = -INFINITY;
+          float nl0, nl1, nd0, nd1;
+          if (kDkDv) {
+            const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
+            const float2 d2 = *reinterpret_cast<const float2*>(vl + 128 + c);
+            nl0 = l2.x; nl1 = l2.y; nd0 = d2.x; nd1 = d2.y;
+          } else {
+            nl0 = nl1 = nl_row;
+            nd0 = nd1 = nd_row;
           }
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          float x0 = nl0, x1 = nl1;
+          fma2_acc(x0, x1, __uint_as_float(sr[2 * jj]), __uint_as_float(sr[2 * jj + 1]), sl2, sl2);
+          const bool v0 = c >= lo_a && c <= hi_a && (c < sink_c || c >= win_c);
+          const bool v1 = c + 1 >= lo_a && c + 1 <= hi_a && (c + 1 < sink_c || c + 1 >= win_c);
+          x0 = v0 ? x0 : -INFINITY;
+          x1 = v1 ? x1 : -INFINITY;
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           float t0 = nd0, t1 = nd1;
-          add2_acc(t0, t1, __uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1]));
-          ds[j] = pack_bf16x2(p0 * t0, p1 * t1);
+          add2_acc(t0, t1, __uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1]));
+          float e0 = 0.f, e1 = 0.f;
+          fma2_acc(e0, e1, p0, p1, t0, t1);                 // dS = P (dP - D)
+          ds[j] = pack_bf16x2(e0, e1);
           if (kDkDv) pp[j] = pack_bf16x2(p0, p1);
+        }
         }
         // the other column half may still be reading the columns these
         // stores overwrite
