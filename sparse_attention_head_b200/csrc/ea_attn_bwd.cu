@@ -74,9 +74,9 @@ struct BwdCfg {
   static constexpr int kOffVec = kOffStage + kStages * 2 * kTileBytes;
   static constexpr int kOffStep = kOffVec + kStages * 2 * 128 * 4;   // step descriptors, 32 B each
   static constexpr int kOffBar = kOffStep + kStages * 32;
-  // res_full, res_empty, st_full[kStages], st_empty[kStages], s_full, ld_done, p_full,
-  // acc_done, acc_empty, drain
-  static constexpr int kNumBars = 2 + 2 * kStages + 6;
+  // res_full, res_empty, st_full[kStages], st_empty[kStages], s_full[2], ld_done,
+  // p_full[2], acc_done, acc_empty, drain (s_full / p_full: one per column half)
+  static constexpr int kNumBars = 2 + 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;    // tmem base, abort flag
   static constexpr int kSmem = kOffMisc + 64 + 1024;         // + alignment slack
   static constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);  // both K-major
@@ -172,10 +172,10 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
   const uint32_t bar0 = smem_u32(bar);
   const uint32_t b_res_full = bar0, b_res_empty = bar0 + 8;
   const uint32_t b_st_full = bar0 + 16, b_st_empty = bar0 + 16 + 8 * C::kStages;
-  const uint32_t b_s_full = bar0 + 16 + 16 * C::kStages;
-  const uint32_t b_ld_done = b_s_full + 8, b_p_full = b_s_full + 16;
-  const uint32_t b_acc_done = b_s_full + 24, b_acc_empty = b_s_full + 32;
-  const uint32_t b_drain = b_s_full + 40;
+  const uint32_t b_s_full = bar0 + 16 + 16 * C::kStages;     // [2]
+  const uint32_t b_ld_done = b_s_full + 16, b_p_full = b_s_full + 24;   // p_full [2]
+  const uint32_t b_acc_done = b_s_full + 40, b_acc_empty = b_s_full + 48;
+  const uint32_t b_drain = b_s_full + 56;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   BwdStep* steps = reinterpret_cast<BwdStep*>(smem + C::kOffStep);
@@ -193,12 +193,14 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
       mbar_init(bar + 2 + i, 1);                  // st_full: producer
       mbar_init(bar + 2 + C::kStages + i, 1);     // st_empty: MMA commit
     }
-    mbar_init(bar + 2 + 2 * C::kStages, 1);       // s_full: MMA commit
-    mbar_init(bar + 3 + 2 * C::kStages, 256);     // ld_done: elementwise threads
-    mbar_init(bar + 4 + 2 * C::kStages, 256);     // p_full: elementwise threads
-    mbar_init(bar + 5 + 2 * C::kStages, 1);       // acc_done: MMA commit
-    mbar_init(bar + 6 + 2 * C::kStages, 256);     // acc_empty: elementwise threads
-    mbar_init(bar + 7 + 2 * C::kStages, 1);       // drain: MMA commit
+    mbar_init(bar + 2 + 2 * C::kStages, 1);       // s_full[0]: MMA commit
+    mbar_init(bar + 3 + 2 * C::kStages, 1);       // s_full[1]: MMA commit
+    mbar_init(bar + 4 + 2 * C::kStages, 128);     // ld_done: column half 0
+    mbar_init(bar + 5 + 2 * C::kStages, 128);     // p_full[0]: column half 0
+    mbar_init(bar + 6 + 2 * C::kStages, 128);     // p_full[1]: column half 1
+    mbar_init(bar + 7 + 2 * C::kStages, 1);       // acc_done: MMA commit
+    mbar_init(bar + 8 + 2 * C::kStages, 256);     // acc_empty: elementwise threads
+    mbar_init(bar + 9 + 2 * C::kStages, 1);       // drain: MMA commit
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -331,6 +333,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
           last = steps[slot].last != 0;
           // scores: kDkDv S^T = K Q^T and dP^T = V dO^T; else S = Q K^T and
           // dP = dO V^T (resident tile 0 / 1 against streamed tile 0 / 1)
+          // (N = 128; splitting them into column halves doubles the MMA
+          // instructions this one thread issues and measured slower)
           const uint64_t s0 = d_stg_k + ((slot * 2 * C::kTileBytes) >> 4);
           const uint64_t s1 = s0 + (C::kTileBytes >> 4);
 #pragma unroll
@@ -341,24 +345,33 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
                    k > 0 ? 1u : 0u);
           }
           mma_commit(b_s_full);
-          if (!(ok = mbar_wait(b_p_full, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT)))
-            break;
-          ++nsteps;
-          tc_fence_after();
+          mma_commit(b_s_full + 8);
           const uint64_t m0 = d_stg_mn + ((slot * 2 * C::kTileBytes) >> 4);
           const uint64_t m1 = m0 + (C::kTileBytes >> 4);
+          // the accumulating products in two K halves (columns 0-63, 64-127
+          // of P / dS), each as soon as its elementwise half is done
 #pragma unroll
-          for (int k = 0; k < EA_BM / 16; ++k) {
-            const uint32_t acc = (!first || k > 0) ? 1u : 0u;
-            if (kDkDv) {
-              mma_ts(tmem + 256, tmem + k * 8, m1 + ((k * 2048) >> 4), C::kIdescTS, acc);  // dV += P^T dO
-              mma_ts(tmem + 384, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
-                     acc);                                                               // dK += dS^T Q
-            } else {
-              mma_ts(tmem + 256, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
-                     acc);                                                               // dQ += dS K
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            if (!(ok = mbar_wait(b_p_full + 8 * hf, nsteps & 1, s_abort, status, tlim,
+                                 EA_ERR_TIMEOUT)))
+              break;
+            tc_fence_after();
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+              const int k = 4 * hf + kq;
+              const uint32_t acc = (!first || k > 0) ? 1u : 0u;
+              if (kDkDv) {
+                mma_ts(tmem + 256, tmem + k * 8, m1 + ((k * 2048) >> 4), C::kIdescTS, acc);  // dV += P^T dO
+                mma_ts(tmem + 384, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
+                       acc);                                                               // dK += dS^T Q
+              } else {
+                mma_ts(tmem + 256, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
+                       acc);                                                               // dQ += dS K
+              }
             }
           }
+          if (!ok) break;
+          ++nsteps;
           first = false;
           mma_commit(b_st_empty + 8 * slot);
           ++pos;
@@ -402,7 +415,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         const BwdStep st = steps[slot];
         last = st.last != 0;
         ++pos;
-        ok = mbar_wait(b_s_full, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        ok = mbar_wait(b_s_full + 8 * half, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint32_t step_parity = nsteps & 1;
@@ -438,7 +451,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         uint32_t sr[32], dr[32];
         tmem_ld32_wait(tmem + lane_off + col0 + 32 * ch, sr);
         tmem_ld32_wait(tmem + lane_off + 128 + col0 + 32 * ch, dr);
-        if (ch == 1) mbar_arrive(b_ld_done);   // all of this warp's columns are read
+        if (ch == 1 && half == 0) mbar_arrive(b_ld_done);   // half 0's columns are read
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           const int j = 16 * ch + jj;
@@ -469,14 +482,17 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         }
         // the other column half may still be reading the columns these
         // stores overwrite
-        ok = mbar_wait(b_ld_done, step_parity, s_abort, status, tlim, EA_ERR_TIMEOUT);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
+        // (only half 1's stores land on columns half 0 reads)
+        if (half == 1) {
+          ok = mbar_wait(b_ld_done, step_parity, s_abort, status, tlim, EA_ERR_TIMEOUT);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
         if (kDkDv) tmem_st32(tmem + lane_off + col0 / 2, pp);
         tmem_st32(tmem + lane_off + 128 + col0 / 2, ds);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(b_p_full);
+        mbar_arrive(b_p_full + 8 * half);
       }
       if (!ok) break;
       // epilogue
