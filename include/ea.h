@@ -236,6 +236,59 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Router training (EA blog §2.1, training trick: the binary routing is made
+ * differentiable with Gumbel-Softmax and a straight-through estimator).
+ *
+ * Reading: the two-way Gumbel-Softmax over (FA, SA) with logits (0, z) and
+ * the caller's Gumbel noise g0 (FA), g1 (SA), device fp32 [B][Hq], gives
+ *   r_soft = sigmoid((z + g1 - g0) / tau),   r_hard = [z + g1 - g0 > 0];
+ * the forward runs r_hard (out = r_hard O_SA + (1 - r_hard) O_FA) and the
+ * backward takes the gradient of r_soft.  The noise is an input so that the
+ * caller owns the random stream (g = -log(-log U), U uniform in (0, 1)).
+ *
+ * ea_router_decide_gumbel: the router's pooling and MLP (bit-identical z to
+ * ea_router_decide), then route_mask = r_hard (device uint8 [B][Hq]);
+ * r_soft_out and logits_out (device fp32 [B][Hq]) are optional (NULL).
+ * workspace >= ea_router_gumbel_workspace_size(...), 16-byte aligned.
+ *
+ * ea_router_ste_backward: with dout, o_fa, o_sa device bf16 [B][Hq][N][d]
+ * (the layer output's gradient and both modes' outputs of every head),
+ *   dr[b,h]  = sum_{n,c} dout * (o_sa - o_fa)          (dL/dr_hard)
+ *   dz       = dr * r_soft (1 - r_soft) / tau
+ * then back through z = W2 ReLU(W1 x + b1) + b2 and the mean pooling:
+ *   dw2 [Hq][hidden], db2 [Hq], dw1 [hidden][Hkv*d], db1 [hidden] (device
+ *   fp32, written, summed over the batch); dr_out (device fp32 [B][Hq],
+ *   optional); dk_pool_out (device fp32 [B][Hkv*d], optional) = dx / N, the
+ *   gradient every key position of (b, kv head) receives through the pool;
+ *   dk_accum (device bf16 [B][Hkv][N][d], optional) gets dk_pool added in
+ *   place (the attention backward's dk plus the router's share).
+ * The forward is recomputed from k (no saved activations).  Gradients are
+ * summed in fp32 in a fixed order (bit-reproducible run to run).
+ * workspace >= ea_router_ste_backward_workspace_size(...), 16-byte aligned.
+ * Limits: those of ea_router_decide, B <= 1024, N <= 32767*256 (backward);
+ * tau finite and > 0 (else EA_ERR_INVALID_ARG).
+ * ---------------------------------------------------------------------- */
+size_t ea_router_gumbel_workspace_size(int B, int Hkv, int N, int d, int hidden, int Hq);
+
+ea_status ea_router_decide_gumbel(const void* k, int B, int Hkv, int N, int d,
+                                  const float* w1, const float* b1, int hidden,
+                                  const float* w2, const float* b2, int Hq,
+                                  const float* g0, const float* g1, float tau,
+                                  uint8_t* route_mask, float* r_soft_out, float* logits_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+size_t ea_router_ste_backward_workspace_size(int B, int Hkv, int N, int d, int hidden, int Hq);
+
+ea_status ea_router_ste_backward(const void* k, int B, int Hkv, int N, int d,
+                                 const float* w1, const float* b1, int hidden,
+                                 const float* w2, const float* b2, int Hq,
+                                 const float* g0, const float* g1, float tau,
+                                 const void* dout, const void* o_fa, const void* o_sa,
+                                 float* dr_out, float* dw1, float* db1, float* dw2, float* db2,
+                                 float* dk_pool_out, void* dk_accum, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Packed variable-length batch (the same attention; not on the pages, which
  * route per input, EA blog §2.1: every sequence is its own square causal
  * prefill).  Sequence b holds tokens [cu_seqlens[b], cu_seqlens[b+1]) of the

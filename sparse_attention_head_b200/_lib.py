@@ -40,7 +40,8 @@ EXPORTED = [
     "ea_hybrid_attn_routed_workspace_size", "ea_hybrid_attn_prefill_routed",
     "ea_hybrid_attn_varlen_routed_workspace_size", "ea_hybrid_attn_prefill_varlen_routed",
     "ea_hybrid_attn_prefill_lse", "ea_hybrid_attn_backward_workspace_size",
-    "ea_hybrid_attn_backward",
+    "ea_hybrid_attn_backward", "ea_router_gumbel_workspace_size", "ea_router_decide_gumbel",
+    "ea_router_ste_backward_workspace_size", "ea_router_ste_backward",
 ]
 
 
@@ -146,6 +147,17 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_backward.restype = c_int
     lib.ea_hybrid_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, pparams, vp, vp, vp, vp,
                                             c_size, vp]
+    for name in ("ea_router_gumbel_workspace_size", "ea_router_ste_backward_workspace_size"):
+        getattr(lib, name).restype = c_size
+        getattr(lib, name).argtypes = [c_int] * 6
+    lib.ea_router_decide_gumbel.restype = c_int
+    lib.ea_router_decide_gumbel.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp,
+                                            c_int, vp, vp, ctypes.c_float, vp, vp, vp, vp,
+                                            c_size, vp]
+    lib.ea_router_ste_backward.restype = c_int
+    lib.ea_router_ste_backward.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp,
+                                           c_int, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, vp, vp, c_size, vp]
     pdec = ctypes.POINTER(EaDecodeParams)
     lib.ea_decode_workspace_size.restype = c_size
     lib.ea_decode_workspace_size.argtypes = [pdec]

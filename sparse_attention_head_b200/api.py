@@ -400,6 +400,84 @@ def ea_hybrid_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return dq, dk, dv
 
 
+def _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau):
+    _need(k, "k", torch.bfloat16, 4)
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1),
+                        ("g0", g0, 2), ("g1", g1, 2)):
+        _need(t, name, torch.float32, nd)
+    B, Hkv, N, d = k.shape
+    hidden, Hq = _router_shapes(w1, b1, w2, b2, Hkv * d)
+    if tuple(g0.shape) != (B, Hq) or tuple(g1.shape) != (B, Hq):
+        raise ValueError("Gumbel noise must be [B, Hq]")
+    if not tau > 0.0:
+        raise ValueError("tau must be positive")
+    return B, Hkv, N, d, hidden, Hq
+
+
+def ea_router_decide_gumbel(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
+                            w2: torch.Tensor, b2: torch.Tensor, g0: torch.Tensor,
+                            g1: torch.Tensor, tau: float, *,
+                            workspace: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None):
+    """Training-time routing: (r_hard uint8 [B, Hq], r_soft fp32, logits fp32)."""
+    lib = _lib.load()
+    B, Hkv, N, d, hidden, Hq = _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau)
+    dev = k.device
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.ea_router_gumbel_workspace_size(
+            B, Hkv, N, d, hidden, Hq)), 16), dtype=torch.uint8, device=dev)
+    r_hard = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+    r_soft = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    rc = lib.ea_router_decide_gumbel(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(),
+                                     hidden, w2.data_ptr(), b2.data_ptr(), Hq, g0.data_ptr(),
+                                     g1.data_ptr(), float(tau), r_hard.data_ptr(),
+                                     r_soft.data_ptr(), logits.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel(), _stream_ptr(stream, dev))
+    check(rc, "ea_router_decide_gumbel")
+    return r_hard, r_soft, logits
+
+
+def ea_router_ste_backward(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
+                           w2: torch.Tensor, b2: torch.Tensor, g0: torch.Tensor,
+                           g1: torch.Tensor, tau: float, dout: torch.Tensor,
+                           o_fa: torch.Tensor, o_sa: torch.Tensor, *,
+                           dk_accum: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None):
+    """Router gradients through the straight-through estimator:
+    (dr [B, Hq], dw1, db1, dw2, db2, dk_pool [B, Hkv*d]) fp32; when dk_accum
+    (bf16 [B, Hkv, N, d]) is given, dk_pool is added to it in place."""
+    lib = _lib.load()
+    B, Hkv, N, d, hidden, Hq = _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau)
+    for name, t in (("dout", dout), ("o_fa", o_fa), ("o_sa", o_sa)):
+        _need(t, name, torch.bfloat16, 4)
+        if tuple(t.shape) != (B, Hq, N, d):
+            raise ValueError(f"{name} must be [B, Hq, N, d]")
+    if dk_accum is not None:
+        _need(dk_accum, "dk_accum", torch.bfloat16, 4)
+        if dk_accum.shape != k.shape:
+            raise ValueError("dk_accum must have the shape of k")
+    dev = k.device
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.ea_router_ste_backward_workspace_size(
+            B, Hkv, N, d, hidden, Hq)), 16), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dr = torch.empty((B, Hq), **f32)
+    dw1, db1 = torch.empty_like(w1), torch.empty_like(b1)
+    dw2, db2 = torch.empty_like(w2), torch.empty_like(b2)
+    dk_pool = torch.empty((B, Hkv * d), **f32)
+    rc = lib.ea_router_ste_backward(
+        k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(), hidden, w2.data_ptr(),
+        b2.data_ptr(), Hq, g0.data_ptr(), g1.data_ptr(), float(tau), dout.data_ptr(),
+        o_fa.data_ptr(), o_sa.data_ptr(), dr.data_ptr(), dw1.data_ptr(), db1.data_ptr(),
+        dw2.data_ptr(), db2.data_ptr(), dk_pool.data_ptr(),
+        dk_accum.data_ptr() if dk_accum is not None else None, workspace.data_ptr(),
+        workspace.numel(), _stream_ptr(stream, dev))
+    check(rc, "ea_router_ste_backward")
+    return dr, dw1, db1, dw2, db2, dk_pool
+
+
 def ea_get_device_status(workspace: torch.Tensor,
                          stream: Optional[torch.cuda.Stream] = None) -> int:
     lib = _lib.load()

@@ -309,6 +309,73 @@ ea_status ea_router_decide_varlen(const void* k, const int32_t* cu_seqlens, int 
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
+// Checks shared by the router training entry points (the router's own limits
+// plus the Gumbel noise and a positive temperature).
+static ea_status check_router_train(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                                    const float* b1, int hidden, const float* w2,
+                                    const float* b2, int Hq, const float* g0, const float* g1,
+                                    float tau) {
+  if (!k || !w1 || !b1 || !w2 || !b2 || !g0 || !g1) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || hidden <= 0 || Hq <= 0) return EA_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || tau == INFINITY) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024 || B > EA_MAX_SEQS)
+    return EA_ERR_UNSUPPORTED;
+  if (hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  return EA_OK;
+}
+
+size_t ea_router_gumbel_workspace_size(int B, int Hkv, int N, int d, int hidden, int Hq) {
+  if (B <= 0 || Hkv <= 0 || N <= 0 || hidden <= 0 || Hq <= 0 || (d != 64 && d != 128)) return 0;
+  return ea::router_gumbel_workspace_bytes(B, Hkv, N, d, hidden, Hq);
+}
+
+ea_status ea_router_decide_gumbel(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                                  const float* b1, int hidden, const float* w2, const float* b2,
+                                  int Hq, const float* g0, const float* g1, float tau,
+                                  uint8_t* route_mask, float* r_soft_out, float* logits_out,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!route_mask) return EA_ERR_INVALID_ARG;
+  const ea_status st = check_router_train(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau);
+  if (st != EA_OK) return st;
+  if (!workspace || workspace_bytes < ea_router_gumbel_workspace_size(B, Hkv, N, d, hidden, Hq))
+    return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  const cudaError_t err = ea::launch_router_gumbel(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq,
+                                                   g0, g1, tau, route_mask, r_soft_out,
+                                                   logits_out, workspace,
+                                                   static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+size_t ea_router_ste_backward_workspace_size(int B, int Hkv, int N, int d, int hidden, int Hq) {
+  if (B <= 0 || Hkv <= 0 || N <= 0 || hidden <= 0 || Hq <= 0 || (d != 64 && d != 128)) return 0;
+  return ea::router_ste_workspace_bytes(B, Hkv, N, d, hidden, Hq);
+}
+
+ea_status ea_router_ste_backward(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                                 const float* b1, int hidden, const float* w2, const float* b2,
+                                 int Hq, const float* g0, const float* g1, float tau,
+                                 const void* dout, const void* o_fa, const void* o_sa,
+                                 float* dr_out, float* dw1, float* db1, float* dw2, float* db2,
+                                 float* dk_pool_out, void* dk_accum, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!dout || !o_fa || !o_sa || !dw1 || !db1 || !dw2 || !db2) return EA_ERR_INVALID_ARG;
+  const ea_status st = check_router_train(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau);
+  if (st != EA_OK) return st;
+  if (N > kMaxSeqLen) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(dout) || !aligned16(o_fa) || !aligned16(o_sa)) return EA_ERR_MISALIGNED;
+  if (!workspace ||
+      workspace_bytes < ea_router_ste_backward_workspace_size(B, Hkv, N, d, hidden, Hq))
+    return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  const cudaError_t err = ea::launch_router_ste(
+      k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau, dout, o_fa, o_sa, dr_out, dw1, db1,
+      dw2, db2, dk_pool_out, dk_accum, workspace, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ attention
 size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p) {
   return check_params(p) == EA_OK ? kAttnWorkspace : 0;

@@ -92,4 +92,20 @@ cudaError_t launch_router(const void* k, const int32_t* cu, int B, int Hkv, int 
                           const float* b2, int Hq, float threshold, uint8_t* mask, float* logits,
                           float* partials, int nsplit, cudaStream_t stream);
 
+// Router training: the Gumbel-Softmax decision and the straight-through
+// gradients.  Workspace layouts are fixed by the *_workspace_bytes sizes.
+size_t router_gumbel_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int Hq);
+cudaError_t launch_router_gumbel(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                                 const float* b1, int hidden, const float* w2, const float* b2,
+                                 int Hq, const float* g0, const float* g1, float tau,
+                                 uint8_t* route_mask, float* r_soft, float* logits_out,
+                                 void* workspace, cudaStream_t s);
+size_t router_ste_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int Hq);
+cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                              const float* b1, int hidden, const float* w2, const float* b2,
+                              int Hq, const float* g0, const float* g1, float tau,
+                              const void* dout, const void* o_fa, const void* o_sa, float* dr_out,
+                              float* dw1, float* db1, float* dw2, float* db2, float* dk_pool_out,
+                              void* dk_accum, void* workspace, cudaStream_t s);
+
 }  // namespace ea

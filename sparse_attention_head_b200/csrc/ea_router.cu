@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <math.h>
 #include <mutex>
 
 #include "ea.h"
@@ -71,6 +72,146 @@ __global__ void __launch_bounds__(kMlpThreads) ea_router_layer_kernel(
       y[static_cast<size_t>(b) * out_dim + o] = fmaxf(v, 0.f);
     }
   }
+}
+
+// ---------------------------------------------------------------- training
+// Gumbel-Softmax straight-through routing (EA blog §2.1, training trick),
+// with the caller's Gumbel noise g0, g1 [B][Hq] and temperature tau:
+//   r_soft = sigmoid((z + g1 - g0) / tau), r_hard = [z + g1 - g0 > 0].
+__global__ void ea_ste_gumbel_kernel(const float* __restrict__ z, const float* __restrict__ g0,
+                                     const float* __restrict__ g1, float tau, int n,
+                                     uint8_t* __restrict__ r_hard, float* __restrict__ r_soft) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float u = z[i] + g1[i] - g0[i];
+  if (r_hard) r_hard[i] = u > 0.f ? 1 : 0;
+  if (r_soft) r_soft[i] = 1.f / (1.f + expf(-u / tau));
+}
+
+// dr partials: CTA (b*Hq + h, split) sums dO * (O_SA - O_FA) over its rows.
+constexpr int kDrThreads = 256;
+__global__ void __launch_bounds__(kDrThreads) ea_ste_dr_kernel(
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o_fa,
+    const __nv_bfloat16* __restrict__ o_sa, int N, int d, int nsplit, float* __restrict__ part) {
+  __shared__ float red[kDrThreads / 32];
+  const int bh = blockIdx.x, split = blockIdx.y;
+  const size_t len = static_cast<size_t>(N) * d;
+  const size_t chunk = (len / 8 + nsplit - 1) / nsplit * 8;   // whole 8-element groups
+  const size_t e0 = split * chunk, e1 = min(len, e0 + chunk);
+  const size_t base = static_cast<size_t>(bh) * len;
+  float acc = 0.f;
+  for (size_t e = e0 + threadIdx.x * 8; e < e1; e += kDrThreads * 8) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + base + e));
+    const uint4 f = __ldg(reinterpret_cast<const uint4*>(o_fa + base + e));
+    const uint4 sx = __ldg(reinterpret_cast<const uint4*>(o_sa + base + e));
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* f2 = reinterpret_cast<const __nv_bfloat162*>(&f);
+    const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sx);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 av = __bfloat1622float2(a2[j]), fv = __bfloat1622float2(f2[j]),
+                   sv = __bfloat1622float2(s2[j]);
+      acc = fmaf(av.x, sv.x - fv.x, acc);
+      acc = fmaf(av.y, sv.y - fv.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kDrThreads / 32; ++w) t += red[w];
+    part[static_cast<size_t>(bh) * nsplit + split] = t;
+  }
+}
+
+// dr (summed in split order) and dz = dr * r (1 - r) / tau per (b, h).
+__global__ void ea_ste_dz_kernel(const float* __restrict__ part, int nsplit,
+                                 const float* __restrict__ z, const float* __restrict__ g0,
+                                 const float* __restrict__ g1, float tau, int n,
+                                 float* __restrict__ dr, float* __restrict__ dz) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float t = 0.f;
+  for (int s = 0; s < nsplit; ++s) t += part[static_cast<size_t>(i) * nsplit + s];
+  const float r = 1.f / (1.f + expf(-(z[i] + g1[i] - g0[i]) / tau));
+  if (dr) dr[i] = t;
+  dz[i] = t * r * (1.f - r) / tau;
+}
+
+// dW2[o][j] = sum_b dz[b][o] h[b][j] (j < hidden); db2[o] = sum_b dz[b][o] (j == hidden).
+__global__ void ea_ste_w2_kernel(const float* __restrict__ dz, const float* __restrict__ h, int B,
+                                 int Hq, int hidden, float* __restrict__ dw2,
+                                 float* __restrict__ db2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= Hq * (hidden + 1)) return;
+  const int o = i / (hidden + 1), j = i % (hidden + 1);
+  float t = 0.f;
+  for (int b = 0; b < B; ++b)
+    t = fmaf(dz[b * Hq + o], j < hidden ? h[static_cast<size_t>(b) * hidden + j] : 1.f, t);
+  if (j < hidden) dw2[static_cast<size_t>(o) * hidden + j] = t;
+  else db2[o] = t;
+}
+
+// dpre[b][j] = [h > 0] * sum_o dz[b][o] W2[o][j]  (h = ReLU(pre): h > 0 iff pre > 0).
+__global__ void ea_ste_dpre_kernel(const float* __restrict__ dz, const float* __restrict__ w2,
+                                   const float* __restrict__ h, int B, int Hq, int hidden,
+                                   float* __restrict__ dpre) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * hidden) return;
+  const int b = i / hidden, j = i % hidden;
+  float t = 0.f;
+  for (int o = 0; o < Hq; ++o) t = fmaf(dz[b * Hq + o], w2[static_cast<size_t>(o) * hidden + j], t);
+  dpre[i] = h[i] > 0.f ? t : 0.f;
+}
+
+// dW1[j][c] = sum_b dpre[b][j] x[b][c] (c < in_dim); db1[j] = sum_b dpre[b][j] (c == in_dim).
+__global__ void ea_ste_w1_kernel(const float* __restrict__ dpre, const float* __restrict__ x,
+                                 int B, int hidden, int in_dim, float* __restrict__ dw1,
+                                 float* __restrict__ db1) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<size_t>(hidden) * (in_dim + 1)) return;
+  const int j = static_cast<int>(i / (in_dim + 1)), c = static_cast<int>(i % (in_dim + 1));
+  float t = 0.f;
+  for (int b = 0; b < B; ++b)
+    t = fmaf(dpre[static_cast<size_t>(b) * hidden + j],
+             c < in_dim ? x[static_cast<size_t>(b) * in_dim + c] : 1.f, t);
+  if (c < in_dim) dw1[static_cast<size_t>(j) * in_dim + c] = t;
+  else db1[j] = t;
+}
+
+// dk_pool[b][c] = (sum_j dpre[b][j] W1[j][c]) / N: the keys' gradient through
+// the mean pooling, the same at every position of (b, c's kv head).
+__global__ void ea_ste_dx_kernel(const float* __restrict__ dpre, const float* __restrict__ w1,
+                                 int B, int hidden, int in_dim, int N,
+                                 float* __restrict__ dk_pool) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * in_dim) return;
+  const int b = i / in_dim, c = i % in_dim;
+  float t = 0.f;
+  for (int j = 0; j < hidden; ++j)
+    t = fmaf(dpre[static_cast<size_t>(b) * hidden + j], w1[static_cast<size_t>(j) * in_dim + c], t);
+  dk_pool[i] = t / static_cast<float>(N);
+}
+
+// dk[b][hk][n][c] += dk_pool[b][hk * d + c] for every position n (bf16 in place).
+__global__ void ea_ste_dk_add_kernel(const float* __restrict__ dk_pool, int B, int Hkv, int N,
+                                     int d, __nv_bfloat16* __restrict__ dk) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t total = static_cast<size_t>(B) * Hkv * N * d;
+  if (i >= total) return;
+  const int c = static_cast<int>(i % d);
+  const size_t row = i / d;                       // (b * Hkv + hk) * N + n
+  const size_t bh = row / N;                      // b * Hkv + hk
+  const int b = static_cast<int>(bh / Hkv), hk = static_cast<int>(bh % Hkv);
+  const float add = dk_pool[static_cast<size_t>(b) * Hkv * d + hk * d + c];
+  dk[i] = __float2bfloat16_rn(__bfloat162float(dk[i]) + add);
+}
+
+int ste_dr_splits(int B, int Hq) {
+  int per = (592 + B * Hq - 1) / (B * Hq);
+  return per < 1 ? 1 : (per > 64 ? 64 : per);
 }
 
 int router_num_splits(int B, int Hkv, int N) {
@@ -168,3 +309,94 @@ extern "C" ea_status ea_router_decide_noalloc(const void* k, int B, int Hkv, int
   return ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold, route_mask,
                           logits_out, scratch, EA_ROUTER_NOALLOC_MAX_BYTES, stream);
 }
+
+// ---------------------------------------------------------------------------
+// Training launches (Gumbel-Softmax straight-through routing, EA blog §2.1).
+namespace ea {
+namespace {
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+}  // namespace
+
+size_t router_gumbel_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int Hq) {
+  return align256(router_workspace_bytes(B, Hkv, N, d, hidden)) +
+         align256(static_cast<size_t>(B) * Hq * 4) + align256(static_cast<size_t>(B) * Hq);
+}
+
+cudaError_t launch_router_gumbel(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                                 const float* b1, int hidden, const float* w2, const float* b2,
+                                 int Hq, const float* g0, const float* g1, float tau,
+                                 uint8_t* route_mask, float* r_soft, float* logits_out,
+                                 void* workspace, cudaStream_t s) {
+  char* ws = static_cast<char*>(workspace);
+  const size_t n = static_cast<size_t>(B) * Hq;
+  size_t off = align256(router_workspace_bytes(B, Hkv, N, d, hidden));
+  float* z = logits_out ? logits_out : reinterpret_cast<float*>(ws + off);
+  off += align256(n * 4);
+  uint8_t* scratch_mask = reinterpret_cast<uint8_t*>(ws + off);
+  cudaError_t err = launch_router(k, nullptr, B, Hkv, N, 0, d, w1, b1, hidden, w2, b2, Hq, 0.f,
+                                  scratch_mask, z, reinterpret_cast<float*>(ws),
+                                  router_num_splits(B, Hkv, N), s);
+  if (err != cudaSuccess) return err;
+  ea_ste_gumbel_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      z, g0, g1, tau, static_cast<int>(n), route_mask, r_soft);
+  return cudaGetLastError();
+}
+
+size_t router_ste_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int Hq) {
+  const size_t n = static_cast<size_t>(B) * Hq;
+  return align256(router_workspace_bytes(B, Hkv, N, d, hidden)) +  // partials, x, h
+         align256(n * 4) +                                          // z
+         align256(n) +                                              // mask (unused)
+         align256(n * ste_dr_splits(B, Hq) * 4) +                   // dr partials
+         align256(n * 4) +                                          // dz
+         align256(static_cast<size_t>(B) * hidden * 4) +            // dpre
+         align256(static_cast<size_t>(B) * Hkv * d * 4);            // dk_pool
+}
+
+cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                              const float* b1, int hidden, const float* w2, const float* b2,
+                              int Hq, const float* g0, const float* g1, float tau,
+                              const void* dout, const void* o_fa, const void* o_sa, float* dr_out,
+                              float* dw1, float* db1, float* dw2, float* db2, float* dk_pool_out,
+                              void* dk_accum, void* workspace, cudaStream_t s) {
+  const size_t n = static_cast<size_t>(B) * Hq;
+  const int nsd = ste_dr_splits(B, Hq);
+  const int ns = router_num_splits(B, Hkv, N);
+  const int in_dim = Hkv * d;
+  char* ws = static_cast<char*>(workspace);
+  float* partials = reinterpret_cast<float*>(ws);
+  const float* x = partials + static_cast<size_t>(B) * Hkv * ns * d;
+  const float* h = x + static_cast<size_t>(B) * in_dim;
+  size_t off = align256(router_workspace_bytes(B, Hkv, N, d, hidden));
+  float* z = reinterpret_cast<float*>(ws + off);       off += align256(n * 4);
+  uint8_t* mask = reinterpret_cast<uint8_t*>(ws + off); off += align256(n);
+  float* drp = reinterpret_cast<float*>(ws + off);     off += align256(n * nsd * 4);
+  float* dz = reinterpret_cast<float*>(ws + off);      off += align256(n * 4);
+  float* dpre = reinterpret_cast<float*>(ws + off);
+  off += align256(static_cast<size_t>(B) * hidden * 4);
+  float* dkp = dk_pool_out ? dk_pool_out : reinterpret_cast<float*>(ws + off);
+  // forward recompute: x, h and z exactly as the router computes them
+  cudaError_t err = launch_router(k, nullptr, B, Hkv, N, 0, d, w1, b1, hidden, w2, b2, Hq, 0.f,
+                                  mask, z, partials, ns, s);
+  if (err != cudaSuccess) return err;
+  ea_ste_dr_kernel<<<dim3(static_cast<unsigned>(n), nsd), kDrThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o_fa),
+      static_cast<const __nv_bfloat16*>(o_sa), N, d, nsd, drp);
+  ea_ste_dz_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      drp, nsd, z, g0, g1, tau, static_cast<int>(n), dr_out, dz);
+  ea_ste_w2_kernel<<<(Hq * (hidden + 1) + 255) / 256, 256, 0, s>>>(dz, h, B, Hq, hidden, dw2,
+                                                                   db2);
+  ea_ste_dpre_kernel<<<(B * hidden + 255) / 256, 256, 0, s>>>(dz, w2, h, B, Hq, hidden, dpre);
+  const size_t nw1 = static_cast<size_t>(hidden) * (in_dim + 1);
+  ea_ste_w1_kernel<<<static_cast<unsigned>((nw1 + 255) / 256), 256, 0, s>>>(dpre, x, B, hidden,
+                                                                            in_dim, dw1, db1);
+  ea_ste_dx_kernel<<<(B * in_dim + 255) / 256, 256, 0, s>>>(dpre, w1, B, hidden, in_dim, N, dkp);
+  if (dk_accum) {
+    const size_t tot = static_cast<size_t>(B) * Hkv * N * d;
+    ea_ste_dk_add_kernel<<<static_cast<unsigned>((tot + 255) / 256), 256, 0, s>>>(
+        dkp, B, Hkv, N, d, static_cast<__nv_bfloat16*>(dk_accum));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ea

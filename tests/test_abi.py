@@ -114,6 +114,40 @@ def test_router_argument_errors(lib):
     assert call(wsb=8) == _lib.EA_ERR_WORKSPACE
 
 
+def test_router_training_argument_errors(lib):
+    ws_need = lib.ea_router_ste_backward_workspace_size(2, 8, 64, 128, 256, 32)
+    assert ws_need > 0 and lib.ea_router_ste_backward_workspace_size(2, 8, 64, 96, 256, 32) == 0
+    assert lib.ea_router_gumbel_workspace_size(2, 8, 64, 128, 256, 32) > 0
+
+    def ste(k=16, B=2, Hkv=8, N=64, d=128, hidden=256, Hq=32, g0=16, tau=1.0, dout=16, dw1=16,
+            ws=256, wsb=ws_need):
+        return lib.ea_router_ste_backward(k, B, Hkv, N, d, 16, 16, hidden, 16, 16, Hq, g0, 16, tau,
+                                          dout, 16, 16, None, dw1, 16, 16, 16, None, None, ws,
+                                          wsb, None)
+    assert ste(k=0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(g0=0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(dout=0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(dw1=0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(tau=0.0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(tau=float("nan")) == _lib.EA_ERR_INVALID_ARG
+    assert ste(tau=float("inf")) == _lib.EA_ERR_INVALID_ARG
+    assert ste(B=0) == _lib.EA_ERR_INVALID_ARG
+    assert ste(d=96) == _lib.EA_ERR_UNSUPPORTED
+    assert ste(hidden=254) == _lib.EA_ERR_UNSUPPORTED
+    assert ste(B=1025) == _lib.EA_ERR_UNSUPPORTED
+    assert ste(k=24) == _lib.EA_ERR_MISALIGNED
+    assert ste(dout=24) == _lib.EA_ERR_MISALIGNED
+    assert ste(ws=0) == _lib.EA_ERR_WORKSPACE
+    assert ste(wsb=ws_need - 1) == _lib.EA_ERR_WORKSPACE
+
+    def gumbel(mask=16, tau=1.0, wsb=1 << 20):
+        return lib.ea_router_decide_gumbel(16, 2, 8, 64, 128, 16, 16, 256, 16, 16, 32, 16, 16, tau,
+                                           mask, None, None, 256, wsb, None)
+    assert gumbel(mask=0) == _lib.EA_ERR_INVALID_ARG
+    assert gumbel(tau=-1.0) == _lib.EA_ERR_INVALID_ARG
+    assert gumbel(wsb=8) == _lib.EA_ERR_WORKSPACE
+
+
 def test_grid_size(lib):
     p = make_params(1, 4, 2, 512, 64, 16, 128)
     assert lib.ea_attn_grid_size(ctypes.byref(p), 148) == 8      # 4 heads x 2 units
