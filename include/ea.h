@@ -211,6 +211,18 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
                                      void* out, float* lse, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* Forward of a training step: every head in BOTH modes, in one launch.  The
+ * mode route_mask chooses goes to out, with its log-sum-exp in lse (as
+ * ea_hybrid_attn_prefill_lse); the other mode to out_other (device bf16
+ * [B][Hq][N][d]).  The straight-through router gradient needs both
+ * (ea_router_ste_backward); only the chosen mode receives an attention
+ * gradient, since the hard route is 0 or 1.  Requires p->select ==
+ * EA_SELECT_ALL and 2*B*Hq <= 4096. */
+ea_status ea_hybrid_attn_prefill_train(const void* q, const void* k, const void* v,
+                                       const uint8_t* route_mask, const ea_attn_params* p,
+                                       void* out, float* lse, void* out_other, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Backward pass (training; EA blog §2.1: the router is trained through a
  * Gumbel-Softmax straight-through estimator, so the attention of each head's
@@ -251,9 +263,12 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
  * r_soft_out and logits_out (device fp32 [B][Hq]) are optional (NULL).
  * workspace >= ea_router_gumbel_workspace_size(...), 16-byte aligned.
  *
- * ea_router_ste_backward: with dout, o_fa, o_sa device bf16 [B][Hq][N][d]
- * (the layer output's gradient and both modes' outputs of every head),
- *   dr[b,h]  = sum_{n,c} dout * (o_sa - o_fa)          (dL/dr_hard)
+ * ea_router_ste_backward: dout, out, out_other device bf16 [B][Hq][N][d]:
+ * the layer output's gradient, each head's output in the mode route_mask
+ * chose and in its other mode (as ea_hybrid_attn_prefill_train writes them);
+ * route_mask == NULL reads as every head having chosen FA, so that out and
+ * out_other are then O_FA and O_SA.  With O_SA - O_FA taken from them,
+ *   dr[b,h]  = sum_{n,c} dout * (O_SA - O_FA)          (dL/dr_hard)
  *   dz       = dr * r_soft (1 - r_soft) / tau
  * then back through z = W2 ReLU(W1 x + b1) + b2 and the mean pooling:
  *   dw2 [Hq][hidden], db2 [Hq], dw1 [hidden][Hkv*d], db1 [hidden] (device
@@ -283,10 +298,11 @@ ea_status ea_router_ste_backward(const void* k, int B, int Hkv, int N, int d,
                                  const float* w1, const float* b1, int hidden,
                                  const float* w2, const float* b2, int Hq,
                                  const float* g0, const float* g1, float tau,
-                                 const void* dout, const void* o_fa, const void* o_sa,
-                                 float* dr_out, float* dw1, float* db1, float* dw2, float* db2,
-                                 float* dk_pool_out, void* dk_accum, void* workspace,
-                                 size_t workspace_bytes, void* stream);
+                                 const void* dout, const void* out, const void* out_other,
+                                 const uint8_t* route_mask, float* dr_out, float* dw1,
+                                 float* db1, float* dw2, float* db2, float* dk_pool_out,
+                                 void* dk_accum, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* ------------------------------------------------------------------------
  * Packed variable-length batch (the same attention; not on the pages, which

@@ -42,6 +42,7 @@ EXPORTED = [
     "ea_hybrid_attn_prefill_lse", "ea_hybrid_attn_backward_workspace_size",
     "ea_hybrid_attn_backward", "ea_router_gumbel_workspace_size", "ea_router_decide_gumbel",
     "ea_router_ste_backward_workspace_size", "ea_router_ste_backward",
+    "ea_hybrid_attn_prefill_train",
 ]
 
 
@@ -142,6 +143,9 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
                                                          c_size, vp]
     lib.ea_hybrid_attn_prefill_lse.restype = c_int
     lib.ea_hybrid_attn_prefill_lse.argtypes = [vp, vp, vp, vp, pparams, vp, vp, vp, c_size, vp]
+    lib.ea_hybrid_attn_prefill_train.restype = c_int
+    lib.ea_hybrid_attn_prefill_train.argtypes = [vp, vp, vp, vp, pparams, vp, vp, vp, vp, c_size,
+                                                 vp]
     lib.ea_hybrid_attn_backward_workspace_size.restype = c_size
     lib.ea_hybrid_attn_backward_workspace_size.argtypes = [pparams]
     lib.ea_hybrid_attn_backward.restype = c_int
@@ -157,7 +161,7 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_router_ste_backward.restype = c_int
     lib.ea_router_ste_backward.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp,
                                            c_int, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp,
-                                           vp, vp, vp, vp, vp, c_size, vp]
+                                           vp, vp, vp, vp, vp, vp, c_size, vp]
     pdec = ctypes.POINTER(EaDecodeParams)
     lib.ea_decode_workspace_size.restype = c_size
     lib.ea_decode_workspace_size.argtypes = [pdec]

@@ -367,6 +367,36 @@ def ea_hybrid_attn_prefill_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
     return out, lse
 
 
+def ea_hybrid_attn_prefill_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                 route_mask: torch.Tensor, sink: int, window: int, *,
+                                 softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                 lse: Optional[torch.Tensor] = None,
+                                 out_other: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None):
+    """Training forward, both modes in one launch: (out [chosen mode], lse
+    fp32 [B, Hq, N], out_other [the other mode])."""
+    lib = _lib.load()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q.shape
+    p = make_params(B, Hq, k.shape[1], N, d, sink, window, softmax_scale)
+    out = torch.empty_like(q) if out is None else out
+    out_other = torch.empty_like(q) if out_other is None else out_other
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = attn_workspace(p, q.device)
+    rc = lib.ea_hybrid_attn_prefill_train(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          route_mask.data_ptr(), ctypes.byref(p), out.data_ptr(),
+                                          lse.data_ptr(), out_other.data_ptr(),
+                                          workspace.data_ptr(), workspace.numel(),
+                                          _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill_train")
+    return out, lse, out_other
+
+
 def ea_hybrid_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                             out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
                             route_mask: torch.Tensor, sink: int, window: int, *,
@@ -441,19 +471,23 @@ def ea_router_decide_gumbel(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
 def ea_router_ste_backward(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
                            w2: torch.Tensor, b2: torch.Tensor, g0: torch.Tensor,
                            g1: torch.Tensor, tau: float, dout: torch.Tensor,
-                           o_fa: torch.Tensor, o_sa: torch.Tensor, *,
+                           out: torch.Tensor, out_other: torch.Tensor,
+                           route_mask: Optional[torch.Tensor] = None, *,
                            dk_accum: Optional[torch.Tensor] = None,
                            workspace: Optional[torch.Tensor] = None,
                            stream: Optional[torch.cuda.Stream] = None):
     """Router gradients through the straight-through estimator:
     (dr [B, Hq], dw1, db1, dw2, db2, dk_pool [B, Hkv*d]) fp32; when dk_accum
-    (bf16 [B, Hkv, N, d]) is given, dk_pool is added to it in place."""
+    (bf16 [B, Hkv, N, d]) is given, dk_pool is added to it in place.  out /
+    out_other: each head's chosen / other mode (route_mask None: O_FA / O_SA)."""
     lib = _lib.load()
     B, Hkv, N, d, hidden, Hq = _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau)
-    for name, t in (("dout", dout), ("o_fa", o_fa), ("o_sa", o_sa)):
+    for name, t in (("dout", dout), ("out", out), ("out_other", out_other)):
         _need(t, name, torch.bfloat16, 4)
         if tuple(t.shape) != (B, Hq, N, d):
             raise ValueError(f"{name} must be [B, Hq, N, d]")
+    if route_mask is not None:
+        _need(route_mask, "route_mask", torch.uint8, 2)
     if dk_accum is not None:
         _need(dk_accum, "dk_accum", torch.bfloat16, 4)
         if dk_accum.shape != k.shape:
@@ -470,7 +504,9 @@ def ea_router_ste_backward(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
     rc = lib.ea_router_ste_backward(
         k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(), hidden, w2.data_ptr(),
         b2.data_ptr(), Hq, g0.data_ptr(), g1.data_ptr(), float(tau), dout.data_ptr(),
-        o_fa.data_ptr(), o_sa.data_ptr(), dr.data_ptr(), dw1.data_ptr(), db1.data_ptr(),
+        out.data_ptr(), out_other.data_ptr(),
+        route_mask.data_ptr() if route_mask is not None else None, dr.data_ptr(), dw1.data_ptr(),
+        db1.data_ptr(),
         dw2.data_ptr(), db2.data_ptr(), dk_pool.data_ptr(),
         dk_accum.data_ptr() if dk_accum is not None else None, workspace.data_ptr(),
         workspace.numel(), _stream_ptr(stream, dev))

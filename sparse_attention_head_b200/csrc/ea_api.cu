@@ -357,22 +357,24 @@ size_t ea_router_ste_backward_workspace_size(int B, int Hkv, int N, int d, int h
 ea_status ea_router_ste_backward(const void* k, int B, int Hkv, int N, int d, const float* w1,
                                  const float* b1, int hidden, const float* w2, const float* b2,
                                  int Hq, const float* g0, const float* g1, float tau,
-                                 const void* dout, const void* o_fa, const void* o_sa,
-                                 float* dr_out, float* dw1, float* db1, float* dw2, float* db2,
+                                 const void* dout, const void* out, const void* out_other,
+                                 const uint8_t* route_mask, float* dr_out, float* dw1,
+                                 float* db1, float* dw2, float* db2,
                                  float* dk_pool_out, void* dk_accum, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  if (!dout || !o_fa || !o_sa || !dw1 || !db1 || !dw2 || !db2) return EA_ERR_INVALID_ARG;
+  if (!dout || !out || !out_other || !dw1 || !db1 || !dw2 || !db2) return EA_ERR_INVALID_ARG;
   const ea_status st = check_router_train(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau);
   if (st != EA_OK) return st;
   if (N > kMaxSeqLen) return EA_ERR_UNSUPPORTED;
-  if (!aligned16(dout) || !aligned16(o_fa) || !aligned16(o_sa)) return EA_ERR_MISALIGNED;
+  if (!aligned16(dout) || !aligned16(out) || !aligned16(out_other)) return EA_ERR_MISALIGNED;
   if (!workspace ||
       workspace_bytes < ea_router_ste_backward_workspace_size(B, Hkv, N, d, hidden, Hq))
     return EA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
   const cudaError_t err = ea::launch_router_ste(
-      k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau, dout, o_fa, o_sa, dr_out, dw1, db1,
-      dw2, db2, dk_pool_out, dk_accum, workspace, static_cast<cudaStream_t>(stream));
+      k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau, dout, out, out_other, route_mask,
+      dr_out, dw1, db1, dw2, db2, dk_pool_out, dk_accum, workspace,
+      static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
@@ -428,14 +430,20 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
-ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v,
-                                     const uint8_t* route_mask, const ea_attn_params* p,
-                                     void* out, float* lse, void* workspace,
-                                     size_t workspace_bytes, void* stream) {
+// Forward of a training step (padded BHSD): the chosen mode with its
+// log-sum-exp, and, when out_other is given, every head's other mode too, in
+// the same launch.
+static ea_status prefill_train(const void* q, const void* k, const void* v,
+                               const uint8_t* route_mask, const ea_attn_params* p, void* out,
+                               float* lse, void* out_other, void* workspace,
+                               size_t workspace_bytes, void* stream) {
   ea_status st = check_params(p);
   if (st != EA_OK) return st;
   if (!q || !k || !v || !route_mask || !out || !lse) return EA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+  if (out_other && p->select != EA_SELECT_ALL) return EA_ERR_INVALID_ARG;
+  if (out_other && 2LL * p->B * p->Hq > EA_MAX_ENTRIES) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (out_other && !aligned16(out_other)))
     return EA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
@@ -447,6 +455,8 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
   args.mask = route_mask;
   args.out = out;
   args.lse = lse;
+  args.out_other = out_other;
+  args.both = out_other != nullptr;
   args.status = static_cast<int*>(workspace);
   args.B = p->B;
   args.Hq = p->Hq;
@@ -461,9 +471,27 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
   args.debug_drop_kv_pos = debug_drop_kv_pos();
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
-  cudaError_t err = ea::launch_attn(p->d, args, ea_attn_grid_size(p, sms),
-                                    static_cast<cudaStream_t>(stream));
+  int grid = ea_attn_grid_size(p, sms);
+  if (args.both) grid = std::min(sms, 2 * grid);
+  cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v,
+                                     const uint8_t* route_mask, const ea_attn_params* p,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return prefill_train(q, k, v, route_mask, p, out, lse, nullptr, workspace, workspace_bytes,
+                       stream);
+}
+
+ea_status ea_hybrid_attn_prefill_train(const void* q, const void* k, const void* v,
+                                       const uint8_t* route_mask, const ea_attn_params* p,
+                                       void* out, float* lse, void* out_other, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!out_other) return EA_ERR_INVALID_ARG;
+  return prefill_train(q, k, v, route_mask, p, out, lse, out_other, workspace, workspace_bytes,
+                       stream);
 }
 
 size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p) {

@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       for (int h0 = 0; h0 < args.Hq; h0 += 32) {
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && ld_mask(args.mask, idx) == 0 && args.select != EA_SELECT_SA;
+        const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) == 0) &&
+                        args.select != EA_SELECT_SA;
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nfa += __popc(bits);
@@ -319,7 +320,8 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       for (int h0 = 0; h0 < args.Hq; h0 += 32) {
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && ld_mask(args.mask, idx) != 0 && args.select != EA_SELECT_FA;
+        const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) != 0) &&
+                        args.select != EA_SELECT_FA;
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nsa += __popc(bits);
@@ -675,13 +677,16 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      if (args.lse != nullptr && !packed && row < seq_len)   // log-sum-exp for the backward
+      // a training forward's other mode goes to out_other, without lse
+      const bool chosen = !args.both || (sparse != 0) == (ld_mask(args.mask, idx) != 0);
+      if (chosen && args.lse != nullptr && !packed && row < seq_len)   // for the backward
         args.lse[static_cast<size_t>(idx) * args.N + row] = (m_ref + __log2f(l)) * 0.6931471805599453f;
       // out row: padded [B][Hq][N][d]; packed [T][Hq][d]
       const size_t orow_index =
           packed ? (static_cast<size_t>(s_tok[seq] + row) * args.Hq + idx % args.Hq)
                  : (static_cast<size_t>(idx) * args.N + row);
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) + orow_index * D;
+      __nv_bfloat16* orow =
+          reinterpret_cast<__nv_bfloat16*>(chosen ? args.out : args.out_other) + orow_index * D;
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
         uint32_t o[64];

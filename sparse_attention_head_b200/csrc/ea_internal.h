@@ -24,6 +24,10 @@ struct alignas(64) AttnArgs {
   const int32_t* cu_seqlens;
   int total;                // T, tokens of a packed batch
   float* lse;               // optional [B][Hq][N]: natural log-sum-exp of each row (padded only)
+  // Training forward (padded only): every head runs in both modes; the mode
+  // the mask chooses goes to `out` (and `lse`), the other one to out_other.
+  void* out_other;
+  int both;
   int B, Hq, Hkv, N;
   int sink, window;
   float scale_log2;         // softmax scale * log2(e)
@@ -104,8 +108,9 @@ size_t router_ste_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int 
 cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const float* w1,
                               const float* b1, int hidden, const float* w2, const float* b2,
                               int Hq, const float* g0, const float* g1, float tau,
-                              const void* dout, const void* o_fa, const void* o_sa, float* dr_out,
-                              float* dw1, float* db1, float* dw2, float* db2, float* dk_pool_out,
-                              void* dk_accum, void* workspace, cudaStream_t s);
+                              const void* dout, const void* out, const void* out_other,
+                              const uint8_t* route_mask, float* dr_out, float* dw1, float* db1,
+                              float* dw2, float* db2, float* dk_pool_out, void* dk_accum,
+                              void* workspace, cudaStream_t s);
 
 }  // namespace ea

@@ -88,11 +88,15 @@ __global__ void ea_ste_gumbel_kernel(const float* __restrict__ z, const float* _
   if (r_soft) r_soft[i] = 1.f / (1.f + expf(-u / tau));
 }
 
-// dr partials: CTA (b*Hq + h, split) sums dO * (O_SA - O_FA) over its rows.
+// dr partials: CTA (b*Hq + h, split) sums dO * (O_SA - O_FA) over its rows,
+// from out (the head's chosen mode) and out_other (its other mode): the sum
+// of dO * (out_other - out), negated where the head chose SA (mask nonzero;
+// mask == nullptr: every head chose FA).
 constexpr int kDrThreads = 256;
 __global__ void __launch_bounds__(kDrThreads) ea_ste_dr_kernel(
-    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o_fa,
-    const __nv_bfloat16* __restrict__ o_sa, int N, int d, int nsplit, float* __restrict__ part) {
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
+    const __nv_bfloat16* __restrict__ out_other, const uint8_t* __restrict__ mask, int N, int d,
+    int nsplit, float* __restrict__ part) {
   __shared__ float red[kDrThreads / 32];
   const int bh = blockIdx.x, split = blockIdx.y;
   const size_t len = static_cast<size_t>(N) * d;
@@ -102,8 +106,8 @@ __global__ void __launch_bounds__(kDrThreads) ea_ste_dr_kernel(
   float acc = 0.f;
   for (size_t e = e0 + threadIdx.x * 8; e < e1; e += kDrThreads * 8) {
     const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + base + e));
-    const uint4 f = __ldg(reinterpret_cast<const uint4*>(o_fa + base + e));
-    const uint4 sx = __ldg(reinterpret_cast<const uint4*>(o_sa + base + e));
+    const uint4 f = __ldg(reinterpret_cast<const uint4*>(out + base + e));
+    const uint4 sx = __ldg(reinterpret_cast<const uint4*>(out_other + base + e));
     const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* f2 = reinterpret_cast<const __nv_bfloat162*>(&f);
     const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sx);
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(kDrThreads) ea_ste_dr_kernel(
   if (threadIdx.x == 0) {
     float t = 0.f;
     for (int w = 0; w < kDrThreads / 32; ++w) t += red[w];
-    part[static_cast<size_t>(bh) * nsplit + split] = t;
+    part[static_cast<size_t>(bh) * nsplit + split] = (mask && mask[bh]) ? -t : t;
   }
 }
 
@@ -356,9 +360,10 @@ size_t router_ste_workspace_bytes(int B, int Hkv, int N, int d, int hidden, int 
 cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const float* w1,
                               const float* b1, int hidden, const float* w2, const float* b2,
                               int Hq, const float* g0, const float* g1, float tau,
-                              const void* dout, const void* o_fa, const void* o_sa, float* dr_out,
-                              float* dw1, float* db1, float* dw2, float* db2, float* dk_pool_out,
-                              void* dk_accum, void* workspace, cudaStream_t s) {
+                              const void* dout, const void* out, const void* out_other,
+                              const uint8_t* route_mask, float* dr_out, float* dw1, float* db1,
+                              float* dw2, float* db2, float* dk_pool_out, void* dk_accum,
+                              void* workspace, cudaStream_t s) {
   const size_t n = static_cast<size_t>(B) * Hq;
   const int nsd = ste_dr_splits(B, Hq);
   const int ns = router_num_splits(B, Hkv, N);
@@ -380,8 +385,8 @@ cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const
                                   mask, z, partials, ns, s);
   if (err != cudaSuccess) return err;
   ea_ste_dr_kernel<<<dim3(static_cast<unsigned>(n), nsd), kDrThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o_fa),
-      static_cast<const __nv_bfloat16*>(o_sa), N, d, nsd, drp);
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out),
+      static_cast<const __nv_bfloat16*>(out_other), route_mask, N, d, nsd, drp);
   ea_ste_dz_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
       drp, nsd, z, g0, g1, tau, static_cast<int>(n), dr_out, dz);
   ea_ste_w2_kernel<<<(Hq * (hidden + 1) + 255) / 256, 256, 0, s>>>(dz, h, B, Hq, hidden, dw2,

@@ -122,8 +122,8 @@ def test_router_training_argument_errors(lib):
     def ste(k=16, B=2, Hkv=8, N=64, d=128, hidden=256, Hq=32, g0=16, tau=1.0, dout=16, dw1=16,
             ws=256, wsb=ws_need):
         return lib.ea_router_ste_backward(k, B, Hkv, N, d, 16, 16, hidden, 16, 16, Hq, g0, 16, tau,
-                                          dout, 16, 16, None, dw1, 16, 16, 16, None, None, ws,
-                                          wsb, None)
+                                          dout, 16, 16, None, None, dw1, 16, 16, 16, None, None,
+                                          ws, wsb, None)
     assert ste(k=0) == _lib.EA_ERR_INVALID_ARG
     assert ste(g0=0) == _lib.EA_ERR_INVALID_ARG
     assert ste(dout=0) == _lib.EA_ERR_INVALID_ARG

@@ -37,7 +37,7 @@ def _lib_built():
     build.build()
 
 
-def _inputs(B, Hkv, N, d, Hq, hidden, seed):
+def _inputs(B, Hkv, N, d, Hq, hidden, seed, mix=False):
     g = torch.Generator().manual_seed(seed)
     k = torch.randn((B, Hkv, N, d), generator=g)
     k += torch.randn((B, Hkv, 1, d), generator=g)          # per-sequence offsets
@@ -65,6 +65,9 @@ def _inputs(B, Hkv, N, d, Hq, hidden, seed):
     close = np.abs(u) < 20 * LOGIT_ABS
     g1[torch.as_tensor(close)] += torch.as_tensor(np.where(u[close] >= 0, 1e-2, -1e-2),
                                                   dtype=torch.float32)
+    if mix:     # head 0 of the first sequence to SA, head 1 to FA
+        g1[0, 0] = float(g0[0, 0] - z[0, 0] + 1.0)
+        g1[0, 1] = float(g0[0, 1] - z[0, 1] - 1.0)
     return k, w1, b1, w2, b2, g0, g1
 
 
@@ -148,3 +151,66 @@ def test_ste_backward_is_deterministic():
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+# ---------------------------------------------------------------- a training step
+from gpu_common import compare  # noqa: E402
+from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_backward,  # noqa: E402
+                                            ea_hybrid_attn_prefill,
+                                            ea_hybrid_attn_prefill_lse,
+                                            ea_hybrid_attn_prefill_train)
+
+LSE_ABS = 4.0e-3          # as for the forward's log-sum-exp (bf16 row-sum terms)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,S,W", [(2, 8, 2, 640, 16, 128), (1, 4, 4, 300, 0, 37)])
+def test_training_step_composes(B, Hq, Hkv, N, S, W):
+    """Gumbel decision -> both-mode forward -> attention backward -> router
+    gradients through the straight-through estimator, all on the GPU."""
+    d, hidden, tau = 128, 64, 1.0
+    k, w1, b1, w2, b2, g0, g1 = _inputs(B, Hkv, N, d, Hq, hidden, seed=N + S, mix=True)
+    g = torch.Generator().manual_seed(N + 1)
+    q = torch.randn((B, Hq, N, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, N, d), generator=g).to(torch.bfloat16)
+    dout = torch.randn((B, Hq, N, d), generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    rw = [t.to(DEV) for t in (w1, b1, w2, b2, g0, g1)]
+    mask, _, _ = ea_router_decide_gumbel(kd, *rw, tau)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+    out, lse, other = ea_hybrid_attn_prefill_train(qd, kd, vd, mask, S, W, workspace=ws[:256])
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws[:256]) == 0
+    hm = mask.cpu().numpy()
+    assert 0 < hm.sum() < hm.size, "the step should mix both modes"
+    # each mode is the single-mode kernel's result, bit for bit
+    out1, lse1 = ea_hybrid_attn_prefill_lse(qd, kd, vd, mask, S, W)
+    other1 = ea_hybrid_attn_prefill(qd, kd, vd, (1 - mask).contiguous(), S, W)
+    assert torch.equal(out, out1) and torch.equal(lse, lse1) and torch.equal(other, other1)
+    # and against the oracle
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    compare(out, oracle.attention(qf, kf, vf, hm, S, W), "train chosen mode")
+    compare(other, oracle.attention(qf, kf, vf, 1 - hm, S, W), "train other mode")
+    assert np.abs(f64(lse) - oracle.attention_lse(qf, kf, hm, S, W)).max() <= LSE_ABS
+    # attention backward of the chosen mode, then the router's share added to dk
+    dq, dk, dv = ea_hybrid_attn_backward(qd, kd, vd, out, dod, lse, mask, S, W, workspace=ws)
+    dk_attn = dk.clone()
+    grads = ea_router_ste_backward(kd, *rw, tau, dod, out, other, mask, dk_accum=dk)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    # the training layout gives exactly what the (O_FA, O_SA) layout gives
+    m4 = mask.bool()[:, :, None, None]
+    o_fa, o_sa = torch.where(m4, other, out), torch.where(m4, out, other)
+    plain = ea_router_ste_backward(kd, *rw, tau, dod, o_fa, o_sa)
+    torch.cuda.synchronize()
+    for a, b in zip(grads, plain):
+        assert torch.equal(a, b)
+    want = (dk_attn.float() + grads[5].view(B, Hkv, 1, d)).to(torch.bfloat16)
+    assert torch.equal(dk, want)
+    # the router gradients against the oracle, on the GPU's own outputs
+    r_dr, r_dz, r_dw1, r_db1, r_dw2, r_db2, r_dk = oracle.router_ste_backward(
+        f64(k), *_np(w1, b1, w2, b2, g0, g1), tau, f64(dout), f64(o_fa), f64(o_sa))
+    terms = np.sum(np.abs(f64(dout) * (f64(o_sa) - f64(o_fa))), axis=(2, 3))
+    assert np.all(np.abs(grads[0].cpu().double().numpy() - r_dr) <= SUM_REL * terms)
+    eps = 4 * (SUM_REL + LOGIT_ABS / tau)
+    scale = np.abs(r_dw2).max()
+    assert np.abs(grads[3].cpu().double().numpy() - r_dw2).max() <= eps * 4 * scale
