@@ -64,8 +64,12 @@ def parse_args():
                     help="run only the decode measurement and print its JSON object")
     ap.add_argument("--packed-seqs", type=int, default=8,
                     help="sequences in the packed-batch measurement (0 skips it)")
-    ap.add_argument("--backward-only", action="store_true",
-                    help="run only the training-step (forward + backward) measurement")
+    ap.add_argument("--training-only", "--backward-only", dest="training_only",
+                    action="store_true",
+                    help="run only the training-step measurement (router, both-mode "
+                         "forward, backward, router gradients)")
+    ap.add_argument("--no-training", action="store_true",
+                    help="skip the training-step measurement of the default line")
     ap.add_argument("--packed-only", action="store_true",
                     help="run only the packed-batch measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
@@ -414,6 +418,9 @@ def run_ours(args, rank, world, local_rank):
     if not args.quick and world == 1 and args.decode_batch > 0:
         result["decode"] = measure_decode(w, args.decode_batch, max(args.steps, 10),
                                           max(args.warmup, 3), dev, stream)
+    if not args.quick and world == 1 and not args.no_training:
+        result["training"] = measure_training(w, max(args.steps, 5), max(args.warmup, 3), dev,
+                                              stream)
     return result
 
 
@@ -518,34 +525,66 @@ def measure_packed(w: workloads.Workload, nseq: int, steps: int, warmup: int, de
 
 
 # ---------------------------------------------------------------- backward
-def measure_backward(w: workloads.Workload, steps: int, warmup: int, dev, stream):
-    """Training step of one layer's attention: the forward with log-sum-exp,
-    then the backward (D, dK/dV, dQ), timed separately with CUDA events.
-    Work: the forward's effective flops, and 2.5x that for the backward (five
-    products of the forward's size against its two)."""
+def measure_training(w: workloads.Workload, steps: int, warmup: int, dev, stream):
+    """One layer's attention training step, every phase timed with CUDA events:
+    the Gumbel-Softmax router decision, the forward of both modes in one
+    launch (the straight-through router gradient needs both outputs), the
+    attention backward of each head's chosen mode (D, dK/dV, dQ), and the
+    router's straight-through gradients (added into dK).  Work: the forward's
+    effective flops of both modes, 2.5x the chosen mode's for the backward
+    (five products of the forward's size against its two)."""
     from sparse_attention_head_b200 import flops
     from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_backward,
-                                                ea_hybrid_attn_prefill_lse)
+                                                ea_hybrid_attn_prefill_lse,
+                                                ea_hybrid_attn_prefill_train,
+                                                ea_router_decide_gumbel, ea_router_ste_backward)
     B, Hq, Hkv, N, d, S, W = w.batch, w.hq, w.hkv, w.seq, w.d, w.sink, w.window
     seed = workloads.layer_seed(w, 0) + 9000
     q, k, v = workloads.make_qkv(w, seed, device=dev)
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
     dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    mask = workloads.make_fixed_mask(dataclasses.replace(w, sparse_frac=workloads.layer_sparse_frac(w, 0)),
-                                     seed).to(dev)
+    frac = workloads.layer_sparse_frac(w, 0)
+    heads = workloads.sparse_head_set(Hq, frac, seed)
+    w1, b1, w2, b2 = (t.to(dev) for t in workloads.make_router_weights(
+        Hkv * d, w.router_hidden, Hq, heads, seed))
+    g0, g1 = workloads.gumbel_noise(B, Hq, seed, device=dev)
+    tau = 1.0
     ws = torch.zeros(1 << 26, dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
+    rws = torch.empty(1 << 26, dtype=torch.uint8, device=dev)
+    out, other = torch.empty_like(q), torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
+
+    r_soft = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+
+    def router():
+        ea_router_decide_gumbel(k, w1, b1, w2, b2, g0, g1, tau, route_mask=mask, r_soft=r_soft,
+                                logits=logits, workspace=rws, stream=stream)
 
     def fwd():
+        ea_hybrid_attn_prefill_train(q, k, v, mask, S, W, out=out, lse=lse, out_other=other,
+                                     workspace=ws[:256], stream=stream)
+
+    def fwd_chosen_only():
         ea_hybrid_attn_prefill_lse(q, k, v, mask, S, W, out=out, lse=lse, workspace=ws[:256],
                                    stream=stream)
 
     def bwd():
         ea_hybrid_attn_backward(q, k, v, out, dout, lse, mask, S, W, dq=dq, dk=dk, dv=dv,
                                 workspace=ws, stream=stream)
+
+    def ste():
+        ea_router_ste_backward(k, w1, b1, w2, b2, g0, g1, tau, dout, out, other, mask,
+                               dk_accum=dk, workspace=rws, stream=stream)
+
+    def step():
+        router()
+        fwd()
+        bwd()
+        ste()
 
     def timed(fn, n):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -556,32 +595,51 @@ def measure_backward(w: workloads.Workload, steps: int, warmup: int, dev, stream
         torch.cuda.synchronize()
         return a.elapsed_time(b) / n
 
-    for _ in range(warmup):
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        r_ms = timed(router, steps)
+        f_ms = timed(fwd, steps)
+        f1_ms = timed(fwd_chosen_only, steps)
         fwd()
-        bwd()
-    torch.cuda.synchronize()
-    f_ms = timed(fwd, steps)
-    b_ms = timed(bwd, steps)
-    if ea_get_device_status(ws) != 0:
-        raise RuntimeError("backward status word reports an error")
-    eff = flops.effective_flops(mask.cpu().numpy(), N, d, S, W)
+        b_ms = timed(bwd, steps)
+        s_ms = timed(ste, steps)
+        t_ms = timed(step, steps)
+    if ea_get_device_status(ws) != 0 or ea_get_device_status(ws[:256]) != 0:
+        raise RuntimeError("a training kernel's status word reports an error")
+    hm = mask.cpu().numpy()
+    eff = flops.effective_flops(hm, N, d, S, W)
+    eff_both = (flops.effective_flops(np.zeros_like(hm), N, d, S, W) +
+                flops.effective_flops(np.ones_like(hm), N, d, S, W))
     peaks, src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     btf = 2.5 * eff / (b_ms * 1e-3) / 1e12
+    # router STE bytes: dO, out, out_other once (the dr reduction), K once
+    # (the forward recompute), dK read and written (the in-place add)
+    ste_bytes = 2 * (3 * B * Hq * N * d + B * Hkv * N * d + 2 * B * Hkv * N * d)
     return {
         "workload": f"{w.name} training step of one layer: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} "
-                    f"S={S} W={W}, SA heads {mask.float().mean():.2f}",
+                    f"S={S} W={W}, Gumbel routes with tau={tau}: SA heads {hm.mean():.2f}",
         "steps": steps, "warmup": warmup,
-        "forward_lse_ms": round(f_ms, 4),
-        "forward_tflops": round(eff / (f_ms * 1e-3) / 1e12, 2),
+        "step_ms": round(t_ms, 4),
+        "router_gumbel_ms": round(r_ms, 4),
+        "forward_both_modes_ms": round(f_ms, 4),
+        "forward_both_modes_tflops": round(eff_both / (f_ms * 1e-3) / 1e12, 2),
+        "forward_chosen_mode_only_ms": round(f1_ms, 4),
         "backward_ms": round(b_ms, 4),
         "backward_tflops": round(btf, 2),
+        "router_ste_ms": round(s_ms, 4),
+        "router_ste_gbs": round(ste_bytes / (s_ms * 1e-3) / 1e9, 1),
+        "router_ste_hbm_frac": round(ste_bytes / (s_ms * 1e-3) / 1e9 / hbm, 4),
         "roofline": {"bound": "tensor", "achieved": round(btf, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(btf / peak, 4),
                      "peak_source": f"{src} bf16_tflops (burst)",
-                     "scope": "backward (rowdot + dK/dV + dQ kernels), 2.5x effective "
-                              "forward flops"},
-        "gpu_launches_per_step": 3,
+                     "scope": "attention backward (rowdot + dK/dV + dQ kernels), 2.5x the "
+                              "chosen mode's effective forward flops"},
+        # router 4 + Gumbel 1; forward 1; backward 3; STE: recompute 4 + 7
+        "gpu_launches_per_step": 5 + 1 + 3 + 11,
     }
 
 
@@ -788,13 +846,13 @@ def main():
             return 0
         print(json.dumps(run_reference(args)), flush=True)
         return 0
-    if args.backward_only:
+    if args.training_only:
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         w = workloads.get(args.workload)
         if args.seq:
             w = dataclasses.replace(w, seq=args.seq)
-        res = measure_backward(w, args.steps, max(args.warmup, 3), dev,
+        res = measure_training(w, args.steps, max(args.warmup, 3), dev,
                                torch.cuda.current_stream(dev))
         if rank == 0:
             print(json.dumps(res), flush=True)

@@ -447,18 +447,30 @@ def _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau):
 def ea_router_decide_gumbel(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
                             w2: torch.Tensor, b2: torch.Tensor, g0: torch.Tensor,
                             g1: torch.Tensor, tau: float, *,
+                            route_mask: Optional[torch.Tensor] = None,
+                            r_soft: Optional[torch.Tensor] = None,
+                            logits: Optional[torch.Tensor] = None,
                             workspace: Optional[torch.Tensor] = None,
                             stream: Optional[torch.cuda.Stream] = None):
-    """Training-time routing: (r_hard uint8 [B, Hq], r_soft fp32, logits fp32)."""
+    """Training-time routing: (r_hard uint8 [B, Hq], r_soft fp32, logits fp32),
+    into the given buffers when passed."""
     lib = _lib.load()
     B, Hkv, N, d, hidden, Hq = _router_train_dims(k, w1, b1, w2, b2, g0, g1, tau)
     dev = k.device
     if workspace is None:
         workspace = torch.empty(max(int(lib.ea_router_gumbel_workspace_size(
             B, Hkv, N, d, hidden, Hq)), 16), dtype=torch.uint8, device=dev)
-    r_hard = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
-    r_soft = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    r_hard = torch.empty((B, Hq), dtype=torch.uint8, device=dev) if route_mask is None \
+        else route_mask
+    if r_soft is None:
+        r_soft = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if logits is None:
+        logits = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    for name, t, dt in (("route_mask", r_hard, torch.uint8), ("r_soft", r_soft, torch.float32),
+                        ("logits", logits, torch.float32)):
+        _need(t, name, dt)
+        if t.numel() != B * Hq:
+            raise ValueError(f"{name} must hold B * Hq values")
     rc = lib.ea_router_decide_gumbel(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(),
                                      hidden, w2.data_ptr(), b2.data_ptr(), Hq, g0.data_ptr(),
                                      g1.data_ptr(), float(tau), r_hard.data_ptr(),

@@ -134,6 +134,16 @@ def make_router_weights(in_dim: int, hidden: int, out_dim: int, sparse_heads,
     return w1.float(), b1.float(), w2.float(), b2.float()
 
 
+def gumbel_noise(batch: int, hq: int, seed: int, device="cpu"):
+    """Two fp32 [batch, hq] draws of standard Gumbel noise, -log(-log U) with
+    U uniform in (0, 1): the noise of the FA and SA choices that a
+    Gumbel-Softmax training step takes as input."""
+    g = _gen(seed + 31, "cpu")
+    u = torch.rand((2, batch, hq), generator=g, dtype=torch.float64).clamp(1e-12, 1.0 - 1e-12)
+    gum = (-torch.log(-torch.log(u))).float()
+    return gum[0].contiguous().to(device), gum[1].contiguous().to(device)
+
+
 def make_fixed_mask(w: Workload, seed: int) -> torch.Tensor:
     """uint8 [B, Hq] mask (1 = sparse), drawn independently per batch row."""
     m = torch.zeros((w.batch, w.hq), dtype=torch.uint8)
