@@ -15,14 +15,15 @@
 //   2. ea_bwd_dkdv_kernel: unit = (b, kv head, 128-key tile j).  K_j and V_j
 //      stay in shared memory; the steps visit (query head of the group,
 //      128-query tile i) pairs that see tile j.  Per step the tensor cores
-//      compute S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM, four warps
-//      turn them into P^T and dS^T (bf16, back into TMEM), and
-//      dV += P^T dO_i, dK += dS^T Q_i accumulate in TMEM (A from TMEM).
+//      compute S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM, eight warps
+//      (two column halves of four) turn them into P^T and dS^T (bf16, back
+//      into TMEM), and dV += P^T dO_i, dK += dS^T Q_i accumulate in TMEM (A
+//      from TMEM), issued half by half as each column half is ready.
 //   3. ea_bwd_dq_kernel: unit = (b, head, 128-query tile i); the steps visit
 //      the key tiles the forward visits: S = Q_i K_j^T, dP = dO_i V_j^T, dS,
 //      dQ += dS K_j.
 // Both are persistent (one CTA per SM), with a TMA producer warp, one MMA
-// issuing thread and four elementwise warps; every wait is bounded.
+// issuing thread and eight elementwise warps; every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
