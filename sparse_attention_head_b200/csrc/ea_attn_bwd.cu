@@ -18,7 +18,9 @@
 //      compute S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM, eight warps
 //      (two column halves of four) turn them into P^T and dS^T (bf16, back
 //      into TMEM), and dV += P^T dO_i, dK += dS^T Q_i accumulate in TMEM (A
-//      from TMEM), issued half by half as each column half is ready.
+//      from TMEM).  The elementwise work runs in two phases (P from S while
+//      dP is computed; dS from dP while dV and the next S are), so the
+//      tensor pipe and the elementwise warps overlap.
 //   3. ea_bwd_dq_kernel: unit = (b, head, 128-query tile i); the steps visit
 //      the key tiles the forward visits: S = Q_i K_j^T, dP = dO_i V_j^T, dS,
 //      dQ += dS K_j.
@@ -61,27 +63,45 @@ __global__ void ea_bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ dout,
   if (lane == 0) dvec[warp] = s;
 }
 
-// Shared-memory plan of both backward kernels (d = 128): two resident tiles
-// (the unit's own operands) and a ring of two stages of two streamed tiles.
+// Shared-memory plan of both backward kernels (d = 128).  The streamed
+// operands come in two rings: tile 0 (kDkDv: Q_i; else K_j) is read by a
+// step's first score product and, one phase later, by its last accumulating
+// product, and the next step's first score product needs the next tile 0
+// while the current one is still in use, so its ring has three slots; tile 1
+// (kDkDv: dO_i; else V_j) is needed later in the step and has two.  The small
+// data (per-step vectors, step descriptors, barriers) comes first and the
+// tiles start 1024-aligned after it, which fills the 227 KB exactly; the
+// kernel requires a 1024-aligned dynamic shared-memory base (checked).
 struct BwdCfg {
   static constexpr int D = 128;
   static constexpr int kThreads = 320;           // warps 0-7 elementwise, 8 producer, 9 MMA
   static constexpr int kBlockBytes = 128 * 128;  // 128 rows x 64 bf16 (one SW128 column block)
   static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kStages = 2;
-  static constexpr int kOffRes = 0;                          // 2 resident tiles
-  static constexpr int kOffStage = 2 * kTileBytes;           // kStages x 2 streamed tiles
-  // per stage: -lse * log2e and -D of the step's 128 query rows (f32)
-  static constexpr int kOffVec = kOffStage + kStages * 2 * kTileBytes;
-  static constexpr int kOffStep = kOffVec + kStages * 2 * 128 * 4;   // step descriptors, 32 B each
-  static constexpr int kOffBar = kOffStep + kStages * 32;
-  // res_full, res_empty, st_full[kStages], st_empty[kStages], s_full[2], ld_done,
-  // p_full[2], acc_done, acc_empty, drain (s_full / p_full: one per column half)
-  static constexpr int kNumBars = 2 + 2 * kStages + 8;
+  static constexpr int kStages0 = 3;             // ring of streamed tile 0
+  static constexpr int kStages1 = 2;             // ring of streamed tile 1
+  // kDkDv: -lse * log2e of the step's 128 query rows per tile-0 slot, and -D
+  // per tile-1 slot (f32)
+  static constexpr int kOffVec0 = 0;
+  static constexpr int kOffVec1 = kOffVec0 + kStages0 * 128 * 4;
+  static constexpr int kOffStep = kOffVec1 + kStages1 * 128 * 4;  // descriptors per tile-0 slot
+  static constexpr int kOffBar = kOffStep + kStages0 * 32;
+  // res_full, res_empty, full0[kStages0], empty0[kStages0], full1[kStages1],
+  // empty1[kStages1], s_full, dp_full, p_full, ds_full, acc_done, acc_empty,
+  // drain
+  static constexpr int kNumBars = 2 + 2 * kStages0 + 2 * kStages1 + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;    // tmem base, abort flag
-  static constexpr int kSmem = kOffMisc + 64 + 1024;         // + alignment slack
+  static constexpr int kOffTiles = 3072;
+  static constexpr int kOffRes = kOffTiles;                  // 2 resident tiles
+  static constexpr int kOffSt0 = kOffRes + 2 * kTileBytes;
+  static constexpr int kOffSt1 = kOffSt0 + kStages0 * kTileBytes;
+  static constexpr int kSmem = kOffSt1 + kStages1 * kTileBytes;
   static constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);  // both K-major
   static constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);    // B MN-major
+  // of every 8 pairs of exponentials in the P phase, this many go to the
+  // FMA-pipe polynomial instead of the MUFU
+  static constexpr int kEmuPairs = 2;
+  static_assert(kOffMisc + 64 <= kOffTiles, "small data overlaps the tiles");
+  static_assert(kOffTiles % 1024 == 0, "tiles must be 1024-aligned");
   static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
@@ -129,6 +149,50 @@ __device__ __forceinline__ bool bwd_block_full(int it, int jt, int N, bool sa, i
 
 
 
+// ---------------------------------------------------------------- phases
+// P phase of one thread's 64 columns (col0 ..): pr = 2^(s * sl2 + nl) on
+// visible pairs and 0 elsewhere, and pk = the same as packed bf16 pairs.
+// kDkDv: nl per column from vl (-lse * log2e of the column's query); else
+// the row's own nl_row.  Visible columns c (0..127 within the tile): c in
+// [lo_a, hi_a] and (c < sink_c or c >= win_c); kFull: every column.
+template <bool kDkDv, bool kFull>
+__device__ __forceinline__ void bwd_phase_p(uint32_t taddr, const float* vl, float nl_row,
+                                            int col0, float sl2, int lo_a, int hi_a, int sink_c,
+                                            int win_c, float (&pr)[64], uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t sr[32];
+    tmem_ld32_wait(taddr + 32 * ch, sr);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = 16 * ch + jj;
+      const int c = col0 + 2 * j;
+      float x0, x1;
+      if (kDkDv) {
+        const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
+        x0 = l2.x;
+        x1 = l2.y;
+      } else {
+        x0 = x1 = nl_row;
+      }
+      fma2_acc(x0, x1, __uint_as_float(sr[2 * jj]), __uint_as_float(sr[2 * jj + 1]), sl2, sl2);
+      if ((j & 7) < BwdCfg::kEmuPairs) {
+        exp2_poly2(x0, x1);
+      } else {
+        x0 = ex2_approx(x0);
+        x1 = ex2_approx(x1);
+      }
+      if (!kFull) {
+        x0 = (c >= lo_a && c <= hi_a && (c < sink_c || c >= win_c)) ? x0 : 0.f;
+        x1 = (c + 1 >= lo_a && c + 1 <= hi_a && (c + 1 < sink_c || c + 1 >= win_c)) ? x1 : 0.f;
+      }
+      pr[2 * j] = x0;
+      pr[2 * j + 1] = x1;
+      pk[j] = pack_bf16x2(x0, x1);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- units
 // kDkDv: unit (b, kv head, key tile), key tile 0 (the most queries) first;
 // else unit (b, head, query tile), the last query tile (the most keys) first.
@@ -165,22 +229,28 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
   using C = BwdCfg;
   constexpr int D = C::D;
   constexpr float kLog2e = 1.4426950408889634f;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the plan fills the 227 KB with no room to align the base: require it
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(args.status, EA_OK, EA_ERR_UNSUPPORTED);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   const uint32_t bar0 = smem_u32(bar);
   const uint32_t b_res_full = bar0, b_res_empty = bar0 + 8;
-  const uint32_t b_st_full = bar0 + 16, b_st_empty = bar0 + 16 + 8 * C::kStages;
-  const uint32_t b_s_full = bar0 + 16 + 16 * C::kStages;     // [2]
-  const uint32_t b_ld_done = b_s_full + 16, b_p_full = b_s_full + 24;   // p_full [2]
-  const uint32_t b_acc_done = b_s_full + 40, b_acc_empty = b_s_full + 48;
-  const uint32_t b_drain = b_s_full + 56;
+  const uint32_t b_full0 = bar0 + 16, b_empty0 = b_full0 + 8 * C::kStages0;
+  const uint32_t b_full1 = b_empty0 + 8 * C::kStages0, b_empty1 = b_full1 + 8 * C::kStages1;
+  const uint32_t b_s_full = b_empty1 + 8 * C::kStages1, b_dp_full = b_s_full + 8;
+  const uint32_t b_p_full = b_s_full + 16, b_ds_full = b_s_full + 24;
+  const uint32_t b_acc_done = b_s_full + 32, b_acc_empty = b_s_full + 40;
+  const uint32_t b_drain = b_s_full + 48;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   BwdStep* steps = reinterpret_cast<BwdStep*>(smem + C::kOffStep);
-  float* vec = reinterpret_cast<float*>(smem + C::kOffVec);
+  float* vec0 = reinterpret_cast<float*>(smem + C::kOffVec0);
+  float* vec1 = reinterpret_cast<float*>(smem + C::kOffVec1);
   const int G = args.Hq / args.Hkv;
   const int nT = ea_cdiv(args.N, EA_BN);
   const int units = args.B * (kDkDv ? args.Hkv : args.Hq) * nT;
@@ -188,20 +258,12 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
   int* status = args.status;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar + 0, 1);                        // res_full: producer
-    mbar_init(bar + 1, 1);                        // res_empty: MMA commit
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(bar + 2 + i, 1);                  // st_full: producer
-      mbar_init(bar + 2 + C::kStages + i, 1);     // st_empty: MMA commit
+    // arrival counts: one (producer arrive or MMA commit) except p_full,
+    // ds_full and acc_empty (all 256 elementwise threads)
+    for (int i = 0; i < C::kNumBars; ++i) {
+      const uint32_t a = bar0 + 8 * i;
+      mbar_init(bar + i, (a == b_p_full || a == b_ds_full || a == b_acc_empty) ? 256 : 1);
     }
-    mbar_init(bar + 2 + 2 * C::kStages, 1);       // s_full[0]: MMA commit
-    mbar_init(bar + 3 + 2 * C::kStages, 1);       // s_full[1]: MMA commit
-    mbar_init(bar + 4 + 2 * C::kStages, 128);     // ld_done: column half 0
-    mbar_init(bar + 5 + 2 * C::kStages, 128);     // p_full[0]: column half 0
-    mbar_init(bar + 6 + 2 * C::kStages, 128);     // p_full[1]: column half 1
-    mbar_init(bar + 7 + 2 * C::kStages, 1);       // acc_done: MMA commit
-    mbar_init(bar + 8 + 2 * C::kStages, 256);     // acc_empty: elementwise threads
-    mbar_init(bar + 9 + 2 * C::kStages, 1);       // drain: MMA commit
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -216,7 +278,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
 
   if (warp == 8) {
     // ============================================================ producer
-    uint32_t pos = 0, nu = 0;
+    uint32_t pos = 0, nu = 0, armed0 = 0, armed1 = 0;
     bool ok = true;
     for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
          u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
@@ -257,42 +319,64 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         for (int i = 0; i < n && ok; ++i) {
           const int it = kDkDv ? tile + i : tile;
           const int jt = kDkDv ? tile : (i < a ? i : lo + (i - a));
-          const uint32_t slot = pos % C::kStages;
-          if (pos >= C::kStages) {
+          const int row = (kDkDv ? it : jt) * EA_BM;
+          const uint32_t s0 = pos % C::kStages0, s1 = pos % C::kStages1;
+          // tile 0 (Q_i or K_j), its -lse vector and the step descriptor
+          if (pos >= C::kStages0) {
             if (lane == 0)
-              ok = mbar_wait(b_st_empty + 8 * slot, ((pos / C::kStages) - 1) & 1, s_abort,
-                             status, tlim, EA_ERR_TIMEOUT);
+              ok = mbar_wait(b_empty0 + 8 * s0, ((pos / C::kStages0) - 1) & 1, s_abort, status,
+                             tlim, EA_ERR_TIMEOUT);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
           if (kDkDv) {
-            // -lse * log2e and -D of the step's query rows
-            float* vl = vec + slot * 256;
+            float* vl = vec0 + s0 * 128;
             for (int r = lane; r < EA_BM; r += 32) {
               const int q = it * EA_BM + r;
               const size_t ri = (static_cast<size_t>(b) * args.Hq + h) * args.N + q;
               vl[r] = q < args.N ? -args.lse[ri] * kLog2e : 0.f;
-              vl[128 + r] = q < args.N ? -args.dvec[ri] : 0.f;
             }
             __syncwarp();
           }
           if (lane == 0) {
-            BwdStep& st = steps[slot];
+            BwdStep& st = steps[s0];
             st.b = b; st.h = h; st.it = it; st.jt = jt; st.sa = sa;
             st.first = (g == 0 && i == 0);
             st.last = (g == ng - 1 && i == n - 1);
             st.full = bwd_block_full(it, jt, args.N, sa, args.sink, args.window);
-            mbar_arrive_expect_tx(b_st_full + 8 * slot, 2 * C::kTileBytes);
-            const uint32_t dst = smem_u32(smem + C::kOffStage) + slot * 2 * C::kTileBytes;
-            const CUtensorMap* m0 = kDkDv ? &args.tm_q : &args.tm_k;
-            const CUtensorMap* m1 = kDkDv ? &args.tm_do : &args.tm_v;
+            mbar_arrive_expect_tx(b_full0 + 8 * s0, C::kTileBytes);
+            ++armed0;
+            const uint32_t dst = smem_u32(smem + C::kOffSt0) + s0 * C::kTileBytes;
+            const CUtensorMap* m = kDkDv ? &args.tm_q : &args.tm_k;
             const int z = kDkDv ? b * args.Hq + h : b * args.Hkv + h / G;
-            const int row = (kDkDv ? it : jt) * EA_BM;
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_3d(dst + c * C::kBlockBytes, m0, b_st_full + 8 * slot, c * 64, row, z);
-              tma_load_3d(dst + C::kTileBytes + c * C::kBlockBytes, m1, b_st_full + 8 * slot,
-                          c * 64, row, z);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + c * C::kBlockBytes, m, b_full0 + 8 * s0, c * 64, row, z);
+          }
+          // tile 1 (dO_i or V_j) and its -D vector
+          if (pos >= C::kStages1) {
+            if (lane == 0)
+              ok = mbar_wait(b_empty1 + 8 * s1, ((pos / C::kStages1) - 1) & 1, s_abort, status,
+                             tlim, EA_ERR_TIMEOUT);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+          }
+          if (kDkDv) {
+            float* vd = vec1 + s1 * 128;
+            for (int r = lane; r < EA_BM; r += 32) {
+              const int q = it * EA_BM + r;
+              const size_t ri = (static_cast<size_t>(b) * args.Hq + h) * args.N + q;
+              vd[r] = q < args.N ? -args.dvec[ri] : 0.f;
             }
+            __syncwarp();
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(b_full1 + 8 * s1, C::kTileBytes);
+            ++armed1;
+            const uint32_t dst = smem_u32(smem + C::kOffSt1) + s1 * C::kTileBytes;
+            const CUtensorMap* m = kDkDv ? &args.tm_do : &args.tm_v;
+            const int z = kDkDv ? b * args.Hq + h : b * args.Hkv + h / G;
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + c * C::kBlockBytes, m, b_full1 + 8 * s1, c * 64, row, z);
           }
           ++pos;
         }
@@ -300,81 +384,113 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     }
     if (lane == 0) {
       // every copy issued must land before the CTA exits
-      const uint32_t n = pos < C::kStages ? pos : C::kStages;
-      for (uint32_t p = pos - n; p < pos; ++p)
-        mbar_wait_drain(b_st_full + 8 * (p % C::kStages), (p / C::kStages) & 1, 200000000ull);
+      const uint32_t n0 = armed0 < C::kStages0 ? armed0 : C::kStages0;
+      for (uint32_t p = armed0 - n0; p < armed0; ++p)
+        mbar_wait_drain(b_full0 + 8 * (p % C::kStages0), (p / C::kStages0) & 1, 200000000ull);
+      const uint32_t n1 = armed1 < C::kStages1 ? armed1 : C::kStages1;
+      for (uint32_t p = armed1 - n1; p < armed1; ++p)
+        mbar_wait_drain(b_full1 + 8 * (p % C::kStages1), (p / C::kStages1) & 1, 200000000ull);
       if (nu > 0) mbar_wait_drain(b_res_full, (nu - 1) & 1, 200000000ull);
     }
   } else if (warp == 9) {
     // ============================================================ MMA issuer
+    // Per step n, the score products and the two phases of the elementwise
+    // warps interleave:
+    //   [E: P from S(n)]    while dP(n) runs
+    //   dV += P^T dO (kDkDv), then S(n + 1)   while E computes dS from dP(n)
+    //   dK += dS^T Q (or dQ += dS K), then dP(n + 1)   while E computes P(n + 1)
+    // so the tensor pipe and the elementwise warps work at the same time.
+    // tcgen05.mma from one thread executes in issue order, so a score
+    // product overwrites the columns the accumulating product before it read.
     if (lane == 0) {
       const uint32_t res = smem_u32(smem + C::kOffRes);
-      const uint32_t stg = smem_u32(smem + C::kOffStage);
-      // K-major views (the two score products) and MN-major views (the B
-      // operand of the accumulating products)
+      // K-major views (the score products) and MN-major views (the B operand
+      // of the accumulating products)
       const uint64_t d_res_k = smem_desc_sw128(res, 16, 1024);
-      const uint64_t d_stg_k = smem_desc_sw128(stg, 16, 1024);
-      const uint64_t d_stg_mn = smem_desc_sw128(stg, C::kBlockBytes, 1024);
+      const uint64_t d_st0_k = smem_desc_sw128(smem_u32(smem + C::kOffSt0), 16, 1024);
+      const uint64_t d_st1_k = smem_desc_sw128(smem_u32(smem + C::kOffSt1), 16, 1024);
+      const uint64_t d_st0_mn = smem_desc_sw128(smem_u32(smem + C::kOffSt0), C::kBlockBytes, 1024);
+      const uint64_t d_st1_mn = smem_desc_sw128(smem_u32(smem + C::kOffSt1), C::kBlockBytes, 1024);
+      // which = 0: kDkDv S^T = K Q^T, else S = Q K^T (TMEM columns 0-127),
+      // resident tile 0 against tile 0 of step p; which = 1: kDkDv
+      // dP^T = V dO^T, else dP = dO V^T (columns 128-255), tiles 1
+      auto scores = [&](uint32_t p, int which) {
+        const uint64_t a = d_res_k + ((which * C::kTileBytes) >> 4);
+        const uint64_t b = which ? d_st1_k + (((p % C::kStages1) * C::kTileBytes) >> 4)
+                                 : d_st0_k + (((p % C::kStages0) * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
+          mma_ss(tmem + 128 * which, a + off, b + off, C::kIdescSS, k > 0 ? 1u : 0u);
+        }
+      };
+      auto wait_full = [&](int which, uint32_t p) {
+        return which ? mbar_wait(b_full1 + 8 * (p % C::kStages1), (p / C::kStages1) & 1, s_abort,
+                                 status, tlim, EA_ERR_TIMEOUT)
+                     : mbar_wait(b_full0 + 8 * (p % C::kStages0), (p / C::kStages0) & 1, s_abort,
+                                 status, tlim, EA_ERR_TIMEOUT);
+      };
       uint32_t pos = 0, nu = 0, nsteps = 0;
       bool ok = true;
       for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
          u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
         if (!(ok = mbar_wait(b_res_full, nu & 1, s_abort, status, tlim, EA_ERR_TIMEOUT))) break;
-        if (nu > 0 && !(ok = mbar_wait(b_acc_empty, (nu - 1) & 1, s_abort, status, tlim,
-                                       EA_ERR_TIMEOUT)))
-          break;
-        tc_fence_after();
-        ++nu;
+        const uint32_t unit = nu++;
+        if (!(ok = wait_full(0, pos))) break;
+        scores(pos, 0);
+        mma_commit(b_s_full);
+        if (!(ok = wait_full(1, pos))) break;
+        scores(pos, 1);
+        mma_commit(b_dp_full);
         bool last = false, first = true;
         while (!last && ok) {
-          const uint32_t slot = pos % C::kStages;
-          if (!(ok = mbar_wait(b_st_full + 8 * slot, (pos / C::kStages) & 1, s_abort, status,
-                               tlim, EA_ERR_TIMEOUT)))
+          const uint32_t s0 = pos % C::kStages0, s1 = pos % C::kStages1;
+          last = steps[s0].last != 0;
+          // the previous unit's accumulators must have been read out
+          if (first && unit > 0 &&
+              !(ok = mbar_wait(b_acc_empty, (unit - 1) & 1, s_abort, status, tlim,
+                               EA_ERR_TIMEOUT)))
             break;
-          last = steps[slot].last != 0;
-          // scores: kDkDv S^T = K Q^T and dP^T = V dO^T; else S = Q K^T and
-          // dP = dO V^T (resident tile 0 / 1 against streamed tile 0 / 1)
-          // (N = 128; splitting them into column halves doubles the MMA
-          // instructions this one thread issues and measured slower)
-          const uint64_t s0 = d_stg_k + ((slot * 2 * C::kTileBytes) >> 4);
-          const uint64_t s1 = s0 + (C::kTileBytes >> 4);
+          const uint64_t m0 = d_st0_mn + ((s0 * C::kTileBytes) >> 4);
+          const uint64_t m1 = d_st1_mn + ((s1 * C::kTileBytes) >> 4);
+          // P done (kDkDv: as bf16 P^T at the start of each column half's
+          // columns) and S read
+          if (!(ok = mbar_wait(b_p_full, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT)))
+            break;
+          tc_fence_after();
+          if (kDkDv) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
-            mma_ss(tmem, d_res_k + off, s0 + off, C::kIdescSS, k > 0 ? 1u : 0u);
-            mma_ss(tmem + 128, d_res_k + (C::kTileBytes >> 4) + off, s1 + off, C::kIdescSS,
-                   k > 0 ? 1u : 0u);
+            for (int k = 0; k < 8; ++k)
+              mma_ts(tmem + 256, tmem + 64 * (k >> 2) + 8 * (k & 3), m1 + ((k * 2048) >> 4),
+                     C::kIdescTS, (!first || k > 0) ? 1u : 0u);            // dV += P^T dO
           }
-          mma_commit(b_s_full);
-          mma_commit(b_s_full + 8);
-          const uint64_t m0 = d_stg_mn + ((slot * 2 * C::kTileBytes) >> 4);
-          const uint64_t m1 = m0 + (C::kTileBytes >> 4);
-          // the accumulating products in two K halves (columns 0-63, 64-127
-          // of P / dS), each as soon as its elementwise half is done
-#pragma unroll
-          for (int hf = 0; hf < 2 && ok; ++hf) {
-            if (!(ok = mbar_wait(b_p_full + 8 * hf, nsteps & 1, s_abort, status, tlim,
-                                 EA_ERR_TIMEOUT)))
-              break;
-            tc_fence_after();
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              const int k = 4 * hf + kq;
-              const uint32_t acc = (!first || k > 0) ? 1u : 0u;
-              if (kDkDv) {
-                mma_ts(tmem + 256, tmem + k * 8, m1 + ((k * 2048) >> 4), C::kIdescTS, acc);  // dV += P^T dO
-                mma_ts(tmem + 384, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
-                       acc);                                                               // dK += dS^T Q
-              } else {
-                mma_ts(tmem + 256, tmem + 128 + k * 8, m0 + ((k * 2048) >> 4), C::kIdescTS,
-                       acc);                                                               // dQ += dS K
-              }
-            }
+          // (TMA-written tiles need no tcgen05 fence: the mbarrier completes
+          // the copy for the tensor cores' reads)
+          if (!last) {
+            if (!(ok = wait_full(0, pos + 1))) break;
+            scores(pos + 1, 0);
+            mma_commit(b_s_full);
           }
-          if (!ok) break;
+          // dS (bf16 at the start of each column half's dP columns)
+          if (!(ok = mbar_wait(b_ds_full, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT)))
+            break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ts(tmem + (kDkDv ? 384 : 256), tmem + 128 + 64 * (k >> 2) + 8 * (k & 3),
+                   m0 + ((k * 2048) >> 4), C::kIdescTS,
+                   (!first || k > 0) ? 1u : 0u);           // dK += dS^T Q  /  dQ += dS K
+          // the step's tiles (and, read by the elementwise warps before
+          // ds_full, its vectors) are free once these products complete
+          mma_commit(b_empty0 + 8 * s0);
+          mma_commit(b_empty1 + 8 * s1);
+          if (!last) {
+            if (!(ok = wait_full(1, pos + 1))) break;
+            scores(pos + 1, 1);
+            mma_commit(b_dp_full);
+          }
           ++nsteps;
           first = false;
-          mma_commit(b_st_empty + 8 * slot);
           ++pos;
         }
         if (!ok) break;
@@ -408,21 +524,18 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
       }
       bool last = false;
       while (!last) {
-        const uint32_t slot = pos % C::kStages;
-        ok = mbar_wait(b_st_full + 8 * slot, (pos / C::kStages) & 1, s_abort, status, tlim,
+        const uint32_t s0 = pos % C::kStages0, s1 = pos % C::kStages1;
+        ok = mbar_wait(b_full0 + 8 * s0, (pos / C::kStages0) & 1, s_abort, status, tlim,
                        EA_ERR_TIMEOUT);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        const BwdStep st = steps[slot];
+        const BwdStep st = steps[s0];
         last = st.last != 0;
-        ++pos;
-        ok = mbar_wait(b_s_full + 8 * half, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        const uint32_t par = nsteps & 1;
+        ok = mbar_wait(b_s_full, par, s_abort, status, tlim, EA_ERR_TIMEOUT);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        const uint32_t step_parity = nsteps & 1;
-        ++nsteps;
         tc_fence_after();
-        const float* vl = vec + slot * 256;
         // visible columns of this row as ranges (branch-free per element):
         // kDkDv (row = key k, column c = query q0 + c): c in [lo_a, hi_a];
         // else (row = query q, column c = key k0 + c): c in [0, hi_a] and
@@ -445,55 +558,67 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
             }
           }
         }
-        uint32_t pp[32], ds[32];
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-        // 32 columns at a time: S (or S^T) and dP (or dP^T) into registers
-        uint32_t sr[32], dr[32];
-        tmem_ld32_wait(tmem + lane_off + col0 + 32 * ch, sr);
-        tmem_ld32_wait(tmem + lane_off + 128 + col0 + 32 * ch, dr);
-        if (ch == 1 && half == 0) mbar_arrive(b_ld_done);   // half 0's columns are read
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int j = 16 * ch + jj;
-          const int c = col0 + 2 * j;
-          float nl0, nl1, nd0, nd1;
+        // phase 1: P kept in registers (and, kDkDv, bf16 P^T at the start of
+        // this half's S columns, all of which this thread has read)
+        float pr[64];
+        {
+          uint32_t pk[32];
+          const float* vl = vec0 + s0 * 128;
+          if (st.full)
+            bwd_phase_p<kDkDv, true>(tmem + lane_off + col0, vl, nl_row, col0, sl2, lo_a, hi_a,
+                                     sink_c, win_c, pr, pk);
+          else
+            bwd_phase_p<kDkDv, false>(tmem + lane_off + col0, vl, nl_row, col0, sl2, lo_a, hi_a,
+                                      sink_c, win_c, pr, pk);
           if (kDkDv) {
-            const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
-            const float2 d2 = *reinterpret_cast<const float2*>(vl + 128 + c);
-            nl0 = l2.x; nl1 = l2.y; nd0 = d2.x; nd1 = d2.y;
-          } else {
-            nl0 = nl1 = nl_row;
-            nd0 = nd1 = nd_row;
+            tmem_st32(tmem + lane_off + col0, pk);
+            tmem_wait_st();
           }
-          float x0 = nl0, x1 = nl1;
-          fma2_acc(x0, x1, __uint_as_float(sr[2 * jj]), __uint_as_float(sr[2 * jj + 1]), sl2, sl2);
-          const bool v0 = c >= lo_a && c <= hi_a && (c < sink_c || c >= win_c);
-          const bool v1 = c + 1 >= lo_a && c + 1 <= hi_a && (c + 1 < sink_c || c + 1 >= win_c);
-          x0 = v0 ? x0 : -INFINITY;
-          x1 = v1 ? x1 : -INFINITY;
-          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          float t0 = nd0, t1 = nd1;
-          add2_acc(t0, t1, __uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1]));
-          float e0 = 0.f, e1 = 0.f;
-          fma2_acc(e0, e1, p0, p1, t0, t1);                 // dS = P (dP - D)
-          ds[j] = pack_bf16x2(e0, e1);
-          if (kDkDv) pp[j] = pack_bf16x2(p0, p1);
         }
-        }
-        // the other column half may still be reading the columns these
-        // stores overwrite
-        // (only half 1's stores land on columns half 0 reads)
-        if (half == 1) {
-          ok = mbar_wait(b_ld_done, step_parity, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        tc_fence_before();
+        mbar_arrive(b_p_full);
+        // phase 2: dS = P (dP - D), bf16 at the start of this half's dP columns
+        if (kDkDv) {   // the step's -D vector comes with tile 1
+          ok = mbar_wait(b_full1 + 8 * s1, (pos / C::kStages1) & 1, s_abort, status, tlim,
+                         EA_ERR_TIMEOUT);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
-        if (kDkDv) tmem_st32(tmem + lane_off + col0 / 2, pp);
-        tmem_st32(tmem + lane_off + 128 + col0 / 2, ds);
-        tmem_wait_st();
+        ++pos;
+        ++nsteps;
+        ok = mbar_wait(b_dp_full, par, s_abort, status, tlim, EA_ERR_TIMEOUT);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          uint32_t ds[32];
+          const float* vd = vec1 + s1 * 128;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t dr[32];
+            tmem_ld32_wait(tmem + lane_off + 128 + col0 + 32 * ch, dr);
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = 16 * ch + jj;
+              const int c = col0 + 2 * j;
+              float t0, t1;
+              if (kDkDv) {
+                const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
+                t0 = d2.x; t1 = d2.y;
+              } else {
+                t0 = t1 = nd_row;
+              }
+              add2_acc(t0, t1, __uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1]));
+              float e0 = 0.f, e1 = 0.f;
+              fma2_acc(e0, e1, pr[2 * j], pr[2 * j + 1], t0, t1);   // dS = P (dP - D)
+              ds[j] = pack_bf16x2(e0, e1);
+            }
+          }
+          tmem_st32(tmem + lane_off + 128 + col0, ds);
+          tmem_wait_st();
+        }
         tc_fence_before();
-        mbar_arrive(b_p_full + 8 * half);
+        mbar_arrive(b_ds_full);
       }
       if (!ok) break;
       // epilogue
