@@ -44,6 +44,16 @@ head h // (Hq // Hkv).
 
 Precision: everything in float64 from inputs the caller has already rounded
 to bf16 (the tests convert the same bf16 tensors the GPU receives).
+
+5. FP8 variant (not on the pages; a throughput variant of the same
+   attention): Q, K, V are stored as e4m3 bytes with one fp32 scale per
+   (batch, head).  What it computes is the attention of section 2/3 over the
+   dequantized values code * scale.  The e4m3 format here is the 8-bit
+   floating-point layout with 1 sign, 4 exponent (bias 7) and 3 mantissa bits,
+   no infinities, the all-ones pattern as NaN, largest finite 448, smallest
+   normal 2^-6 and subnormals m * 2^-9; conversion rounds to nearest, ties to
+   even, and saturates to +-448.  A head is quantized with s = amax / 448 and
+   codes e4m3(x * (448 / amax)), all in fp32.
 """
 from __future__ import annotations
 
@@ -74,6 +84,12 @@ __all__ = [
     "attention_backward",
     "router_gumbel_forward",
     "router_ste_backward",
+    "e4m3_decode",
+    "e4m3_encode",
+    "quantize_e4m3_per_head",
+    "dequantize_e4m3",
+    "attention_fp8",
+    "fp8_p_rounding_bound",
 ]
 
 
@@ -525,3 +541,114 @@ def router_ste_backward(k, w1, b1, w2, b2, g0, g1, tau: float, dout, o_fa, o_sa)
     dx = dpre @ w1
     dk_router = np.broadcast_to((dx / N).reshape(B, Hkv, 1, d), (B, Hkv, N, d)).copy()
     return dr, dz, dw1, db1, dw2, db2, dk_router
+
+
+# --------------------------------------------------------------------------
+# FP8 (e4m3) variant: codec, per-head quantization, reference and the error
+# bound of an e4m3 probability matrix
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 value of each e4m3 byte (NaN for 0x7f / 0xff)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 15) & ((c & 7) == 7), np.nan, val)
+    return sign * val
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """uint8 e4m3 codes of fp32 values: round to nearest, ties to even, magnitudes
+    above 448 saturate to 448; the sign of a zero result is kept."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    neg = np.signbit(x)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    # binade of a (at least the subnormal one, 2^-6 with quantum 2^-9)
+    _, ex = np.frexp(a)                      # a = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)
+    quantum = np.exp2(e - 3.0)
+    v = np.rint(a / quantum) * quantum       # rint: ties to even (448 stays 448)
+    # code: subnormals (and 2^-6 itself) are v / 2^-9; normals (E << 3) | M
+    _, ev = np.frexp(v)
+    en = ev - 1
+    normal = v >= 2.0 ** -6
+    m_norm = np.where(normal, v / np.exp2(en) * 8.0 - 8.0, 0.0)
+    code = np.where(normal, ((en + 7) << 3) + m_norm.astype(np.int64),
+                    (v / 2.0 ** -9).astype(np.int64))
+    code = np.where(np.isnan(x), 0x7F, code)
+    return (code | np.where(neg, 0x80, 0)).astype(np.uint8)
+
+
+def quantize_e4m3_per_head(x):
+    """x: [B, H, N, d] (values already exact in fp32).  Per (b, h): amax =
+    max |x|, inv = 448 / amax and scale = amax / 448 in fp32 (1 and 1 when
+    amax = 0), codes = e4m3(fp32(x * inv)).  Returns (codes uint8, scale
+    float32 [B, H])."""
+    x = np.asarray(x, dtype=np.float32)
+    B, H = x.shape[:2]
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scale = np.empty((B, H), dtype=np.float32)
+    for b in range(B):
+        for h in range(H):
+            amax = np.float32(np.max(np.abs(x[b, h]))) if x[b, h].size else np.float32(0)
+            if amax > 0:
+                inv = np.float32(E4M3_MAX) / amax
+                scale[b, h] = amax / np.float32(E4M3_MAX)
+            else:
+                inv = np.float32(1.0)
+                scale[b, h] = np.float32(1.0)
+            codes[b, h] = e4m3_encode((x[b, h] * inv).astype(np.float32))
+    return codes, scale
+
+
+def dequantize_e4m3(codes, scale) -> np.ndarray:
+    """float64 code * scale, scale per (b, h) of [B, H, N, d] codes."""
+    return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[:, :, None, None]
+
+
+def attention_fp8(q_codes, q_scale, k_codes, k_scale, v_codes, v_scale, mask, sink: int,
+                  window: int, scale: float | None = None) -> np.ndarray:
+    """The FP8 variant's result: the attention of the dequantized Q, K, V."""
+    return attention(dequantize_e4m3(q_codes, q_scale), dequantize_e4m3(k_codes, k_scale),
+                     dequantize_e4m3(v_codes, v_scale), mask, sink, window, scale)
+
+
+def fp8_p_rounding_bound(q, k, v, mask, sink: int, window: int,
+                         scale: float | None = None) -> np.ndarray:
+    """Elementwise bound [B, Hq, N, d] on how far a kernel that rounds the
+    probabilities to e4m3 before the P.V product can be from the exact result.
+
+    Exact weights: w_j = p_j / l with p_j = exp(s_j - m) over the row's
+    visible keys, m the row max and l = sum p_j (>= 1, the max term is 1).
+    The kernel works in a unit c >= 1 (its running reference max is at or
+    below the row max) and forms sum_j e4m3(c p_j) v_j / (c l): the
+    probabilities are rounded, the row sum is not.  e4m3 rounding moves a
+    normal value by at most 2^-4 of itself and a subnormal one by at most
+    2^-10 (half its spacing), so |e4m3(c p_j) - c p_j| <= max(2^-4 c p_j,
+    2^-10) and
+        |out - out*| <= sum_j max(2^-4 w_j, 2^-10 / (c l)) |v_j|
+                     <= sum_j max(2^-4 w_j, 2^-10 / l) |v_j|.
+    Returns that last sum per element."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    g = Hq // k.shape[1]
+    out = np.empty((B, Hq, N, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            p, s = _head_probs(q, k, mask, b, h, sink, window, scale)
+            vis = np.isfinite(s)
+            m = np.max(s, axis=1, keepdims=True)
+            ell = np.sum(np.where(vis, np.exp(s - m), 0.0), axis=1, keepdims=True)
+            per = np.maximum(2.0 ** -4 * p, 2.0 ** -10 / ell)
+            per = np.where(vis, per, 0.0)
+            out[b, h] = per @ np.abs(v[b, h // g])
+    return out

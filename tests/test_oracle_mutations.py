@@ -61,6 +61,16 @@ MUTATIONS = {
                         "dz = dr * r_soft * (1.0 - r_soft)"),
     "ste_relu_mask_dropped": ("dpre = np.where(pre > 0.0, dh, 0.0)", "dpre = dh"),
     "ste_pool_not_divided": ("(dx / N).reshape(B, Hkv, 1, d)", "dx.reshape(B, Hkv, 1, d)"),
+    "e4m3_ties_away": ("v = np.rint(a / quantum) * quantum", "v = np.floor(a / quantum + 0.5) * quantum"),
+    "e4m3_no_saturation": ("a = np.minimum(np.abs(x), E4M3_MAX)", "a = np.abs(x)"),
+    "e4m3_subnormal_quantum": ("e = np.maximum(ex - 1, -6)", "e = np.maximum(ex - 1, -7)"),
+    "e4m3_bias_8": ("(1.0 + m / 8.0) * np.exp2(e - 7.0)", "(1.0 + m / 8.0) * np.exp2(e - 8.0)"),
+    "quant_scale_inverted": ("scale[b, h] = amax / np.float32(E4M3_MAX)",
+                             "scale[b, h] = np.float32(E4M3_MAX) / amax"),
+    "quant_amax_signed": ("amax = np.float32(np.max(np.abs(x[b, h])))", "amax = np.float32(np.max(x[b, h]))"),
+    "fp8_bound_relative_only": ("per = np.maximum(2.0 ** -4 * p, 2.0 ** -10 / ell)", "per = 2.0 ** -4 * p"),
+    "fp8_attention_v_scale_of_k": ("dequantize_e4m3(v_codes, v_scale), mask, sink, window, scale)",
+                                   "dequantize_e4m3(v_codes, k_scale), mask, sink, window, scale)"),
     "ste_diff_sign": ("diff = np.asarray(o_sa, dtype=np.float64) - np.asarray(o_fa",
                       "diff = np.asarray(o_fa, dtype=np.float64) - np.asarray(o_sa"),
 }

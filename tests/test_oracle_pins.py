@@ -493,3 +493,131 @@ def test_gumbel_hard_decision_is_the_soft_argmax():
     # a small temperature makes the soft decision hard
     _, r_cold, _ = oracle.router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, 1e-6)
     np.testing.assert_allclose(r_cold, r_hard, atol=1e-6)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3)
+# The format is fixed by its definition (1 sign, 4 exponent bits with bias 7,
+# 3 mantissa bits, no infinities, 0x7f / 0xff NaN, largest finite 448), not by
+# the pages; the pins below are closed forms of that definition, ties to even
+# at every midpoint, and an independent library conversion.
+
+def test_e4m3_codes_closed_forms():
+    x = np.array([1.0, 0.5, 2.0 ** -6, 2.0 ** -9, 7 * 2.0 ** -9, 448.0, 240.0, 1.125, -3.5,
+                  -0.0, 0.0], np.float32)
+    want = [0x38, 0x30, 0x08, 0x01, 0x07, 0x7E, 0x77, 0x39, 0xC6, 0x80, 0x00]
+    assert oracle.e4m3_encode(x).tolist() == want
+    np.testing.assert_array_equal(oracle.e4m3_decode(np.array(want)), x.astype(np.float64))
+    # saturation: everything above 448 in magnitude stays finite
+    assert oracle.e4m3_encode(np.array([449.0, 464.0, 1e9, -1e30], np.float32)).tolist() == \
+        [0x7E, 0x7E, 0x7E, 0xFE]
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF]))).all()
+
+
+def test_e4m3_round_trip_and_ties_to_even():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    np.testing.assert_array_equal(oracle.e4m3_encode(vals.astype(np.float32)), codes)
+    pos = np.arange(0, 0x7E, dtype=np.int64)            # c and c + 1 both finite, positive
+    lo, hi = oracle.e4m3_decode(pos), oracle.e4m3_decode(pos + 1)
+    mid = ((lo + hi) / 2).astype(np.float32)             # exact in fp32
+    even = np.where(pos % 2 == 0, pos, pos + 1)
+    np.testing.assert_array_equal(oracle.e4m3_encode(mid), even)
+    up = np.nextafter(mid, np.float32(np.inf))
+    down = np.nextafter(mid, np.float32(0))
+    np.testing.assert_array_equal(oracle.e4m3_encode(up), pos + 1)
+    np.testing.assert_array_equal(oracle.e4m3_encode(down), pos)
+
+
+def test_e4m3_encode_matches_library_conversion():
+    rng = np.random.default_rng(80)
+    x = np.concatenate([rng.standard_normal(4000) * 30, rng.standard_normal(2000) * 0.01,
+                        rng.uniform(-448, 448, 2000)]).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_encode(x), lib)
+
+
+def test_quantize_per_head_properties():
+    rng = np.random.default_rng(81)
+    x = (rng.standard_normal((2, 3, 50, 16)) * np.array([1.0, 0.01, 20.0])[None, :, None, None])
+    x = x.astype(np.float32)
+    x[1, 2] = 0.0                                          # an all-zero head
+    codes, scale = oracle.quantize_e4m3_per_head(x)
+    for b in range(2):
+        for h in range(3):
+            amax = np.abs(x[b, h]).max()
+            if amax == 0:
+                assert scale[b, h] == 1.0 and not codes[b, h].any()
+                continue
+            assert scale[b, h] == np.float32(amax) / np.float32(448)
+            # the largest magnitude maps to the largest code
+            i = np.unravel_index(np.argmax(np.abs(x[b, h])), x[b, h].shape)
+            assert codes[b, h][i] & 0x7F == 0x7E
+    deq = oracle.dequantize_e4m3(codes, scale)
+    err = np.abs(deq - x)
+    # relative 2^-4 in the normal range, half a subnormal step below it
+    s = scale.astype(np.float64)[:, :, None, None]
+    bound = np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * s) * (1 + 1e-6)
+    assert np.all(err <= bound)
+
+
+@pytest.mark.parametrize("S,W", [(4, 16), (0, 3)])
+def test_fp8_bound_holds_for_a_simulated_kernel(S, W):
+    """A numpy model of the kernel's arithmetic (probabilities in a unit c >=
+    1, rounded to e4m3, unrounded row sum) stays within the bound, and the
+    bound is far from vacuous."""
+    rng = np.random.default_rng(82 + S)
+    B, Hq, Hkv, N, d = 1, 2, 1, 96, 8
+    q = rng.standard_normal((B, Hq, N, d)) * 2.5
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    mask = np.array([[0, 1]], np.uint8)
+    ref = oracle.attention(q, k, v, mask, S, W)
+    bound = oracle.fp8_p_rounding_bound(q, k, v, mask, S, W)
+    scale = 1.0 / math.sqrt(d)
+    for h in range(Hq):
+        for i in range(N):
+            keys = oracle.visible_keys(i, bool(mask[0, h]), S, W)
+            s = (k[0, 0, keys] @ q[0, h, i]) * scale
+            p = np.exp(s - s.max())
+            c = 2.0 ** rng.uniform(0, 8)                  # the kernel's unit
+            pq = oracle.e4m3_decode(oracle.e4m3_encode((p * c).astype(np.float32))) / c
+            out = (pq @ v[0, 0, keys]) / p.sum()
+            assert np.all(np.abs(out - ref[0, h, i]) <= bound[0, h, i] + 1e-12), (h, i)
+    assert bound.mean() < 0.1 * np.abs(v).mean()
+
+
+def test_fp8_bound_covers_flushed_probabilities():
+    """One dominant key and 90 keys at p = 2^-11, which e4m3 flushes to zero
+    in the unit c = 1: the error is the whole mass of those keys, which only
+    the absolute (subnormal) term of the bound covers."""
+    N = 91
+    q = np.ones((1, 1, N, 1))
+    k = np.full((1, 1, N, 1), math.log(2.0 ** -11))
+    k[0, 0, 0, 0] = 0.0
+    v = np.full((1, 1, N, 1), 10.0)
+    v[0, 0, 0, 0] = 0.0
+    mask = np.zeros((1, 1), np.uint8)
+    ref = oracle.attention(q, k, v, mask, 0, 1, scale=1.0)
+    bound = oracle.fp8_p_rounding_bound(q, k, v, mask, 0, 1, scale=1.0)
+    s = k[0, 0, :, 0]
+    p = np.exp(s - s.max())
+    pq = oracle.e4m3_decode(oracle.e4m3_encode(p.astype(np.float32)))
+    out = (pq @ v[0, 0, :, 0]) / p.sum()
+    err = abs(out - ref[0, 0, N - 1, 0])
+    assert err > 0.4                                   # the flushed mass
+    assert err <= bound[0, 0, N - 1, 0]
+
+
+def test_attention_fp8_dequantizes_before_attending():
+    rng = np.random.default_rng(83)
+    x = rng.standard_normal((3, 1, 2, 40, 8)).astype(np.float32)
+    (qc, qs), (kc, ks), (vc, vs) = (oracle.quantize_e4m3_per_head(t) for t in x)
+    mask = np.array([[0, 1]], np.uint8)
+    # SA heads with S = 0, W = 1: every row attends to itself only, so out is
+    # the dequantized v
+    out = oracle.attention_fp8(qc, qs, kc, ks, vc, vs, np.ones_like(mask), 0, 1)
+    np.testing.assert_allclose(out, oracle.dequantize_e4m3(vc, vs), rtol=0, atol=1e-12)
+    full = oracle.attention_fp8(qc, qs, kc, ks, vc, vs, mask, 2, 5)
+    ref = oracle.attention(oracle.dequantize_e4m3(qc, qs), oracle.dequantize_e4m3(kc, ks),
+                           oracle.dequantize_e4m3(vc, vs), mask, 2, 5)
+    np.testing.assert_allclose(full, ref, rtol=0, atol=0)
