@@ -68,6 +68,10 @@ def parse_args():
                     action="store_true",
                     help="run only the training-step measurement (router, both-mode "
                          "forward, backward, router gradients)")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the FP8-variant measurement of the default line")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="run only the FP8-variant measurement and print its JSON object")
     ap.add_argument("--no-training", action="store_true",
                     help="skip the training-step measurement of the default line")
     ap.add_argument("--packed-only", action="store_true",
@@ -418,10 +422,98 @@ def run_ours(args, rank, world, local_rank):
     if not args.quick and world == 1 and args.decode_batch > 0:
         result["decode"] = measure_decode(w, args.decode_batch, max(args.steps, 10),
                                           max(args.warmup, 3), dev, stream)
+    if not args.quick and world == 1 and not args.no_fp8 and w.d == 128:
+        result["fp8"] = measure_fp8(w, max(args.steps, 5), max(args.warmup, 3), dev, stream)
     if not args.quick and world == 1 and not args.no_training:
         result["training"] = measure_training(w, max(args.steps, 5), max(args.warmup, 3), dev,
                                               stream)
     return result
+
+
+# ---------------------------------------------------------------- FP8 variant
+def measure_fp8(w: workloads.Workload, steps: int, warmup: int, dev, stream):
+    """The FP8 (e4m3) variant of the fused attention on the same layer: Q, K, V
+    quantized per head once (the quantization timed on its own), then the
+    attention timed with CUDA events on resident e4m3 inputs; the bf16 kernel
+    on the same layer and mask beside it."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (ea_get_device_status, ea_hybrid_attn_prefill,
+                                                ea_hybrid_attn_prefill_fp8, ea_quantize_fp8)
+    B, Hq, Hkv, N, d, S, W = w.batch, w.hq, w.hkv, w.seq, w.d, w.sink, w.window
+    seed = workloads.layer_seed(w, 0)
+    q, k, v = workloads.make_qkv(w, seed, device=dev)
+    heads = workloads.sparse_head_set(Hq, workloads.layer_sparse_frac(w, 0), seed)
+    mask_h = np.zeros((B, Hq), np.uint8)
+    mask_h[:, heads] = 1
+    mask = torch.as_tensor(mask_h, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    qw = torch.empty(1 << 16, dtype=torch.uint8, device=dev)
+
+    def quant():
+        a = ea_quantize_fp8(q, workspace=qw, stream=stream)
+        b = ea_quantize_fp8(k, workspace=qw, stream=stream)
+        c = ea_quantize_fp8(v, transpose=True, workspace=qw, stream=stream)
+        return a, b, c
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    with torch.cuda.stream(stream):
+        (q8, qs), (k8, ks), (vt8, vs) = quant()
+
+        def fp8():
+            ea_hybrid_attn_prefill_fp8(q8, k8, vt8, qs, ks, vs, mask, S, W, out=out,
+                                       workspace=ws, stream=stream)
+
+        def bf16():
+            ea_hybrid_attn_prefill(q, k, v, mask, S, W, out=out, workspace=ws, stream=stream)
+
+        for _ in range(warmup):
+            quant()
+            fp8()
+            bf16()
+        torch.cuda.synchronize()
+        q_ms = timed(quant, steps)
+        f_ms = timed(fp8, steps)
+        b_ms = timed(bf16, steps)
+    if ea_get_device_status(ws) != 0:
+        raise RuntimeError("attention status word reports an error")
+    eff = flops.effective_flops(mask_h, N, d, S, W)
+    peaks, src = load_peaks()
+    peak8 = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tf = eff / (f_ms * 1e-3) / 1e12
+    # quantization bytes: bf16 read twice (amax, then convert), e4m3 written once
+    nval = (B * Hq + 2 * B * Hkv) * N * d
+    qbytes = nval * (2 + 2 + 1)
+    return {
+        "workload": f"{w.name} FP8 (e4m3 Q/K/V, per-head scales) prefill: B={B} Hq={Hq} "
+                    f"Hkv={Hkv} N={N} d={d} S={S} W={W}, SA heads {mask_h.mean():.2f}",
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": round(f_ms, 4),
+        "effective_tflops": round(tf, 2),
+        "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": round(peak8, 1),
+                     "unit": "TFLOP/s", "frac": round(tf / peak8, 4),
+                     "peak_source": f"{src} bf16_tflops (burst) x 2, the nominal e4m3/bf16 "
+                                    "dense ratio",
+                     "scope": "fused FP8 attention kernel, effective flops"},
+        "bf16_ms_per_step": round(b_ms, 4),
+        "speedup_vs_bf16": round(b_ms / f_ms, 3),
+        "quantize_ms": round(q_ms, 4),
+        "quantize_gbs": round(qbytes / (q_ms * 1e-3) / 1e9, 1),
+        "quantize_hbm_frac": round(qbytes / (q_ms * 1e-3) / 1e9 / hbm, 4),
+        "gpu_launches_per_step": 1,
+        "l2": (f"e4m3 inputs {(B * Hq + 2 * B * Hkv) * N * d / 1e6:.0f} MB "
+               + ("exceed L2 (126 MB), no flush" if (B * Hq + 2 * B * Hkv) * N * d > 126e6
+                  else "fit in L2 (126 MB): timed warm")),
+    }
 
 
 # ---------------------------------------------------------------- packed batches
@@ -845,6 +937,16 @@ def main():
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.fp8_only:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = measure_fp8(w, args.steps, max(args.warmup, 3), dev, torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
         return 0
     if args.training_only:
         dev = torch.device("cuda", local_rank)

@@ -248,6 +248,45 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * FP8 (e4m3) variant of the fused attention.  Not on the pages: the same
+ * attention (FA causal, SA sink + window, one launch) over inputs stored as
+ * e4m3 bytes with one fp32 dequantization scale per (batch, head); what it
+ * computes is the attention of code * scale.  e4m3: 1 sign, 4 exponent bits
+ * (bias 7), 3 mantissa bits, largest finite 448, subnormals m * 2^-9.
+ *
+ * ea_quantize_fp8: x device bf16 [heads][N][d] (heads = B * H, d = 128).
+ *   Per head, amax = max |x|, scale[h] = amax / 448 and every value becomes
+ *   e4m3(x * (448 / amax)) (fp32 arithmetic, round to nearest even,
+ *   saturating); an all-zero head gets scale 1.  transpose = 0 writes codes
+ *   [heads][N][d]; transpose = 1 writes [heads][d][ea_fp8_vt_stride(N)] (the
+ *   layout the attention reads V in; positions >= N are zero).  scale: device
+ *   fp32 [heads].  workspace >= ea_quantize_fp8_workspace_size(heads) bytes
+ *   (per-head amax, reset by the call).  Deterministic (max is order-free).
+ *
+ * ea_hybrid_attn_prefill_fp8: q8 [B][Hq][N][128], k8 [B][Hkv][N][128] and
+ *   vt8 [B][Hkv][128][ea_fp8_vt_stride(N)] e4m3 codes (as ea_quantize_fp8
+ *   writes them), q_scale [B*Hq], k_scale and v_scale [B*Hkv] fp32, all device;
+ *   out bf16 [B][Hq][N][128].  Both products run on the tensor cores as
+ *   e4m3 x e4m3 -> fp32; the probabilities are rounded to e4m3 for the P.V
+ *   product (the row sum is not), so results are within the e4m3 rounding of
+ *   P of the exact attention of the dequantized inputs.  Params, mask,
+ *   workspace and status as for ea_hybrid_attn_prefill; d must be 128; padded
+ *   batches only.
+ * ---------------------------------------------------------------------- */
+int ea_fp8_vt_stride(int N);
+
+size_t ea_quantize_fp8_workspace_size(int heads);
+
+ea_status ea_quantize_fp8(const void* x, int heads, int N, int d, int transpose, void* codes,
+                          float* scale, void* workspace, size_t workspace_bytes, void* stream);
+
+ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void* vt8,
+                                     const float* q_scale, const float* k_scale,
+                                     const float* v_scale, const uint8_t* route_mask,
+                                     const ea_attn_params* p, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Router training (EA blog §2.1, training trick: the binary routing is made
  * differentiable with Gumbel-Softmax and a straight-through estimator).
  *

@@ -90,6 +90,7 @@ __all__ = [
     "dequantize_e4m3",
     "attention_fp8",
     "fp8_p_rounding_bound",
+    "fp8_p_rounding_bound_rows",
 ]
 
 
@@ -651,4 +652,26 @@ def fp8_p_rounding_bound(q, k, v, mask, sink: int, window: int,
             per = np.maximum(2.0 ** -4 * p, 2.0 ** -10 / ell)
             per = np.where(vis, per, 0.0)
             out[b, h] = per @ np.abs(v[b, h // g])
+    return out
+
+
+def fp8_p_rounding_bound_rows(q, k, v, mask, b: int, h: int, rows, sink: int, window: int,
+                              scale: float | None = None) -> np.ndarray:
+    """fp8_p_rounding_bound for the listed query rows of head (b, h) only
+    ([len(rows), d]), computed row by row from the visible keys."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    g = Hq // np.asarray(k).shape[1]
+    kh = np.asarray(k[b, h // g], dtype=np.float64)
+    vh = np.asarray(v[b, h // g], dtype=np.float64)
+    out = np.empty((len(rows), d), dtype=np.float64)
+    for r, i in enumerate(rows):
+        keys = visible_keys(int(i), bool(mask[b, h]), sink, window)
+        s = (kh[keys] @ q[b, h, i]) * scale
+        e = np.exp(s - np.max(s))
+        ell = np.sum(e)
+        per = np.maximum(2.0 ** -4 * e / ell, 2.0 ** -10 / ell)
+        out[r] = per @ np.abs(vh[keys])
     return out

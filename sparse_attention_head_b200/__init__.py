@@ -17,5 +17,6 @@ from .api import (HostPrefill, attn_workspace, decode_workspace, ea_decode_kv_po
                   make_varlen_params, ea_router_decide_varlen, ea_hybrid_attn_prefill_routed,
                   ea_hybrid_attn_prefill_varlen_routed, ea_hybrid_attn_prefill_lse,
                   ea_hybrid_attn_backward, ea_router_decide_gumbel, ea_router_ste_backward,
-                  ea_hybrid_attn_prefill_train)
+                  ea_hybrid_attn_prefill_train, ea_quantize_fp8, ea_hybrid_attn_prefill_fp8,
+                  ea_fp8_vt_stride)
 from .flops import attn_visible_pairs, effective_flops, tile_flops  # noqa: F401

@@ -42,7 +42,8 @@ EXPORTED = [
     "ea_hybrid_attn_prefill_lse", "ea_hybrid_attn_backward_workspace_size",
     "ea_hybrid_attn_backward", "ea_router_gumbel_workspace_size", "ea_router_decide_gumbel",
     "ea_router_ste_backward_workspace_size", "ea_router_ste_backward",
-    "ea_hybrid_attn_prefill_train",
+    "ea_hybrid_attn_prefill_train", "ea_fp8_vt_stride", "ea_quantize_fp8_workspace_size",
+    "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8",
 ]
 
 
@@ -143,6 +144,15 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
                                                          c_size, vp]
     lib.ea_hybrid_attn_prefill_lse.restype = c_int
     lib.ea_hybrid_attn_prefill_lse.argtypes = [vp, vp, vp, vp, pparams, vp, vp, vp, c_size, vp]
+    lib.ea_fp8_vt_stride.restype = c_int
+    lib.ea_fp8_vt_stride.argtypes = [c_int]
+    lib.ea_quantize_fp8_workspace_size.restype = c_size
+    lib.ea_quantize_fp8_workspace_size.argtypes = [c_int]
+    lib.ea_quantize_fp8.restype = c_int
+    lib.ea_quantize_fp8.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, vp, c_size, vp]
+    lib.ea_hybrid_attn_prefill_fp8.restype = c_int
+    lib.ea_hybrid_attn_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, pparams, vp, vp, c_size,
+                                               vp]
     lib.ea_hybrid_attn_prefill_train.restype = c_int
     lib.ea_hybrid_attn_prefill_train.argtypes = [vp, vp, vp, vp, pparams, vp, vp, vp, vp, c_size,
                                                  vp]

@@ -397,6 +397,77 @@ def ea_hybrid_attn_prefill_train(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     return out, lse, out_other
 
 
+# ---------------------------------------------------------------- FP8
+def ea_fp8_vt_stride(N: int) -> int:
+    """Row stride (bytes) of the transposed e4m3 V layout: N rounded up to 16."""
+    return int(_lib.load().ea_fp8_vt_stride(int(N)))
+
+
+def ea_quantize_fp8(x: torch.Tensor, transpose: bool = False, *,
+                    codes: Optional[torch.Tensor] = None, scale: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """Per-head e4m3 quantization of bf16 x [B, H, N, d]: (codes uint8
+    [B, H, N, d], or [B, H, d, ea_fp8_vt_stride(N)] when transposed; scale
+    fp32 [B, H])."""
+    lib = _lib.load()
+    _need(x, "x", torch.bfloat16, 4)
+    B, H, N, d = x.shape
+    dev = x.device
+    shape = (B, H, d, ea_fp8_vt_stride(N)) if transpose else (B, H, N, d)
+    if codes is None:
+        codes = torch.empty(shape, dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _need(codes, "codes", torch.uint8, 4)
+    _need(scale, "scale", torch.float32)
+    if tuple(codes.shape) != shape or scale.numel() != B * H:
+        raise ValueError("codes / scale buffers do not match x")
+    if workspace is None:
+        workspace = torch.empty(int(lib.ea_quantize_fp8_workspace_size(B * H)), dtype=torch.uint8,
+                                device=dev)
+    rc = lib.ea_quantize_fp8(x.data_ptr(), B * H, N, d, 1 if transpose else 0, codes.data_ptr(),
+                             scale.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                             _stream_ptr(stream, dev))
+    check(rc, "ea_quantize_fp8")
+    return codes, scale
+
+
+def ea_hybrid_attn_prefill_fp8(q8: torch.Tensor, k8: torch.Tensor, vt8: torch.Tensor,
+                               q_scale: torch.Tensor, k_scale: torch.Tensor,
+                               v_scale: torch.Tensor, route_mask: torch.Tensor, sink: int,
+                               window: int, *, softmax_scale: float = 0.0,
+                               select: int = EA_SELECT_ALL, out: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None,
+                               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The fused attention over e4m3 inputs (as ea_quantize_fp8 writes them):
+    out bf16 [B, Hq, N, d]."""
+    lib = _lib.load()
+    for name, t in (("q8", q8), ("k8", k8), ("vt8", vt8)):
+        _need(t, name, torch.uint8, 4)
+    for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+        _need(t, name, torch.float32)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q8.shape
+    Hkv = k8.shape[1]
+    if tuple(k8.shape) != (B, Hkv, N, d) or tuple(vt8.shape) != (B, Hkv, d, ea_fp8_vt_stride(N)):
+        raise ValueError("k8 / vt8 shapes do not match q8")
+    if q_scale.numel() != B * Hq or k_scale.numel() != B * Hkv or v_scale.numel() != B * Hkv:
+        raise ValueError("one scale per (batch, head) is required")
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale, select)
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q8.device)
+    if workspace is None:
+        workspace = attn_workspace(p, q8.device)
+    rc = lib.ea_hybrid_attn_prefill_fp8(q8.data_ptr(), k8.data_ptr(), vt8.data_ptr(),
+                                        q_scale.data_ptr(), k_scale.data_ptr(),
+                                        v_scale.data_ptr(), route_mask.data_ptr(),
+                                        ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel(), _stream_ptr(stream, q8.device))
+    check(rc, "ea_hybrid_attn_prefill_fp8")
+    return out
+
+
 def ea_hybrid_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                             out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
                             route_mask: torch.Tensor, sink: int, window: int, *,

@@ -124,6 +124,23 @@ bool encode_bhsd(CUtensorMap* m, const void* ptr, int d, int n, int rows3) {
   return r == CUDA_SUCCESS;
 }
 
+// e4m3 bytes as a 3-D tensor (inner, rows, planes) with the given row and
+// plane strides in bytes; box 128 x 128 x 1 (128-byte rows), 128-byte swizzle.
+bool encode_u8(CUtensorMap* m, const void* ptr, int inner, int rows, int planes,
+               uint64_t row_stride, uint64_t plane_stride) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {row_stride, plane_stride};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Packed [T][heads][d] memory as a (d, T, heads) tensor: tokens step by
 // heads * d elements, heads by d; the same 64 x 128 x 1 box.
 bool encode_packed(CUtensorMap* m, const void* ptr, int d, int total, int heads) {
@@ -492,6 +509,72 @@ ea_status ea_hybrid_attn_prefill_train(const void* q, const void* k, const void*
   if (!out_other) return EA_ERR_INVALID_ARG;
   return prefill_train(q, k, v, route_mask, p, out, lse, out_other, workspace, workspace_bytes,
                        stream);
+}
+
+// ---------------------------------------------------------------- FP8
+int ea_fp8_vt_stride(int N) { return N > 0 ? ea::fp8_npad(N) : 0; }
+
+size_t ea_quantize_fp8_workspace_size(int heads) {
+  return heads > 0 ? ea::fp8_quant_workspace_bytes(heads) : 0;
+}
+
+ea_status ea_quantize_fp8(const void* x, int heads, int N, int d, int transpose, void* codes,
+                          float* scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !codes || !scale || heads <= 0 || N <= 0 || d <= 0) return EA_ERR_INVALID_ARG;
+  if (transpose != 0 && transpose != 1) return EA_ERR_INVALID_ARG;
+  if (d != 128) return EA_ERR_UNSUPPORTED;
+  if (N > kMaxSeqLen || static_cast<long long>(heads) > 65535) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes)) return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < ea_quantize_fp8_workspace_size(heads))
+    return EA_ERR_WORKSPACE;
+  const cudaError_t err = ea::launch_fp8_quant(x, heads, N, d, transpose, codes, scale, workspace,
+                                               static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void* vt8,
+                                     const float* q_scale, const float* k_scale,
+                                     const float* v_scale, const uint8_t* route_mask,
+                                     const ea_attn_params* p, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (!q8 || !k8 || !vt8 || !q_scale || !k_scale || !v_scale || !route_mask || !out)
+    return EA_ERR_INVALID_ARG;
+  if (p->d != 128) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(vt8) || !aligned16(out))
+    return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < kAttnWorkspace) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  const uint64_t npad = static_cast<uint64_t>(ea::fp8_npad(p->N));
+  const uint64_t d = static_cast<uint64_t>(p->d);
+  ea::AttnArgs args = {};
+  if (!encode_u8(&args.tm_q, q8, p->d, p->N, p->B * p->Hq, d, d * p->N) ||
+      !encode_u8(&args.tm_k, k8, p->d, p->N, p->B * p->Hkv, d, d * p->N) ||
+      !encode_u8(&args.tm_v, vt8, p->N, p->d, p->B * p->Hkv, npad, npad * d))
+    return EA_ERR_CUDA;
+  args.mask = route_mask;
+  args.out = out;
+  args.q_scale = q_scale;
+  args.k_scale = k_scale;
+  args.v_scale = v_scale;
+  args.status = static_cast<int*>(workspace);
+  args.B = p->B;
+  args.Hq = p->Hq;
+  args.Hkv = p->Hkv;
+  args.N = p->N;
+  args.sink = p->sink;
+  args.window = p->window;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->d));
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.select = p->select;
+  args.timeout_ns = wait_timeout_ns();
+  args.debug_drop_kv_pos = -1;
+  const int sms = device_sms();
+  if (sms <= 0) return EA_ERR_CUDA;
+  const cudaError_t err = ea::launch_attn_fp8(args, ea_attn_grid_size(p, sms),
+                                              static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
 size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p) {

@@ -48,15 +48,21 @@ namespace ea {
 // FMA pipe instead of the MUFU (the two units then share the work).
 constexpr int kEmuPairs = 0;
 
-template <int D>
+// kFp8: q, k as e4m3 rows of d bytes; v transposed (d rows of keys); both
+// products of kind::f8f6f4 with P rounded to e4m3 (d = 128 only).
+template <int D, bool kFp8 = false>
 struct AttnCfg {
   static constexpr int kThreads = 384;
   static constexpr uint32_t kRegsSoftmax = 192;
   static constexpr uint32_t kRegsOther = 120;
-  static constexpr int kBlockBytes = 128 * 128;             // 128 rows x 64 bf16
-  static constexpr int kDBlocks = D / 64;                   // 128-byte column blocks
-  static constexpr int kTileBytes = 128 * D * 2;            // one Q slot / K / V tile
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kElem = kFp8 ? 1 : 2;                // bytes per value
+  static constexpr int kBlockBytes = 128 * 128;             // 128 rows x 128 bytes
+  static constexpr int kBlockElems = 128 / kElem;           // values per 128-byte row
+  static constexpr int kDBlocks = D * kElem / 128;          // 128-byte column blocks
+  static constexpr int kTileBytes = 128 * D * kElem;        // one Q slot / K / V tile
+  static constexpr int kStages = (kTileBytes == 32768) ? 4 : 8;
+  static constexpr int kKSteps = D * kElem / 32;            // S product: 32 bytes of K each
+  static constexpr int kPVSteps = 128 * kElem / 32;         // P.V product: 32 bytes of keys each
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
@@ -75,8 +81,12 @@ struct AttnCfg {
   static constexpr int kOffP = kOffOrder + EA_MAX_SEQS * 2;
   static constexpr int kSmem = kOffP + EA_MAX_SEQS * 2 + 1024;  // + alignment slack
   static_assert(kSmem <= 232448, "shared memory per CTA");
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
-  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+  static constexpr uint32_t kIdescS =
+      kFp8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
+  // bf16: V [keys][d] is an MN-major B; e4m3: V^T [d][keys] is K-major
+  static constexpr uint32_t kIdescPV =
+      kFp8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
+  static_assert(!kFp8 || D == 128, "the FP8 variant is built for d = 128");
 };
 
 // Shared-memory addresses (32-bit) of the kernel's mbarriers; the arrays
@@ -182,9 +192,9 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
   return grid_sync(args, s_flag);
 }
 
-template <int D, bool kRouted>
+template <int D, bool kRouted, bool kFp8 = false>
 __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
-  using C = AttnCfg<D>;
+  using C = AttnCfg<D, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -386,7 +396,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         for (int s = 0; s < ut.nslots; ++s)
           for (int c = 0; c < C::kDBlocks; ++c)
             tma_load_3d(smem_u32(sQ) + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
-                        c * 64, tok + ut.r0 + s * EA_BM, qz);
+                        c * C::kBlockElems, tok + ut.r0 + s * EA_BM, qz);
         ++n_units;
         for (int i = 0; i < ut.n && ok; ++i) {
           const int t = ea_tile_at(ut, i);
@@ -403,9 +413,15 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
             }
             mbar_arrive_expect_tx(bars.kv_full + 8 * st, C::kTileBytes);
             const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
-            for (int c = 0; c < C::kDBlocks; ++c)
-              tma_load_3d(smem_u32(sKV) + st * C::kTileBytes + c * C::kBlockBytes, map, bars.kv_full + 8 * st,
-                          c * 64, tok + t * EA_BN, kvz);
+            if (kFp8 && which) {
+              // V^T: the tile's 128 keys along the row, all d rows
+              tma_load_3d(smem_u32(sKV) + st * C::kTileBytes, map, bars.kv_full + 8 * st,
+                          tok + t * EA_BN, 0, kvz);
+            } else {
+              for (int c = 0; c < C::kDBlocks; ++c)
+                tma_load_3d(smem_u32(sKV) + st * C::kTileBytes + c * C::kBlockBytes, map,
+                            bars.kv_full + 8 * st, c * C::kBlockElems, tok + t * EA_BN, kvz);
+            }
             ++kv_pos;
           }
         }
@@ -443,17 +459,28 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         const uint64_t a0 = dq + ((s * C::kTileBytes) >> 4);
         const uint64_t b0 = dkv_k + ((st * C::kTileBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < C::kKSteps; ++k) {
           const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
-          mma_ss(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
+          if (kFp8)
+            mma_ss_f8(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
         }
       };
+      // P from TMEM (32 bytes of keys = 8 columns per K step); B: bf16 V
+      // MN-major (16 key rows per step), or e4m3 V^T K-major (32 key bytes)
       auto issue_pv = [&](int s, uint32_t st, bool acc) {
-        const uint64_t b0 = dkv_v + ((st * C::kTileBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < EA_BN / 16; ++k)
-          mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8, b0 + ((k * 2048) >> 4),
-                 C::kIdescPV, (acc || k > 0) ? 1u : 0u);
+        for (int k = 0; k < C::kPVSteps; ++k) {
+          if (kFp8)
+            mma_ts_f8(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
+                      dkv_k + ((st * C::kTileBytes + k * 32) >> 4), C::kIdescPV,
+                      (acc || k > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
+                   dkv_v + ((st * C::kTileBytes + k * 2048) >> 4), C::kIdescPV,
+                   (acc || k > 0) ? 1u : 0u);
+        }
       };
       EaCursor cur;
       ea_cursor_init(cur, view);
@@ -550,7 +577,6 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + slot * 128;
     const uint32_t tO = tmem + lane_off + 256 + slot * 128;
-    const float sl2 = args.scale_log2;
     uint32_t s_cnt = 0;
     uint32_t pv_cnt = 0;
     bool ok = true;
@@ -568,6 +594,10 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
       if (slot >= ut.nslots) continue;
       const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
+      // FP8: the scores carry the q and k dequantization scales
+      const int kvh = seq * args.Hkv + (idx % args.Hq) / G;
+      const float sl2 = kFp8 ? args.scale_log2 * args.q_scale[idx] * args.k_scale[kvh]
+                             : args.scale_log2;
       float m_ref = -INFINITY;
       float l = 0.f;
       bool has_o = false;
@@ -626,6 +656,24 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         float acc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        if constexpr (kFp8) {
+          // e4m3 P, four keys per column (32 columns); the row sum adds the
+          // unrounded values
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float p0, p1, p2, p3;
+            fma2_sc(p0, p1, x[4 * j], x[4 * j + 1], sl2, -msub);
+            fma2_sc(p2, p3, x[4 * j + 2], x[4 * j + 3], sl2, -msub);
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
+            p2 = ex2_approx(p2);
+            p3 = ex2_approx(p3);
+            pk[j] = pack_e4m3x4(p0, p1, p2, p3);
+            add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], p0 + p2, p1 + p3);
+          }
+          tmem_st32(tS, pk);
+        } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -646,6 +694,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                      __uint_as_float(pk[j] & 0xffff0000u));
           }
           tmem_st16(tS + c * 16, pk);
+        }
         }
         l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         if (__any_sync(0xffffffffu, rescale)) {
@@ -676,7 +725,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = kFp8 ? args.v_scale[kvh] / l : 1.f / l;
       // a training forward's other mode goes to out_other, without lse
       const bool chosen = !args.both || (sparse != 0) == (ld_mask(args.mask, idx) != 0);
       if (chosen && args.lse != nullptr && !packed && row < seq_len)   // for the backward
@@ -722,21 +771,21 @@ int attn_smem_bytes(int D) {
   return D == 128 ? AttnCfg<128>::kSmem : AttnCfg<64>::kSmem;
 }
 
-template <int D, bool kRouted>
+template <int D, bool kRouted, bool kFp8 = false>
 static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream) {
-  const int smem = AttnCfg<D>::kSmem;
+  const int smem = AttnCfg<D, kFp8>::kSmem;
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev >= 64 || !configured[dev]) {
-    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D, kRouted>,
+    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D, kRouted, kFp8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     if (dev < 64) configured[dev] = 1;
   }
   if (!kRouted) {
-    ea_hybrid_attn_kernel<D, false><<<grid, AttnCfg<D>::kThreads, smem, stream>>>(args);
+    ea_hybrid_attn_kernel<D, false, kFp8><<<grid, AttnCfg<D, kFp8>::kThreads, smem, stream>>>(args);
     return cudaGetLastError();
   }
   // every CTA must be resident at once: the runtime refuses a cooperative
@@ -750,6 +799,10 @@ cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stre
   if (D == 128) return launch_d<128, false>(args, grid, stream);
   if (D == 64) return launch_d<64, false>(args, grid, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_fp8(const AttnArgs& args, int grid, cudaStream_t stream) {
+  return launch_d<128, false, true>(args, grid, stream);
 }
 
 cudaError_t launch_attn_routed(int D, const AttnArgs& args, int grid, cudaStream_t stream) {

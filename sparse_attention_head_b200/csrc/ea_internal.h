@@ -28,6 +28,11 @@ struct alignas(64) AttnArgs {
   // the mask chooses goes to `out` (and `lse`), the other one to out_other.
   void* out_other;
   int both;
+  // FP8 variant (q, k e4m3 BHSD, v e4m3 transposed [B*Hkv][d][Npad]): the
+  // per-(batch, head) dequantization scales of q, k and v.
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
   int B, Hq, Hkv, N;
   int sink, window;
   float scale_log2;         // softmax scale * log2(e)
@@ -85,6 +90,15 @@ cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stre
 // The routed kernel (router in the prologue), as a cooperative launch: all
 // CTAs resident at once (they meet at grid barriers), or an error.
 cudaError_t launch_attn_routed(int D, const AttnArgs& args, int grid, cudaStream_t stream);
+// The FP8 variant of the fused kernel (d = 128, not routed).
+cudaError_t launch_attn_fp8(const AttnArgs& args, int grid, cudaStream_t stream);
+
+// bf16 -> e4m3 per-head quantization (x: [heads][N][d], d = 128): codes
+// [heads][N][d], or transposed [heads][d][fp8_npad(N)]; scale [heads].
+int fp8_npad(int N);
+size_t fp8_quant_workspace_bytes(int heads);
+cudaError_t launch_fp8_quant(const void* x, int heads, int N, int d, int transpose, void* codes,
+                             float* scale, void* workspace, cudaStream_t stream);
 
 // Router: pooled partial sums, then the MLP and the threshold.
 int router_num_splits(int B, int Hkv, int N);

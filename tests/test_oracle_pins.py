@@ -621,3 +621,17 @@ def test_attention_fp8_dequantizes_before_attending():
     ref = oracle.attention(oracle.dequantize_e4m3(qc, qs), oracle.dequantize_e4m3(kc, ks),
                            oracle.dequantize_e4m3(vc, vs), mask, 2, 5)
     np.testing.assert_allclose(full, ref, rtol=0, atol=0)
+
+
+def test_fp8_bound_rows_equals_the_dense_bound():
+    rng = np.random.default_rng(84)
+    q = rng.standard_normal((1, 4, 70, 8))
+    k = rng.standard_normal((1, 2, 70, 8))
+    v = rng.standard_normal((1, 2, 70, 8))
+    mask = np.array([[0, 1, 0, 1]], np.uint8)
+    dense = oracle.fp8_p_rounding_bound(q, k, v, mask, 3, 9)
+    rows = [0, 1, 5, 9, 12, 69]
+    for h in range(4):
+        np.testing.assert_allclose(
+            oracle.fp8_p_rounding_bound_rows(q, k, v, mask, 0, h, rows, 3, 9), dense[0, h, rows],
+            rtol=1e-12, atol=1e-15)
