@@ -47,6 +47,9 @@ namespace ea {
 // Of every 8 exp2 pairs of a score row, this many run as a polynomial on the
 // FMA pipe instead of the MUFU (the two units then share the work).
 constexpr int kEmuPairs = 0;
+// The same for the FP8 variant, per 8 groups of four scores: its MUFU pipe
+// also carries the e4m3 conversions.
+constexpr int kEmuQuadsFp8 = 2;
 
 // kFp8: q, k as e4m3 rows of d bytes; v transposed (d rows of keys); both
 // products of kind::f8f6f4 with P rounded to e4m3 (d = 128 only).
@@ -665,10 +668,15 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
             float p0, p1, p2, p3;
             fma2_sc(p0, p1, x[4 * j], x[4 * j + 1], sl2, -msub);
             fma2_sc(p2, p3, x[4 * j + 2], x[4 * j + 3], sl2, -msub);
-            p0 = ex2_approx(p0);
-            p1 = ex2_approx(p1);
-            p2 = ex2_approx(p2);
-            p3 = ex2_approx(p3);
+            if ((j & 7) < kEmuQuadsFp8) {
+              exp2_poly2(p0, p1);
+              exp2_poly2(p2, p3);
+            } else {
+              p0 = ex2_approx(p0);
+              p1 = ex2_approx(p1);
+              p2 = ex2_approx(p2);
+              p3 = ex2_approx(p3);
+            }
             pk[j] = pack_e4m3x4(p0, p1, p2, p3);
             add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], p0 + p2, p1 + p3);
           }
