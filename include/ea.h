@@ -319,7 +319,8 @@ ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void*
  * The forward is recomputed from k (no saved activations).  Gradients are
  * summed in fp32 in a fixed order (bit-reproducible run to run).
  * workspace >= ea_router_ste_backward_workspace_size(...), 16-byte aligned.
- * Limits: those of ea_router_decide, B <= 1024, N <= 32767*256 (backward);
+ * Limits: those of ea_router_decide, B <= 1024, N <= 32767*256 and
+ * B * Hkv <= 65535 (backward); dk_accum 16-byte aligned;
  * tau finite and > 0 (else EA_ERR_INVALID_ARG).
  * ---------------------------------------------------------------------- */
 size_t ea_router_gumbel_workspace_size(int B, int Hkv, int N, int d, int hidden, int Hq);

@@ -382,8 +382,9 @@ ea_status ea_router_ste_backward(const void* k, int B, int Hkv, int N, int d, co
   if (!dout || !out || !out_other || !dw1 || !db1 || !dw2 || !db2) return EA_ERR_INVALID_ARG;
   const ea_status st = check_router_train(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, g0, g1, tau);
   if (st != EA_OK) return st;
-  if (N > kMaxSeqLen) return EA_ERR_UNSUPPORTED;
+  if (N > kMaxSeqLen || static_cast<long long>(B) * Hkv > 65535) return EA_ERR_UNSUPPORTED;
   if (!aligned16(dout) || !aligned16(out) || !aligned16(out_other)) return EA_ERR_MISALIGNED;
+  if (dk_accum && !aligned16(dk_accum)) return EA_ERR_MISALIGNED;
   if (!workspace ||
       workspace_bytes < ea_router_ste_backward_workspace_size(B, Hkv, N, d, hidden, Hq))
     return EA_ERR_WORKSPACE;

@@ -26,6 +26,7 @@
 
 #include "ea.h"
 #include "ea_internal.h"
+#include "ea_ptx.cuh"
 #include "ea_router_dev.cuh"
 
 namespace ea {
@@ -199,18 +200,34 @@ __global__ void ea_ste_dx_kernel(const float* __restrict__ dpre, const float* __
   dk_pool[i] = t / static_cast<float>(N);
 }
 
-// dk[b][hk][n][c] += dk_pool[b][hk * d + c] for every position n (bf16 in place).
-__global__ void ea_ste_dk_add_kernel(const float* __restrict__ dk_pool, int B, int Hkv, int N,
-                                     int d, __nv_bfloat16* __restrict__ dk) {
-  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const size_t total = static_cast<size_t>(B) * Hkv * N * d;
-  if (i >= total) return;
-  const int c = static_cast<int>(i % d);
-  const size_t row = i / d;                       // (b * Hkv + hk) * N + n
-  const size_t bh = row / N;                      // b * Hkv + hk
-  const int b = static_cast<int>(bh / Hkv), hk = static_cast<int>(bh % Hkv);
-  const float add = dk_pool[static_cast<size_t>(b) * Hkv * d + hk * d + c];
-  dk[i] = __float2bfloat16_rn(__bfloat162float(dk[i]) + add);
+// dk[b][hk][n][c] += dk_pool[b][hk * d + c] for every position n (bf16 in
+// place): CTA (position chunk, b * Hkv + hk), thread per 8 channels of a row
+// (16-byte loads and stores), the plane's d pooled values in registers.
+constexpr int kDkAddThreads = 256;
+__global__ void __launch_bounds__(kDkAddThreads) ea_ste_dk_add_kernel(
+    const float* __restrict__ dk_pool, int N, int d, int rows_per_cta,
+    __nv_bfloat16* __restrict__ dk) {
+  const int bh = blockIdx.y;
+  const int tpr = d / 8;                          // threads per row
+  const int c0 = (threadIdx.x % tpr) * 8;
+  float add[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) add[j] = dk_pool[static_cast<size_t>(bh) * d + c0 + j];
+  const int n0 = blockIdx.x * rows_per_cta;
+  const int n1 = min(N, n0 + rows_per_cta);
+  __nv_bfloat16* plane = dk + static_cast<size_t>(bh) * N * d;
+  for (int n = n0 + threadIdx.x / tpr; n < n1; n += kDkAddThreads / tpr) {
+    uint4* ptr = reinterpret_cast<uint4*>(plane + static_cast<size_t>(n) * d + c0);
+    uint4 v = *ptr;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16) + add[2 * j];
+      const float hi = __uint_as_float(w[j] & 0xffff0000u) + add[2 * j + 1];
+      w[j] = pack_bf16x2(lo, hi);
+    }
+    *ptr = v;
+  }
 }
 
 int ste_dr_splits(int B, int Hq) {
@@ -397,9 +414,13 @@ cudaError_t launch_router_ste(const void* k, int B, int Hkv, int N, int d, const
                                                                             in_dim, dw1, db1);
   ea_ste_dx_kernel<<<(B * in_dim + 255) / 256, 256, 0, s>>>(dpre, w1, B, hidden, in_dim, N, dkp);
   if (dk_accum) {
-    const size_t tot = static_cast<size_t>(B) * Hkv * N * d;
-    ea_ste_dk_add_kernel<<<static_cast<unsigned>((tot + 255) / 256), 256, 0, s>>>(
-        dkp, B, Hkv, N, d, static_cast<__nv_bfloat16*>(dk_accum));
+    // about four CTAs per SM over all planes, whole rows per CTA
+    const int planes = B * Hkv;
+    int chunks = (592 + planes - 1) / planes;
+    if (chunks > N) chunks = N;
+    const int rows = (N + chunks - 1) / chunks;
+    ea_ste_dk_add_kernel<<<dim3((N + rows - 1) / rows, planes), kDkAddThreads, 0, s>>>(
+        dkp, N, d, rows, static_cast<__nv_bfloat16*>(dk_accum));
   }
   return cudaGetLastError();
 }
