@@ -633,15 +633,18 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
             if (!vis) x[j] = -INFINITY;
           }
         }
-        // row max: eight independent chains of three-input max, then a tree
+        // row max: eight independent chains of three-input max over x[8..119],
+        // the last eight columns, then a tree
         float mk[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mk[k] = x[k];
 #pragma unroll
-        for (int j = 8; j < 128; j += 16) {
+        for (int j = 8; j < 120; j += 16) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], x[j + k], x[j + 8 + k]);
         }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mk[k] = fmaxf(mk[k], x[120 + k]);
         const float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]),
                                fmaxf(mk[6], mk[7]));
         const float m_tile = mx * sl2;
