@@ -306,7 +306,8 @@ def run_ours(args, rank, world, local_rank):
         "tile_granular_tflops": round(tile * world / (ms_per_step * 1e-3) / 1e12, 2),
         "attn_ms": round(attn_avg_ms, 4),
         "router_ms": round(statistics.mean(router_ms), 4),
-        "gpu_launches": K * nlayers * (3 if layers[0]["router"] is not None else 1),
+        # router: pool, reduce and the two MLP layers; then the attention launch
+        "gpu_launches": K * nlayers * (5 if layers[0]["router"] is not None else 1),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
@@ -409,10 +410,11 @@ def run_ours(args, rank, world, local_rank):
                          "h2d_bytes_per_step": hp.h2d_bytes(),
                          "d2h_bytes_per_step": hp.d2h_bytes(),
                          "ms_per_step": round(e2e_ms, 4),
-                         "path": "HostPrefill: pinned host q,k,v -> " +
+                         "path": "ea_hybrid_attn_prefill_host: pinned host q,k,v -> " +
                                  ("ea_router_decide" if L["router"] is not None
                                   else "route mask copy") +
-                                 " -> ea_hybrid_attn_prefill -> pinned host out"
+                                 f" -> {hp.chunks} kv-head chunks (upload, fused attention, "
+                                 "download overlapped) -> pinned host out"
                                  + (" (layer 0)" if nlayers > 1 else "")}
         if rank == 0:
             result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)

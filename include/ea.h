@@ -13,9 +13,10 @@
  *  - Tensors are dense, contiguous, row-major, in BHSD order:
  *      q, out : bf16 [B][Hq][N][d]      k, v : bf16 [B][Hkv][N][d]
  *    Query head h reads kv head h / (Hq / Hkv).
- *  - Every data pointer is a DEVICE pointer owned by the caller; the library
- *    never allocates, frees or keeps device memory of its own.  Parameter
- *    structs are HOST pointers, read before the call returns.
+ *  - Every data pointer is a DEVICE pointer owned by the caller (the
+ *    *_host arguments of ea_hybrid_attn_prefill_host are the exception); the
+ *    library never allocates, frees or keeps device memory of its own.
+ *    Parameter structs are HOST pointers, read before the call returns.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point synchronises except ea_get_device_status.
  *  - Argument errors are returned synchronously, before anything is
@@ -479,6 +480,70 @@ ea_status ea_hybrid_attn_decode(const void* q, const void* k_new, const void* v_
  * on invalid arguments. */
 int ea_decode_kv_policy(const uint8_t* mask, int B, int Hq, int Hkv, int32_t* cache_slot,
                         int* n_full, int* n_sa);
+
+/* ------------------------------------------------------------------------
+ * Prefill from HOST buffers, transfers overlapped with the attention.
+ *
+ * The pages move no data between host and device; this entry point serves a
+ * caller whose q, k, v live in host memory (and who wants out back there).
+ * It runs the same method as ea_router_decide followed by
+ * ea_hybrid_attn_prefill (Elastic Attention blog §2.1 router, §3 fused
+ * kernel) on device copies of the inputs, with bit-identical results, but
+ * splits the transfers so that most of them overlap the compute:
+ *   1. k (all of it: the router pools every kv head) and, without a router,
+ *      the caller's mask are uploaded; the router runs on k.
+ *   2. The heads are walked in chunks of c kv heads (with their c*Hq/Hkv
+ *      query heads) of one batch element: the chunk's q and v are uploaded,
+ *      its attention runs (ea_hybrid_attn_prefill on that head range), and
+ *      its rows of out are downloaded, so one chunk's upload and another's
+ *      download overlap a third chunk's attention.
+ *
+ * q_host, k_host, v_host : HOST bf16 BHSD.  Pinned memory (cudaHostAlloc or
+ *             cudaHostRegister) is needed for the copies to overlap anything;
+ *             pageable memory gives the same results without the overlap.
+ * route_mask_host : HOST uint8 [B][Hq] (0 = FA, nonzero = SA) when w1 is
+ *             NULL; ignored when the router runs.
+ * w1, b1, hidden, w2, b2, threshold : the router as for ea_router_decide
+ *             (DEVICE pointers: weights stay resident), or w1 = NULL to use
+ *             route_mask_host.
+ * p         : host pointer; p->select must be EA_SELECT_ALL.
+ * out_host  : HOST bf16 [B][Hq][N][d] (pinned for the overlap).
+ * route_mask_out_host : HOST uint8 [B][Hq] that receives the mask used, or
+ *             NULL.
+ * kv_heads_per_chunk : c in 1..Hkv (larger values are clamped to Hkv), or 0
+ *             for about eight chunks in all (ea_hybrid_attn_host_chunks
+ *             gives the count).
+ * workspace : DEVICE, >= ea_hybrid_attn_host_workspace_size(p, hidden)
+ *             bytes (hidden = 0 without a router), 16-byte aligned, ZEROED
+ *             once before its first use.  Its first 256 bytes are the
+ *             attention status block, read by ea_get_device_status(workspace,
+ *             ...); the rest holds the device mask, the router's scratch and
+ *             device copies of q, k, v and out.
+ * stream    : the call's work starts after the work already enqueued on
+ *             `stream`, and work enqueued on `stream` afterwards starts after
+ *             all of it, the last download included: synchronise `stream`
+ *             before reading out_host.  The copies themselves run on two
+ *             non-blocking streams that the library creates per device on
+ *             first use and keeps until the process exits.  The call never
+ *             synchronises.
+ * Argument errors are returned before anything is enqueued; a CUDA failure
+ * part way returns EA_ERR_CUDA with earlier chunks already enqueued.  Limits:
+ * those of ea_hybrid_attn_prefill (and of ea_router_decide with a router).
+ * Two calls in flight at once need separate workspaces and host buffers.
+ * ---------------------------------------------------------------------- */
+size_t ea_hybrid_attn_host_workspace_size(const ea_attn_params* p, int hidden);
+
+/* Number of chunks (kernel launches) a call with these arguments makes; 0
+ * if p is invalid or kv_heads_per_chunk < 0. */
+int ea_hybrid_attn_host_chunks(const ea_attn_params* p, int kv_heads_per_chunk);
+
+ea_status ea_hybrid_attn_prefill_host(const void* q_host, const void* k_host,
+                                      const void* v_host, const uint8_t* route_mask_host,
+                                      const float* w1, const float* b1, int hidden,
+                                      const float* w2, const float* b2, float threshold,
+                                      const ea_attn_params* p, void* out_host,
+                                      uint8_t* route_mask_out_host, int kv_heads_per_chunk,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Host-side view of the fused kernel's work schedule, for inspection and

@@ -43,7 +43,8 @@ EXPORTED = [
     "ea_hybrid_attn_backward", "ea_router_gumbel_workspace_size", "ea_router_decide_gumbel",
     "ea_router_ste_backward_workspace_size", "ea_router_ste_backward",
     "ea_hybrid_attn_prefill_train", "ea_fp8_vt_stride", "ea_quantize_fp8_workspace_size",
-    "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8",
+    "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8", "ea_hybrid_attn_host_workspace_size",
+    "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host",
 ]
 
 
@@ -107,6 +108,13 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
                                              vp, c_int, c_float, vp, vp, vp]
     lib.ea_hybrid_attn_workspace_size.restype = c_size
     lib.ea_hybrid_attn_workspace_size.argtypes = [pparams]
+    lib.ea_hybrid_attn_host_workspace_size.restype = c_size
+    lib.ea_hybrid_attn_host_workspace_size.argtypes = [pparams, c_int]
+    lib.ea_hybrid_attn_host_chunks.restype = c_int
+    lib.ea_hybrid_attn_host_chunks.argtypes = [pparams, c_int]
+    lib.ea_hybrid_attn_prefill_host.restype = c_int
+    lib.ea_hybrid_attn_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, vp, c_float,
+                                                pparams, vp, vp, c_int, vp, c_size, vp]
     lib.ea_hybrid_attn_prefill.restype = c_int
     lib.ea_hybrid_attn_prefill.argtypes = [vp, vp, vp, vp, pparams, vp, vp, c_size, vp]
     lib.ea_get_device_status.restype = c_int

@@ -6,6 +6,7 @@ CUDA stream; every step of the computation runs in libea.so's kernels.
 from __future__ import annotations
 
 import ctypes
+import math
 from typing import Optional, Tuple
 
 import numpy as np
@@ -658,54 +659,109 @@ def ea_attn_grid_size(p: EaAttnParams, num_sms: int) -> int:
 
 
 # ---------------------------------------------------------------- host-buffer path
+def ea_hybrid_attn_host_workspace_size(p: EaAttnParams, hidden: int = 0) -> int:
+    return int(_lib.load().ea_hybrid_attn_host_workspace_size(ctypes.byref(p), int(hidden)))
+
+
+def ea_hybrid_attn_host_chunks(p: EaAttnParams, kv_heads_per_chunk: int = 0) -> int:
+    return int(_lib.load().ea_hybrid_attn_host_chunks(ctypes.byref(p), int(kv_heads_per_chunk)))
+
+
+def _host_ptr(t: torch.Tensor, name: str, dtype, numel: int) -> int:
+    if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous() or t.numel() != numel:
+        raise ValueError(f"{name} must be a contiguous host {dtype} tensor of {numel} elements")
+    return t.data_ptr()
+
+
+def ea_hybrid_attn_prefill_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                                sink: int, window: int, *, out_host: torch.Tensor,
+                                workspace: torch.Tensor, router=None, threshold: float = 0.0,
+                                route_mask_host: Optional[torch.Tensor] = None,
+                                route_mask_out_host: Optional[torch.Tensor] = None,
+                                kv_heads_per_chunk: int = 0, softmax_scale: float = 0.0,
+                                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Prefill from host buffers (q, k, v, out on the host; pinned for the
+    copies to overlap the compute).  router = (w1, b1, w2, b2) device tensors,
+    or None with route_mask_host given.  The work is enqueued on `stream`;
+    synchronise it before reading out_host."""
+    lib = _lib.load()
+    B, Hq, N, d = q_host.shape
+    Hkv = k_host.shape[1]
+    if tuple(k_host.shape) != (B, Hkv, N, d) or v_host.shape != k_host.shape:
+        raise ValueError("k_host and v_host must be [B, Hkv, N, d] matching q_host")
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale)
+    nq, nkv = B * Hq * N * d, B * Hkv * N * d
+    args = [_host_ptr(q_host, "q_host", torch.bfloat16, nq),
+            _host_ptr(k_host, "k_host", torch.bfloat16, nkv),
+            _host_ptr(v_host, "v_host", torch.bfloat16, nkv)]
+    if router is not None:
+        w1, b1, w2, b2 = router
+        for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+            _need(t, name, torch.float32, nd)
+        args += [None, w1.data_ptr(), b1.data_ptr(), int(w1.shape[0]), w2.data_ptr(),
+                 b2.data_ptr(), float(threshold)]
+        device = w1.device
+    else:
+        if route_mask_host is None:
+            raise ValueError("route_mask_host is required without a router")
+        args += [_host_ptr(route_mask_host, "route_mask_host", torch.uint8, B * Hq), None, None,
+                 0, None, None, 0.0]
+        device = workspace.device
+    _host_ptr(out_host, "out_host", torch.bfloat16, nq)
+    mask_out = None
+    if route_mask_out_host is not None:
+        mask_out = _host_ptr(route_mask_out_host, "route_mask_out_host", torch.uint8, B * Hq)
+    if workspace.device.type != "cuda" or workspace.dtype != torch.uint8:
+        raise ValueError("workspace must be a device uint8 tensor")
+    rc = lib.ea_hybrid_attn_prefill_host(*args, ctypes.byref(p), out_host.data_ptr(), mask_out,
+                                         int(kv_heads_per_chunk), workspace.data_ptr(),
+                                         workspace.numel(), _stream_ptr(stream, device))
+    check(rc, "ea_hybrid_attn_prefill_host")
+    return out_host
+
+
 class HostPrefill:
-    """One layer's prefill from HOST buffers: copies q, k, v (pinned host) to
-    the device, runs ea_router_decide (or, with no router weights, copies the
-    caller's route mask) then ea_hybrid_attn_prefill, and copies the output
-    back into a pinned host buffer.  Device buffers are allocated once and
-    reused across calls."""
+    """One layer's prefill from HOST buffers through ea_hybrid_attn_prefill_host:
+    the router (resident device weights) or the caller's mask, then the fused
+    attention, with the q/k/v uploads and the out download split by kv-head
+    chunks so they overlap the compute.  The device workspace (device copies
+    of the inputs and output) and the pinned host output are allocated once
+    and reused across calls."""
 
     def __init__(self, B, Hq, Hkv, N, d, w1, b1, w2, b2, sink, window, device="cuda",
-                 threshold=0.0):
+                 threshold=0.0, kv_heads_per_chunk=0):
         self.has_router = w1 is not None
         self.shape_q = (B, Hq, N, d)
         self.shape_kv = (B, Hkv, N, d)
         self.sink, self.window, self.threshold = int(sink), int(window), float(threshold)
+        self.kv_heads_per_chunk = int(kv_heads_per_chunk)
         dev = torch.device(device)
-        self.q = torch.empty(self.shape_q, dtype=torch.bfloat16, device=dev)
-        self.k = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
-        self.v = torch.empty(self.shape_kv, dtype=torch.bfloat16, device=dev)
-        self.out = torch.empty(self.shape_q, dtype=torch.bfloat16, device=dev)
+        self.router = None
+        hidden = 0
         if self.has_router:
-            self.w1, self.b1 = w1.to(dev).contiguous(), b1.to(dev).contiguous()
-            self.w2, self.b2 = w2.to(dev).contiguous(), b2.to(dev).contiguous()
-        self.mask = torch.empty((B, Hq), dtype=torch.uint8, device=dev)
-        self.rws = torch.empty(max(ea_router_workspace_size(B, Hkv, N, d), 16),
-                               dtype=torch.uint8, device=dev)
-        self.aws = attn_workspace(make_params(B, Hq, Hkv, N, d, sink, window), dev)
+            self.router = tuple(t.to(dev).contiguous() for t in (w1, b1, w2, b2))
+            hidden = int(w1.shape[0])
+        p = make_params(B, Hq, Hkv, N, d, sink, window)
+        n = ea_hybrid_attn_host_workspace_size(p, hidden)
+        if n == 0:
+            raise ValueError("invalid prefill parameters")
+        self.workspace = torch.zeros(n, dtype=torch.uint8, device=dev)
+        self.chunks = ea_hybrid_attn_host_chunks(p, self.kv_heads_per_chunk)
         self.out_host = torch.empty(self.shape_q, dtype=torch.bfloat16, pin_memory=True)
 
     def h2d_bytes(self) -> int:
-        n = (self.q.numel() + self.k.numel() + self.v.numel()) * 2
-        return n if self.has_router else n + self.mask.numel()
+        n = (math.prod(self.shape_q) + 2 * math.prod(self.shape_kv)) * 2
+        return n if self.has_router else n + self.shape_q[0] * self.shape_q[1]
 
     def d2h_bytes(self) -> int:
-        return self.out.numel() * 2
+        return math.prod(self.shape_q) * 2
 
     def __call__(self, q_host, k_host, v_host, mask_host=None, stream=None):
-        self.q.copy_(q_host, non_blocking=True)
-        self.k.copy_(k_host, non_blocking=True)
-        self.v.copy_(v_host, non_blocking=True)
-        if self.has_router:
-            ea_router_decide(self.k, self.w1, self.b1, self.w2, self.b2, self.threshold,
-                             workspace=self.rws, route_mask=self.mask, want_logits=False,
-                             stream=stream)
-        else:
-            self.mask.copy_(mask_host.reshape(self.mask.shape), non_blocking=True)
-        ea_hybrid_attn_prefill(self.q, self.k, self.v, self.mask, self.sink, self.window,
-                               out=self.out, workspace=self.aws, stream=stream)
-        self.out_host.copy_(self.out, non_blocking=True)
-        return self.out_host
+        return ea_hybrid_attn_prefill_host(
+            q_host, k_host, v_host, self.sink, self.window, out_host=self.out_host,
+            workspace=self.workspace, router=self.router, threshold=self.threshold,
+            route_mask_host=None if self.has_router else mask_host.reshape(-1),
+            kv_heads_per_chunk=self.kv_heads_per_chunk, stream=stream)
 
 
 # ---------------------------------------------------------------- decode

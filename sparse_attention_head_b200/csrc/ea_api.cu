@@ -883,4 +883,199 @@ int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int ran
   return ut.n;
 }
 
+
+// ------------------------------------------------------------------ host buffers
+namespace {
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Device workspace of ea_hybrid_attn_prefill_host: the attention status block,
+// then the route mask, the router's scratch and device copies of q, k, v, out.
+struct HostLayout {
+  size_t mask, router, q, k, v, out, total;
+  size_t q_bytes, kv_bytes;
+};
+
+HostLayout host_layout(const ea_attn_params* p, int hidden) {
+  HostLayout L;
+  const size_t head = static_cast<size_t>(p->N) * p->d * 2;
+  L.q_bytes = head * p->B * p->Hq;
+  L.kv_bytes = head * p->B * p->Hkv;
+  size_t off = kAttnWorkspace;
+  L.mask = off;
+  off += up256(static_cast<size_t>(p->B) * p->Hq);
+  L.router = off;
+  if (hidden > 0) off += up256(ea::router_workspace_bytes(p->B, p->Hkv, p->N, p->d, kRouterMaxHidden));
+  L.q = off;
+  off += up256(L.q_bytes);
+  L.k = off;
+  off += up256(L.kv_bytes);
+  L.v = off;
+  off += up256(L.kv_bytes);
+  L.out = off;
+  off += up256(L.q_bytes);
+  L.total = off;
+  return L;
+}
+
+// Kv heads per chunk: the caller's choice, or about eight chunks in all.
+int host_chunk(const ea_attn_params* p, int kv_heads_per_chunk) {
+  int c = kv_heads_per_chunk;
+  if (c <= 0) c = (p->B * p->Hkv + 7) / 8;
+  return std::max(1, std::min(c, p->Hkv));
+}
+
+// The two copy streams (upload, download) of the current device, created
+// non-blocking on first use and kept until the process exits.
+bool host_copy_streams(cudaStream_t* up, cudaStream_t* down) {
+  static cudaStream_t s_up[ea::kMaxSmDevices] = {};
+  static cudaStream_t s_down[ea::kMaxSmDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= ea::kMaxSmDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!s_up[dev]) {
+    cudaStream_t a = nullptr, b = nullptr;
+    if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaStreamDestroy(a);
+      return false;
+    }
+    s_up[dev] = a;
+    s_down[dev] = b;
+  }
+  *up = s_up[dev];
+  *down = s_down[dev];
+  return true;
+}
+
+// Events of one call, destroyed when the call returns (a recorded event may
+// be destroyed before it completes; its resources are released afterwards).
+struct CallEvents {
+  std::vector<cudaEvent_t> ev;
+  ~CallEvents() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  }
+  cudaEvent_t make() {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    ev.push_back(e);
+    return e;
+  }
+};
+
+}  // namespace
+
+size_t ea_hybrid_attn_host_workspace_size(const ea_attn_params* p, int hidden) {
+  if (check_params(p) != EA_OK || hidden < 0 || hidden > kRouterMaxHidden) return 0;
+  return host_layout(p, hidden).total;
+}
+
+int ea_hybrid_attn_host_chunks(const ea_attn_params* p, int kv_heads_per_chunk) {
+  if (check_params(p) != EA_OK || kv_heads_per_chunk < 0) return 0;
+  const int c = host_chunk(p, kv_heads_per_chunk);
+  return p->B * ((p->Hkv + c - 1) / c);
+}
+
+ea_status ea_hybrid_attn_prefill_host(const void* q_host, const void* k_host,
+                                      const void* v_host, const uint8_t* route_mask_host,
+                                      const float* w1, const float* b1, int hidden,
+                                      const float* w2, const float* b2, float threshold,
+                                      const ea_attn_params* p, void* out_host,
+                                      uint8_t* route_mask_out_host, int kv_heads_per_chunk,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  ea_status st = check_params(p);
+  if (st != EA_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_host || kv_heads_per_chunk < 0)
+    return EA_ERR_INVALID_ARG;
+  if (p->select != EA_SELECT_ALL) return EA_ERR_INVALID_ARG;
+  const bool routed = w1 != nullptr;
+  if (!routed && !route_mask_host) return EA_ERR_INVALID_ARG;
+  if (!workspace) return EA_ERR_WORKSPACE;
+  const HostLayout L = host_layout(p, routed ? 1 : 0);
+  char* ws = static_cast<char*>(workspace);
+  uint8_t* dmask = reinterpret_cast<uint8_t*>(ws + L.mask);
+  if (routed) {
+    st = check_router_args(w1, b1, w2, b2, dmask, p->Hkv, p->d, hidden, p->Hq, threshold);
+    if (st != EA_OK) return st;
+  }
+  if (workspace_bytes < L.total) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaStream_t up = nullptr, down = nullptr;
+  if (!host_copy_streams(&up, &down)) return EA_ERR_CUDA;
+  char* dq = ws + L.q;
+  char* dk = ws + L.k;
+  char* dv = ws + L.v;
+  char* dout = ws + L.out;
+  const char* hq = static_cast<const char*>(q_host);
+  const char* hv = static_cast<const char*>(v_host);
+  char* hout = static_cast<char*>(out_host);
+  const size_t head = static_cast<size_t>(p->N) * p->d * 2;
+  const int G = p->Hq / p->Hkv;
+  const int c = host_chunk(p, kv_heads_per_chunk);
+  const size_t mask_bytes = static_cast<size_t>(p->B) * p->Hq;
+
+  CallEvents E;
+  cudaEvent_t ev_start = E.make(), ev_k = E.make();
+  if (!ev_start || !ev_k) return EA_ERR_CUDA;
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // The copies start after the work already on the caller's stream (the
+  // device buffers may still be read by an earlier call).
+  if (!ok(cudaEventRecord(ev_start, cs)) || !ok(cudaStreamWaitEvent(up, ev_start, 0)) ||
+      !ok(cudaStreamWaitEvent(down, ev_start, 0)))
+    return EA_ERR_CUDA;
+  // k (all of it: the router pools every kv head) and the caller's mask first.
+  if (!ok(cudaMemcpyAsync(dk, k_host, L.kv_bytes, cudaMemcpyHostToDevice, up))) return EA_ERR_CUDA;
+  if (!routed &&
+      !ok(cudaMemcpyAsync(dmask, route_mask_host, mask_bytes, cudaMemcpyHostToDevice, up)))
+    return EA_ERR_CUDA;
+  if (!ok(cudaEventRecord(ev_k, up)) || !ok(cudaStreamWaitEvent(cs, ev_k, 0))) return EA_ERR_CUDA;
+  if (routed) {
+    st = ea_router_decide(dk, p->B, p->Hkv, p->N, p->d, w1, b1, hidden, w2, b2, p->Hq,
+                          threshold, dmask, nullptr, ws + L.router, L.q - L.router, cs);
+    if (st != EA_OK) return st;
+  }
+  if (route_mask_out_host) {
+    cudaEvent_t ev_mask = E.make();
+    if (!ev_mask || !ok(cudaEventRecord(ev_mask, cs)) || !ok(cudaStreamWaitEvent(down, ev_mask, 0)) ||
+        !ok(cudaMemcpyAsync(route_mask_out_host, dmask, mask_bytes, cudaMemcpyDeviceToHost, down)))
+      return EA_ERR_CUDA;
+  }
+  // Chunks of c kv heads (and their G*c query heads) of one batch element:
+  // upload q and v, attend, download out.
+  for (int b = 0; b < p->B; ++b) {
+    for (int g0 = 0; g0 < p->Hkv; g0 += c) {
+      const int gc = std::min(c, p->Hkv - g0);
+      const size_t qoff = (static_cast<size_t>(b) * p->Hq + static_cast<size_t>(g0) * G) * head;
+      const size_t kvoff = (static_cast<size_t>(b) * p->Hkv + g0) * head;
+      const size_t qlen = static_cast<size_t>(gc) * G * head;
+      const size_t kvlen = static_cast<size_t>(gc) * head;
+      cudaEvent_t ev_in = E.make(), ev_done = E.make();
+      if (!ev_in || !ev_done) return EA_ERR_CUDA;
+      if (!ok(cudaMemcpyAsync(dq + qoff, hq + qoff, qlen, cudaMemcpyHostToDevice, up)) ||
+          !ok(cudaMemcpyAsync(dv + kvoff, hv + kvoff, kvlen, cudaMemcpyHostToDevice, up)) ||
+          !ok(cudaEventRecord(ev_in, up)) || !ok(cudaStreamWaitEvent(cs, ev_in, 0)))
+        return EA_ERR_CUDA;
+      ea_attn_params sub = *p;
+      sub.B = 1;
+      sub.Hq = gc * G;
+      sub.Hkv = gc;
+      st = ea_hybrid_attn_prefill(dq + qoff, dk + kvoff, dv + kvoff,
+                                  dmask + static_cast<size_t>(b) * p->Hq + g0 * G, &sub,
+                                  dout + qoff, workspace, kAttnWorkspace, cs);
+      if (st != EA_OK) return st;
+      if (!ok(cudaEventRecord(ev_done, cs)) || !ok(cudaStreamWaitEvent(down, ev_done, 0)) ||
+          !ok(cudaMemcpyAsync(hout + qoff, dout + qoff, qlen, cudaMemcpyDeviceToHost, down)))
+        return EA_ERR_CUDA;
+    }
+  }
+  // Work enqueued on the caller's stream later runs after the last download.
+  cudaEvent_t ev_end = E.make();
+  if (!ev_end || !ok(cudaEventRecord(ev_end, down)) || !ok(cudaStreamWaitEvent(cs, ev_end, 0)))
+    return EA_ERR_CUDA;
+  return EA_OK;
+}
+
 }  // extern "C"

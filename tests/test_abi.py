@@ -163,3 +163,50 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def _host(lib, p, qh=16, kh=16, vh=16, mask=16, w1=None, hidden=0, out=16, chunk=0, ws=256,
+          wsbytes=1 << 40):
+    return lib.ea_hybrid_attn_prefill_host(qh, kh, vh, mask, w1, 16 if w1 else None, hidden,
+                                           16 if w1 else None, 16 if w1 else None, 0.0,
+                                           ctypes.byref(p), out, None, chunk, ws, wsbytes, None)
+
+
+def test_host_entry_argument_errors(lib):
+    """ea_hybrid_attn_prefill_host rejects bad arguments before anything is
+    enqueued (so these calls need no GPU)."""
+    good = make_params(1, 8, 4, 700, 128, 16, 200)
+    assert _host(lib, make_params(0, 8, 4, 700, 128, 16, 200)) == _lib.EA_ERR_INVALID_ARG
+    assert _host(lib, good, qh=0) == _lib.EA_ERR_INVALID_ARG
+    assert _host(lib, good, out=0) == _lib.EA_ERR_INVALID_ARG
+    assert _host(lib, good, chunk=-1) == _lib.EA_ERR_INVALID_ARG
+    assert _host(lib, good, mask=0) == _lib.EA_ERR_INVALID_ARG          # no mask, no router
+    assert _host(lib, make_params(1, 8, 4, 700, 128, 16, 200, select=1)) == \
+        _lib.EA_ERR_INVALID_ARG
+    assert _host(lib, good, ws=0) == _lib.EA_ERR_WORKSPACE
+    assert _host(lib, good, w1=16, hidden=0) == _lib.EA_ERR_INVALID_ARG  # router, hidden 0
+    assert _host(lib, good, w1=24, hidden=64) == _lib.EA_ERR_MISALIGNED
+    assert _host(lib, good, wsbytes=1024) == _lib.EA_ERR_WORKSPACE
+    assert _host(lib, good, ws=264) == _lib.EA_ERR_MISALIGNED
+
+
+def test_host_workspace_and_chunks(lib):
+    """Workspace: the 256-byte status block, the mask, the router's scratch
+    (with a router) and device copies of q, k, v, out; about eight chunks by
+    default, never straddling a batch element."""
+    from sparse_attention_head_b200.api import (ea_hybrid_attn_host_chunks,
+                                                ea_hybrid_attn_host_workspace_size)
+    p = make_params(1, 32, 8, 32768, 128, 64, 1024)
+    tensors = (2 * 32 + 2 * 8) * 32768 * 128 * 2
+    n0 = ea_hybrid_attn_host_workspace_size(p, 0)
+    n1 = ea_hybrid_attn_host_workspace_size(p, 256)
+    assert tensors + 512 <= n0 < tensors + 4096
+    assert n1 > n0
+    assert ea_hybrid_attn_host_workspace_size(make_params(1, 8, 3, 64, 128, 0, 1), 0) == 0
+    assert ea_hybrid_attn_host_chunks(p, 0) == 8
+    assert ea_hybrid_attn_host_chunks(p, 3) == 3          # 3 + 3 + 2 kv heads
+    assert ea_hybrid_attn_host_chunks(p, 100) == 1
+    assert ea_hybrid_attn_host_chunks(make_params(2, 32, 8, 65536, 128, 64, 2048), 0) == 8
+    assert ea_hybrid_attn_host_chunks(make_params(4, 32, 8, 16384, 128, 128, 512), 0) == 8
+    assert ea_hybrid_attn_host_chunks(make_params(3, 4, 2, 512, 64, 16, 128), 0) == 6
+    assert ea_hybrid_attn_host_chunks(p, -1) == 0
