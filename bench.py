@@ -730,10 +730,10 @@ def measure_training(w: workloads.Workload, steps: int, warmup: int, dev, stream
         "roofline": {"bound": "tensor", "achieved": round(btf, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(btf / peak, 4),
                      "peak_source": f"{src} bf16_tflops (burst)",
-                     "scope": "attention backward (rowdot + dK/dV + dQ kernels), 2.5x the "
+                     "scope": "attention backward (rowdot + schedule + dK/dV + dQ kernels), 2.5x the "
                               "chosen mode's effective forward flops"},
-        # router 4 + Gumbel 1; forward 1; backward 3; STE: recompute 4 + 7
-        "gpu_launches_per_step": 5 + 1 + 3 + 11,
+        # router 4 + Gumbel 1; forward 1; backward 4 (rowdot, schedule, dK/dV, dQ); STE: recompute 4 + 7
+        "gpu_launches_per_step": 5 + 1 + 4 + 11,
     }
 
 

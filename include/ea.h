@@ -237,7 +237,9 @@ ea_status ea_hybrid_attn_prefill_train(const void* q, const void* k, const void*
  * route_mask : the forward's mask.
  * dq         : device bf16 [B][Hq][N][d]; dk, dv: [B][Hkv][N][d]; written.
  * workspace  : >= ea_hybrid_attn_backward_workspace_size(p) bytes, zeroed
- *              once; status word, then D (fp32 [B][Hq][N]).
+ *              once; status word, then D (fp32 [B][Hq][N]), then the two
+ *              kernels' work schedules (per-CTA unit lists, rebuilt by every
+ *              call from route_mask).
  * Arithmetic: bf16 tensor-core operands (P and dS rounded to bf16), fp32
  * accumulation, bf16 results.  Limits: d = 128, p->select == EA_SELECT_ALL,
  * plus those of ea_hybrid_attn_prefill. */

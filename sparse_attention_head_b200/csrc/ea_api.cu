@@ -581,7 +581,8 @@ ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void*
 size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p) {
   if (check_params(p) != EA_OK || p->d != 128) return 0;
   const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
-  return kAttnWorkspace + (rows * sizeof(float) + 255) / 256 * 256;
+  return kAttnWorkspace + (rows * sizeof(float) + 255) / 256 * 256 +
+         ea::bwd_sched_ints(p->B, p->Hq, p->Hkv, p->N) * sizeof(int);
 }
 
 ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, const void* out,
@@ -606,6 +607,25 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
       !encode_bhsd(&a.tm_do, dout, p->d, p->N, p->B * p->Hq))
     return EA_ERR_CUDA;
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + kAttnWorkspace);
+  {
+    // the schedule's unit lists after D
+    const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
+    int* w = reinterpret_cast<int*>(static_cast<char*>(workspace) + kAttnWorkspace +
+                                    (rows * sizeof(float) + 255) / 256 * 256);
+    const size_t nT = static_cast<size_t>((p->N + EA_BN - 1) / EA_BN);
+    const size_t ukv = static_cast<size_t>(p->B) * p->Hkv * nT;
+    const size_t uq = static_cast<size_t>(p->B) * p->Hq * nT;
+    a.offs_kv = w;
+    a.offs_q = w + (ea::kBwdMaxGrid + 1);
+    w += 2 * (ea::kBwdMaxGrid + 1);
+    a.list_kv = w;
+    a.sorted_kv = w + ukv;
+    a.cta_kv = w + 2 * ukv;
+    w += 3 * ukv;
+    a.list_q = w;
+    a.sorted_q = w + uq;
+    a.cta_q = w + 2 * uq;
+  }
   a.lse = lse;
   a.dvec = dvec;
   a.mask = route_mask;

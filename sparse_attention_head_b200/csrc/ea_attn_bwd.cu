@@ -10,9 +10,12 @@
 // a kv head's dK, dV summed over its query heads (GQA).  P is recomputed from
 // the forward's log-sum-exp: P = 2^(s * scale * log2e - lse * log2e).
 //
-// Three launches on the caller's stream:
+// Four launches on the caller's stream:
 //   1. ea_bwd_rowdot_kernel: D = rowsum(dO * O), fp32 (HBM-bound);
-//   2. ea_bwd_dkdv_kernel: unit = (b, kv head, 128-key tile j).  K_j and V_j
+//   2. ea_bwd_sched_kernel: the units of the two kernels below sorted by
+//      cost and assigned to CTAs (longest first; for dK/dV each to the
+//      least-loaded CTA), as per-CTA lists in the workspace;
+//   3. ea_bwd_dkdv_kernel: unit = (b, kv head, 128-key tile j).  K_j and V_j
 //      stay in shared memory; the steps visit (query head of the group,
 //      128-query tile i) pairs that see tile j.  Per step the tensor cores
 //      compute S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM, eight warps
@@ -21,7 +24,7 @@
 //      from TMEM).  The elementwise work runs in two phases (P from S while
 //      dP is computed; dS from dP while dV and the next S are), so the
 //      tensor pipe and the elementwise warps overlap.
-//   3. ea_bwd_dq_kernel: unit = (b, head, 128-query tile i); the steps visit
+//   4. ea_bwd_dq_kernel: unit = (b, head, 128-query tile i); the steps visit
 //      the key tiles the forward visits: S = Q_i K_j^T, dP = dO_i V_j^T, dS,
 //      dQ += dS K_j.
 // Both are persistent (one CTA per SM), with a TMA producer warp, one MMA
@@ -196,10 +199,9 @@ __device__ __forceinline__ void bwd_phase_p(uint32_t taddr, const float* vl, flo
 }
 
 // ---------------------------------------------------------------- units
-// kDkDv: unit (b, kv head, key tile), key tile 0 (the most queries) first;
-// else unit (b, head, query tile), the last query tile (the most keys) first.
-// Units are dealt to CTAs in a snake (ea_rank_for), so a CTA that takes one
-// of the first, longest units takes one of the last, shortest ones next.
+// kDkDv: unit (b, kv head, key tile); else unit (b, head, query tile).  The
+// index u enumerates them; the order in which CTAs run them is the
+// schedule's (ea_bwd_sched_kernel below).
 template <bool kDkDv>
 __device__ __forceinline__ void bwd_unit_of(const BwdArgs& a, int u, int* b, int* hx, int* tile) {
   const int nT = ea_cdiv(a.N, EA_BN);
@@ -214,6 +216,186 @@ __device__ __forceinline__ void bwd_unit_of(const BwdArgs& a, int u, int* b, int
     *b = (u % per) / a.Hq;
     *hx = (u % per) % a.Hq;
   }
+}
+
+// ---------------------------------------------------------------- schedule
+// A unit's cost in steps (plus one for its fixed work: resident loads and
+// the accumulator read-out).  kDkDv: the query tiles of the group's heads
+// that see the key tile; else the key tiles the query tile visits.
+template <bool kDkDv>
+__device__ __forceinline__ int bwd_unit_cost(const BwdArgs& a, const uint8_t* mask, int u) {
+  int b, hx, tile;
+  bwd_unit_of<kDkDv>(a, u, &b, &hx, &tile);
+  const int nT = ea_cdiv(a.N, EA_BN);
+  if (kDkDv) {
+    const int G = a.Hq / a.Hkv;
+    int c = 1;
+    for (int g = 0; g < G; ++g) {
+      const bool sa = mask[b * a.Hq + hx * G + g] != 0;
+      c += bwd_last_query_tile(tile, sa, nT, a.sink, a.window) - tile + 1;
+    }
+    return c;
+  }
+  int a0, lo;
+  bwd_key_tiles(tile, mask[b * a.Hq + hx] != 0, a.sink, a.window, &a0, &lo);
+  return 1 + a0 + (tile - lo + 1);
+}
+
+constexpr int kSchedBins = 4096;
+
+// Per-CTA unit lists of one backward kernel, longest units first.  One CTA
+// of 1024 threads per kernel (blockIdx.x 0: dK/dV, 1: dQ):
+//   1. units are counted by cost bin (cost >> shift, so every bin index is
+//      below kSchedBins) and sorted by decreasing bin, ties by unit index;
+//   2. dK/dV: each unit in that order goes to the least-loaded CTA (ties to
+//      the lowest index), since a few key tiles carry far more steps than
+//      the rest; dQ: the sorted units are dealt in a snake, which already
+//      balances its many similar units;
+//   3. each CTA's units are listed in sorted order.
+// Every step is deterministic (the scatters run in order on one warp), so
+// the schedule is the same on every run.  Results do not depend on it: a
+// unit owns its output tile.
+template <bool kDkDv>
+__device__ void bwd_schedule(const BwdArgs& a, int grid, int* hist, long long* load,
+                             uint8_t* mask, int& shift_s) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nT = ea_cdiv(a.N, EA_BN);
+  const int units = a.B * (kDkDv ? a.Hkv : a.Hq) * nT;
+  int* offs = kDkDv ? a.offs_kv : a.offs_q;
+  int* list = kDkDv ? a.list_kv : a.list_q;
+  int* sorted = kDkDv ? a.sorted_kv : a.sorted_q;
+  int* cta = kDkDv ? a.cta_kv : a.cta_q;
+  const int max_cost = 1 + (kDkDv ? a.Hq / a.Hkv : 1) * nT;
+  if (tid == 0) {
+    int sh = 0;
+    while ((max_cost >> sh) >= kSchedBins) ++sh;
+    shift_s = sh;
+  }
+  for (int i = tid; i < kSchedBins; i += blockDim.x) hist[i] = 0;
+  for (int i = tid; i < kBwdMaxGrid; i += blockDim.x) load[i] = 0;
+  for (int i = tid; i < a.B * a.Hq; i += blockDim.x) mask[i] = a.mask[i];
+  __syncthreads();
+  const int shift = shift_s;
+  for (int u = tid; u < units; u += blockDim.x)
+    atomicAdd(&hist[bwd_unit_cost<kDkDv>(a, mask, u) >> shift], 1);
+  __syncthreads();
+  // hist[bin] becomes the first sorted position of the bin (decreasing bins)
+  if (tid == 0) {
+    int run = 0;
+    for (int bin = kSchedBins - 1; bin >= 0; --bin) {
+      const int n = hist[bin];
+      hist[bin] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  if (warp == 0) {
+    // stable scatter by bin
+    for (int base = 0; base < units; base += 32) {
+      const int u = base + lane;
+      const int bin = u < units ? bwd_unit_cost<kDkDv>(a, mask, u) >> shift : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      const int pos = u < units ? hist[bin] + __popc(peers & lt) : 0;
+      __syncwarp();
+      if (u < units) {
+        sorted[pos] = u;
+        if ((peers & lt) == 0) hist[bin] += __popc(peers);
+      }
+      __syncwarp();
+    }
+    // assignment of sorted position r to a CTA
+    for (int base = 0; base < units; base += 32) {
+      if (kDkDv) {
+        // the 32 costs of this batch are read at once, then taken in order
+        const int mine = base + lane < units ? bwd_unit_cost<kDkDv>(a, mask, sorted[base + lane]) : 0;
+        for (int j = 0; j < 32 && base + j < units; ++j) {
+          const int r = base + j;
+          const int c = __shfl_sync(0xffffffffu, mine, j);
+          long long best = 0x7fffffffffffffffll;
+          int bi = 0;
+          for (int i = lane; i < grid; i += 32)
+            if (load[i] < best) {
+              best = load[i];
+              bi = i;
+            }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const long long ob = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ob < best || (ob == best && oi < bi)) {
+              best = ob;
+              bi = oi;
+            }
+          }
+          if (lane == 0) {
+            cta[r] = bi;
+            load[bi] += c;
+          }
+          __syncwarp();
+        }
+      } else {
+        const int r = base + lane;
+        if (r < units) {
+          const int k = r / grid, c = r % grid;
+          cta[r] = (k & 1) ? grid - 1 - c : c;
+        }
+      }
+    }
+    __syncwarp();
+    // per-CTA counts, offsets, then the lists in sorted order
+    for (int i = lane; i < grid; i += 32) load[i] = 0;
+    __syncwarp();
+    for (int base = 0; base < units; base += 32) {
+      const int r = base + lane;
+      const int c = r < units ? cta[r] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      if (r < units && (peers & lt) == 0) load[c] += __popc(peers);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      int run = 0;
+      for (int i = 0; i < grid; ++i) {
+        offs[i] = run;
+        const int n = static_cast<int>(load[i]);
+        load[i] = run;
+        run += n;
+      }
+      offs[grid] = run;
+    }
+    __syncwarp();
+    for (int base = 0; base < units; base += 32) {
+      const int r = base + lane;
+      const int c = r < units ? cta[r] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int pos = r < units ? static_cast<int>(load[c]) + __popc(peers & lt) : 0;
+      __syncwarp();
+      if (r < units) {
+        list[pos] = sorted[r];
+        if ((peers & lt) == 0) load[c] += __popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024, 1) ea_bwd_sched_kernel(const __grid_constant__ BwdArgs a,
+                                                               int grid_kv, int grid_q) {
+  __shared__ int hist[kSchedBins];
+  __shared__ long long load[kBwdMaxGrid];
+  __shared__ uint8_t mask[EA_MAX_ENTRIES];
+  __shared__ int shift_s;
+  if (blockIdx.x == 0)
+    bwd_schedule<true>(a, grid_kv, hist, load, mask, shift_s);
+  else
+    bwd_schedule<false>(a, grid_q, hist, load, mask, shift_s);
+}
+
+size_t bwd_sched_ints(int B, int Hq, int Hkv, int N) {
+  const size_t nT = static_cast<size_t>(ea_cdiv(N, EA_BN));
+  const size_t units_kv = static_cast<size_t>(B) * Hkv * nT;
+  const size_t units_q = static_cast<size_t>(B) * Hq * nT;
+  return 2 * (kBwdMaxGrid + 1) + 3 * (units_kv + units_q);
 }
 
 // One backward kernel per flavour (see the file comment):
@@ -255,7 +437,9 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
   float* vec1 = reinterpret_cast<float*>(smem + C::kOffVec1);
   const int G = args.Hq / args.Hkv;
   const int nT = ea_cdiv(args.N, EA_BN);
-  const int units = args.B * (kDkDv ? args.Hkv : args.Hq) * nT;
+  // this CTA's units, longest first (ea_bwd_sched_kernel)
+  const int* uoffs = kDkDv ? args.offs_kv : args.offs_q;
+  const int* ulist = kDkDv ? args.list_kv : args.list_q;
   const uint64_t tlim = args.timeout_ns;
   int* status = args.status;
 
@@ -282,8 +466,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     // ============================================================ producer
     uint32_t pos = 0, nu = 0, armed0 = 0, armed1 = 0;
     bool ok = true;
-    for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
-         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
+    for (int kk = uoffs[blockIdx.x], kend = uoffs[blockIdx.x + 1]; kk < kend && ok; ++kk) {
+      const int u = ulist[kk];
       int b, hx, tile;
       bwd_unit_of<kDkDv>(args, u, &b, &hx, &tile);
       if (nu > 0) {
@@ -434,8 +618,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
       };
       uint32_t pos = 0, nu = 0, nsteps = 0;
       bool ok = true;
-      for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
-         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
+      for (int kk = uoffs[blockIdx.x], kend = uoffs[blockIdx.x + 1]; kk < kend && ok; ++kk) {
         if (!(ok = mbar_wait(b_res_full, nu & 1, s_abort, status, tlim, EA_ERR_TIMEOUT))) break;
         const uint32_t unit = nu++;
         if (!(ok = wait_full(0, pos))) break;
@@ -512,8 +695,8 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     const float sl2 = args.scale_log2;
     uint32_t pos = 0, nsteps = 0, nu = 0;
     bool ok = true;
-    for (int kk = 0, u = ea_rank_for(0, blockIdx.x, gridDim.x, units); u >= 0 && ok;
-         u = ea_rank_for(++kk, blockIdx.x, gridDim.x, units)) {
+    for (int kk = uoffs[blockIdx.x], kend = uoffs[blockIdx.x + 1]; kk < kend && ok; ++kk) {
+      const int u = ulist[kk];
       int b, hx, tile;
       bwd_unit_of<kDkDv>(args, u, &b, &hx, &tile);
       const int row = tile * EA_BM + t;
@@ -709,11 +892,14 @@ cudaError_t launch_backward(const BwdArgs& a, const void* dout, const void* out,
   }
   const int nT = ea_cdiv(a.N, EA_BN);
   const int units_kv = a.B * a.Hkv * nT, units_q = a.B * a.Hq * nT;
-  ea_bwd_attn_kernel<true><<<units_kv < grid_sms ? units_kv : grid_sms, BwdCfg::kThreads,
-                             BwdCfg::kSmem, stream>>>(a);
+  const int sms = grid_sms < kBwdMaxGrid ? grid_sms : kBwdMaxGrid;
+  const int grid_kv = units_kv < sms ? units_kv : sms;
+  const int grid_q = units_q < sms ? units_q : sms;
+  ea_bwd_sched_kernel<<<2, 1024, 0, stream>>>(a, grid_kv, grid_q);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  ea_bwd_attn_kernel<false><<<units_q < grid_sms ? units_q : grid_sms, BwdCfg::kThreads,
-                              BwdCfg::kSmem, stream>>>(a);
+  ea_bwd_attn_kernel<true><<<grid_kv, BwdCfg::kThreads, BwdCfg::kSmem, stream>>>(a);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  ea_bwd_attn_kernel<false><<<grid_q, BwdCfg::kThreads, BwdCfg::kSmem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -72,7 +72,22 @@ struct BwdArgs {
   int B, Hq, Hkv, N, sink, window;
   float scale, scale_log2;
   unsigned long long timeout_ns;
+  // Unit lists of the two kernels (written by ea_bwd_sched_kernel): CTA c
+  // runs units list[offs[c]] .. list[offs[c + 1] - 1] in that order.  sorted
+  // and cta are the schedule's scratch (one int per unit each).
+  int* offs_kv;
+  int* list_kv;
+  int* sorted_kv;
+  int* cta_kv;
+  int* offs_q;
+  int* list_q;
+  int* sorted_q;
+  int* cta_q;
 };
+// Upper bound of the CTAs a backward kernel is launched with.
+constexpr int kBwdMaxGrid = 1024;
+// Ints of backward workspace the unit lists need, after D.
+size_t bwd_sched_ints(int B, int Hq, int Hkv, int N);
 // D = rowsum(dO * O) into dvec, then the dK/dV and dQ kernels.
 cudaError_t launch_backward(const BwdArgs& a, const void* dout, const void* out, float* dvec,
                             int grid_sms, cudaStream_t stream);
