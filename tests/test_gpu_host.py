@@ -169,3 +169,28 @@ def test_host_prefill_reuse():
         outs.append(hp.out_host.clone())
     assert not torch.equal(outs[0], outs[1])
     assert ea_get_device_status(hp.workspace) == 0
+
+
+def test_llama8b_full_size_matches_device_path():
+    """The bench's e2e configuration (llama8b layer, router, automatic
+    chunks): the host path's mask and output equal the device path's bit for
+    bit, and its rows match the oracle on a sample of every head."""
+    w = workloads.get("llama8b")
+    seed = workloads.layer_seed(w)
+    q, k, v = workloads.make_qkv(w, seed)
+    q, k, v = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    heads = workloads.sparse_head_set(w.hq, w.sparse_frac, seed)
+    router = workloads.make_router_weights(w.hkv * w.d, w.router_hidden, w.hq, heads, seed)
+    hp = HostPrefill(w.batch, w.hq, w.hkv, w.seq, w.d, *router, w.sink, w.window, device=DEV)
+    assert hp.chunks == 8
+    hp(q, k, v)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(hp.workspace) == 0
+    ref_out, ref_mask = _device_path(q, k, v, w.sink, w.window, router=router)
+    assert int(ref_mask.sum()) == 22
+    assert torch.equal(hp.out_host, ref_out)
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    rows = [0, 1, 63, 64, 1023, 1024, 1087, 1088, 20000, w.seq - 1]
+    for h in range(0, w.hq, 5):
+        ref = oracle.attention_rows(qf, kf, vf, ref_mask.numpy(), 0, h, rows, w.sink, w.window)
+        compare(hp.out_host[0, h, rows], ref, f"llama8b host path head {h}")
