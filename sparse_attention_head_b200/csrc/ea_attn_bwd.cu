@@ -276,20 +276,56 @@ __device__ void bwd_schedule(const BwdArgs& a, int grid, int* hist, long long* l
   for (int i = tid; i < a.B * a.Hq; i += blockDim.x) mask[i] = a.mask[i];
   __syncthreads();
   const int shift = shift_s;
-  for (int u = tid; u < units; u += blockDim.x)
-    atomicAdd(&hist[bwd_unit_cost<kDkDv>(a, mask, u) >> shift], 1);
-  __syncthreads();
-  // hist[bin] becomes the first sorted position of the bin (decreasing bins)
-  if (tid == 0) {
-    int run = 0;
-    for (int bin = kSchedBins - 1; bin >= 0; --bin) {
-      const int n = hist[bin];
-      hist[bin] = run;
-      run += n;
-    }
+  const unsigned lt = (1u << lane) - 1u;
+  // counts per bin; lanes of a warp that share a bin add once (most units
+  // of a mask share a handful of costs)
+  for (int base = warp * 32; base < units; base += blockDim.x) {
+    const int u = base + lane;
+    const int bin = u < units ? bwd_unit_cost<kDkDv>(a, mask, u) >> shift : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (u < units && (peers & lt) == 0) atomicAdd(&hist[bin], __popc(peers));
   }
   __syncthreads();
-  const unsigned lt = (1u << lane) - 1u;
+  // hist[bin] becomes the first sorted position of the bin, bins in
+  // decreasing order: each thread sums four consecutive bins from the top,
+  // a block scan of the thread sums gives each group's start
+  {
+    static_assert(kSchedBins == 4 * 1024, "four bins per thread of the 1024");
+    int* wsum = reinterpret_cast<int*>(load);   // 32 warp totals (load is reset below)
+    int v[4], t = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = hist[kSchedBins - 1 - (4 * tid + i)];
+      t += v[i];
+    }
+    int incl = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = wsum[lane], wi = w;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wi, off);
+        if (lane >= off) wi += y;
+      }
+      wsum[lane] = wi - w;                      // exclusive over warps
+    }
+    __syncthreads();
+    int run = wsum[warp] + incl - t;            // exclusive start of this thread's four bins
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hist[kSchedBins - 1 - (4 * tid + i)] = run;
+      run += v[i];
+    }
+    __syncthreads();
+    for (int i = tid; i < kBwdMaxGrid; i += blockDim.x) load[i] = 0;
+    __syncthreads();
+  }
   if (warp == 0) {
     // stable scatter by bin
     for (int base = 0; base < units; base += 32) {
@@ -304,43 +340,92 @@ __device__ void bwd_schedule(const BwdArgs& a, int grid, int* hist, long long* l
       }
       __syncwarp();
     }
-    // assignment of sorted position r to a CTA
-    for (int base = 0; base < units; base += 32) {
-      if (kDkDv) {
-        // the 32 costs of this batch are read at once, then taken in order
-        const int mine = base + lane < units ? bwd_unit_cost<kDkDv>(a, mask, sorted[base + lane]) : 0;
-        for (int j = 0; j < 32 && base + j < units; ++j) {
-          const int r = base + j;
-          const int c = __shfl_sync(0xffffffffu, mine, j);
-          long long best = 0x7fffffffffffffffll;
-          int bi = 0;
-          for (int i = lane; i < grid; i += 32)
-            if (load[i] < best) {
-              best = load[i];
-              bi = i;
-            }
+  }
+  if (!kDkDv) {
+    // dQ: the sorted units dealt in a snake.  Rank r = k * grid + j goes to
+    // CTA j (k even) or grid - 1 - j (k odd), at position k of its list; a
+    // CTA's list has units / grid entries, plus one if the last, partial
+    // round reaches it, so the offsets and positions are closed forms.
+    __syncthreads();
+    const int F = units / grid, R = units % grid;
+    auto first = [&](int c) {
+      int extra = 0;
+      if (R > 0) extra = (F & 1) == 0 ? min(c, R) : max(0, c - (grid - R));
+      return c * F + extra;
+    };
+    for (int c = tid; c <= grid; c += blockDim.x) offs[c] = first(c);
+    for (int r = tid; r < units; r += blockDim.x) {
+      const int k = r / grid, j = r % grid;
+      const int c = (k & 1) ? grid - 1 - j : j;
+      list[first(c) + k] = sorted[r];
+    }
+    return;
+  }
+  if (warp == 0) {
+    // dK/dV: each unit in sorted order to the least-loaded CTA (ties to the
+    // lowest index).  Lane l keeps the loads of CTAs l, l + 32, ... in
+    // registers (grid <= 32 * kPer) and the warp takes their minimum with
+    // reductions.  Loads stay below 2^31 (units * max_cost); past that, or
+    // for a larger grid, the units are dealt in a snake instead.
+    constexpr int kPer = 8;
+    const bool greedy = grid <= 32 * kPer &&
+                        static_cast<long long>(units) * max_cost < (1ll << 31);
+    // Packed keys (load << 8 | CTA) when every load stays below 2^24: the
+    // key minimum is then the least load with the lowest index, one
+    // reduction per unit.
+    const bool packed = greedy && static_cast<long long>(units) * max_cost < (1ll << 24);
+    unsigned ld[kPer];
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            const long long ob = __shfl_xor_sync(0xffffffffu, best, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ob < best || (ob == best && oi < bi)) {
-              best = ob;
-              bi = oi;
-            }
-          }
-          if (lane == 0) {
-            cta[r] = bi;
-            load[bi] += c;
-          }
-          __syncwarp();
-        }
-      } else {
+    for (int m = 0; m < kPer; ++m)
+      ld[m] = (m * 32 + lane < grid) ? (packed ? static_cast<unsigned>(m * 32 + lane) : 0u)
+                                     : 0xffffffffu;
+    for (int base = 0; base < units; base += 32) {
+      const int mine = base + lane < units ? bwd_unit_cost<kDkDv>(a, mask, sorted[base + lane]) : 0;
+      if (!greedy) {
         const int r = base + lane;
         if (r < units) {
-          const int k = r / grid, c = r % grid;
-          cta[r] = (k & 1) ? grid - 1 - c : c;
+          const int k = r / grid, j = r % grid;
+          cta[r] = (k & 1) ? grid - 1 - j : j;
         }
+        continue;
       }
+      unsigned mywin = 0;   // lane j keeps the CTA of unit base + j
+      for (int j = 0; j < 32 && base + j < units; ++j) {
+        const unsigned c = static_cast<unsigned>(__shfl_sync(0xffffffffu, mine, j));
+        unsigned win;
+        if (packed) {
+          const unsigned m01 = min(ld[0], ld[1]), m23 = min(ld[2], ld[3]);
+          const unsigned m45 = min(ld[4], ld[5]), m67 = min(ld[6], ld[7]);
+          const unsigned key = __reduce_min_sync(0xffffffffu, min(min(m01, m23), min(m45, m67)));
+          win = key & 0xffu;
+          // branch-free: only the winning slot adds
+#pragma unroll
+          for (int m = 0; m < kPer; ++m)
+            ld[m] += (static_cast<unsigned>(m * 32 + lane) == win) ? (c << 8) : 0u;
+        } else {
+          unsigned best = ld[0];
+          int bm = 0;
+#pragma unroll
+          for (int m = 1; m < kPer; ++m)
+            if (ld[m] < best) {
+              best = ld[m];
+              bm = m;
+            }
+          const unsigned wmin = __reduce_min_sync(0xffffffffu, best);
+          // CTA index of this lane's minimum (lane + 32 m); the smallest
+          // index among the lanes that hold the warp minimum wins
+          const unsigned idx =
+              (best == wmin) ? static_cast<unsigned>(bm * 32 + lane) : 0xffffffffu;
+          win = __reduce_min_sync(0xffffffffu, idx);
+          if (static_cast<int>(win & 31) == lane) {
+#pragma unroll
+            for (int m = 0; m < kPer; ++m)
+              if (m == static_cast<int>(win >> 5)) ld[m] += c;
+          }
+        }
+        mywin = (lane == j) ? win : mywin;
+      }
+      if (base + lane < units) cta[base + lane] = static_cast<int>(mywin);
     }
     __syncwarp();
     // per-CTA counts, offsets, then the lists in sorted order
