@@ -386,8 +386,13 @@ def run_ours(args, rank, world, local_rank):
                 "routed_one_launch_ms": round(routed_ms, 4),
                 "routed_speedup_vs_two_launches": round(two_ms / routed_ms, 3),
             })
-        # end to end through the public API with host buffers (layer 0; for a
-        # multi-layer workload the metric uses that layer's work only)
+        if rank == 0:
+            result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
+    if not args.quick:
+        # end to end through the public API with host buffers, on every rank
+        # (layer 0; for a multi-layer workload the metric uses that layer's
+        # work only); the timed region is the slowest rank's
+        L = layers[0]
         ek = args.e2e_steps or K
         router = L["router"] if L["router"] is not None else (None, None, None, None)
         hp = HostPrefill(B, Hq, Hkv, N, d, *router, w.sink, w.window, device=dev)
@@ -398,26 +403,31 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(2):
             hp(qh, kh, vh, mh)
         torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(ek):
             hp(qh, kh, vh, mh)
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / ek
+        if world > 1:
+            torch.distributed.barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / ek, world, dev)
+        if ea_get_device_status(hp.workspace) != 0:
+            raise RuntimeError("host-buffer path status word reports an error")
         eff0 = flops.effective_flops(mask_host[0], N, d, w.sink, w.window)
-        result["e2e"] = {"value": round(eff0 / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
-                         "h2d_bytes_per_step": hp.h2d_bytes(),
-                         "d2h_bytes_per_step": hp.d2h_bytes(),
+        result["e2e"] = {"value": round(eff0 * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                         "h2d_bytes_per_step": hp.h2d_bytes() * world,
+                         "d2h_bytes_per_step": hp.d2h_bytes() * world,
                          "ms_per_step": round(e2e_ms, 4),
                          "path": "ea_hybrid_attn_prefill_host: pinned host q,k,v -> " +
                                  ("ea_router_decide" if L["router"] is not None
                                   else "route mask copy") +
                                  f" -> {hp.chunks} kv-head chunks (upload, fused attention, "
                                  "download overlapped) -> pinned host out"
-                                 + (" (layer 0)" if nlayers > 1 else "")}
-        if rank == 0:
-            result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
+                                 + (" (layer 0)" if nlayers > 1 else "")
+                                 + (f", one replica per rank x{world}" if world > 1 else "")}
     if not args.quick and world == 1 and args.packed_seqs > 0:
         result["packed"] = measure_packed(w, args.packed_seqs, max(args.steps, 5),
                                           max(args.warmup, 3), dev, stream)
