@@ -535,6 +535,16 @@ int ea_decode_kv_policy(const uint8_t* mask, int B, int Hq, int Hkv, int32_t* ca
  * ---------------------------------------------------------------------- */
 size_t ea_hybrid_attn_host_workspace_size(const ea_attn_params* p, int hidden);
 
+/* Releases what the library holds between calls: the copy streams of
+ * ea_hybrid_attn_prefill_host, on every device that created them (after the
+ * work already on them finishes; the current device is restored).  Call it
+ * with no library call in flight; a later host-buffer call creates the
+ * streams again.  Nothing else is held: every other buffer is the caller's,
+ * and ea_router_decide_noalloc's fixed scratch is static device memory that
+ * lives until the process exits.  EA_OK, or EA_ERR_CUDA if a CUDA call
+ * failed (the streams are forgotten either way). */
+ea_status ea_shutdown(void);
+
 /* Number of chunks (kernel launches) a call with these arguments makes; 0
  * if p is invalid or kv_heads_per_chunk < 0. */
 int ea_hybrid_attn_host_chunks(const ea_attn_params* p, int kv_heads_per_chunk);

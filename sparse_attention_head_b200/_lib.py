@@ -44,7 +44,7 @@ EXPORTED = [
     "ea_router_ste_backward_workspace_size", "ea_router_ste_backward",
     "ea_hybrid_attn_prefill_train", "ea_fp8_vt_stride", "ea_quantize_fp8_workspace_size",
     "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8", "ea_hybrid_attn_host_workspace_size",
-    "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host",
+    "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host", "ea_shutdown",
 ]
 
 
@@ -110,6 +110,8 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_workspace_size.argtypes = [pparams]
     lib.ea_hybrid_attn_host_workspace_size.restype = c_size
     lib.ea_hybrid_attn_host_workspace_size.argtypes = [pparams, c_int]
+    lib.ea_shutdown.restype = c_int
+    lib.ea_shutdown.argtypes = []
     lib.ea_hybrid_attn_host_chunks.restype = c_int
     lib.ea_hybrid_attn_host_chunks.argtypes = [pparams, c_int]
     lib.ea_hybrid_attn_prefill_host.restype = c_int

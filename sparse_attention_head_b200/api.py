@@ -663,6 +663,11 @@ def ea_hybrid_attn_host_workspace_size(p: EaAttnParams, hidden: int = 0) -> int:
     return int(_lib.load().ea_hybrid_attn_host_workspace_size(ctypes.byref(p), int(hidden)))
 
 
+def ea_shutdown() -> None:
+    """Release the library's copy streams (see include/ea.h)."""
+    check(_lib.load().ea_shutdown(), "ea_shutdown")
+
+
 def ea_hybrid_attn_host_chunks(p: EaAttnParams, kv_heads_per_chunk: int = 0) -> int:
     return int(_lib.load().ea_hybrid_attn_host_chunks(ctypes.byref(p), int(kv_heads_per_chunk)))
 

@@ -945,15 +945,18 @@ int host_chunk(const ea_attn_params* p, int kv_heads_per_chunk) {
   return std::max(1, std::min(c, p->Hkv));
 }
 
-// The two copy streams (upload, download) of the current device, created
-// non-blocking on first use and kept until the process exits.
+// The two copy streams (upload, download) of each device, created
+// non-blocking on first use and kept until ea_shutdown or the process exits.
+cudaStream_t g_up[ea::kMaxSmDevices] = {};
+cudaStream_t g_down[ea::kMaxSmDevices] = {};
+std::mutex g_stream_mu;
+
 bool host_copy_streams(cudaStream_t* up, cudaStream_t* down) {
-  static cudaStream_t s_up[ea::kMaxSmDevices] = {};
-  static cudaStream_t s_down[ea::kMaxSmDevices] = {};
-  static std::mutex mu;
+  cudaStream_t* s_up = g_up;
+  cudaStream_t* s_down = g_down;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= ea::kMaxSmDevices) return false;
-  std::lock_guard<std::mutex> lock(mu);
+  std::lock_guard<std::mutex> lock(g_stream_mu);
   if (!s_up[dev]) {
     cudaStream_t a = nullptr, b = nullptr;
     if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return false;
@@ -985,6 +988,30 @@ struct CallEvents {
 };
 
 }  // namespace
+
+ea_status ea_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_stream_mu);
+  int cur = -1;
+  bool any = false;
+  ea_status st = EA_OK;
+  for (int dev = 0; dev < ea::kMaxSmDevices; ++dev) {
+    if (!g_up[dev]) continue;
+    if (!any) {
+      if (cudaGetDevice(&cur) != cudaSuccess) return EA_ERR_CUDA;
+      any = true;
+    }
+    // a stream's work finishes before it is destroyed
+    if (cudaSetDevice(dev) != cudaSuccess || cudaStreamSynchronize(g_up[dev]) != cudaSuccess ||
+        cudaStreamSynchronize(g_down[dev]) != cudaSuccess ||
+        cudaStreamDestroy(g_up[dev]) != cudaSuccess ||
+        cudaStreamDestroy(g_down[dev]) != cudaSuccess)
+      st = EA_ERR_CUDA;
+    g_up[dev] = nullptr;
+    g_down[dev] = nullptr;
+  }
+  if (any && cudaSetDevice(cur) != cudaSuccess) st = EA_ERR_CUDA;
+  return st;
+}
 
 size_t ea_hybrid_attn_host_workspace_size(const ea_attn_params* p, int hidden) {
   if (check_params(p) != EA_OK || hidden < 0 || hidden > kRouterMaxHidden) return 0;

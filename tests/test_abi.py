@@ -210,3 +210,9 @@ def test_host_workspace_and_chunks(lib):
     assert ea_hybrid_attn_host_chunks(make_params(4, 32, 8, 16384, 128, 128, 512), 0) == 8
     assert ea_hybrid_attn_host_chunks(make_params(3, 4, 2, 512, 64, 16, 128), 0) == 6
     assert ea_hybrid_attn_host_chunks(p, -1) == 0
+
+
+def test_shutdown_without_streams(lib):
+    """With no host-buffer call made, ea_shutdown has nothing to release and
+    makes no CUDA call (so it runs without a GPU)."""
+    assert lib.ea_shutdown() == _lib.EA_OK

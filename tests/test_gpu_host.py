@@ -194,3 +194,18 @@ def test_llama8b_full_size_matches_device_path():
     for h in range(0, w.hq, 5):
         ref = oracle.attention_rows(qf, kf, vf, ref_mask.numpy(), 0, h, rows, w.sink, w.window)
         compare(hp.out_host[0, h, rows], ref, f"llama8b host path head {h}")
+
+
+def test_shutdown_then_call_again():
+    """ea_shutdown releases the copy streams; the next call recreates them
+    and gives the same bits."""
+    from sparse_attention_head_b200.api import ea_shutdown
+    B, Hq, Hkv, N, d, S, W = 1, 4, 2, 400, 64, 8, 100
+    q, k, v = _qkv(B, Hq, Hkv, N, d, seed=71)
+    mask = torch.tensor([[0, 1, 1, 0]], dtype=torch.uint8)
+    first, _ = _host_path(q, k, v, S, W, 1, mask=mask)
+    ea_shutdown()
+    again, _ = _host_path(q, k, v, S, W, 1, mask=mask)
+    assert torch.equal(first, again)
+    ea_shutdown()
+    ea_shutdown()
