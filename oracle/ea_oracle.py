@@ -508,7 +508,9 @@ def router_gumbel_forward(k, w1, b1, w2, b2, g0, g1, tau: float):
     """Training-time routing: (r_hard [B,Hq] uint8, r_soft [B,Hq], z [B,Hq])."""
     z = router_mlp(router_pool(k), w1, b1, w2, b2)
     u = (z + np.asarray(g1, dtype=np.float64) - np.asarray(g0, dtype=np.float64)) / tau
-    r_soft = 1.0 / (1.0 + np.exp(-u))
+    # exp(-u) overflows to inf for u < -709, where the sigmoid is 0 anyway
+    with np.errstate(over="ignore"):
+        r_soft = 1.0 / (1.0 + np.exp(-u))
     r_hard = (u > 0.0).astype(np.uint8)
     return r_hard, r_soft, z
 
