@@ -762,6 +762,8 @@ class HostPrefill:
         return math.prod(self.shape_q) * 2
 
     def __call__(self, q_host, k_host, v_host, mask_host=None, stream=None):
+        if not self.has_router and mask_host is None:
+            raise ValueError("HostPrefill without router weights needs mask_host [B, Hq]")
         return ea_hybrid_attn_prefill_host(
             q_host, k_host, v_host, self.sink, self.window, out_host=self.out_host,
             workspace=self.workspace, router=self.router, threshold=self.threshold,

@@ -216,3 +216,14 @@ def test_shutdown_without_streams(lib):
     """With no host-buffer call made, ea_shutdown has nothing to release and
     makes no CUDA call (so it runs without a GPU)."""
     assert lib.ea_shutdown() == _lib.EA_OK
+
+
+def test_host_prefill_needs_a_mask_without_router():
+    """Without router weights the host-buffer wrapper needs the caller's mask
+    (checked before any CUDA work)."""
+    import torch
+    from sparse_attention_head_b200.api import HostPrefill
+    hp = HostPrefill.__new__(HostPrefill)
+    hp.has_router = False
+    with pytest.raises(ValueError):
+        hp(torch.zeros(1), torch.zeros(1), torch.zeros(1), None)
