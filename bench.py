@@ -41,6 +41,7 @@ import workloads  # noqa: E402
 
 METRIC = "effective prefill attention TFLOPS and tokens/s at 1 B200; % of bf16 tensor peak"
 UNIT = "TFLOP/s"
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 per B200 (the 2:4-sparse figure halved)
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
@@ -303,6 +304,8 @@ def run_ours(args, rank, world, local_rank):
                          % ((B * (Hq + 2 * Hkv) * N * d * 2) / 2 ** 20)},
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_bf16_peak": round(100.0 * value / world / peak, 2),
+        # the same against the nominal dense bf16 figure (2.25 PFLOP/s per GPU)
+        "pct_of_nominal_bf16_dense": round(100.0 * value / world / NOMINAL_BF16_TFLOPS, 2),
         "tile_granular_tflops": round(tile * world / (ms_per_step * 1e-3) / 1e12, 2),
         "attn_ms": round(attn_avg_ms, 4),
         "router_ms": round(statistics.mean(router_ms), 4),
