@@ -25,6 +25,10 @@
  *    back with ea_get_device_status.
  *  - Calls on different streams may run concurrently as long as each has its
  *    own workspace and output buffers.
+ *  - ea_router_decide, ea_hybrid_attn_prefill and ea_hybrid_attn_decode may
+ *    be captured into a CUDA graph once each has run eagerly on the device
+ *    (the first call sets the kernels' shared-memory attributes); replays
+ *    read the captured buffers' current contents.
  */
 #ifndef EA_H_
 #define EA_H_
