@@ -252,7 +252,8 @@ constexpr int kSchedBins = 4096;
 //      the rest; dQ: the sorted units are dealt in a snake, which already
 //      balances its many similar units;
 //   3. each CTA's units are listed in sorted order.
-// Every step is deterministic (the scatters run in order on one warp), so
+// Every step is deterministic: the sort's scatter and the dK/dV assignment
+// and lists run in order on one warp, and the dQ lists are closed forms, so
 // the schedule is the same on every run.  Results do not depend on it: a
 // unit owns its output tile.
 template <bool kDkDv>
