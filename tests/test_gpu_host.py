@@ -209,3 +209,24 @@ def test_shutdown_then_call_again():
     assert torch.equal(first, again)
     ea_shutdown()
     ea_shutdown()
+
+
+def test_two_calls_in_flight_on_two_streams():
+    """Two host-buffer calls with their own workspaces, enqueued on two
+    streams before either is synchronised, share the library's copy streams;
+    each still equals the device path."""
+    B, Hq, Hkv, N, d, S, W = 1, 8, 4, 900, 128, 16, 200
+    calls = []
+    for seed in (81, 82):
+        q, k, v = _qkv(B, Hq, Hkv, N, d, seed=seed)
+        router, _ = _router(k, Hq, 32, seed=seed + 100)
+        hp = HostPrefill(B, Hq, Hkv, N, d, *router, S, W, device=DEV, kv_heads_per_chunk=1)
+        calls.append((hp, (q, k, v), router, torch.cuda.Stream()))
+    torch.cuda.synchronize()
+    for hp, (q, k, v), _, stream in calls:
+        hp(q, k, v, stream=stream)
+    torch.cuda.synchronize()
+    for hp, (q, k, v), router, _ in calls:
+        ref_out, _ = _device_path(q, k, v, S, W, router=router)
+        assert torch.equal(hp.out_host, ref_out)
+        assert ea_get_device_status(hp.workspace) == 0
