@@ -215,8 +215,8 @@ int list_units(const HostSched& h, int Hq, int S, int W, int32_t* units_out, int
     EaCursor cur;
     ea_cursor_init(cur, h.view);
     for (int r = 0; r < total && r < max_units; ++r) {
-      int sparse, e, pair;
-      ea_cursor_seek(cur, h.view, r, &sparse, &e, &pair);
+      int sparse = 0, e = 0, pair = 0;
+      if (!ea_cursor_seek(cur, h.view, r, &sparse, &e, &pair)) break;
       const int idx = h.ent[sparse ? h.nfa + e : e];
       const EaShape sh = ea_make_shape(h.len[idx / Hq], S, W);
       const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
@@ -888,8 +888,8 @@ int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int ran
   if (rank < 0 || rank >= total) return -1;
   EaCursor cur;
   ea_cursor_init(cur, h.view);
-  int sparse, e, pair;
-  ea_cursor_seek(cur, h.view, rank, &sparse, &e, &pair);
+  int sparse = 0, e = 0, pair = 0;
+  if (!ea_cursor_seek(cur, h.view, rank, &sparse, &e, &pair)) return -1;
   const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
   const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
   for (int i = 0; i < ut.n && i < max_tiles; ++i) {
