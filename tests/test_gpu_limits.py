@@ -87,3 +87,31 @@ def test_router_at_its_largest_sizes():
     np.testing.assert_array_equal(mask.cpu().numpy(), mask_ref)
     # fp32 sums of 8192 and 4096 terms: measured max |z - z_ref| ~5e-6 on a B200
     np.testing.assert_allclose(f64(z), z_ref, rtol=0, atol=LOGIT_ABS)
+
+
+def test_decode_step_at_the_group_limit():
+    """B * Hkv = 4096 (sequence, kv head) groups, every kind of group (all
+    SA with a compact cache, mixed, all FA), ragged positions."""
+    from test_gpu_decode import _caches, _history, _mask, _prefill_caches, _step
+    from sparse_attention_head_b200.api import (decode_workspace, ea_decode_kv_policy,
+                                                make_decode_params)
+    B, Hq, Hkv, d, S, W, max_len = 512, 32, 8, 64, 4, 32, 80
+    pos = np.random.default_rng(5).integers(0, max_len, size=B).tolist()
+    L = max(pos) + 1
+    q, k, v = _history(B, Hq, Hkv, L, d, seed=99)
+    mask = _mask(B, Hq, Hkv, seed=98)
+    slots, n_full, n_sa = ea_decode_kv_policy(mask, Hkv)
+    caches = _caches(slots, n_full, n_sa, max_len, S, W, d)
+    _prefill_caches(caches, slots, k, v, pos, S, W)
+    ws = decode_workspace(make_decode_params(B, Hq, Hkv, d, S, W, max_len, n_full, n_sa), DEV)
+    idx = torch.as_tensor(pos, dtype=torch.long)
+    bi = torch.arange(B)
+    q_t, k_t, v_t = q[bi, :, idx], k[bi, :, idx], v[bi, :, idx]
+    out = _step(q_t, k_t, v_t, pos, mask, slots, caches, S, W, max_len, ws)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    ref = oracle.decode_step(f64(q_t), f64(k), f64(v), pos, mask, S, W)
+    # position 0 sees one key and positions 1-3 at most four: the few-key
+    # allowance of bf16 output rounding applies to those rows
+    few = np.array([p <= 3 for p in pos], dtype=bool)[:, None, None]
+    compare(out, ref, "decode at 4096 groups", few_rows=few)
