@@ -115,3 +115,28 @@ def test_decode_step_at_the_group_limit():
     # allowance of bf16 output rounding applies to those rows
     few = np.array([p <= 3 for p in pos], dtype=bool)[:, None, None]
     compare(out, ref, "decode at 4096 groups", few_rows=few)
+
+
+def test_backward_with_many_heads():
+    """2048 (batch, head) entries with eight query heads per kv head, two key
+    tiles: the backward's cost-sorted schedule over 512 dK/dV units and 4096
+    dQ units, against the oracle."""
+    from sparse_attention_head_b200.api import (ea_hybrid_attn_backward,
+                                                ea_hybrid_attn_prefill_lse)
+    B, Hq, Hkv, N, d, S, W = 32, 64, 8, 150, 128, 8, 64
+    q, k, v, dout = (_rand(s, 30 + i) for i, s in
+                     enumerate(((B, Hq, N, d), (B, Hkv, N, d), (B, Hkv, N, d), (B, Hq, N, d))))
+    mn = np.random.default_rng(31).integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    m = torch.as_tensor(mn, device=DEV)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    out, lse = ea_hybrid_attn_prefill_lse(qd, kd, vd, m, S, W)
+    dq, dk, dv = ea_hybrid_attn_backward(qd, kd, vd, out, dod, lse, m, S, W)
+    torch.cuda.synchronize()
+    rq, rk, rv = oracle.attention_backward(f64(q), f64(k), f64(v), f64(dout), mn, S, W)
+    # the normwise bound of the backward tests: P and dS enter the tensor cores
+    # as bf16 and the results are bf16 (2^-6 of the max, 2^-7 of the mean)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        err = np.abs(f64(got) - ref)
+        assert np.all(np.isfinite(f64(got))), name
+        assert err.max() <= 2.0 ** -6 * np.abs(ref).max(), (name, float(err.max()))
+        assert err.mean() <= 2.0 ** -7 * np.abs(ref).mean(), (name, float(err.mean()))
