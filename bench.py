@@ -80,6 +80,9 @@ def parse_args():
                     help="run only the packed-batch measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
+    ap.add_argument("--host-timeline", action="store_true",
+                    help="one host-buffer call under the torch profiler: device busy and "
+                         "overlap times of the uploads, downloads and kernels (JSON)")
     return ap.parse_args()
 
 
@@ -650,6 +653,70 @@ def measure_packed(w: workloads.Workload, nseq: int, steps: int, warmup: int, de
 
 
 # ---------------------------------------------------------------- backward
+
+def _union_ms(intervals):
+    """Total length of a union of (start, end) intervals (microseconds in,
+    milliseconds out)."""
+    total, cur_s, cur_e = 0.0, None, None
+    for a, b in sorted(intervals):
+        if cur_e is None or a > cur_e:
+            if cur_e is not None:
+                total += cur_e - cur_s
+            cur_s, cur_e = a, b
+        else:
+            cur_e = max(cur_e, b)
+    if cur_e is not None:
+        total += cur_e - cur_s
+    return total / 1000.0
+
+
+def host_timeline(w: workloads.Workload, dev):
+    """One call of the host-buffer path (after two warm-up calls) under the
+    torch profiler, whose CUDA activity records give every copy and kernel
+    its device start and end: the span of the call, the busy time of the
+    uploads, the downloads and our kernels, and how much of the kernels' and
+    the downloads' time overlaps the uploads."""
+    from torch.profiler import ProfilerActivity, profile
+    from sparse_attention_head_b200.api import HostPrefill
+    L = make_layer(w, 0, 0, dev)
+    B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
+    router = L["router"] if L["router"] is not None else (None, None, None, None)
+    hp = HostPrefill(B, Hq, Hkv, N, d, *router, w.sink, w.window, device=dev)
+    qh, kh, vh = (L[x].cpu().pin_memory() for x in ("q", "k", "v"))
+    mh = None if L["router"] is not None else L["mask"].cpu().pin_memory()
+    for _ in range(2):
+        hp(qh, kh, vh, mh)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        hp(qh, kh, vh, mh)
+        torch.cuda.synchronize()
+    h2d, d2h, kern = [], [], []
+    for e in prof.events():
+        if e.device_type.name != "CUDA":
+            continue
+        iv = (e.time_range.start, e.time_range.end)
+        name = e.name.lower()
+        if "memcpy" in name and "htod" in name:
+            h2d.append(iv)
+        elif "memcpy" in name and "dtoh" in name:
+            d2h.append(iv)
+        elif name.startswith("ea::") or "ea::" in name:
+            kern.append(iv)
+    every = h2d + d2h + kern
+    span = (max(b for _, b in every) - min(a for a, _ in every)) / 1000.0 if every else 0.0
+    up = _union_ms(h2d)
+    return {
+        "workload": w.name, "chunks": hp.chunks,
+        "span_ms": round(span, 3),
+        "h2d_busy_ms": round(up, 3), "d2h_busy_ms": round(_union_ms(d2h), 3),
+        "kernel_busy_ms": round(_union_ms(kern), 3),
+        "kernel_overlapping_h2d_ms": round(_union_ms(kern) + up - _union_ms(kern + h2d), 3),
+        "d2h_overlapping_h2d_ms": round(_union_ms(d2h) + up - _union_ms(d2h + h2d), 3),
+        "copies": {"h2d": len(h2d), "d2h": len(d2h)}, "kernels": len(kern),
+        "h2d_bytes": hp.h2d_bytes(), "d2h_bytes": hp.d2h_bytes(),
+    }
+
+
 def measure_training(w: workloads.Workload, steps: int, warmup: int, dev, stream):
     """One layer's attention training step, every phase timed with CUDA events:
     the Gumbel-Softmax router decision, the forward of both modes in one
@@ -989,6 +1056,16 @@ def main():
             w = dataclasses.replace(w, seq=args.seq)
         res = measure_training(w, args.steps, max(args.warmup, 3), dev,
                                torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return 0
+    if args.host_timeline:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = host_timeline(w, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
         return 0
