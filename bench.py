@@ -80,6 +80,9 @@ def parse_args():
                     help="run only the packed-batch measurement and print its JSON object")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
+    ap.add_argument("--unit-trace", action="store_true",
+                    help="one fused-attention launch with the per-unit trace: the CTAs' "
+                         "finish spread, busy fraction and FA/SA interleave (JSON)")
     ap.add_argument("--host-timeline", action="store_true",
                     help="one host-buffer call under the torch profiler: device busy and "
                          "overlap times of the uploads, downloads and kernels (JSON)")
@@ -654,6 +657,66 @@ def measure_packed(w: workloads.Workload, nseq: int, steps: int, warmup: int, de
 
 # ---------------------------------------------------------------- backward
 
+
+def unit_trace(w: workloads.Workload, dev):
+    """Layer 0's fused attention launch with the per-unit trace (after two
+    untraced warm-up launches): how evenly the persistent CTAs finish, how
+    busy they are, how much of the launch runs FA and SA units at the same
+    time, and the time per KV tile of each mode."""
+    from sparse_attention_head_b200.api import (attn_workspace, ea_hybrid_attn_prefill,
+                                                ea_hybrid_attn_prefill_traced,
+                                                ea_router_decide, make_params)
+    L = make_layer(w, 0, 0, dev)
+    B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
+    if L["router"] is not None:
+        mask, _ = ea_router_decide(L["k"], *L["router"], want_logits=False)
+    else:
+        mask = L["mask"]
+    ws = attn_workspace(make_params(B, Hq, Hkv, N, d, w.sink, w.window), dev)
+    out = torch.empty_like(L["q"])
+    for _ in range(2):
+        ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], mask, w.sink, w.window, out=out,
+                               workspace=ws)
+    torch.cuda.synchronize()
+    _, rec, total = ea_hybrid_attn_prefill_traced(L["q"], L["k"], L["v"], mask, w.sink,
+                                                  w.window, out=out, workspace=ws,
+                                                  max_records=1 << 17)
+    start, end, cta, sparse, tiles = rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 4], rec[:, 5]
+    t0 = start.min()
+    span = float(end.max() - t0) / 1e3
+    ctas = np.unique(cta)
+    last_end = np.array([end[cta == c].max() for c in ctas], dtype=np.float64)
+    busy = np.array([(end[cta == c] - start[cta == c]).sum() for c in ctas], dtype=np.float64)
+    # time during which an FA unit and an SA unit are both in progress
+    ev = sorted([(int(a), 1, int(sp)) for a, sp in zip(start, sparse)] +
+                [(int(b), -1, int(sp)) for b, sp in zip(end, sparse)])
+    live = [0, 0]
+    both, prev = 0, None
+    for t, delta, sp in ev:
+        if prev is not None and live[0] > 0 and live[1] > 0:
+            both += t - prev
+        live[sp] += delta
+        prev = t
+    per_tile = {}
+    for sp, name in ((0, "fa"), (1, "sa")):
+        sel = sparse == sp
+        if sel.any():
+            per_tile[name + "_us_per_tile"] = round(
+                float((end[sel] - start[sel]).sum()) / 1e3 / float(tiles[sel].sum()), 3)
+    return {
+        "workload": w.name, "units": int(total), "ctas": int(len(ctas)),
+        "fa_units": int((sparse == 0).sum()), "sa_units": int((sparse == 1).sum()),
+        "span_us": round(span, 1),
+        "cta_finish_us": {"min": round(float(last_end.min() - t0) / 1e3, 1),
+                          "median": round(float(np.median(last_end) - t0) / 1e3, 1),
+                          "max": round(float(last_end.max() - t0) / 1e3, 1)},
+        "tail_us": round(float(last_end.max() - np.median(last_end)) / 1e3, 1),
+        "busy_fraction": round(float(busy.sum()) / (len(ctas) * span * 1e3), 4),
+        "fa_sa_concurrent_fraction": round(both / (span * 1e3), 4),
+        **per_tile,
+    }
+
+
 def _union_ms(intervals):
     """Total length of a union of (start, end) intervals (microseconds in,
     milliseconds out)."""
@@ -1056,6 +1119,16 @@ def main():
             w = dataclasses.replace(w, seq=args.seq)
         res = measure_training(w, args.steps, max(args.warmup, 3), dev,
                                torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return 0
+    if args.unit_trace:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        w = workloads.get(args.workload)
+        if args.seq:
+            w = dataclasses.replace(w, seq=args.seq)
+        res = unit_trace(w, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
         return 0

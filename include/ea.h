@@ -216,6 +216,23 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
                                      void* out, float* lse, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* ea_hybrid_attn_prefill with a per-unit trace, for load-balance
+ * measurements (the results are those of the untraced call, bit for bit).
+ * trace: device
+ * uint64 [4 + 4 * trace_records], 8-byte aligned, ZEROED by the caller before
+ * the call.  trace[0] receives the number of work units the launch ran; the
+ * first trace_records units, in completion order, each leave four values at
+ * trace[4 + 4 i]: the unit's start and end on the device's global timer
+ * (ns; start when its first query slot begins, end when that slot's rows are
+ * stored), (CTA index << 32) | schedule rank, and (1 if SA << 32) | its KV
+ * tile count.  Errors as for ea_hybrid_attn_prefill, plus EA_ERR_INVALID_ARG
+ * for a NULL trace or negative trace_records. */
+ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,
+                                        const uint8_t* route_mask, const ea_attn_params* p,
+                                        void* out, void* workspace, size_t workspace_bytes,
+                                        unsigned long long* trace, int trace_records,
+                                        void* stream);
+
 /* Forward of a training step: every head in BOTH modes, in one launch.  The
  * mode route_mask chooses goes to out, with its log-sum-exp in lse (as
  * ea_hybrid_attn_prefill_lse); the other mode to out_other (device bf16

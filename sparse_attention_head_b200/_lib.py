@@ -45,6 +45,7 @@ EXPORTED = [
     "ea_hybrid_attn_prefill_train", "ea_fp8_vt_stride", "ea_quantize_fp8_workspace_size",
     "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8", "ea_hybrid_attn_host_workspace_size",
     "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host", "ea_shutdown",
+    "ea_hybrid_attn_prefill_traced",
 ]
 
 
@@ -110,6 +111,9 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_workspace_size.argtypes = [pparams]
     lib.ea_hybrid_attn_host_workspace_size.restype = c_size
     lib.ea_hybrid_attn_host_workspace_size.argtypes = [pparams, c_int]
+    lib.ea_hybrid_attn_prefill_traced.restype = c_int
+    lib.ea_hybrid_attn_prefill_traced.argtypes = [vp, vp, vp, vp, pparams, vp, vp, c_size, vp,
+                                                  c_int, vp]
     lib.ea_shutdown.restype = c_int
     lib.ea_shutdown.argtypes = []
     lib.ea_hybrid_attn_host_chunks.restype = c_int

@@ -192,6 +192,39 @@ def ea_hybrid_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out
 
 
+def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  route_mask: torch.Tensor, sink: int, window: int, *,
+                                  max_records: int = 65536, out: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None):
+    """ea_hybrid_attn_prefill with a per-unit trace: (out, records int64
+    [n, 6] = start_ns, end_ns, cta, rank, sparse, kv_tiles, total units).
+    Synchronises the device to read the trace back."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    _need(route_mask, "route_mask", torch.uint8)
+    B, Hq, N, d = q.shape
+    p = make_params(B, Hq, k.shape[1], N, d, sink, window)
+    out = torch.empty_like(q) if out is None else out
+    workspace = attn_workspace(p, q.device) if workspace is None else workspace
+    trace = torch.zeros(4 + 4 * int(max_records), dtype=torch.int64, device=q.device)
+    rc = lib.ea_hybrid_attn_prefill_traced(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           route_mask.data_ptr(), ctypes.byref(p),
+                                           out.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), trace.data_ptr(),
+                                           int(max_records), _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill_traced")
+    t = trace.cpu().numpy()
+    total = int(t[0])
+    n = min(total, int(max_records))
+    rec = t[4:4 + 4 * n].reshape(n, 4)
+    cols = np.stack([rec[:, 0], rec[:, 1], rec[:, 2] >> 32, rec[:, 2] & 0xffffffff,
+                     rec[:, 3] >> 32, rec[:, 3] & 0xffffffff], axis=1)
+    return out, cols, total
+
+
 # ---------------------------------------------------------------- packed batches
 def make_varlen_params(B, Hq, Hkv, total, max_seqlen, d, sink, window, softmax_scale=0.0,
                        select=EA_SELECT_ALL) -> EaVarlenParams:

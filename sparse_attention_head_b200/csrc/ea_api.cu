@@ -408,9 +408,10 @@ int ea_attn_grid_size(const ea_attn_params* p, int num_sms) {
   return static_cast<int>(units < num_sms ? units : num_sms);
 }
 
-ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
-                                 const uint8_t* route_mask, const ea_attn_params* p, void* out,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+static ea_status prefill_impl(const void* q, const void* k, const void* v,
+                              const uint8_t* route_mask, const ea_attn_params* p, void* out,
+                              void* workspace, size_t workspace_bytes,
+                              unsigned long long* trace, int trace_max, void* stream) {
   ea_status st = check_params(p);
   if (st != EA_OK) return st;
   if (!q || !k || !v || !route_mask || !out) return EA_ERR_INVALID_ARG;
@@ -440,12 +441,32 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.trace = trace;
+  args.trace_max = trace_max;
 
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
   const int grid = ea_attn_grid_size(p, sms);
   cudaError_t err = ea::launch_attn(p->d, args, grid, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
+                                 const uint8_t* route_mask, const ea_attn_params* p, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, nullptr, 0,
+                      stream);
+}
+
+ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,
+                                        const uint8_t* route_mask, const ea_attn_params* p,
+                                        void* out, void* workspace, size_t workspace_bytes,
+                                        unsigned long long* trace, int trace_records,
+                                        void* stream) {
+  if (!trace || trace_records < 0) return EA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(trace) & 7u) != 0) return EA_ERR_MISALIGNED;
+  return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, trace,
+                      trace_records, stream);
 }
 
 // Forward of a training step (padded BHSD): the chosen mode with its

@@ -596,6 +596,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       const EaShape shape = ea_make_shape(seq_len, args.sink, args.window);
       const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
       if (slot >= ut.nslots) continue;
+      const uint64_t unit_t0 = (args.trace && warp == 0 && lane == 0) ? global_ns() : 0;
       const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
       // FP8: the scores carry the q and k dequantization scales
       const int kvh = seq * args.Hkv + (idx % args.Hq) / G;
@@ -766,6 +767,17 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       }
       tc_fence_before();
       mbar_arrive(bars.o_empty + 8 * slot);
+      if (args.trace && warp == 0 && lane == 0) {
+        // slot 0's rows are stored: the unit's record
+        const unsigned long long k = atomicAdd(args.trace, 1ull);
+        if (k < static_cast<unsigned long long>(args.trace_max)) {
+          unsigned long long* rec = args.trace + 4 + 4 * k;
+          rec[0] = unit_t0;
+          rec[1] = global_ns();
+          rec[2] = (static_cast<unsigned long long>(blockIdx.x) << 32) | static_cast<unsigned>(r);
+          rec[3] = (static_cast<unsigned long long>(sparse) << 32) | static_cast<unsigned>(ut.n);
+        }
+      }
     }
   }
 

@@ -1,0 +1,58 @@
+"""The per-unit trace of the fused prefill (ea_hybrid_attn_prefill_traced):
+the output equals the untraced call's bits, and the trace holds one record
+per unit of the host schedule view, each on the CTA the snake deal assigns,
+with that unit's mode and tile count."""
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_head_b200 import build
+from sparse_attention_head_b200.api import (attn_workspace, ea_attn_grid_size,
+                                            ea_get_device_status, ea_hybrid_attn_prefill,
+                                            ea_hybrid_attn_prefill_traced, ea_schedule_units,
+                                            make_params)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,S,W", [
+    (1, 8, 2, 2048, 128, 64, 256),
+    (2, 16, 4, 700, 64, 8, 100),
+])
+def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
+    g = torch.Generator().manual_seed(N)
+    q, k, v = (torch.randn(s, generator=g).to(torch.bfloat16).to(DEV) for s in
+               ((B, Hq, N, d), (B, Hkv, N, d), (B, Hkv, N, d)))
+    m = np.random.default_rng(N).integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    mask = torch.from_numpy(m).to(DEV)
+    p = make_params(B, Hq, Hkv, N, d, S, W)
+    ws = attn_workspace(p, DEV)
+    plain = ea_hybrid_attn_prefill(q, k, v, mask, S, W, workspace=ws)
+    traced, rec, total = ea_hybrid_attn_prefill_traced(q, k, v, mask, S, W, workspace=ws)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    assert torch.equal(plain, traced)
+    units = ea_schedule_units(m, p)                 # rows: sparse, b, h, pair, n_kv_tiles
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    grid = ea_attn_grid_size(p, sms)
+    assert total == len(units) == len(rec)
+    start, end, cta, rank, sparse, tiles = (rec[:, i] for i in range(6))
+    assert sorted(rank.tolist()) == list(range(total))
+    assert np.all(end >= start) and np.all(start > 0)
+    k_round, j = rank // grid, rank % grid
+    np.testing.assert_array_equal(cta, np.where(k_round % 2 == 0, j, grid - 1 - j))
+    np.testing.assert_array_equal(sparse, units[rank, 0])
+    np.testing.assert_array_equal(tiles, units[rank, 4])
+    # a CTA runs its units one after another, in rank order
+    for c in np.unique(cta):
+        sel = np.where(cta == c)[0]
+        order = sel[np.argsort(rank[sel])]
+        assert np.all(start[order][1:] >= start[order][:-1])
