@@ -681,7 +681,8 @@ def unit_trace(w: workloads.Workload, dev):
     _, rec, total = ea_hybrid_attn_prefill_traced(L["q"], L["k"], L["v"], mask, w.sink,
                                                   w.window, out=out, workspace=ws,
                                                   max_records=1 << 17)
-    start, end, cta, sparse, tiles = rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 4], rec[:, 5]
+    start, first_s, last_p, end = rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 3]
+    cta, sparse, tiles = rec[:, 4], rec[:, 6], rec[:, 7]
     t0 = start.min()
     span = float(end.max() - t0) / 1e3
     ctas = np.unique(cta)
@@ -714,6 +715,13 @@ def unit_trace(w: workloads.Workload, dev):
         "busy_fraction": round(float(busy.sum()) / (len(ctas) * span * 1e3), 4),
         "fa_sa_concurrent_fraction": round(both / (span * 1e3), 4),
         **per_tile,
+        # a unit's phases, as its first query slot sees them (mean, us): from
+        # its start to its first score tile, from there to its last P, and
+        # from its last P to its rows stored
+        "unit_ramp_us": round(float((first_s - start).mean()) / 1e3, 3),
+        "unit_body_us": round(float((last_p - first_s).mean()) / 1e3, 3),
+        "unit_drain_us": round(float((end - last_p).mean()) / 1e3, 3),
+        "unit_tiles_mean": round(float(tiles.mean()), 2),
     }
 
 

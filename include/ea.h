@@ -218,15 +218,19 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
 
 /* ea_hybrid_attn_prefill with a per-unit trace, for load-balance
  * measurements (the results are those of the untraced call, bit for bit).
+ * It launches a kernel instantiation of its own, the untraced kernel plus the
+ * trace stores, so ea_hybrid_attn_prefill carries none of that code.
  * trace: device
- * uint64 [4 + 4 * trace_records], 8-byte aligned, ZEROED by the caller before
+ * uint64 [8 + 6 * trace_records], 8-byte aligned, ZEROED by the caller before
  * the call.  trace[0] receives the number of work units the launch ran; the
- * first trace_records units, in completion order, each leave four values at
- * trace[4 + 4 i]: the unit's start and end on the device's global timer
- * (ns; start when its first query slot begins, end when that slot's rows are
- * stored), (CTA index << 32) | schedule rank, and (1 if SA << 32) | its KV
- * tile count.  Errors as for ea_hybrid_attn_prefill, plus EA_ERR_INVALID_ARG
- * for a NULL trace or negative trace_records. */
+ * first trace_records units, in completion order, each leave six values at
+ * trace[8 + 6 i], times on the device's global timer in ns, all seen by the
+ * unit's first query slot: its start, the moment its first score tile was
+ * ready, the moment it handed over its last probabilities, its end (its rows
+ * stored); then (CTA index << 32) | schedule rank, and (1 if SA << 32) | its
+ * KV tile count.  Errors as for ea_hybrid_attn_prefill, plus EA_ERR_INVALID_ARG
+ * for a NULL trace or negative trace_records and EA_ERR_MISALIGNED for a trace
+ * that is not 8-byte aligned. */
 ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,
                                         const uint8_t* route_mask, const ea_attn_params* p,
                                         void* out, void* workspace, size_t workspace_bytes,

@@ -198,8 +198,8 @@ def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
                                   workspace: Optional[torch.Tensor] = None,
                                   stream: Optional[torch.cuda.Stream] = None):
     """ea_hybrid_attn_prefill with a per-unit trace: (out, records int64
-    [n, 6] = start_ns, end_ns, cta, rank, sparse, kv_tiles, total units).
-    Synchronises the device to read the trace back."""
+    [n, 8] = start_ns, first_s_ns, last_p_ns, end_ns, cta, rank, sparse,
+    kv_tiles, total units).  Synchronises the device to read the trace back."""
     lib = _lib.load()
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
@@ -209,7 +209,7 @@ def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
     p = make_params(B, Hq, k.shape[1], N, d, sink, window)
     out = torch.empty_like(q) if out is None else out
     workspace = attn_workspace(p, q.device) if workspace is None else workspace
-    trace = torch.zeros(4 + 4 * int(max_records), dtype=torch.int64, device=q.device)
+    trace = torch.zeros(8 + 6 * int(max_records), dtype=torch.int64, device=q.device)
     rc = lib.ea_hybrid_attn_prefill_traced(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                            route_mask.data_ptr(), ctypes.byref(p),
                                            out.data_ptr(), workspace.data_ptr(),
@@ -219,9 +219,9 @@ def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
     t = trace.cpu().numpy()
     total = int(t[0])
     n = min(total, int(max_records))
-    rec = t[4:4 + 4 * n].reshape(n, 4)
-    cols = np.stack([rec[:, 0], rec[:, 1], rec[:, 2] >> 32, rec[:, 2] & 0xffffffff,
-                     rec[:, 3] >> 32, rec[:, 3] & 0xffffffff], axis=1)
+    rec = t[8:8 + 6 * n].reshape(n, 6)
+    cols = np.stack([rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 3], rec[:, 4] >> 32,
+                     rec[:, 4] & 0xffffffff, rec[:, 5] >> 32, rec[:, 5] & 0xffffffff], axis=1)
     return out, cols, total
 
 

@@ -195,7 +195,9 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
   return grid_sync(args, s_flag);
 }
 
-template <int D, bool kRouted, bool kFp8 = false>
+// kTrace: the per-unit trace (its own instantiation, so the others carry none
+// of its code or registers)
+template <int D, bool kRouted, bool kFp8 = false, bool kTrace = false>
 __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_constant__ AttnArgs args) {
   using C = AttnCfg<D, kFp8>;
   extern __shared__ uint8_t smem_raw[];
@@ -228,6 +230,9 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_counts = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // nFA, nSA
+  // per-unit trace times of softmax warp 0 lane 0 (unit start, first S ready,
+  // last P handed over): kept in shared memory, off the softmax registers
+  uint64_t* s_trace_ts = reinterpret_cast<uint64_t*>(smem + C::kOffMisc + 32);
   uint16_t* s_ent = reinterpret_cast<uint16_t*>(smem + C::kOffEnt);
 
 
@@ -596,7 +601,12 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       const EaShape shape = ea_make_shape(seq_len, args.sink, args.window);
       const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
       if (slot >= ut.nslots) continue;
-      const uint64_t unit_t0 = (args.trace && warp == 0 && lane == 0) ? global_ns() : 0;
+      const bool tracing = kTrace && warp == 0 && lane == 0;
+      if (tracing) {
+        s_trace_ts[0] = global_ns();
+        s_trace_ts[1] = 0;
+        s_trace_ts[2] = 0;
+      }
       const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
       // FP8: the scores carry the q and k dequantization scales
       const int kvh = seq * args.Hkv + (idx % args.Hq) / G;
@@ -613,6 +623,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++s_cnt;
+        if (tracing && s_trace_ts[1] == 0) s_trace_ts[1] = global_ns();   // first S ready
         tc_fence_after();
         float x[128];
         {
@@ -732,6 +743,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         has_o = true;
       }
       if (!ok) break;
+      if (tracing) s_trace_ts[2] = global_ns();   // the unit's last P is handed over
       // Epilogue: O / l -> bf16 -> out[b, h, row, :].
       ok = mbar_wait(bars.o_done + 8 * slot, (pv_cnt - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
       ok = __all_sync(0xffffffffu, ok);
@@ -767,15 +779,17 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       }
       tc_fence_before();
       mbar_arrive(bars.o_empty + 8 * slot);
-      if (args.trace && warp == 0 && lane == 0) {
+      if (tracing) {
         // slot 0's rows are stored: the unit's record
         const unsigned long long k = atomicAdd(args.trace, 1ull);
         if (k < static_cast<unsigned long long>(args.trace_max)) {
-          unsigned long long* rec = args.trace + 4 + 4 * k;
-          rec[0] = unit_t0;
-          rec[1] = global_ns();
-          rec[2] = (static_cast<unsigned long long>(blockIdx.x) << 32) | static_cast<unsigned>(r);
-          rec[3] = (static_cast<unsigned long long>(sparse) << 32) | static_cast<unsigned>(ut.n);
+          unsigned long long* rec = args.trace + 8 + 6 * k;
+          rec[0] = s_trace_ts[0];
+          rec[1] = s_trace_ts[1];
+          rec[2] = s_trace_ts[2];
+          rec[3] = global_ns();
+          rec[4] = (static_cast<unsigned long long>(blockIdx.x) << 32) | static_cast<unsigned>(r);
+          rec[5] = (static_cast<unsigned long long>(sparse) << 32) | static_cast<unsigned>(ut.n);
         }
       }
     }
@@ -794,7 +808,7 @@ int attn_smem_bytes(int D) {
   return D == 128 ? AttnCfg<128>::kSmem : AttnCfg<64>::kSmem;
 }
 
-template <int D, bool kRouted, bool kFp8 = false>
+template <int D, bool kRouted, bool kFp8 = false, bool kTrace = false>
 static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream) {
   const int smem = AttnCfg<D, kFp8>::kSmem;
   static int configured[64] = {0};
@@ -802,13 +816,13 @@ static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream)
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev >= 64 || !configured[dev]) {
-    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D, kRouted, kFp8>,
+    err = cudaFuncSetAttribute(ea_hybrid_attn_kernel<D, kRouted, kFp8, kTrace>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     if (dev < 64) configured[dev] = 1;
   }
   if (!kRouted) {
-    ea_hybrid_attn_kernel<D, false, kFp8><<<grid, AttnCfg<D, kFp8>::kThreads, smem, stream>>>(args);
+    ea_hybrid_attn_kernel<D, false, kFp8, kTrace><<<grid, AttnCfg<D, kFp8>::kThreads, smem, stream>>>(args);
     return cudaGetLastError();
   }
   // every CTA must be resident at once: the runtime refuses a cooperative
@@ -819,8 +833,13 @@ static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream)
 }
 
 cudaError_t launch_attn(int D, const AttnArgs& args, int grid, cudaStream_t stream) {
-  if (D == 128) return launch_d<128, false>(args, grid, stream);
-  if (D == 64) return launch_d<64, false>(args, grid, stream);
+  const bool trace = args.trace != nullptr;
+  if (D == 128)
+    return trace ? launch_d<128, false, false, true>(args, grid, stream)
+                 : launch_d<128, false>(args, grid, stream);
+  if (D == 64)
+    return trace ? launch_d<64, false, false, true>(args, grid, stream)
+                 : launch_d<64, false>(args, grid, stream);
   return cudaErrorInvalidValue;
 }
 

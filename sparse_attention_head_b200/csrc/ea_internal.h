@@ -42,8 +42,9 @@ struct alignas(64) AttnArgs {
   // this K/V ring position, so the kernel's bounded wait for it runs out.
   int debug_drop_kv_pos;
   // Per-unit trace (nullptr = off): trace[0] counts records; record i sits
-  // at trace[4 + 4 i] .. +3 = {start ns, end ns, CTA << 32 | rank,
-  // sparse << 32 | KV tiles}; records past trace_max are counted, not kept.
+  // at trace[8 + 6 i] .. +5 = {start, first S ready, last P handed over,
+  // end (ns), CTA << 32 | rank, sparse << 32 | KV tiles}; records past
+  // trace_max are counted, not kept.
   unsigned long long* trace;
   int trace_max;
   // Routed launch only: the router runs in the kernel's prologue (pool,

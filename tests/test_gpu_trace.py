@@ -44,9 +44,10 @@ def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     grid = ea_attn_grid_size(p, sms)
     assert total == len(units) == len(rec)
-    start, end, cta, rank, sparse, tiles = (rec[:, i] for i in range(6))
+    start, first_s, last_p, end, cta, rank, sparse, tiles = (rec[:, i] for i in range(8))
     assert sorted(rank.tolist()) == list(range(total))
-    assert np.all(end >= start) and np.all(start > 0)
+    assert np.all(start > 0)
+    assert np.all(first_s >= start) and np.all(last_p >= first_s) and np.all(end >= last_p)
     k_round, j = rank // grid, rank % grid
     np.testing.assert_array_equal(cta, np.where(k_round % 2 == 0, j, grid - 1 - j))
     np.testing.assert_array_equal(sparse, units[rank, 0])
