@@ -681,6 +681,14 @@ def unit_trace(w: workloads.Workload, dev):
     _, rec, total = ea_hybrid_attn_prefill_traced(L["q"], L["k"], L["v"], mask, w.sink,
                                                   w.window, out=out, workspace=ws,
                                                   max_records=1 << 17)
+    return {"workload": w.name, **summarize_unit_trace(rec, total)}
+
+
+def summarize_unit_trace(rec: np.ndarray, total: int) -> dict:
+    """Balance figures of one traced launch.  rec: int64 [n, 8] rows of
+    (start, first S ready, last P handed over, end) in ns, CTA, rank, sparse,
+    KV tiles, as ea_hybrid_attn_prefill_traced returns them; total: units
+    the launch ran."""
     start, first_s, last_p, end = rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 3]
     cta, sparse, tiles = rec[:, 4], rec[:, 6], rec[:, 7]
     t0 = start.min()
@@ -688,7 +696,8 @@ def unit_trace(w: workloads.Workload, dev):
     ctas = np.unique(cta)
     last_end = np.array([end[cta == c].max() for c in ctas], dtype=np.float64)
     busy = np.array([(end[cta == c] - start[cta == c]).sum() for c in ctas], dtype=np.float64)
-    # time during which an FA unit and an SA unit are both in progress
+    # time during which an FA unit and an SA unit are both in progress (an end
+    # sorts before a start at the same instant: touching units do not overlap)
     ev = sorted([(int(a), 1, int(sp)) for a, sp in zip(start, sparse)] +
                 [(int(b), -1, int(sp)) for b, sp in zip(end, sparse)])
     live = [0, 0]
@@ -705,7 +714,7 @@ def unit_trace(w: workloads.Workload, dev):
             per_tile[name + "_us_per_tile"] = round(
                 float((end[sel] - start[sel]).sum()) / 1e3 / float(tiles[sel].sum()), 3)
     return {
-        "workload": w.name, "units": int(total), "ctas": int(len(ctas)),
+        "units": int(total), "ctas": int(len(ctas)),
         "fa_units": int((sparse == 0).sum()), "sa_units": int((sparse == 1).sum()),
         "span_us": round(span, 1),
         "cta_finish_us": {"min": round(float(last_end.min() - t0) / 1e3, 1),
