@@ -18,7 +18,7 @@ Sources are two pages about one method:
    layer's Key hidden states and a simple MLP emits one routing signal r per
    head; r = 0 sends the head to Full Attention (FA), r = 1 to Sparse
    Attention (SA).  The pages fix neither pooling, activation nor widths.
-   Readings taken here (all plain, all listed in the design doc):
+   Readings taken here (the plainest ones the text supports):
      - pooled input x[b] = mean over all N positions of K[b, :, n, :], flattened
        in (kv_head, channel) order;
      - h = ReLU(W1 x + b1), z = W2 h + b2 (nn.Linear convention, W is out x in);
