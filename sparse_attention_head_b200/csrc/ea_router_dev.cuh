@@ -95,8 +95,18 @@ __device__ __forceinline__ float router_x(const float* partials,
   int t0;
   const int len = router_seq_rows(cu, N, total, b, &t0);
   const float* p = partials + (static_cast<size_t>(b) * Hkv + hk) * nsplit * d + c;
+  // the partials are added in split order; the loads of 16 splits are issued
+  // before their adds, so their L2 latencies overlap instead of queueing
   float s = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) s += __ldcg(p + static_cast<size_t>(sp) * d);
+  int sp = 0;
+  for (; sp + 16 <= nsplit; sp += 16) {
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = __ldcg(p + static_cast<size_t>(sp + u) * d);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) s += v[u];
+  }
+  for (; sp < nsplit; ++sp) s += __ldcg(p + static_cast<size_t>(sp) * d);
   return len > 0 ? s * (1.0f / static_cast<float>(len)) : 0.f;
 }
 
