@@ -87,6 +87,24 @@ def test_attention_argument_errors(lib):
         _lib.EA_ERR_INVALID_ARG
 
 
+def test_traced_prefill_argument_errors(lib):
+    """The traced entry point's own checks (trace buffer, record count), then
+    the untraced call's; every case returns before any CUDA call."""
+    good = make_params(1, 4, 2, 512, 64, 16, 128)
+
+    def traced(p, trace=256, records=8, q=16, ws=256, wsbytes=256):
+        return lib.ea_hybrid_attn_prefill_traced(q, 16, 16, 16, ctypes.byref(p), 16, ws, wsbytes,
+                                                 trace, records, None)
+    assert traced(good, trace=None) == _lib.EA_ERR_INVALID_ARG
+    assert traced(good, records=-1) == _lib.EA_ERR_INVALID_ARG
+    assert traced(good, trace=260) == _lib.EA_ERR_MISALIGNED      # 4-byte aligned only
+    assert traced(make_params(0, 4, 2, 512, 64, 16, 128)) == _lib.EA_ERR_INVALID_ARG
+    assert traced(make_params(1, 4, 2, 512, 96, 16, 128)) == _lib.EA_ERR_UNSUPPORTED
+    assert traced(good, q=0) == _lib.EA_ERR_INVALID_ARG
+    assert traced(good, q=24) == _lib.EA_ERR_MISALIGNED
+    assert traced(good, wsbytes=4) == _lib.EA_ERR_WORKSPACE
+
+
 def test_workspace_sizes(lib):
     p = make_params(1, 32, 8, 32768, 128, 64, 1024)
     assert lib.ea_hybrid_attn_workspace_size(ctypes.byref(p)) >= 4
