@@ -4,6 +4,10 @@
 One step = one attention layer's prefill: the Attention Router
 (ea_router_decide) on the key states, then the fused hybrid FA/SA attention
 (ea_hybrid_attn_prefill), on seeded synthetic inputs already resident in HBM.
+The headline workload is the largest single-GPU configuration, a 256K-token
+layer (B1 N262144, 32 query / 8 kv heads, d128, sink 128, window 4096,
+router-chosen ~75% sparse heads); the other configurations follow under
+"workloads", each with its own roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -53,7 +57,13 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama8b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="ext256k", choices=sorted(workloads.WORKLOADS),
+                    help="headline workload (default: the largest single-GPU configuration)")
+    ap.add_argument("--side-workload", default="llama8b", choices=sorted(workloads.WORKLOADS),
+                    help="layer shape of the secondary measurements (packed batch, decode, "
+                         "FP8, training) when the headline workload is ext256k")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the attention measurements of the other configurations")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of the host-buffer end-to-end measurement (default: --steps)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -78,6 +88,8 @@ def parse_args():
                     help="skip the training-step measurement of the default line")
     ap.add_argument("--packed-only", action="store_true",
                     help="run only the packed-batch measurement and print its JSON object")
+    ap.add_argument("--ab-reps", type=int, default=20,
+                    help="calls of each arm in the interleaved comparator timings")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no comparators, e2e or CPU baseline")
     ap.add_argument("--unit-trace", action="store_true",
@@ -168,9 +180,10 @@ def visible_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
-def traffic_for_current_kernel():
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, only if it was taken on the current kernel source."""
+def traffic_for_current_kernel(workload: str, seq: int):
+    """Per-launch DRAM bytes of the attention kernel on this workload, from the
+    committed ncu summary: only if a capture exists for this workload at this
+    sequence length and was taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", "attn_traffic.json")
     src = os.path.join(ROOT, "sparse_attention_head_b200", "csrc", "ea_attn.cu")
     if not os.path.exists(path):
@@ -180,7 +193,54 @@ def traffic_for_current_kernel():
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if d.get("kernel_sha256_16") != h:
         return None
-    return d.get("dram_bytes_per_launch_full_workload")
+    e = d.get("workloads", {}).get(workload)
+    if not e or int(e.get("seq", -1)) != int(seq):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def roofline_peak(timed_region_ms: float):
+    """The bf16 peak a kernel is held against: the burst figure for a kernel
+    timed alone, the sustained one (seconds back to back under the power cap)
+    when the timed region keeps the kernel busy for a second or more.
+    Returns (peak, kind, burst peak, source)."""
+    peaks, src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if timed_region_ms >= 1000.0:
+        return sustained, "sustained", burst, src
+    return burst, "burst", burst, src
+
+
+def bench_config(w: workloads.Workload, sparse_frac: float, world: int) -> dict:
+    """The `config` of the JSON line; both arms print the same dict."""
+    in_bytes = w.layers * w.batch * (w.hq + 2 * w.hkv) * w.seq * w.d * 2
+    l2 = (("inputs %.1f MiB fit in L2: 256 MiB flush between timed steps, each step timed on "
+           "its own" % (in_bytes / 2 ** 20)) if in_bytes < 2 * L2_BYTES else
+          ("inputs exceed L2 (Q+K+V %.0f MiB > 126 MB), no flush" % (in_bytes / 2 ** 20)))
+    return {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch * world,
+            "seq_len": w.seq, "parallelism": f"replicas x{world}", "l2": l2}
+
+
+def ab_medians(fns, reps: int, stream):
+    """Median device time (ms) of each function, called in interleaved order
+    (a, b, ..., a, b, ...) after one warm call each, every call timed with its
+    own CUDA events on `stream`."""
+    for fn in fns:
+        fn()
+    torch.cuda.synchronize()
+    times = [[] for _ in fns]
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(reps)] for _ in fns]
+    for r in range(reps):
+        for i, fn in enumerate(fns):
+            evs[i][r][0].record(stream)
+            fn()
+            evs[i][r][1].record(stream)
+    torch.cuda.synchronize()
+    for i in range(len(fns)):
+        times[i] = [a.elapsed_time(b) for a, b in evs[i]]
+    return [statistics.median(t) for t in times], times
 
 
 # ---------------------------------------------------------------- ranks
@@ -308,8 +368,7 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / K
     value = eff * world / (ms_per_step * 1e-3) / 1e12
     tokens_per_s = B * N * world / (ms_per_step * 1e-3)
-    peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_kind, burst, peak_src = roofline_peak(total_ms)
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = (eff / nlayers) / (attn_avg_ms * 1e-3) / 1e12
 
@@ -318,15 +377,10 @@ def run_ours(args, rank, world, local_rank):
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_desc(w, sparse_frac), "global_batch": B * world,
-                   "seq_len": N, "parallelism": f"replicas x{world}",
-                   "l2": ("inputs %.1f MiB fit in L2: 256 MiB flush between timed steps, "
-                          "each step timed on its own" % (in_bytes / 2 ** 20))
-                         if flush is not None else
-                         ("inputs exceed L2 (Q+K+V %.0f MiB > 126 MB), no flush"
-                          % (in_bytes / 2 ** 20))},
+        "config": bench_config(w, sparse_frac, world),
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_bf16_peak": round(100.0 * value / world / peak, 2),
+        "pct_of_burst_bf16_peak": round(100.0 * value / world / burst, 2),
         # the same against the nominal dense bf16 figure (2.25 PFLOP/s per GPU)
         "pct_of_nominal_bf16_dense": round(100.0 * value / world / NOMINAL_BF16_TFLOPS, 2),
         "tile_granular_tflops": round(tile * world / (ms_per_step * 1e-3) / 1e12, 2),
@@ -336,29 +390,25 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": K * nlayers * (5 if layers[0]["router"] is not None else 1),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "traffic": traffic_for_current_kernel(),
+                     "peak_source": (f"{peak_src} bf16_tflops_{peak_kind}" if peak_kind ==
+                                     "sustained" else f"{peak_src} bf16_tflops (burst)"),
+                     "peak_rule": ("sustained: the timed region keeps the kernel busy back to "
+                                   "back for %.1f s (>= 1 s, under the power cap)"
+                                   % (total_ms / 1e3)) if peak_kind == "sustained" else
+                                  ("burst: the timed region is %.0f ms (< 1 s)" % total_ms),
+                     "frac_of_burst_peak": round(achieved / burst, 4),
+                     "traffic": traffic_for_current_kernel(w.name, N),
                      "kernel": "ea_hybrid_attn_kernel<128>"},
         "clocks": clocks,
     }
 
     if not args.quick and world == 1:
-        # comparators on the same inputs (outside the timed region)
+        # comparators on the same inputs (outside the timed region), each pair
+        # timed call by call in interleaved order, medians reported
         L = layers[0]
         m0 = masks[0]
-
-        def timeit(fn, reps=5):
-            fn()
-            torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            return a.elapsed_time(b) / reps
-
         out_tmp = torch.empty_like(L["q"])
+        reps = args.ab_reps
 
         def split_pass():
             ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], m0, w.sink, w.window,
@@ -374,14 +424,18 @@ def run_ours(args, rank, world, local_rank):
         def full_causal():
             ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], all_fa, w.sink, w.window,
                                    out=out_tmp, workspace=aws)
-        fused_ms = timeit(fused)
-        split_ms = timeit(split_pass)
-        full_ms = timeit(full_causal, reps=3)
+        (fused_ms, split_ms), (fused_t, split_t) = ab_medians([fused, split_pass], reps, stream)
+        (full_ms,), _ = ab_medians([full_causal], max(3, min(reps, 5)), stream)
         full_eff = flops.effective_flops(all_fa.cpu().numpy(), N, d, w.sink, w.window)
+        wins = sum(1 for a, b in zip(fused_t, split_t) if a < b)
         result["comparators"] = {
+            "timing": f"interleaved A/B, {reps} calls each after one warm call, medians",
             "fused_attn_ms": round(fused_ms, 4),
             "split_fa_then_sa_ms": round(split_ms, 4),
-            "fused_speedup_vs_split": round(split_ms / fused_ms, 3),
+            "fused_speedup_vs_split": round(split_ms / fused_ms, 4),
+            "fused_faster_in_pairs": f"{wins}/{reps}",
+            "fused_ms_range": [round(min(fused_t), 4), round(max(fused_t), 4)],
+            "split_ms_range": [round(min(split_t), 4), round(max(split_t), 4)],
             "full_causal_ms": round(full_ms, 4),
             "full_causal_tflops": round(full_eff / (full_ms * 1e-3) / 1e12, 2),
             "elastic_speedup_vs_full_causal": round(full_ms / fused_ms, 3),
@@ -391,7 +445,9 @@ def run_ours(args, rank, world, local_rank):
             # (cooperative) launch that runs the router in its prologue
             from sparse_attention_head_b200.api import ea_hybrid_attn_prefill_routed
             m_tmp = torch.empty_like(masks[0])
-            ws_routed = torch.zeros(1 << 24, dtype=torch.uint8, device=dev)
+            ws_routed = torch.zeros(
+                max(1 << 24, ea_router_workspace_size(B, Hkv, N, d) + (1 << 20)),
+                dtype=torch.uint8, device=dev)
 
             def two_launch():
                 ea_router_decide(L["k"], *L["router"], workspace=rws, route_mask=m_tmp,
@@ -403,14 +459,16 @@ def run_ours(args, rank, world, local_rank):
                 ea_hybrid_attn_prefill_routed(L["q"], L["k"], L["v"], *L["router"], w.sink,
                                               w.window, route_mask=m_tmp, out=out_tmp,
                                               workspace=ws_routed)
-            two_ms = timeit(two_launch)
-            routed_ms = timeit(routed)
+            (two_ms, routed_ms), (two_t, routed_t) = ab_medians([two_launch, routed], reps,
+                                                                stream)
             if ea_get_device_status(ws_routed) != 0:
                 raise RuntimeError("routed launch status word reports an error")
             result["comparators"].update({
                 "router_then_attn_ms": round(two_ms, 4),
                 "routed_one_launch_ms": round(routed_ms, 4),
-                "routed_speedup_vs_two_launches": round(two_ms / routed_ms, 3),
+                "routed_speedup_vs_two_launches": round(two_ms / routed_ms, 4),
+                "routed_faster_in_pairs":
+                    f"{sum(1 for a, b in zip(routed_t, two_t) if a < b)}/{reps}",
             })
         if rank == 0:
             result["cpu_baseline"] = cpu_baseline(w, L, m0.cpu().numpy(), args.cpu_seconds)
@@ -454,19 +512,111 @@ def run_ours(args, rank, world, local_rank):
                                  "download overlapped) -> pinned host out"
                                  + (" (layer 0)" if nlayers > 1 else "")
                                  + (f", one replica per rank x{world}" if world > 1 else "")}
+    # The secondary measurements run on layers of their own: the headline's
+    # tensors are released first.  With the 256K headline they take the
+    # side workload's layer shape (each names its workload).
+    layers.clear()
+    outs.clear()
+    masks.clear()
+    L = hp = qh = kh = vh = mh = out_tmp = None
+    torch.cuda.empty_cache()
+    side = workloads.get(args.side_workload) if w.name == "ext256k" else w
+    if not args.quick and world == 1 and not args.no_extra_workloads and args.seq is None:
+        result["workloads"] = {}
+        for name in ("llama8b", "qwen4b", "qwen8b36", "ext256k"):
+            if name != w.name:
+                result["workloads"][name] = measure_workload(workloads.get(name), dev, stream)
+                torch.cuda.empty_cache()
     if not args.quick and world == 1 and args.packed_seqs > 0:
-        result["packed"] = measure_packed(w, args.packed_seqs, max(args.steps, 5),
+        result["packed"] = measure_packed(side, args.packed_seqs, max(args.steps, 5),
                                           max(args.warmup, 3), dev, stream)
     if not args.quick and world == 1 and args.decode_batch > 0:
-        result["decode"] = measure_decode(w, args.decode_batch, max(args.steps, 10),
+        result["decode"] = measure_decode(side, args.decode_batch, max(args.steps, 10),
                                           max(args.warmup, 3), dev, stream)
-    if not args.quick and world == 1 and not args.no_fp8 and w.d == 128:
-        result["fp8"] = measure_fp8(w, max(args.steps, 5), max(args.warmup, 3), dev, stream)
+    if not args.quick and world == 1 and not args.no_fp8 and side.d == 128:
+        result["fp8"] = measure_fp8(side, max(args.steps, 5), max(args.warmup, 3), dev, stream)
     # the backward kernels are built for d = 128 (as the FP8 kernel)
-    if not args.quick and world == 1 and not args.no_training and w.d == 128:
-        result["training"] = measure_training(w, max(args.steps, 5), max(args.warmup, 3), dev,
-                                              stream)
+    if not args.quick and world == 1 and not args.no_training and side.d == 128:
+        result["training"] = measure_training(side, max(args.steps, 5), max(args.warmup, 3),
+                                              dev, stream)
     return result
+
+
+def measure_workload(w: workloads.Workload, dev, stream, steps: int = 5, warmup: int = 3):
+    """One more configuration's step (router, when it has one, then the fused
+    attention, every layer), timed as the headline is (CUDA events per launch;
+    inputs under 2x L2 get a 256 MiB flush between steps), with the attention
+    kernel's own roofline."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import (attn_workspace, ea_get_device_status,
+                                                ea_hybrid_attn_prefill, ea_router_decide,
+                                                ea_router_workspace_size, make_params)
+    B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
+    layers = [make_layer(w, l, 0, dev) for l in range(w.layers)]
+    aws = attn_workspace(make_params(B, Hq, Hkv, N, d, w.sink, w.window), dev)
+    rws = torch.empty(max(ea_router_workspace_size(B, Hkv, N, d), 16), dtype=torch.uint8,
+                      device=dev)
+    outs = [torch.empty_like(L["q"]) for L in layers]
+    masks = [torch.empty((B, Hq), dtype=torch.uint8, device=dev) if L["router"] is not None
+             else L["mask"] for L in layers]
+    in_bytes = w.layers * B * (Hq + 2 * Hkv) * N * d * 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES \
+        else None
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
+          for _ in range(steps)]
+
+    def step(e=None):
+        for li, L in enumerate(layers):
+            if e is not None:
+                e[li][0].record(stream)
+            if L["router"] is not None:
+                ea_router_decide(L["k"], *L["router"], workspace=rws, route_mask=masks[li],
+                                 want_logits=False)
+            if e is not None:
+                e[li][1].record(stream)
+            ea_hybrid_attn_prefill(L["q"], L["k"], L["v"], masks[li], w.sink, w.window,
+                                   out=outs[li], workspace=aws)
+            if e is not None:
+                e[li][2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        step(ev[i])
+    torch.cuda.synchronize()
+    if ea_get_device_status(aws) != 0:
+        raise RuntimeError(f"{w.name}: device status word reports an error")
+    step_ms = [ev[i][0][0].elapsed_time(ev[i][-1][2]) for i in range(steps)]
+    attn_ms = [ev[i][l][1].elapsed_time(ev[i][l][2]) for i in range(steps)
+               for l in range(w.layers)]
+    router_ms = [ev[i][l][0].elapsed_time(ev[i][l][1]) for i in range(steps)
+                 for l in range(w.layers)]
+    mask_host = [m.cpu().numpy() for m in masks]
+    eff = sum(flops.effective_flops(m, N, d, w.sink, w.window) for m in mask_host)
+    sparse_frac = float(np.mean([m.mean() for m in mask_host]))
+    ms = statistics.mean(step_ms)
+    attn_avg = statistics.mean(attn_ms)
+    achieved = (eff / w.layers) / (attn_avg * 1e-3) / 1e12
+    peak, kind, burst, src = roofline_peak(sum(step_ms))
+    return {
+        "config": bench_config(w, sparse_frac, 1),
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": round(ms, 4),
+        "effective_tflops": round(eff / (ms * 1e-3) / 1e12, 2),
+        "tokens_per_s": round(B * N / (ms * 1e-3), 1),
+        "attn_ms_per_layer": round(attn_avg, 4),
+        "router_ms_per_layer": round(statistics.mean(router_ms), 4),
+        "gpu_launches_per_step": w.layers * (5 if layers[0]["router"] is not None else 1),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{src} bf16_tflops ({kind})",
+                     "frac_of_burst_peak": round(achieved / burst, 4),
+                     "traffic": traffic_for_current_kernel(w.name, N),
+                     "kernel": "ea_hybrid_attn_kernel<128>"},
+    }
 
 
 # ---------------------------------------------------------------- FP8 variant
@@ -1098,8 +1248,9 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch,
-                   "seq_len": w.seq, "parallelism": "host cores"},
+        # the same config dict as our arm's line (the oracle's host cores are
+        # described in cpu_baseline)
+        "config": bench_config(w, sparse_frac, args.gpus),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(),
                          "kind": "oracle", "sample": desc + " per step"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -137,15 +137,25 @@ ea_status ea_router_decide_varlen(const void* k, const int32_t* cu_seqlens, int 
  * ea_router_workspace_size(B, Hkv, N, d), exceeds that size is rejected with
  * EA_ERR_SCRATCH_LIMIT before anything is enqueued.
  *
+ * Arguments are checked exactly as ea_router_decide checks them, with the
+ * same codes; only then is the scratch need compared with the limit.  The
+ * scratch used is the CURRENT device's copy of the array, so k, the weights,
+ * route_mask and logits_out must be device memory of the current device
+ * (EA_ERR_INVALID_ARG otherwise), and `stream` must belong to that device.
+ *
  * The first call on a device looks up that device's copy of the array (a
  * runtime symbol query, no allocation), so make the first call on each
  * device before any stream capture.  The entry point never calls cudaMalloc,
- * cudaFree or any allocating routine.
+ * cudaFree or any allocating routine.  A device reset invalidates the
+ * looked-up address: call ea_shutdown before resetting a device.
  *
  * All calls on one device share the array: two calls whose work overlaps on
  * the GPU (different streams, no ordering between them) race on it and give
- * undefined results.  Calls ordered on one stream are safe; each call
- * overwrites every scratch value it reads, so stale contents never matter.
+ * undefined results.  A CUDA graph captured from this call uses the same
+ * array, so its replays must be ordered with each other, with the replays of
+ * any other such graph and with eager calls, in the same way.  Calls ordered
+ * on one stream are safe; each call overwrites every scratch value it reads,
+ * so stale contents never matter.
  * ---------------------------------------------------------------------- */
 #define EA_ROUTER_NOALLOC_MAX_BYTES (1u << 20)
 
@@ -566,8 +576,10 @@ size_t ea_hybrid_attn_host_workspace_size(const ea_attn_params* p, int hidden);
  * with no library call in flight; a later host-buffer call creates the
  * streams again.  Nothing else is held: every other buffer is the caller's,
  * and ea_router_decide_noalloc's fixed scratch is static device memory that
- * lives until the process exits.  EA_OK, or EA_ERR_CUDA if a CUDA call
- * failed (the streams are forgotten either way). */
+ * lives until the process exits (ea_shutdown only forgets the device
+ * addresses it looked up for it, so the next call looks them up again: call
+ * ea_shutdown before resetting a device).  EA_OK, or EA_ERR_CUDA if a CUDA
+ * call failed (the streams are forgotten either way). */
 ea_status ea_shutdown(void);
 
 /* Number of chunks (kernel launches) a call with these arguments makes; 0

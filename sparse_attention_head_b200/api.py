@@ -122,25 +122,52 @@ def ea_router_decide_varlen(k: torch.Tensor, cu_seqlens: torch.Tensor, max_seqle
     return route_mask, logits
 
 
+def _padded_router_shapes(k_shape, w1, b1, w2, b2):
+    """(B, Hkv, N, d, hidden, Hq) of a padded router call; raises ValueError if
+    the weights do not fit the key states."""
+    if len(k_shape) != 4 or any(t.dim() != n for t, n in ((w1, 2), (b1, 1), (w2, 2), (b2, 1))):
+        raise ValueError("k must be [B, Hkv, N, d]; w1, w2 2-D and b1, b2 1-D")
+    B, Hkv, N, d = (int(x) for x in k_shape)
+    hidden, Hq = int(w1.shape[0]), int(w2.shape[0])
+    if w1.shape[1] != Hkv * d or b1.shape[0] != hidden or w2.shape[1] != hidden \
+            or b2.shape[0] != Hq:
+        raise ValueError("router weight shapes do not match the key states")
+    return B, Hkv, N, d, hidden, Hq
+
+
 def ea_router_decide_noalloc(k: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor,
                              w2: torch.Tensor, b2: torch.Tensor, threshold: float = 0.0, *,
                              route_mask: torch.Tensor, logits: Optional[torch.Tensor] = None,
                              stream: Optional[torch.cuda.Stream] = None) -> None:
     """The router without a workspace argument, for callers that cannot
     allocate device memory when they route a layer (its scratch is a fixed
-    array inside libea.so).  The caller passes the output buffers; this
-    wrapper allocates nothing either."""
+    array inside libea.so).  The caller passes the output buffers, route_mask
+    uint8 [B, Hq] and optionally logits fp32 [B, Hq], on k's device; this
+    wrapper allocates nothing either.  The call runs with k's device current,
+    because the library uses the current device's copy of its scratch."""
     lib = _lib.load()
+    B, Hkv, N, d, hidden, Hq = _padded_router_shapes(k.shape, w1, b1, w2, b2)
+    if tuple(route_mask.shape) != (B, Hq):
+        raise ValueError(f"route_mask must be [B, Hq] = [{B}, {Hq}]")
+    if logits is not None and tuple(logits.shape) != (B, Hq):
+        raise ValueError(f"logits must be [B, Hq] = [{B}, {Hq}]")
     _need(k, "k", torch.bfloat16, 4)
     for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
         _need(t, name, torch.float32, nd)
-    _need(route_mask, "route_mask", torch.uint8)
-    B, Hkv, N, d = k.shape
-    rc = lib.ea_router_decide_noalloc(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(), b1.data_ptr(),
-                                      w1.shape[0], w2.data_ptr(), b2.data_ptr(), w2.shape[0],
-                                      float(threshold), route_mask.data_ptr(),
-                                      logits.data_ptr() if logits is not None else None,
-                                      _stream_ptr(stream, k.device))
+    _need(route_mask, "route_mask", torch.uint8, 2)
+    if logits is not None:
+        _need(logits, "logits", torch.float32, 2)
+    dev = k.device
+    for name, t in (("w1", w1), ("b1", b1), ("w2", w2), ("b2", b2), ("route_mask", route_mask),
+                    ("logits", logits)):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} must be on {dev}, like k")
+    with torch.cuda.device(dev):
+        rc = lib.ea_router_decide_noalloc(k.data_ptr(), B, Hkv, N, d, w1.data_ptr(),
+                                          b1.data_ptr(), hidden, w2.data_ptr(), b2.data_ptr(),
+                                          Hq, float(threshold), route_mask.data_ptr(),
+                                          logits.data_ptr() if logits is not None else None,
+                                          _stream_ptr(stream, dev))
     check(rc, "ea_router_decide_noalloc")
 
 

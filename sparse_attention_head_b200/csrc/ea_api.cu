@@ -18,6 +18,8 @@
 namespace ea {
 
 constexpr int kMaxSmDevices = 64;
+// Widest router hidden layer the workspaces are sized for.
+constexpr int kRouterMaxHidden = 4096;
 
 int device_sms() {
   static int sms[kMaxSmDevices] = {0};
@@ -44,11 +46,30 @@ unsigned long long wait_timeout_ns() {
   return ns;
 }
 
+// Argument checks of ea_router_decide, shared with the entry point that
+// uses the library's fixed scratch array (same codes for the same arguments).
+ea_status router_check_args(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                            const float* b1, int hidden, const float* w2, const float* b2,
+                            int Hq, float threshold, const uint8_t* route_mask) {
+  if (!k || !w1 || !b1 || !w2 || !b2 || !route_mask) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || hidden <= 0 || Hq <= 0)
+    return EA_ERR_INVALID_ARG;
+  if (threshold != threshold) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(w1) & 15u) ||
+      (reinterpret_cast<uintptr_t>(w2) & 15u))
+    return EA_ERR_MISALIGNED;
+  return EA_OK;
+}
+
 }  // namespace ea
 
 namespace {
 
 using ea::device_sms;
+using ea::kRouterMaxHidden;
 using ea::wait_timeout_ns;
 
 
@@ -231,19 +252,30 @@ int list_units(const HostSched& h, int Hq, int S, int W, int32_t* units_out, int
   return total;
 }
 
-// EA_DEBUG_DROP_KV_POS=<n> makes the attention producer skip K/V ring
-// position n of every CTA (a test of the bounded waits; off by default).
+#ifdef EA_TEST_HOOKS
+// Failure-injection hooks of the test build (libea_testhooks.so), read once
+// per process: EA_DEBUG_DROP_KV_POS=<n> makes the attention producer skip
+// K/V ring position n of every CTA; EA_DEBUG_SKIP_GRID_SYNC=<n> makes CTA 0
+// of a routed launch leave without arriving at grid barrier n (0-3).  Each
+// makes a bounded device wait run out.  The release library has neither.
+int debug_env(const char* name) {
+  const char* e = getenv(name);
+  return e ? atoi(e) : -1;
+}
 int debug_drop_kv_pos() {
-  static int pos = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    if (const char* e = getenv("EA_DEBUG_DROP_KV_POS")) pos = atoi(e);
-  });
+  static const int pos = debug_env("EA_DEBUG_DROP_KV_POS");
   return pos;
 }
+int debug_skip_grid_sync() {
+  static const int phase = debug_env("EA_DEBUG_SKIP_GRID_SYNC");
+  return phase;
+}
+#else
+int debug_drop_kv_pos() { return -1; }
+int debug_skip_grid_sync() { return -1; }
+#endif
 
 constexpr size_t kAttnWorkspace = 256;
-constexpr int kRouterMaxHidden = 4096;
 
 }  // namespace
 
@@ -277,14 +309,9 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const fl
                            const float* b1, int hidden, const float* w2, const float* b2,
                            int Hq, float threshold, uint8_t* route_mask, float* logits_out,
                            void* workspace, size_t workspace_bytes, void* stream) {
-  if (!k || !w1 || !b1 || !w2 || !b2 || !route_mask) return EA_ERR_INVALID_ARG;
-  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || hidden <= 0 || Hq <= 0)
-    return EA_ERR_INVALID_ARG;
-  if (threshold != threshold) return EA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
-  if (Hkv * d > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
-  if ((Hkv * d) % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
-  if (!aligned16(k) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  const ea_status chk = ea::router_check_args(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq,
+                                              threshold, route_mask);
+  if (chk != EA_OK) return chk;
   const size_t need = ea_router_workspace_size(B, Hkv, N, d);
   if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
@@ -441,6 +468,7 @@ static ea_status prefill_impl(const void* q, const void* k, const void* v,
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.debug_skip_grid_sync = debug_skip_grid_sync();
   args.trace = trace;
   args.trace_max = trace_max;
 
@@ -508,6 +536,7 @@ static ea_status prefill_train(const void* q, const void* k, const void* v,
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.debug_skip_grid_sync = debug_skip_grid_sync();
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
   int grid = ea_attn_grid_size(p, sms);
@@ -592,6 +621,7 @@ ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void*
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = -1;
+  args.debug_skip_grid_sync = -1;
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
   const cudaError_t err = ea::launch_attn_fp8(args, ea_attn_grid_size(p, sms),
@@ -721,6 +751,7 @@ ea_status ea_hybrid_attn_prefill_varlen(const void* q, const void* k, const void
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.debug_skip_grid_sync = debug_skip_grid_sync();
 
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
@@ -812,6 +843,7 @@ ea_status ea_hybrid_attn_prefill_routed(const void* q, const void* k, const void
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.debug_skip_grid_sync = debug_skip_grid_sync();
   set_router_args(args, k, w1, b1, hidden, w2, b2, threshold, route_mask, logits_out, workspace,
                   ea::router_num_splits(p->B, p->Hkv, p->N));
   const int sms = device_sms();
@@ -867,6 +899,7 @@ ea_status ea_hybrid_attn_prefill_varlen_routed(const void* q, const void* k, con
   args.select = p->select;
   args.timeout_ns = wait_timeout_ns();
   args.debug_drop_kv_pos = debug_drop_kv_pos();
+  args.debug_skip_grid_sync = debug_skip_grid_sync();
   set_router_args(args, k, w1, b1, hidden, w2, b2, threshold, route_mask, logits_out, workspace,
                   ea::router_num_splits(p->B, p->Hkv, p->max_seqlen > 0 ? p->max_seqlen : 1));
   const int sms = device_sms();
@@ -1011,6 +1044,7 @@ struct CallEvents {
 }  // namespace
 
 ea_status ea_shutdown(void) {
+  ea::router_noalloc_forget();
   std::lock_guard<std::mutex> lock(g_stream_mu);
   int cur = -1;
   bool any = false;

@@ -117,8 +117,14 @@ __device__ __forceinline__ uint8_t ld_mask(const uint8_t* mask, int idx) {
 // others wait for (no reset between launches is needed).  Bounded: returns
 // false, with EA_ERR_TIMEOUT in the status word, if the others do not arrive
 // in time.  Needs every CTA resident at once (a cooperative launch).
-__device__ bool grid_sync(const AttnArgs& args, volatile int* s_flag) {
+__device__ bool grid_sync(const AttnArgs& args, volatile int* s_flag, int phase) {
   __syncthreads();
+#ifdef EA_TEST_HOOKS
+  // test build only: CTA 0 leaves without arriving, so the others time out
+  if (phase == args.debug_skip_grid_sync && blockIdx.x == 0) return false;
+#else
+  (void)phase;
+#endif
   if (threadIdx.x == 0) {
     volatile unsigned int* gen = args.bar_gen;
     const unsigned int g = *gen;
@@ -170,11 +176,11 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
                           args.total, Hkv, b, hk, split, ns, partials, red, tid, 1);
     }
   }
-  if (!grid_sync(args, s_flag)) return false;
+  if (!grid_sync(args, s_flag, 0)) return false;
   for (int i = blockIdx.x * blockDim.x + tid; i < B * in_dim; i += gridDim.x * blockDim.x)
     xbuf[i] = router_x(partials, args.cu_seqlens, Hkv, args.N, args.total, D, ns, i / in_dim,
                        i % in_dim);
-  if (!grid_sync(args, s_flag)) return false;
+  if (!grid_sync(args, s_flag, 1)) return false;
   const int nw = blockDim.x / 32;
   for (int o = blockIdx.x * nw + warp; o < B * hidden; o += gridDim.x * nw) {
     const int b = o / hidden, oo = o % hidden;
@@ -182,7 +188,7 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
                                     args.b1, oo, lane);
     if (lane == 0) hbuf[static_cast<size_t>(b) * hidden + oo] = fmaxf(v, 0.f);
   }
-  if (!grid_sync(args, s_flag)) return false;
+  if (!grid_sync(args, s_flag, 2)) return false;
   for (int o = blockIdx.x * nw + warp; o < B * args.Hq; o += gridDim.x * nw) {
     const int b = o / args.Hq, oo = o % args.Hq;
     const float v = router_warp_dot(hbuf + static_cast<size_t>(b) * hidden, hidden, args.w2,
@@ -192,7 +198,7 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
       args.mask_out[o] = (v > args.threshold) ? 1 : 0;
     }
   }
-  return grid_sync(args, s_flag);
+  return grid_sync(args, s_flag, 3);
 }
 
 // kTrace: the per-unit trace (its own instantiation, so the others carry none
@@ -415,10 +421,12 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                              tlim, EA_ERR_TIMEOUT);
               if (!ok) break;
             }
+#ifdef EA_TEST_HOOKS
             if (static_cast<int>(kv_pos) == args.debug_drop_kv_pos) {
-              ++kv_pos;           // test hook: this copy never happens
+              ++kv_pos;           // test build only: this copy never happens
               continue;
             }
+#endif
             mbar_arrive_expect_tx(bars.kv_full + 8 * st, C::kTileBytes);
             const CUtensorMap* map = which ? &args.tm_v : &args.tm_k;
             if (kFp8 && which) {

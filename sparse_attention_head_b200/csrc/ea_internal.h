@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ea.h"
+
 namespace ea {
 
 // Arguments of the fused hybrid attention kernel.  The tensor maps describe
@@ -38,9 +40,14 @@ struct alignas(64) AttnArgs {
   float scale_log2;         // softmax scale * log2(e)
   int select;               // ea_select
   unsigned long long timeout_ns;
-  // Failure-detection test hook (-1 = off): the producer skips the copy of
-  // this K/V ring position, so the kernel's bounded wait for it runs out.
+  // Failure-detection test hooks, compiled only into the library built with
+  // EA_TEST_HOOKS (-1 = off; the release library never sets them): the
+  // producer skips the copy of K/V ring position debug_drop_kv_pos, so the
+  // kernel's bounded wait for it runs out; CTA 0 of a routed launch leaves
+  // without arriving at grid barrier number debug_skip_grid_sync, so the
+  // other CTAs' bounded barrier waits run out.
   int debug_drop_kv_pos;
+  int debug_skip_grid_sync;
   // Per-unit trace (nullptr = off): trace[0] counts records; record i sits
   // at trace[8 + 6 i] .. +5 = {start, first S ready, last P handed over,
   // end (ns), CTA << 32 | rank, sparse << 32 | KV tiles}; records past
@@ -122,6 +129,13 @@ cudaError_t launch_fp8_quant(const void* x, int heads, int N, int d, int transpo
                              float* scale, void* workspace, cudaStream_t stream);
 
 // Router: pooled partial sums, then the MLP and the threshold.
+// The argument checks of ea_router_decide (status codes as its header states).
+ea_status router_check_args(const void* k, int B, int Hkv, int N, int d, const float* w1,
+                            const float* b1, int hidden, const float* w2, const float* b2,
+                            int Hq, float threshold, const uint8_t* route_mask);
+// Forget the device addresses of the fixed router scratch array (they are
+// looked up again on the next call that needs them).
+void router_noalloc_forget();
 int router_num_splits(int B, int Hkv, int N);
 size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden);
 // cu == nullptr: padded K [B][Hkv][N][d]; else packed K [total][Hkv][d] with

@@ -301,10 +301,10 @@ static __device__ __align__(256) unsigned char g_router_noalloc_scratch[EA_ROUTE
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoallocMaxDevices] = {nullptr};
 
-// Device address of this device's scratch array, or nullptr on failure.
-void* noalloc_scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+// Device address of device dev's copy of the scratch array, or nullptr on
+// failure.  dev must be the current device: the symbol lookup uses it.
+void* noalloc_scratch_for_device(int dev) {
+  if (dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
@@ -314,18 +314,47 @@ void* noalloc_scratch_for_current_device() {
   return g_noalloc_ptr[dev];
 }
 
+// True if p is device memory of device dev (the only memory the router's
+// kernels may be given).
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();   // an unknown pointer leaves no sticky error
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
 }  // namespace
+
+namespace ea {
+void router_noalloc_forget() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (int i = 0; i < kNoallocMaxDevices; ++i) g_noalloc_ptr[i] = nullptr;
+}
+}  // namespace ea
 
 extern "C" ea_status ea_router_decide_noalloc(const void* k, int B, int Hkv, int N, int d,
                                               const float* w1, const float* b1, int hidden,
                                               const float* w2, const float* b2, int Hq,
                                               float threshold, uint8_t* route_mask,
                                               float* logits_out, void* stream) {
+  // the same checks, in the same order, as ea_router_decide; the scratch
+  // limit only after them
+  const ea_status chk = ea::router_check_args(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq,
+                                              threshold, route_mask);
+  if (chk != EA_OK) return chk;
   const size_t need = ea_router_workspace_size(B, Hkv, N, d);
   if (need > EA_ROUTER_NOALLOC_MAX_BYTES) return EA_ERR_SCRATCH_LIMIT;
-  if (need == 0) return ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold,
-                                         route_mask, logits_out, nullptr, 0, stream);
-  void* scratch = noalloc_scratch_for_current_device();
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EA_ERR_CUDA;
+  // the scratch is the current device's copy: the keys and the outputs must
+  // live there too
+  if (!on_device(k, dev) || !on_device(w1, dev) || !on_device(b1, dev) || !on_device(w2, dev) ||
+      !on_device(b2, dev) || !on_device(route_mask, dev) ||
+      (logits_out && !on_device(logits_out, dev)))
+    return EA_ERR_INVALID_ARG;
+  void* scratch = noalloc_scratch_for_device(dev);
   if (!scratch) return EA_ERR_CUDA;
   return ea_router_decide(k, B, Hkv, N, d, w1, b1, hidden, w2, b2, Hq, threshold, route_mask,
                           logits_out, scratch, EA_ROUTER_NOALLOC_MAX_BYTES, stream);
