@@ -12,9 +12,10 @@ router-chosen ~75% sparse heads); the other configurations follow under
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints ONE JSON line on rank 0.  Multi-GPU runs (torchrun, one rank per GPU)
-are independent replicas of the workload on every rank (the path splits into
-independent (batch, head) problems, so there is no data-path collective); the
-time is the max over ranks and `value` counts the work of all ranks.
+shard one layer over the ranks by (batch, kv group), balanced by the mask's
+per-group cost; the router's pooled key vector is the one exchange (an NCCL
+all-gather of the ranks' pooled slices).  The work is fixed as N grows
+(strong scaling); the time is the max over ranks.
 
 --impl reference times the CPU oracle (float64 numpy, the plain definition of
 the method) on a bounded sample of the same workload, on the host cores.
@@ -218,8 +219,12 @@ def bench_config(w: workloads.Workload, sparse_frac: float, world: int) -> dict:
     l2 = (("inputs %.1f MiB fit in L2: 256 MiB flush between timed steps, each step timed on "
            "its own" % (in_bytes / 2 ** 20)) if in_bytes < 2 * L2_BYTES else
           ("inputs exceed L2 (Q+K+V %.0f MiB > 126 MB), no flush" % (in_bytes / 2 ** 20)))
-    return {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch * world,
-            "seq_len": w.seq, "parallelism": f"replicas x{world}", "l2": l2}
+    return {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch,
+            "seq_len": w.seq,
+            "parallelism": ("single GPU" if world == 1 else
+                            f"(batch, kv group) shards x{world}: LPT on the mask's tile cost, "
+                            "all-gather of the router's pooled slices"),
+            "l2": l2}
 
 
 def ab_medians(fns, reps: int, stream):
@@ -539,6 +544,143 @@ def run_ours(args, rank, world, local_rank):
     if not args.quick and world == 1 and not args.no_training and side.d == 128:
         result["training"] = measure_training(side, max(args.steps, 5), max(args.warmup, 3),
                                               dev, stream)
+    return result
+
+
+def run_sharded(args, rank, world, local_rank):
+    """N > 1: ONE layer's prefill (per layer of the workload) head-sharded over
+    the ranks: each rank pools its share of the (b, kv head) rows, one NCCL
+    all-gather of the pooled slices feeds the router on every rank, the
+    (b, kv group) groups are assigned by LPT on their cost under the mask,
+    and each rank runs the fused attention on its groups.  Total work is
+    fixed (strong scaling); the time is the slowest rank's."""
+    from sparse_attention_head_b200 import flops
+    from sparse_attention_head_b200.api import ea_get_device_status
+    from sparse_attention_head_b200.shard import ShardedPrefill, rank_loads, group_costs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    if args.seq:
+        w = dataclasses.replace(w, seq=args.seq)
+    B, Hq, Hkv, N, d = w.batch, w.hq, w.hkv, w.seq, w.d
+    stream = torch.cuda.current_stream(dev)
+    # every rank holds the same layer (rank 0's seed): the shards split it
+    layers = [make_layer(w, l, 0, dev) for l in range(w.layers)]
+    sps = []
+    for L in layers:
+        r = L["router"] if L["router"] is not None else (None, None, None, None)
+        sps.append(ShardedPrefill(B, Hq, Hkv, N, d, *r, w.sink, w.window, rank, world, dev,
+                                  mask=L["mask"]))
+    outs = [torch.empty_like(L["q"]) for L in layers]
+
+    def step(ev=None):
+        for li, (L, sp) in enumerate(zip(layers, sps)):
+            if ev is not None:
+                ev[li][0].record(stream)
+            sp.route(L["k"], stream)
+            sp.assign(stream)
+            if ev is not None:
+                ev[li][1].record(stream)
+            sp.attend(L["q"], L["k"], L["v"], outs[li], stream)
+            if ev is not None:
+                ev[li][2].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(visible_gpu_index(local_rank)) if rank == 0 else None
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    for sp in sps:
+        if ea_get_device_status(sp.attn_ws) != 0:
+            raise RuntimeError("device status word reports an error")
+    masks = [sp.mask.cpu().numpy() for sp in sps]
+    eff = sum(flops.effective_flops(m, N, d, w.sink, w.window) for m in masks)
+    sparse_frac = float(np.mean([m.mean() for m in masks]))
+    # this rank's share of the work, and its attention launches' time
+    mine = 0.0
+    for m, sp in zip(masks, sps):
+        sel = sp.owner == rank
+        for b in range(B):
+            for hk in range(Hkv):
+                if sel[b, hk]:
+                    mine += flops.effective_flops(m[b, hk * (Hq // Hkv):(hk + 1) * (Hq // Hkv)],
+                                                  N, d, w.sink, w.window)
+    attn_ms = statistics.mean(evs[i][l][1].elapsed_time(evs[i][l][2]) for i in range(K)
+                              for l in range(w.layers))
+    route_ms = statistics.mean(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K)
+                               for l in range(w.layers))
+    ms_per_step = total_ms / K
+    value = eff / (ms_per_step * 1e-3) / 1e12
+    peak, peak_kind, burst, peak_src = roofline_peak(total_ms)
+    achieved = (mine / w.layers) / (attn_ms * 1e-3) / 1e12
+    loads = rank_loads(group_costs(masks[0], Hkv, N, w.sink, w.window), sps[0].owner, world)
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": bench_config(w, sparse_frac, world),
+        "tokens_per_s": round(B * N / (ms_per_step * 1e-3), 1),
+        "pct_of_bf16_peak": round(100.0 * value / world / peak, 2),
+        "route_ms_rank0": round(route_ms, 4),
+        "attn_ms_rank0": round(attn_ms, 4),
+        "lpt_tile_loads_layer0": loads,
+        # per layer: pool rows + reduce (2), MLP (2), attention (1)
+        "gpu_launches": K * w.layers * (5 if layers[0]["router"] is not None else 1),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops ({peak_kind})",
+                     "frac_of_burst_peak": round(achieved / burst, 4),
+                     "scope": "rank 0's fused attention launch on its groups",
+                     "traffic": None, "kernel": "ea_hybrid_attn_kernel<128>"},
+        "clocks": clocks,
+    }
+    if not args.quick:
+        # end to end from pinned host buffers: each rank uploads the keys of
+        # its pooling rows and the q, k, v of its groups, downloads its heads
+        L, sp = layers[0], sps[0]
+        qh, kh, vh = (L[n].cpu().pin_memory() for n in ("q", "k", "v"))
+        oh = torch.empty_like(qh).pin_memory()
+        for _ in range(2):
+            sp.host_step(qh, kh, vh, oh, L["q"], L["k"], L["v"], outs[0], stream)
+        torch.cuda.synchronize()
+        torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ek = args.e2e_steps or K
+        up = down = 0
+        a.record(stream)
+        for _ in range(ek):
+            up, down = sp.host_step(qh, kh, vh, oh, L["q"], L["k"], L["v"], outs[0], stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        torch.distributed.barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / ek, world, dev)
+        tot = torch.tensor([up, down], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tot)
+        eff0 = flops.effective_flops(masks[0], N, d, w.sink, w.window)
+        result["e2e"] = {"value": round(eff0 / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                         "h2d_bytes_per_step": int(tot[0].item()),
+                         "d2h_bytes_per_step": int(tot[1].item()),
+                         "ms_per_step": round(e2e_ms, 4),
+                         "path": "ShardedPrefill.host_step: pooling rows' keys up, router "
+                                 "all-gather, LPT groups' q/k/v up, fused attention, own heads "
+                                 "down (layer 0)"}
     return result
 
 
@@ -1338,7 +1480,8 @@ def main():
             "nccl", timeout=datetime.timedelta(seconds=180),
             device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        res = run_sharded(args, rank, world, local_rank) if world > 1 else \
+            run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -212,6 +212,59 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
                                  void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* ------------------------------------------------------------------------
+ * Head-sharded multi-GPU prefill (one process per GPU).  The path splits
+ * into independent (batch, kv group) problems, so the work is sharded over
+ * (b, kv head) pairs; the only exchange is the router's pooled vector, which
+ * needs the keys of every kv head of a batch row (Elastic Attention blog
+ * §2.1: the router reads the layer's Key hidden states).  Per layer, on
+ * every rank:
+ *   1. ea_router_pool_rows pools the rank's rows of the flattened (b, kv
+ *      head) index into its slice of x;
+ *   2. the caller all-gathers the slices (NCCL) into x [B][Hkv*d];
+ *   3. ea_router_mlp runs the router's MLP and threshold on x (every rank
+ *      gets the same mask);
+ *   4. ea_hybrid_attn_prefill_groups computes the (b, kv head) groups the
+ *      rank was assigned (a balanced assignment by the mask's per-group
+ *      cost), writing only those heads' output rows.
+ * Steps 1 + 3 give the bits of ea_router_decide, and step 4 over the union
+ * of the ranks' groups the bits of ea_hybrid_attn_prefill.
+ * ---------------------------------------------------------------------- */
+
+/* Pools the key rows of flattened (b, kv head) indices [row0, row0 + nrows)
+ * of a padded K (device bf16 [B][Hkv][N][d], 16-byte aligned), row r being
+ * (b = r / Hkv, hk = r % Hkv): x_out (device fp32 [nrows][d]) receives
+ * mean over n of K[b][hk][n][:], with the pooling kernels and split count
+ * ea_router_decide uses for the whole [B][Hkv] problem, so every value has
+ * its bits.  workspace: >= ea_router_workspace_size(B, Hkv, N, d) bytes.
+ * Errors: EA_ERR_INVALID_ARG for NULL pointers or a row range outside
+ * [0, B*Hkv); otherwise as ea_router_decide.  nrows = 0 enqueues nothing. */
+ea_status ea_router_pool_rows(const void* k, int B, int Hkv, int N, int d, int row0, int nrows,
+                             float* x_out, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Bytes of workspace ea_router_mlp needs (B * hidden fp32); 0 if invalid. */
+size_t ea_router_mlp_workspace_size(int B, int hidden);
+
+/* The router's MLP and decision on a pooled x (device fp32 [B][in_dim],
+ * in_dim = Hkv * d, 16-byte aligned): z = W2 ReLU(W1 x + b1) + b2 and
+ * route_mask = z > threshold, with the kernels of ea_router_decide (same
+ * bits for the same x).  Weights, outputs and limits as ea_router_decide. */
+ea_status ea_router_mlp(const float* x, int B, int in_dim, const float* w1, const float* b1,
+                        int hidden, const float* w2, const float* b2, int Hq, float threshold,
+                        uint8_t* route_mask, float* logits_out, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ea_hybrid_attn_prefill restricted to a shard: group_sel (device uint8
+ * [B][Hkv], required) marks the (b, kv head) groups whose query heads run;
+ * the output rows of the other heads are left untouched.  Each head's rows
+ * have the bits the unrestricted call gives them.  Other arguments, limits
+ * and errors as ea_hybrid_attn_prefill (NULL group_sel: EA_ERR_INVALID_ARG). */
+ea_status ea_hybrid_attn_prefill_groups(const void* q, const void* k, const void* v,
+                                        const uint8_t* route_mask, const uint8_t* group_sel,
+                                        const ea_attn_params* p, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word kept
  * in `workspace` (an attention workspace).  *status_out receives EA_OK or
  * the error a kernel recorded (EA_ERR_TIMEOUT when a bounded device wait ran

@@ -82,6 +82,7 @@ __all__ = [
     "attention_varlen",
     "attention_lse",
     "attention_backward",
+    "attention_backward_sampled",
     "router_gumbel_forward",
     "router_ste_backward",
     "e4m3_decode",
@@ -501,6 +502,92 @@ def attention_backward(q, k, v, dout, mask, sink: int, window: int,
             ds = p * (dp - dd)
             dq[b, h] = scale * (ds @ k[b, hk])
             dk[b, hk] += scale * (ds.T @ q[b, h])
+    return dq, dk, dv
+
+
+def _visible_grid(rows, cols, sparse: bool, sink: int, window: int) -> np.ndarray:
+    """bool [len(rows), len(cols)]: visible(i, j) for every pair, elementwise."""
+    i = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.asarray(cols, dtype=np.int64)[None, :]
+    vis = j <= i
+    if sparse:
+        vis &= (j < sink) | ((i - j) < window)
+    return vis
+
+
+def attention_backward_sampled(q, k, v, dout, mask, b: int, hk: int, q_rows, key_rows,
+                               sink: int, window: int, scale: float | None = None,
+                               block: int = 512):
+    """Sampled gradients of L = sum(dout * out) for one kv group (batch b, kv
+    head hk) at any N, from the same definitions as attention_backward:
+    (dq [G, len(q_rows), d] for the group's query heads at rows q_rows,
+     dk [len(key_rows), d], dv [len(key_rows), d] of kv head hk at key_rows).
+
+    Per query head h of the group and per row i, over the keys i sees:
+      P_ij = exp(scale q_i.k_j - lse_i),  O_i = sum_j P_ij v_j,
+      D_i = dO_i . O_i,  dS_ij = P_ij (dO_i . v_j - D_i);
+    then dq_i = scale sum_j dS_ij k_j, and for a key j the sums run over the
+    rows i that see j and over the group's query heads:
+      dv_j = sum_h sum_i P_ij dO_i,  dk_j = scale sum_h sum_i dS_ij q_i.
+    lse_i and D_i come first, for every row: rows are taken in blocks, each
+    block's scores formed against the key range its rows may see with the
+    exact element mask applied, so every row's values are those of the
+    row-by-row definition."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    kh, vh = k[b, hk], v[b, hk]
+    q_rows = np.asarray(q_rows, dtype=np.int64)
+    key_rows = np.asarray(key_rows, dtype=np.int64)
+    dq = np.zeros((g, len(q_rows), d))
+    dk = np.zeros((len(key_rows), d))
+    dv = np.zeros((len(key_rows), d))
+    for hh in range(g):
+        h = hk * g + hh
+        sparse = bool(mask[b, h])
+        qh, doh = q[b, h], dout[b, h]
+        lse = np.empty(N)
+        dd = np.empty(N)
+        for i0 in range(0, N, block):
+            i1 = min(N, i0 + block)
+            rows = np.arange(i0, i1)
+            # keys any row of the block may see: [0, i1) for FA; the sinks and
+            # [i0 - window + 1, i1) for SA
+            if sparse:
+                lo = max(0, i0 - window + 1)
+                cols = np.unique(np.concatenate([np.arange(0, min(sink, i1)),
+                                                 np.arange(lo, i1)]))
+            else:
+                cols = np.arange(0, i1)
+            sc = (qh[rows] @ kh[cols].T) * scale
+            sc = np.where(_visible_grid(rows, cols, sparse, sink, window), sc, -np.inf)
+            m = np.max(sc, axis=1, keepdims=True)
+            e = np.exp(sc - m)
+            tot = np.sum(e, axis=1, keepdims=True)
+            lse[i0:i1] = (m + np.log(tot))[:, 0]
+            o = (e / tot) @ vh[cols]
+            dd[i0:i1] = np.sum(doh[rows] * o, axis=1)
+        for r, i in enumerate(q_rows):
+            cols = visible_keys(int(i), sparse, sink, window)
+            p = np.exp((kh[cols] @ qh[i]) * scale - lse[i])
+            ds = p * (vh[cols] @ doh[i] - dd[i])
+            dq[hh, r] = scale * (ds @ kh[cols])
+        for r, j in enumerate(key_rows):
+            j = int(j)
+            rows = np.arange(j, N)
+            rows = rows[_visible_grid(rows, [j], sparse, sink, window)[:, 0]]
+            if len(rows) == 0:
+                continue
+            p = np.exp((qh[rows] @ kh[j]) * scale - lse[rows])
+            dv[r] += p @ doh[rows]
+            ds = p * (doh[rows] @ vh[j] - dd[rows])
+            dk[r] += scale * (ds @ qh[rows])
     return dq, dk, dv
 
 

@@ -45,7 +45,8 @@ EXPORTED = [
     "ea_hybrid_attn_prefill_train", "ea_fp8_vt_stride", "ea_quantize_fp8_workspace_size",
     "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8", "ea_hybrid_attn_host_workspace_size",
     "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host", "ea_shutdown",
-    "ea_hybrid_attn_prefill_traced",
+    "ea_hybrid_attn_prefill_traced", "ea_router_pool_rows", "ea_router_mlp_workspace_size",
+    "ea_router_mlp", "ea_hybrid_attn_prefill_groups",
 ]
 
 
@@ -121,6 +122,17 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_prefill_host.restype = c_int
     lib.ea_hybrid_attn_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, vp, c_float,
                                                 pparams, vp, vp, c_int, vp, c_size, vp]
+    lib.ea_router_pool_rows.restype = c_int
+    lib.ea_router_pool_rows.argtypes = [vp, c_int, c_int, c_int, c_int, c_int, c_int, vp, vp,
+                                        c_size, vp]
+    lib.ea_router_mlp_workspace_size.restype = c_size
+    lib.ea_router_mlp_workspace_size.argtypes = [c_int, c_int]
+    lib.ea_router_mlp.restype = c_int
+    lib.ea_router_mlp.argtypes = [vp, c_int, c_int, vp, vp, c_int, vp, vp, c_int, c_float, vp,
+                                  vp, vp, c_size, vp]
+    lib.ea_hybrid_attn_prefill_groups.restype = c_int
+    lib.ea_hybrid_attn_prefill_groups.argtypes = [vp, vp, vp, vp, vp, pparams, vp, vp, c_size,
+                                                  vp]
     lib.ea_hybrid_attn_prefill.restype = c_int
     lib.ea_hybrid_attn_prefill.argtypes = [vp, vp, vp, vp, pparams, vp, vp, c_size, vp]
     lib.ea_get_device_status.restype = c_int

@@ -122,6 +122,56 @@ def ea_router_decide_varlen(k: torch.Tensor, cu_seqlens: torch.Tensor, max_seqle
     return route_mask, logits
 
 
+def ea_router_pool_rows(k: torch.Tensor, row0: int, nrows: int, *, x_out: torch.Tensor,
+                        workspace: torch.Tensor,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Pooled key rows [row0, row0 + nrows) of the flattened (b, kv head)
+    index of k [B, Hkv, N, d] into x_out (fp32, at least nrows * d values)."""
+    lib = _lib.load()
+    _need(k, "k", torch.bfloat16, 4)
+    _need(x_out, "x_out", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    B, Hkv, N, d = k.shape
+    if x_out.numel() < nrows * d:
+        raise ValueError("x_out must hold nrows * d values")
+    rc = lib.ea_router_pool_rows(k.data_ptr(), B, Hkv, N, d, int(row0), int(nrows),
+                                 x_out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream_ptr(stream, k.device))
+    check(rc, "ea_router_pool_rows")
+    return x_out
+
+
+def ea_router_mlp_workspace_size(B: int, hidden: int) -> int:
+    return int(_lib.load().ea_router_mlp_workspace_size(B, hidden))
+
+
+def ea_router_mlp(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor,
+                  b2: torch.Tensor, threshold: float = 0.0, *, route_mask: torch.Tensor,
+                  logits: Optional[torch.Tensor] = None, workspace: torch.Tensor,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The router's MLP and threshold on pooled x [B, in_dim] (fp32)."""
+    lib = _lib.load()
+    _need(x, "x", torch.float32, 2)
+    for name, t, nd in (("w1", w1, 2), ("b1", b1, 1), ("w2", w2, 2), ("b2", b2, 1)):
+        _need(t, name, torch.float32, nd)
+    _need(route_mask, "route_mask", torch.uint8)
+    _need(workspace, "workspace", torch.uint8)
+    B, in_dim = x.shape
+    hidden, Hq = w1.shape[0], w2.shape[0]
+    if w1.shape[1] != in_dim or b1.shape[0] != hidden or w2.shape[1] != hidden \
+            or b2.shape[0] != Hq:
+        raise ValueError("router weight shapes do not match x")
+    if route_mask.numel() != B * Hq or (logits is not None and logits.numel() != B * Hq):
+        raise ValueError("route_mask and logits must hold B * Hq entries")
+    rc = lib.ea_router_mlp(x.data_ptr(), B, in_dim, w1.data_ptr(), b1.data_ptr(), hidden,
+                           w2.data_ptr(), b2.data_ptr(), Hq, float(threshold),
+                           route_mask.data_ptr(),
+                           logits.data_ptr() if logits is not None else None,
+                           workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, x.device))
+    check(rc, "ea_router_mlp")
+    return route_mask
+
+
 def _padded_router_shapes(k_shape, w1, b1, w2, b2):
     """(B, Hkv, N, d, hidden, Hq) of a padded router call; raises ValueError if
     the weights do not fit the key states."""
@@ -216,6 +266,44 @@ def ea_hybrid_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                     workspace.data_ptr(), workspace.numel(),
                                     _stream_ptr(stream, q.device))
     check(rc, "ea_hybrid_attn_prefill")
+    return out
+
+
+def ea_hybrid_attn_prefill_groups(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  route_mask: torch.Tensor, group_sel: torch.Tensor,
+                                  sink: int, window: int, *, softmax_scale: float = 0.0,
+                                  out: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The fused prefill on one shard: only the query heads of the (b, kv
+    head) groups with group_sel[b, hk] != 0 run; other heads' rows of `out`
+    are left as they were."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    _need(route_mask, "route_mask", torch.uint8)
+    _need(group_sel, "group_sel", torch.uint8)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    if route_mask.numel() != B * Hq or group_sel.numel() != B * Hkv:
+        raise ValueError("route_mask must hold B * Hq entries and group_sel B * Hkv")
+    p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if workspace is None:
+        workspace = attn_workspace(p, q.device)
+    rc = lib.ea_hybrid_attn_prefill_groups(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           route_mask.data_ptr(), group_sel.data_ptr(),
+                                           ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), _stream_ptr(stream, q.device))
+    check(rc, "ea_hybrid_attn_prefill_groups")
     return out
 
 

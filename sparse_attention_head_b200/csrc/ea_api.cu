@@ -323,6 +323,51 @@ ea_status ea_router_decide(const void* k, int B, int Hkv, int N, int d, const fl
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
+ea_status ea_router_pool_rows(const void* k, int B, int Hkv, int N, int d, int row0, int nrows,
+                             float* x_out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!k || !x_out) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if (Hkv * d > 8192) return EA_ERR_UNSUPPORTED;
+  if (row0 < 0 || nrows < 0 || static_cast<long long>(row0) + nrows >
+                                   static_cast<long long>(B) * Hkv)
+    return EA_ERR_INVALID_ARG;
+  if (!aligned16(k)) return EA_ERR_MISALIGNED;
+  const size_t need = ea_router_workspace_size(B, Hkv, N, d);
+  if (!workspace || workspace_bytes < need) return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  if (nrows == 0) return EA_OK;
+  cudaError_t err = ea::launch_router_pool_rows(k, B, Hkv, N, d, row0, nrows,
+                                                static_cast<float*>(workspace), x_out,
+                                                static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+size_t ea_router_mlp_workspace_size(int B, int hidden) {
+  if (B <= 0 || hidden <= 0 || hidden > kRouterMaxHidden) return 0;
+  return static_cast<size_t>(B) * hidden * sizeof(float);
+}
+
+ea_status ea_router_mlp(const float* x, int B, int in_dim, const float* w1, const float* b1,
+                        int hidden, const float* w2, const float* b2, int Hq, float threshold,
+                        uint8_t* route_mask, float* logits_out, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!x || !w1 || !b1 || !w2 || !b2 || !route_mask) return EA_ERR_INVALID_ARG;
+  if (B <= 0 || in_dim <= 0 || hidden <= 0 || Hq <= 0) return EA_ERR_INVALID_ARG;
+  if (threshold != threshold) return EA_ERR_INVALID_ARG;
+  if (in_dim > 8192 || hidden > kRouterMaxHidden || Hq > 1024) return EA_ERR_UNSUPPORTED;
+  if (in_dim % 4 != 0 || hidden % 4 != 0) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2)) return EA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < ea_router_mlp_workspace_size(B, hidden))
+    return EA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return EA_ERR_MISALIGNED;
+  cudaError_t err = ea::launch_router_mlp(x, B, in_dim, w1, b1, hidden, w2, b2, Hq, threshold,
+                                          route_mask, logits_out, static_cast<float*>(workspace),
+                                          static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
 size_t ea_router_varlen_workspace_size(int B, int Hkv, int max_seqlen, int d) {
   if (B <= 0 || Hkv <= 0 || max_seqlen < 0 || (d != 64 && d != 128)) return 0;
   return ea::router_workspace_bytes(B, Hkv, max_seqlen > 0 ? max_seqlen : 1, d,
@@ -438,7 +483,8 @@ int ea_attn_grid_size(const ea_attn_params* p, int num_sms) {
 static ea_status prefill_impl(const void* q, const void* k, const void* v,
                               const uint8_t* route_mask, const ea_attn_params* p, void* out,
                               void* workspace, size_t workspace_bytes,
-                              unsigned long long* trace, int trace_max, void* stream) {
+                              unsigned long long* trace, int trace_max, void* stream,
+                              const uint8_t* group_sel = nullptr) {
   ea_status st = check_params(p);
   if (st != EA_OK) return st;
   if (!q || !k || !v || !route_mask || !out) return EA_ERR_INVALID_ARG;
@@ -471,6 +517,7 @@ static ea_status prefill_impl(const void* q, const void* k, const void* v,
   args.debug_skip_grid_sync = debug_skip_grid_sync();
   args.trace = trace;
   args.trace_max = trace_max;
+  args.group_sel = group_sel;
 
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
@@ -484,6 +531,15 @@ ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v,
                                  void* workspace, size_t workspace_bytes, void* stream) {
   return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, nullptr, 0,
                       stream);
+}
+
+ea_status ea_hybrid_attn_prefill_groups(const void* q, const void* k, const void* v,
+                                       const uint8_t* route_mask, const uint8_t* group_sel,
+                                       const ea_attn_params* p, void* out, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!group_sel) return EA_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, nullptr, 0, stream,
+                      group_sel);
 }
 
 ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,

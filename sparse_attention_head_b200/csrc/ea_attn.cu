@@ -112,6 +112,12 @@ __device__ __forceinline__ uint8_t ld_mask(const uint8_t* mask, int idx) {
   return idx >= 0 ? *reinterpret_cast<const volatile uint8_t*>(mask + idx) : 0;
 }
 
+// Does the launch's shard run the query heads of (sequence b, kv head of h)?
+__device__ __forceinline__ bool in_shard(const AttnArgs& args, int b, int h) {
+  return args.group_sel == nullptr ||
+         args.group_sel[b * args.Hkv + h / (args.Hq / args.Hkv)] != 0;
+}
+
 // Grid barrier of the routed prologue.  Every CTA arrives once per phase;
 // the last arrival resets the count and advances the generation, which the
 // others wait for (no reset between launches is needed).  Bounded: returns
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
         const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) == 0) &&
-                        args.select != EA_SELECT_SA;
+                        args.select != EA_SELECT_SA && in_shard(args, b, h);
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nfa += __popc(bits);
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         const int h = h0 + lane;
         const int idx = b * args.Hq + h;
         const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) != 0) &&
-                        args.select != EA_SELECT_FA;
+                        args.select != EA_SELECT_FA && in_shard(args, b, h);
         const unsigned bits = __ballot_sync(0xffffffffu, ok);
         if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
         nsa += __popc(bits);

@@ -48,6 +48,10 @@ struct alignas(64) AttnArgs {
   // other CTAs' bounded barrier waits run out.
   int debug_drop_kv_pos;
   int debug_skip_grid_sync;
+  // Shard of the launch (nullptr = every head): [B*Hkv], nonzero where the
+  // query heads of (batch, kv head) run; the others' output rows are not
+  // written.
+  const uint8_t* group_sel;
   // Per-unit trace (nullptr = off): trace[0] counts records; record i sits
   // at trace[8 + 6 i] .. +5 = {start, first S ready, last P handed over,
   // end (ns), CTA << 32 | rank, sparse << 32 | KV tiles}; records past
@@ -138,6 +142,18 @@ ea_status router_check_args(const void* k, int B, int Hkv, int N, int d, const f
 void router_noalloc_forget();
 int router_num_splits(int B, int Hkv, int N);
 size_t router_workspace_bytes(int B, int Hkv, int N, int d, int hidden);
+// Pooled rows [row0, row0 + nrows) of the flattened (batch, kv head) index of
+// a padded K [B][Hkv][N][d] into x_out [nrows][d], with the split count of the
+// whole problem (so the bits equal those launch_router computes).
+cudaError_t launch_router_pool_rows(const void* k, int B, int Hkv, int N, int d, int row0,
+                                    int nrows, float* partials, float* x_out,
+                                    cudaStream_t stream);
+// The router's two MLP layers and threshold on a pooled x [B][in_dim];
+// hbuf holds B * hidden floats.
+cudaError_t launch_router_mlp(const float* x, int B, int in_dim, const float* w1,
+                              const float* b1, int hidden, const float* w2, const float* b2,
+                              int Hq, float threshold, uint8_t* mask, float* logits, float* hbuf,
+                              cudaStream_t stream);
 // cu == nullptr: padded K [B][Hkv][N][d]; else packed K [total][Hkv][d] with
 // sequence b at tokens [cu[b], cu[b + 1]).
 cudaError_t launch_router(const void* k, const int32_t* cu, int B, int Hkv, int N, int total,

@@ -42,6 +42,29 @@ __global__ void __launch_bounds__(kPoolThreads) ea_router_pool_kernel(
                       partials, red, threadIdx.x, 1);
 }
 
+// The same pooling items for rows row0 + blockIdx.y of the flattened (batch,
+// kv head) index of a padded K (one shard's rows), with the whole problem's
+// split count.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) ea_router_pool_rows_kernel(
+    const __nv_bfloat16* __restrict__ k, int N, int Hkv, int row0, int nsplit,
+    float* __restrict__ partials) {
+  __shared__ float red[(kPoolThreads / (D / 8)) * D];
+  const int r = row0 + static_cast<int>(blockIdx.y);
+  router_pool_item<D>(k, nullptr, N, 0, Hkv, r / Hkv, r % Hkv, blockIdx.x, nsplit, partials, red,
+                      threadIdx.x, 1);
+}
+
+// x of those rows, [nrows][d] (one channel per thread).
+__global__ void ea_router_reduce_rows_kernel(const float* __restrict__ partials, int Hkv, int N,
+                                             int d, int nsplit, int row0, int nrows,
+                                             float* __restrict__ x_out) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // (row - row0) * d + c
+  if (e >= nrows * d) return;
+  const int r = row0 + e / d;
+  x_out[e] = router_x(partials, nullptr, Hkv, N, 0, d, nsplit, r / Hkv, (r % Hkv) * d + e % d);
+}
+
 // x[b][j] for one channel per thread.
 __global__ void ea_router_reduce_kernel(const float* __restrict__ partials,
                                         const int32_t* __restrict__ cu, int Hkv, int N, int total,
@@ -277,6 +300,38 @@ cudaError_t launch_router(const void* k, const int32_t* cu, int B, int Hkv, int 
   ea_router_layer_kernel<false><<<dim3((hidden + kWarps - 1) / kWarps, B), kMlpThreads, 0,
                                   stream>>>(xbuf, in_dim, w1, b1, hidden, hbuf, 0.f, nullptr);
   err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ea_router_layer_kernel<true><<<dim3((Hq + kWarps - 1) / kWarps, B), kMlpThreads, 0,
+                                 stream>>>(hbuf, hidden, w2, b2, Hq, logits, threshold, mask);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_pool_rows(const void* k, int B, int Hkv, int N, int d, int row0,
+                                    int nrows, float* partials, float* x_out,
+                                    cudaStream_t stream) {
+  const int nsplit = router_num_splits(B, Hkv, N);
+  dim3 grid(nsplit, nrows);
+  if (d == 128)
+    ea_router_pool_rows_kernel<128><<<grid, kPoolThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k), N, Hkv, row0, nsplit, partials);
+  else
+    ea_router_pool_rows_kernel<64><<<grid, kPoolThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k), N, Hkv, row0, nsplit, partials);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ea_router_reduce_rows_kernel<<<(nrows * d + 255) / 256, 256, 0, stream>>>(
+      partials, Hkv, N, d, nsplit, row0, nrows, x_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_mlp(const float* x, int B, int in_dim, const float* w1,
+                              const float* b1, int hidden, const float* w2, const float* b2,
+                              int Hq, float threshold, uint8_t* mask, float* logits, float* hbuf,
+                              cudaStream_t stream) {
+  constexpr int kWarps = kMlpThreads / 32;
+  ea_router_layer_kernel<false><<<dim3((hidden + kWarps - 1) / kWarps, B), kMlpThreads, 0,
+                                  stream>>>(x, in_dim, w1, b1, hidden, hbuf, 0.f, nullptr);
+  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   ea_router_layer_kernel<true><<<dim3((Hq + kWarps - 1) / kWarps, B), kMlpThreads, 0,
                                  stream>>>(hbuf, hidden, w2, b2, Hq, logits, threshold, mask);

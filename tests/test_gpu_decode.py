@@ -100,6 +100,9 @@ CASES = [
     (1, 8, 4, 64, 130, 257, 1300, [1299]),                 # GQA 2, sinks span two chunks
     (2, 8, 8, 128, 1, 512, 1541, [1540, 1024]),            # ragged split tail
     (1, 8, 1, 128, 2000, 300, 1800, [1799]),               # sinks beyond max_len (all sink)
+    # the bench's layer shape at the positions it decodes (16K-32K): long
+    # full caches split many ways, wrapped rings
+    (3, 32, 8, 128, 64, 1024, 32768, [32767, 16384, 24001]),
 ]
 
 

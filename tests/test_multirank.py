@@ -1,6 +1,7 @@
 """The multi-rank plumbing of bench.py on CPU with gloo, world size 2: every
-rank runs its own replica (distinct seeds and inputs), the timed region is
-the slowest rank's, and only rank 0 prints the JSON line."""
+rank holds the same layer (the shards split one layer), the timed region is
+the slowest rank's, only rank 0 prints the JSON line, and both arms print
+the same config."""
 import json
 import os
 import socket
@@ -29,7 +30,7 @@ def _worker(rank, world, port, out):
     try:
         w = workloads.get("tiny")
         t = bench.max_over_ranks(1.5 + rank, world, "cpu")
-        L = bench.make_layer(w, 0, rank, "cpu")
+        L = bench.make_layer(w, 0, 0, "cpu")          # the sharded run's inputs
         q0 = L["q"].float()
         gathered = [torch.zeros_like(q0) for _ in range(world)]
         dist.all_gather(gathered, q0)
@@ -39,7 +40,7 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_replicas_and_max_time():
+def test_two_gloo_ranks_same_layer_and_max_time():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -52,8 +53,7 @@ def test_two_gloo_ranks_replicas_and_max_time():
         assert p.exitcode == 0
     (r0, t0, s0, same0), (r1, t1, s1, same1) = res
     assert t0 == t1 == 2.5               # both ranks see the slowest rank's time
-    assert s0 != s1                      # each rank has its own inputs
-    assert not same0 and not same1
+    assert same0 and same1               # both ranks hold the layer the shards split
 
 
 def test_reference_arm_prints_on_rank_zero_only():
@@ -69,3 +69,19 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_both_arms_print_the_same_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    base = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+            "--workload", "tiny", "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"]
+    for gpus in (1, 2):
+        env0 = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+        r0 = subprocess.run(base + ["--gpus", str(gpus)], env=env0, capture_output=True,
+                            text=True, timeout=300)
+        assert r0.returncode == 0, r0.stderr
+        line = json.loads(r0.stdout.strip().splitlines()[-1])
+        # tiny routes heads 1 and 3 of 4 sparse: fraction 0.5
+        assert line["config"] == bench.bench_config(workloads.get("tiny"), 0.5, gpus)

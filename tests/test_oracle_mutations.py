@@ -56,6 +56,13 @@ MUTATIONS = {
     "bwd_dk_unscaled": ("dk[b, hk] += scale * (ds.T @ q[b, h])", "dk[b, hk] += ds.T @ q[b, h]"),
     "bwd_dv_untransposed": ("dv[b, hk] += p.T @ dout[b, h]", "dv[b, hk] += p @ dout[b, h]"),
     "bwd_gqa_overwrite": ("dv[b, hk] += p.T @ dout[b, h]", "dv[b, hk] = p.T @ dout[b, h]"),
+    "bwd_sampled_missing_rowsum": ("ds = p * (vh[cols] @ doh[i] - dd[i])",
+                                   "ds = p * (vh[cols] @ doh[i])"),
+    "bwd_sampled_keys_strict": ("rows = np.arange(j, N)\n", "rows = np.arange(j + 1, N)\n"),
+    "bwd_sampled_block_window": ("lo = max(0, i0 - window + 1)", "lo = max(0, i0 - window + 2)"),
+    "bwd_sampled_dk_unscaled": ("dk[r] += scale * (ds @ qh[rows])", "dk[r] += ds @ qh[rows]"),
+    "bwd_sampled_lse_unshifted": ("lse[i0:i1] = (m + np.log(tot))[:, 0]",
+                                  "lse[i0:i1] = np.log(tot)[:, 0]"),
     "lse_without_max": ("out[b, h] = m + np.log(", "out[b, h] = np.log("),
     "ste_missing_tau": ("dz = dr * r_soft * (1.0 - r_soft) / tau",
                         "dz = dr * r_soft * (1.0 - r_soft)"),

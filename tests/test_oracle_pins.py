@@ -430,6 +430,52 @@ def test_attention_backward_matches_finite_differences():
     np.testing.assert_allclose(dv, _fd_grad(loss, v), rtol=0, atol=1e-6)
 
 
+def test_sampled_backward_matches_finite_differences():
+    """The sampled gradients of one kv group at every row and key against
+    central differences of the brute-force forward (independent of both
+    backward functions); a block smaller than N so the row blocks meet."""
+    rng = np.random.default_rng(73)
+    B, Hq, Hkv, N, d, S, W = 2, 4, 2, 8, 2, 2, 3
+    q = rng.standard_normal((B, Hq, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    dout = rng.standard_normal((B, Hq, N, d))
+    mask = np.array([[0, 1, 1, 1], [1, 0, 0, 1]], np.uint8)
+
+    def loss():
+        return float(np.sum(dout * oracle.brute_force_attention(q, k, v, mask, S, W)))
+    fq, fk, fv = _fd_grad(loss, q), _fd_grad(loss, k), _fd_grad(loss, v)
+    for b in range(B):
+        for hk in range(Hkv):
+            dq, dk, dv = oracle.attention_backward_sampled(
+                q, k, v, dout, mask, b, hk, np.arange(N), np.arange(N), S, W, block=3)
+            np.testing.assert_allclose(dq, fq[b, 2 * hk:2 * hk + 2], rtol=0, atol=1e-6)
+            np.testing.assert_allclose(dk, fk[b, hk], rtol=0, atol=1e-6)
+            np.testing.assert_allclose(dv, fv[b, hk], rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("S,W,block", [(4, 16, 32), (0, 1, 8), (3, 200, 64), (70, 5, 16)])
+def test_sampled_backward_equals_dense_backward(S, W, block):
+    """Sampled rows and keys (the first and last, block edges, sinks, window
+    edges) equal the dense backward's, for mixed FA/SA groups."""
+    rng = np.random.default_rng(74 + W)
+    B, Hq, Hkv, N, d = 1, 8, 2, 150, 8
+    q = rng.standard_normal((B, Hq, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    dout = rng.standard_normal((B, Hq, N, d))
+    mask = np.array([[1, 0, 1, 1, 1, 1, 0, 0]], np.uint8)
+    rq, rk, rv = oracle.attention_backward(q, k, v, dout, mask, S, W)
+    rows = sorted({0, 1, max(S - 1, 0), S, W - 1, W, block - 1, block, 2 * block, N - 2, N - 1}
+                  & set(range(N)))
+    for hk in range(Hkv):
+        dq, dk, dv = oracle.attention_backward_sampled(q, k, v, dout, mask, 0, hk, rows, rows,
+                                                       S, W, block=block)
+        np.testing.assert_allclose(dq, rq[0, 4 * hk:4 * hk + 4][:, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dk, rk[0, hk, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv, rv[0, hk, rows], rtol=0, atol=1e-12)
+
+
 def test_attention_lse_matches_the_definition():
     rng = np.random.default_rng(72)
     B, Hq, Hkv, N, d, S, W = 1, 2, 1, 11, 4, 2, 3
