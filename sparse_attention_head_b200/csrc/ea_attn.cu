@@ -11,8 +11,9 @@
 //   warps 4-7  the same for slot 1 (rows r0+128..r0+255)
 //   warp  8    TMA producer: Q slots once per unit, then K and V tiles of the
 //              unit's tile list through a ring of shared-memory stages
-//   warp  9    tcgen05 issuer (one thread): S_s = Q_s K^T into TMEM, then
-//              O_s += P_s V with P read from TMEM (P overwrites S in place)
+//   warp  9    tcgen05 issuer (the whole warp runs the loop, the elected
+//              lane issues): S_s = Q_s K^T into TMEM, then O_s += P_s V with
+//              P read from TMEM (P overwrites S in place)
 //   warps 10-11 idle (they complete the third warpgroup)
 // Registers: launched at 168 per thread (384 x 168 = 64512); the third
 // warpgroup drops to 120 and the two softmax warpgroups rise to 192
@@ -24,7 +25,10 @@
 // Softmax runs one query row per thread in fp32 on the log2 scale.  The row
 // reference max is only moved when a tile's max exceeds it by more than 8
 // (2^8 headroom in fp32/bf16), so most tiles need no O rescale; the final
-// O / l uses the same reference, so the result is unchanged.
+// O / l uses the same reference, so the result is unchanged.  The row sum l
+// adds the fp32 probabilities on fully visible tiles and the bf16-rounded
+// ones (those the P.V product sees) on masked tiles, which hold every key of
+// the rows that see fewer than 128 keys.
 //
 // Every wait is bounded: on timeout the kernel records EA_ERR_TIMEOUT in the
 // status word, every role leaves its loop, in-flight copies and MMAs are
@@ -70,8 +74,8 @@ struct AttnCfg {
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   // q_full, q_empty, drain, kv_full[kStages], kv_empty[kStages],
-  // s_full[2], p_full[2], o_done[2], o_empty[2]
-  static constexpr int kNumBars = 3 + 2 * kStages + 8;
+  // s_full[2], p_full[2], o_done[2], o_empty[2], p_half[2]
+  static constexpr int kNumBars = 3 + 2 * kStages + 10;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, counts
   static constexpr int kOffEnt = kOffMisc + 64;
   // sequence tables: token offset and length by index, order and unit count by
@@ -104,6 +108,7 @@ struct Bars {
   uint32_t p_full;
   uint32_t o_done;
   uint32_t o_empty;
+  uint32_t p_half;
 };
 
 // Route bit of entry idx, read through the coherent path: in a routed launch
@@ -207,6 +212,42 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
   return grid_sync(args, s_flag, 3);
 }
 
+// One row's probabilities p = 2^(x * sl2 - msub) over keys [32 C0, 32 C1)
+// of a 128-key tile:
+// packed FMA, then exp2 on the MUFU for most pairs and on the FMA pipe for
+// kEmuPairs of every 8 pairs; P is stored to TMEM as bf16 pairs (columns
+// [0, 64) of the row's score columns) and acc gathers the row sum.  The sum
+// adds the bf16-rounded values the P.V product sees when kRoundedSum, else
+// the fp32 values, each within 2^-9 of its rounding (unpacking the rounded
+// values costs 128 instructions per row and tile: 4-8% of the launch when
+// every tile pays it).
+template <bool kRoundedSum, int C0, int C1>
+__device__ __forceinline__ void softmax_p_bf16(const float (&x)[128], float sl2, float msub,
+                                               uint32_t tS, float (&acc)[8]) {
+#pragma unroll
+  for (int c = C0; c < C1; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float p0, p1;
+      fma2_sc(p0, p1, x[c * 32 + 2 * j], x[c * 32 + 2 * j + 1], sl2, -msub);
+      if ((j & 7) < kEmuPairs) {
+        exp2_poly2(p0, p1);
+      } else {
+        p0 = ex2_approx(p0);
+        p1 = ex2_approx(p1);
+      }
+      pk[j] = pack_bf16x2(p0, p1);
+      if (kRoundedSum)
+        add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], __uint_as_float(pk[j] << 16),
+                 __uint_as_float(pk[j] & 0xffff0000u));
+      else
+        add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], p0, p1);
+    }
+    tmem_st16(tS + c * 16, pk);
+  }
+}
+
 // kTrace: the per-unit trace (its own instantiation, so the others carry none
 // of its code or registers)
 template <int D, bool kRouted, bool kFp8 = false, bool kTrace = false>
@@ -238,6 +279,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     bars.p_full = bars.s_full + 16;
     bars.o_done = bars.p_full + 16;
     bars.o_empty = bars.o_done + 16;
+    bars.p_half = bars.o_empty + 16;
   }
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -251,7 +293,8 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     // bar_base layout: q_full, q_empty, drain, kv_full[kStages],
-    // kv_empty[kStages], s_full[2], p_full[2], o_done[2], o_empty[2]
+    // kv_empty[kStages], s_full[2], p_full[2], o_done[2], o_empty[2],
+    // p_half[2]
     mbar_init(bar_base + 0, 1);                        // q_full: producer
     mbar_init(bar_base + 1, 1);                        // q_empty: MMA issuer
     mbar_init(bar_base + 2, 1);                        // drain: MMA issuer
@@ -264,6 +307,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       mbar_init(bar_base + 3 + 2 * C::kStages + 2 + s, 128);  // p_full
       mbar_init(bar_base + 3 + 2 * C::kStages + 4 + s, 1);    // o_done
       mbar_init(bar_base + 3 + 2 * C::kStages + 6 + s, 128);  // o_empty
+      mbar_init(bar_base + 3 + 2 * C::kStages + 8 + s, 128);  // p_half
     }
     *s_abort = 0;
     fence_mbar_init();
@@ -457,13 +501,17 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     __syncwarp();
     } else if (warp == 9) {
     // ============================================================ MMA issuer
-    // One thread issues both slots' MMAs in the order PV0(i), S0(i+1),
-    // PV1(i), S1(i+1): each group of eight MMAs is contiguous, and the
-    // tensor pipe always has the other slot's group queued while a softmax
-    // runs.  The pipe's queue is shallow, so the thread keeps everything but
-    // MMAs and the waits they need off this path (K/V waits come from the
-    // async proxy and need no tcgen05 fence; only P handoffs do).
-    if (lane == 0) {
+    // Both slots' MMAs go out in the order PV0(i), S0(i+1), PV1(i), S1(i+1):
+    // each group of eight MMAs is contiguous, and the tensor pipe always has
+    // the other slot's group queued while a softmax runs.  The whole warp
+    // runs this loop (its waits, tile lists and descriptors are warp-uniform
+    // values) and the elected lane's tcgen05.mma / commit take effect: issued
+    // from one lane inside a lane-0 branch, the same loop ran 5% slower on
+    // every workload.  Only the MMAs and the waits they need are on this
+    // path (K/V waits come from the async proxy and need no tcgen05 fence;
+    // only P handoffs do).
+    {
+      const uint32_t leader = elect_one();
       uint32_t kv_pos = 0;
       uint32_t n_units = 0;
       uint32_t p_cnt[2] = {0, 0};
@@ -484,22 +532,22 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         for (int k = 0; k < C::kKSteps; ++k) {
           const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
           if (kFp8)
-            mma_ss_f8(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
+            mma_ss_f8_w(leader, tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
           else
-            mma_ss(tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
+            mma_ss_w(leader, tmem + s * 128, a0 + off, b0 + off, C::kIdescS, k > 0 ? 1u : 0u);
         }
       };
       // P from TMEM (32 bytes of keys = 8 columns per K step); B: bf16 V
       // MN-major (16 key rows per step), or e4m3 V^T K-major (32 key bytes)
-      auto issue_pv = [&](int s, uint32_t st, bool acc) {
+      auto issue_pv = [&](int s, uint32_t st, bool acc, int k0, int k1) {
 #pragma unroll
-        for (int k = 0; k < C::kPVSteps; ++k) {
+        for (int k = k0; k < k1; ++k) {
           if (kFp8)
-            mma_ts_f8(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
+            mma_ts_f8_w(leader, tmem + 256 + s * 128, tmem + s * 128 + k * 8,
                       dkv_k + ((st * C::kTileBytes + k * 32) >> 4), C::kIdescPV,
                       (acc || k > 0) ? 1u : 0u);
           else
-            mma_ts(tmem + 256 + s * 128, tmem + s * 128 + k * 8,
+            mma_ts_w(leader, tmem + 256 + s * 128, tmem + s * 128 + k * 8,
                    dkv_v + ((st * C::kTileBytes + k * 2048) >> 4), C::kIdescPV,
                    (acc || k > 0) ? 1u : 0u);
         }
@@ -529,9 +577,9 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           for (int s = 0; s < 2; ++s)
             if (ea_tile_code(shape, ut, sparse, s, t0)) {
               issue_s(s, st);
-              mma_commit(bars.s_full + 8 * s);
+              mma_commit_w(leader, bars.s_full + 8 * s);
             }
-          mma_commit(bars.kv_empty + 8 * st);
+          mma_commit_w(leader, bars.kv_empty + 8 * st);
         }
         bool first_pv[2] = {true, true};
         for (int i = 0; i < ut.n && ok; ++i) {
@@ -554,10 +602,9 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (ea_tile_code(shape, ut, sparse, s, t)) {
-              ok = mbar_wait(bars.p_full + 8 * s, p_cnt[s] & 1, s_abort, status, tlim,
+              ok = mbar_wait(bars.p_half + 8 * s, p_cnt[s] & 1, s_abort, status, tlim,
                              EA_ERR_TIMEOUT);
               if (!ok) break;
-              ++p_cnt[s];
               if (first_pv[s]) {
                 if (u_cnt[s] > 0) {
                   ok = mbar_wait(bars.o_empty + 8 * s, (u_cnt[s] - 1) & 1, s_abort, status, tlim,
@@ -566,26 +613,34 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                 }
                 ++u_cnt[s];
               }
+              // P.V over the first 64 keys as soon as their P is stored,
+              // the rest when the whole P is
               tc_fence_after();
-              issue_pv(s, vst, !first_pv[s]);
+              issue_pv(s, vst, !first_pv[s], 0, C::kPVSteps / 2);
+              ok = mbar_wait(bars.p_full + 8 * s, p_cnt[s] & 1, s_abort, status, tlim,
+                             EA_ERR_TIMEOUT);
+              if (!ok) break;
+              ++p_cnt[s];
+              tc_fence_after();
+              issue_pv(s, vst, true, C::kPVSteps / 2, C::kPVSteps);
               first_pv[s] = false;
-              mma_commit(bars.o_done + 8 * s);
+              mma_commit_w(leader, bars.o_done + 8 * s);
             }
             if (has_next && ea_tile_code(shape, ut, sparse, s, tn)) {
               issue_s(s, kst);
-              mma_commit(bars.s_full + 8 * s);
+              mma_commit_w(leader, bars.s_full + 8 * s);
             }
           }
           if (!ok) break;
-          mma_commit(bars.kv_empty + 8 * vst);
-          if (has_next) mma_commit(bars.kv_empty + 8 * kst);
+          mma_commit_w(leader, bars.kv_empty + 8 * vst);
+          if (has_next) mma_commit_w(leader, bars.kv_empty + 8 * kst);
         }
         if (!ok) break;
-        mma_commit(bars.q_empty);
+        mma_commit_w(leader, bars.q_empty);
         kv_pos += 2 * ut.n;
       }
-      // Drain: wait for every MMA this thread issued.
-      mma_commit(bars.drain);
+      // Drain: wait for every MMA the elected lane issued.
+      mma_commit_w(leader, bars.drain);
       mbar_wait_drain(bars.drain, 0, 200000000ull);
     }
     __syncwarp();
@@ -683,8 +738,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           m_ref = m_tile;
         }
         const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // p = 2^(s * scale * log2e - m): packed FMA, then exp2 on the MUFU for
-        // most pairs and on the FMA pipe for kEmuPairs of every 8 pairs
+        // p = 2^(s * scale * log2e - m)
         float acc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.f;
@@ -711,29 +765,19 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           }
           tmem_st32(tS, pk);
         } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float p0, p1;
-            fma2_sc(p0, p1, x[c * 32 + 2 * j], x[c * 32 + 2 * j + 1], sl2, -msub);
-            if ((j & 7) < kEmuPairs) {
-              exp2_poly2(p0, p1);
-            } else {
-              p0 = ex2_approx(p0);
-              p1 = ex2_approx(p1);
-            }
-            pk[j] = pack_bf16x2(p0, p1);
-            // the row sum adds the bf16 values the P.V product sees, so the
-            // weights applied to V sum to one even in rows with few keys
-            add2_acc(acc[2 * (j & 3)], acc[2 * (j & 3) + 1], __uint_as_float(pk[j] << 16),
-                     __uint_as_float(pk[j] & 0xffff0000u));
-          }
-          tmem_st16(tS + c * 16, pk);
+          // a tile with masked pairs (code 2) holds every key of the rows
+          // that see fewer than 128 keys; there the row sum adds the
+          // bf16-rounded probabilities, so such rows' weights sum to one
+          // exactly (a one-key row gives v itself)
+          if (code == 2)
+            softmax_p_bf16<true, 0, 2>(x, sl2, msub, tS, acc);
+          else
+            softmax_p_bf16<false, 0, 2>(x, sl2, msub, tS, acc);
         }
-        }
-        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        // O is rescaled (rarely) before the first half of P is handed over,
+        // so the first half's P.V product accumulates onto the rescaled O;
+        // the previous P.V is complete, since this tile's S product followed
+        // it on the same issuing thread
         if (__any_sync(0xffffffffu, rescale)) {
           ok = mbar_wait(bars.o_done + 8 * slot, (pv_cnt - 1) & 1, s_abort, status, tlim,
                          EA_ERR_TIMEOUT);
@@ -750,6 +794,18 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
             tmem_st64(tO + h * 64, o);
           }
         }
+        // the first 64 keys' P: the issuer starts their P.V while the
+        // second half is computed
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars.p_half + 8 * slot);
+        if constexpr (!kFp8) {
+          if (code == 2)
+            softmax_p_bf16<true, 2, 4>(x, sl2, msub, tS, acc);
+          else
+            softmax_p_bf16<false, 2, 4>(x, sl2, msub, tS, acc);
+        }
+        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bars.p_full + 8 * slot);
