@@ -685,10 +685,17 @@ ea_status ea_hybrid_attn_prefill_fp8(const void* q8, const void* k8, const void*
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
+// Backward workspace: status block; D [B*Hq*N]; the dK/dV kernel's padded
+// vectors -lse*log2e and -D [B*Hq][npad] each; the schedule's unit lists.
+size_t bwd_pad_rows(const ea_attn_params* p) {
+  return static_cast<size_t>(p->B) * p->Hq * ((p->N + EA_BN - 1) / EA_BN) * EA_BN;
+}
+
 size_t ea_hybrid_attn_backward_workspace_size(const ea_attn_params* p) {
   if (check_params(p) != EA_OK || p->d != 128) return 0;
   const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
   return kAttnWorkspace + (rows * sizeof(float) + 255) / 256 * 256 +
+         2 * bwd_pad_rows(p) * sizeof(float) +
          ea::bwd_sched_ints(p->B, p->Hq, p->Hkv, p->N) * sizeof(int);
 }
 
@@ -714,11 +721,14 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
       !encode_bhsd(&a.tm_do, dout, p->d, p->N, p->B * p->Hq))
     return EA_ERR_CUDA;
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + kAttnWorkspace);
+  const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
+  // the padded vectors after D (512-byte aligned: every tile's vector is one
+  // aligned bulk copy), then the schedule's unit lists
+  float* vl_pad = reinterpret_cast<float*>(static_cast<char*>(workspace) + kAttnWorkspace +
+                                           (rows * sizeof(float) + 255) / 256 * 256);
+  float* vd_pad = vl_pad + bwd_pad_rows(p);
   {
-    // the schedule's unit lists after D
-    const size_t rows = static_cast<size_t>(p->B) * p->Hq * p->N;
-    int* w = reinterpret_cast<int*>(static_cast<char*>(workspace) + kAttnWorkspace +
-                                    (rows * sizeof(float) + 255) / 256 * 256);
+    int* w = reinterpret_cast<int*>(vd_pad + bwd_pad_rows(p));
     const size_t nT = static_cast<size_t>((p->N + EA_BN - 1) / EA_BN);
     const size_t ukv = static_cast<size_t>(p->B) * p->Hkv * nT;
     const size_t uq = static_cast<size_t>(p->B) * p->Hq * nT;
@@ -735,6 +745,9 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
   }
   a.lse = lse;
   a.dvec = dvec;
+  a.vl_pad = vl_pad;
+  a.vd_pad = vd_pad;
+  a.npad = static_cast<int>(((p->N + EA_BN - 1) / EA_BN) * EA_BN);
   a.mask = route_mask;
   a.dq = static_cast<__nv_bfloat16*>(dq);
   a.dk = static_cast<__nv_bfloat16*>(dk);
@@ -751,7 +764,8 @@ ea_status ea_hybrid_attn_backward(const void* q, const void* k, const void* v, c
   a.timeout_ns = wait_timeout_ns();
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
-  cudaError_t err = ea::launch_backward(a, dout, out, dvec, sms, static_cast<cudaStream_t>(stream));
+  cudaError_t err = ea::launch_backward(a, dout, out, dvec, vl_pad, vd_pad, sms,
+                                        static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

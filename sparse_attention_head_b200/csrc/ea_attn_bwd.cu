@@ -46,16 +46,27 @@ namespace ea {
 
 // D[row] = sum_c dO[row][c] * O[row][c] over rows of [rows][d] (d = 128):
 // 16 lanes per row with 16-byte loads (two rows per warp step), the 16
-// partial sums reduced by xor shuffles in a fixed order.
+// partial sums reduced by xor shuffles in a fixed order.  Rows are visited as
+// (b*Hq + h, q) over q < npad: for q < N the kernel writes D to dvec and, for
+// the dK/dV kernel's bulk copies, -D to vd_pad and -lse * log2(e) to vl_pad;
+// the padding (q >= N) gets zeros there.
 __global__ void ea_bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ dout,
-                                     const __nv_bfloat16* __restrict__ out, int rows, int d,
-                                     float* __restrict__ dvec) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  const int row = t >> 4, c0 = (t & 15) * 8;
+                                     const __nv_bfloat16* __restrict__ out,
+                                     const float* __restrict__ lse, int bh_count, int N, int npad,
+                                     int d, float* __restrict__ dvec, float* __restrict__ vl_pad,
+                                     float* __restrict__ vd_pad) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long prow = t >> 4;                   // padded row: bh * npad + q
+  const int c0 = static_cast<int>(t & 15) * 8;
+  const bool in_range = prow < static_cast<long long>(bh_count) * npad;
+  const int bh = in_range ? static_cast<int>(prow / npad) : 0;
+  const int q = in_range ? static_cast<int>(prow % npad) : 0;
+  const bool valid = in_range && q < N;
+  const size_t row = static_cast<size_t>(bh) * N + q;
   float s = 0.f;
-  if (row < rows) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + static_cast<size_t>(row) * d + c0));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + static_cast<size_t>(row) * d + c0));
+  if (valid) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + row * d + c0));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + row * d + c0));
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -65,7 +76,16 @@ __global__ void ea_bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ dout,
   }
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if ((t & 15) == 0 && row < rows) dvec[row] = s;
+  if ((t & 15) == 0 && in_range) {
+    if (valid) {
+      dvec[row] = s;
+      vd_pad[prow] = -s;
+      vl_pad[prow] = -lse[row] * 1.4426950408889634f;
+    } else {
+      vd_pad[prow] = 0.f;
+      vl_pad[prow] = 0.f;
+    }
+  }
 }
 
 // Shared-memory plan of both backward kernels (d = 128).  The streamed
@@ -601,23 +621,19 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
-          if (kDkDv) {
-            float* vl = vec0 + s0 * 128;
-            for (int r = lane; r < EA_BM; r += 32) {
-              const int q = it * EA_BM + r;
-              const size_t ri = (static_cast<size_t>(b) * args.Hq + h) * args.N + q;
-              vl[r] = q < args.N ? -args.lse[ri] * kLog2e : 0.f;
-            }
-            __syncwarp();
-          }
           if (lane == 0) {
             BwdStep& st = steps[s0];
             st.b = b; st.h = h; st.it = it; st.jt = jt; st.sa = sa;
             st.first = (g == 0 && i == 0);
             st.last = (g == ng - 1 && i == n - 1);
             st.full = bwd_block_full(it, jt, args.N, sa, args.sink, args.window);
-            mbar_arrive_expect_tx(b_full0 + 8 * s0, C::kTileBytes);
+            mbar_arrive_expect_tx(b_full0 + 8 * s0, C::kTileBytes + (kDkDv ? 512u : 0u));
             ++armed0;
+            if (kDkDv)   // the query tile's -lse * log2e: one 512-byte copy
+              bulk_load(smem_u32(vec0 + s0 * 128),
+                        args.vl_pad + (static_cast<size_t>(b) * args.Hq + h) * args.npad +
+                            it * EA_BM,
+                        512, b_full0 + 8 * s0);
             const uint32_t dst = smem_u32(smem + C::kOffSt0) + s0 * C::kTileBytes;
             const CUtensorMap* m = kDkDv ? &args.tm_q : &args.tm_k;
             const int z = kDkDv ? b * args.Hq + h : b * args.Hkv + h / G;
@@ -632,18 +648,14 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
-          if (kDkDv) {
-            float* vd = vec1 + s1 * 128;
-            for (int r = lane; r < EA_BM; r += 32) {
-              const int q = it * EA_BM + r;
-              const size_t ri = (static_cast<size_t>(b) * args.Hq + h) * args.N + q;
-              vd[r] = q < args.N ? -args.dvec[ri] : 0.f;
-            }
-            __syncwarp();
-          }
           if (lane == 0) {
-            mbar_arrive_expect_tx(b_full1 + 8 * s1, C::kTileBytes);
+            mbar_arrive_expect_tx(b_full1 + 8 * s1, C::kTileBytes + (kDkDv ? 512u : 0u));
             ++armed1;
+            if (kDkDv)   // the query tile's -D
+              bulk_load(smem_u32(vec1 + s1 * 128),
+                        args.vd_pad + (static_cast<size_t>(b) * args.Hq + h) * args.npad +
+                            it * EA_BM,
+                        512, b_full1 + 8 * s1);
             const uint32_t dst = smem_u32(smem + C::kOffSt1) + s1 * C::kTileBytes;
             const CUtensorMap* m = kDkDv ? &args.tm_do : &args.tm_v;
             const int z = kDkDv ? b * args.Hq + h : b * args.Hkv + h / G;
@@ -674,7 +686,11 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
     // so the tensor pipe and the elementwise warps work at the same time.
     // tcgen05.mma from one thread executes in issue order, so a score
     // product overwrites the columns the accumulating product before it read.
-    if (lane == 0) {
+    // The whole warp runs this loop and the elected lane's MMAs and commits
+    // take effect (warp-uniform descriptors and counters; the fused forward
+    // runs 5% faster this way than from a lane-0 branch).
+    {
+      const uint32_t leader = elect_one();
       const uint32_t res = smem_u32(smem + C::kOffRes);
       // K-major views (the score products) and MN-major views (the B operand
       // of the accumulating products)
@@ -693,7 +709,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k >> 2) * C::kBlockBytes + (k & 3) * 32) >> 4;
-          mma_ss(tmem + 128 * which, a + off, b + off, C::kIdescSS, k > 0 ? 1u : 0u);
+          mma_ss_w(leader, tmem + 128 * which, a + off, b + off, C::kIdescSS, k > 0 ? 1u : 0u);
         }
       };
       auto wait_full = [&](int which, uint32_t p) {
@@ -709,10 +725,10 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
         const uint32_t unit = nu++;
         if (!(ok = wait_full(0, pos))) break;
         scores(pos, 0);
-        mma_commit(b_s_full);
+        mma_commit_w(leader, b_s_full);
         if (!(ok = wait_full(1, pos))) break;
         scores(pos, 1);
-        mma_commit(b_dp_full);
+        mma_commit_w(leader, b_dp_full);
         bool last = false, first = true;
         while (!last && ok) {
           const uint32_t s0 = pos % C::kStages0, s1 = pos % C::kStages1;
@@ -732,7 +748,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
           if (kDkDv) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              mma_ts(tmem + 256, tmem + 64 * (k >> 2) + 8 * (k & 3), m1 + ((k * 2048) >> 4),
+              mma_ts_w(leader, tmem + 256, tmem + 64 * (k >> 2) + 8 * (k & 3), m1 + ((k * 2048) >> 4),
                      C::kIdescTS, (!first || k > 0) ? 1u : 0u);            // dV += P^T dO
           }
           // (TMA-written tiles need no tcgen05 fence: the mbarrier completes
@@ -740,7 +756,7 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
           if (!last) {
             if (!(ok = wait_full(0, pos + 1))) break;
             scores(pos + 1, 0);
-            mma_commit(b_s_full);
+            mma_commit_w(leader, b_s_full);
           }
           // dS (bf16 at the start of each column half's dP columns)
           if (!(ok = mbar_wait(b_ds_full, nsteps & 1, s_abort, status, tlim, EA_ERR_TIMEOUT)))
@@ -748,28 +764,28 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ts(tmem + (kDkDv ? 384 : 256), tmem + 128 + 64 * (k >> 2) + 8 * (k & 3),
+            mma_ts_w(leader, tmem + (kDkDv ? 384 : 256), tmem + 128 + 64 * (k >> 2) + 8 * (k & 3),
                    m0 + ((k * 2048) >> 4), C::kIdescTS,
                    (!first || k > 0) ? 1u : 0u);           // dK += dS^T Q  /  dQ += dS K
           // the step's tiles (and, read by the elementwise warps before
           // ds_full, its vectors) are free once these products complete
-          mma_commit(b_empty0 + 8 * s0);
-          mma_commit(b_empty1 + 8 * s1);
+          mma_commit_w(leader, b_empty0 + 8 * s0);
+          mma_commit_w(leader, b_empty1 + 8 * s1);
           if (!last) {
             if (!(ok = wait_full(1, pos + 1))) break;
             scores(pos + 1, 1);
-            mma_commit(b_dp_full);
+            mma_commit_w(leader, b_dp_full);
           }
           ++nsteps;
           first = false;
           ++pos;
         }
         if (!ok) break;
-        mma_commit(b_acc_done);
-        mma_commit(b_res_empty);
+        mma_commit_w(leader, b_acc_done);
+        mma_commit_w(leader, b_res_empty);
       }
-      // drain: wait for every MMA this thread issued
-      mma_commit(b_drain);
+      // drain: wait for every MMA the elected lane issued
+      mma_commit_w(leader, b_drain);
       mbar_wait_drain(b_drain, 0, 200000000ull);
     }
   } else {
@@ -956,11 +972,11 @@ __global__ void __launch_bounds__(BwdCfg::kThreads, 1) ea_bwd_attn_kernel(
 static int g_bwd_configured[64] = {0};
 
 cudaError_t launch_backward(const BwdArgs& a, const void* dout, const void* out, float* dvec,
-                            int grid_sms, cudaStream_t stream) {
-  const int rows = a.B * a.Hq * a.N;
-  ea_bwd_rowdot_kernel<<<(rows + 15) / 16, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), rows,
-      BwdCfg::D, dvec);
+                            float* vl_pad, float* vd_pad, int grid_sms, cudaStream_t stream) {
+  const long long prows = static_cast<long long>(a.B) * a.Hq * a.npad;
+  ea_bwd_rowdot_kernel<<<static_cast<unsigned>((prows + 15) / 16), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), a.lse,
+      a.B * a.Hq, a.N, a.npad, BwdCfg::D, dvec, vl_pad, vd_pad);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   int dev = 0;

@@ -81,6 +81,13 @@ struct BwdArgs {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // (d, N, B*heads) boxes of 64 x 128 x 1
   const float* lse;                      // [B][Hq][N] natural log-sum-exp
   const float* dvec;                     // [B][Hq][N] rowsum(dO * O) (computed first)
+  // The dK/dV kernel's per-step vectors, written with dvec: for query q of
+  // (b, h), row b * Hq + h of [B*Hq][npad] (npad = 128 * ceil(N / 128)):
+  // -lse * log2(e) and -D, zero for q >= N.  Each 128-query tile's vector is
+  // one 512-byte bulk copy.
+  const float* vl_pad;
+  const float* vd_pad;
+  int npad;
   const uint8_t* mask;                   // [B][Hq]
   __nv_bfloat16* dq;                     // [B][Hq][N][d]
   __nv_bfloat16* dk;                     // [B][Hkv][N][d]
@@ -105,9 +112,10 @@ struct BwdArgs {
 constexpr int kBwdMaxGrid = 1024;
 // Ints of backward workspace the unit lists need, after D.
 size_t bwd_sched_ints(int B, int Hq, int Hkv, int N);
-// D = rowsum(dO * O) into dvec, then the dK/dV and dQ kernels.
+// D = rowsum(dO * O) into dvec (and the padded vectors vl_pad, vd_pad), then
+// the dK/dV and dQ kernels.
 cudaError_t launch_backward(const BwdArgs& a, const void* dout, const void* out, float* dvec,
-                            int grid_sms, cudaStream_t stream);
+                            float* vl_pad, float* vd_pad, int grid_sms, cudaStream_t stream);
 
 // SM count of the current device (cached per device); 0 on error.
 int device_sms();

@@ -23,11 +23,12 @@ def _lib_built():
 
 def _read_lists(ws, B, Hq, Hkv, N):
     """Workspace: 256-byte status block, D (fp32 [B][Hq][N], padded to 256
-    bytes), then int32 offs_kv[1025], offs_q[1025], list/sorted/cta of dK/dV,
+    bytes), the dK/dV kernel's two padded vectors (fp32 [B*Hq][128 nT] each),
+    then int32 offs_kv[1025], offs_q[1025], list/sorted/cta of dK/dV,
     list/sorted/cta of dQ."""
     nT = -(-N // m.BN)
     ukv, uq = B * Hkv * nT, B * Hq * nT
-    base = 256 + (B * Hq * N * 4 + 255) // 256 * 256
+    base = 256 + (B * Hq * N * 4 + 255) // 256 * 256 + 2 * B * Hq * nT * 128 * 4
     ints = ws[base:].view(torch.int32).cpu().numpy().astype(np.int64)
     g = m.MAX_GRID + 1
     offs_kv, offs_q = ints[:g], ints[g:2 * g]
