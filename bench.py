@@ -181,18 +181,30 @@ def visible_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
+ATTN_KERNEL_SOURCES = ("ea_attn.cu", "ea_sched.h", "ea_internal.h", "ea_ptx.cuh", "ea_tmem.cuh",
+                       "ea_math.cuh")
+
+
+def attn_kernel_source_hash() -> str:
+    """sha256 (16 hex digits) over the fused attention kernel's source files,
+    in the order of ATTN_KERNEL_SOURCES."""
+    h = hashlib.sha256()
+    for name in ATTN_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_attention_head_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_for_current_kernel(workload: str, seq: int):
     """Per-launch DRAM bytes of the attention kernel on this workload, from the
     committed ncu summary: only if a capture exists for this workload at this
     sequence length and was taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", "attn_traffic.json")
-    src = os.path.join(ROOT, "sparse_attention_head_b200", "csrc", "ea_attn.cu")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("kernel_sha256_16") != h:
+    if d.get("kernel_sha256_16") != attn_kernel_source_hash():
         return None
     e = d.get("workloads", {}).get(workload)
     if not e or int(e.get("seq", -1)) != int(seq):

@@ -200,9 +200,13 @@ size_t ea_hybrid_attn_workspace_size(const ea_attn_params* p);
  * out       : device bf16 [B][Hq][N][d]; rows of heads not selected by
  *             p->select are left untouched.
  * workspace : device, >= ea_hybrid_attn_workspace_size(p) bytes, ZEROED
- *             once before its first use; the kernel only ever writes a
- *             nonzero error code into it (ea_get_device_status reads it and,
- *             after an error, clears the 256-byte status block).
+ *             once before its first use.  Its first 256 bytes are the status
+ *             block: the kernel writes a nonzero error code into its status
+ *             word, and keeps its dispatch counters (CTAs take work units
+ *             from a global counter) at bytes 192-231, back at zero when the
+ *             launch ends.  ea_get_device_status reads the status word and,
+ *             after an error, clears the whole block.  Launches that may
+ *             run at the same time need separate workspaces.
  * Limits: d in {64, 128}; Hq % Hkv == 0; B <= 1024; B*Hq <= 4096;
  * N <= 32767 * 256.
  */
@@ -651,7 +655,9 @@ ea_status ea_hybrid_attn_prefill_host(const void* q_host, const void* k_host,
  * Host-side view of the fused kernel's work schedule, for inspection and
  * tests (no GPU needed).  A unit is (mode, b, h, pair): 256 query rows
  * [256*pair, 256*pair + 256) of head h in batch b, run by one CTA.  Units
- * are ordered longest first and dealt to CTAs in a snake order.
+ * are ordered longest first; a CTA takes the next unit of that order from a
+ * global counter whenever it starts one (the order is fixed, the CTA that
+ * runs a unit is not).
  *
  * mask        : host uint8 [B][Hq].
  * units_out   : host int32 [max_units][5] = {sparse, b, h, pair, n_kv_tiles}

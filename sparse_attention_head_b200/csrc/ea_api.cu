@@ -230,14 +230,15 @@ void build_host_sched(const uint8_t* mask, int B, int Hq, int select, const int*
 }
 
 // Units of a schedule in rank order: {sparse, b, h, pair, n_kv_tiles}.
-int list_units(const HostSched& h, int Hq, int S, int W, int32_t* units_out, int max_units) {
+int list_units(const HostSched& h, int Hq, int Hkv, int d, int S, int W, int32_t* units_out,
+               int max_units) {
   const int total = ea_total_units(h.view);
   if (units_out) {
     EaCursor cur;
-    ea_cursor_init(cur, h.view);
+    ea_cursor_init(cur, h.view, h.ent.data(), Hq, Hkv, ea_group_major(h.view.Pmax, d));
     for (int r = 0; r < total && r < max_units; ++r) {
       int sparse = 0, e = 0, pair = 0;
-      if (!ea_cursor_seek(cur, h.view, r, &sparse, &e, &pair)) break;
+      if (!ea_cursor_seek(cur, h.view, h.ent.data(), r, &sparse, &e, &pair)) break;
       const int idx = h.ent[sparse ? h.nfa + e : e];
       const EaShape sh = ea_make_shape(h.len[idx / Hq], S, W);
       const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
@@ -985,7 +986,7 @@ int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p, int32_t* uni
   std::vector<int> lens(p->B, p->N);
   HostSched h;
   build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
-  return list_units(h, p->Hq, p->sink, p->window, units_out, max_units);
+  return list_units(h, p->Hq, p->Hkv, p->d, p->sink, p->window, units_out, max_units);
 }
 
 int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
@@ -999,7 +1000,7 @@ int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
   }
   HostSched h;
   build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
-  return list_units(h, p->Hq, p->sink, p->window, units_out, max_units);
+  return list_units(h, p->Hq, p->Hkv, p->d, p->sink, p->window, units_out, max_units);
 }
 
 int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int rank,
@@ -1011,9 +1012,9 @@ int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int ran
   const int total = ea_total_units(h.view);
   if (rank < 0 || rank >= total) return -1;
   EaCursor cur;
-  ea_cursor_init(cur, h.view);
+  ea_cursor_init(cur, h.view, h.ent.data(), p->Hq, p->Hkv, ea_group_major(h.view.Pmax, p->d));
   int sparse = 0, e = 0, pair = 0;
-  if (!ea_cursor_seek(cur, h.view, rank, &sparse, &e, &pair)) return -1;
+  if (!ea_cursor_seek(cur, h.view, h.ent.data(), rank, &sparse, &e, &pair)) return -1;
   const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
   const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
   for (int i = 0; i < ut.n && i < max_tiles; ++i) {

@@ -74,10 +74,13 @@ struct AttnCfg {
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   // q_full, q_empty, drain, kv_full[kStages], kv_empty[kStages],
-  // s_full[2], p_full[2], o_done[2], o_empty[2], p_half[2]
-  static constexpr int kNumBars = 3 + 2 * kStages + 10;
+  // s_full[2], p_full[2], o_done[2], o_empty[2], p_half[2],
+  // unit_full[kUnitRing], unit_empty[kUnitRing]
+  static constexpr int kUnitRing = 4;                       // units the producer runs ahead
+  static constexpr int kNumBars = 3 + 2 * kStages + 10 + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, counts
-  static constexpr int kOffEnt = kOffMisc + 64;
+  static constexpr int kOffUnit = kOffMisc + 64;            // the unit ring: {rank, unit word}
+  static constexpr int kOffEnt = kOffUnit + 64;
   // sequence tables: token offset and length by index, order and unit count by
   // sorted position, FA / SA entry prefix counts by sorted position
   static constexpr int kOffTok = kOffEnt + EA_MAX_ENTRIES * 2;
@@ -109,6 +112,8 @@ struct Bars {
   uint32_t o_done;
   uint32_t o_empty;
   uint32_t p_half;
+  uint32_t unit_full;
+  uint32_t unit_empty;
 };
 
 // Route bit of entry idx, read through the coherent path: in a routed launch
@@ -121,6 +126,19 @@ __device__ __forceinline__ uint8_t ld_mask(const uint8_t* mask, int idx) {
 __device__ __forceinline__ bool in_shard(const AttnArgs& args, int b, int h) {
   return args.group_sel == nullptr ||
          args.group_sel[b * args.Hkv + h / (args.Hq / args.Hkv)] != 0;
+}
+
+// This CTA takes no more tickets (its producer has stopped, or never
+// started); the last CTA of the launch to get here resets the dispatch
+// counters for the next launch on this workspace.
+__device__ __forceinline__ void release_dispatch(const AttnArgs& args) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(args.done_ctas, 1u) == gridDim.x - 1) {
+      atomicExch(args.ticket, 0u);
+      atomicExch(args.done_ctas, 0u);
+    }
+  }
 }
 
 // Grid barrier of the routed prologue.  Every CTA arrives once per phase;
@@ -257,8 +275,10 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   if constexpr (kRouted) {
-    if (!routed_prologue<D>(args, smem, reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16)))
+    if (!routed_prologue<D>(args, smem, reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16))) {
+      release_dispatch(args);
       return;   // a grid barrier timed out; nothing is allocated or in flight yet
+    }
   }
 
   const int warp = threadIdx.x >> 5;
@@ -280,6 +300,8 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     bars.o_done = bars.p_full + 16;
     bars.o_empty = bars.o_done + 16;
     bars.p_half = bars.o_empty + 16;
+    bars.unit_full = bars.p_half + 16;
+    bars.unit_empty = bars.unit_full + 8 * C::kUnitRing;
   }
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -288,13 +310,14 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   // last P handed over): kept in shared memory, off the softmax registers
   uint64_t* s_trace_ts = reinterpret_cast<uint64_t*>(smem + C::kOffMisc + 32);
   uint16_t* s_ent = reinterpret_cast<uint16_t*>(smem + C::kOffEnt);
+  volatile int* s_unit = reinterpret_cast<volatile int*>(smem + C::kOffUnit);
 
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     // bar_base layout: q_full, q_empty, drain, kv_full[kStages],
     // kv_empty[kStages], s_full[2], p_full[2], o_done[2], o_empty[2],
-    // p_half[2]
+    // p_half[2], unit_full[kUnitRing], unit_empty[kUnitRing]
     mbar_init(bar_base + 0, 1);                        // q_full: producer
     mbar_init(bar_base + 1, 1);                        // q_empty: MMA issuer
     mbar_init(bar_base + 2, 1);                        // drain: MMA issuer
@@ -308,6 +331,11 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       mbar_init(bar_base + 3 + 2 * C::kStages + 4 + s, 1);    // o_done
       mbar_init(bar_base + 3 + 2 * C::kStages + 6 + s, 128);  // o_empty
       mbar_init(bar_base + 3 + 2 * C::kStages + 8 + s, 128);  // p_half
+    }
+    for (int u = 0; u < C::kUnitRing; ++u) {
+      mbar_init(bar_base + 3 + 2 * C::kStages + 10 + u, 1);   // unit_full: producer
+      // unit_empty: the MMA warp's elected lane and lane 0 of the 8 softmax warps
+      mbar_init(bar_base + 3 + 2 * C::kStages + 10 + C::kUnitRing + u, 9);
     }
     *s_abort = 0;
     fence_mbar_init();
@@ -437,13 +465,33 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       uint32_t n_units = 0;
       bool ok = true;
       EaCursor cur;
-      ea_cursor_init(cur, view);
+      ea_cursor_init(cur, view, s_ent, args.Hq, args.Hkv, ea_group_major(view.Pmax, D));
+      // Tickets come one unit ahead: the counter's reply (a global atomic, up
+      // to microseconds under the launch's memory traffic) returns while this
+      // unit's loads are issued, instead of delaying the next unit's Q load.
+      unsigned int next_ticket = atomicAdd(args.ticket, 1u);
       for (int kk = 0; ok; ++kk) {
-        const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+        // the next unit, published to the MMA and softmax warps through the
+        // unit ring
+        const int us = kk % C::kUnitRing;
+        if (kk >= C::kUnitRing) {
+          ok = mbar_wait(bars.unit_empty + 8 * us, ((kk / C::kUnitRing) - 1) & 1, s_abort, status,
+                         tlim, EA_ERR_TIMEOUT);
+          if (!ok) break;
+        }
+        const unsigned int ticket = next_ticket;
+        const int r = ticket < static_cast<unsigned int>(total) ? static_cast<int>(ticket) : -1;
+        int sparse = 0, e = 0, pair = 0;
+        if (r >= 0) ea_cursor_seek(cur, view, s_ent, r, &sparse, &e, &pair);
+        const int idx = r >= 0 ? static_cast<int>(s_ent[sparse ? nFA + e : e]) : 0;
+        // Only this thread runs the cursor: the other roles read the unit
+        // decoded, {rank, pair << 13 | sparse << 12 | entry} (an entry index
+        // is below 4096, a pair below 32768).
+        s_unit[2 * us] = r;
+        s_unit[2 * us + 1] = (pair << 13) | (sparse << 12) | idx;
+        mbar_arrive(bars.unit_full + 8 * us);
         if (r < 0) break;
-        int sparse, e, pair;
-        ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
-        const int idx = s_ent[sparse ? nFA + e : e];
+        next_ticket = atomicAdd(args.ticket, 1u);
         const int b = idx / args.Hq, h = idx % args.Hq;
         // tensor coordinates: padded batch (row, head index b*H + h); packed
         // batch (token, head)
@@ -552,14 +600,17 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                    (acc || k > 0) ? 1u : 0u);
         }
       };
-      EaCursor cur;
-      ea_cursor_init(cur, view);
       for (int kk = 0; ok; ++kk) {
-        const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+        const int us = kk % C::kUnitRing;
+        ok = mbar_wait(bars.unit_full + 8 * us, (kk / C::kUnitRing) & 1, s_abort, status, tlim,
+                       EA_ERR_TIMEOUT);
+        if (!ok) break;
+        const int r = s_unit[2 * us];
+        const int word = s_unit[2 * us + 1];
+        __syncwarp();
+        if (leader) mbar_arrive(bars.unit_empty + 8 * us);
         if (r < 0) break;
-        int sparse, e, pair;
-        ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
-        const int idx = s_ent[sparse ? nFA + e : e];
+        const int sparse = (word >> 12) & 1, pair = word >> 13, idx = word & 4095;
         const EaShape shape = ea_make_shape(s_len[idx / args.Hq], args.sink, args.window);
         const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
 
@@ -657,14 +708,18 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     uint32_t s_cnt = 0;
     uint32_t pv_cnt = 0;
     bool ok = true;
-    EaCursor cur;
-    ea_cursor_init(cur, view);
     for (int kk = 0; ok; ++kk) {
-      const int r = ea_rank_for(kk, blockIdx.x, gridDim.x, total);
+      const int us = kk % C::kUnitRing;
+      ok = mbar_wait(bars.unit_full + 8 * us, (kk / C::kUnitRing) & 1, s_abort, status, tlim,
+                     EA_ERR_TIMEOUT);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int r = s_unit[2 * us];
+      const int word = s_unit[2 * us + 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.unit_empty + 8 * us);
       if (r < 0) break;
-      int sparse, e, pair;
-      ea_cursor_seek(cur, view, r, &sparse, &e, &pair);
-      const int idx = s_ent[sparse ? nFA + e : e];
+      const int sparse = (word >> 12) & 1, pair = word >> 13, idx = word & 4095;
       const int seq = idx / args.Hq;
       const int seq_len = s_len[seq];
       const EaShape shape = ea_make_shape(seq_len, args.sink, args.window);
@@ -872,6 +927,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  release_dispatch(args);
 }
 
 int attn_smem_bytes(int D) {
@@ -879,8 +935,13 @@ int attn_smem_bytes(int D) {
 }
 
 template <int D, bool kRouted, bool kFp8 = false, bool kTrace = false>
-static cudaError_t launch_d(const AttnArgs& args, int grid, cudaStream_t stream) {
+static cudaError_t launch_d(const AttnArgs& args_in, int grid, cudaStream_t stream) {
   const int smem = AttnCfg<D, kFp8>::kSmem;
+  // the dispatch counters sit in the caller's status block (status word at
+  // 0, the routed prologue's grid barrier at 64 and 128)
+  AttnArgs args = args_in;
+  args.ticket = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(args.status) + 192);
+  args.done_ctas = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(args.status) + 224);
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);

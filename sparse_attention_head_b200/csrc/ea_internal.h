@@ -52,6 +52,11 @@ struct alignas(64) AttnArgs {
   // query heads of (batch, kv head) run; the others' output rows are not
   // written.
   const uint8_t* group_sel;
+  // Dynamic unit dispatch, inside the caller's 256-byte status block: the
+  // launch's ticket counter and the count of CTAs done taking tickets (the
+  // last one resets both to zero for the next launch).  Set by the launcher.
+  unsigned int* ticket;
+  unsigned int* done_ctas;
   // Per-unit trace (nullptr = off): trace[0] counts records; record i sits
   // at trace[8 + 6 i] .. +5 = {start, first S ready, last P handed over,
   // end (ns), CTA << 32 | rank, sparse << 32 | KV tiles}; records past

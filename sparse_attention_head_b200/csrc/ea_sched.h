@@ -12,13 +12,26 @@
 //   tiles = the 128-key KV tiles the unit visits.  FA: 0..last.  SA: the sink
 //           tiles [0, ceil(S/128)) and the window tiles [lo, last], where lo
 //           is the tile of the first row's window start.
-//   order = longest first: FA units longer than any SA unit (largest pair
-//           first), then every SA unit, then the remaining FA units; inside
-//           one pair index the heads of one kv group are adjacent, so their
-//           K/V tiles are reused from L2.  Sequences of a batch may differ in
-//           length (EaSeqView).
-//   deal  = rank r goes to CTA c in a snake: round k = r / G covers ranks
-//           [kG, kG+G) left to right when k is even, right to left when odd.
+//   order = longest first: FA units longer than any SA unit, then every SA
+//           unit, then the remaining FA units, each run pair descending; at
+//           one pair the entries go in list order, so the heads of one kv
+//           group are adjacent and their K/V tiles are reused from L2.  For
+//           long sequences (one kv head's K and V at least half the L2) the
+//           long FA units instead go kv group by kv group (a sequence's kv
+//           head and the query heads that read it): the CTAs running at any
+//           moment then stream one or two groups' prefixes, which L2 holds.
+//           Sequences of a batch may differ in length (EaSeqView).
+//   deal  = dynamic: a CTA's producer warp takes the next rank from a
+//           global ticket counter as it starts a unit, so no CTA waits on a
+//           static share, and the units running at any moment stay adjacent
+//           in the order.  The producer alone runs the cursor below and hands
+//           each unit, decoded, to the other roles.
+//   Measured at 256K tokens (32 query, 8 kv heads, d = 128, 24 of 32 heads
+//   SA; one B200): dealt statically in a snake, the CTAs drifted apart and
+//   DRAM reads were ~70x one pass over q, k, v; dealt dynamically, ~44x;
+//   with the long FA units by kv group as well, ~1.4x and 8% less time.  At
+//   192K tokens by group was 4% faster; at 16K-64K tokens by pair was as fast
+//   or faster (up to 7%).
 #pragma once
 
 #include <stdint.h>
@@ -86,16 +99,36 @@ EA_HD int ea_split_pair(int S, int W, int Pmax) {
   return ea_min(sa_cap / 2, Pmax);
 }
 
-// Order (longest first): FA units with pair >= pA (pair descending), then
-// every SA unit (pair descending), then the FA units with pair < pA (pair
-// descending); inside one (phase, pair), entries in list order.  A cursor
-// walks it; ranks must be asked in increasing order.
+// K and V elements of one kv head (of the longest sequence, in whole units)
+// from which the long FA units go kv group by kv group: 2 * 131072 * 128,
+// 64 MB of bf16 K and V, half the L2.
+#define EA_GROUP_MAJOR_ELEMS (1ll << 25)
+
+EA_HD bool ea_group_major(int Pmax, int d) {
+  return 2ll * Pmax * EA_UNIT_ROWS * d >= EA_GROUP_MAJOR_ELEMS;
+}
+
+// Order (longest first): FA units with pair >= pA, then every SA unit (pair
+// descending), then the FA units with pair < pA (pair descending); inside
+// one (phase, pair), entries in list order.  The long FA units go pair
+// descending the same way, or, group-major, kv group by kv group: the
+// groups in (sorted sequence, kv head) order, a group's units pair
+// descending, its heads in order inside a pair.  A group's FA entries are a
+// contiguous run of the FA list (grouped by sorted sequence, heads
+// increasing).  A cursor walks the order; ranks must be asked in increasing
+// order.
 struct EaCursor {
   int phase;   // 0: long FA, 1: SA, 2: short FA, 3: past the end
   int p;       // pair
-  int base;    // rank of the first unit at (phase, p)
-  int cnt;     // units at (phase, p)
+  int base;    // rank of the first unit at (phase, p), or of the group
+  int cnt;     // units at (phase, p), or of the group
   int m;       // sorted sequences with more than p units
+  // phase 0, group-major
+  int gm;      // 1: the long FA units go kv group by kv group
+  int Hq, G, Hkv;
+  int k, hk;   // the group: sorted sequence position, kv head
+  int fa0, nf; // its FA entries: list positions [fa0, fa0 + nf)
+  int fa_end;  // scan position in the sequence's FA run
 };
 
 EA_HD int ea_phase_top(const EaSeqView& v, int phase) {
@@ -117,26 +150,82 @@ EA_HD void ea_cursor_settle(EaCursor& c, const EaSeqView& v) {
   c.cnt = (c.phase == 1 ? v.prefSA : v.prefFA)[c.m];
 }
 
-EA_HD void ea_cursor_init(EaCursor& c, const EaSeqView& v) {
+// Group-major phase 0: the next kv group with long FA units, or phase 1.
+template <class T>
+EA_HD void ea_cursor_next_group(EaCursor& c, const EaSeqView& v, const T* ent) {
+  for (;;) {
+    if (++c.hk >= c.Hkv) {
+      c.hk = 0;
+      ++c.k;
+    }
+    if (c.k >= v.nseq) {
+      c.phase = 1;
+      c.p = ea_phase_top(v, 1);
+      c.m = 0;
+      ea_cursor_settle(c, v);
+      return;
+    }
+    if (c.hk == 0) c.fa_end = v.prefFA[c.k];   // a new sequence: its FA run
+    int a = c.fa_end;
+    const int e = v.prefFA[c.k + 1];
+    while (a < e && (static_cast<int>(ent[a]) % c.Hq) / c.G < c.hk) ++a;
+    int b = a;
+    while (b < e && (static_cast<int>(ent[b]) % c.Hq) / c.G == c.hk) ++b;
+    c.fa0 = a;
+    c.nf = b - a;
+    c.fa_end = b;
+    c.cnt = c.nf * ea_max(v.P[c.k] - v.pA, 0);
+    if (c.cnt > 0) return;
+  }
+}
+
+// ent: the entry lists (FA entries, then SA entries), read by the
+// group-major walk only.
+template <class T>
+EA_HD void ea_cursor_init(EaCursor& c, const EaSeqView& v, const T* ent, int Hq, int Hkv,
+                          bool group_major) {
   c.phase = 0;
   c.p = ea_phase_top(v, 0);
   c.base = 0;
   c.m = 0;
-  ea_cursor_settle(c, v);
+  c.gm = group_major ? 1 : 0;
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.G = Hq / Hkv;
+  c.k = 0;
+  c.hk = -1;
+  c.fa0 = c.nf = c.fa_end = 0;
+  if (c.gm && v.nseq > 0 && v.pA < v.Pmax) {
+    ea_cursor_next_group(c, v, ent);
+  } else {
+    ea_cursor_settle(c, v);
+  }
 }
 
 // Unit of rank r: (sparse, entry index within its list, pair); false past
 // the end.
-EA_HD bool ea_cursor_seek(EaCursor& c, const EaSeqView& v, int r, int* sparse, int* e,
-                          int* pair) {
+template <class T>
+EA_HD bool ea_cursor_seek(EaCursor& c, const EaSeqView& v, const T* ent, int r, int* sparse,
+                          int* e, int* pair) {
   while (c.phase < 3 && r >= c.base + c.cnt) {
     c.base += c.cnt;
-    --c.p;
-    ea_cursor_settle(c, v);
+    if (c.phase == 0 && c.gm) {
+      ea_cursor_next_group(c, v, ent);
+    } else {
+      --c.p;
+      ea_cursor_settle(c, v);
+    }
   }
   if (c.phase >= 3) return false;
+  const int u = r - c.base;
+  if (c.phase == 0 && c.gm) {
+    *sparse = 0;
+    *e = c.fa0 + u % c.nf;
+    *pair = v.P[c.k] - 1 - u / c.nf;
+    return true;
+  }
   *sparse = c.phase == 1;
-  *e = r - c.base;
+  *e = u;
   *pair = c.p;
   return true;
 }
@@ -146,12 +235,6 @@ EA_HD int ea_total_units(const EaSeqView& v) {
   for (int k = 0; k < v.nseq; ++k)
     total += v.P[k] * ((v.prefFA[k + 1] - v.prefFA[k]) + (v.prefSA[k + 1] - v.prefSA[k]));
   return total;
-}
-
-// k-th rank dealt to CTA c of G (or -1 past the end).
-EA_HD int ea_rank_for(int k, int c, int G, int total) {
-  int r = k * G + ((k & 1) ? (G - 1 - c) : c);
-  return r < total ? r : -1;
 }
 
 // Tile list of one unit: [0, a) then [lo, last].

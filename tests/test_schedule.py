@@ -1,7 +1,10 @@
 """Host logic of the fused kernel's schedule (no GPU): every selected
 (b, h, query row) is covered by exactly one unit slot, every tile a slot
 needs is visited with the right masking code, units are ordered longest
-first, and the snake deal gives each rank to exactly one CTA."""
+first (at one pair, the entries in (sorted sequence, head) order, so a kv
+group's heads are adjacent; for long sequences the long FA units kv group by
+kv group), and dynamic dispatch of that order over 148 CTAs balances their
+loads."""
 import numpy as np
 import pytest
 
@@ -91,7 +94,72 @@ def test_unit_tiles_match_definition(B, Hq, Hkv, N, d, S, W, sel):
         assert np.all(codes.max(axis=1) > 0)
 
 
-def test_order_longest_first_and_snake_deal():
+def _dynamic_loads(cost, ctas=148):
+    """Each CTA takes the next unit of the order when it finishes its last
+    one (the kernel's ticket counter); a unit costs its tiles plus an
+    overhead of two tiles."""
+    import heapq
+    heap = [(0.0, c) for c in range(ctas)]
+    for x in cost:
+        t, c = heapq.heappop(heap)
+        heapq.heappush(heap, (t + float(x) + 2.0, c))
+    return np.array([t for t, _ in heap])
+
+
+def _check_pairs_in_entry_order(units, seq_order):
+    """Inside each run of one mode, pair descending; at one pair, the entries
+    in (sorted sequence, head) order."""
+    pos = {b: i for i, b in enumerate(seq_order)}
+    key = [(-int(pair), pos[int(b)], int(h)) for _, b, h, pair, _ in units]
+    assert key == sorted(key)
+
+
+def _group_major(n_max, d):
+    """The order's switch, restated: the long FA units go kv group by kv
+    group from 2 * 131072 * 128 K/V elements per kv head (64 MB of bf16, half
+    the L2), counting the longest sequence in whole 256-row units."""
+    return 2 * (-(-n_max // 256) * 256) * d >= 2 * 131072 * 128
+
+
+def _check_order(units, Hq, Hkv, S, W, seq_order, group_major):
+    """The order's rules from the unit list alone: the long FA units (pair >=
+    pA, longer than any SA unit) first, then every SA unit, then the short FA
+    units.  Group-major, the long FA units of one (b, kv group) are
+    consecutive, the groups in (sorted sequence, kv head) order, inside a
+    group pair descending with heads ascending; otherwise, like the other two
+    runs, pair descending with the entries of one pair in (sorted sequence,
+    head) order.  Returns the number of long FA units."""
+    G = Hq // Hkv
+    pA = (-(-S // 128) + 2 + -(-(W - 1) // 128)) // 2
+    pos = {b: i for i, b in enumerate(seq_order)}
+    long_fa = (units[:, 0] == 0) & (units[:, 3] >= pA)
+    n0 = int(long_fa.sum())
+    assert np.all(long_fa[:n0]) and not np.any(long_fa[n0:])
+    if group_major:
+        runs = []
+        for i, (_, b, h, _, _) in enumerate(units[:n0]):
+            key = (int(b), int(h) // G)
+            if not runs or runs[-1][0] != key:
+                runs.append([key, i, i + 1])
+            else:
+                runs[-1][2] = i + 1
+        assert len({r[0] for r in runs}) == len(runs), "a group's units are not consecutive"
+        order = [(pos[b], hk) for (b, hk), _, _ in runs]
+        assert order == sorted(order)
+        for _, a, e in runs:
+            key = [(-int(pair), int(h)) for _, _, h, pair, _ in units[a:e]]
+            assert key == sorted(key)
+    else:
+        _check_pairs_in_entry_order(units[:n0], seq_order)
+    rest = units[n0:]
+    nsa = int(np.sum(rest[:, 0] == 1))
+    assert np.all(rest[:nsa, 0] == 1) and np.all(rest[nsa:, 0] == 0)
+    _check_pairs_in_entry_order(rest[:nsa], seq_order)
+    _check_pairs_in_entry_order(rest[nsa:], seq_order)
+    return n0
+
+
+def test_order_longest_first_and_dynamic_balance():
     B, Hq, Hkv, N, d, S, W = 1, 32, 8, 32768, 128, 64, 1024
     mask = np.zeros((B, Hq), np.uint8)
     mask[0, [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]] = 1
@@ -105,28 +173,41 @@ def test_order_longest_first_and_snake_deal():
     assert np.all(long_fa[:, 0] == 0)
     assert np.all(np.diff(long_fa[:, 4]) <= 0)
     assert np.all(long_fa[:, 4] > sa_cap)
+    # the first pair: every FA head, kv groups in order
+    assert [int(h) for _, _, h, _, _ in units[:nfa]] == [0, 3, 4, 6, 8, 10, 14, 16, 21, 27]
     # then SA units, then the short FA units
     rest = units[len(long_fa):]
     assert np.all(rest[: 22 * 128, 0] == 1)
     assert np.all(rest[22 * 128:, 0] == 0)
     assert np.all(rest[22 * 128:, 4] <= sa_cap)
-    # snake deal: each rank exactly once, loads within one longest unit
-    G = 148
-    total = len(units)
-    owner = -np.ones(total, dtype=np.int64)
-    load = np.zeros(G, dtype=np.int64)
-    for c in range(G):
-        k = 0
-        while True:
-            r = k * G + ((G - 1 - c) if (k & 1) else c)
-            if r >= total:
-                break
-            assert owner[r] == -1
-            owner[r] = c
-            load[c] += cost[r]
-            k += 1
-    assert np.all(owner >= 0)
-    assert load.max() - load.min() <= cost.max()
+    for part in (long_fa, rest[: 22 * 128], rest[22 * 128:]):
+        _check_pairs_in_entry_order(part, [0])
+    # dynamic dispatch: the CTAs' finish times within 1% of the mean load
+    loads = _dynamic_loads(cost)
+    assert loads.max() <= (cost.sum() + 2.0 * len(units)) / 148 * 1.01
+
+
+@pytest.mark.parametrize("N,d", [(262144, 128), (131072, 128), (130817, 128), (130816, 128),
+                                 (65536, 128), (262144, 64), (261889, 64), (261888, 64)])
+def test_order_group_major_switch_and_dynamic_balance(N, d):
+    B, Hq, Hkv, S, W = 1, 32, 8, 128, 4096
+    mask = np.zeros((B, Hq), np.uint8)
+    mask[0, [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]] = 1
+    units = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, d, S, W))
+    gm = _group_major(N, d)
+    assert gm == (N > 130816 if d == 128 else N > 261888)
+    n0 = _check_order(units, Hq, Hkv, S, W, [0], gm)
+    first_groups = list(dict.fromkeys(int(h) // 4 for _, _, h, _, _ in units[:n0]))
+    if gm:
+        # FA heads 0, 3, 4, 6, 8, 10, 14, 16, 21, 27 lie in kv groups 0-6;
+        # group 7 (heads 28-31) is all SA
+        assert first_groups == list(range(7))
+        assert [int(h) for _, _, h, _, _ in units[:4]] == [0, 3, 0, 3]
+    else:
+        assert [int(h) for _, _, h, _, _ in units[:10]] == [0, 3, 4, 6, 8, 10, 14, 16, 21, 27]
+    cost = units[:, 4]
+    loads = _dynamic_loads(cost)
+    assert loads.max() <= (cost.sum() + 2.0 * len(units)) / 148 * 1.01
 
 
 @pytest.mark.parametrize("N,S,W", [(1, 0, 1), (77, 3, 5), (512, 16, 128), (300, 400, 2)])
@@ -222,8 +303,10 @@ def test_varlen_equal_lengths_schedule_like_the_padded_batch():
     np.testing.assert_array_equal(padded, packed)
 
 
-def test_varlen_order_longest_first_and_balance():
-    cu = np.cumsum([0, 32768, 1000, 9000, 300, 20000, 0, 4096]).tolist()
+@pytest.mark.parametrize("lens", [[32768, 1000, 9000, 300, 20000, 0, 4096],
+                                  [2000, 140000, 9000, 0, 131000, 700]])
+def test_varlen_order_longest_first_and_dynamic_balance(lens):
+    cu = np.cumsum([0] + lens).tolist()
     B, Hq, Hkv, d, S, W = len(cu) - 1, 32, 8, 128, 64, 1024
     rng = np.random.default_rng(11)
     mask = (rng.random((B, Hq)) < 0.7).astype(np.uint8)
@@ -231,22 +314,14 @@ def test_varlen_order_longest_first_and_balance():
     units = ea_schedule_units_varlen(mask, p, cu)
     _units_cover(units, cu, mask, 0)
     cost = units[:, 4]
-    sa_cap = int(np.ceil(S / 128)) + 2 + int(np.ceil((W - 1) / 128))
-    pA = sa_cap // 2
-    # long FA units first by pair, descending; then every SA unit; then short FA
-    nlong = int(np.sum((units[:, 0] == 0) & (units[:, 3] >= pA)))
-    assert np.all(units[:nlong, 0] == 0) and np.all(np.diff(units[:nlong, 3]) <= 0)
-    nsa = int(np.sum(units[:, 0] == 1))
-    assert np.all(units[nlong:nlong + nsa, 0] == 1)
-    assert np.all(units[nlong + nsa:, 0] == 0) and np.all(units[nlong + nsa:, 3] < pA)
-    # snake deal over 148 CTAs: loads within one longest unit
-    G = 148
-    load = np.zeros(G, np.int64)
-    for r in range(len(units)):
-        k = r // G
-        c = (r % G) if k % 2 == 0 else G - 1 - (r % G)
-        load[c] += cost[r]
-    assert load.max() - load.min() <= cost.max()
+    lens = np.diff(cu)
+    # sequences sorted by unit count, longest first, ties by index
+    pb = [-(-int(n) // 256) for n in lens]
+    seq_order = sorted(range(B), key=lambda b: (-pb[b], b))
+    _check_order(units, Hq, Hkv, S, W, seq_order, _group_major(int(lens.max()), d))
+    # dynamic dispatch over 148 CTAs: finish times within 1% of the mean load
+    loads = _dynamic_loads(cost)
+    assert loads.max() <= (cost.sum() + 2.0 * len(units)) / 148 * 1.01
 
 
 def test_varlen_schedule_rejects_inconsistent_offsets():
