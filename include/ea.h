@@ -514,7 +514,7 @@ ea_status ea_hybrid_attn_prefill_varlen_routed(const void* q, const void* k, con
 
 /* Host view of the packed batch's schedule, like ea_schedule_units below:
  * cu_seqlens_host is a HOST int32 [B+1] copy; units_out rows are
- * {sparse, b, h, pair, n_kv_tiles}.  Returns the unit count or -1. */
+ * {sparse, b, h0, h1, row0, n_kv_tiles}.  Returns the unit count or -1. */
 int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
                              const int32_t* cu_seqlens_host, int32_t* units_out, int max_units);
 
@@ -653,23 +653,27 @@ ea_status ea_hybrid_attn_prefill_host(const void* q_host, const void* k_host,
 
 /* ------------------------------------------------------------------------
  * Host-side view of the fused kernel's work schedule, for inspection and
- * tests (no GPU needed).  A unit is (mode, b, h, pair): 256 query rows
- * [256*pair, 256*pair + 256) of head h in batch b, run by one CTA.  Units
- * are ordered longest first; a CTA takes the next unit of that order from a
- * global counter whenever it starts one (the order is fixed, the CTA that
- * runs a unit is not).
+ * tests (no GPU needed).  A unit is two 128-row query slots run by one CTA
+ * over the same K/V tiles: a paired unit holds rows [row0, row0 + 128) of
+ * two query heads h0 != h1 of one kv group with the same route (the group's
+ * heads of that mode two by two, in head order); a single unit holds rows
+ * [row0, row0 + 256) of one head h0 (= h1), an odd one out of its group.
+ * Units are ordered longest first; a CTA takes the next unit of that order
+ * from a global counter whenever it starts one (the order is fixed, the CTA
+ * that runs a unit is not).
  *
  * mask        : host uint8 [B][Hq].
- * units_out   : host int32 [max_units][5] = {sparse, b, h, pair, n_kv_tiles}
- *               in schedule rank order (may be NULL to only count).
+ * units_out   : host int32 [max_units][6] = {sparse, b, h0, h1, row0,
+ *               n_kv_tiles} in schedule rank order (may be NULL to only
+ *               count).
  * Returns the number of units (>= 0), or -1 on invalid arguments.
  * ---------------------------------------------------------------------- */
 int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p,
                       int32_t* units_out, int max_units);
 
 /* The KV tiles (128 keys each) unit `rank` visits, in visiting order, and
- * per tile and query slot (slot 0: rows 256*pair..+127, slot 1: the next
- * 128) a code: 0 = skipped, 1 = every pair visible, 2 = needs the element
+ * per tile and query slot (slot 0: head h0 at rows row0..row0+127; slot 1:
+ * head h1 at the same rows, or, single, head h0 at the next 128) a code: 0 = skipped, 1 = every pair visible, 2 = needs the element
  * mask.  tiles_out: host int32 [max_tiles]; codes_out: host int32
  * [max_tiles][2].  Returns the tile count, or -1 on invalid arguments. */
 int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p,

@@ -763,26 +763,28 @@ def _host_mask(mask) -> np.ndarray:
 
 
 def ea_schedule_units(mask, p: EaAttnParams) -> np.ndarray:
-    """[U, 5] int32 rows (sparse, b, h, pair, n_kv_tiles) in schedule order."""
+    """[U, 6] int32 rows (sparse, b, h0, h1, row0, n_kv_tiles) in schedule order.
+    A paired unit (h1 != h0) holds rows [row0, row0 + 128) of heads h0 and h1;
+    a single unit (h1 == h0) rows [row0, row0 + 256) of head h0."""
     lib = _lib.load()
     m = _host_mask(mask)
     n = lib.ea_schedule_units(m.ctypes.data, ctypes.byref(p), None, 0)
     if n < 0:
         raise ValueError("invalid schedule arguments")
-    out = np.zeros((max(n, 1), 5), dtype=np.int32)
+    out = np.zeros((max(n, 1), 6), dtype=np.int32)
     lib.ea_schedule_units(m.ctypes.data, ctypes.byref(p), out.ctypes.data, n)
     return out[:n]
 
 
 def ea_schedule_units_varlen(mask, p: EaVarlenParams, cu_seqlens) -> np.ndarray:
-    """Schedule of a packed batch (cu_seqlens on the host): [U, 5] int32 rows."""
+    """Schedule of a packed batch (cu_seqlens on the host): [U, 6] int32 rows."""
     lib = _lib.load()
     m = _host_mask(mask)
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     n = lib.ea_schedule_units_varlen(m.ctypes.data, ctypes.byref(p), cu.ctypes.data, None, 0)
     if n < 0:
         raise ValueError("invalid schedule arguments")
-    out = np.zeros((max(n, 1), 5), dtype=np.int32)
+    out = np.zeros((max(n, 1), 6), dtype=np.int32)
     lib.ea_schedule_units_varlen(m.ctypes.data, ctypes.byref(p), cu.ctypes.data,
                                  out.ctypes.data, n)
     return out[:n]

@@ -182,54 +182,72 @@ bool encode_packed(CUtensorMap* m, const void* ptr, int d, int total, int heads)
 // Host copy of the kernel's sequence tables (EaSeqView): the schedule views
 // build exactly what the kernel's prologue builds.
 struct HostSched {
-  std::vector<int16_t> P;
-  std::vector<int32_t> prefFA, prefSA;
+  std::vector<int16_t> nT, P;
+  std::vector<int16_t> pref[4];
   std::vector<int> ent, len;
-  int nfa = 0, nsa = 0;
   EaSeqView view;
 };
 
-void build_host_sched(const uint8_t* mask, int B, int Hq, int select, const int* lens, int S,
-                      int W, HostSched& h) {
-  std::vector<int> order(B), pb(B);
-  for (int b = 0; b < B; ++b) {
-    order[b] = b;
-    pb[b] = ea_cdiv(lens[b], EA_UNIT_ROWS);
-  }
-  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return pb[x] > pb[y]; });
-  h.len.assign(lens, lens + B);
-  h.P.resize(B);
-  h.prefFA.assign(B + 1, 0);
-  h.prefSA.assign(B + 1, 0);
-  h.ent.clear();
-  for (int k = 0; k < B; ++k) {
-    h.P[k] = static_cast<int16_t>(pb[order[k]]);
-    h.prefFA[k] = static_cast<int32_t>(h.ent.size());
-    for (int hh = 0; hh < Hq; ++hh) {
-      const int idx = order[k] * Hq + hh;
-      if (!mask[idx] && select != EA_SELECT_SA) h.ent.push_back(idx);
+// The entry runs of one mode for sorted sequence b: per kv group, the
+// group's selected heads two by two (paired), an odd one out single; every
+// head single when a group has more than EA_MAX_PAIR_GROUP heads.
+static void host_entries(const uint8_t* mask, int b, int Hq, int Hkv, int select, int mode,
+                         std::vector<int>& paired, std::vector<int>& single) {
+  const int G = Hq / Hkv;
+  for (int hk = 0; hk < Hkv; ++hk) {
+    std::vector<int> heads;
+    for (int g = 0; g < G; ++g) {
+      const int idx = b * Hq + hk * G + g;
+      const bool sa = mask[idx] != 0;
+      if (sa == (mode == 1) && select != (mode == 1 ? EA_SELECT_FA : EA_SELECT_SA))
+        heads.push_back(idx);
     }
+    const int n = static_cast<int>(heads.size());
+    const int npair = G <= EA_MAX_PAIR_GROUP ? n / 2 : 0;
+    for (int i = 0; i < 2 * npair; ++i) paired.push_back(heads[i]);
+    for (int i = 2 * npair; i < n; ++i) single.push_back(heads[i]);
   }
-  h.nfa = static_cast<int>(h.ent.size());
-  h.prefFA[B] = h.nfa;
-  for (int k = 0; k < B; ++k) {
-    h.prefSA[k] = static_cast<int32_t>(h.ent.size()) - h.nfa;
-    for (int hh = 0; hh < Hq; ++hh) {
-      const int idx = order[k] * Hq + hh;
-      if (mask[idx] && select != EA_SELECT_FA) h.ent.push_back(idx);
-    }
-  }
-  h.nsa = static_cast<int>(h.ent.size()) - h.nfa;
-  h.prefSA[B] = h.nsa;
-  h.view.nseq = B;
-  h.view.P = h.P.data();
-  h.view.prefFA = h.prefFA.data();
-  h.view.prefSA = h.prefSA.data();
-  h.view.Pmax = B > 0 ? h.P[0] : 0;
-  h.view.pA = ea_split_pair(S, W, h.view.Pmax);
 }
 
-// Units of a schedule in rank order: {sparse, b, h, pair, n_kv_tiles}.
+void build_host_sched(const uint8_t* mask, int B, int Hq, int Hkv, int select, const int* lens,
+                      int S, int W, HostSched& h) {
+  std::vector<int> order(B), nb(B);
+  for (int b = 0; b < B; ++b) {
+    order[b] = b;
+    nb[b] = ea_cdiv(lens[b], EA_BN);
+  }
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return nb[x] > nb[y]; });
+  h.len.assign(lens, lens + B);
+  h.nT.resize(B);
+  h.P.resize(B);
+  std::vector<int> runs[4];
+  for (int j = 0; j < 4; ++j) h.pref[j].assign(B + 1, 0);
+  for (int k = 0; k < B; ++k) {
+    h.nT[k] = static_cast<int16_t>(nb[order[k]]);
+    h.P[k] = static_cast<int16_t>(ea_cdiv(nb[order[k]], 2));
+    for (int mode = 0; mode < 2; ++mode) {
+      h.pref[2 * mode][k] = static_cast<int16_t>(runs[2 * mode].size() / 2);
+      h.pref[2 * mode + 1][k] = static_cast<int16_t>(runs[2 * mode + 1].size());
+      host_entries(mask, order[k], Hq, Hkv, select, mode, runs[2 * mode], runs[2 * mode + 1]);
+    }
+  }
+  h.ent.clear();
+  for (int j = 0; j < 4; ++j) {
+    h.pref[j][B] = static_cast<int16_t>(j % 2 == 0 ? runs[j].size() / 2 : runs[j].size());
+    h.view.run0[j] = static_cast<int>(h.ent.size());
+    h.ent.insert(h.ent.end(), runs[j].begin(), runs[j].end());
+    h.view.pref[j] = h.pref[j].data();
+  }
+  h.view.nseq = B;
+  h.view.nT = h.nT.data();
+  h.view.P = h.P.data();
+  h.view.Pmax = B > 0 ? h.P[0] : 0;
+  h.view.mA = ea_long_level(S, W);
+}
+
+// Units of a schedule in rank order: {sparse, b, h0, h1, row0, n_kv_tiles}.
+// A paired unit (h1 != h0) holds rows [row0, row0 + 128) of both heads; a
+// single unit (h1 == h0) rows [row0, row0 + 256) of one head.
 int list_units(const HostSched& h, int Hq, int Hkv, int d, int S, int W, int32_t* units_out,
                int max_units) {
   const int total = ea_total_units(h.view);
@@ -237,17 +255,19 @@ int list_units(const HostSched& h, int Hq, int Hkv, int d, int S, int W, int32_t
     EaCursor cur;
     ea_cursor_init(cur, h.view, h.ent.data(), Hq, Hkv, ea_group_major(h.view.Pmax, d));
     for (int r = 0; r < total && r < max_units; ++r) {
-      int sparse = 0, e = 0, pair = 0;
-      if (!ea_cursor_seek(cur, h.view, h.ent.data(), r, &sparse, &e, &pair)) break;
-      const int idx = h.ent[sparse ? h.nfa + e : e];
+      EaUnitRef u;
+      if (!ea_cursor_seek(cur, h.view, h.ent.data(), r, &u)) break;
+      const int idx = h.ent[u.pos];
+      const int idx1 = u.paired ? h.ent[u.pos + 1] : idx;
       const EaShape sh = ea_make_shape(h.len[idx / Hq], S, W);
-      const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
-      int32_t* u = units_out + 5 * r;
-      u[0] = sparse;
-      u[1] = idx / Hq;
-      u[2] = idx % Hq;
-      u[3] = pair;
-      u[4] = ut.n;
+      const EaUnitTiles ut = ea_unit_tiles(sh, u.sparse, u.paired, u.level);
+      int32_t* o = units_out + 6 * r;
+      o[0] = u.sparse;
+      o[1] = idx / Hq;
+      o[2] = idx % Hq;
+      o[3] = idx1 % Hq;
+      o[4] = ut.r0;
+      o[5] = ut.n;
     }
   }
   return total;
@@ -985,7 +1005,7 @@ int ea_schedule_units(const uint8_t* mask, const ea_attn_params* p, int32_t* uni
   if (!mask || check_params(p) != EA_OK) return -1;
   std::vector<int> lens(p->B, p->N);
   HostSched h;
-  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  build_host_sched(mask, p->B, p->Hq, p->Hkv, p->select, lens.data(), p->sink, p->window, h);
   return list_units(h, p->Hq, p->Hkv, p->d, p->sink, p->window, units_out, max_units);
 }
 
@@ -999,7 +1019,7 @@ int ea_schedule_units_varlen(const uint8_t* mask, const ea_varlen_params* p,
     if (lens[b] < 0) return -1;
   }
   HostSched h;
-  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  build_host_sched(mask, p->B, p->Hq, p->Hkv, p->select, lens.data(), p->sink, p->window, h);
   return list_units(h, p->Hq, p->Hkv, p->d, p->sink, p->window, units_out, max_units);
 }
 
@@ -1008,21 +1028,21 @@ int ea_schedule_unit_tiles(const uint8_t* mask, const ea_attn_params* p, int ran
   if (!mask || check_params(p) != EA_OK) return -1;
   std::vector<int> lens(p->B, p->N);
   HostSched h;
-  build_host_sched(mask, p->B, p->Hq, p->select, lens.data(), p->sink, p->window, h);
+  build_host_sched(mask, p->B, p->Hq, p->Hkv, p->select, lens.data(), p->sink, p->window, h);
   const int total = ea_total_units(h.view);
   if (rank < 0 || rank >= total) return -1;
   EaCursor cur;
   ea_cursor_init(cur, h.view, h.ent.data(), p->Hq, p->Hkv, ea_group_major(h.view.Pmax, p->d));
-  int sparse = 0, e = 0, pair = 0;
-  if (!ea_cursor_seek(cur, h.view, h.ent.data(), rank, &sparse, &e, &pair)) return -1;
+  EaUnitRef u;
+  if (!ea_cursor_seek(cur, h.view, h.ent.data(), rank, &u)) return -1;
   const EaShape sh = ea_make_shape(p->N, p->sink, p->window);
-  const EaUnitTiles ut = ea_unit_tiles(sh, sparse, pair);
+  const EaUnitTiles ut = ea_unit_tiles(sh, u.sparse, u.paired, u.level);
   for (int i = 0; i < ut.n && i < max_tiles; ++i) {
     const int t = ea_tile_at(ut, i);
     if (tiles_out) tiles_out[i] = t;
     if (codes_out) {
-      codes_out[2 * i] = ea_tile_code(sh, ut, sparse, 0, t);
-      codes_out[2 * i + 1] = ea_tile_code(sh, ut, sparse, 1, t);
+      codes_out[2 * i] = ea_tile_code(sh, ut, u.sparse, 0, t);
+      codes_out[2 * i + 1] = ea_tile_code(sh, ut, u.sparse, 1, t);
     }
   }
   return ut.n;

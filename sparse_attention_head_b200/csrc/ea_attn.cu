@@ -79,17 +79,19 @@ struct AttnCfg {
   static constexpr int kUnitRing = 4;                       // units the producer runs ahead
   static constexpr int kNumBars = 3 + 2 * kStages + 10 + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, counts
-  static constexpr int kOffUnit = kOffMisc + 64;            // the unit ring: {rank, unit word}
+  static constexpr int kOffUnit = kOffMisc + 64;            // the unit ring: {rank, word, head}
   static constexpr int kOffEnt = kOffUnit + 64;
-  // sequence tables: token offset and length by index, order and unit count by
-  // sorted position, FA / SA entry prefix counts by sorted position
+  // sequence tables: token offset and length by index; order, block count and
+  // pair count by sorted position; the four entry runs' prefix counts by
+  // sorted position
   static constexpr int kOffTok = kOffEnt + EA_MAX_ENTRIES * 2;
   static constexpr int kOffLen = kOffTok + EA_MAX_SEQS * 4;
-  static constexpr int kOffPrefFA = kOffLen + EA_MAX_SEQS * 4;
-  static constexpr int kOffPrefSA = kOffPrefFA + (EA_MAX_SEQS + 1) * 4;
-  static constexpr int kOffOrder = kOffPrefSA + (EA_MAX_SEQS + 1) * 4;
+  static constexpr int kPrefLen = EA_MAX_SEQS + 2;          // int16 entries, even
+  static constexpr int kOffPref = kOffLen + EA_MAX_SEQS * 4;
+  static constexpr int kOffOrder = kOffPref + 4 * kPrefLen * 2;
   static constexpr int kOffP = kOffOrder + EA_MAX_SEQS * 2;
-  static constexpr int kSmem = kOffP + EA_MAX_SEQS * 2 + 1024;  // + alignment slack
+  static constexpr int kOffNT = kOffP + EA_MAX_SEQS * 2;
+  static constexpr int kSmem = kOffNT + EA_MAX_SEQS * 2 + 1024;  // + alignment slack
   static_assert(kSmem <= 232448, "shared memory per CTA");
   static constexpr uint32_t kIdescS =
       kFp8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
@@ -305,7 +307,6 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   }
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  int* s_counts = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // nFA, nSA
   // per-unit trace times of softmax warp 0 lane 0 (unit start, first S ready,
   // last P handed over): kept in shared memory, off the softmax registers
   uint64_t* s_trace_ts = reinterpret_cast<uint64_t*>(smem + C::kOffMisc + 32);
@@ -355,10 +356,10 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   // and records EA_ERR_INVALID_ARG.
   int32_t* s_tok = reinterpret_cast<int32_t*>(smem + C::kOffTok);
   int32_t* s_len = reinterpret_cast<int32_t*>(smem + C::kOffLen);
-  int32_t* s_prefFA = reinterpret_cast<int32_t*>(smem + C::kOffPrefFA);
-  int32_t* s_prefSA = reinterpret_cast<int32_t*>(smem + C::kOffPrefSA);
+  int16_t* s_pref = reinterpret_cast<int16_t*>(smem + C::kOffPref);   // [4][kPrefLen]
   int16_t* s_order = reinterpret_cast<int16_t*>(smem + C::kOffOrder);
   int16_t* s_P = reinterpret_cast<int16_t*>(smem + C::kOffP);
+  int16_t* s_nT = reinterpret_cast<int16_t*>(smem + C::kOffNT);
   const bool packed = args.cu_seqlens != nullptr;
   if (packed) {
     bool good = true;
@@ -381,59 +382,81 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
     }
   }
   __syncthreads();
-  // Sorted order: by unit count, longest first, ties by index (a padded batch
-  // keeps the identity order).
+  // Sorted order: by block count, longest first, ties by index (a padded
+  // batch keeps the identity order).
   for (int b = threadIdx.x; b < args.B; b += blockDim.x) {
-    const int pb = ea_cdiv(s_len[b], EA_UNIT_ROWS);
+    const int nb = ea_cdiv(s_len[b], EA_BN);
     int rank = b;
     if (packed) {
       rank = 0;
       for (int o = 0; o < args.B; ++o) {
-        const int po = ea_cdiv(s_len[o], EA_UNIT_ROWS);
-        rank += (po > pb) || (po == pb && o < b);
+        const int no = ea_cdiv(s_len[o], EA_BN);
+        rank += (no > nb) || (no == nb && o < b);
       }
     }
     s_order[rank] = static_cast<int16_t>(b);
-    s_P[rank] = static_cast<int16_t>(pb);
+    s_nT[rank] = static_cast<int16_t>(nb);
+    s_P[rank] = static_cast<int16_t>(ea_cdiv(nb, 2));
   }
   __syncthreads();
-  // Entry lists: FA heads first, then SA heads, filtered by args.select, each
-  // grouped by sorted sequence with heads in order.  Warp 0 builds them with
-  // ballots, and the prefix counts per sorted position with them.
+  // Entry runs (FA paired, FA single, SA paired, SA single), filtered by
+  // args.select and the shard, each grouped by sorted sequence, kv groups in
+  // order, heads increasing; a kv group's heads of one mode are paired two
+  // by two, an odd one out is single (all single when a group has more than
+  // EA_MAX_PAIR_GROUP heads).  Warp 0 builds them with ballots in two passes:
+  // the prefix counts, then the heads at their positions.
   if (warp == 0) {
-    int nfa = 0;
-    for (int k = 0; k < args.B; ++k) {
-      const int b = s_order[k];
-      if (lane == 0) s_prefFA[k] = nfa;
-      for (int h0 = 0; h0 < args.Hq; h0 += 32) {
-        const int h = h0 + lane;
-        const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) == 0) &&
-                        args.select != EA_SELECT_SA && in_shard(args, b, h);
-        const unsigned bits = __ballot_sync(0xffffffffu, ok);
-        if (ok) s_ent[nfa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
-        nfa += __popc(bits);
+    const int Gq = args.Hq / args.Hkv;
+    const bool pairing = Gq <= EA_MAX_PAIR_GROUP;
+    // a chunk of lanes covers whole kv groups when pairing
+    const int chunk = pairing ? (32 / Gq) * Gq : 32;
+    const int gl = pairing ? (lane / Gq) * Gq : 0;
+    const unsigned gmask =
+        pairing ? ((Gq == 32 ? 0xffffffffu : ((1u << Gq) - 1u)) << gl) : 0u;
+    const unsigned below = (1u << lane) - 1u;
+    int run0[4] = {0, 0, 0, 0};
+    for (int pass = 0; pass < 2; ++pass) {
+      int cnt[4] = {0, 0, 0, 0};   // heads written to each run so far
+      for (int k = 0; k < args.B; ++k) {
+        const int b = s_order[k];
+#pragma unroll
+        for (int mode = 0; mode < 2; ++mode) {
+          if (pass == 0 && lane == 0) {
+            s_pref[(2 * mode) * C::kPrefLen + k] = static_cast<int16_t>(cnt[2 * mode] / 2);
+            s_pref[(2 * mode + 1) * C::kPrefLen + k] = static_cast<int16_t>(cnt[2 * mode + 1]);
+          }
+          for (int h0 = 0; h0 < args.Hq; h0 += chunk) {
+            const int h = h0 + lane;
+            const int idx = b * args.Hq + h;
+            const bool ok = lane < chunk && h < args.Hq &&
+                            (args.both || (ld_mask(args.mask, idx) != 0) == (mode == 1)) &&
+                            args.select != (mode == 1 ? EA_SELECT_FA : EA_SELECT_SA) &&
+                            in_shard(args, b, h);
+            const unsigned bits = __ballot_sync(0xffffffffu, ok);
+            const int rank = __popc(bits & gmask & below);
+            const int n = __popc(bits & gmask);
+            const bool pr = ok && pairing && rank < (n & ~1);
+            const unsigned pbits = __ballot_sync(0xffffffffu, pr);
+            const unsigned sbits = __ballot_sync(0xffffffffu, ok && !pr);
+            if (pass == 1 && ok) {
+              const int pos = pr ? run0[2 * mode] + cnt[2 * mode] + __popc(pbits & below)
+                                 : run0[2 * mode + 1] + cnt[2 * mode + 1] + __popc(sbits & below);
+              s_ent[pos] = static_cast<uint16_t>(idx);
+            }
+            cnt[2 * mode] += __popc(pbits);
+            cnt[2 * mode + 1] += __popc(sbits);
+          }
+        }
       }
-    }
-    int nsa = 0;
-    for (int k = 0; k < args.B; ++k) {
-      const int b = s_order[k];
-      if (lane == 0) s_prefSA[k] = nsa;
-      for (int h0 = 0; h0 < args.Hq; h0 += 32) {
-        const int h = h0 + lane;
-        const int idx = b * args.Hq + h;
-        const bool ok = h < args.Hq && (args.both || ld_mask(args.mask, idx) != 0) &&
-                        args.select != EA_SELECT_FA && in_shard(args, b, h);
-        const unsigned bits = __ballot_sync(0xffffffffu, ok);
-        if (ok) s_ent[nfa + nsa + __popc(bits & ((1u << lane) - 1u))] = static_cast<uint16_t>(idx);
-        nsa += __popc(bits);
+      if (pass == 0) {
+        if (lane == 0)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            s_pref[j * C::kPrefLen + args.B] = static_cast<int16_t>(j % 2 == 0 ? cnt[j] / 2 : cnt[j]);
+        run0[1] = cnt[0];
+        run0[2] = run0[1] + cnt[1];
+        run0[3] = run0[2] + cnt[2];
       }
-    }
-    if (lane == 0) {
-      s_prefFA[args.B] = nfa;
-      s_prefSA[args.B] = nsa;
-      s_counts[0] = nfa;
-      s_counts[1] = nsa;
     }
   }
   tc_fence_before();
@@ -441,14 +464,18 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
   tc_fence_after();
 
   const uint32_t tmem = *s_tmem;
-  const int nFA = s_counts[0];
   EaSeqView view;
   view.nseq = args.B;
+  view.nT = s_nT;
   view.P = s_P;
-  view.prefFA = s_prefFA;
-  view.prefSA = s_prefSA;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) view.pref[j] = s_pref + j * C::kPrefLen;
+  view.run0[0] = 0;
+  view.run0[1] = 2 * view.pref[0][args.B];
+  view.run0[2] = view.run0[1] + view.pref[1][args.B];
+  view.run0[3] = view.run0[2] + 2 * view.pref[2][args.B];
   view.Pmax = args.B > 0 ? s_P[0] : 0;
-  view.pA = ea_split_pair(args.sink, args.window, view.Pmax);
+  view.mA = ea_long_level(args.sink, args.window);
   const int total = ea_total_units(view);
   const int G = args.Hq / args.Hkv;
   const uint64_t tlim = args.timeout_ns;
@@ -481,34 +508,40 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         }
         const unsigned int ticket = next_ticket;
         const int r = ticket < static_cast<unsigned int>(total) ? static_cast<int>(ticket) : -1;
-        int sparse = 0, e = 0, pair = 0;
-        if (r >= 0) ea_cursor_seek(cur, view, s_ent, r, &sparse, &e, &pair);
-        const int idx = r >= 0 ? static_cast<int>(s_ent[sparse ? nFA + e : e]) : 0;
+        EaUnitRef u = {0, 0, 0, 0};
+        if (r >= 0) ea_cursor_seek(cur, view, s_ent, r, &u);
+        const int idx = r >= 0 ? static_cast<int>(s_ent[u.pos]) : 0;
+        const int idx1 = (r >= 0 && u.paired) ? static_cast<int>(s_ent[u.pos + 1]) : idx;
         // Only this thread runs the cursor: the other roles read the unit
-        // decoded, {rank, pair << 13 | sparse << 12 | entry} (an entry index
-        // is below 4096, a pair below 32768).
-        s_unit[2 * us] = r;
-        s_unit[2 * us + 1] = (pair << 13) | (sparse << 12) | idx;
+        // decoded, {rank, level << 14 | paired << 13 | sparse << 12 | head
+        // of slot 0, head of slot 1} (a head index is below 4096, a level
+        // below 65536).
+        s_unit[4 * us] = r;
+        s_unit[4 * us + 1] = (u.level << 14) | (u.paired << 13) | (u.sparse << 12) | idx;
+        s_unit[4 * us + 2] = idx1;
         mbar_arrive(bars.unit_full + 8 * us);
         if (r < 0) break;
         next_ticket = atomicAdd(args.ticket, 1u);
+        const int sparse = u.sparse;
         const int b = idx / args.Hq, h = idx % args.Hq;
         // tensor coordinates: padded batch (row, head index b*H + h); packed
-        // batch (token, head)
+        // batch (token, head); both heads of a paired unit read kv head h / G
         const int tok = s_tok[b];
-        const int qz = packed ? h : idx;
         const int kvz = packed ? h / G : b * args.Hkv + h / G;
         const EaShape shape = ea_make_shape(s_len[b], args.sink, args.window);
-        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, u.paired, u.level);
         if (n_units > 0) {
           ok = mbar_wait(bars.q_empty, (n_units - 1) & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
           if (!ok) break;
         }
         mbar_arrive_expect_tx(bars.q_full, ut.nslots * C::kTileBytes);
-        for (int s = 0; s < ut.nslots; ++s)
+        for (int s = 0; s < ut.nslots; ++s) {
+          const int qidx = s ? idx1 : idx;
+          const int qz = packed ? qidx % args.Hq : qidx;
           for (int c = 0; c < C::kDBlocks; ++c)
             tma_load_3d(smem_u32(sQ) + s * C::kTileBytes + c * C::kBlockBytes, &args.tm_q, bars.q_full,
-                        c * C::kBlockElems, tok + ut.r0 + s * EA_BM, qz);
+                        c * C::kBlockElems, tok + ut.r0 + s * ut.rstep, qz);
+        }
         ++n_units;
         for (int i = 0; i < ut.n && ok; ++i) {
           const int t = ea_tile_at(ut, i);
@@ -605,14 +638,14 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         ok = mbar_wait(bars.unit_full + 8 * us, (kk / C::kUnitRing) & 1, s_abort, status, tlim,
                        EA_ERR_TIMEOUT);
         if (!ok) break;
-        const int r = s_unit[2 * us];
-        const int word = s_unit[2 * us + 1];
+        const int r = s_unit[4 * us];
+        const int word = s_unit[4 * us + 1];
         __syncwarp();
         if (leader) mbar_arrive(bars.unit_empty + 8 * us);
         if (r < 0) break;
-        const int sparse = (word >> 12) & 1, pair = word >> 13, idx = word & 4095;
+        const int sparse = (word >> 12) & 1, idx = word & 4095;
         const EaShape shape = ea_make_shape(s_len[idx / args.Hq], args.sink, args.window);
-        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+        const EaUnitTiles ut = ea_unit_tiles(shape, sparse, (word >> 13) & 1, word >> 14);
 
         ok = mbar_wait(bars.q_full, n_units & 1, s_abort, status, tlim, EA_ERR_TIMEOUT);
         if (!ok) break;
@@ -714,16 +747,18 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                      EA_ERR_TIMEOUT);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const int r = s_unit[2 * us];
-      const int word = s_unit[2 * us + 1];
+      const int r = s_unit[4 * us];
+      const int word = s_unit[4 * us + 1];
+      const int idx1 = s_unit[4 * us + 2];
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.unit_empty + 8 * us);
       if (r < 0) break;
-      const int sparse = (word >> 12) & 1, pair = word >> 13, idx = word & 4095;
+      const int sparse = (word >> 12) & 1;
+      const int idx = slot ? idx1 : (word & 4095);   // this slot's head
       const int seq = idx / args.Hq;
       const int seq_len = s_len[seq];
       const EaShape shape = ea_make_shape(seq_len, args.sink, args.window);
-      const EaUnitTiles ut = ea_unit_tiles(shape, sparse, pair);
+      const EaUnitTiles ut = ea_unit_tiles(shape, sparse, (word >> 13) & 1, word >> 14);
       if (slot >= ut.nslots) continue;
       const bool tracing = kTrace && warp == 0 && lane == 0;
       if (tracing) {
@@ -731,7 +766,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         s_trace_ts[1] = 0;
         s_trace_ts[2] = 0;
       }
-      const int row = ut.r0 + slot * EA_BM + row_local;   // global query row
+      const int row = ut.r0 + slot * ut.rstep + row_local;   // global query row
       // FP8: the scores carry the q and k dequantization scales
       const int kvh = seq * args.Hkv + (idx % args.Hq) / G;
       const float sl2 = kFp8 ? args.scale_log2 * args.q_scale[idx] * args.k_scale[kvh]

@@ -43,7 +43,7 @@ def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
     torch.cuda.synchronize()
     assert ea_get_device_status(ws) == 0
     assert torch.equal(plain, traced)
-    units = ea_schedule_units(m, p)                 # rows: sparse, b, h, pair, n_kv_tiles
+    units = ea_schedule_units(m, p)       # rows: sparse, b, h0, h1, row0, n_kv_tiles
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     grid = ea_attn_grid_size(p, sms)
     assert total == len(units) == len(rec)
@@ -58,7 +58,7 @@ def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
     assert np.all(first_s >= start) and np.all(last_p >= first_s) and np.all(end >= last_p)
     assert set(np.unique(cta).tolist()) <= set(range(grid))
     np.testing.assert_array_equal(sparse, units[rank, 0])
-    np.testing.assert_array_equal(tiles, units[rank, 4])
+    np.testing.assert_array_equal(tiles, units[rank, 5])
     # a CTA runs its units one after another, in the increasing rank order of
     # its tickets
     for c in np.unique(cta):

@@ -1,10 +1,14 @@
 """Host logic of the fused kernel's schedule (no GPU): every selected
-(b, h, query row) is covered by exactly one unit slot, every tile a slot
-needs is visited with the right masking code, units are ordered longest
-first (at one pair, the entries in (sorted sequence, head) order, so a kv
-group's heads are adjacent; for long sequences the long FA units kv group by
-kv group), and dynamic dispatch of that order over 148 CTAs balances their
-loads."""
+(b, h, query row) is covered by exactly one unit slot; a kv group's heads of
+one mode are paired two by two in head order (an odd one out runs single);
+every tile a slot needs is visited with the right masking code; units are
+ordered longest first (level descending; at one level the paired units, then
+the single ones, entries in (sorted sequence, head) order; for long sequences
+the long FA units kv group by kv group); and dynamic dispatch of that order
+over 148 CTAs balances their loads.
+
+Unit rows are (sparse, b, h0, h1, row0, n_kv_tiles): paired (h1 != h0) rows
+[row0, row0 + 128) of both heads; single (h1 == h0) rows [row0, row0 + 256)."""
 import numpy as np
 import pytest
 
@@ -32,6 +36,65 @@ def brute_codes(N, sparse, S, W, r0, tile):
     return 1 if all_vis else 2
 
 
+def _slots(unit):
+    """[(head, first row)] of a unit's two slots."""
+    _, _, h0, h1, row0, _ = (int(x) for x in unit)
+    return [(h0, row0), (h1, row0)] if h1 != h0 else [(h0, row0), (h0, row0 + 128)]
+
+
+def _level(unit):
+    """The unit's level m: a paired unit's block; 2p + 1 for a single unit of pair p."""
+    _, _, h0, h1, row0, _ = (int(x) for x in unit)
+    return row0 // 128 if h1 != h0 else 2 * (row0 // 256) + 1
+
+
+def _expected_pairing(mask, Hq, Hkv, sel):
+    """{(mode, b, h0, h1)}: per (b, kv group, mode) the selected heads in order,
+    two by two; an odd one out as (mode, b, h, h)."""
+    B = mask.shape[0]
+    G = Hq // Hkv
+    want = set()
+    for b in range(B):
+        for hk in range(Hkv):
+            for mode in (0, 1):
+                if sel == 1 and mode == 1 or sel == 2 and mode == 0:
+                    continue
+                heads = [hk * G + g for g in range(G) if int(mask[b, hk * G + g] != 0) == mode]
+                npair = len(heads) // 2 if G <= 32 else 0
+                for i in range(npair):
+                    want.add((mode, b, heads[2 * i], heads[2 * i + 1]))
+                for h in heads[2 * npair:]:
+                    want.add((mode, b, h, h))
+    return want
+
+
+def _check_cover(units, lens, mask, Hq, Hkv, sel):
+    """Every selected (b, h, row) in exactly one slot; the units' head pairs
+    are the pairing rule's."""
+    B = mask.shape[0]
+    covered = [np.zeros((Hq, n), np.int32) for n in lens]
+    pairs = set()
+    for u in units:
+        sparse, b = int(u[0]), int(u[1])
+        h0, h1 = int(u[2]), int(u[3])
+        assert sel == 0 or (sel == 1 and not sparse) or (sel == 2 and sparse)
+        assert h0 // (Hq // Hkv) == h1 // (Hq // Hkv)
+        pairs.add((sparse, b, h0, h1))
+        for h, r0 in _slots(u):
+            assert sparse == int(mask[b, h] != 0)
+            assert r0 < lens[b] or h1 == h0
+            if r0 < lens[b]:
+                covered[b][h, r0:min(lens[b], r0 + 128)] += 1
+    for b in range(B):
+        for h in range(Hq):
+            selected = sel == 0 or (sel == 1) == (mask[b, h] == 0)
+            assert np.all(covered[b][h] == (1 if selected else 0)), (b, h)
+    want = _expected_pairing(mask, Hq, Hkv, sel)
+    if any(n > 0 for n in lens):
+        present = {(m, b, h0, h1) for (m, b, h0, h1) in want if lens[b] > 0}
+        assert pairs == present
+
+
 CASES = [
     # B, Hq, Hkv, N, d, S, W, select
     (1, 4, 2, 512, 64, 16, 128, 0),
@@ -42,6 +105,8 @@ CASES = [
     (1, 4, 2, 640, 64, 1, 129, 1),
     (1, 4, 2, 640, 64, 1, 129, 2),
     (2, 6, 3, 257, 64, 300, 5, 0),
+    (1, 12, 2, 385, 64, 16, 100, 0),
+    (2, 8, 1, 129, 128, 0, 64, 0),
 ]
 
 
@@ -51,17 +116,16 @@ def test_units_cover_rows_once(B, Hq, Hkv, N, d, S, W, sel):
     mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
     p = make_params(B, Hq, Hkv, N, d, S, W, select=sel)
     units = ea_schedule_units(mask, p)
-    covered = np.zeros((B, Hq, N), dtype=np.int32)
-    for sparse, b, h, pair, ntiles in units:
-        assert sparse == mask[b, h]
-        assert sel == 0 or (sel == 1 and not sparse) or (sel == 2 and sparse)
-        r0 = 256 * pair
-        covered[b, h, r0:min(N, r0 + 256)] += 1
-    for b in range(B):
-        for h in range(Hq):
-            selected = sel == 0 or (sel == 1) == (mask[b, h] == 0)
-            want = 1 if selected else 0
-            assert np.all(covered[b, h] == want)
+    _check_cover(units, [N] * B, mask, Hq, Hkv, sel)
+
+
+def test_pairing_with_more_than_32_heads_per_group_is_single():
+    B, Hq, Hkv, N = 1, 64, 1, 300
+    mask = np.zeros((B, Hq), np.uint8)
+    mask[0, ::3] = 1
+    units = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, 64, 4, 64))
+    assert np.all(units[:, 2] == units[:, 3])
+    _check_cover(units, [N], mask, Hq, Hkv, 0)
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,d,S,W,sel", CASES)
@@ -72,17 +136,16 @@ def test_unit_tiles_match_definition(B, Hq, Hkv, N, d, S, W, sel):
     units = ea_schedule_units(mask, p)
     ntiles_total = (N + 127) // 128
     seen_kinds = set()
-    for rank, (sparse, b, h, pair, n) in enumerate(units):
-        key = (sparse, pair)
+    for rank, u in enumerate(units):
+        sparse, n = int(u[0]), int(u[5])
+        key = (sparse, int(u[2]) != int(u[3]), int(u[4]))
         if key in seen_kinds:
             continue
         seen_kinds.add(key)
         tiles, codes = ea_schedule_unit_tiles(mask, p, rank)
         assert len(tiles) == n
         assert len(set(tiles.tolist())) == n and list(tiles) == sorted(tiles)
-        r0 = 256 * pair
-        for slot in range(2):
-            rs = r0 + 128 * slot
+        for slot, (_, rs) in enumerate(_slots(u)):
             for t in range(ntiles_total):
                 want = brute_codes(N, bool(sparse), S, W, rs, t) if rs < N else 0
                 if t in tiles:
@@ -106,11 +169,11 @@ def _dynamic_loads(cost, ctas=148):
     return np.array([t for t, _ in heap])
 
 
-def _check_pairs_in_entry_order(units, seq_order):
-    """Inside each run of one mode, pair descending; at one pair, the entries
-    in (sorted sequence, head) order."""
+def _check_levels_in_entry_order(units, seq_order):
+    """Inside a run of one mode: level descending; at one level the paired
+    units, then the single ones, each in (sorted sequence, head) order."""
     pos = {b: i for i, b in enumerate(seq_order)}
-    key = [(-int(pair), pos[int(b)], int(h)) for _, b, h, pair, _ in units]
+    key = [(-_level(u), int(u[2]) == int(u[3]), pos[int(u[1])], int(u[2])) for u in units]
     assert key == sorted(key)
 
 
@@ -121,24 +184,30 @@ def _group_major(n_max, d):
     return 2 * (-(-n_max // 256) * 256) * d >= 2 * 131072 * 128
 
 
+def _long_level(S, W):
+    """Levels from which an FA unit is longer than any SA unit."""
+    return -(-S // 128) + 2 + -(-(W - 1) // 128)
+
+
 def _check_order(units, Hq, Hkv, S, W, seq_order, group_major):
-    """The order's rules from the unit list alone: the long FA units (pair >=
-    pA, longer than any SA unit) first, then every SA unit, then the short FA
-    units.  Group-major, the long FA units of one (b, kv group) are
+    """The order's rules from the unit list alone: the long FA units (level
+    >= mA, longer than any SA unit) first, then every SA unit, then the short
+    FA units.  Group-major, the long FA units of one (b, kv group) are
     consecutive, the groups in (sorted sequence, kv head) order, inside a
-    group pair descending with heads ascending; otherwise, like the other two
-    runs, pair descending with the entries of one pair in (sorted sequence,
-    head) order.  Returns the number of long FA units."""
+    group level descending (paired before single, heads ascending);
+    otherwise, like the other two runs, level descending with the units of
+    one level in (paired first, sorted sequence, head) order.  Returns the
+    number of long FA units."""
     G = Hq // Hkv
-    pA = (-(-S // 128) + 2 + -(-(W - 1) // 128)) // 2
+    mA = _long_level(S, W)
     pos = {b: i for i, b in enumerate(seq_order)}
-    long_fa = (units[:, 0] == 0) & (units[:, 3] >= pA)
+    long_fa = np.array([int(u[0]) == 0 and _level(u) >= mA for u in units], dtype=bool)
     n0 = int(long_fa.sum())
     assert np.all(long_fa[:n0]) and not np.any(long_fa[n0:])
     if group_major:
         runs = []
-        for i, (_, b, h, _, _) in enumerate(units[:n0]):
-            key = (int(b), int(h) // G)
+        for i, u in enumerate(units[:n0]):
+            key = (int(u[1]), int(u[2]) // G)
             if not runs or runs[-1][0] != key:
                 runs.append([key, i, i + 1])
             else:
@@ -147,42 +216,45 @@ def _check_order(units, Hq, Hkv, S, W, seq_order, group_major):
         order = [(pos[b], hk) for (b, hk), _, _ in runs]
         assert order == sorted(order)
         for _, a, e in runs:
-            key = [(-int(pair), int(h)) for _, _, h, pair, _ in units[a:e]]
+            key = [(-_level(u), int(u[2]) == int(u[3]), int(u[2])) for u in units[a:e]]
             assert key == sorted(key)
     else:
-        _check_pairs_in_entry_order(units[:n0], seq_order)
+        _check_levels_in_entry_order(units[:n0], seq_order)
     rest = units[n0:]
     nsa = int(np.sum(rest[:, 0] == 1))
     assert np.all(rest[:nsa, 0] == 1) and np.all(rest[nsa:, 0] == 0)
-    _check_pairs_in_entry_order(rest[:nsa], seq_order)
-    _check_pairs_in_entry_order(rest[nsa:], seq_order)
+    _check_levels_in_entry_order(rest[:nsa], seq_order)
+    _check_levels_in_entry_order(rest[nsa:], seq_order)
     return n0
+
+
+_MASK22 = [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]
 
 
 def test_order_longest_first_and_dynamic_balance():
     B, Hq, Hkv, N, d, S, W = 1, 32, 8, 32768, 128, 64, 1024
     mask = np.zeros((B, Hq), np.uint8)
-    mask[0, [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]] = 1
-    p = make_params(B, Hq, Hkv, N, d, S, W)
-    units = ea_schedule_units(mask, p)
-    cost = units[:, 4]
+    mask[0, _MASK22] = 1
+    units = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, d, S, W))
+    n0 = _check_order(units, Hq, Hkv, S, W, [0], False)
+    # FA heads by kv group: {0, 3} {4, 6} {8, 10} {14} {16} {21} {27}: 3 pairs
+    # and 4 singles; SA: {1, 2} {5, 7} {9, 11} {12, 13} {15} {17, 18} {19}
+    # {20, 22} {23} {24, 25} {26} {28, 29} {30, 31}: 9 pairs, 4 singles
+    assert len(units) == 3 * 256 + 4 * 128 + 9 * 256 + 4 * 128
+    mA = _long_level(S, W)
+    # single units at odd levels 2p + 1 >= mA: p >= mA // 2
+    assert n0 == 3 * (256 - mA) + 4 * (128 - mA // 2)
+    # the top level (255, odd): the three FA pairs, then the four FA singles
+    top = [(int(u[2]), int(u[3]), int(u[4])) for u in units[:7]]
+    assert top == [(0, 3, 255 * 128), (4, 6, 255 * 128), (8, 10, 255 * 128),
+                   (14, 14, 127 * 256), (16, 16, 127 * 256), (21, 21, 127 * 256),
+                   (27, 27, 127 * 256)]
+    # the next level (254): the pairs only
+    assert [(int(u[2]), int(u[4])) for u in units[7:10]] == [(0, 254 * 128), (4, 254 * 128),
+                                                             (8, 254 * 128)]
+    cost = units[:, 5]
     sa_cap = max(cost[units[:, 0] == 1])
-    nfa = int((mask == 0).sum())
-    # long FA units first, strictly non-increasing
-    long_fa = units[: nfa * (128 - sa_cap // 2)]
-    assert np.all(long_fa[:, 0] == 0)
-    assert np.all(np.diff(long_fa[:, 4]) <= 0)
-    assert np.all(long_fa[:, 4] > sa_cap)
-    # the first pair: every FA head, kv groups in order
-    assert [int(h) for _, _, h, _, _ in units[:nfa]] == [0, 3, 4, 6, 8, 10, 14, 16, 21, 27]
-    # then SA units, then the short FA units
-    rest = units[len(long_fa):]
-    assert np.all(rest[: 22 * 128, 0] == 1)
-    assert np.all(rest[22 * 128:, 0] == 0)
-    assert np.all(rest[22 * 128:, 4] <= sa_cap)
-    for part in (long_fa, rest[: 22 * 128], rest[22 * 128:]):
-        _check_pairs_in_entry_order(part, [0])
-    # dynamic dispatch: the CTAs' finish times within 1% of the mean load
+    assert np.all(cost[:n0] > sa_cap - 1)
     loads = _dynamic_loads(cost)
     assert loads.max() <= (cost.sum() + 2.0 * len(units)) / 148 * 1.01
 
@@ -192,20 +264,20 @@ def test_order_longest_first_and_dynamic_balance():
 def test_order_group_major_switch_and_dynamic_balance(N, d):
     B, Hq, Hkv, S, W = 1, 32, 8, 128, 4096
     mask = np.zeros((B, Hq), np.uint8)
-    mask[0, [1, 2, 5, 7, 9, 11, 12, 13, 15, 17, 18, 19, 20, 22, 23, 24, 25, 26, 28, 29, 30, 31]] = 1
+    mask[0, _MASK22] = 1
     units = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, d, S, W))
     gm = _group_major(N, d)
     assert gm == (N > 130816 if d == 128 else N > 261888)
     n0 = _check_order(units, Hq, Hkv, S, W, [0], gm)
-    first_groups = list(dict.fromkeys(int(h) // 4 for _, _, h, _, _ in units[:n0]))
+    first_groups = list(dict.fromkeys(int(u[2]) // 4 for u in units[:n0]))
     if gm:
-        # FA heads 0, 3, 4, 6, 8, 10, 14, 16, 21, 27 lie in kv groups 0-6;
-        # group 7 (heads 28-31) is all SA
+        # FA heads lie in kv groups 0-6; group 7 (heads 28-31) is all SA
         assert first_groups == list(range(7))
-        assert [int(h) for _, _, h, _, _ in units[:4]] == [0, 3, 0, 3]
+        # group 0: the pair (0, 3) at every level, nothing single
+        assert [(int(u[2]), int(u[3])) for u in units[:3]] == [(0, 3)] * 3
     else:
-        assert [int(h) for _, _, h, _, _ in units[:10]] == [0, 3, 4, 6, 8, 10, 14, 16, 21, 27]
-    cost = units[:, 4]
+        assert [int(u[2]) for u in units[:7]] == [0, 4, 8, 14, 16, 21, 27]
+    cost = units[:, 5]
     loads = _dynamic_loads(cost)
     assert loads.max() <= (cost.sum() + 2.0 * len(units)) / 148 * 1.01
 
@@ -257,23 +329,12 @@ VARLEN_CASES = [
     ([0, 700, 900, 2000], 4, 2, 128, 130, 200, 1),
     ([0, 700, 900, 2000], 4, 2, 128, 130, 200, 2),
     ([0, 0, 0, 129], 2, 1, 64, 5, 3, 0),
+    ([0, 129, 385, 386, 900], 8, 2, 64, 8, 200, 0),
 ]
 
 
-def _units_cover(units, cu, mask, sel):
-    B, Hq = mask.shape
-    lens = np.diff(cu)
-    covered = [np.zeros((Hq, n), np.int32) for n in lens]
-    for sparse, b, h, pair, ntiles in units:
-        assert sparse == mask[b, h]
-        assert sel == 0 or (sel == 1 and not sparse) or (sel == 2 and sparse)
-        r0 = 256 * pair
-        assert r0 < lens[b]
-        covered[b][h, r0:min(lens[b], r0 + 256)] += 1
-    for b in range(B):
-        for h in range(Hq):
-            selected = sel == 0 or (sel == 1) == (mask[b, h] == 0)
-            assert np.all(covered[b][h] == (1 if selected else 0)), (b, h)
+def _units_cover(units, cu, mask, sel, Hkv):
+    _check_cover(units, list(np.diff(cu)), mask, mask.shape[1], Hkv, sel)
 
 
 @pytest.mark.parametrize("cu,Hq,Hkv,d,S,W,sel", VARLEN_CASES)
@@ -283,14 +344,15 @@ def test_varlen_units_cover_rows_once(cu, Hq, Hkv, d, S, W, sel):
     mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
     p = make_varlen_params(B, Hq, Hkv, cu[-1], max(np.diff(cu)), d, S, W, select=sel)
     units = ea_schedule_units_varlen(mask, p, cu)
-    _units_cover(units, cu, mask, sel)
+    _units_cover(units, cu, mask, sel, Hkv)
     # each unit's tile count is that of its own sequence's shape
-    for sparse, b, h, pair, n in units:
+    for u in units:
+        sparse, b, n = int(u[0]), int(u[1]), int(u[5])
         N_b = cu[b + 1] - cu[b]
         tiles = [t for t in range((N_b + 127) // 128)
-                 if any(brute_codes(N_b, bool(sparse), S, W, 256 * pair + 128 * s, t)
-                        for s in range(2) if 256 * pair + 128 * s < N_b)]
-        assert n == len(tiles), (b, pair, n, tiles)
+                 if any(brute_codes(N_b, bool(sparse), S, W, rs, t)
+                        for _, rs in _slots(u) if rs < N_b)]
+        assert n == len(tiles), (b, int(u[4]), n, tiles)
 
 
 def test_varlen_equal_lengths_schedule_like_the_padded_batch():
@@ -312,12 +374,12 @@ def test_varlen_order_longest_first_and_dynamic_balance(lens):
     mask = (rng.random((B, Hq)) < 0.7).astype(np.uint8)
     p = make_varlen_params(B, Hq, Hkv, cu[-1], max(np.diff(cu)), d, S, W)
     units = ea_schedule_units_varlen(mask, p, cu)
-    _units_cover(units, cu, mask, 0)
-    cost = units[:, 4]
+    _units_cover(units, cu, mask, 0, Hkv)
+    cost = units[:, 5]
     lens = np.diff(cu)
-    # sequences sorted by unit count, longest first, ties by index
-    pb = [-(-int(n) // 256) for n in lens]
-    seq_order = sorted(range(B), key=lambda b: (-pb[b], b))
+    # sequences sorted by 128-row block count, longest first, ties by index
+    nb = [-(-int(n) // 128) for n in lens]
+    seq_order = sorted(range(B), key=lambda b: (-nb[b], b))
     _check_order(units, Hq, Hkv, S, W, seq_order, _group_major(int(lens.max()), d))
     # dynamic dispatch over 148 CTAs: finish times within 1% of the mean load
     loads = _dynamic_loads(cost)
