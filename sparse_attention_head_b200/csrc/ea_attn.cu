@@ -232,6 +232,12 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
   return grid_sync(args, s_flag, 3);
 }
 
+// Bits [0, n) of a 32-bit word (n clamped to [0, 32]).
+__device__ __forceinline__ uint32_t bits_below(int n) {
+  n = n < 0 ? 0 : n;
+  return n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+}
+
 // One row's probabilities p = 2^(x * sl2 - msub) over keys [32 C0, 32 C1)
 // of a 128-key tile:
 // packed FMA, then exp2 on the MUFU for most pairs and on the FMA pipe for
@@ -767,6 +773,13 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         s_trace_ts[2] = 0;
       }
       const int row = ut.r0 + slot * ut.rstep + row_local;   // global query row
+      // does some row of this slot see fewer than 128 keys?  (the count of
+      // visible keys grows with the row, so the slot's first row decides)
+      const int r0s = ut.r0 + slot * ut.rstep;
+      const int keys0 = sparse ? ea_min(r0s + 1, args.window) +
+                                     ea_min(args.sink, ea_max(0, r0s - args.window + 1))
+                               : r0s + 1;
+      const bool few_keys = keys0 < 128;
       // FP8: the scores carry the q and k dequantization scales
       const int kvh = seq * args.Hkv + (idx % args.Hq) / G;
       const float sl2 = kFp8 ? args.scale_log2 * args.q_scale[idx] * args.k_scale[kvh]
@@ -794,15 +807,19 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         if (code == 2) {
           const int c0 = t * EA_BN;
           // visible key j (local): j <= row - c0, and for SA also
-          // (j < sink - c0 || j >= row - window + 1 - c0)
+          // (j < sink - c0 || j >= row - window + 1 - c0); built as a
+          // 128-bit mask, four words of intervals, then one bit test per key
           const int lim = row - c0;
           const int sink_hi = sparse ? args.sink - c0 : 1 << 30;
           const int win_lo = sparse ? row - args.window + 1 - c0 : -(1 << 30);
+          uint32_t vm[4];
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            const bool vis = (j <= lim) && (j < sink_hi || j >= win_lo);
-            if (!vis) x[j] = -INFINITY;
-          }
+          for (int w = 0; w < 4; ++w)
+            vm[w] = bits_below(lim + 1 - 32 * w) &
+                    (bits_below(sink_hi - 32 * w) | ~bits_below(win_lo - 32 * w));
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (!((vm[j >> 5] >> (j & 31)) & 1u)) x[j] = -INFINITY;
         }
         // row max: eight independent chains of three-input max over x[8..119],
         // the last eight columns, then a tree
@@ -856,10 +873,10 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           tmem_st32(tS, pk);
         } else {
           // a tile with masked pairs (code 2) holds every key of the rows
-          // that see fewer than 128 keys; there the row sum adds the
-          // bf16-rounded probabilities, so such rows' weights sum to one
-          // exactly (a one-key row gives v itself)
-          if (code == 2)
+          // that see fewer than 128 keys; in a slot that has such rows the
+          // row sum adds the bf16-rounded probabilities there, so their
+          // weights sum to one exactly (a one-key row gives v itself)
+          if (code == 2 && few_keys)
             softmax_p_bf16<true, 0, 2>(x, sl2, msub, tS, acc);
           else
             softmax_p_bf16<false, 0, 2>(x, sl2, msub, tS, acc);
@@ -890,7 +907,7 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(bars.p_half + 8 * slot);
         if constexpr (!kFp8) {
-          if (code == 2)
+          if (code == 2 && few_keys)
             softmax_p_bf16<true, 2, 4>(x, sl2, msub, tS, acc);
           else
             softmax_p_bf16<false, 2, 4>(x, sl2, msub, tS, acc);
