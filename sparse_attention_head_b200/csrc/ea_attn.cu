@@ -937,20 +937,28 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
                  : (static_cast<size_t>(idx) * args.N + row);
       __nv_bfloat16* orow =
           reinterpret_cast<__nv_bfloat16*>(chosen ? args.out : args.out_other) + orow_index * D;
+      // 32-byte stores when the output base is 32-byte aligned (every row
+      // starts a multiple of 2 d bytes after it), else 16-byte ones
+      const bool st32 =
+          (reinterpret_cast<uintptr_t>(chosen ? args.out : args.out_other) & 31u) == 0;
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
         uint32_t o[64];
         tmem_ld64_wait(tO + h * 64, o);
         if (row < seq_len) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + h * 64);
+          uint32_t w[32];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint32_t w[4];
+          for (int j = 0; j < 32; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l,
+                               __uint_as_float(o[2 * j + 1]) * inv_l);
+          if (st32) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              w[j] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * j]) * inv_l,
-                                 __uint_as_float(o[8 * q + 2 * j + 1]) * inv_l);
-            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int q = 0; q < 4; ++q) st_global_v8(orow + h * 64 + 16 * q, &w[8 * q]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + h * 64);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           }
         }
       }
