@@ -605,8 +605,14 @@ def run_ours(args, rank, world, local_rank):
         result["packed"] = measure_packed(side, args.packed_seqs, max(args.steps, 5),
                                           max(args.warmup, 3), dev, stream)
     if not args.quick and world == 1 and args.decode_batch > 0:
+        dec_sampler = ClockSampler(visible_gpu_index(local_rank))
+        dec_sampler.start()
         result["decode"] = measure_decode(side, args.decode_batch, max(args.steps, 10),
                                           max(args.warmup, 3), dev, stream)
+        # sampled over the whole measurement (setup and both arms): the decode
+        # step is partly issue-bound, so its time follows the SM clock, which
+        # the prefill workloads before it leave under the power cap
+        result["decode"]["clocks_during_measurement"] = dec_sampler.stop()
     if not args.quick and world == 1 and not args.no_fp8 and side.d == 128:
         result["fp8"] = measure_fp8(side, max(args.steps, 5), max(args.warmup, 3), dev, stream)
     # the backward kernels are built for d = 128 (as the FP8 kernel)
@@ -1538,8 +1544,11 @@ def main():
         w = workloads.get(args.workload)
         if args.seq:
             w = dataclasses.replace(w, seq=args.seq)
+        sampler = ClockSampler(visible_gpu_index(local_rank))
+        sampler.start()
         res = measure_decode(w, max(args.decode_batch, 1), args.steps, max(args.warmup, 3), dev,
                              torch.cuda.current_stream(dev))
+        res["clocks_during_measurement"] = sampler.stop()
         if rank == 0:
             print(json.dumps(res), flush=True)
         return 0

@@ -164,3 +164,27 @@ def test_router_small_shapes(d, N):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(mask.cpu().numpy(), mask_ref)
     np.testing.assert_allclose(f64(z), z_ref, rtol=0, atol=1e-4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_output_only_16_byte_aligned(d):
+    """The C ABI asks 16-byte alignment of out; the epilogue uses 32-byte
+    stores only on a 32-byte aligned base.  An out buffer 16 bytes past a
+    32-byte boundary gives the same bits as an aligned one."""
+    B, Hq, Hkv, N, S, W = 1, 4, 2, 300, 8, 64
+    q, k, v = (t.to(DEV) for t in _qkv(B, Hq, Hkv, N, d, 31 + d))
+    mask = torch.tensor([[0, 1, 1, 0]], dtype=torch.uint8, device=DEV)
+    ws = attn_workspace(make_params(B, Hq, Hkv, N, d, S, W), DEV)
+    aligned = ea_hybrid_attn_prefill(q, k, v, mask, S, W, workspace=ws)
+    n = q.numel()
+    buf = torch.empty(n + 64, dtype=torch.bfloat16, device=DEV)
+    base = buf.data_ptr()
+    skip = ((32 - base % 32) % 32 + 16) // 2     # elements to a 16-mod-32 address
+    out16 = buf[skip:skip + n].view(q.shape)
+    assert out16.data_ptr() % 32 == 16
+    ea_hybrid_attn_prefill(q, k, v, mask, S, W, workspace=ws, out=out16)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(ws) == 0
+    assert torch.equal(aligned, out16)
+    ref = oracle.attention(f64(q.cpu()), f64(k.cpu()), f64(v.cpu()), mask.cpu().numpy(), S, W)
+    compare(out16, ref, "out16")
