@@ -232,12 +232,6 @@ __device__ bool routed_prologue(const AttnArgs& args, uint8_t* smem, volatile in
   return grid_sync(args, s_flag, 3);
 }
 
-// Bits [0, n) of a 32-bit word (n clamped to [0, 32]).
-__device__ __forceinline__ uint32_t bits_below(int n) {
-  n = n < 0 ? 0 : n;
-  return n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
-}
-
 // One row's probabilities p = 2^(x * sl2 - msub) over keys [32 C0, 32 C1)
 // of a 128-key tile:
 // packed FMA, then exp2 on the MUFU for most pairs and on the FMA pipe for
@@ -965,14 +959,16 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(bars.o_empty + 8 * slot);
       if (tracing) {
-        // slot 0's rows are stored: the unit's record
+        // slot 0's rows are stored: the unit's record (the end stamped before
+        // the record's slot is taken, so the atomic's round trip is not in it)
+        const unsigned long long t_end = global_ns();
         const unsigned long long k = atomicAdd(args.trace, 1ull);
         if (k < static_cast<unsigned long long>(args.trace_max)) {
           unsigned long long* rec = args.trace + 8 + 6 * k;
           rec[0] = s_trace_ts[0];
           rec[1] = s_trace_ts[1];
           rec[2] = s_trace_ts[2];
-          rec[3] = global_ns();
+          rec[3] = t_end;
           rec[4] = (static_cast<unsigned long long>(blockIdx.x) << 32) | static_cast<unsigned>(r);
           rec[5] = (static_cast<unsigned long long>(sparse) << 32) | static_cast<unsigned>(ut.n);
         }

@@ -184,6 +184,17 @@ template <bool kDkDv, bool kFull>
 __device__ __forceinline__ void bwd_phase_p(uint32_t taddr, const float* vl, float nl_row,
                                             int col0, float sl2, int lo_a, int hi_a, int sink_c,
                                             int win_c, float (&pr)[64], uint32_t (&pk)[32]) {
+  // visible columns col0 + lc (lc < 64) as 64 bits: lc in [lo_a, hi_a] and
+  // (lc < sink_c or lc >= win_c), shifted by col0
+  uint32_t vm[2] = {0xffffffffu, 0xffffffffu};
+  if (!kFull) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int base = col0 + 32 * w;
+      vm[w] = bits_below(hi_a + 1 - base) & ~bits_below(lo_a - base) &
+              (bits_below(sink_c - base) | ~bits_below(win_c - base));
+    }
+  }
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     uint32_t sr[32];
@@ -208,8 +219,9 @@ __device__ __forceinline__ void bwd_phase_p(uint32_t taddr, const float* vl, flo
         x1 = ex2_approx(x1);
       }
       if (!kFull) {
-        x0 = (c >= lo_a && c <= hi_a && (c < sink_c || c >= win_c)) ? x0 : 0.f;
-        x1 = (c + 1 >= lo_a && c + 1 <= hi_a && (c + 1 < sink_c || c + 1 >= win_c)) ? x1 : 0.f;
+        // local column 2 j (and 2 j + 1) of this thread's 64: word ch, bits 2 jj, 2 jj + 1
+        x0 = ((vm[ch] >> (2 * jj)) & 1u) ? x0 : 0.f;
+        x1 = ((vm[ch] >> (2 * jj + 1)) & 1u) ? x1 : 0.f;
       }
       pr[2 * j] = x0;
       pr[2 * j + 1] = x1;

@@ -7,6 +7,13 @@
 
 namespace ea {
 
+// Bits [0, n) of a 32-bit word (n clamped to [0, 32]): element masks as
+// interval bits, one bit test per element instead of several compares.
+__device__ __forceinline__ uint32_t bits_below(int n) {
+  n = n < 0 ? 0 : n;
+  return n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
