@@ -1283,6 +1283,9 @@ def measure_training(w: workloads.Workload, steps: int, warmup: int, dev, stream
 
 
 # ---------------------------------------------------------------- decode
+DECODE_WARMUP_S = 0.5
+
+
 def measure_decode(w: workloads.Workload, batch: int, steps: int, warmup: int, dev, stream):
     """One decode step per sequence of a ragged serving batch (positions in
     [seq/2, seq)), caches under the per-head policy, timed with CUDA events;
@@ -1330,8 +1333,18 @@ def measure_decode(w: workloads.Workload, batch: int, steps: int, warmup: int, d
         def step(i):
             ea_hybrid_attn_decode(q, kn, vn, pos_steps[i], m_dev, slots, *caches, S, W,
                                   max_len, out=out, workspace=ws, stream=stream)
-        for i in range(warmup):
-            step(i)
+        # warm-up: the W steps, then the last of them again (it rewrites the
+        # same cache rows) until DECODE_WARMUP_S of steps have run, so the
+        # timed steps start from steady clocks: right after a prefill
+        # measurement the GPU is still coming out of its power cap, and a
+        # step took 286 us there against 235 us half a second later
+        t_end = time.perf_counter() + DECODE_WARMUP_S
+        n = 0
+        while n < warmup or time.perf_counter() < t_end:
+            step(min(n, warmup - 1))
+            n += 1
+            if n % 32 == 0:
+                torch.cuda.synchronize()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -1358,6 +1371,8 @@ def measure_decode(w: workloads.Workload, batch: int, steps: int, warmup: int, d
                     f"ragged in [{w.seq // 2}, {w.seq}) + step, SA heads {mask.float().mean():.2f},"
                     f" all-SA kv groups {byts['n_sa_groups']}/{byts['n_groups']}",
         "steps": steps, "warmup": warmup,
+        "warmup_rule": f"{warmup} steps, then the last one repeated until {DECODE_WARMUP_S} s "
+                       "of steps have run",
         "us_per_step": round(ms * 1e3, 2),
         "tokens_per_s": round(B / (ms * 1e-3), 1),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
