@@ -294,8 +294,11 @@ ea_status ea_hybrid_attn_prefill_lse(const void* q, const void* k, const void* v
  * trace[8 + 6 i], times on the device's global timer in ns, all seen by the
  * unit's first query slot: its start, the moment its first score tile was
  * ready, the moment it handed over its last probabilities, its end (its rows
- * stored); then (CTA index << 32) | schedule rank, and (1 if SA << 32) | its
- * KV tile count.  Errors as for ea_hybrid_attn_prefill, plus EA_ERR_INVALID_ARG
+ * stored); then (CTA index << 48) | (level << 32) | schedule rank, and
+ * (1 if SA << 62) | (head of slot 0 << 44) | (head of slot 1 << 32) | its KV
+ * tile count, a head given as b * Hq + h (the two equal for a single unit;
+ * the level is a paired unit's 128-row block, 2p + 1 for a single unit of
+ * 256-row pair p).  Errors as for ea_hybrid_attn_prefill, plus EA_ERR_INVALID_ARG
  * for a NULL trace or negative trace_records and EA_ERR_MISALIGNED for a trace
  * that is not 8-byte aligned. */
 ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,

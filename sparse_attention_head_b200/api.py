@@ -313,8 +313,9 @@ def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
                                   workspace: Optional[torch.Tensor] = None,
                                   stream: Optional[torch.cuda.Stream] = None):
     """ea_hybrid_attn_prefill with a per-unit trace: (out, records int64
-    [n, 8] = start_ns, first_s_ns, last_p_ns, end_ns, cta, rank, sparse,
-    kv_tiles, total units).  Synchronises the device to read the trace back."""
+    [n, 11] = start_ns, first_s_ns, last_p_ns, end_ns, cta, rank, sparse,
+    kv_tiles, level, head of slot 0, head of slot 1 (heads as b * Hq + h),
+    total units).  Synchronises the device to read the trace back."""
     lib = _lib.load()
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
@@ -335,8 +336,10 @@ def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
     total = int(t[0])
     n = min(total, int(max_records))
     rec = t[8:8 + 6 * n].reshape(n, 6)
-    cols = np.stack([rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 3], rec[:, 4] >> 32,
-                     rec[:, 4] & 0xffffffff, rec[:, 5] >> 32, rec[:, 5] & 0xffffffff], axis=1)
+    cols = np.stack([rec[:, 0], rec[:, 1], rec[:, 2], rec[:, 3], rec[:, 4] >> 48,
+                     rec[:, 4] & 0xffffffff, (rec[:, 5] >> 62) & 1, rec[:, 5] & 0xffffffff,
+                     (rec[:, 4] >> 32) & 0xffff, (rec[:, 5] >> 44) & 0xfff,
+                     (rec[:, 5] >> 32) & 0xfff], axis=1)
     return out, cols, total
 
 

@@ -969,8 +969,11 @@ __global__ void __launch_bounds__(384, 1) ea_hybrid_attn_kernel(const __grid_con
           rec[1] = s_trace_ts[1];
           rec[2] = s_trace_ts[2];
           rec[3] = t_end;
-          rec[4] = (static_cast<unsigned long long>(blockIdx.x) << 32) | static_cast<unsigned>(r);
-          rec[5] = (static_cast<unsigned long long>(sparse) << 32) | static_cast<unsigned>(ut.n);
+          rec[4] = (static_cast<unsigned long long>(blockIdx.x) << 48) |
+                   (static_cast<unsigned long long>(word >> 14) << 32) | static_cast<unsigned>(r);
+          rec[5] = (static_cast<unsigned long long>(sparse) << 62) |
+                   (static_cast<unsigned long long>(word & 4095) << 44) |
+                   (static_cast<unsigned long long>(idx1) << 32) | static_cast<unsigned>(ut.n);
         }
       }
     }

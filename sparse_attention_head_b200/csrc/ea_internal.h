@@ -59,8 +59,9 @@ struct alignas(64) AttnArgs {
   unsigned int* done_ctas;
   // Per-unit trace (nullptr = off): trace[0] counts records; record i sits
   // at trace[8 + 6 i] .. +5 = {start, first S ready, last P handed over,
-  // end (ns), CTA << 32 | rank, sparse << 32 | KV tiles}; records past
-  // trace_max are counted, not kept.
+  // end (ns), CTA << 48 | level << 32 | rank, sparse << 62 | head of slot 0
+  // << 44 | head of slot 1 << 32 | KV tiles}; records past trace_max are
+  // counted, not kept.
   unsigned long long* trace;
   int trace_max;
   // Routed launch only: the router runs in the kernel's prologue (pool,

@@ -1,8 +1,8 @@
 """The per-unit trace of the fused prefill (ea_hybrid_attn_prefill_traced):
 the output equals the untraced call's bits, and the trace holds one record
-per unit of the host schedule view, with that unit's mode and tile count;
-units are dispatched dynamically, so each CTA runs the ranks it took from
-the ticket counter in increasing order, one after another."""
+per unit of the host schedule view, with that unit's mode, heads, rows and
+tile count; units are dispatched dynamically, so each CTA runs the ranks it
+took from the ticket counter in increasing order, one after another."""
 import numpy as np
 import pytest
 import torch
@@ -59,6 +59,15 @@ def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
     assert set(np.unique(cta).tolist()) <= set(range(grid))
     np.testing.assert_array_equal(sparse, units[rank, 0])
     np.testing.assert_array_equal(tiles, units[rank, 5])
+    # the unit each rank ran is the host view's: both slots' heads and rows
+    level, head0, head1 = rec[:, 8], rec[:, 9], rec[:, 10]
+    u = units[rank]
+    np.testing.assert_array_equal(head0, u[:, 1] * Hq + u[:, 2])
+    np.testing.assert_array_equal(head1, u[:, 1] * Hq + u[:, 3])
+    paired = u[:, 2] != u[:, 3]
+    np.testing.assert_array_equal(np.where(paired, level * 128, (level >> 1) * 256), u[:, 4])
+    if Hq // Hkv >= 2:
+        assert np.any(paired)
     # a CTA runs its units one after another, in the increasing rank order of
     # its tickets
     for c in np.unique(cta):
