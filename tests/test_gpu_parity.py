@@ -188,3 +188,27 @@ def test_output_only_16_byte_aligned(d):
     assert torch.equal(aligned, out16)
     ref = oracle.attention(f64(q.cpu()), f64(k.cpu()), f64(v.cpu()), mask.cpu().numpy(), S, W)
     compare(out16, ref, "out16")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d", [
+    (2, 3, 1, 300, 64),      # G = 3: a pair and a single per mode at most
+    (1, 16, 2, 261, 128),    # G = 8
+    (1, 32, 1, 200, 64),     # G = 32: the largest group that pairs
+    (1, 64, 1, 130, 64),     # G = 64: every head runs single
+    (1, 6, 6, 257, 128),     # G = 1: nothing to pair
+])
+def test_group_sizes_pairing(B, Hq, Hkv, N, d):
+    """Query heads of one kv group and one route share paired units; every
+    group size and odd-one-out case matches the oracle, and the split pass
+    (one mode per launch) gives the same bits."""
+    S, W = 16, 96
+    q, k, v = _qkv(B, Hq, Hkv, N, d, 700 + Hq)
+    mask = torch.from_numpy(np.random.default_rng(Hq + N).integers(0, 2, size=(B, Hq))
+                            .astype(np.uint8))
+    out = _run(q, k, v, mask, S, W)
+    ref = oracle.attention(f64(q), f64(k), f64(v), mask.numpy(), S, W)
+    compare(out, ref, f"G={Hq // Hkv}")
+    fa = _run(q, k, v, mask, S, W, select=EA_SELECT_FA)
+    sa = _run(q, k, v, mask, S, W, select=EA_SELECT_SA)
+    m = mask.to(DEV).bool()[:, :, None, None]
+    assert torch.equal(torch.where(m, sa, fa), out)
