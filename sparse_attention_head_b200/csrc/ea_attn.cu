@@ -7,10 +7,14 @@
 // W keys including the diagonal); full heads are plain causal attention.
 //
 // Design (one persistent CTA per SM, 12 warps = 3 warpgroups):
-//   warps 0-3  softmax/correction/epilogue of query slot 0 (rows r0..r0+127)
-//   warps 4-7  the same for slot 1 (rows r0+128..r0+255)
-//   warp  8    TMA producer: Q slots once per unit, then K and V tiles of the
-//              unit's tile list through a ring of shared-memory stages
+//   warps 0-3  softmax/correction/epilogue of query slot 0 (a paired unit:
+//              head h0, rows r0..r0+127; a single unit: rows r0..r0+127)
+//   warps 4-7  the same for slot 1 (head h1 at the same rows; a single unit:
+//              rows r0+128..r0+255 of the one head)
+//   warp  8    TMA producer: takes the unit tickets, walks the schedule and
+//              hands each unit on through a shared-memory ring; loads the
+//              Q slots once per unit, then K and V tiles of the unit's tile
+//              list through a ring of shared-memory stages
 //   warp  9    tcgen05 issuer (the whole warp runs the loop, the elected
 //              lane issues): S_s = Q_s K^T into TMEM, then O_s += P_s V with
 //              P read from TMEM (P overwrites S in place)
@@ -26,9 +30,9 @@
 // reference max is only moved when a tile's max exceeds it by more than 8
 // (2^8 headroom in fp32/bf16), so most tiles need no O rescale; the final
 // O / l uses the same reference, so the result is unchanged.  The row sum l
-// adds the fp32 probabilities on fully visible tiles and the bf16-rounded
-// ones (those the P.V product sees) on masked tiles, which hold every key of
-// the rows that see fewer than 128 keys.
+// adds the fp32 probabilities, except on the masked tiles of slots holding a
+// row that sees fewer than 128 keys: there it adds the bf16-rounded ones
+// (those the P.V product sees), so such rows' weights sum to one exactly.
 //
 // Every wait is bounded: on timeout the kernel records EA_ERR_TIMEOUT in the
 // status word, every role leaves its loop, in-flight copies and MMAs are

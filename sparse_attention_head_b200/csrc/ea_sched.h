@@ -38,7 +38,7 @@
 //   Measured at 256K tokens (32 query, 8 kv heads, d = 128, 24 of 32 heads
 //   SA; one B200): dealt statically in a snake, the CTAs drifted apart and
 //   DRAM reads were ~70x one pass over q, k, v; dealt dynamically, ~44x;
-//   with the long FA units by kv group as well, ~1.4x and 8% less time.  At
+//   with the long FA units by kv group as well, ~1.7x and 8% less time.  At
 //   192K tokens by group was 4% faster; at 16K-64K tokens by level was as
 //   fast or faster (up to 7%).
 #pragma once
