@@ -196,6 +196,8 @@ def test_output_only_16_byte_aligned(d):
     (1, 32, 1, 200, 64),     # G = 32: the largest group that pairs
     (1, 64, 1, 130, 64),     # G = 64: every head runs single
     (1, 6, 6, 257, 128),     # G = 1: nothing to pair
+    (1, 48, 16, 140, 64),    # G = 3 over two 30-lane chunks of the prologue's ballots
+    (2, 40, 8, 129, 64),     # G = 5 over two chunks
 ])
 def test_group_sizes_pairing(B, Hq, Hkv, N, d):
     """Query heads of one kv group and one route share paired units; every

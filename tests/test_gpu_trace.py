@@ -28,6 +28,8 @@ def _lib():
     (1, 8, 2, 2048, 128, 64, 256),
     (2, 16, 4, 700, 64, 8, 100),
     (1, 8, 2, 131072, 128, 64, 1024),    # long FA units kv group by kv group
+    (1, 48, 16, 600, 64, 8, 64),         # G = 3: groups over the prologue's 30-lane chunks
+    (1, 64, 2, 300, 64, 8, 64),          # G = 32 over two chunks
 ])
 def test_trace_matches_the_schedule(B, Hq, Hkv, N, d, S, W):
     g = torch.Generator().manual_seed(N)

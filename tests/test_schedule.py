@@ -415,3 +415,15 @@ def test_backward_schedule_mirror_balances():
             assert np.all(c[:-1] >= c[1:])
         load = m.per_cta_load(offs, lst, cost)
         assert load.max() / load.mean() < 1.02, (kdkdv, load.max() / load.mean())
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(48, 16), (40, 8), (96, 3), (64, 2)])
+def test_pairing_across_prologue_chunks(Hq, Hkv):
+    """Groups whose heads span the kernel prologue's 32-lane chunks (G = 3, 5:
+    chunks of 30 lanes; G = 32; G = 32 over several chunks) pair as the rule
+    says, and every row is covered once."""
+    B, N, d, S, W = 2, 300, 64, 8, 64
+    rng = np.random.default_rng(Hq * Hkv)
+    mask = rng.integers(0, 2, size=(B, Hq)).astype(np.uint8)
+    units = ea_schedule_units(mask, make_params(B, Hq, Hkv, N, d, S, W))
+    _check_cover(units, [N] * B, mask, Hq, Hkv, 0)
