@@ -234,7 +234,8 @@ def bench_config(w: workloads.Workload, sparse_frac: float, world: int) -> dict:
     return {"workload": workload_desc(w, sparse_frac), "global_batch": w.batch,
             "seq_len": w.seq,
             "parallelism": ("single GPU" if world == 1 else
-                            f"(batch, kv group) shards x{world}: LPT on the mask's tile cost, "
+                            f"(batch, kv group) shards x{world}, a group over a rank's share split "
+                            "by query head: LPT on the mask's tile cost, "
                             "all-gather of the router's pooled slices"),
             "l2": l2}
 
@@ -626,12 +627,13 @@ def run_sharded(args, rank, world, local_rank):
     """N > 1: ONE layer's prefill (per layer of the workload) head-sharded over
     the ranks: each rank pools its share of the (b, kv head) rows, one NCCL
     all-gather of the pooled slices feeds the router on every rank, the
-    (b, kv group) groups are assigned by LPT on their cost under the mask,
+    (b, kv group) groups are assigned by LPT on their cost under the mask (a
+    group costlier than a rank's share split by query head),
     and each rank runs the fused attention on its groups.  Total work is
     fixed (strong scaling); the time is the slowest rank's."""
     from sparse_attention_head_b200 import flops
     from sparse_attention_head_b200.api import ea_get_device_status
-    from sparse_attention_head_b200.shard import ShardedPrefill, rank_loads, group_costs
+    from sparse_attention_head_b200.shard import ShardedPrefill, head_costs, rank_loads
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = workloads.get(args.workload)
@@ -690,12 +692,11 @@ def run_sharded(args, rank, world, local_rank):
     # this rank's share of the work, and its attention launches' time
     mine = 0.0
     for m, sp in zip(masks, sps):
-        sel = sp.owner == rank
+        sel = sp.owner == rank          # [B, Hq]
         for b in range(B):
-            for hk in range(Hkv):
-                if sel[b, hk]:
-                    mine += flops.effective_flops(m[b, hk * (Hq // Hkv):(hk + 1) * (Hq // Hkv)],
-                                                  N, d, w.sink, w.window)
+            for h in range(Hq):
+                if sel[b, h]:
+                    mine += flops.effective_flops(m[b, h:h + 1], N, d, w.sink, w.window)
     attn_ms = statistics.mean(evs[i][l][1].elapsed_time(evs[i][l][2]) for i in range(K)
                               for l in range(w.layers))
     route_ms = statistics.mean(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K)
@@ -704,7 +705,7 @@ def run_sharded(args, rank, world, local_rank):
     value = eff / (ms_per_step * 1e-3) / 1e12
     peak, peak_kind, burst, peak_src = roofline_peak(total_ms)
     achieved = (mine / w.layers) / (attn_ms * 1e-3) / 1e12
-    loads = rank_loads(group_costs(masks[0], Hkv, N, w.sink, w.window), sps[0].owner, world)
+    loads = rank_loads(head_costs(masks[0], N, w.sink, w.window), sps[0].owner, world)
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),

@@ -269,6 +269,17 @@ ea_status ea_hybrid_attn_prefill_groups(const void* q, const void* k, const void
                                         const ea_attn_params* p, void* out, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* The same restricted by query head: head_sel (device uint8 [B][Hq]) is
+ * nonzero where head (b, h) runs.  For a shard that splits a kv group whose
+ * heads cost more than a rank's share: the ranks holding its heads each read
+ * the group's K and V.  Each head's rows have the bits of the unrestricted
+ * call; the other heads' rows are left untouched.  NULL head_sel:
+ * EA_ERR_INVALID_ARG; otherwise as ea_hybrid_attn_prefill. */
+ea_status ea_hybrid_attn_prefill_heads(const void* q, const void* k, const void* v,
+                                       const uint8_t* route_mask, const uint8_t* head_sel,
+                                       const ea_attn_params* p, void* out, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word kept
  * in `workspace` (an attention workspace).  *status_out receives EA_OK or
  * the error a kernel recorded (EA_ERR_TIMEOUT when a bounded device wait ran

@@ -46,7 +46,7 @@ EXPORTED = [
     "ea_quantize_fp8", "ea_hybrid_attn_prefill_fp8", "ea_hybrid_attn_host_workspace_size",
     "ea_hybrid_attn_host_chunks", "ea_hybrid_attn_prefill_host", "ea_shutdown",
     "ea_hybrid_attn_prefill_traced", "ea_router_pool_rows", "ea_router_mlp_workspace_size",
-    "ea_router_mlp", "ea_hybrid_attn_prefill_groups",
+    "ea_router_mlp", "ea_hybrid_attn_prefill_groups", "ea_hybrid_attn_prefill_heads",
 ]
 
 
@@ -133,6 +133,9 @@ def load(build_if_missing: bool = False) -> ctypes.CDLL:
     lib.ea_hybrid_attn_prefill_groups.restype = c_int
     lib.ea_hybrid_attn_prefill_groups.argtypes = [vp, vp, vp, vp, vp, pparams, vp, vp, c_size,
                                                   vp]
+    lib.ea_hybrid_attn_prefill_heads.restype = c_int
+    lib.ea_hybrid_attn_prefill_heads.argtypes = [vp, vp, vp, vp, vp, pparams, vp, vp, c_size,
+                                                 vp]
     lib.ea_hybrid_attn_prefill.restype = c_int
     lib.ea_hybrid_attn_prefill.argtypes = [vp, vp, vp, vp, pparams, vp, vp, c_size, vp]
     lib.ea_get_device_status.restype = c_int

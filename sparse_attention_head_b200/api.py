@@ -269,27 +269,28 @@ def ea_hybrid_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out
 
 
-def ea_hybrid_attn_prefill_groups(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                                  route_mask: torch.Tensor, group_sel: torch.Tensor,
-                                  sink: int, window: int, *, softmax_scale: float = 0.0,
-                                  out: Optional[torch.Tensor] = None,
-                                  workspace: Optional[torch.Tensor] = None,
-                                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """The fused prefill on one shard: only the query heads of the (b, kv
-    head) groups with group_sel[b, hk] != 0 run; other heads' rows of `out`
-    are left as they were."""
+def _prefill_selected(name: str, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      route_mask: torch.Tensor, sel: torch.Tensor, sink: int, window: int, *,
+                      softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The fused prefill on one shard, through the C entry point `name`:
+    ea_hybrid_attn_prefill_groups (sel [B, Hkv] by kv group) or
+    ea_hybrid_attn_prefill_heads (sel [B, Hq] by query head).  Only the
+    selected heads run; other heads' rows of `out` are left as they were."""
     lib = _lib.load()
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
     _need(route_mask, "route_mask", torch.uint8)
-    _need(group_sel, "group_sel", torch.uint8)
+    _need(sel, "selection", torch.uint8)
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
         raise ValueError("k and v must be [B, Hkv, N, d] matching q")
-    if route_mask.numel() != B * Hq or group_sel.numel() != B * Hkv:
-        raise ValueError("route_mask must hold B * Hq entries and group_sel B * Hkv")
+    want = B * Hkv if name == "ea_hybrid_attn_prefill_groups" else B * Hq
+    if route_mask.numel() != B * Hq or sel.numel() != want:
+        raise ValueError("route_mask must hold B * Hq entries and the selection %d" % want)
     p = make_params(B, Hq, Hkv, N, d, sink, window, softmax_scale)
     if out is None:
         out = torch.empty_like(q)
@@ -299,12 +300,32 @@ def ea_hybrid_attn_prefill_groups(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
             raise ValueError("out must have q's shape")
     if workspace is None:
         workspace = attn_workspace(p, q.device)
-    rc = lib.ea_hybrid_attn_prefill_groups(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                           route_mask.data_ptr(), group_sel.data_ptr(),
-                                           ctypes.byref(p), out.data_ptr(), workspace.data_ptr(),
-                                           workspace.numel(), _stream_ptr(stream, q.device))
-    check(rc, "ea_hybrid_attn_prefill_groups")
+    rc = getattr(lib, name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), route_mask.data_ptr(),
+                            sel.data_ptr(), ctypes.byref(p), out.data_ptr(),
+                            workspace.data_ptr(), workspace.numel(),
+                            _stream_ptr(stream, q.device))
+    check(rc, name)
     return out
+
+
+def ea_hybrid_attn_prefill_groups(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  route_mask: torch.Tensor, group_sel: torch.Tensor,
+                                  sink: int, window: int, **kw) -> torch.Tensor:
+    """The fused prefill on one shard: only the query heads of the (b, kv
+    head) groups with group_sel[b, hk] != 0 run; other heads' rows of `out`
+    are left as they were."""
+    return _prefill_selected("ea_hybrid_attn_prefill_groups", q, k, v, route_mask, group_sel,
+                             sink, window, **kw)
+
+
+def ea_hybrid_attn_prefill_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                 route_mask: torch.Tensor, head_sel: torch.Tensor,
+                                 sink: int, window: int, **kw) -> torch.Tensor:
+    """The fused prefill on one shard: only the query heads with
+    head_sel[b, h] != 0 run; other heads' rows of `out` are left as they
+    were."""
+    return _prefill_selected("ea_hybrid_attn_prefill_heads", q, k, v, route_mask, head_sel,
+                             sink, window, **kw)
 
 
 def ea_hybrid_attn_prefill_traced(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -505,7 +505,8 @@ static ea_status prefill_impl(const void* q, const void* k, const void* v,
                               const uint8_t* route_mask, const ea_attn_params* p, void* out,
                               void* workspace, size_t workspace_bytes,
                               unsigned long long* trace, int trace_max, void* stream,
-                              const uint8_t* group_sel = nullptr) {
+                              const uint8_t* group_sel = nullptr,
+                              const uint8_t* head_sel = nullptr) {
   ea_status st = check_params(p);
   if (st != EA_OK) return st;
   if (!q || !k || !v || !route_mask || !out) return EA_ERR_INVALID_ARG;
@@ -539,6 +540,7 @@ static ea_status prefill_impl(const void* q, const void* k, const void* v,
   args.trace = trace;
   args.trace_max = trace_max;
   args.group_sel = group_sel;
+  args.head_sel = head_sel;
 
   const int sms = device_sms();
   if (sms <= 0) return EA_ERR_CUDA;
@@ -561,6 +563,15 @@ ea_status ea_hybrid_attn_prefill_groups(const void* q, const void* k, const void
   if (!group_sel) return EA_ERR_INVALID_ARG;
   return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, nullptr, 0, stream,
                       group_sel);
+}
+
+ea_status ea_hybrid_attn_prefill_heads(const void* q, const void* k, const void* v,
+                                      const uint8_t* route_mask, const uint8_t* head_sel,
+                                      const ea_attn_params* p, void* out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!head_sel) return EA_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, route_mask, p, out, workspace, workspace_bytes, nullptr, 0, stream,
+                      nullptr, head_sel);
 }
 
 ea_status ea_hybrid_attn_prefill_traced(const void* q, const void* k, const void* v,

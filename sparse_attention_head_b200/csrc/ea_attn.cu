@@ -128,10 +128,12 @@ __device__ __forceinline__ uint8_t ld_mask(const uint8_t* mask, int idx) {
   return idx >= 0 ? *reinterpret_cast<const volatile uint8_t*>(mask + idx) : 0;
 }
 
-// Does the launch's shard run the query heads of (sequence b, kv head of h)?
+// Does the launch's shard run query head h of sequence b (its kv group
+// selected, and the head itself when a head selection is given)?
 __device__ __forceinline__ bool in_shard(const AttnArgs& args, int b, int h) {
-  return args.group_sel == nullptr ||
-         args.group_sel[b * args.Hkv + h / (args.Hq / args.Hkv)] != 0;
+  return (args.group_sel == nullptr ||
+          args.group_sel[b * args.Hkv + h / (args.Hq / args.Hkv)] != 0) &&
+         (args.head_sel == nullptr || args.head_sel[b * args.Hq + h] != 0);
 }
 
 // This CTA takes no more tickets (its producer has stopped, or never

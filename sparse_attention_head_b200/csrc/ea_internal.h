@@ -52,6 +52,9 @@ struct alignas(64) AttnArgs {
   // query heads of (batch, kv head) run; the others' output rows are not
   // written.
   const uint8_t* group_sel;
+  // The same by query head (nullptr = every head): [B*Hq], nonzero where
+  // head (batch, h) runs.
+  const uint8_t* head_sel;
   // Dynamic unit dispatch, inside the caller's 256-byte status block: the
   // launch's ticket counter and the count of CTAs done taking tickets (the
   // last one resets both to zero for the next launch).  Set by the launcher.

@@ -11,7 +11,11 @@ all-gather of those fp32 slices (B * Hkv * d values) gives every rank the
 same pooled vector, hence the same mask.  The mask then fixes each group's
 cost, and the groups are assigned to ranks by longest-processing-time
 (largest cost first, to the least-loaded rank): deterministic, so every rank
-computes the same assignment without another exchange.
+computes the same assignment without another exchange.  A group that costs
+more than a rank's share (total / ranks) is split into its query heads, each
+assigned on its own; the ranks holding its heads each read the group's K/V.
+With few groups per rank (8 kv groups over 8 ranks) whole groups cannot
+balance: one with two or three full-attention heads sets the time.
 
 Host logic only (ownership, costs, assignment) plus the per-layer step that
 strings the C ABI calls together with torch.distributed; every step of the
@@ -55,6 +59,44 @@ def group_costs(mask, Hkv: int, N: int, sink: int, window: int) -> np.ndarray:
     return (n_sa * t_sa + (G - n_sa) * t_fa).astype(np.int64)
 
 
+def head_costs(mask, N: int, sink: int, window: int) -> np.ndarray:
+    """[B, Hq] int64: the score tiles each query head runs under the mask."""
+    m = np.asarray(mask)
+    m = m.reshape(m.shape[0], -1)
+    t_fa = _visible_tiles(N, False, sink, window)
+    t_sa = _visible_tiles(N, True, sink, window)
+    return np.where(m != 0, t_sa, t_fa).astype(np.int64)
+
+
+def lpt_assign_split(mask, Hkv: int, N: int, sink: int, window: int, world: int) -> np.ndarray:
+    """owner [B, Hq] by query head.  The items are the (b, kv group) groups,
+    except that a group costing more than total / world becomes one item per
+    query head; then longest processing time first over the items (ties:
+    lower first head index first; least-loaded rank, ties to the lower
+    rank).  Depends only on the mask, so every rank computes the same one."""
+    hc = head_costs(mask, N, sink, window)
+    B, Hq = hc.shape
+    G = Hq // Hkv
+    gc = hc.reshape(B, Hkv, G).sum(axis=2)
+    share = gc.sum() / max(world, 1)
+    items = []          # (cost, first head flat index, heads as flat indices)
+    for b in range(B):
+        for hk in range(Hkv):
+            heads = [b * Hq + hk * G + j for j in range(G)]
+            if world > 1 and G > 1 and gc[b, hk] > share:
+                items.extend((int(hc.reshape(-1)[i]), i, [i]) for i in heads)
+            else:
+                items.append((int(gc[b, hk]), heads[0], heads))
+    items.sort(key=lambda it: (-it[0], it[1]))
+    load = [0] * world
+    owner = np.empty(B * Hq, dtype=np.int64)
+    for cost, _, heads in items:
+        r = min(range(world), key=lambda x: (load[x], x))
+        owner[heads] = r
+        load[r] += cost
+    return owner.reshape(B, Hq)
+
+
 def lpt_assign(costs, world: int) -> np.ndarray:
     """owner [B, Hkv]: longest processing time first.  Groups are taken in
     order of decreasing cost (ties: lower flattened index first) and each
@@ -70,6 +112,12 @@ def lpt_assign(costs, world: int) -> np.ndarray:
         owner[i] = r
         load[r] += int(flat[i])
     return owner.reshape(c.shape)
+
+
+def heads_of(owner_h, rank: int) -> Sequence[Tuple[int, int]]:
+    """(b, h) query heads a per-head assignment gives `rank`."""
+    o = np.asarray(owner_h)
+    return [(b, h) for b in range(o.shape[0]) for h in range(o.shape[1]) if o[b, h] == rank]
 
 
 def group_select(owner, rank: int) -> np.ndarray:
@@ -99,8 +147,10 @@ def gather_pooled(x_local: torch.Tensor, B: int, Hkv: int, d: int, world: int,
 
 class ShardedPrefill:
     """One layer's sharded prefill on this rank: router pooling of the rank's
-    rows, the all-gather of the pooled slices, the router MLP, the group
-    assignment, and the fused attention on the rank's groups.
+    rows, the all-gather of the pooled slices, the router MLP, the
+    assignment (by group, a group costlier than a rank's share split by
+    query head; split_groups=False keeps whole groups), and the fused
+    attention on the rank's query heads.
 
     Every rank holds the layer's full q, k, v (for instance after an
     all-gather of the projections); a rank reads the keys of its pooling
@@ -110,7 +160,8 @@ class ShardedPrefill:
 
     def __init__(self, B: int, Hq: int, Hkv: int, N: int, d: int, w1, b1, w2, b2,
                  sink: int, window: int, rank: int, world: int, device, group=None,
-                 threshold: float = 0.0, mask: Optional[torch.Tensor] = None):
+                 threshold: float = 0.0, mask: Optional[torch.Tensor] = None,
+                 split_groups: bool = True):
         """w1..b2: the router's weights on `device`; or all None with `mask`
         (device uint8 [B, Hq]) given, for a layer whose routing is fixed (no
         router step, no exchange)."""
@@ -135,7 +186,8 @@ class ShardedPrefill:
             torch.empty((B, Hq), dtype=torch.uint8, device=self.dev)
         self.mask_host = torch.empty((B, Hq), dtype=torch.uint8).pin_memory() \
             if torch.cuda.is_available() else torch.empty((B, Hq), dtype=torch.uint8)
-        self.sel = torch.empty((B, Hkv), dtype=torch.uint8, device=self.dev)
+        self.split_groups = split_groups
+        self.sel = torch.empty((B, Hq), dtype=torch.uint8, device=self.dev)
         self.attn_ws = attn_workspace(make_params(B, Hq, Hkv, N, d, sink, window), self.dev)
         self.owner = None
 
@@ -154,30 +206,37 @@ class ShardedPrefill:
 
     def assign(self, stream=None) -> np.ndarray:
         """Step 4a: the host copy of the mask (synchronises the stream), the
-        groups' costs and the LPT assignment; uploads this rank's selection."""
+        costs and the LPT assignment; uploads this rank's head selection.
+        Returns the owner of every query head, [B, Hq]."""
         s = stream if stream is not None else torch.cuda.current_stream(self.dev)
         with torch.cuda.stream(s):
             self.mask_host.copy_(self.mask, non_blocking=True)
             s.synchronize()
             m = self.mask_host.numpy().copy()
-            self.owner = lpt_assign(group_costs(m, self.Hkv, self.N, self.sink, self.window),
-                                    self.world)
-            self.sel.copy_(torch.as_tensor(group_select(self.owner, self.rank)))
+            if self.split_groups:
+                self.owner = lpt_assign_split(m, self.Hkv, self.N, self.sink, self.window,
+                                              self.world)
+            else:
+                g = lpt_assign(group_costs(m, self.Hkv, self.N, self.sink, self.window),
+                               self.world)
+                self.owner = np.repeat(g, self.Hq // self.Hkv, axis=1)
+            self.sel.copy_(torch.as_tensor((self.owner == self.rank).astype(np.uint8)))
         return self.owner
 
     def attend(self, q, k, v, out, stream=None) -> torch.Tensor:
-        """Step 4b: the fused attention on this rank's groups."""
-        from .api import ea_hybrid_attn_prefill_groups
-        return ea_hybrid_attn_prefill_groups(q, k, v, self.mask, self.sel, self.sink,
-                                             self.window, out=out, workspace=self.attn_ws,
-                                             stream=stream)
+        """Step 4b: the fused attention on this rank's query heads."""
+        from .api import ea_hybrid_attn_prefill_heads
+        return ea_hybrid_attn_prefill_heads(q, k, v, self.mask, self.sel, self.sink,
+                                            self.window, out=out, workspace=self.attn_ws,
+                                            stream=stream)
 
     def host_step(self, q_host, k_host, v_host, out_host, q, k, v, out, stream=None):
         """The step from pinned host buffers: the keys of the rank's pooling
-        rows go up first; after the assignment, the q, k, v of the rank's
-        groups; its heads' output rows come back into out_host (valid after
-        the stream synchronises).  q, k, v, out: full-size device buffers of
-        which the rank uses its parts.  Returns (bytes up, bytes down)."""
+        rows go up first; after the assignment, the q rows of the rank's
+        heads and the k, v of their kv groups; its heads' output rows come
+        back into out_host (valid after the stream synchronises).  q, k, v,
+        out: full-size device buffers of which the rank uses its parts.
+        Returns (bytes up, bytes down)."""
         s = stream if stream is not None else torch.cuda.current_stream(self.dev)
         G = self.Hq // self.Hkv
         up = down = 0
@@ -188,24 +247,24 @@ class ShardedPrefill:
                 up += k[b, hk].numel() * k.element_size()
             self.route(k, s)
             owner = self.assign(s)
+            mine = owner == self.rank
             for b in range(self.B):
                 for hk in range(self.Hkv):
-                    if owner[b, hk] != self.rank:
+                    hs = [hk * G + j for j in range(G) if mine[b, hk * G + j]]
+                    if not hs:
                         continue
-                    hs = slice(hk * G, (hk + 1) * G)
-                    q[b, hs].copy_(q_host[b, hs], non_blocking=True)
+                    for h in hs:
+                        q[b, h].copy_(q_host[b, h], non_blocking=True)
+                        up += q[b, h].numel() * q.element_size()
                     v[b, hk].copy_(v_host[b, hk], non_blocking=True)
-                    up += q[b, hs].numel() * q.element_size() + v[b, hk].numel() * v.element_size()
+                    up += v[b, hk].numel() * v.element_size()
                     if not (self.row0 <= b * self.Hkv + hk < self.row0 + self.nrows):
                         k[b, hk].copy_(k_host[b, hk], non_blocking=True)
                         up += k[b, hk].numel() * k.element_size()
             self.attend(q, k, v, out, s)
-            for b in range(self.B):
-                for hk in range(self.Hkv):
-                    if owner[b, hk] == self.rank:
-                        hs = slice(hk * G, (hk + 1) * G)
-                        out_host[b, hs].copy_(out[b, hs], non_blocking=True)
-                        down += out[b, hs].numel() * out.element_size()
+            for b, h in heads_of(owner, self.rank):
+                out_host[b, h].copy_(out[b, h], non_blocking=True)
+                down += out[b, h].numel() * out.element_size()
         return up, down
 
     def __call__(self, q, k, v, out, stream=None) -> torch.Tensor:

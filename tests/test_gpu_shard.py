@@ -4,8 +4,10 @@ emulated one after another on one GPU (no kernel waits on another):
   all-gather lays them, then ea_router_mlp, gives ea_router_decide's mask
   and logits bit for bit;
 - each rank's ea_hybrid_attn_prefill_groups launch on its LPT-assigned
-  groups writes exactly its heads' rows, with the bits of the unsharded
-  fused launch, and leaves every other row untouched."""
+  groups, and each rank's ea_hybrid_attn_prefill_heads launch on its heads
+  under the split assignment (a group costlier than a rank's share split by
+  query head), writes exactly its heads' rows, with the bits of the
+  unsharded fused launch, and leaves every other row untouched."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +15,8 @@ import torch
 from sparse_attention_head_b200 import build, shard
 from sparse_attention_head_b200.api import (attn_workspace, ea_get_device_status,
                                             ea_hybrid_attn_prefill,
-                                            ea_hybrid_attn_prefill_groups, ea_router_decide,
+                                            ea_hybrid_attn_prefill_groups,
+                                            ea_hybrid_attn_prefill_heads, ea_router_decide,
                                             ea_router_mlp, ea_router_mlp_workspace_size,
                                             ea_router_pool_rows, ea_router_workspace_size,
                                             make_params)
@@ -95,6 +98,24 @@ def test_sharded_router_and_attention_equal_the_single_launch(B, Hq, Hkv, N, d, 
             mine[b, h] = True
         covered |= mine
         own = mine.to(DEV)
+        assert torch.equal(out[own].view(torch.int16), out_ref[own].view(torch.int16)), r
+        assert bool((out[~own] == 7.0).all()), r
+    assert bool(covered.all())
+
+    # step 4, split assignment: every rank's query heads
+    owner_h = shard.lpt_assign_split(m, Hkv, N, S, W, world)
+    covered = torch.zeros((B, Hq), dtype=torch.bool)
+    for r in range(world):
+        sel = torch.as_tensor((owner_h == r).astype(np.uint8), device=DEV)
+        out = torch.full_like(q, 7.0)
+        ws = attn_workspace(make_params(B, Hq, Hkv, N, d, S, W), DEV)
+        ea_hybrid_attn_prefill_heads(q, k, v, mask, sel, S, W, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        assert ea_get_device_status(ws) == 0
+        own = torch.as_tensor(owner_h == r)
+        assert not bool((covered & own).any())
+        covered |= own
+        own = own.to(DEV)
         assert torch.equal(out[own].view(torch.int16), out_ref[own].view(torch.int16)), r
         assert bool((out[~own] == 7.0).all()), r
     assert bool(covered.all())

@@ -4,7 +4,9 @@
   contiguous equal chunks.
 - Group costs: the score tiles of each group's heads, against a count made
   tile by tile from the visibility definition.
-- LPT assignment: a partition, deterministic, and within the LPT bound.
+- LPT assignment: a partition, deterministic, and within the LPT bound; the
+  split assignment splits exactly the groups costlier than a rank's share,
+  keeps the others whole, and balances the bench's 8-group layer on 8 ranks.
 - World-size 2 and 3 gloo ranks: each rank pools only its own rows (the
   oracle's pooling stands in for the pooling kernel), the package's
   all-gather assembles the pooled vector, and the router MLP on it gives
@@ -84,6 +86,64 @@ def test_lpt_assignment_partition_and_bound():
     assert owner.tolist() == [[0, 1, 1, 0, 1]]
 
 
+@pytest.mark.parametrize("N,S,W", [(300, 4, 100), (1000, 0, 1)])
+def test_head_costs_count_visible_tiles(N, S, W):
+    rng = np.random.default_rng(N + 1)
+    mask = (rng.random((2, 8)) < 0.5).astype(np.uint8)
+    hc = shard.head_costs(mask, N, S, W)
+    t_fa, t_sa = _tiles_by_definition(N, False, S, W), _tiles_by_definition(N, True, S, W)
+    np.testing.assert_array_equal(hc, np.where(mask != 0, t_sa, t_fa))
+    np.testing.assert_array_equal(hc.reshape(2, 2, 4).sum(axis=2), shard.group_costs(mask, 2, N, S, W))
+
+
+def test_split_assignment_splits_only_heavy_groups():
+    rng = np.random.default_rng(3)
+    N, S, W = 8192, 64, 512
+    for world in (1, 2, 3, 4, 8):
+        for _ in range(10):
+            B, Hkv, G = int(rng.integers(1, 4)), int(rng.choice([2, 4, 8])), int(rng.choice([1, 2, 4]))
+            Hq = Hkv * G
+            mask = (rng.random((B, Hq)) < 0.6).astype(np.uint8)
+            owner = shard.lpt_assign_split(mask, Hkv, N, S, W, world)
+            assert owner.shape == (B, Hq) and set(np.unique(owner)) <= set(range(world))
+            np.testing.assert_array_equal(owner, shard.lpt_assign_split(mask.copy(), Hkv, N, S, W,
+                                                                        world))
+            gc = shard.group_costs(mask, Hkv, N, S, W)
+            share = gc.sum() / world
+            g_owner = owner.reshape(B, Hkv, G)
+            for b in range(B):
+                for hk in range(Hkv):
+                    whole = len(set(g_owner[b, hk].tolist())) == 1
+                    if gc[b, hk] <= share or world == 1 or G == 1:
+                        assert whole, (world, b, hk)
+            hc = shard.head_costs(mask, N, S, W)
+            loads = shard.rank_loads(hc, owner, world)
+            assert sum(loads) == int(hc.sum())
+            # LPT bound over the items: mean load + the largest item
+            assert max(loads) <= hc.sum() / world + max(int(hc.max()), int(gc[gc <= share].max())
+                                                          if np.any(gc <= share) else 0)
+
+
+def test_split_assignment_balances_eight_groups_on_eight_ranks():
+    # the bench's 256K layer shape: FA heads per kv group 2 1 2 0 1 1 0 1
+    fa = [2, 1, 2, 0, 1, 1, 0, 1]
+    mask = np.ones((1, 32), np.uint8)
+    for g, n in enumerate(fa):
+        mask[0, 4 * g:4 * g + n] = 0
+    N, S, W = 262144, 128, 4096
+    whole = shard.lpt_assign(shard.group_costs(mask, 8, N, S, W), 8)
+    hc = shard.head_costs(mask, N, S, W)
+    loads_whole = shard.rank_loads(shard.group_costs(mask, 8, N, S, W), whole, 8)
+    split = shard.lpt_assign_split(mask, 8, N, S, W, 8)
+    loads_split = shard.rank_loads(hc, split, 8)
+    mean = hc.sum() / 8
+    assert mean / max(loads_whole) < 0.6
+    assert mean / max(loads_split) > 0.95
+    # each rank runs one full-attention head
+    for r in range(8):
+        assert sum(1 for h in range(32) if split[0, h] == r and mask[0, h] == 0) == 1
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -121,8 +181,8 @@ def _rank_main(rank, world, port, out_dir):
         x = shard.gather_pooled(torch.as_tensor(x_local.reshape(-1)), B, Hkv, d, world)
         z = oracle.router_mlp(x.numpy(), w1, b1, w2, b2)
         mask = (z > 0.0).astype(np.uint8)
-        owner = shard.lpt_assign(shard.group_costs(mask, Hkv, N, 8, 20), world)
-        heads = shard.head_rows_of(owner, rank, Hq // Hkv)
+        owner = shard.lpt_assign_split(mask, Hkv, N, 8, 20, world)
+        heads = shard.heads_of(owner, rank)
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), x=x.numpy(), z=z, mask=mask,
                  owner=owner, heads=np.array(heads, dtype=np.int64).reshape(-1, 2))
         dist.barrier()
