@@ -120,3 +120,31 @@ def test_sharded_router_and_attention_equal_the_single_launch(B, Hq, Hkv, N, d, 
         assert bool((out[~own] == 7.0).all()), r
     assert bool(covered.all())
     assert ea_get_device_status(ws_ref) == 0
+
+
+@pytest.mark.parametrize("split", [True, False])
+def test_sharded_prefill_class_one_rank(split):
+    """ShardedPrefill on one rank (no exchange: the gathered vector is the
+    rank's own slice): route, assign and attend give the unsharded launch's
+    mask and output bits, and host_step moves every head up and down."""
+    B, Hq, Hkv, N, d, S, W = 2, 16, 4, 700, 128, 16, 128
+    q, k, v, w1, b1, w2, b2 = _layer(B, Hq, Hkv, N, d, 64, seed=77)
+    mask_ref, _ = ea_router_decide(k, w1, b1, w2, b2)
+    out_ref = ea_hybrid_attn_prefill(q, k, v, mask_ref, S, W)
+    sp = shard.ShardedPrefill(B, Hq, Hkv, N, d, w1, b1, w2, b2, S, W, 0, 1, DEV,
+                              split_groups=split)
+    out = torch.full_like(q, 7.0)
+    sp(q, k, v, out)
+    torch.cuda.synchronize()
+    assert ea_get_device_status(sp.attn_ws) == 0
+    assert torch.equal(sp.mask, mask_ref)
+    assert np.all(sp.owner == 0)
+    assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16))
+    # from pinned host buffers
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd, od = (torch.empty_like(t) for t in (q, k, v, q))
+    up, down = sp.host_step(qh, kh, vh, oh, qd, kd, vd, od)
+    torch.cuda.synchronize()
+    assert torch.equal(oh.view(torch.int16), out_ref.cpu().view(torch.int16))
+    assert up == (q.numel() + k.numel() + v.numel()) * 2 and down == q.numel() * 2
